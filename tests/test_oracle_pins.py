@@ -1,0 +1,415 @@
+"""Pins of the CPU oracle to facts fixed outside it: the pages' worked example and
+printed numbers, closed forms, invariants, brute force on tiny inputs and library
+routines.  Each test is chosen so that a plausible mistake (dropped term, wrong
+sign or index, transposed operand) in the oracle fails it.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import golden_path
+from oracle import dg_oracle as O
+from block_diffusion_lm_masked_b200 import roofline as R
+from block_diffusion_lm_masked_b200 import synth
+
+
+def _read_golden(name):
+    rows = []
+    with open(golden_path(name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ---------------------------------------------------------------- mask
+
+def test_block_mask_matches_worked_example():
+    """The printed 7x7 prefix/block mask (P=3 prefix rows, 4 block rows)."""
+    want = np.array([[int(v) for v in r] for r in _read_golden("block_mask_p3_c4.txt")], dtype=bool)
+    assert want.shape == (7, 7)
+    np.testing.assert_array_equal(O.block_mask(3, 4), want)
+
+
+def test_causal_rows_are_prefix_rows_of_mask():
+    # prefill of T tokens after P cached ones = the causal rows P..P+T-1 of a mask with no block
+    full = O.block_mask(9, 0)
+    np.testing.assert_array_equal(O.causal_rows(4, 5), full[4:9, :9])
+
+
+# ---------------------------------------------------------------- RNG
+
+def test_splitmix64_known_answers():
+    want = [int(r[0], 16) for r in _read_golden("splitmix64_seed0.txt")]
+    assert [O.splitmix64(0, i) for i in range(3)] == want
+    # the input generator's own implementation agrees with the published values too
+    got = synth.splitmix64(0, np.arange(3, dtype=np.uint64))
+    assert [int(v) for v in got] == want
+
+
+def test_renoise_tokens_uniform_chi2():
+    V, n = 64, 64 * 400
+    draws = [O.renoise_token(1236, s, p, V) for s in range(4) for p in range(n // 4)]
+    counts = np.bincount(draws, minlength=V)
+    exp = n / V
+    chi2 = ((counts - exp) ** 2 / exp).sum()
+    # 63 degrees of freedom: mean 63, sd ~11.2; 130 is > 6 sd out
+    assert chi2 < 130
+    assert min(draws) >= 0 and max(draws) < V
+
+
+def test_renoise_tokens_in_range_for_non_power_of_two():
+    V = 1000
+    toks = [O.renoise_token(7, 3, p, V) for p in range(5000)]
+    assert 0 <= min(toks) and max(toks) < V
+    assert len(set(toks)) > 900
+
+
+# ---------------------------------------------------------------- rounding
+
+def test_round_bf16_ties_and_library():
+    assert O.round_bf16(np.array([1.0]))[0] == 1.0
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0                    # tie -> even
+    assert O.round_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6    # tie -> even (up)
+    assert O.round_bf16(np.array([-1.0 - 2.0 ** -8 - 2.0 ** -20]))[0] == -1.0 - 2.0 ** -7
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x.astype(np.float64)), lib)
+
+
+def test_widen_bf16_bits():
+    bits = np.array([0x3F80, 0xBF80, 0x4049, 0x0000], dtype=np.uint16)
+    np.testing.assert_array_equal(O.widen(bits), [1.0, -1.0, 3.140625, 0.0])
+
+
+# ---------------------------------------------------------------- norms, rope, silu
+
+def test_rms_norm_closed_forms():
+    x = np.full((1, 8), 3.0)
+    np.testing.assert_allclose(O.rms_norm(x, 1e-6), 3.0 / np.sqrt(9.0 + 1e-6), rtol=1e-15)
+    rng = np.random.default_rng(1)
+    y = O.rms_norm(rng.standard_normal((5, 64)) * 7.0, 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-12)
+
+
+def test_rope_closed_form_and_relative_position():
+    # d = 2: the single pair rotates by the position itself
+    x = np.array([[[1.0, 0.0]]] * 1)
+    for pos in (0, 1, 5):
+        r = O.rope(x, np.array([pos]), 10000.0)
+        np.testing.assert_allclose(r[0, 0], [math.cos(pos), math.sin(pos)], atol=1e-15)
+    # pair i rotates at theta^(-2i/d); rotate-half pairs (i, i + d/2)
+    d, theta = 8, 100.0
+    e = np.zeros((1, 1, d))
+    e[0, 0, 1] = 1.0
+    r = O.rope(e, np.array([3]), theta)[0, 0]
+    ang = 3 * theta ** (-2.0 / d)
+    np.testing.assert_allclose(r[[1, 1 + d // 2]], [math.cos(ang), math.sin(ang)], atol=1e-14)
+    assert np.abs(np.delete(r, [1, 1 + d // 2])).max() == 0.0
+    # dot products depend on the position difference only, norms are preserved
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((1, 1, 16))
+    k = rng.standard_normal((1, 1, 16))
+    dots = [float(O.rope(q, np.array([m]), 1e4)[0, 0] @ O.rope(k, np.array([m - 3]), 1e4)[0, 0])
+            for m in (3, 10, 77, 1000)]
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-9)
+    np.testing.assert_allclose(np.linalg.norm(O.rope(q, np.array([12345]), 1e4)), np.linalg.norm(q), rtol=1e-12)
+
+
+def test_silu_closed_forms():
+    np.testing.assert_allclose(O.silu(np.array([0.0, 50.0, -50.0, 1.0])),
+                               [0.0, 50.0, -50.0 * math.exp(-50.0) / (1 + math.exp(-50.0)), 1 / (1 + math.exp(-1))],
+                               rtol=1e-12, atol=1e-300)
+
+
+# ---------------------------------------------------------------- attention
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(3)
+    d = 16
+    # all keys equal -> uniform weights -> mean of the allowed values
+    q = rng.standard_normal((1, 2, d))
+    k = np.tile(rng.standard_normal((1, 1, d)), (1, 5, 1))
+    v = rng.standard_normal((1, 5, d))
+    allowed = np.array([[1, 1, 1, 0, 0], [1, 1, 1, 1, 1]], dtype=bool)
+    o = O.attention(q, k, v, allowed)
+    np.testing.assert_allclose(o[0, 0], v[0, :3].mean(axis=0), rtol=1e-12)
+    np.testing.assert_allclose(o[0, 1], v[0].mean(axis=0), rtol=1e-12)
+    # one allowed key -> that value
+    o1 = O.attention(q, rng.standard_normal((1, 5, d)), v, np.eye(2, 5, 2, dtype=bool))
+    np.testing.assert_allclose(o1[0, 0], v[0, 2], rtol=1e-12)
+    np.testing.assert_allclose(o1[0, 1], v[0, 3], rtol=1e-12)
+
+
+def test_attention_two_keys_logistic_scale():
+    d = 4
+    q = np.zeros((1, 1, d)); q[0, 0, 0] = 1.0
+    k = np.zeros((1, 2, d)); k[0, 0, 0] = 3.0; k[0, 1, 0] = -1.0
+    v = np.zeros((1, 2, d)); v[0, 0, 1] = 1.0; v[0, 1, 2] = 1.0
+    o = O.attention(q, k, v, np.ones((1, 2), dtype=bool))
+    p0 = 1.0 / (1.0 + math.exp((-1.0 - 3.0) / math.sqrt(d)))
+    np.testing.assert_allclose(o[0, 0], [0.0, p0, 1 - p0, 0.0], rtol=1e-12)
+
+
+def test_attention_gqa_head_mapping():
+    # 4 query heads, 2 kv heads: heads 0,1 read kv 0; heads 2,3 read kv 1 (contiguous groups)
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((4, 3, 8))
+    k = rng.standard_normal((2, 6, 8))
+    v = np.zeros((2, 6, 8)); v[0] += 1.5; v[1] -= 2.5
+    o = O.attention(q, k, v, np.ones((3, 6), dtype=bool))
+    np.testing.assert_allclose(o[:2], 1.5, rtol=1e-12)
+    np.testing.assert_allclose(o[2:], -2.5, rtol=1e-12)
+
+
+def test_attention_block_rows_bidirectional_prefix_rows_causal():
+    rng = np.random.default_rng(5)
+    P, C, d = 3, 4, 8
+    q = rng.standard_normal((1, P + C, d)); k = rng.standard_normal((1, P + C, d)); v = rng.standard_normal((1, P + C, d))
+    m = O.block_mask(P, C)
+    base = O.attention(q, k, v, m)
+    # perturbing the last block key changes every block row but no prefix row
+    k2 = k.copy(); k2[0, -1] += 1.0
+    pert = O.attention(q, k2, v, m)
+    np.testing.assert_array_equal(pert[0, :P], base[0, :P])
+    assert np.all(np.abs(pert[0, P:] - base[0, P:]).max(axis=1) > 0)
+    # permuting block keys/values together leaves block rows unchanged (bidirectional, no order)
+    perm = np.concatenate([np.arange(P), P + rng.permutation(C)])
+    np.testing.assert_allclose(O.attention(q, k[:, perm], v[:, perm], m)[0, P:], base[0, P:], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- router / permutation
+
+def test_router_topk_brute_force_subsets():
+    rng = np.random.default_rng(6)
+    for E, k in ((6, 2), (7, 3), (5, 1)):
+        logits = rng.standard_normal((20, E))
+        idx, w, margin = O.router_topk(logits, k)
+        for t in range(20):
+            best = max(itertools.combinations(range(E), k), key=lambda s: sum(logits[t, list(s)]))
+            assert set(idx[t]) == set(best)
+            srt = sorted(logits[t], reverse=True)
+            assert margin[t] == pytest.approx(srt[k - 1] - srt[k])
+            ch = logits[t, idx[t]]
+            assert list(ch) == sorted(ch, reverse=True)
+            np.testing.assert_allclose(w[t], np.exp(ch) / np.exp(ch).sum(), rtol=1e-12)
+
+
+def test_router_topk_special_cases():
+    lg = np.array([[0.3, -1.0, 2.0, 0.5]])
+    idx, w, _ = O.router_topk(lg, 4)           # k = E: dense mixture = full softmax
+    np.testing.assert_allclose(w[0], np.exp(lg[0, idx[0]]) / np.exp(lg[0]).sum(), rtol=1e-12)
+    idx1, w1, _ = O.router_topk(lg, 1)         # k = 1: single expert, weight 1
+    assert idx1[0, 0] == 2 and w1[0, 0] == 1.0
+    idxt, _, mt = O.router_topk(np.zeros((1, 5)), 2)   # all tied: lowest ids
+    assert list(idxt[0]) == [0, 1] and mt[0] == 0.0
+
+
+def test_expert_permutation_invariants():
+    rng = np.random.default_rng(7)
+    T, k, E = 37, 3, 9
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    counts, offsets, perm, inv, union = O.expert_permutation(idx, E)
+    assert counts.sum() == T * k
+    assert sorted(perm.tolist()) == list(range(T * k))
+    assert union == len({int(e) for e in idx.reshape(-1)})
+    assert k <= union <= min(E, T * k)
+    flat = idx.reshape(-1)
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert all(flat[a] == e for a in seg)
+        assert list(seg) == sorted(seg)        # (token, slot) ascending within an expert
+    np.testing.assert_array_equal(perm[inv], np.arange(T * k))
+
+
+# ---------------------------------------------------------------- MoE
+
+def _tiny_cfg(**over):
+    cfg = dict(n_layers=1, hidden=16, n_q_heads=2, n_kv_heads=1, head_dim=8, n_experts=4, top_k=2,
+               expert_ffn=12, vocab=40, rope_theta=10000.0, rms_eps=1e-6, dtype="f32")
+    cfg.update(over)
+    return cfg
+
+
+class _M:
+    def __init__(self, cfg, seed=11):
+        rng = np.random.default_rng(seed)
+        H, nq, nkv, d, E, F, V = (cfg[x] for x in ("hidden", "n_q_heads", "n_kv_heads", "head_dim",
+                                                   "n_experts", "expert_ffn", "vocab"))
+        self.cfg = cfg
+        self.embed = rng.standard_normal((V, H)) * 0.5
+        self.w_out = rng.standard_normal((V, H)) * 0.3
+        self.layers = [dict(w_q=rng.standard_normal((nq * d, H)) * 0.3, w_k=rng.standard_normal((nkv * d, H)) * 0.3,
+                            w_v=rng.standard_normal((nkv * d, H)) * 0.3, w_o=rng.standard_normal((H, nq * d)) * 0.3,
+                            w_router=rng.standard_normal((E, H)), w_gate=rng.standard_normal((E, F, H)) * 0.3,
+                            w_up=rng.standard_normal((E, F, H)) * 0.3, w_down=rng.standard_normal((E, H, F)) * 0.3)
+                       for _ in range(cfg["n_layers"])]
+
+
+def _swiglu(x, wg, wu, wd):
+    g = x @ wg.T
+    return ((g / (1 + np.exp(-g))) * (x @ wu.T)) @ wd.T
+
+
+def test_moe_identical_experts_equals_dense_swiglu():
+    cfg = _tiny_cfg()
+    m = _M(cfg)
+    L = m.layers[0]
+    for e in range(1, cfg["n_experts"]):
+        L["w_gate"][e] = L["w_gate"][0]; L["w_up"][e] = L["w_up"][0]; L["w_down"][e] = L["w_down"][0]
+    x = np.random.default_rng(8).standard_normal((9, cfg["hidden"]))
+    xn = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + cfg["rms_eps"])
+    got = O.moe(m, 0, x, O.Precision("f32"))
+    np.testing.assert_allclose(got, _swiglu(xn, L["w_gate"][0], L["w_up"][0], L["w_down"][0]), rtol=1e-12, atol=1e-13)
+
+
+def test_moe_k1_routes_each_token_to_its_argmax_expert():
+    cfg = _tiny_cfg(top_k=1)
+    m = _M(cfg)
+    L = m.layers[0]
+    x = np.random.default_rng(9).standard_normal((7, cfg["hidden"]))
+    xn = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + cfg["rms_eps"])
+    got = O.moe(m, 0, x, O.Precision("f32"))
+    for t in range(7):
+        e = int(np.argmax(xn[t] @ L["w_router"].T))
+        want = _swiglu(xn[t:t + 1], L["w_gate"][e], L["w_up"][e], L["w_down"][e])[0]
+        np.testing.assert_allclose(got[t], want, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- whole pass
+
+def test_single_token_pass_closed_form():
+    """C=1, empty cache, one expert: attention over one key returns its value, so the
+    pass reduces to plain matrix products written out here."""
+    cfg = _tiny_cfg(n_experts=1, top_k=1, n_q_heads=2, n_kv_heads=1)
+    m = _M(cfg)
+    L = m.layers[0]
+    tok = np.array([17])
+    logits, _ = O.denoise_pass(m, O.Cache.empty(cfg), tok, O.Precision("f32"))
+    eps = cfg["rms_eps"]
+    nrm = lambda z: z / np.sqrt(np.mean(z * z) + eps)
+    x = m.embed[17].copy()
+    v = nrm(x) @ L["w_v"].T                     # one kv head, position 0 (no rotation of v)
+    x = x + np.concatenate([v, v]) @ L["w_o"].T   # both query heads read that kv head
+    x = x + _swiglu(nrm(x)[None], L["w_gate"][0], L["w_up"][0], L["w_down"][0])[0]
+    np.testing.assert_allclose(logits[0], nrm(x) @ m.w_out.T, rtol=1e-11, atol=1e-12)
+
+
+def test_zero_mixing_weights_pass_is_embedding_readout():
+    cfg = _tiny_cfg(n_layers=2)
+    m = _M(cfg)
+    for L in m.layers:
+        L["w_o"][:] = 0.0
+        L["w_down"][:] = 0.0
+    toks = np.array([3, 9, 3, 27, 0])
+    cache = O.Cache([(np.random.default_rng(1).standard_normal((1, 6, 8)),) * 2] * 2)
+    logits, _ = O.denoise_pass(m, cache, toks, O.Precision("f32"))
+    e = m.embed[toks]
+    np.testing.assert_allclose(logits, (e / np.sqrt(np.mean(e * e, axis=1, keepdims=True) + 1e-6)) @ m.w_out.T,
+                               rtol=1e-12)
+
+
+def test_prefix_kv_reuse_equals_full_recompute():
+    """The cached path (causal prefill of the prefix, then a denoising pass against the
+    cache) equals recomputing prefix and block together under the prefix/block mask."""
+    cfg = _tiny_cfg(n_layers=2)
+    m = _M(cfg)
+    pre = np.array([5, 1, 33, 8, 20, 2])
+    can = np.array([11, 39, 0, 7])
+    prec = O.Precision("f32")
+    cache = O.prefill_append(m, O.Cache.empty(cfg), pre, prec)
+    logits, _ = O.denoise_pass(m, cache, can, prec)
+    ks, vs, full_logits = O.full_sequence_states(m, pre, can, prec)
+    P = len(pre)
+    for l in range(cfg["n_layers"]):
+        np.testing.assert_allclose(cache.k[l], ks[l][:, :P], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(cache.v[l], vs[l][:, :P], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(logits, full_logits, rtol=1e-10, atol=1e-11)
+
+
+def test_chunked_prefill_equals_single_prefill():
+    cfg = _tiny_cfg(n_layers=2)
+    m = _M(cfg)
+    toks = np.array([4, 8, 15, 16, 23, 42 % 40, 1, 2])
+    prec = O.Precision("bf16")
+    one = O.prefill_append(m, O.Cache.empty(cfg), toks, prec)
+    two = O.prefill_append(m, O.prefill_append(m, O.Cache.empty(cfg), toks[:3], prec), toks[3:], prec)
+    for l in range(2):
+        np.testing.assert_allclose(two.k[l], one.k[l], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(two.v[l], one.v[l], rtol=1e-12, atol=1e-13)
+
+
+def test_denoise_pass_leaves_cache_untouched():
+    cfg = _tiny_cfg()
+    m = _M(cfg)
+    cache = O.prefill_append(m, O.Cache.empty(cfg), np.array([1, 2, 3]), O.Precision("f32"))
+    before = cache.copy()
+    O.denoise_pass(m, cache, np.array([4, 5]), O.Precision("f32"))
+    for l in range(cfg["n_layers"]):
+        np.testing.assert_array_equal(cache.k[l], before.k[l])
+        np.testing.assert_array_equal(cache.v[l], before.v[l])
+
+
+# ---------------------------------------------------------------- canvas update
+
+def test_canvas_update_special_cases():
+    rng = np.random.default_rng(10)
+    C, V = 12, 50
+    lg = rng.standard_normal((C, V))
+    u0 = O.canvas_update(lg, 0, 99, 0)
+    np.testing.assert_array_equal(u0["canvas"], np.argmax(lg, axis=1))
+    uc = O.canvas_update(lg, C, 99, 5)
+    np.testing.assert_array_equal(uc["canvas"], [O.renoise_token(99, 5, i, V) for i in range(C)])
+    # confidence closed form: one logit a, the rest 0
+    lg2 = np.zeros((2, V)); lg2[0, 3] = 2.0; lg2[1, 7] = 40.0
+    u2 = O.canvas_update(lg2, 0, 1, 0)
+    np.testing.assert_allclose(u2["conf"][0], math.exp(2.0) / (math.exp(2.0) + V - 1), rtol=1e-14)
+    assert u2["conf"][1] == pytest.approx(1.0, abs=1e-15)
+    assert list(u2["argmax"]) == [3, 7]
+    # ties: argmax takes the lowest id; equal confidences re-noise lower positions first
+    u3 = O.canvas_update(np.zeros((4, 6)), 2, 1, 0)
+    assert list(u3["argmax"]) == [0, 0, 0, 0] and list(u3["renoised"]) == [0, 1]
+
+
+def test_canvas_update_renoise_set_brute_force():
+    rng = np.random.default_rng(11)
+    C, V, n = 30, 20, 11
+    lg = rng.standard_normal((C, V)) * 2
+    u = O.canvas_update(lg, n, 5, 3)
+    conf = [math.exp(max(r)) / sum(math.exp(x) for x in r) for r in lg.tolist()]
+    want = sorted(sorted(range(C), key=lambda i: (conf[i], i))[:n])
+    assert list(u["renoised"]) == want
+    keep = [i for i in range(C) if i not in want]
+    assert all(u["canvas"][i] == int(np.argmax(lg[i])) for i in keep)
+    assert all(u["cut_margin"] >= 0)
+
+
+def test_renoise_schedule_golden():
+    g = {r[0]: [int(v) for v in r[1:]] for r in _read_golden("renoise_schedule.txt")}
+    assert [O.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]
+    assert [O.renoise_count(256, 8, s, 0.5, 0.0) for s in range(8)] == g["S8"]
+    assert O.renoise_count(256, 1, 0, 0.25, 0.25) == g["S1_C256_q25"][0]
+    assert O.renoise_count(32, 1, 0, 0.25, 0.25) == g["S1_C32_q25"][0]
+
+
+# ---------------------------------------------------------------- roofline calculator
+
+def test_roofline_reproduces_exercise_arithmetic():
+    g = {r[0]: float(r[1]) for r in _read_golden("roofline_h100_model.txt")}
+    bw, peak = 3.35e12, 990e12
+    assert R.dense_weight_read_s(8e9, 2, bw) * 1e3 == pytest.approx(g["weight_read_bf16_ms"], abs=5e-4)
+    assert R.dense_weight_read_s(8e9, 0.5, bw) * 1e3 == pytest.approx(g["weight_read_4bit_ms"], abs=5e-4)
+    assert 2 * 8e9 * 256 / peak * 1e3 == pytest.approx(g["compute_floor_256_ms"], abs=5e-4)
+    ar = R.dense_pass_s(8e9, 1, 2, bw, peak)
+    assert ar == pytest.approx(g["ar_pass_s"], rel=1e-6)
+    assert 1.0 / ar == pytest.approx(g["ar_ceiling_tok_s"], rel=1e-6)
+    t1024 = R.dense_pass_s(8e9, 1024, 2, bw, peak)     # compute-bound: the larger bound wins
+    assert t1024 == pytest.approx(g["diffusion_pass_1024_s"], rel=1e-6)
+    s = R.breakeven_steps(1024, t1024, 1.0 / ar)
+    assert s == pytest.approx(g["breakeven_steps"], abs=5e-3)
+    assert math.floor(s) == int(g["max_steps"])

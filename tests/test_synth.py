@@ -1,0 +1,31 @@
+"""The seeded input generator: determinism, chunking independence, distribution."""
+import numpy as np
+
+from block_diffusion_lm_masked_b200 import synth
+from oracle import dg_oracle as O
+
+
+def test_normal_is_deterministic_and_chunk_independent(monkeypatch):
+    a = synth.normal(5, 77, (3000,), 0.02, "bf16")
+    monkeypatch.setattr(synth, "_CHUNK", 257)
+    b = synth.normal(5, 77, (3000,), 0.02, "bf16")
+    np.testing.assert_array_equal(a, b)
+    c = synth.normal(5, 78, (3000,), 0.02, "bf16")
+    assert (a != c).mean() > 0.9
+
+
+def test_normal_moments_and_bf16_exactness():
+    f = synth.normal(1234, 9, (200000,), 0.02, "f32").astype(np.float64)
+    assert abs(f.mean()) < 3 * 0.02 / np.sqrt(2e5)
+    assert abs(f.std() - 0.02) < 0.02 * 0.01
+    bits = synth.normal(1234, 9, (200000,), 0.02, "bf16")
+    wide = O.widen(bits)
+    np.testing.assert_array_equal(O.round_bf16(f), O.round_bf16(wide))   # same draws, bf16-representable
+    assert np.abs(wide - f).max() <= 0.02 * 6 * 2.0 ** -8
+
+
+def test_tokens_uniform_in_range():
+    t = synth.tokens(1235, 3, 100000, 1000)
+    assert t.min() >= 0 and t.max() < 1000
+    cnt = np.bincount(t, minlength=1000)
+    assert cnt.min() > 40 and cnt.max() < 170
