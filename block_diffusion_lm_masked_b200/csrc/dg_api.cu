@@ -1,0 +1,751 @@
+// C-ABI of libdg: validation, workspace carving, TMA tensor-map encoding and the
+// launch sequences of the prefill, denoising pass, canvas update and canvas
+// generation (declared in include/dg.h and include/dg_debug.h).
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "../../include/dg_debug.h"
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+using dg::bf16;
+
+// ---------------------------------------------------------------- errors
+static thread_local std::string g_err;
+static dg_status fail(dg_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+#define DG_CHECK_ARG(cond, ...) \
+  do {                          \
+    if (!(cond)) return fail(DG_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+// ---------------------------------------------------------------- profiling
+namespace {
+struct ProfPair {
+  cudaEvent_t a, b;
+  int kind;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfPair> g_prof_pending;
+std::vector<ProfPair> g_prof_free;
+double g_prof_ms[DG_K_COUNT];
+int g_prof_n[DG_K_COUNT];
+int64_t g_launches = 0;
+
+void prof_flush_locked() {
+  for (auto& p : g_prof_pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+      g_prof_ms[p.kind] += ms;
+      g_prof_n[p.kind] += 1;
+    }
+    g_prof_free.push_back(p);
+  }
+  g_prof_pending.clear();
+}
+
+struct ProfScope {
+  ProfPair pair{};
+  bool on = false;
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_launches++;
+    if (!g_prof_on) return;
+    if (g_prof_pending.size() >= 8192) prof_flush_locked();
+    if (!g_prof_free.empty()) {
+      pair = g_prof_free.back();
+      g_prof_free.pop_back();
+    } else {
+      if (cudaEventCreate(&pair.a) != cudaSuccess || cudaEventCreate(&pair.b) != cudaSuccess) return;
+    }
+    pair.kind = kind;
+    on = cudaEventRecord(pair.a, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (cudaEventRecord(pair.b, st) == cudaSuccess) g_prof_pending.push_back(pair);
+  }
+};
+}  // namespace
+
+#define LAUNCH(kind, st, call)                                                                          \
+  do {                                                                                                  \
+    cudaError_t _e;                                                                                     \
+    {                                                                                                   \
+      ProfScope _ps((kind), (st));                                                                      \
+      _e = (call);                                                                                      \
+    }                                                                                                   \
+    if (_e != cudaSuccess) return fail(DG_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(_e));          \
+  } while (0)
+
+// ---------------------------------------------------------------- tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static dg_status get_encoder() {
+  if (g_encode) return DG_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || fn == nullptr || q != cudaDriverEntryPointSuccess)
+    return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(e));
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return DG_OK;
+}
+
+// bf16 tensor, up to 3 dims (dims[0] innermost), 128-byte swizzle
+static dg_status encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                             const uint64_t* strides_bytes /* rank-1 entries */, const uint32_t* box) {
+  if (get_encoder() != DG_OK) return DG_ERR_CUDA;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) gd[i] = dims[i], bx[i] = box[i];
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx,
+                        es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DG_OK;
+}
+// row-major [rows][cols] bf16 matrix as a 2-D map with box (64 cols, box_rows rows)
+static dg_status map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return encode_bf16(m, base, 2, dims, strides, box);
+}
+
+// ---------------------------------------------------------------- model
+struct LayerMaps {
+  CUtensorMap qkv, o, gate_up, down;
+};
+struct dg_model {
+  dg_config cfg;
+  const void* embed;
+  const void* w_out;
+  std::vector<dg_layer_weights> layers;
+  std::vector<LayerMaps> maps;
+  CUtensorMap out_map;
+  bool taps_on = false;
+  std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
+  std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
+  int32_t* tap_unions = nullptr;
+};
+
+static bool is_bf16(const dg_config& c) { return c.dtype == DG_DTYPE_BF16; }
+static size_t act_bytes(const dg_config& c) { return is_bf16(c) ? 2 : 4; }
+static int qkv_rows(const dg_config& c) { return (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim; }
+
+static dg_status validate_config(const dg_config* c) {
+  DG_CHECK_ARG(c, "config is NULL");
+  DG_CHECK_ARG(c->n_layers >= 1 && c->hidden > 0 && c->n_q_heads > 0 && c->n_kv_heads > 0 && c->head_dim > 0 &&
+                   c->n_experts > 0 && c->top_k > 0 && c->expert_ffn > 0 && c->vocab > 0,
+               "config sizes must be positive");
+  DG_CHECK_ARG(c->dtype == DG_DTYPE_BF16 || c->dtype == DG_DTYPE_F32, "dtype must be DG_DTYPE_BF16 or DG_DTYPE_F32");
+  DG_CHECK_ARG(c->n_q_heads % c->n_kv_heads == 0, "n_q_heads %% n_kv_heads != 0");
+  DG_CHECK_ARG(c->top_k <= c->n_experts && c->top_k <= 16, "top_k must be <= min(16, n_experts)");
+  DG_CHECK_ARG(c->n_experts <= 256, "n_experts must be <= 256");
+  DG_CHECK_ARG(c->hidden % 64 == 0 && c->expert_ffn % 64 == 0, "hidden and expert_ffn must be multiples of 64");
+  DG_CHECK_ARG(c->head_dim % 2 == 0 && c->head_dim <= 128, "head_dim must be even and <= 128");
+  DG_CHECK_ARG(c->vocab % 4 == 0, "vocab must be a multiple of 4");
+  DG_CHECK_ARG(c->rms_eps >= 0.f && c->rope_theta > 0.f, "bad rms_eps / rope_theta");
+  if (is_bf16(*c)) {
+    DG_CHECK_ARG(c->head_dim == 128, "bf16 model: head_dim must be 128");
+    DG_CHECK_ARG(c->vocab % 128 == 0, "bf16 model: vocab must be a multiple of 128");
+    DG_CHECK_ARG(qkv_rows(*c) % 128 == 0 && c->hidden % 128 == 0, "bf16 model: hidden must be a multiple of 128");
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out) {
+  dg_status s = validate_config(cfg);
+  if (s != DG_OK) return s;
+  DG_CHECK_ARG(w && out && w->embed && w->w_out && w->layers, "weights / out pointer is NULL");
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const dg_layer_weights& L = w->layers[l];
+    DG_CHECK_ARG(L.w_qkv && L.w_o && L.w_router && L.w_gate_up && L.w_down, "layer %d has a NULL weight", l);
+  }
+  dg_model* m = new dg_model();
+  m->cfg = *cfg;
+  m->embed = w->embed;
+  m->w_out = w->w_out;
+  m->layers.assign(w->layers, w->layers + cfg->n_layers);
+  if (is_bf16(*cfg)) {
+    const dg_config& c = *cfg;
+    m->maps.resize(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const dg_layer_weights& L = m->layers[l];
+      LayerMaps& M = m->maps[l];
+      if ((s = map_rows(&M.qkv, L.w_qkv, qkv_rows(c), c.hidden, 128)) != DG_OK ||
+          (s = map_rows(&M.o, L.w_o, c.hidden, (uint64_t)c.n_q_heads * c.head_dim, 128)) != DG_OK ||
+          (s = map_rows(&M.gate_up, L.w_gate_up, (uint64_t)c.n_experts * 2 * c.expert_ffn, c.hidden, 128)) != DG_OK ||
+          (s = map_rows(&M.down, L.w_down, (uint64_t)c.n_experts * c.hidden, c.expert_ffn, 128)) != DG_OK) {
+        delete m;
+        return s;
+      }
+    }
+    if ((s = map_rows(&m->out_map, m->w_out, c.vocab, c.hidden, 128)) != DG_OK) {
+      delete m;
+      return s;
+    }
+  }
+  *out = m;
+  return DG_OK;
+}
+
+extern "C" void dg_model_destroy(dg_model* m) { delete m; }
+
+// ---------------------------------------------------------------- workspace layout
+namespace {
+constexpr int kMaxAttnSplits = 16;
+inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t err, upd, x, xn, qkv, q, o, part_o, part_lse, logits_r, topk_idx, topk_w, counts, offsets, perm, inv, uni, xs,
+      h, gu, ys, total;
+};
+
+size_t upd_bytes(int C, int V) { return al((size_t)C * dg::update_splits(C, V) * sizeof(dg::UpdPart)); }
+
+WsLayout layout(const dg_config& c, int T) {
+  WsLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o += al(bytes);
+    return r;
+  };
+  const size_t ab = act_bytes(c);
+  const size_t H = c.hidden, E = c.n_experts, k = c.top_k, F = c.expert_ffn, d = c.head_dim;
+  L.err = take(256);
+  size_t upd_max = 0;
+  for (int C = 1; C <= T; ++C) upd_max = upd_max > upd_bytes(C, c.vocab) ? upd_max : upd_bytes(C, c.vocab);
+  L.upd = take(upd_max);
+  L.x = take((size_t)T * H * 4);
+  L.xn = take((size_t)T * H * ab);
+  L.qkv = take((size_t)T * qkv_rows(c) * 4);
+  L.q = take((size_t)c.n_q_heads * T * d * ab);
+  L.o = take((size_t)T * c.n_q_heads * d * ab);
+  L.part_o = take(is_bf16(c) ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
+  L.part_lse = take(is_bf16(c) ? (size_t)kMaxAttnSplits * c.n_q_heads * T * 4 : 0);
+  L.logits_r = take((size_t)T * E * 4);
+  L.topk_idx = take((size_t)T * k * 4);
+  L.topk_w = take((size_t)T * k * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.perm = take((size_t)T * k * 4);
+  L.inv = take((size_t)T * k * 4);
+  L.uni = take(4);
+  L.xs = take((size_t)T * k * H * ab);
+  L.h = take((size_t)T * k * F * ab);
+  L.gu = take(is_bf16(c) ? 0 : (size_t)T * k * 2 * F * 4);
+  L.ys = take((size_t)T * k * H * 4);
+  L.total = o;
+  return L;
+}
+
+struct Ws {
+  char* base;
+  WsLayout L;
+  template <typename P>
+  P* at(size_t off) const {
+    return reinterpret_cast<P*>(base + off);
+  }
+  int* err() const { return at<int>(L.err); }
+};
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+}  // namespace
+
+extern "C" size_t dg_workspace_bytes(const dg_config* cfg, int32_t max_tokens) {
+  if (validate_config(cfg) != DG_OK || max_tokens <= 0) return 0;
+  return layout(*cfg, max_tokens).total;
+}
+extern "C" size_t dg_update_workspace_bytes(int32_t C, int32_t V) {
+  if (C <= 0 || V <= 0) return 0;
+  return 256 + upd_bytes(C, V);
+}
+
+// ---------------------------------------------------------------- the layer stack
+namespace {
+
+// GEMM smem budget: about half the SM so that two CTAs can share it
+constexpr int kGemmSmem = 100 * 1024;
+
+dg_status gemm_bf16(int kind, int epi, const CUtensorMap& A, const void* X, int x_rows, int K, int a_rows_per_group,
+                    int n_groups, const int* group_off, int max_rows_per_group, void* out, int ld_out, int* err,
+                    cudaStream_t st) {
+  CUtensorMap B;
+  dg_status s = map_rows(&B, X, (uint64_t)x_rows, (uint64_t)K, 16);
+  if (s != DG_OK) return s;
+  dg::TcGemmParams p;
+  p.K = K;
+  p.a_rows_per_group = a_rows_per_group;
+  p.group_off = group_off;
+  p.n_tokens = x_rows;
+  p.out = out;
+  p.ld_out = ld_out;
+  p.smem_budget = kGemmSmem;
+  p.err = err;
+  const int m_tiles = (epi == dg::EPI_SWIGLU_BF16) ? a_rows_per_group / 128 : a_rows_per_group / 128;
+  LAUNCH(kind, st, dg::launch_tc_gemm(epi, A, B, p, m_tiles, n_groups, max_rows_per_group, st));
+  return DG_OK;
+}
+
+int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
+  const int nch = ceil_div(n_keys, 128);
+  const int base = ceil_div(n_q, 128) * nq;
+  int splits = ceil_div(2 * 148, base);
+  if (splits > kMaxAttnSplits) splits = kMaxAttnSplits;
+  if (splits > ceil_div(nch, 2)) splits = ceil_div(nch, 2);
+  if (splits < 1) splits = 1;
+  *chunks_per_split = ceil_div(nch, splits);
+  splits = ceil_div(nch, *chunks_per_split);
+  return splits;
+}
+
+// attention of n_q new rows at positions pos0.. over cache keys [0, n_keys)
+dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0, int n_keys,
+                    int causal, cudaStream_t st) {
+  const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
+  if (!is_bf16(c)) {
+    LAUNCH(DG_K_ATTENTION, st,
+           dg::launch_simt_attention_f32(ws.at<float>(ws.L.q), (const float*)kc, (const float*)vtc, cap, n_q, pos0,
+                                         n_keys, causal, nq, nkv, d, ws.at<float>(ws.L.o), st));
+    return DG_OK;
+  }
+  CUtensorMap mq, mk, mv;
+  dg_status s;
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)n_q * d * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mq, ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mk, kc, 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)n_keys, (uint64_t)d, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)cap * 2, (uint64_t)d * cap * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mv, vtc, 3, dims, str, box)) != DG_OK) return s;
+  }
+  dg::TcAttnParams p;
+  p.n_q = n_q;
+  p.q_pos0 = pos0;
+  p.n_keys = n_keys;
+  p.causal = causal;
+  p.group = nq / nkv;
+  p.nq = nq;
+  p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  p.out = ws.at<bf16>(ws.L.o);
+  p.part_o = ws.at<float>(ws.L.part_o);
+  p.part_lse = ws.at<float>(ws.L.part_lse);
+  p.err = ws.err();
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mq, mk, mv, p, st));
+  if (p.n_splits > 1)
+    LAUNCH(DG_K_ATTN_MERGE, st,
+           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<void>(ws.L.o), 1, st));
+  return DG_OK;
+}
+
+// one transformer layer over n rows at positions pos0.. whose residual is in ws.x.
+// stop_after_kv: write this layer's K/V and return (last layer of a prefill).
+template <typename T>
+dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, int n, int pos0, int causal,
+                bool stop_after_kv, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& W = m->layers[l];
+  const int H = c.hidden, nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
+  const int E = c.n_experts, k = c.top_k, F = c.expert_ffn;
+  const bool bf = is_bf16(c);
+  int* err = ws.err();
+  dg_status s;
+  // attention block: RMSNorm -> QKV -> RoPE (+ K/V into the cache) -> attention -> O + residual
+  LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<T>(ws.at<float>(ws.L.x), n, H, c.rms_eps, ws.at<T>(ws.L.xn), st));
+  if (bf) {
+    if ((s = gemm_bf16(DG_K_GEMM_QKV, dg::EPI_STORE_F32, m->maps[l].qkv, ws.at<void>(ws.L.xn), n, H, qkv_rows(c), 1,
+                       nullptr, n, ws.at<float>(ws.L.qkv), qkv_rows(c), err, st)) != DG_OK)
+      return s;
+  } else {
+    LAUNCH(DG_K_GEMM_QKV, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_qkv, ws.at<float>(ws.L.xn), nullptr, 1, n, n, qkv_rows(c),
+                                    H, ws.at<float>(ws.L.qkv), qkv_rows(c), st));
+  }
+  LAUNCH(DG_K_ROPE_KV, st,
+         dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), n, nq, nkv, d, pos0, c.rope_theta, ws.at<T>(ws.L.q),
+                                    (T*)kc, (T*)vtc, cap, st));
+  if (stop_after_kv) return DG_OK;
+  if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
+  if (bf) {
+    if ((s = gemm_bf16(DG_K_GEMM_O, dg::EPI_ADD_F32, m->maps[l].o, ws.at<void>(ws.L.o), n, nq * d, H, 1, nullptr, n,
+                       ws.at<float>(ws.L.x), H, err, st)) != DG_OK)
+      return s;
+  } else {
+    LAUNCH(DG_K_GEMM_O, st,
+           dg::launch_simt_gemm_f32(1, (const float*)W.w_o, ws.at<float>(ws.L.o), nullptr, 1, n, n, H, nq * d,
+                                    ws.at<float>(ws.L.x), H, st));
+  }
+  if (m->taps_on && !m->tap_x_attn.empty() && m->tap_x_attn[l])
+    if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return fail(DG_ERR_CUDA, "tap copy failed");
+  // MoE block: router (fp32) -> top-k -> histogram/permutation -> gather -> experts -> combine
+  LAUNCH(DG_K_ROUTER, st,
+         dg::launch_router<T>(ws.at<float>(ws.L.x), W.w_router, n, H, E, c.rms_eps, ws.at<float>(ws.L.logits_r),
+                              ws.at<T>(ws.L.xn), st));
+  LAUNCH(DG_K_TOPK, st,
+         dg::launch_topk(ws.at<float>(ws.L.logits_r), n, E, k, ws.at<int32_t>(ws.L.topk_idx),
+                         ws.at<float>(ws.L.topk_w), st));
+  LAUNCH(DG_K_PERMUTE, st,
+         dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
+                            ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
+                            ws.at<int32_t>(ws.L.uni), st));
+  LAUNCH(DG_K_GATHER, st,
+         dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), ws.at<int32_t>(ws.L.perm), n * k, k, H, ws.at<T>(ws.L.xs), st));
+  const int* off = ws.at<int>(ws.L.offsets);
+  if (bf) {
+    if ((s = gemm_bf16(DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, m->maps[l].gate_up, ws.at<void>(ws.L.xs), n * k, H,
+                       2 * F, E, off, n, ws.at<void>(ws.L.h), F, err, st)) != DG_OK)
+      return s;
+    if ((s = gemm_bf16(DG_K_GEMM_DOWN, dg::EPI_STORE_F32, m->maps[l].down, ws.at<void>(ws.L.h), n * k, F, H, E, off,
+                       n, ws.at<float>(ws.L.ys), H, err, st)) != DG_OK)
+      return s;
+  } else {
+    LAUNCH(DG_K_GEMM_GATE_UP, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_gate_up, ws.at<float>(ws.L.xs), off, E, n, n * k, 2 * F, H,
+                                    ws.at<float>(ws.L.gu), 2 * F, st));
+    LAUNCH(DG_K_SWIGLU, st,
+           dg::launch_swiglu_packed_f32(ws.at<float>(ws.L.gu), n * k, F, ws.at<float>(ws.L.h), st));
+    LAUNCH(DG_K_GEMM_DOWN, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_down, ws.at<float>(ws.L.h), off, E, n, n * k, H, F,
+                                    ws.at<float>(ws.L.ys), H, st));
+  }
+  LAUNCH(DG_K_COMBINE, st,
+         dg::launch_combine(ws.at<float>(ws.L.ys), ws.at<int32_t>(ws.L.inv), ws.at<float>(ws.L.topk_w), n, k, H,
+                            ws.at<float>(ws.L.x), st));
+  if (m->taps_on) {
+    auto cp = [&](void* dst, const void* src, size_t bytes) {
+      return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
+    };
+    cudaError_t e = cudaSuccess;
+    if (!m->tap_x_out.empty()) e = cp(m->tap_x_out[l], ws.at<float>(ws.L.x), (size_t)n * H * 4);
+    if (e == cudaSuccess && !m->tap_topk_idx.empty())
+      e = cp(m->tap_topk_idx[l], ws.at<int32_t>(ws.L.topk_idx), (size_t)n * k * 4);
+    if (e == cudaSuccess && !m->tap_topk_w.empty())
+      e = cp(m->tap_topk_w[l], ws.at<float>(ws.L.topk_w), (size_t)n * k * 4);
+    if (e == cudaSuccess && !m->tap_counts.empty()) e = cp(m->tap_counts[l], ws.at<int32_t>(ws.L.counts), E * 4);
+    if (e == cudaSuccess && !m->tap_perm.empty())
+      e = cp(m->tap_perm[l], ws.at<int32_t>(ws.L.perm), (size_t)n * k * 4);
+    if (e == cudaSuccess && m->tap_unions) e = cp(m->tap_unions + l, ws.at<int32_t>(ws.L.uni), 4);
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "tap copy failed: %s", cudaGetErrorString(e));
+  }
+  return DG_OK;
+}
+
+dg_status check_ws(const dg_config& c, void* d_ws, size_t ws_bytes, int n, Ws* ws) {
+  DG_CHECK_ARG(d_ws, "workspace is NULL");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_ws) & 255) == 0, "workspace must be 256-byte aligned");
+  ws->base = static_cast<char*>(d_ws);
+  ws->L = layout(c, n);
+  if (ws_bytes < ws->L.total)
+    return fail(DG_ERR_CAPACITY, "workspace too small: %zu < %zu bytes", ws_bytes, ws->L.total);
+  return DG_OK;
+}
+
+dg_status check_cache(const dg_config& c, const dg_kv_cache* cache) {
+  DG_CHECK_ARG(cache && cache->k && cache->vt, "cache is NULL");
+  DG_CHECK_ARG(cache->capacity > 0 && cache->capacity % 8 == 0, "cache capacity must be a positive multiple of 8");
+  DG_CHECK_ARG(cache->len >= 0 && cache->len <= cache->capacity, "cache len out of range");
+  for (int l = 0; l < c.n_layers; ++l) {
+    DG_CHECK_ARG(cache->k[l] && cache->vt[l], "cache layer %d is NULL", l);
+    DG_CHECK_ARG((reinterpret_cast<uintptr_t>(cache->k[l]) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(cache->vt[l]) & 15) == 0,
+                 "cache buffers must be 16-byte aligned");
+  }
+  return DG_OK;
+}
+
+template <typename T>
+dg_status run_stack(dg_model* m, const dg_kv_cache* cache, const int32_t* tokens, int n, int causal,
+                    bool skip_last_block, const Ws& ws, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int pos0 = cache->len;
+  LAUNCH(DG_K_EMBED_NORM, st,
+         dg::launch_embed_norm<T>(tokens, (const T*)m->embed, n, c.vocab, c.hidden, c.rms_eps, ws.at<float>(ws.L.x),
+                                  ws.at<T>(ws.L.xn), ws.err(), st));
+  for (int l = 0; l < c.n_layers; ++l) {
+    const bool last = (l == c.n_layers - 1) && skip_last_block;
+    dg_status s = layer<T>(m, l, ws, cache->k[l], cache->vt[l], cache->capacity, n, pos0, causal, last, st);
+    if (s != DG_OK) return s;
+  }
+  return DG_OK;
+}
+
+}  // namespace
+
+extern "C" dg_status dg_prefill_append(dg_model* m, dg_kv_cache* cache, const int32_t* d_tokens, int32_t T,
+                                       void* d_ws, size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  DG_CHECK_ARG(d_tokens && T > 0, "tokens NULL or T <= 0");
+  if ((int64_t)cache->len + T > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache overflow: len %d + T %d > capacity %d", cache->len, T, cache->capacity);
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, T, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool saved = m->taps_on;
+  m->taps_on = false;
+  s = is_bf16(m->cfg) ? run_stack<bf16>(m, cache, d_tokens, T, 1, true, ws, st)
+                      : run_stack<float>(m, cache, d_tokens, T, 1, true, ws, st);
+  m->taps_on = saved;
+  if (s != DG_OK) return s;
+  cache->len += T;
+  return DG_OK;
+}
+
+extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, const int32_t* d_canvas, int32_t C,
+                                     float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  DG_CHECK_ARG(d_canvas && d_logits && C > 0, "canvas / logits NULL or C <= 0");
+  if ((int64_t)cache->len + C > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
+                cache->capacity);
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, C, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dg_config& c = m->cfg;
+  s = is_bf16(c) ? run_stack<bf16>(m, cache, d_canvas, C, 0, false, ws, st)
+                 : run_stack<float>(m, cache, d_canvas, C, 0, false, ws, st);
+  if (s != DG_OK) return s;
+  // final RMSNorm + vocabulary projection to fp32 logits
+  if (is_bf16(c)) {
+    LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<bf16>(ws.at<float>(ws.L.x), C, c.hidden, c.rms_eps,
+                                                        ws.at<bf16>(ws.L.xn), st));
+    if ((s = gemm_bf16(DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, m->out_map, ws.at<void>(ws.L.xn), C, c.hidden, c.vocab, 1,
+                       nullptr, C, d_logits, c.vocab, ws.err(), st)) != DG_OK)
+      return s;
+  } else {
+    LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<float>(ws.at<float>(ws.L.x), C, c.hidden, c.rms_eps,
+                                                         ws.at<float>(ws.L.xn), st));
+    LAUNCH(DG_K_GEMM_VOCAB, st,
+           dg::launch_simt_gemm_f32(0, (const float*)m->w_out, ws.at<float>(ws.L.xn), nullptr, 1, C, C, c.vocab,
+                                    c.hidden, d_logits, c.vocab, st));
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t V, int32_t n_renoise, uint64_t seed,
+                                      uint32_t step, int32_t* d_canvas, float* d_conf, void* d_ws, size_t ws_bytes,
+                                      dg_stream stream) {
+  DG_CHECK_ARG(d_logits && d_canvas && d_ws, "logits / canvas / workspace is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(V > 0 && V % 4 == 0, "V must be a positive multiple of 4");
+  DG_CHECK_ARG(n_renoise >= 0 && n_renoise <= C, "n_renoise must be in [0, C]");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_logits) & 15) == 0, "logits must be 16-byte aligned");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_ws) & 255) == 0, "workspace must be 256-byte aligned");
+  if (ws_bytes < dg_update_workspace_bytes(C, V))
+    return fail(DG_ERR_CAPACITY, "workspace too small for the update: %zu < %zu", ws_bytes,
+                dg_update_workspace_bytes(C, V));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dg::UpdPart* part = reinterpret_cast<dg::UpdPart*>(static_cast<char*>(d_ws) + 256);
+  const int splits = dg::update_splits(C, V);
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, part, st));
+  LAUNCH(DG_K_UPDATE_SELECT, st,
+         dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, st));
+  return DG_OK;
+}
+
+static int renoise_count(int C, int S, int s, double r0, double r1) {
+  const double f = (S == 1) ? r0 : (r0 * (S - 1 - s) + r1 * s) / (double)(S - 1);
+  return (int)floor((double)C * f + 1e-9);
+}
+extern "C" int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end) {
+  if (C < 0 || S < 1 || step < 0 || step >= S) return -1;
+  return renoise_count(C, S, step, r_start, r_end);
+}
+
+extern "C" dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t S,
+                                        float r_start, float r_end, uint64_t seed, int32_t append, float* d_logits,
+                                        void* d_ws, size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(S >= 1, "S must be >= 1");
+  DG_CHECK_ARG(r_start >= 0.f && r_start <= 1.f && r_end >= 0.f && r_end <= 1.f, "re-noise fractions must be in [0,1]");
+  DG_CHECK_ARG(C <= 1024, "C must be <= 1024");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  if ((int64_t)cache->len + C > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
+                cache->capacity);
+  for (int step = 0; step < S; ++step) {
+    if ((s = dg_denoise_pass(m, cache, d_canvas, C, d_logits, d_ws, ws_bytes, stream)) != DG_OK) return s;
+    const int n = renoise_count(C, S, step, r_start, r_end);
+    if ((s = dg_canvas_update(d_logits, C, m->cfg.vocab, n, seed, (uint32_t)step, d_canvas, nullptr, d_ws, ws_bytes,
+                              stream)) != DG_OK)
+      return s;
+  }
+  if (append) return dg_prefill_append(m, cache, d_canvas, C, d_ws, ws_bytes, stream);
+  return DG_OK;
+}
+
+extern "C" dg_status dg_pack_gate_up(const void* d_gate, const void* d_up, void* d_out, int32_t E, int32_t F,
+                                     int32_t H, int32_t elem_bytes, dg_stream stream) {
+  DG_CHECK_ARG(d_gate && d_up && d_out, "NULL pointer");
+  DG_CHECK_ARG(E > 0 && F > 0 && H > 0 && F % 64 == 0, "E, F, H must be positive and F a multiple of 64");
+  DG_CHECK_ARG(elem_bytes == 2 || elem_bytes == 4, "elem_bytes must be 2 or 4");
+  DG_CHECK_ARG(((size_t)H * elem_bytes) % 16 == 0, "rows must be a multiple of 16 bytes");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dg::launch_pack_gate_up(d_gate, d_up, d_out, E, F, H, elem_bytes, st);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "pack_gate_up: %s", cudaGetErrorString(e));
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_launches++;
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_device_status(void* d_ws, dg_stream stream) {
+  DG_CHECK_ARG(d_ws, "workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, d_ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(d_ws, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (v == DG_DEVERR_BAD_TOKEN) return fail(DG_ERR_INVALID_ARG, "a token id was outside [0, vocab)");
+    return fail(DG_ERR_TIMEOUT, "device error word %d (a bounded wait gave up)", v);
+  }
+  return DG_OK;
+}
+
+extern "C" const char* dg_last_error(void) { return g_err.c_str(); }
+
+// ---------------------------------------------------------------- debug / profiling
+extern "C" dg_status dg_set_taps(dg_model* m, const dg_taps* t) {
+  DG_CHECK_ARG(m, "model is NULL");
+  const int L = m->cfg.n_layers;
+  auto grab = [&](auto* const* src, auto& dst) {
+    dst.clear();
+    if (src) dst.assign(src, src + L);
+  };
+  if (!t) {
+    m->taps_on = false;
+    return DG_OK;
+  }
+  grab(t->x_attn, m->tap_x_attn);
+  grab(t->x_out, m->tap_x_out);
+  grab(t->topk_w, m->tap_topk_w);
+  grab(t->topk_idx, m->tap_topk_idx);
+  grab(t->counts, m->tap_counts);
+  grab(t->perm, m->tap_perm);
+  m->tap_unions = t->unions;
+  m->taps_on = true;
+  return DG_OK;
+}
+
+extern "C" dg_status dg_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return DG_OK;
+}
+extern "C" void dg_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  prof_flush_locked();
+  for (int i = 0; i < DG_K_COUNT; ++i) g_prof_ms[i] = 0.0, g_prof_n[i] = 0;
+}
+extern "C" dg_status dg_profile_read(int32_t kind, double* total_ms, int32_t* launches) {
+  DG_CHECK_ARG(kind >= 0 && kind < DG_K_COUNT && total_ms && launches, "bad kind / NULL output");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  prof_flush_locked();
+  *total_ms = g_prof_ms[kind];
+  *launches = g_prof_n[kind];
+  return DG_OK;
+}
+extern "C" const char* dg_kernel_name(int32_t kind) {
+  static const char* names[DG_K_COUNT] = {"embed_norm", "rms_norm",   "gemm_qkv",   "rope_kv",        "attention",
+                                          "attn_merge", "gemm_o",     "router",     "topk",           "permute",
+                                          "gather",     "gemm_gate_up", "swiglu",   "gemm_down",      "combine",
+                                          "gemm_vocab", "update_partial", "update_select"};
+  return (kind >= 0 && kind < DG_K_COUNT) ? names[kind] : "?";
+}
+extern "C" int64_t dg_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_launches;
+}
+
+extern "C" dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups,
+                                        const void* X, int32_t x_rows, int32_t K, const int32_t* group_off,
+                                        int32_t max_rows_per_group, void* out, int32_t ld_out, int32_t* d_err,
+                                        dg_stream stream) {
+  DG_CHECK_ARG(W && X && out && d_err, "NULL pointer");
+  DG_CHECK_ARG(epi >= 0 && epi <= 2, "epi must be 0, 1 or 2");
+  DG_CHECK_ARG(K > 0 && K % 64 == 0 && a_rows_per_group > 0 && a_rows_per_group % 128 == 0 && n_groups > 0 &&
+                   x_rows > 0 && max_rows_per_group > 0,
+               "bad GEMM shape");
+  DG_CHECK_ARG(group_off || n_groups == 1, "several groups need group_off");
+  CUtensorMap A;
+  dg_status s = map_rows(&A, W, (uint64_t)n_groups * a_rows_per_group, (uint64_t)K, 128);
+  if (s != DG_OK) return s;
+  return gemm_bf16(DG_K_GEMM_QKV, epi, A, X, x_rows, K, a_rows_per_group, n_groups, group_off, max_rows_per_group,
+                   out, ld_out, d_err, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,
+                                             int32_t pos0, int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv,
+                                             void* out, void* d_ws, size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(q && k && vt && out && d_ws, "NULL pointer");
+  DG_CHECK_ARG(nq > 0 && nkv > 0 && nq % nkv == 0 && n_q > 0 && n_keys > 0 && n_keys <= cap && cap % 8 == 0,
+               "bad attention shape");
+  DG_CHECK_ARG(!causal || pos0 + n_q <= n_keys, "causal rows need their own keys");
+  dg_config c{};
+  c.n_layers = 1;
+  c.hidden = 128;
+  c.n_q_heads = nq;
+  c.n_kv_heads = nkv;
+  c.head_dim = 128;
+  c.n_experts = 1;
+  c.top_k = 1;
+  c.expert_ffn = 64;
+  c.vocab = 128;
+  c.rope_theta = 10000.f;
+  c.rms_eps = 1e-6f;
+  c.dtype = DG_DTYPE_BF16;
+  Ws ws;
+  dg_status s = check_ws(c, d_ws, ws_bytes, n_q, &ws);
+  if (s != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the pass reads q from the workspace's q buffer and writes o to its o buffer
+  cudaError_t e = cudaMemcpyAsync(ws.at<void>(ws.L.q), q, (size_t)nq * n_q * 128 * 2, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy q: %s", cudaGetErrorString(e));
+  if ((s = attention(c, ws, const_cast<void*>(k), const_cast<void*>(vt), cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
+    return s;
+  e = cudaMemcpyAsync(out, ws.at<void>(ws.L.o), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy o: %s", cudaGetErrorString(e));
+  return DG_OK;
+}

@@ -1,0 +1,679 @@
+// Non-tensor-core kernels of the pass: embedding + RMSNorm, RoPE and KV-cache
+// writes, the router and its top-k, the expert histogram / stable permutation /
+// row gather, the weighted combine, the canvas update (softmax confidence,
+// argmax, lowest-confidence re-noising), and fp32 GEMM / attention used by the
+// fp32 model (tcgen05 has no fp32 operand kind).
+#include <math.h>
+
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+// ---------------------------------------------------------------- block reductions
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = (threadIdx.x < nw) ? red[threadIdx.x] : 0.0f;
+  if (warp == 0) t = warp_sum(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  return red[0];
+}
+
+// ---------------------------------------------------------------- embedding + RMSNorm
+// x[t] = embed[tokens[t]] (fp32), xn[t] = x[t] / sqrt(mean(x[t]^2) + eps) in the activation dtype
+template <typename T>
+__global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ embed, int V, int H,
+                                  float eps, float* __restrict__ x, T* __restrict__ xn, int* __restrict__ err) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  int tok = tokens[t];
+  if (tok < 0 || tok >= V) {  // never read outside the table: flag and use token 0
+    if (threadIdx.x == 0) atomicCAS(err, 0, DG_DEVERR_BAD_TOKEN);
+    tok = 0;
+  }
+  const T* e = embed + (size_t)tok * H;
+  float* xr = x + (size_t)t * H;
+  float ss = 0.0f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const float v = to_f32(e[h]);
+    xr[h] = v;
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)H + eps);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) xn[(size_t)t * H + h] = from_f32<T>(xr[h] * inv);
+}
+
+template <typename T>
+__global__ void rms_norm_kernel(const float* __restrict__ x, int H, float eps, T* __restrict__ xn) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  const float* xr = x + (size_t)t * H;
+  float ss = 0.0f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) ss += xr[h] * xr[h];
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / (float)H + eps);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) xn[(size_t)t * H + h] = from_f32<T>(xr[h] * inv);
+}
+
+template <typename T>
+cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int V, int H, float eps, float* x, T* xn,
+                              int* err, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  embed_norm_kernel<T><<<n, 256, 0, st>>>(tokens, embed, V, H, eps, x, xn, err);
+  return cudaGetLastError();
+}
+template <typename T>
+cudaError_t launch_rms_norm(const float* x, int n, int H, float eps, T* xn, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  rms_norm_kernel<T><<<n, 256, 0, st>>>(x, H, eps, xn);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- RoPE + KV cache write
+// qkv[t] = [q heads | k heads | v heads] (fp32).  Rotate-half RoPE at position pos0 + t
+// (angles in double precision), then q -> q[h][t][:], k -> K[kvh][pos][:],
+// v -> V^T[kvh][:][pos], all in the activation dtype.
+template <typename T>
+__global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nq, int nkv, int d, int pos0, float theta,
+                                    int n, T* __restrict__ q, T* __restrict__ kc, T* __restrict__ vtc, int cap) {
+  extern __shared__ float cs[];  // [d/2] cos, [d/2] sin
+  const int t = blockIdx.x;
+  const int half = d / 2;
+  const int pos = pos0 + t;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)d);
+    double sn, cn;
+    sincos((double)pos * inv_freq, &sn, &cn);
+    cs[i] = (float)cn;
+    cs[half + i] = (float)sn;
+  }
+  __syncthreads();
+  const int W = (nq + 2 * nkv) * d;
+  const float* row = qkv + (size_t)t * W;
+  // q and k heads: pairs (i, i + d/2)
+  for (int idx = threadIdx.x; idx < (nq + nkv) * half; idx += blockDim.x) {
+    const int hh = idx / half, i = idx % half;
+    const float x1 = row[hh * d + i], x2 = row[hh * d + i + half];
+    const float c = cs[i], s = cs[half + i];
+    const float o1 = x1 * c - x2 * s, o2 = x2 * c + x1 * s;
+    if (hh < nq) {
+      T* dst = q + ((size_t)hh * n + t) * d;
+      dst[i] = from_f32<T>(o1);
+      dst[i + half] = from_f32<T>(o2);
+    } else {
+      T* dst = kc + ((size_t)(hh - nq) * cap + pos) * d;
+      dst[i] = from_f32<T>(o1);
+      dst[i + half] = from_f32<T>(o2);
+    }
+  }
+  for (int idx = threadIdx.x; idx < nkv * d; idx += blockDim.x) {
+    const int hh = idx / d, dd = idx % d;
+    vtc[((size_t)hh * d + dd) * cap + pos] = from_f32<T>(row[(nq + nkv) * d + idx]);
+  }
+}
+
+template <typename T>
+cudaError_t launch_rope_scatter(const float* qkv, int n, int nq, int nkv, int d, int pos0, float theta, T* q,
+                                T* kcache, T* vtcache, int cap, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  rope_scatter_kernel<T><<<n, 256, d * sizeof(float), st>>>(qkv, nq, nkv, d, pos0, theta, n, q, kcache, vtcache,
+                                                             cap);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- fp32 GEMM (fp32 model)
+// out[row][feat] (+)= sum_k W[g*M + feat][k] * X[row][k] for rows of group g
+constexpr int SG_BT = 32, SG_BF = 64, SG_BK = 32;
+__global__ void simt_gemm_f32_kernel(int epi_add, const float* __restrict__ W, const float* __restrict__ X,
+                                     const int* __restrict__ group_off, int n_tokens, int M, int K,
+                                     float* __restrict__ out, int ld_out) {
+  __shared__ float sx[SG_BT][SG_BK + 1];
+  __shared__ float sw[SG_BF][SG_BK + 1];
+  const int g = blockIdx.y;
+  int r_begin = 0, r_end = n_tokens;
+  if (group_off) {
+    r_begin = group_off[g];
+    r_end = group_off[g + 1];
+  }
+  const int r0 = r_begin + blockIdx.z * SG_BT;
+  if (r0 >= r_end) return;
+  const int f0 = blockIdx.x * SG_BF;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;  // 16 x 16 threads: 2 rows x 4 features each
+  float acc[2][4] = {};
+  const float* Wg = W + (size_t)g * M * K;
+  for (int k0 = 0; k0 < K; k0 += SG_BK) {
+    for (int i = threadIdx.x; i < SG_BT * SG_BK; i += blockDim.x) {
+      const int r = i / SG_BK, kk = i % SG_BK;
+      sx[r][kk] = (r0 + r < r_end && k0 + kk < K) ? X[(size_t)(r0 + r) * K + k0 + kk] : 0.0f;
+    }
+    for (int i = threadIdx.x; i < SG_BF * SG_BK; i += blockDim.x) {
+      const int f = i / SG_BK, kk = i % SG_BK;
+      sw[f][kk] = (f0 + f < M && k0 + kk < K) ? Wg[(size_t)(f0 + f) * K + k0 + kk] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      float a[2], b[4];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) a[i] = sx[ty * 2 + i][kk];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = sw[tx + 16 * j][kk];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r = r0 + ty * 2 + i;
+    if (r >= r_end) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int f = f0 + tx + 16 * j;
+      if (f >= M) continue;
+      float* dst = out + (size_t)r * ld_out + f;
+      if (epi_add)
+        *dst += acc[i][j];
+      else
+        *dst = acc[i][j];
+    }
+  }
+}
+
+cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, const int* group_off, int n_groups,
+                                 int max_rows_per_group, int n_tokens, int M, int K, float* out, int ld_out,
+                                 cudaStream_t st) {
+  if (max_rows_per_group <= 0 || n_groups <= 0) return cudaSuccess;
+  dim3 grid((M + SG_BF - 1) / SG_BF, n_groups, (max_rows_per_group + SG_BT - 1) / SG_BT);
+  simt_gemm_f32_kernel<<<grid, 256, 0, st>>>(epi_add, W, X, group_off, n_tokens, M, K, out, ld_out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- fp32 attention (fp32 model)
+// one warp per (query row, head); lane = key within a 32-key chunk, online softmax
+__global__ void simt_attention_f32_kernel(const float* __restrict__ q, const float* __restrict__ kc,
+                                          const float* __restrict__ vtc, int cap, int n_q, int q_pos0, int n_keys,
+                                          int causal, int nq, int nkv, int d, float* __restrict__ out) {
+  __shared__ float sq[128];
+  const int qrow = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+  const int kvh = h / (nq / nkv);
+  for (int i = lane; i < d; i += 32) sq[i] = q[((size_t)h * n_q + qrow) * d + i];
+  __syncwarp();
+  const int lim = causal ? min(n_keys, q_pos0 + qrow + 1) : n_keys;
+  const float scale = 1.0f / sqrtf((float)d);
+  float m = -INFINITY, l = 0.0f;
+  float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const float* K = kc + (size_t)kvh * cap * d;
+  const float* Vt = vtc + (size_t)kvh * d * cap;
+  for (int k0 = 0; k0 < lim; k0 += 32) {
+    const int key = k0 + lane;
+    float s = -INFINITY;
+    if (key < lim) {
+      float acc = 0.0f;
+      for (int i = 0; i < d; ++i) acc = fmaf(sq[i], K[(size_t)key * d + i], acc);
+      s = acc * scale;
+    }
+    const float cm = warp_max(s);
+    const float mn = fmaxf(m, cm);
+    const float alpha = (m == -INFINITY) ? 0.0f : expf(m - mn);
+    const float p = (key < lim) ? expf(s - mn) : 0.0f;
+    l = l * alpha + warp_sum(p);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] *= alpha;
+    const int nk = min(32, lim - k0);
+    for (int kk = 0; kk < nk; ++kk) {
+      const float pk = __shfl_sync(0xffffffffu, p, kk);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int dd = lane + 32 * j;
+        if (dd < d) o[j] = fmaf(pk, Vt[(size_t)dd * cap + k0 + kk], o[j]);
+      }
+    }
+    m = mn;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int dd = lane + 32 * j;
+    if (dd < d) out[(size_t)qrow * nq * d + (size_t)h * d + dd] = o[j] / l;
+  }
+}
+
+cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const float* vtcache, int cap, int n_q,
+                                      int q_pos0, int n_keys, int causal, int nq, int nkv, int d, float* out,
+                                      cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  simt_attention_f32_kernel<<<dim3(n_q, nq), 32, 0, st>>>(q, kcache, vtcache, cap, n_q, q_pos0, n_keys, causal, nq,
+                                                          nkv, d, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- router
+// logits[t][e] = sum_h xn[t][h] * w_router[e][h], xn = x / rms(x) in fp32.
+// CTA: 8 tokens x 32 experts; column-block 0 also writes xn in the activation dtype
+// (the expert input).
+constexpr int RT_TOK = 8, RT_EXP = 32, RT_K = 64;
+template <typename T>
+__global__ void router_kernel(const float* __restrict__ x, const float* __restrict__ wr, int n, int H, int E,
+                              float eps, float* __restrict__ logits, T* __restrict__ xn_out) {
+  __shared__ float inv_s[RT_TOK];
+  __shared__ float sx[RT_TOK][RT_K];
+  __shared__ float sw[RT_EXP][RT_K + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * RT_TOK, e0 = blockIdx.y * RT_EXP;
+  {
+    const int t = t0 + warp;
+    float ss = 0.0f;
+    if (t < n)
+      for (int h = lane; h < H; h += 32) ss += x[(size_t)t * H + h] * x[(size_t)t * H + h];
+    ss = warp_sum(ss);
+    if (lane == 0) inv_s[warp] = 1.0f / sqrtf(ss / (float)H + eps);
+  }
+  __syncthreads();
+  if (blockIdx.y == 0) {
+    for (int i = threadIdx.x; i < RT_TOK * H; i += blockDim.x) {
+      const int tt = i / H, h = i % H;
+      if (t0 + tt < n) xn_out[(size_t)(t0 + tt) * H + h] = from_f32<T>(x[(size_t)(t0 + tt) * H + h] * inv_s[tt]);
+    }
+  }
+  const int tt = warp, e = e0 + lane;
+  float acc = 0.0f;
+  for (int k0 = 0; k0 < H; k0 += RT_K) {
+    for (int i = threadIdx.x; i < RT_TOK * RT_K; i += blockDim.x) {
+      const int a = i / RT_K, kk = i % RT_K;
+      const int t = t0 + a;
+      sx[a][kk] = (t < n && k0 + kk < H) ? x[(size_t)t * H + k0 + kk] * inv_s[a] : 0.0f;
+    }
+    for (int i = threadIdx.x; i < RT_EXP * RT_K; i += blockDim.x) {
+      const int a = i / RT_K, kk = i % RT_K;
+      sw[a][kk] = (e0 + a < E && k0 + kk < H) ? wr[(size_t)(e0 + a) * H + k0 + kk] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 16
+    for (int kk = 0; kk < RT_K; ++kk) acc = fmaf(sx[tt][kk], sw[lane][kk], acc);
+    __syncthreads();
+  }
+  if (t0 + tt < n && e < E) logits[(size_t)(t0 + tt) * E + e] = acc;
+}
+
+template <typename T>
+cudaError_t launch_router(const float* x, const float* w_router, int n, int H, int E, float eps, float* logits,
+                          T* xn, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  dim3 grid((n + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
+  router_kernel<T><<<grid, 256, 0, st>>>(x, w_router, n, H, E, eps, logits, xn);
+  return cudaGetLastError();
+}
+
+// top-k by value (ties to the lower expert id), weights = softmax over the k chosen logits
+__global__ void topk_kernel(const float* __restrict__ logits, int n, int E, int k, int32_t* __restrict__ idx,
+                            float* __restrict__ w) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= n) return;
+  const float* lg = logits + (size_t)warp * E;
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? lg[e] : -INFINITY;
+  }
+  float chosen[16];
+  int chosen_id[16];
+  unsigned taken = 0u;  // bit i: entry lane + 32 i already chosen
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv || (v[i] == bv && e < bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    chosen[j] = bv;
+    chosen_id[j] = bi;
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+  }
+  if (lane == 0) {
+    float den = 0.0f;
+    for (int j = 0; j < k; ++j) den += expf(chosen[j] - chosen[0]);
+    for (int j = 0; j < k; ++j) {
+      idx[(size_t)warp * k + j] = chosen_id[j];
+      w[(size_t)warp * k + j] = expf(chosen[j] - chosen[0]) / den;
+    }
+  }
+}
+
+cudaError_t launch_topk(const float* logits, int n, int E, int k, int32_t* idx, float* w, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  if (E > 256 || k > 16 || k > E) return cudaErrorInvalidValue;
+  const int threads = 256;
+  topk_kernel<<<(n * 32 + threads - 1) / threads, threads, 0, st>>>(logits, n, E, k, idx, w);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- expert histogram + stable permutation
+// counts[e], offsets[e] (exclusive scan, offsets[E] = n*k), perm[p] = flattened (t*k + j)
+// of the p-th row when assignments are ordered by (expert, t, j); inv = inverse of perm;
+// union_out = number of experts with at least one row.  One CTA of 1024 threads.
+constexpr int PM_EMAX = 256;
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int total, int E,
+                                                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                       int32_t* __restrict__ union_out) {
+  __shared__ int cnt[PM_EMAX], base[PM_EMAX], run[PM_EMAX];
+  __shared__ int wcnt[32][PM_EMAX];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0, run[e] = 0;
+  __syncthreads();
+  for (int a = tid; a < total; a += blockDim.x) {
+    const int e = idx[a];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, u = 0;
+    for (int e = 0; e < E; ++e) {
+      base[e] = acc;
+      offsets[e] = acc;
+      counts[e] = cnt[e];
+      acc += cnt[e];
+      u += cnt[e] > 0;
+    }
+    offsets[E] = acc;
+    *union_out = u;
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < total; c0 += blockDim.x) {
+    const int a = c0 + tid;
+    const int e = (a < total) ? idx[a] : -1;
+    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i / E][i % E] = 0;
+    __syncthreads();
+    const unsigned match = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(match & lt_mask);
+    if (e >= 0 && e < E && rank == 0) wcnt[warp][e] = __popc(match);
+    __syncthreads();
+    if (e >= 0 && e < E) {
+      int pre = 0;
+      for (int w2 = 0; w2 < warp; ++w2) pre += wcnt[w2][e];
+      const int pos = base[e] + run[e] + pre + rank;
+      perm[pos] = a;
+      inv[a] = pos;
+    }
+    __syncthreads();
+    for (int e2 = tid; e2 < E; e2 += blockDim.x) {
+      int s = 0;
+      for (int w2 = 0; w2 < 32; ++w2) s += wcnt[w2][e2];
+      run[e2] += s;
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_permute(const int32_t* idx, int n, int k, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm, int32_t* inv, int32_t* union_out, cudaStream_t st) {
+  if (E > PM_EMAX) return cudaErrorInvalidValue;
+  permute_kernel<<<1, 1024, 0, st>>>(idx, n * k, E, counts, offsets, perm, inv, union_out);
+  return cudaGetLastError();
+}
+
+// xs[p] = xn[perm[p] / k]  (16-byte vector copies; H * sizeof(T) is a multiple of 16)
+template <typename T>
+__global__ void gather_rows_kernel(const T* __restrict__ xn, const int32_t* __restrict__ perm, int k, int H,
+                                   T* __restrict__ xs) {
+  const int p = blockIdx.x;
+  const int t = perm[p] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * H);
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
+  const int nv = H * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+}
+
+template <typename T>
+cudaError_t launch_gather_rows(const T* xn, const int32_t* perm, int rows, int k, int H, T* xs, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  gather_rows_kernel<T><<<rows, 128, 0, st>>>(xn, perm, k, H, xs);
+  return cudaGetLastError();
+}
+
+// fp32 model: gu rows in the packed gate/up order -> h = silu(gate) * up
+__global__ void swiglu_packed_f32_kernel(const float* __restrict__ gu, int F, float* __restrict__ h) {
+  const int p = blockIdx.x;
+  const float* r = gu + (size_t)p * 2 * F;
+  for (int f = threadIdx.x; f < F; f += blockDim.x) {
+    const int blk = f / 64, i = f % 64;
+    const float g = r[blk * 128 + i], u = r[blk * 128 + 64 + i];
+    h[(size_t)p * F + f] = g / (1.0f + expf(-g)) * u;
+  }
+}
+cudaError_t launch_swiglu_packed_f32(const float* gu, int rows, int F, float* h, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  swiglu_packed_f32_kernel<<<rows, 256, 0, st>>>(gu, F, h);
+  return cudaGetLastError();
+}
+
+// x[t] += sum_j w[t][j] * ys[inv[t*k + j]], slots in order j = 0..k-1
+__global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __restrict__ inv,
+                               const float* __restrict__ w, int k, int H, float* __restrict__ x) {
+  const int t = blockIdx.x;
+  __shared__ int rows[16];
+  __shared__ float ws[16];
+  if (threadIdx.x < k) {
+    rows[threadIdx.x] = inv[t * k + threadIdx.x];
+    ws[threadIdx.x] = w[t * k + threadIdx.x];
+  }
+  __syncthreads();
+  float4* xr = reinterpret_cast<float4*>(x + (size_t)t * H);
+  for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 y = reinterpret_cast<const float4*>(ys + (size_t)rows[j] * H)[i];
+      acc.x = fmaf(ws[j], y.x, acc.x);
+      acc.y = fmaf(ws[j], y.y, acc.y);
+      acc.z = fmaf(ws[j], y.z, acc.z);
+      acc.w = fmaf(ws[j], y.w, acc.w);
+    }
+    float4 v = xr[i];
+    v.x += acc.x;
+    v.y += acc.y;
+    v.z += acc.z;
+    v.w += acc.w;
+    xr[i] = v;
+  }
+}
+cudaError_t launch_combine(const float* ys, const int32_t* inv, const float* w, int n, int k, int H, float* x,
+                           cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  if (k > 16 || (H % 4) != 0) return cudaErrorInvalidValue;
+  combine_kernel<<<n, 256, 0, st>>>(ys, inv, w, k, H, x);
+  return cudaGetLastError();
+}
+
+// packed[e][b*128 + r] = r < 64 ? gate[e][b*64 + r] : up[e][b*64 + r - 64]  (rows of H elements)
+__global__ void pack_gate_up_kernel(const uint8_t* __restrict__ gate, const uint8_t* __restrict__ up,
+                                    uint8_t* __restrict__ out, int F, size_t row_bytes) {
+  const int prow = blockIdx.x;  // over E * 2F
+  const int e = prow / (2 * F), r2 = prow % (2 * F);
+  const int blk = r2 / 128, r = r2 % 128;
+  const uint8_t* src = (r < 64) ? gate + ((size_t)e * F + blk * 64 + r) * row_bytes
+                                : up + ((size_t)e * F + blk * 64 + r - 64) * row_bytes;
+  uint8_t* dst = out + (size_t)prow * row_bytes;
+  for (size_t i = threadIdx.x * 16; i < row_bytes; i += blockDim.x * 16)
+    *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<const uint4*>(src + i);
+}
+cudaError_t launch_pack_gate_up(const void* gate, const void* up, void* out, int E, int F, int H, int elem_bytes,
+                                cudaStream_t st) {
+  const size_t row_bytes = (size_t)H * elem_bytes;
+  if ((row_bytes % 16) != 0 || (F % 64) != 0) return cudaErrorInvalidValue;
+  pack_gate_up_kernel<<<E * 2 * F, 128, 0, st>>>((const uint8_t*)gate, (const uint8_t*)up, (uint8_t*)out, F,
+                                                  row_bytes);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- canvas update
+__device__ __forceinline__ void upd_merge(float& m, float& s, int& a, float m2, float s2, int a2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2, s = s2, a = a2;
+    return;
+  }
+  if (m2 > m) {
+    s = s * expf(m - m2) + s2;
+    m = m2;
+    a = a2;
+  } else if (m2 < m) {
+    s += s2 * expf(m2 - m);
+  } else {
+    s += s2;
+    a = min(a, a2);
+  }
+}
+
+int update_splits(int C, int V) {
+  // about four CTAs per SM over the canvas, slices of at least 4096 logits
+  int s = (4 * 148 + C - 1) / (C > 0 ? C : 1);
+  const int max_s = (V + 4095) / 4096;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  return s;
+}
+
+// per (row, slice): max, first argmax and sum exp(l - max), one streaming pass
+__global__ void update_partial_kernel(const float* __restrict__ logits, int V, int splits, UpdPart* __restrict__ part) {
+  __shared__ float sm[32], ss[32];
+  __shared__ int sa[32];
+  const int row = blockIdx.x, sp = blockIdx.y;
+  const int slice = ((V + splits - 1) / splits + 3) & ~3;
+  const int lo = sp * slice, hi = min(V, lo + slice);
+  const float* lg = logits + (size_t)row * V;
+  float m = -INFINITY, s = 0.0f;
+  int a = 0x7fffffff;
+  for (int i = lo + threadIdx.x * 4; i < hi; i += blockDim.x * 4) {
+    const float4 v4 = *reinterpret_cast<const float4*>(lg + i);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float x = v[u];
+      if (x > m) {
+        s = s * __expf(m - x) + 1.0f;
+        m = x;
+        a = i + u;
+      } else {
+        s += __expf(x - m);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
+    upd_merge(m, s, a, m2, s2, a2);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) sm[warp] = m, ss[warp] = s, sa[warp] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w2 = 1; w2 < (int)(blockDim.x >> 5); ++w2) upd_merge(m, s, a, sm[w2], ss[w2], sa[w2]);
+    UpdPart r;
+    r.m = m;
+    r.s = s;
+    r.a = a;
+    r.pad = 0;
+    part[(size_t)row * splits + sp] = r;
+  }
+}
+
+__device__ __forceinline__ uint64_t splitmix64_out(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// merge slices, confidence = 1 / sum exp(l - max); every position takes its argmax, then
+// the n_renoise lowest-confidence positions (ties: lower position first) take a fresh
+// token: SplitMix64(seed) draw number (step << 32 | position), multiply-shift onto [0, V).
+__global__ void update_select_kernel(const UpdPart* __restrict__ part, int C, int V, int splits, int n_renoise,
+                                     uint64_t seed, uint32_t step, int32_t* __restrict__ canvas,
+                                     float* __restrict__ conf) {
+  extern __shared__ float den[];  // [C]
+  const int i = threadIdx.x;
+  float m = -INFINITY, s = 0.0f;
+  int a = 0x7fffffff;
+  if (i < C) {
+    for (int sp = 0; sp < splits; ++sp) {
+      const UpdPart q = part[(size_t)i * splits + sp];
+      upd_merge(m, s, a, q.m, q.s, q.a);
+    }
+    den[i] = s;
+  }
+  __syncthreads();
+  if (i < C) {
+    int rank = 0;
+    for (int j = 0; j < C; ++j) {
+      const float dj = den[j];
+      rank += (dj > s) || (dj == s && j < i);
+    }
+    int tok = a;
+    if (rank < n_renoise) {
+      const uint64_t x = splitmix64_out(seed, ((uint64_t)step << 32) | (uint64_t)i);
+      tok = (int)(((x >> 32) * (uint64_t)V) >> 32);
+    }
+    canvas[i] = tok;
+    if (conf) conf[i] = 1.0f / s;
+  }
+}
+
+cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, UpdPart* part, cudaStream_t st) {
+  if (C <= 0) return cudaSuccess;
+  update_partial_kernel<<<dim3(C, splits), 256, 0, st>>>(logits, V, splits, part);
+  return cudaGetLastError();
+}
+cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
+                                 uint32_t step, int32_t* canvas, float* conf, cudaStream_t st) {
+  if (C <= 0) return cudaSuccess;
+  if (C > 1024) return cudaErrorInvalidValue;
+  const int threads = (C + 31) & ~31;
+  update_select_kernel<<<1, threads, C * sizeof(float), st>>>(part, C, V, splits, n_renoise, seed, step, canvas,
+                                                              conf);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- explicit instantiations
+template cudaError_t launch_embed_norm<float>(const int32_t*, const float*, int, int, int, float, float*, float*,
+                                              int*, cudaStream_t);
+template cudaError_t launch_embed_norm<bf16>(const int32_t*, const bf16*, int, int, int, float, float*, bf16*, int*,
+                                             cudaStream_t);
+template cudaError_t launch_rms_norm<float>(const float*, int, int, float, float*, cudaStream_t);
+template cudaError_t launch_rms_norm<bf16>(const float*, int, int, float, bf16*, cudaStream_t);
+template cudaError_t launch_rope_scatter<float>(const float*, int, int, int, int, int, float, float*, float*, float*,
+                                                int, cudaStream_t);
+template cudaError_t launch_rope_scatter<bf16>(const float*, int, int, int, int, int, float, bf16*, bf16*, bf16*, int,
+                                               cudaStream_t);
+template cudaError_t launch_router<float>(const float*, const float*, int, int, int, float, float*, float*,
+                                          cudaStream_t);
+template cudaError_t launch_router<bf16>(const float*, const float*, int, int, int, float, float*, bf16*,
+                                         cudaStream_t);
+template cudaError_t launch_gather_rows<float>(const float*, const int32_t*, int, int, int, float*, cudaStream_t);
+template cudaError_t launch_gather_rows<bf16>(const bf16*, const int32_t*, int, int, int, bf16*, cudaStream_t);
+
+}  // namespace dg

@@ -1,0 +1,168 @@
+/*
+ * dg.h -- C-ABI of libdg: the denoising pass of a block-diffusion ("uniform-state")
+ * MoE language model on one B200 (sm_100a).
+ *
+ * What the calls compute (page title -- section):
+ *   "DiffusionGemma" video explainer -- "The fix: a 256-token canvas": a canvas of
+ *       token slots is refined in parallel over several denoising passes;
+ *   same page -- "Uniform State Diffusion": noise is random vocabulary tokens, every
+ *       position is updated in parallel, low-confidence tokens are re-noised with
+ *       fresh random tokens, and passes repeat until the canvas converges;
+ *   same page -- "Two modes, one model": prefill mode reads tokens with causal
+ *       attention and writes the KV cache; denoising mode lets every canvas token
+ *       attend to all canvas tokens and to the KV cache;
+ *   same page -- "Long-form text: chaining canvases": each completed canvas is
+ *       appended to the KV cache by a prefill step before the next canvas opens;
+ *   "Module 12. Diffusion Language Models" exercises -- prefix/block mask solution:
+ *       prefix rows causal, block rows see prefix and block; prefix K/V is reused
+ *       across denoising steps unchanged;
+ *   same page -- MoE remark: one pass reads the union of the experts its canvas
+ *       positions route to.
+ *
+ * Conventions for every call:
+ *   - All device pointers are owned by the caller; the library never frees them and
+ *     allocates no device memory of its own.  Host structs are read during the call
+ *     only (dg_model_create copies what it needs).
+ *   - Work is enqueued asynchronously on the given stream (NULL = legacy default
+ *     stream); the return code covers argument validation and launch errors only.
+ *     Device-side failures (a bounded wait that timed out) are recorded in the
+ *     workspace's error word and reported by dg_device_status.
+ *   - On any error no kernel has been launched unless the code is DG_ERR_CUDA.
+ *   - dg_last_error() returns a thread-local message for the last non-OK status.
+ *
+ * Data layouts (row-major; "bf16" = IEEE bfloat16 bits; the fp32 model uses float):
+ *   weights, all [out_features][in_features] (y = x W^T):
+ *     embed, w_out   [V][H]
+ *     w_qkv          [(nq + 2 nkv) d][H]    rows of W_q, then W_k, then W_v
+ *     w_o            [H][nq d]
+ *     w_router       [E][H]                 always fp32
+ *     w_gate_up      [E][2F][H]             packed: for b = 0..F/64-1, rows 128b..128b+63
+ *                                            are gate rows 64b..64b+63, rows 128b+64..128b+127
+ *                                            the up rows 64b..64b+63 (see dg_pack_gate_up)
+ *     w_down         [E][H][F]
+ *   KV cache, per layer:  K [nkv][capacity][d],  V transposed: Vt [nkv][d][capacity]
+ *   canvas / tokens int32 [n];  logits fp32 [C][V]
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dg_stream; /* a cudaStream_t */
+
+typedef enum dg_status {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = -1, /* null pointer, bad size, unsupported shape for the dtype    */
+  DG_ERR_CAPACITY = -2,    /* KV cache or workspace too small; nothing was changed        */
+  DG_ERR_CUDA = -3,        /* a CUDA call failed; see dg_last_error()                      */
+  DG_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up (from dg_device_status)   */
+  DG_ERR_UNSUPPORTED = -5  /* valid shape that this build does not implement               */
+} dg_status;
+
+typedef enum dg_dtype { DG_DTYPE_BF16 = 0, DG_DTYPE_F32 = 1 } dg_dtype;
+
+typedef struct dg_config {
+  int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim;
+  int32_t n_experts, top_k, expert_ffn, vocab;
+  float rope_theta; /* RoPE base (rotate-half pairs, absolute positions)             */
+  float rms_eps;    /* RMSNorm epsilon (unit gain)                                   */
+  int32_t dtype;    /* dg_dtype of weights, activations and KV cache                 */
+} dg_config;
+/* Shape rules.  Both dtypes: n_q_heads % n_kv_heads == 0, top_k <= min(16, n_experts),
+ * n_experts <= 256, hidden % 64 == 0, expert_ffn % 64 == 0.  bf16 additionally:
+ * head_dim == 128, vocab % 128 == 0, (n_q_heads + 2 n_kv_heads) * 128 % 128 == 0.
+ * fp32: head_dim <= 128. */
+
+typedef struct dg_layer_weights {
+  const void* w_qkv;
+  const void* w_o;
+  const float* w_router;
+  const void* w_gate_up;
+  const void* w_down;
+} dg_layer_weights;
+
+typedef struct dg_weights {
+  const void* embed;
+  const void* w_out;
+  const dg_layer_weights* layers; /* host array of n_layers */
+} dg_weights;
+
+typedef struct dg_kv_cache {
+  void* const* k;   /* host array [n_layers] of device pointers, K  [nkv][capacity][d] */
+  void* const* vt;  /* host array [n_layers] of device pointers, Vt [nkv][d][capacity] */
+  int32_t capacity; /* positions per layer, multiple of 8                               */
+  int32_t len;      /* valid positions [0, len); dg_prefill_append advances it          */
+} dg_kv_cache;
+
+typedef struct dg_model dg_model;
+
+/* Validate the config, copy it and the weight pointers, and pre-encode the weight
+ * tensor maps.  The weights must stay alive and unchanged while the model exists. */
+dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);
+void dg_model_destroy(dg_model* m);
+
+/* Bytes of device workspace for calls on up to max_tokens tokens per call (canvas or
+ * prefill length).  The caller allocates it (256-byte aligned) and passes it to every
+ * call; its first 4 bytes are the device error word (zero it once after allocating). */
+size_t dg_workspace_bytes(const dg_config* cfg, int32_t max_tokens);
+/* Workspace bytes dg_canvas_update needs on its own for a C x V logits matrix. */
+size_t dg_update_workspace_bytes(int32_t C, int32_t V);
+
+/* Prefill mode.  Runs the T tokens at positions len..len+T-1 through the stack with
+ * causal attention over [0, len + i] and writes their K/V into every layer's cache at
+ * [len, len + T); then cache->len += T.  No logits are produced.
+ * DG_ERR_CAPACITY if len + T > capacity (cache and len unchanged). */
+dg_status dg_prefill_append(dg_model* m, dg_kv_cache* cache, const int32_t* d_tokens, int32_t T, void* d_ws,
+                            size_t ws_bytes, dg_stream stream);
+
+/* Denoising mode.  One pass over the canvas at positions len..len+C-1: every canvas
+ * query attends to cached keys [0, len) and all C canvas keys.  Writes
+ * d_logits[C][V] (fp32).  The canvas K/V are written to cache slots [len, len+C) as
+ * scratch; cache->len and slots [0, len) are never modified.
+ * DG_ERR_CAPACITY if len + C > capacity. */
+dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, const int32_t* d_canvas, int32_t C,
+                          float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream);
+
+/* Canvas update.  For each row i of d_logits[C][V]: argmax (lowest id on ties) and
+ * confidence = largest softmax probability.  Every position takes its argmax, then
+ * the n_renoise lowest-confidence positions (lower position first on ties) take a
+ * fresh token: SplitMix64 draw number (step << 32 | i) of the stream seeded with
+ * `seed`, mapped to [0, V) as (draw >> 32) * V >> 32.  Writes d_canvas[C]; writes
+ * d_conf[C] if not NULL.  C <= 1024, V % 4 == 0, 0 <= n_renoise <= C. */
+dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t V, int32_t n_renoise, uint64_t seed,
+                           uint32_t step, int32_t* d_canvas, float* d_conf, void* d_ws, size_t ws_bytes,
+                           dg_stream stream);
+
+/* S denoising passes with re-noising, then (if append) the canvas is appended to the
+ * cache by dg_prefill_append.  After pass s (0-based) the number of re-noised
+ * positions is floor(C * f_s + 1e-9), f_s = (r_start (S-1-s) + r_end s) / (S-1)
+ * (f_0 = r_start when S == 1); the update of pass s uses step = s.  d_canvas holds
+ * the initial noise on entry and the result on return.  d_logits ([C][V]) receives
+ * the last pass's logits. */
+dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t S,
+                             float r_start, float r_end, uint64_t seed, int32_t append, float* d_logits,
+                             void* d_ws, size_t ws_bytes, dg_stream stream);
+
+/* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
+int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
+
+/* Lay out separate gate and up weights ([E][F][H] each) in the packed w_gate_up layout.
+ * elem_bytes: 2 (bf16) or 4 (fp32).  Pure data movement on the stream. */
+dg_status dg_pack_gate_up(const void* d_gate, const void* d_up, void* d_out, int32_t E, int32_t F, int32_t H,
+                          int32_t elem_bytes, dg_stream stream);
+
+/* Synchronize the stream, read and clear the workspace error word.  DG_OK or
+ * DG_ERR_TIMEOUT (a kernel's bounded wait gave up; its outputs are not valid). */
+dg_status dg_device_status(void* d_ws, dg_stream stream);
+
+const char* dg_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

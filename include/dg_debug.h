@@ -1,0 +1,94 @@
+/*
+ * dg_debug.h -- inspection entry points of libdg: per-layer taps of the denoising
+ * pass (for layer-by-layer comparison with an independent implementation) and
+ * per-kernel timing with CUDA events.  None of these change what the pass computes.
+ */
+#ifndef DG_DEBUG_H
+#define DG_DEBUG_H
+
+#include "dg.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Per-layer copies taken during dg_denoise_pass.  Each member is a host array of
+ * n_layers device pointers (the array itself or any entry may be NULL = not taken).
+ *   x_attn   fp32 [C][H]   residual after the attention block
+ *   x_out    fp32 [C][H]   residual after the MoE block
+ *   topk_idx int32 [C][k]  routed experts, descending router logit
+ *   topk_w   fp32 [C][k]   combine weights (softmax over the k chosen logits)
+ *   counts   int32 [E]     rows routed to each expert
+ *   perm     int32 [C k]   perm[p] = t*k + j of the p-th row in expert order
+ *   unions   device int32 [n_layers] (single pointer): experts with at least one row */
+typedef struct dg_taps {
+  float* const* x_attn;
+  float* const* x_out;
+  int32_t* const* topk_idx;
+  float* const* topk_w;
+  int32_t* const* counts;
+  int32_t* const* perm;
+  int32_t* unions;
+} dg_taps;
+
+/* Copy the tap pointers into the model (NULL turns taps off). */
+dg_status dg_set_taps(dg_model* m, const dg_taps* taps);
+
+/* Kernel kinds timed by the profiler. */
+typedef enum dg_kernel_kind {
+  DG_K_EMBED_NORM = 0,
+  DG_K_RMS_NORM,
+  DG_K_GEMM_QKV,
+  DG_K_ROPE_KV,
+  DG_K_ATTENTION,
+  DG_K_ATTN_MERGE,
+  DG_K_GEMM_O,
+  DG_K_ROUTER,
+  DG_K_TOPK,
+  DG_K_PERMUTE,
+  DG_K_GATHER,
+  DG_K_GEMM_GATE_UP,
+  DG_K_SWIGLU,
+  DG_K_GEMM_DOWN,
+  DG_K_COMBINE,
+  DG_K_GEMM_VOCAB,
+  DG_K_UPDATE_PARTIAL,
+  DG_K_UPDATE_SELECT,
+  DG_K_COUNT
+} dg_kernel_kind;
+
+/* When on, every kernel launch of the library is bracketed by a pair of CUDA events
+ * recorded on the launching stream.  Off by default. */
+dg_status dg_profile_enable(int32_t on);
+/* Wait for the recorded events and return, for one kind, the summed device time (ms)
+ * and the number of launches since the last reset. */
+dg_status dg_profile_read(int32_t kind, double* total_ms, int32_t* launches);
+void dg_profile_reset(void);
+const char* dg_kernel_name(int32_t kind);
+
+/* One launch of the tcgen05 GEMM alone (bf16):
+ *   out[r][f] (op)= sum_k W[g * a_rows_per_group + f][k] * X[r][k]
+ * for rows r of group g = [group_off[g], group_off[g+1]) (group_off: device int32
+ * [n_groups + 1], or NULL for one group of x_rows rows).  epi 0: store fp32 out,
+ * 1: add into fp32 out, 2: packed gate/up rows -> bf16 silu(gate) * up with
+ * a_rows_per_group / 2 output columns.  W [n_groups * a_rows_per_group][K], X [x_rows][K]
+ * bf16; K % 64 == 0, a_rows_per_group % 128 == 0.  d_err: device int32 error word. */
+dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups, const void* X,
+                             int32_t x_rows, int32_t K, const int32_t* group_off, int32_t max_rows_per_group,
+                             void* out, int32_t ld_out, int32_t* d_err, dg_stream stream);
+
+/* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
+ * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
+ * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128].  d_ws: a workspace sized by
+ * dg_workspace_bytes for a config with these heads and >= n_q tokens. */
+dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q, int32_t pos0,
+                                  int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv, void* out, void* d_ws,
+                                  size_t ws_bytes, dg_stream stream);
+
+/* Kernels launched by the library since it was loaded (all kinds, profiling or not). */
+int64_t dg_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_DEBUG_H */

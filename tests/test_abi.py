@@ -1,0 +1,70 @@
+"""The C-ABI library: it loads, exports every symbol the headers declare, and its
+host-side validation and arithmetic work without a GPU (no compute calls here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from conftest import ROOT, golden_path
+from block_diffusion_lm_masked_b200 import configs as CF
+from block_diffusion_lm_masked_b200 import dg
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \t\*]*?\b(dg_[a-z0-9_]+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert {"dg_prefill_append", "dg_denoise_pass", "dg_canvas_update", "dg_generate_canvas"} <= names
+    lib = ctypes.CDLL(dg.LIB_PATH)
+    missing = [n for n in sorted(names) if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_workspace_sizes_for_every_config():
+    for name in CF.ORDER:
+        cfg = CF.CONFIGS[name]
+        n = dg.workspace_bytes(cfg, max(cfg["canvas"], cfg.get("prompt", 0)))
+        assert n > 0 and n % 256 == 0
+    assert dg.update_workspace_bytes(256, 262144) > 256
+
+
+def test_invalid_configs_rejected_on_host():
+    bad = dict(CF.CONFIGS["layer1_bf16"], head_dim=64)          # bf16 path needs d = 128
+    assert dg.workspace_bytes(bad, 256) == 0
+    c = dg.make_config(bad)
+    w = dg.Weights(None, None, None)
+    h = ctypes.c_void_p()
+    assert dg.lib.dg_model_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == dg.DG_ERR_INVALID_ARG
+    assert "head_dim" in dg.lib.dg_last_error().decode()
+    for over in (dict(n_q_heads=6, n_kv_heads=4), dict(top_k=17), dict(n_experts=300), dict(expert_ffn=100)):
+        assert dg.workspace_bytes(dict(CF.CONFIGS["tiny_fp32"], **over), 32) == 0, over
+
+
+def test_null_arguments_rejected_on_host():
+    assert dg.lib.dg_canvas_update(None, 4, 8, 1, 0, 0, None, None, None, 0, None) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_denoise_pass(None, None, None, 4, None, None, 0, None) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_prefill_append(None, None, None, 4, None, 0, None) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_device_status(None, None) == dg.DG_ERR_INVALID_ARG
+
+
+def test_renoise_schedule_matches_golden():
+    g = {}
+    for line in open(golden_path("renoise_schedule.txt")):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            g[k] = [int(x) for x in v]
+    assert [dg.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]
+    assert [dg.renoise_count(256, 8, s, 0.5, 0.0) for s in range(8)] == g["S8"]
+    assert dg.renoise_count(256, 1, 0, 0.25, 0.25) == g["S1_C256_q25"][0]
+    assert dg.renoise_count(32, 1, 0, 0.25, 0.25) == g["S1_C32_q25"][0]
+    assert dg.renoise_count(256, 4, 4, 0.5, 0.0) == -1

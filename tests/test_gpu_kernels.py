@@ -1,0 +1,132 @@
+"""Single-kernel checks of the tcgen05 GEMM and attention launches against plain
+PyTorch fp32 on the same device (the GPU's own reference of the same op), on
+shapes with ragged token counts, several tiles and empty groups."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from block_diffusion_lm_masked_b200 import dg as _dg
+    return _dg
+
+
+def _bf(*shape, scale=1.0, gen=None):
+    return (torch.randn(*shape, generator=gen, device="cuda") * scale).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,K,n", [(128, 64, 1), (256, 128, 16), (384, 512, 100), (128, 2048, 256), (256, 256, 300),
+                                   (1408, 2816, 37)])
+def test_dense_gemm_store(dg, M, K, n):
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + n)
+    W, X = _bf(M, K, gen=g), _bf(n, K, gen=g)
+    out = torch.full((n, M), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dg.debug_gemm_bf16(0, W, M, 1, X, None, n, out, M, err)
+    torch.cuda.synchronize()
+    ref = X.float() @ W.float().T
+    assert err.item() == 0
+    torch.testing.assert_close(out, ref, rtol=1e-4, atol=1e-3 * ref.abs().max().item())
+
+
+def test_dense_gemm_add(dg):
+    g = torch.Generator(device="cuda").manual_seed(3)
+    M, K, n = 256, 512, 77
+    W, X = _bf(M, K, gen=g), _bf(n, K, gen=g)
+    base = torch.randn(n, M, generator=g, device="cuda")
+    out = base.clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dg.debug_gemm_bf16(1, W, M, 1, X, None, n, out, M, err)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out, base + X.float() @ W.float().T, rtol=1e-4, atol=1e-3 * 20)
+
+
+def _groups(counts):
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    return torch.from_numpy(off).cuda(), int(off[-1])
+
+
+@pytest.mark.parametrize("counts", [[0, 3, 17, 40, 1], [16, 0, 0, 256, 5, 33], [300, 2]])
+def test_grouped_gemm(dg, counts):
+    g = torch.Generator(device="cuda").manual_seed(sum(counts))
+    E, M, K = len(counts), 256, 192
+    off, rows = _groups(counts)
+    W, X = _bf(E * M, K, gen=g), _bf(rows, K, gen=g)
+    out = torch.full((rows, M), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dg.debug_gemm_bf16(0, W, M, E, X, off, max(counts), out, M, err)
+    torch.cuda.synchronize()
+    ref = torch.empty_like(out)
+    o = off.cpu().numpy()
+    for e in range(E):
+        ref[o[e]:o[e + 1]] = X[o[e]:o[e + 1]].float() @ W[e * M:(e + 1) * M].float().T
+    torch.testing.assert_close(out, ref, rtol=1e-4, atol=1e-3 * ref.abs().max().item())
+
+
+def test_gate_up_swiglu_epilogue(dg):
+    g = torch.Generator(device="cuda").manual_seed(5)
+    counts = [5, 0, 70, 16]
+    E, F, K = len(counts), 128, 256
+    off, rows = _groups(counts)
+    gate, up = _bf(E, F, K, scale=0.1, gen=g), _bf(E, F, K, scale=0.1, gen=g)
+    packed = torch.empty(E, 2 * F, K, dtype=torch.bfloat16, device="cuda")
+    dg._check(dg.lib.dg_pack_gate_up(dg._ptr(gate), dg._ptr(up), dg._ptr(packed), E, F, K, 2, dg._stream()))
+    X = _bf(rows, K, gen=g)
+    h = torch.zeros(rows, F, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dg.debug_gemm_bf16(2, packed.view(E * 2 * F, K), 2 * F, E, X, off, max(counts), h, F, err)
+    torch.cuda.synchronize()
+    o = off.cpu().numpy()
+    ref = torch.empty(rows, F, device="cuda")
+    for e in range(E):
+        xs = X[o[e]:o[e + 1]].float()
+        a, b = xs @ gate[e].float().T, xs @ up[e].float().T
+        ref[o[e]:o[e + 1]] = torch.nn.functional.silu(a) * b
+    torch.testing.assert_close(h.float(), ref, rtol=2e-2, atol=2e-2 * ref.abs().max().item())
+
+
+def _attn_ref(q, k, vt, n_keys, pos0, causal):
+    nq, n_q, d = q.shape
+    nkv = k.shape[0]
+    g = nq // nkv
+    out = torch.empty(n_q, nq * d, device="cuda")
+    kk = k[:, :n_keys].float()
+    vv = vt[:, :, :n_keys].float().transpose(1, 2)
+    pos = torch.arange(n_q, device="cuda") + pos0
+    keys = torch.arange(n_keys, device="cuda")
+    mask = keys[None, :] <= pos[:, None] if causal else torch.ones(n_q, n_keys, dtype=torch.bool, device="cuda")
+    for h in range(nq):
+        s = (q[h].float() @ kk[h // g].T) / d ** 0.5
+        s = s.masked_fill(~mask, float("-inf"))
+        out[:, h * d:(h + 1) * d] = torch.softmax(s, dim=1) @ vv[h // g]
+    return out
+
+
+@pytest.mark.parametrize("n_q,pos0,n_keys,causal,nq,nkv", [
+    (100, 200, 300, False, 4, 2),      # canvas rows over a ragged prefix + canvas
+    (256, 1024, 1280, False, 16, 4),   # the single-layer workload's shape
+    (200, 50, 250, True, 4, 1),        # prefill rows, causal, ragged
+    (64, 4900, 4964, False, 2, 2),     # long keys: split-KV + merge
+    (300, 0, 300, True, 2, 1),         # prefill from an empty cache
+])
+def test_attention(dg, n_q, pos0, n_keys, causal, nq, nkv):
+    from block_diffusion_lm_masked_b200 import configs as CF
+    g = torch.Generator(device="cuda").manual_seed(n_q + n_keys)
+    d, cap = 128, ((n_keys + 7) // 8) * 8 + 8
+    q = _bf(nq, n_q, d, gen=g)
+    k = _bf(nkv, cap, d, gen=g)
+    vt = _bf(nkv, d, cap, gen=g)
+    cfg = dict(CF.CONFIGS["layer1_bf16"], n_q_heads=nq, n_kv_heads=nkv, hidden=128, expert_ffn=64, n_experts=1,
+               top_k=1, vocab=128, n_layers=1)
+    ws = dg.Workspace(cfg, n_q)
+    out = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device="cuda")
+    dg.debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws)
+    dg.device_status(ws)
+    ref = _attn_ref(q, k, vt, n_keys, pos0, causal)
+    err = (out.float() - ref).abs().max().item() / ref.pow(2).mean().sqrt().item()
+    assert err < 2e-2, err
