@@ -1,0 +1,326 @@
+"""Benchmark of one denoising step: a full denoising pass plus the canvas update.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Workload (default): the single-layer bf16 pass -- hidden 2048, 16 query / 4 KV heads
+of 128, 64 experts top-4 with FFN 1024, vocabulary 32768, 1024 cached prefix
+positions (K/V ~ N(0,1)), a 256-slot canvas of uniform random tokens; one step =
+dg_denoise_pass + dg_canvas_update (25% re-noised).  Weights are seeded N(0, 0.02)
+bf16 (synthetic, random init).  The metric is canvas tokens per second per pass
+(C / step latency), summed over ranks; each rank runs its own replica (no data-path
+collective: the pass does not shard), so scaling is weak.
+
+Prints ONE JSON line on rank 0.  --impl reference times the CPU oracle instead (a
+bounded sample of the same workload on the host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from block_diffusion_lm_masked_b200 import configs as CF  # noqa: E402
+from block_diffusion_lm_masked_b200 import roofline as RF  # noqa: E402
+from block_diffusion_lm_masked_b200 import synth  # noqa: E402
+
+METRIC = "canvas tokens/sec per denoising pass and pass latency (µs); % of roofline, 1×B200"
+UNIT = "canvas tokens/s"
+DATA = "synthetic: seeded random-init weights N(0,0.02) bf16, cached prefix K/V N(0,1), uniform canvas tokens"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _workload_desc(name, cfg):
+    return (f"{name}: {cfg['n_layers']} layer(s), H{cfg['hidden']}, {cfg['n_q_heads']}q/{cfg['n_kv_heads']}kv "
+            f"d{cfg['head_dim']}, E{cfg['n_experts']} top-{cfg['top_k']}, F{cfg['expert_ffn']}, V{cfg['vocab']}, "
+            f"P{cfg['prefix']}, C{cfg['canvas']}; step = 1 denoising pass + canvas update")
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except Exception:
+            self.p.kill()
+            out, _ = self.p.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _oracle_step(host, ocache, canvas, n, prec, step):
+    from oracle import dg_oracle as O
+    logits, _ = O.denoise_pass(host, ocache, canvas, prec)
+    return O.canvas_update(logits, n, synth.SEED_RENOISE, step)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i.get("num_threads", 1) for i in threadpool_info())
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg, name):
+    """The CPU oracle on the host cores, one oracle step per timed step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import dg_oracle as O
+    P, C = cfg["prefix"], cfg["canvas"]
+    host = synth.Model(cfg)
+    ocache = O.Cache(synth.prefix_cache(cfg, P))
+    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
+    prec = O.Precision(cfg["dtype"])
+    n = O.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+    for w in range(args.warmup):
+        _oracle_step(host, ocache, canvas, n, prec, 0)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        _oracle_step(host, ocache, canvas, n, prec, 0)
+    dt = time.perf_counter() - t0
+    ms = dt * 1e3 / max(1, args.steps)
+    value = C / (ms / 1e3)
+    cores = _blas_threads()
+    sample = f"{args.steps} full oracle steps (pass + update) of the workload, fp64 numpy"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": {"workload": _workload_desc(name, cfg)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(cfg, budget_s=30.0):
+    """Time the oracle as it stands on a bounded sample: whole oracle steps until ~budget."""
+    from oracle import dg_oracle as O
+    P, C = cfg["prefix"], cfg["canvas"]
+    host = synth.Model(cfg)
+    ocache = O.Cache(synth.prefix_cache(cfg, P))
+    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
+    prec = O.Precision(cfg["dtype"])
+    n = O.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+    times = []
+    t_start = time.perf_counter()
+    while not times or (time.perf_counter() - t_start < budget_s / 2 and len(times) < 5):
+        t0 = time.perf_counter()
+        _oracle_step(host, ocache, canvas, n, prec, 0)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.median(times) * 1e3
+    return {"value": C / (ms / 1e3), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{len(times)} whole oracle steps (denoising pass + update, fp64 numpy) of the workload; "
+                      f"median {ms:.0f} ms per step"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
+    ap.add_argument("--workload", default="layer1_bf16", choices=[n for n in CF.ORDER if n != "chained8_bf16"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    name = args.workload
+    cfg = CF.CONFIGS[name]
+    if args.impl == "reference":
+        return run_reference(args, cfg, name)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from block_diffusion_lm_masked_b200 import dg
+
+    P, C, V = cfg["prefix"], cfg["canvas"], cfg["vocab"]
+    host = synth.Model(cfg)
+    model = dg.Model(host, dev)
+    cache = dg.KVCache(cfg, ((P + C + 7) // 8) * 8, dev)
+    cache.load_prefix(synth.prefix_cache(cfg, P))
+    ws = dg.Workspace(cfg, C, dev)
+    noise = torch.from_numpy(synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(rank), C, V))
+    canvas = noise.to(dev)
+    logits = torch.empty(C, V, device=dev)
+    n_ren = dg.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
+
+    # every step denoises the same input canvas; the update writes a second buffer
+    canvas_in = canvas
+    canvas_out = torch.empty_like(canvas)
+
+    def step(s):
+        dg.denoise_pass(model, cache, canvas_in, logits, ws)
+        dg.canvas_update(logits, n_ren, synth.SEED_RENOISE, s, canvas_out, ws)
+
+    # expert union per layer of this input (read once, outside the timed region)
+    unions = torch.zeros(cfg["n_layers"], dtype=torch.int32, device=dev)
+    model.set_taps({"unions": unions})
+    step(0)
+    model.set_taps(None)
+    torch.cuda.synchronize(dev)
+    unions_h = [int(u) for u in unions.cpu()]
+
+    for w in range(args.warmup):
+        step(w)
+    dg.device_status(ws)
+
+    def timed(K, profile):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if profile:
+            dg.profile_reset()
+            dg.profile_enable(True)
+        l0 = dg.launch_count()
+        for s in range(K):
+            flush.zero_()
+            ev[s][0].record(stream)
+            step(s)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if profile:
+            dg.profile_enable(False)
+        return sum(a.elapsed_time(b) for a, b in ev), dg.launch_count() - l0
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clk = Clocks(local)
+    clk.start()
+    total_ms, launches = timed(args.steps, profile=False)
+    clocks = clk.stop()
+    dg.device_status(ws)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+
+    # per-kernel breakdown with CUDA events on the launching stream (separate timed run)
+    prof_ms, _ = timed(args.steps, profile=True)
+    kern = {}
+    for kname in dg.KERNEL_KINDS:
+        ms, n = dg.profile_read(kname)
+        if n:
+            kern[kname] = {"launches": n, "avg_us": ms * 1e3 / n, "share": ms / max(prof_ms, 1e-9)}
+
+    # end to end through the public API with host buffers: H2D canvas, pass, update, D2H canvas
+    h_in = noise.clone().pin_memory()
+    h_out = torch.empty_like(h_in).pin_memory()
+    e2e_ms = []
+    for s in range(args.steps + args.warmup):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        canvas_in.copy_(h_in, non_blocking=True)
+        step(s)
+        h_out.copy_(canvas_out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if s >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+
+    ms_step = total_ms / args.steps
+    value = world * C * args.steps / (total_ms / 1e3)
+    e2e_value = world * C * args.steps / (e2e_total / 1e3)
+    hbm, tf_burst, tf_sust, peak_src = _peaks()
+
+    # whole-pass roofline (slower of FLOPs at the bf16 peak and bytes at HBM bandwidth)
+    flops = RF.pass_flops(cfg, P, C)
+    nbytes = RF.pass_bytes(cfg, P, C, unions_h) + RF.update_bytes(cfg, C)
+    t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
+    # dominant kernel: the gate/up grouped GEMM, HBM-bound on the union of expert weights
+    gu = kern.get("gemm_gate_up")
+    roof = None
+    if gu:
+        per_launch = RF.gate_up_bytes(cfg, unions_h[0], C * cfg["top_k"])
+        achieved = per_launch / (gu["avg_us"] * 1e-6) / 1e9
+        roof = {"kernel": "gemm_gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                "bytes_per_launch": per_launch}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "pass_latency_us": ms_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": _workload_desc(name, cfg), "l2": "flushed between steps (256 MB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "expert_union": unions_h},
+        "roofline": roof,
+        "pass_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof * 1e3 / ms_step, "flops": flops,
+                          "bytes": nbytes, "bound": "hbm" if nbytes / (hbm * 1e9) > flops / (tf_burst * 1e12)
+                          else "tensor", "peak_source": peak_src},
+        "kernels": kern,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": C * 4, "d2h_bytes_per_step": C * 4},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

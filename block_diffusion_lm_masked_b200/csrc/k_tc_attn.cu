@@ -9,7 +9,10 @@
 // transposed in the cache ([d][position]) so both MMAs read K-major operands.
 // The running max is only raised when it grows by more than 2^8 (log2 domain), so
 // O in TMEM is rescaled rarely; P and l use the same (possibly stale) max, which
-// leaves O / l exact.
+// leaves O / l exact.  P is carried as two bf16 terms, hi = bf16(p) and
+// lo = bf16(p - hi), and O accumulates hi V + lo V: the probabilities keep about 16
+// significant bits instead of 8, which keeps the attention output within a few
+// fp32-accumulation ulps of exact softmax attention.
 #include <math.h>
 
 #include "dg_common.cuh"
@@ -21,7 +24,7 @@ constexpr int AT_BQ = 128;
 constexpr int AT_BKEYS = 128;
 constexpr int AT_D = 128;
 constexpr uint32_t AT_HALF = 128 * 128;  // one [128 rows][64 bf16] swizzled block: 16 KB
-constexpr int AT_SMEM = 1024 + 12 * AT_HALF;  // Q (2 blocks), K[2] (4), Vt[2] (4), P (2)
+constexpr int AT_SMEM = 1024 + 14 * AT_HALF;  // Q (2 blocks), K[2] (4), Vt[2] (4), P hi (2), P lo (2)
 
 __global__ void __launch_bounds__(128, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -63,7 +66,8 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sQ = smem;                    // 2 blocks: d 0..63, d 64..127
   uint8_t* sK = smem + 2 * AT_HALF;      // [buf][2 blocks]
   uint8_t* sV = smem + 6 * AT_HALF;      // [buf][2 blocks]: V^T rows = d, K = keys 0..63 / 64..127
-  uint8_t* sP = smem + 10 * AT_HALF;     // 2 blocks: keys 0..63, 64..127
+  uint8_t* sP = smem + 10 * AT_HALF;     // P hi, 2 blocks: keys 0..63, 64..127
+  uint8_t* sPl = smem + 12 * AT_HALF;    // P lo, same layout
 
   if (warp == 0) tmem_alloc(&tmem_base_s, 256);
   if (tid == 32) {
@@ -183,23 +187,27 @@ __global__ void __launch_bounds__(128, 1)
       l *= alpha;
       m_used = rmax;
     }
-    // P = exp2(s - m_used) in bf16, written as the K-major A operand of the PV MMA
+    // P = exp2(s - m_used) as hi + lo bf16 terms, written as K-major A operands of the PV MMAs
 #pragma unroll
     for (int blk = 0; blk < 2; ++blk) {
       uint8_t* pb = sP + blk * AT_HALF;
+      uint8_t* pl = sPl + blk * AT_HALF;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
+        uint32_t wh[4], wl[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i0 = blk * 64 + c * 8 + 2 * e;
           const float p0 = (s[i0] == -INFINITY) ? 0.0f : exp2f(s[i0] - m_used);
           const float p1 = (s[i0 + 1] == -INFINITY) ? 0.0f : exp2f(s[i0 + 1] - m_used);
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          l += __low2float(pr) + __high2float(pr);
-          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+          l += p0 + p1;
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
+          wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
+          wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
         }
-        *reinterpret_cast<uint4*>(pb + sw128_offset(tid, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(pb + sw128_offset(tid, c)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(pl + sw128_offset(tid, c)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
     }
     fence_proxy_async_smem();
@@ -208,13 +216,16 @@ __global__ void __launch_bounds__(128, 1)
     if (tid == 0) {
       if (!abort_s) {
         tc_fence_after();
-        const uint32_t pp = smem_u32(sP), v = smem_u32(sV + buf * 2 * AT_HALF);
+        const uint32_t pp = smem_u32(sP), pl = smem_u32(sPl), v = smem_u32(sV + buf * 2 * AT_HALF);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma(tmem_O, sw128_kmajor_desc(pp + kb * AT_HALF + kk * 32),
-                   sw128_kmajor_desc(v + kb * AT_HALF + kk * 32), idesc, (j > 0 || (kb | kk) != 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t vd = sw128_kmajor_desc(v + kb * AT_HALF + kk * 32);
+            tc_mma(tmem_O, sw128_kmajor_desc(pp + kb * AT_HALF + kk * 32), vd, idesc,
+                   (j > 0 || (kb | kk) != 0) ? 1u : 0u);
+            tc_mma(tmem_O, sw128_kmajor_desc(pl + kb * AT_HALF + kk * 32), vd, idesc, 1u);
+          }
       }
       tc_commit(&pv_bar);
     }

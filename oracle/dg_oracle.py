@@ -324,7 +324,7 @@ def denoise_pass(model, cache: Cache, canvas: np.ndarray, prec: Precision, logit
     return vocab_logits(model, x, prec, rows=logit_rows), taps
 
 
-def prefill_append(model, cache: Cache, tokens: np.ndarray, prec: Precision) -> Cache:
+def prefill_append(model, cache: Cache, tokens: np.ndarray, prec: Precision, taps: list | None = None) -> Cache:
     """Causal prefill of T tokens at positions P..P+T-1, appending their K/V (prefill mode).
 
     [DG-explainer] "Two modes, one model" / "Long-form text: chaining canvases": the
@@ -347,7 +347,10 @@ def prefill_append(model, cache: Cache, tokens: np.ndarray, prec: Precision) -> 
             break
         o = attention(q, out.k[l], out.v[l], mask)
         x = x + _attn_out(model, l, o, prec)
-        x = x + moe(model, l, x, prec)
+        tap = {} if taps is not None else None
+        x = x + moe(model, l, x, prec, tap)
+        if taps is not None:
+            taps.append(tap)
     return out
 
 

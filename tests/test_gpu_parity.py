@@ -82,15 +82,22 @@ def test_prefill_append_matches_oracle(dg):
     ws = st.workspace(300)
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 77, cfg["vocab"])
     more = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(9), 150, cfg["vocab"])
+    near_tie = set()   # positions whose oracle routing margin is below 1e-3 in some layer
     for toks in (prompt, more):
+        P0 = st.ocache.len
         dg.prefill_append(st.model, st.cache, torch.from_numpy(toks).cuda(), ws)
-        st.ocache = O.prefill_append(st.host, st.ocache, toks, st.prec)
+        taps = []
+        st.ocache = O.prefill_append(st.host, st.ocache, toks, st.prec, taps)
+        for t in taps:
+            near_tie |= {P0 + int(i) for i in np.nonzero(t["router_margin"] < PL.ROUTE_MARGIN)[0]}
     dg.device_status(ws)
     assert st.cache.len == 227 == st.ocache.len
+    keep = [p for p in range(227) if p not in near_tie]
     for l in range(cfg["n_layers"]):
         k, v = st.cache.logical(l)
-        assert PL.rel_err(k.reshape(-1, 128), st.ocache.k[l].reshape(-1, 128)) < 2e-2
-        assert PL.rel_err(v.reshape(-1, 128), st.ocache.v[l].reshape(-1, 128)) < 2e-2
+        ok, ov = st.ocache.k[l], st.ocache.v[l]
+        assert PL.rel_err(k[:, keep].reshape(-1, 128), ok[:, keep].reshape(-1, 128)) < 2e-2, l
+        assert PL.rel_err(v[:, keep].reshape(-1, 128), ov[:, keep].reshape(-1, 128)) < 2e-2, l
 
 
 def test_mask_worked_example_on_gpu(dg):
@@ -115,7 +122,7 @@ def test_chained_canvases_small(dg):
     cfg = dict(SMALL_BF16, n_layers=2)
     C, S, n_can = 64, 3, 2
     st = PL.Setup(cfg, 0, capacity=512, with_prefix=False)
-    ws = st.workspace(C)
+    ws = st.workspace(96)
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 96, cfg["vocab"])
     dg.prefill_append(st.model, st.cache, torch.from_numpy(prompt).cuda(), ws)
     oc = O.prefill_append(st.host, st.ocache, prompt, st.prec)
