@@ -214,11 +214,15 @@ extern "C" void dg_model_destroy(dg_model* m) { delete m; }
 // ---------------------------------------------------------------- workspace layout
 namespace {
 constexpr int kMaxAttnSplits = 16;
+constexpr int kMaxKsQkv = 4;   // split-K of the QKV projection
+constexpr int kMaxKsO = 8;     // split-K of the output projection
+constexpr int kSmemShared = 100 * 1024;  // GEMM stage budget when two CTAs share an SM
+constexpr int kSmemSolo = 200 * 1024;    // ... when one CTA owns the SM
 inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t err, upd, x, xn, qkv, q, o, part_o, part_lse, logits_r, topk_idx, topk_w, counts, offsets, perm, inv, uni, xs,
-      h, gu, ys, total;
+  size_t err, upd, x, xn, xn_lo, qkv, q, o, o_lo, part_o, part_lse, opart, topk_idx, topk_w, counts, offsets, perm,
+      inv, uni, xs, xs_lo, h, h_lo, gu, ys, total;
 };
 
 size_t upd_bytes(int C, int V) { return al((size_t)C * dg::update_splits(C, V) * sizeof(dg::UpdPart)); }
@@ -231,20 +235,23 @@ WsLayout layout(const dg_config& c, int T) {
     o += al(bytes);
     return r;
   };
+  const bool bf = is_bf16(c);
   const size_t ab = act_bytes(c);
-  const size_t H = c.hidden, E = c.n_experts, k = c.top_k, F = c.expert_ffn, d = c.head_dim;
+  const size_t H = c.hidden, k = c.top_k, F = c.expert_ffn, d = c.head_dim, E = c.n_experts;
   L.err = take(256);
   size_t upd_max = 0;
   for (int C = 1; C <= T; ++C) upd_max = upd_max > upd_bytes(C, c.vocab) ? upd_max : upd_bytes(C, c.vocab);
   L.upd = take(upd_max);
   L.x = take((size_t)T * H * 4);
   L.xn = take((size_t)T * H * ab);
-  L.qkv = take((size_t)T * qkv_rows(c) * 4);
+  L.xn_lo = take(bf ? (size_t)T * H * 2 : 0);
+  L.qkv = take((size_t)(bf ? kMaxKsQkv : 1) * T * qkv_rows(c) * 4);
   L.q = take((size_t)c.n_q_heads * T * d * ab);
   L.o = take((size_t)T * c.n_q_heads * d * ab);
-  L.part_o = take(is_bf16(c) ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
-  L.part_lse = take(is_bf16(c) ? (size_t)kMaxAttnSplits * c.n_q_heads * T * 4 : 0);
-  L.logits_r = take((size_t)T * E * 4);
+  L.o_lo = take(bf ? (size_t)T * c.n_q_heads * d * 2 : 0);
+  L.part_o = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
+  L.part_lse = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * 4 : 0);
+  L.opart = take((size_t)(bf ? kMaxKsO : 1) * T * H * 4);
   L.topk_idx = take((size_t)T * k * 4);
   L.topk_w = take((size_t)T * k * 4);
   L.counts = take(E * 4);
@@ -253,8 +260,10 @@ WsLayout layout(const dg_config& c, int T) {
   L.inv = take((size_t)T * k * 4);
   L.uni = take(4);
   L.xs = take((size_t)T * k * H * ab);
+  L.xs_lo = take(bf ? (size_t)T * k * H * 2 : 0);
   L.h = take((size_t)T * k * F * ab);
-  L.gu = take(is_bf16(c) ? 0 : (size_t)T * k * 2 * F * 4);
+  L.h_lo = take(bf ? (size_t)T * k * F * 2 : 0);
+  L.gu = take(bf ? 0 : (size_t)T * k * 2 * F * 4);
   L.ys = take((size_t)T * k * H * 4);
   L.total = o;
   return L;
@@ -271,6 +280,15 @@ struct Ws {
 };
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// split-K factor: a divisor of the k-block count, at most max_ks, keeping >= 2 k-blocks
+// per CTA and about two CTAs per SM at most
+int pick_ksplit(int m_tiles, int token_chunks, int nkb, int max_ks) {
+  int best = 1;
+  for (int ks = 1; ks <= max_ks; ++ks)
+    if (nkb % ks == 0 && nkb / ks >= 2 && m_tiles * token_chunks * ks <= 2 * 148) best = ks;
+  return best;
+}
 }  // namespace
 
 extern "C" size_t dg_workspace_bytes(const dg_config* cfg, int32_t max_tokens) {
@@ -285,26 +303,46 @@ extern "C" size_t dg_update_workspace_bytes(int32_t C, int32_t V) {
 // ---------------------------------------------------------------- the layer stack
 namespace {
 
-// GEMM smem budget: about half the SM so that two CTAs can share it
-constexpr int kGemmSmem = 100 * 1024;
+struct GemmCall {
+  int kind, epi;
+  const CUtensorMap* A;
+  const void* X;
+  const void* X_lo;  // null: single term
+  int x_rows, K, a_rows_per_group, n_groups;
+  const int* group_off;
+  int max_rows_per_group;
+  void* out;
+  void* out_lo;
+  int ld_out;
+  int k_splits;
+  size_t split_stride;
+  int smem_budget;
+};
 
-dg_status gemm_bf16(int kind, int epi, const CUtensorMap& A, const void* X, int x_rows, int K, int a_rows_per_group,
-                    int n_groups, const int* group_off, int max_rows_per_group, void* out, int ld_out, int* err,
-                    cudaStream_t st) {
-  CUtensorMap B;
-  dg_status s = map_rows(&B, X, (uint64_t)x_rows, (uint64_t)K, 16);
+dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
+  CUtensorMap B, B2;
+  dg_status s = map_rows(&B, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 16);
   if (s != DG_OK) return s;
+  if (g.X_lo) {
+    if ((s = map_rows(&B2, g.X_lo, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
+  } else {
+    B2 = B;
+  }
   dg::TcGemmParams p;
-  p.K = K;
-  p.a_rows_per_group = a_rows_per_group;
-  p.group_off = group_off;
-  p.n_tokens = x_rows;
-  p.out = out;
-  p.ld_out = ld_out;
-  p.smem_budget = kGemmSmem;
+  p.K = g.K;
+  p.a_rows_per_group = g.a_rows_per_group;
+  p.group_off = g.group_off;
+  p.n_tokens = g.x_rows;
+  p.out = g.out;
+  p.out_lo = g.out_lo;
+  p.ld_out = g.ld_out;
+  p.two_terms = g.X_lo != nullptr;
+  p.k_splits = g.k_splits;
+  p.split_stride = g.split_stride;
+  p.smem_budget = g.smem_budget;
   p.err = err;
-  const int m_tiles = (epi == dg::EPI_SWIGLU_BF16) ? a_rows_per_group / 128 : a_rows_per_group / 128;
-  LAUNCH(kind, st, dg::launch_tc_gemm(epi, A, B, p, m_tiles, n_groups, max_rows_per_group, st));
+  LAUNCH(g.kind, st,
+         dg::launch_tc_gemm(g.epi, *g.A, B, B2, p, g.a_rows_per_group / 128, g.n_groups, g.max_rows_per_group, st));
   return DG_OK;
 }
 
@@ -320,7 +358,7 @@ int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
   return splits;
 }
 
-// attention of n_q new rows at positions pos0.. over cache keys [0, n_keys)
+// attention of n_q new rows at positions pos0.. over cache keys [0, n_keys) -> ws.o (+ ws.o_lo)
 dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0, int n_keys,
                     int causal, cudaStream_t st) {
   const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
@@ -360,91 +398,99 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
   p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   p.out = ws.at<bf16>(ws.L.o);
+  p.out_lo = ws.at<bf16>(ws.L.o_lo);
   p.part_o = ws.at<float>(ws.L.part_o);
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
   LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mq, mk, mv, p, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
-           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<void>(ws.L.o), 1, st));
+           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),
+                                 ws.at<bf16>(ws.L.o_lo), st));
   return DG_OK;
 }
 
-// one transformer layer over n rows at positions pos0.. whose residual is in ws.x.
+// One transformer layer over n rows at positions pos0..  On entry ws.x holds the
+// residual stream and ws.xn (+ xn_lo) its RMSNorm; on exit the same for the next layer
+// (final: ws.xn single-term, the vocabulary projection's input).
 // stop_after_kv: write this layer's K/V and return (last layer of a prefill).
 template <typename T>
 dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, int n, int pos0, int causal,
-                bool stop_after_kv, cudaStream_t st) {
+                bool stop_after_kv, bool final_layer, cudaStream_t st) {
   const dg_config& c = m->cfg;
   const dg_layer_weights& W = m->layers[l];
   const int H = c.hidden, nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
-  const int E = c.n_experts, k = c.top_k, F = c.expert_ffn;
+  const int E = c.n_experts, k = c.top_k, F = c.expert_ffn, QR = qkv_rows(c);
   const bool bf = is_bf16(c);
   int* err = ws.err();
+  T* xn_lo = bf ? ws.at<T>(ws.L.xn_lo) : nullptr;
   dg_status s;
-  // attention block: RMSNorm -> QKV -> RoPE (+ K/V into the cache) -> attention -> O + residual
-  LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<T>(ws.at<float>(ws.L.x), n, H, c.rms_eps, ws.at<T>(ws.L.xn), st));
+  const int chunks = ceil_div(n, 256);
+  // ---- attention block: QKV (split-K partials) -> RoPE + K/V into the cache -> attention -> output projection
+  int ks_qkv = 1, ks_o = 1;
   if (bf) {
-    if ((s = gemm_bf16(DG_K_GEMM_QKV, dg::EPI_STORE_F32, m->maps[l].qkv, ws.at<void>(ws.L.xn), n, H, qkv_rows(c), 1,
-                       nullptr, n, ws.at<float>(ws.L.qkv), qkv_rows(c), err, st)) != DG_OK)
-      return s;
+    ks_qkv = pick_ksplit(QR / 128, chunks, H / 64, kMaxKsQkv);
+    GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, ws.at<void>(ws.L.xn), xn_lo, n, H, QR, 1,
+               nullptr, n, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemSolo};
+    if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_QKV, st,
-           dg::launch_simt_gemm_f32(0, (const float*)W.w_qkv, ws.at<float>(ws.L.xn), nullptr, 1, n, n, qkv_rows(c),
-                                    H, ws.at<float>(ws.L.qkv), qkv_rows(c), st));
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_qkv, ws.at<float>(ws.L.xn), nullptr, 1, n, n, QR, H,
+                                    ws.at<float>(ws.L.qkv), QR, st));
   }
   LAUNCH(DG_K_ROPE_KV, st,
-         dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), n, nq, nkv, d, pos0, c.rope_theta, ws.at<T>(ws.L.q),
-                                    (T*)kc, (T*)vtc, cap, st));
+         dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), ks_qkv, (size_t)n * QR, n, nq, nkv, d, pos0, c.rope_theta,
+                                    ws.at<T>(ws.L.q), (T*)kc, (T*)vtc, cap, st));
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
-    if ((s = gemm_bf16(DG_K_GEMM_O, dg::EPI_ADD_F32, m->maps[l].o, ws.at<void>(ws.L.o), n, nq * d, H, 1, nullptr, n,
-                       ws.at<float>(ws.L.x), H, err, st)) != DG_OK)
-      return s;
+    ks_o = pick_ksplit(H / 128, chunks, nq * d / 64, kMaxKsO);
+    GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo), n,
+               nq * d, H, 1, nullptr, n, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H, kSmemSolo};
+    if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_O, st,
-           dg::launch_simt_gemm_f32(1, (const float*)W.w_o, ws.at<float>(ws.L.o), nullptr, 1, n, n, H, nq * d,
-                                    ws.at<float>(ws.L.x), H, st));
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_o, ws.at<float>(ws.L.o), nullptr, 1, n, n, H, nq * d,
+                                    ws.at<float>(ws.L.opart), H, st));
   }
+  // ---- MoE block: residual + RMSNorm + router + top-k -> histogram / permutation -> experts -> combine + RMSNorm
+  LAUNCH(DG_K_ROUTER, st,
+         dg::launch_router_fused<T>(ws.at<float>(ws.L.x), ws.at<float>(ws.L.opart), ks_o, (size_t)n * H, W.w_router,
+                                    n, H, E, k, c.rms_eps, nullptr, ws.at<int32_t>(ws.L.topk_idx),
+                                    ws.at<float>(ws.L.topk_w), ws.at<T>(ws.L.xn), xn_lo, st));
   if (m->taps_on && !m->tap_x_attn.empty() && m->tap_x_attn[l])
     if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
         cudaSuccess)
       return fail(DG_ERR_CUDA, "tap copy failed");
-  // MoE block: router (fp32) -> top-k -> histogram/permutation -> gather -> experts -> combine
-  LAUNCH(DG_K_ROUTER, st,
-         dg::launch_router<T>(ws.at<float>(ws.L.x), W.w_router, n, H, E, c.rms_eps, ws.at<float>(ws.L.logits_r),
-                              ws.at<T>(ws.L.xn), st));
-  LAUNCH(DG_K_TOPK, st,
-         dg::launch_topk(ws.at<float>(ws.L.logits_r), n, E, k, ws.at<int32_t>(ws.L.topk_idx),
-                         ws.at<float>(ws.L.topk_w), st));
   LAUNCH(DG_K_PERMUTE, st,
          dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
                             ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
                             ws.at<int32_t>(ws.L.uni), st));
+  T* xs_lo = bf ? ws.at<T>(ws.L.xs_lo) : nullptr;
   LAUNCH(DG_K_GATHER, st,
-         dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), ws.at<int32_t>(ws.L.perm), n * k, k, H, ws.at<T>(ws.L.xs), st));
+         dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), xn_lo, ws.at<int32_t>(ws.L.perm), n * k, k, H,
+                                   ws.at<T>(ws.L.xs), xs_lo, st));
   const int* off = ws.at<int>(ws.L.offsets);
   if (bf) {
-    if ((s = gemm_bf16(DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, m->maps[l].gate_up, ws.at<void>(ws.L.xs), n * k, H,
-                       2 * F, E, off, n, ws.at<void>(ws.L.h), F, err, st)) != DG_OK)
-      return s;
-    if ((s = gemm_bf16(DG_K_GEMM_DOWN, dg::EPI_STORE_F32, m->maps[l].down, ws.at<void>(ws.L.h), n * k, F, H, E, off,
-                       n, ws.at<float>(ws.L.ys), H, err, st)) != DG_OK)
-      return s;
+    GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate_up, ws.at<void>(ws.L.xs), xs_lo, n * k, H,
+                2 * F, E, off, n, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0, kSmemShared};
+    if ((s = gemm_bf16(gu, err, st)) != DG_OK) return s;
+    GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo),
+                n * k, F, H, E, off, n, ws.at<float>(ws.L.ys), nullptr, H, 1, 0, kSmemShared};
+    if ((s = gemm_bf16(dn, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_GATE_UP, st,
            dg::launch_simt_gemm_f32(0, (const float*)W.w_gate_up, ws.at<float>(ws.L.xs), off, E, n, n * k, 2 * F, H,
                                     ws.at<float>(ws.L.gu), 2 * F, st));
-    LAUNCH(DG_K_SWIGLU, st,
-           dg::launch_swiglu_packed_f32(ws.at<float>(ws.L.gu), n * k, F, ws.at<float>(ws.L.h), st));
+    LAUNCH(DG_K_SWIGLU, st, dg::launch_swiglu_packed_f32(ws.at<float>(ws.L.gu), n * k, F, ws.at<float>(ws.L.h), st));
     LAUNCH(DG_K_GEMM_DOWN, st,
            dg::launch_simt_gemm_f32(0, (const float*)W.w_down, ws.at<float>(ws.L.h), off, E, n, n * k, H, F,
                                     ws.at<float>(ws.L.ys), H, st));
   }
   LAUNCH(DG_K_COMBINE, st,
-         dg::launch_combine(ws.at<float>(ws.L.ys), ws.at<int32_t>(ws.L.inv), ws.at<float>(ws.L.topk_w), n, k, H,
-                            ws.at<float>(ws.L.x), st));
+         dg::launch_combine_norm<T>(ws.at<float>(ws.L.ys), ws.at<int32_t>(ws.L.inv), ws.at<float>(ws.L.topk_w), n, k,
+                                    H, c.rms_eps, ws.at<float>(ws.L.x), ws.at<T>(ws.L.xn),
+                                    final_layer ? nullptr : xn_lo, st));
   if (m->taps_on) {
     auto cp = [&](void* dst, const void* src, size_t bytes) {
       return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
@@ -487,17 +533,21 @@ dg_status check_cache(const dg_config& c, const dg_kv_cache* cache) {
   return DG_OK;
 }
 
+// prefill: causal, the last layer stops after its K/V; denoise: bidirectional, the last
+// layer leaves the vocabulary projection's input in ws.xn
 template <typename T>
-dg_status run_stack(dg_model* m, const dg_kv_cache* cache, const int32_t* tokens, int n, int causal,
-                    bool skip_last_block, const Ws& ws, cudaStream_t st) {
+dg_status run_stack(dg_model* m, const dg_kv_cache* cache, const int32_t* tokens, int n, bool prefill, const Ws& ws,
+                    cudaStream_t st) {
   const dg_config& c = m->cfg;
   const int pos0 = cache->len;
+  T* xn_lo = is_bf16(c) ? ws.at<T>(ws.L.xn_lo) : nullptr;
   LAUNCH(DG_K_EMBED_NORM, st,
          dg::launch_embed_norm<T>(tokens, (const T*)m->embed, n, c.vocab, c.hidden, c.rms_eps, ws.at<float>(ws.L.x),
-                                  ws.at<T>(ws.L.xn), ws.err(), st));
+                                  ws.at<T>(ws.L.xn), xn_lo, ws.err(), st));
   for (int l = 0; l < c.n_layers; ++l) {
-    const bool last = (l == c.n_layers - 1) && skip_last_block;
-    dg_status s = layer<T>(m, l, ws, cache->k[l], cache->vt[l], cache->capacity, n, pos0, causal, last, st);
+    const bool last = l == c.n_layers - 1;
+    dg_status s = layer<T>(m, l, ws, cache->k[l], cache->vt[l], cache->capacity, n, pos0, prefill ? 1 : 0,
+                           last && prefill, last && !prefill, st);
     if (s != DG_OK) return s;
   }
   return DG_OK;
@@ -518,8 +568,8 @@ extern "C" dg_status dg_prefill_append(dg_model* m, dg_kv_cache* cache, const in
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool saved = m->taps_on;
   m->taps_on = false;
-  s = is_bf16(m->cfg) ? run_stack<bf16>(m, cache, d_tokens, T, 1, true, ws, st)
-                      : run_stack<float>(m, cache, d_tokens, T, 1, true, ws, st);
+  s = is_bf16(m->cfg) ? run_stack<bf16>(m, cache, d_tokens, T, true, ws, st)
+                      : run_stack<float>(m, cache, d_tokens, T, true, ws, st);
   m->taps_on = saved;
   if (s != DG_OK) return s;
   cache->len += T;
@@ -539,19 +589,15 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
   if ((s = check_ws(m->cfg, d_ws, ws_bytes, C, &ws)) != DG_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const dg_config& c = m->cfg;
-  s = is_bf16(c) ? run_stack<bf16>(m, cache, d_canvas, C, 0, false, ws, st)
-                 : run_stack<float>(m, cache, d_canvas, C, 0, false, ws, st);
+  s = is_bf16(c) ? run_stack<bf16>(m, cache, d_canvas, C, false, ws, st)
+                 : run_stack<float>(m, cache, d_canvas, C, false, ws, st);
   if (s != DG_OK) return s;
-  // final RMSNorm + vocabulary projection to fp32 logits
+  // vocabulary projection of the final RMSNorm (left in ws.xn by the last layer) to fp32 logits
   if (is_bf16(c)) {
-    LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<bf16>(ws.at<float>(ws.L.x), C, c.hidden, c.rms_eps,
-                                                        ws.at<bf16>(ws.L.xn), st));
-    if ((s = gemm_bf16(DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, m->out_map, ws.at<void>(ws.L.xn), C, c.hidden, c.vocab, 1,
-                       nullptr, C, d_logits, c.vocab, ws.err(), st)) != DG_OK)
-      return s;
+    GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, ws.at<void>(ws.L.xn), nullptr, C, c.hidden, c.vocab,
+               1, nullptr, C, d_logits, nullptr, c.vocab, 1, 0, kSmemShared};
+    if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
   } else {
-    LAUNCH(DG_K_RMS_NORM, st, dg::launch_rms_norm<float>(ws.at<float>(ws.L.x), C, c.hidden, c.rms_eps,
-                                                         ws.at<float>(ws.L.xn), st));
     LAUNCH(DG_K_GEMM_VOCAB, st,
            dg::launch_simt_gemm_f32(0, (const float*)m->w_out, ws.at<float>(ws.L.xn), nullptr, 1, C, C, c.vocab,
                                     c.hidden, d_logits, c.vocab, st));
@@ -700,9 +746,9 @@ extern "C" int64_t dg_launch_count(void) {
 }
 
 extern "C" dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups,
-                                        const void* X, int32_t x_rows, int32_t K, const int32_t* group_off,
-                                        int32_t max_rows_per_group, void* out, int32_t ld_out, int32_t* d_err,
-                                        dg_stream stream) {
+                                        const void* X, const void* X_lo, int32_t x_rows, int32_t K,
+                                        const int32_t* group_off, int32_t max_rows_per_group, void* out,
+                                        void* out_lo, int32_t ld_out, int32_t* d_err, dg_stream stream) {
   DG_CHECK_ARG(W && X && out && d_err, "NULL pointer");
   DG_CHECK_ARG(epi >= 0 && epi <= 2, "epi must be 0, 1 or 2");
   DG_CHECK_ARG(K > 0 && K % 64 == 0 && a_rows_per_group > 0 && a_rows_per_group % 128 == 0 && n_groups > 0 &&
@@ -712,13 +758,14 @@ extern "C" dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_ro
   CUtensorMap A;
   dg_status s = map_rows(&A, W, (uint64_t)n_groups * a_rows_per_group, (uint64_t)K, 128);
   if (s != DG_OK) return s;
-  return gemm_bf16(DG_K_GEMM_QKV, epi, A, X, x_rows, K, a_rows_per_group, n_groups, group_off, max_rows_per_group,
-                   out, ld_out, d_err, reinterpret_cast<cudaStream_t>(stream));
+  GemmCall g{DG_K_GEMM_QKV, epi, &A, X, X_lo, x_rows, K, a_rows_per_group, n_groups, group_off, max_rows_per_group,
+             out, out_lo, ld_out, 1, 0, kSmemShared};
+  return gemm_bf16(g, d_err, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,
                                              int32_t pos0, int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv,
-                                             void* out, void* d_ws, size_t ws_bytes, dg_stream stream) {
+                                             void* out, void* out_lo, void* d_ws, size_t ws_bytes, dg_stream stream) {
   DG_CHECK_ARG(q && k && vt && out && d_ws, "NULL pointer");
   DG_CHECK_ARG(nq > 0 && nkv > 0 && nq % nkv == 0 && n_q > 0 && n_keys > 0 && n_keys <= cap && cap % 8 == 0,
                "bad attention shape");
@@ -746,6 +793,17 @@ extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const
   if ((s = attention(c, ws, const_cast<void*>(k), const_cast<void*>(vt), cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
     return s;
   e = cudaMemcpyAsync(out, ws.at<void>(ws.L.o), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && out_lo)
+    e = cudaMemcpyAsync(out_lo, ws.at<void>(ws.L.o_lo), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy o: %s", cudaGetErrorString(e));
+  return DG_OK;
+}
+
+extern "C" dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream) {
+  DG_CHECK_ARG(d_ws, "workspace is NULL");
+  DG_CHECK_ARG(timeout_ms >= 1 && timeout_ms <= 10000, "timeout_ms must be in [1, 10000]");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LAUNCH(DG_K_COUNT - 1, st,
+         dg::launch_bounded_wait_selftest(static_cast<int*>(d_ws), (uint64_t)timeout_ms * 1000000ull, st));
   return DG_OK;
 }

@@ -93,6 +93,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Same bounded wait with a caller-chosen limit (used by the timeout self-test).
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns, int* err, int code) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) {
+      if (err) atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Bounded wait used only while winding down after an abort: waits for work already
 // issued (TMA loads, MMAs) to land, ignoring the abort flag, for at most DG_WAIT_NS.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {

@@ -25,10 +25,21 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 }
 
 // ---------------------------------------------------------------- embedding + RMSNorm
-// x[t] = embed[tokens[t]] (fp32), xn[t] = x[t] / sqrt(mean(x[t]^2) + eps) in the activation dtype
+// An fp32 activation v handed to a bf16 GEMM is stored as hi = bf16(v) and
+// lo = bf16(v - hi); the GEMM accumulates W hi + W lo, which carries ~16 significant
+// bits of v.  For the fp32 model T = float and there is no lo part.
+template <typename T>
+__device__ __forceinline__ void store_act(T* hi, T* lo, size_t i, float v) {
+  const T h = from_f32<T>(v);
+  hi[i] = h;
+  if (lo) lo[i] = from_f32<T>(v - to_f32(h));
+}
+
+// x[t] = embed[tokens[t]] (fp32), xn[t] = x[t] / sqrt(mean(x[t]^2) + eps)
 template <typename T>
 __global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ embed, int V, int H,
-                                  float eps, float* __restrict__ x, T* __restrict__ xn, int* __restrict__ err) {
+                                  float eps, float* __restrict__ x, T* __restrict__ xn, T* __restrict__ xn_lo,
+                                  int* __restrict__ err) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   int tok = tokens[t];
@@ -46,32 +57,14 @@ __global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, const T* _
   }
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)H + eps);
-  for (int h = threadIdx.x; h < H; h += blockDim.x) xn[(size_t)t * H + h] = from_f32<T>(xr[h] * inv);
-}
-
-template <typename T>
-__global__ void rms_norm_kernel(const float* __restrict__ x, int H, float eps, T* __restrict__ xn) {
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  const float* xr = x + (size_t)t * H;
-  float ss = 0.0f;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) ss += xr[h] * xr[h];
-  ss = block_sum(ss, red);
-  const float inv = 1.0f / sqrtf(ss / (float)H + eps);
-  for (int h = threadIdx.x; h < H; h += blockDim.x) xn[(size_t)t * H + h] = from_f32<T>(xr[h] * inv);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) store_act(xn, xn_lo, (size_t)t * H + h, xr[h] * inv);
 }
 
 template <typename T>
 cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int V, int H, float eps, float* x, T* xn,
-                              int* err, cudaStream_t st) {
+                              T* xn_lo, int* err, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  embed_norm_kernel<T><<<n, 256, 0, st>>>(tokens, embed, V, H, eps, x, xn, err);
-  return cudaGetLastError();
-}
-template <typename T>
-cudaError_t launch_rms_norm(const float* x, int n, int H, float eps, T* xn, cudaStream_t st) {
-  if (n <= 0) return cudaSuccess;
-  rms_norm_kernel<T><<<n, 256, 0, st>>>(x, H, eps, xn);
+  embed_norm_kernel<T><<<n, 256, 0, st>>>(tokens, embed, V, H, eps, x, xn, xn_lo, err);
   return cudaGetLastError();
 }
 
@@ -80,9 +73,10 @@ cudaError_t launch_rms_norm(const float* x, int n, int H, float eps, T* xn, cuda
 // (angles in double precision), then q -> q[h][t][:], k -> K[kvh][pos][:],
 // v -> V^T[kvh][:][pos], all in the activation dtype.
 template <typename T>
-__global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nq, int nkv, int d, int pos0, float theta,
-                                    int n, T* __restrict__ q, T* __restrict__ kc, T* __restrict__ vtc, int cap) {
-  extern __shared__ float cs[];  // [d/2] cos, [d/2] sin
+__global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, size_t part_stride, int nq, int nkv,
+                                    int d, int pos0, float theta, int n, T* __restrict__ q, T* __restrict__ kc,
+                                    T* __restrict__ vtc, int cap) {
+  extern __shared__ float cs[];  // [d/2] cos, [d/2] sin, then the summed qkv row
   const int t = blockIdx.x;
   const int half = d / 2;
   const int pos = pos0 + t;
@@ -93,9 +87,14 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nq, int n
     cs[i] = (float)cn;
     cs[half + i] = (float)sn;
   }
-  __syncthreads();
   const int W = (nq + 2 * nkv) * d;
-  const float* row = qkv + (size_t)t * W;
+  float* row = cs + d;  // qkv row = sum of the split-K partials, in a fixed order
+  for (int i = threadIdx.x; i < W; i += blockDim.x) {
+    float v = 0.0f;
+    for (int s = 0; s < n_parts; ++s) v += qkv[s * part_stride + (size_t)t * W + i];
+    row[i] = v;
+  }
+  __syncthreads();
   // q and k heads: pairs (i, i + d/2)
   for (int idx = threadIdx.x; idx < (nq + nkv) * half; idx += blockDim.x) {
     const int hh = idx / half, i = idx % half;
@@ -119,11 +118,12 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nq, int n
 }
 
 template <typename T>
-cudaError_t launch_rope_scatter(const float* qkv, int n, int nq, int nkv, int d, int pos0, float theta, T* q,
-                                T* kcache, T* vtcache, int cap, cudaStream_t st) {
+cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
+                                int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  rope_scatter_kernel<T><<<n, 256, d * sizeof(float), st>>>(qkv, nq, nkv, d, pos0, theta, n, q, kcache, vtcache,
-                                                             cap);
+  const size_t smem = (size_t)(d + (nq + 2 * nkv) * d) * sizeof(float);
+  rope_scatter_kernel<T><<<n, 256, smem, st>>>(qkv, n_parts, part_stride, nq, nkv, d, pos0, theta, n, q, kcache,
+                                                vtcache, cap);
   return cudaGetLastError();
 }
 
@@ -255,117 +255,122 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- router
-// logits[t][e] = sum_h xn[t][h] * w_router[e][h], xn = x / rms(x) in fp32.
-// CTA: 8 tokens x 32 experts; column-block 0 also writes xn in the activation dtype
-// (the expert input).
-constexpr int RT_TOK = 8, RT_EXP = 32, RT_K = 64;
+// ---------------------------------------------------------------- residual + RMSNorm + router + top-k
+// Per token: x += sum of the output-projection partials (fixed order); xn = x / rms(x)
+// in fp32; router logits l[e] = xn . w_router[e] (fp32); the k largest (ties to the
+// lower expert id) and their softmax weights.  xn is also stored (hi/lo) as the expert
+// input.  CTA = RTF_TOK tokens, 256 threads; warp w handles experts w, w + 8, ...
+constexpr int RTF_TOK = 4;
 template <typename T>
-__global__ void router_kernel(const float* __restrict__ x, const float* __restrict__ wr, int n, int H, int E,
-                              float eps, float* __restrict__ logits, T* __restrict__ xn_out) {
-  __shared__ float inv_s[RT_TOK];
-  __shared__ float sx[RT_TOK][RT_K];
-  __shared__ float sw[RT_EXP][RT_K + 1];
+__global__ void __launch_bounds__(256) router_fused_kernel(
+    float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
+    const float* __restrict__ wr, int n, int H, int E, int k, float eps, float* __restrict__ logits_out,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, T* __restrict__ xn, T* __restrict__ xn_lo) {
+  extern __shared__ float sm[];  // xs[RTF_TOK][H], lg[RTF_TOK][E]
+  float* xs = sm;
+  float* lg = sm + RTF_TOK * H;
+  __shared__ float inv_s[RTF_TOK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * RT_TOK, e0 = blockIdx.y * RT_EXP;
-  {
-    const int t = t0 + warp;
+  const int t0 = blockIdx.x * RTF_TOK;
+  const int nt = min(RTF_TOK, n - t0);
+  // residual add of the partials
+  for (int i = threadIdx.x; i < nt * H; i += blockDim.x) {
+    const int a = i / H, h = i % H;
+    const size_t o = (size_t)(t0 + a) * H + h;
+    float v = x[o];
+    for (int s = 0; s < n_parts; ++s) v += parts[s * part_stride + o];
+    x[o] = v;
+    xs[a * H + h] = v;
+  }
+  __syncthreads();
+  if (warp < RTF_TOK) {
     float ss = 0.0f;
-    if (t < n)
-      for (int h = lane; h < H; h += 32) ss += x[(size_t)t * H + h] * x[(size_t)t * H + h];
+    if (warp < nt)
+      for (int h = lane; h < H; h += 32) ss += xs[warp * H + h] * xs[warp * H + h];
     ss = warp_sum(ss);
     if (lane == 0) inv_s[warp] = 1.0f / sqrtf(ss / (float)H + eps);
   }
   __syncthreads();
-  if (blockIdx.y == 0) {
-    for (int i = threadIdx.x; i < RT_TOK * H; i += blockDim.x) {
-      const int tt = i / H, h = i % H;
-      if (t0 + tt < n) xn_out[(size_t)(t0 + tt) * H + h] = from_f32<T>(x[(size_t)(t0 + tt) * H + h] * inv_s[tt]);
+  for (int i = threadIdx.x; i < nt * H; i += blockDim.x) {
+    const int a = i / H;
+    const float v = xs[i] * inv_s[a];
+    xs[i] = v;
+    store_act(xn, xn_lo, (size_t)t0 * H + i, v);
+  }
+  __syncthreads();
+  // logits: one expert row per warp iteration, float4 over H, all tokens of the CTA at once
+  for (int e = warp; e < E; e += 8) {
+    const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)e * H);
+    float acc[RTF_TOK] = {};
+    for (int i = lane; i < H / 4; i += 32) {
+      const float4 w = w4[i];
+#pragma unroll
+      for (int a = 0; a < RTF_TOK; ++a) {
+        const float4 v = reinterpret_cast<const float4*>(xs + a * H)[i];
+        acc[a] = fmaf(w.x, v.x, fmaf(w.y, v.y, fmaf(w.z, v.z, fmaf(w.w, v.w, acc[a]))));
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < RTF_TOK; ++a) {
+      const float r = warp_sum(acc[a]);
+      if (lane == 0) lg[a * E + e] = r;
     }
   }
-  const int tt = warp, e = e0 + lane;
-  float acc = 0.0f;
-  for (int k0 = 0; k0 < H; k0 += RT_K) {
-    for (int i = threadIdx.x; i < RT_TOK * RT_K; i += blockDim.x) {
-      const int a = i / RT_K, kk = i % RT_K;
-      const int t = t0 + a;
-      sx[a][kk] = (t < n && k0 + kk < H) ? x[(size_t)t * H + k0 + kk] * inv_s[a] : 0.0f;
+  __syncthreads();
+  if (logits_out)
+    for (int i = threadIdx.x; i < nt * E; i += blockDim.x) logits_out[(size_t)t0 * E + i] = lg[i];
+  // top-k: warp a < nt selects for token a
+  if (warp < nt) {
+    const float* l = lg + warp * E;
+    float chosen[16];
+    int chosen_id[16];
+    unsigned taken = 0u;  // bit i: entry lane + 32 i already chosen
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || l[e] > bv || (l[e] == bv && e < bi))) {
+          bv = l[e];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      chosen[j] = bv;
+      chosen_id[j] = bi;
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     }
-    for (int i = threadIdx.x; i < RT_EXP * RT_K; i += blockDim.x) {
-      const int a = i / RT_K, kk = i % RT_K;
-      sw[a][kk] = (e0 + a < E && k0 + kk < H) ? wr[(size_t)(e0 + a) * H + k0 + kk] : 0.0f;
+    if (lane == 0) {
+      float den = 0.0f;
+      for (int j = 0; j < k; ++j) den += expf(chosen[j] - chosen[0]);
+      for (int j = 0; j < k; ++j) {
+        topk_idx[(size_t)(t0 + warp) * k + j] = chosen_id[j];
+        topk_w[(size_t)(t0 + warp) * k + j] = expf(chosen[j] - chosen[0]) / den;
+      }
     }
-    __syncthreads();
-#pragma unroll 16
-    for (int kk = 0; kk < RT_K; ++kk) acc = fmaf(sx[tt][kk], sw[lane][kk], acc);
-    __syncthreads();
   }
-  if (t0 + tt < n && e < E) logits[(size_t)(t0 + tt) * E + e] = acc;
 }
 
 template <typename T>
-cudaError_t launch_router(const float* x, const float* w_router, int n, int H, int E, float eps, float* logits,
-                          T* xn, cudaStream_t st) {
+cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_t part_stride, const float* w_router,
+                                int n, int H, int E, int k, float eps, float* logits, int32_t* topk_idx, float* topk_w,
+                                T* xn, T* xn_lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  dim3 grid((n + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
-  router_kernel<T><<<grid, 256, 0, st>>>(x, w_router, n, H, E, eps, logits, xn);
-  return cudaGetLastError();
-}
-
-// top-k by value (ties to the lower expert id), weights = softmax over the k chosen logits
-__global__ void topk_kernel(const float* __restrict__ logits, int n, int E, int k, int32_t* __restrict__ idx,
-                            float* __restrict__ w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= n) return;
-  const float* lg = logits + (size_t)warp * E;
-  float v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = (e < E) ? lg[e] : -INFINITY;
-  }
-  float chosen[16];
-  int chosen_id[16];
-  unsigned taken = 0u;  // bit i: entry lane + 32 i already chosen
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    chosen[j] = bv;
-    chosen_id[j] = bi;
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-  }
-  if (lane == 0) {
-    float den = 0.0f;
-    for (int j = 0; j < k; ++j) den += expf(chosen[j] - chosen[0]);
-    for (int j = 0; j < k; ++j) {
-      idx[(size_t)warp * k + j] = chosen_id[j];
-      w[(size_t)warp * k + j] = expf(chosen[j] - chosen[0]) / den;
-    }
-  }
-}
-
-cudaError_t launch_topk(const float* logits, int n, int E, int k, int32_t* idx, float* w, cudaStream_t st) {
-  if (n <= 0) return cudaSuccess;
-  if (E > 256 || k > 16 || k > E) return cudaErrorInvalidValue;
-  const int threads = 256;
-  topk_kernel<<<(n * 32 + threads - 1) / threads, threads, 0, st>>>(logits, n, E, k, idx, w);
+  if (E > 256 || k > 16 || k > E || (H % 4) != 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)RTF_TOK * (H + E) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  router_fused_kernel<T><<<(n + RTF_TOK - 1) / RTF_TOK, 256, smem, st>>>(x, parts, n_parts, part_stride, w_router, n,
+                                                                          H, E, k, eps, logits, topk_idx, topk_w, xn,
+                                                                          xn_lo);
   return cudaGetLastError();
 }
 
@@ -435,22 +440,31 @@ cudaError_t launch_permute(const int32_t* idx, int n, int k, int E, int32_t* cou
   return cudaGetLastError();
 }
 
-// xs[p] = xn[perm[p] / k]  (16-byte vector copies; H * sizeof(T) is a multiple of 16)
+// xs[p] = xn[perm[p] / k] for the hi and (if present) lo parts; 16-byte vector copies
 template <typename T>
-__global__ void gather_rows_kernel(const T* __restrict__ xn, const int32_t* __restrict__ perm, int k, int H,
-                                   T* __restrict__ xs) {
+__global__ void gather_rows_kernel(const T* __restrict__ xn, const T* __restrict__ xn_lo,
+                                   const int32_t* __restrict__ perm, int k, int H, T* __restrict__ xs,
+                                   T* __restrict__ xs_lo) {
   const int p = blockIdx.x;
   const int t = perm[p] / k;
-  const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * H);
-  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
   const int nv = H * (int)sizeof(T) / 16;
-  for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  }
+  if (xn_lo) {
+    const uint4* src = reinterpret_cast<const uint4*>(xn_lo + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs_lo + (size_t)p * H);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  }
 }
 
 template <typename T>
-cudaError_t launch_gather_rows(const T* xn, const int32_t* perm, int rows, int k, int H, T* xs, cudaStream_t st) {
+cudaError_t launch_gather_rows(const T* xn, const T* xn_lo, const int32_t* perm, int rows, int k, int H, T* xs,
+                               T* xs_lo, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  gather_rows_kernel<T><<<rows, 128, 0, st>>>(xn, perm, k, H, xs);
+  gather_rows_kernel<T><<<rows, 128, 0, st>>>(xn, xn_lo, perm, k, H, xs, xs_lo);
   return cudaGetLastError();
 }
 
@@ -470,18 +484,24 @@ cudaError_t launch_swiglu_packed_f32(const float* gu, int rows, int F, float* h,
   return cudaGetLastError();
 }
 
-// x[t] += sum_j w[t][j] * ys[inv[t*k + j]], slots in order j = 0..k-1
-__global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __restrict__ inv,
-                               const float* __restrict__ w, int k, int H, float* __restrict__ x) {
+// x[t] += sum_j w[t][j] * ys[inv[t*k + j]] (slots in order j = 0..k-1), then
+// xn[t] = x[t] / rms(x[t]) for the next consumer (next layer's QKV, or the vocabulary
+// projection with xn_lo = null).
+template <typename T>
+__global__ void combine_norm_kernel(const float* __restrict__ ys, const int32_t* __restrict__ inv,
+                                    const float* __restrict__ w, int k, int H, float eps, float* __restrict__ x,
+                                    T* __restrict__ xn, T* __restrict__ xn_lo) {
   const int t = blockIdx.x;
   __shared__ int rows[16];
   __shared__ float ws[16];
+  __shared__ float red[32];
   if (threadIdx.x < k) {
     rows[threadIdx.x] = inv[t * k + threadIdx.x];
     ws[threadIdx.x] = w[t * k + threadIdx.x];
   }
   __syncthreads();
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * H);
+  float ss = 0.0f;
   for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
@@ -497,13 +517,25 @@ __global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __re
     v.z += acc.z;
     v.w += acc.w;
     xr[i] = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = block_sum(ss, red);
+  const float invr = 1.0f / sqrtf(ss / (float)H + eps);
+  for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+    const float4 v = xr[i];
+    const size_t o = (size_t)t * H + 4 * i;
+    store_act(xn, xn_lo, o + 0, v.x * invr);
+    store_act(xn, xn_lo, o + 1, v.y * invr);
+    store_act(xn, xn_lo, o + 2, v.z * invr);
+    store_act(xn, xn_lo, o + 3, v.w * invr);
   }
 }
-cudaError_t launch_combine(const float* ys, const int32_t* inv, const float* w, int n, int k, int H, float* x,
-                           cudaStream_t st) {
+template <typename T>
+cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float* w, int n, int k, int H, float eps,
+                                float* x, T* xn, T* xn_lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   if (k > 16 || (H % 4) != 0) return cudaErrorInvalidValue;
-  combine_kernel<<<n, 256, 0, st>>>(ys, inv, w, k, H, x);
+  combine_norm_kernel<T><<<n, 256, 0, st>>>(ys, inv, w, k, H, eps, x, xn, xn_lo);
   return cudaGetLastError();
 }
 
@@ -658,22 +690,35 @@ cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- timeout self-test
+// One thread waits on an mbarrier that nothing will complete; the bounded wait gives
+// up after limit_ns, records the error code and the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel(int* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait_ns(&bar, 0, limit_ns, err, DG_DEVERR_TIMEOUT_FULL);
+  }
+}
+cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- explicit instantiations
-template cudaError_t launch_embed_norm<float>(const int32_t*, const float*, int, int, int, float, float*, float*,
-                                              int*, cudaStream_t);
-template cudaError_t launch_embed_norm<bf16>(const int32_t*, const bf16*, int, int, int, float, float*, bf16*, int*,
-                                             cudaStream_t);
-template cudaError_t launch_rms_norm<float>(const float*, int, int, float, float*, cudaStream_t);
-template cudaError_t launch_rms_norm<bf16>(const float*, int, int, float, bf16*, cudaStream_t);
-template cudaError_t launch_rope_scatter<float>(const float*, int, int, int, int, int, float, float*, float*, float*,
-                                                int, cudaStream_t);
-template cudaError_t launch_rope_scatter<bf16>(const float*, int, int, int, int, int, float, bf16*, bf16*, bf16*, int,
-                                               cudaStream_t);
-template cudaError_t launch_router<float>(const float*, const float*, int, int, int, float, float*, float*,
-                                          cudaStream_t);
-template cudaError_t launch_router<bf16>(const float*, const float*, int, int, int, float, float*, bf16*,
-                                         cudaStream_t);
-template cudaError_t launch_gather_rows<float>(const float*, const int32_t*, int, int, int, float*, cudaStream_t);
-template cudaError_t launch_gather_rows<bf16>(const bf16*, const int32_t*, int, int, int, bf16*, cudaStream_t);
+#define DG_INST(T)                                                                                                \
+  template cudaError_t launch_embed_norm<T>(const int32_t*, const T*, int, int, int, float, float*, T*, T*, int*, \
+                                            cudaStream_t);                                                        \
+  template cudaError_t launch_rope_scatter<T>(const float*, int, size_t, int, int, int, int, int, float, T*, T*,  \
+                                              T*, int, cudaStream_t);                                             \
+  template cudaError_t launch_router_fused<T>(float*, const float*, int, size_t, const float*, int, int, int, int, \
+                                              float, float*, int32_t*, float*, T*, T*, cudaStream_t);             \
+  template cudaError_t launch_gather_rows<T>(const T*, const T*, const int32_t*, int, int, int, T*, T*,          \
+                                             cudaStream_t);                                                       \
+  template cudaError_t launch_combine_norm<T>(const float*, const int32_t*, const float*, int, int, int, float,   \
+                                              float*, T*, T*, cudaStream_t);
+DG_INST(float)
+DG_INST(bf16)
 
 }  // namespace dg

@@ -239,20 +239,30 @@ __global__ void __launch_bounds__(128, 1)
     const bool valid = qrow < p.n_q;
     const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
     if (p.n_splits == 1) {
-      __nv_bfloat16* o = p.out + (size_t)qrow * p.nq * AT_D + (size_t)h * AT_D;
+      const size_t base = (size_t)qrow * p.nq * AT_D + (size_t)h * AT_D;
 #pragma unroll
       for (int c = 0; c < AT_D / 16; ++c) {
         uint32_t r[16];
         tmem_ld16(tmem_O + lane_off + c * 16, r);
         tc_wait_ld();
         if (valid) {
-          uint32_t w[8];
+          uint32_t w[8], wl[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(o + c * 16);
+          for (int e = 0; e < 8; ++e) {
+            const float a = __uint_as_float(r[2 * e]) * inv_l, b = __uint_as_float(r[2 * e + 1]) * inv_l;
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
+            w[e] = *reinterpret_cast<const uint32_t*>(&hi);
+            wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.out + base + c * 16);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (p.out_lo) {
+            uint4* dl = reinterpret_cast<uint4*>(p.out_lo + base + c * 16);
+            dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+          }
         }
       }
     } else {
@@ -285,7 +295,7 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_splits,
-                                  int nq, int n_q, int d, void* out, int out_is_bf16) {
+                                  int nq, int n_q, int d, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
   const int qrow = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
   float mx = -INFINITY;
   for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, part_lse[((size_t)s * nq + h) * n_q + qrow]);
@@ -302,10 +312,9 @@ __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float*
     }
     const float v = den > 0.0f ? num / den : 0.0f;
     const size_t o = (size_t)qrow * nq * d + (size_t)h * d + dd;
-    if (out_is_bf16)
-      reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
-    else
-      reinterpret_cast<float*>(out)[o] = v;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    out[o] = hi;
+    if (out_lo) out_lo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 
@@ -319,8 +328,8 @@ cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& K, cons
 }
 
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
-                              void* out, int out_is_bf16, cudaStream_t st) {
-  attn_merge_kernel<<<dim3(n_q, nq), 128, 0, st>>>(part_o, part_lse, n_splits, nq, n_q, d, out, out_is_bf16);
+                              __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
+  attn_merge_kernel<<<dim3(n_q, nq), 128, 0, st>>>(part_o, part_lse, n_splits, nq, n_q, d, out, out_lo);
   return cudaGetLastError();
 }
 

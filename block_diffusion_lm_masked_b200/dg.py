@@ -83,8 +83,9 @@ def _load():
         "dg_kernel_name": (ctypes.c_char_p, [I32]),
         "dg_launch_count": (ctypes.c_int64, []),
         "dg_renoise_count": (I32, [I32, I32, I32, F32, F32]),
-        "dg_debug_gemm_bf16": (I32, [I32, P, I32, I32, P, I32, I32, P, I32, P, I32, P, P]),
-        "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, SZ, P]),
+        "dg_debug_bounded_wait": (I32, [P, I32, P]),
+        "dg_debug_gemm_bf16": (I32, [I32, P, I32, I32, P, P, I32, I32, P, I32, P, P, I32, P, P]),
+        "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -309,15 +310,22 @@ def launch_count() -> int:
 
 
 def debug_gemm_bf16(epi, W, a_rows_per_group, n_groups, X, group_off, max_rows_per_group, out, ld_out, err,
-                    stream=None):
+                    X_lo=None, out_lo=None, stream=None):
     """One tcgen05 GEMM launch (see include/dg_debug.h)."""
-    _check(lib.dg_debug_gemm_bf16(epi, _ptr(W), a_rows_per_group, n_groups, _ptr(X), X.shape[0], X.shape[1],
-                                  _ptr(group_off), max_rows_per_group, _ptr(out), ld_out, _ptr(err), _stream(stream)))
+    _check(lib.dg_debug_gemm_bf16(epi, _ptr(W), a_rows_per_group, n_groups, _ptr(X), _ptr(X_lo), X.shape[0],
+                                  X.shape[1], _ptr(group_off), max_rows_per_group, _ptr(out), _ptr(out_lo), ld_out,
+                                  _ptr(err), _stream(stream)))
 
 
-def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, stream=None):
+def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out_lo=None, stream=None):
     """One attention launch (see include/dg_debug.h): q [nq][n_q][128], k [nkv][cap][128], vt [nkv][128][cap]."""
     nq, n_q, _ = q.shape
     nkv, cap, _ = k.shape
     _check(lib.dg_debug_attention_bf16(_ptr(q), _ptr(k), _ptr(vt), cap, n_q, pos0, n_keys, 1 if causal else 0, nq,
-                                       nkv, _ptr(out), ws.ptr, ws.nbytes, _stream(stream)))
+                                       nkv, _ptr(out), _ptr(out_lo), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def debug_bounded_wait(ws, timeout_ms, stream=None):
+    """Launch the bounded-wait self-test kernel (see include/dg_debug.h)."""
+    ptr = ws.ptr if isinstance(ws, Workspace) else ctypes.c_void_p(ws.data_ptr())
+    _check(lib.dg_debug_bounded_wait(ptr, timeout_ms, _stream(stream)))

@@ -67,23 +67,34 @@ void dg_profile_reset(void);
 const char* dg_kernel_name(int32_t kind);
 
 /* One launch of the tcgen05 GEMM alone (bf16):
- *   out[r][f] (op)= sum_k W[g * a_rows_per_group + f][k] * X[r][k]
+ *   out[r][f] (op)= sum_k W[g * a_rows_per_group + f][k] * (X[r][k] + X_lo[r][k])
  * for rows r of group g = [group_off[g], group_off[g+1]) (group_off: device int32
- * [n_groups + 1], or NULL for one group of x_rows rows).  epi 0: store fp32 out,
- * 1: add into fp32 out, 2: packed gate/up rows -> bf16 silu(gate) * up with
- * a_rows_per_group / 2 output columns.  W [n_groups * a_rows_per_group][K], X [x_rows][K]
- * bf16; K % 64 == 0, a_rows_per_group % 128 == 0.  d_err: device int32 error word. */
+ * [n_groups + 1], or NULL for one group of x_rows rows; X_lo NULL: X alone).  epi 0:
+ * store fp32 out, 1: add into fp32 out, 2: packed gate/up rows -> silu(gate) * up with
+ * a_rows_per_group / 2 output columns, written as bf16 hi (out) and lo (out_lo, or
+ * NULL).  W [n_groups * a_rows_per_group][K], X [x_rows][K] bf16; K % 64 == 0,
+ * a_rows_per_group % 128 == 0.  d_err: device int32 error word. */
 dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups, const void* X,
-                             int32_t x_rows, int32_t K, const int32_t* group_off, int32_t max_rows_per_group,
-                             void* out, int32_t ld_out, int32_t* d_err, dg_stream stream);
+                             const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off,
+                             int32_t max_rows_per_group, void* out, void* out_lo, int32_t ld_out, int32_t* d_err,
+                             dg_stream stream);
 
 /* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
  * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
- * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128].  d_ws: a workspace sized by
- * dg_workspace_bytes for a config with these heads and >= n_q tokens. */
+ * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128] (hi part); out_lo (nullable)
+ * receives the lo part, out + out_lo = the fp32 attention output to ~16 bits.  d_ws: a
+ * workspace sized by dg_workspace_bytes for a config with these heads, hidden 128 and
+ * >= n_q tokens. */
 dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q, int32_t pos0,
-                                  int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv, void* out, void* d_ws,
-                                  size_t ws_bytes, dg_stream stream);
+                                  int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv, void* out, void* out_lo,
+                                  void* d_ws, size_t ws_bytes, dg_stream stream);
+
+/* Failure-detection self-test: launches one kernel whose thread waits, with the
+ * library's bounded wait, on an mbarrier that nothing completes.  After timeout_ms
+ * the wait gives up, records a timeout code in the workspace error word and the
+ * kernel returns normally (no trap, the context stays usable); dg_device_status then
+ * returns DG_ERR_TIMEOUT.  timeout_ms in [1, 10000]. */
+dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream);
 
 /* Kernels launched by the library since it was loaded (all kinds, profiling or not). */
 int64_t dg_launch_count(void);

@@ -31,12 +31,16 @@ Readings where the pages are silent (each one listed in the design notes):
   takes its argmax (ties to the lowest id), then the n lowest-confidence
   positions (ties to the lower position) get a fresh random token.
 
-Precision model.  The fp32 model computes everything in float64 here.  For bf16
-models the CUDA path stores some activations in bf16; where a later integer
-decision (routing, argmax, re-noise set) depends on them, both sides must take
-it at the same precision, so `Precision('bf16')` rounds (round-to-nearest-even)
-at exactly those storage points: the normed GEMM inputs, post-RoPE q/k and v,
-the attention output, and the SwiGLU output.  Everything else stays float64.
+Precision model.  The pages fix no precision beyond bf16 weights, so the oracle
+follows the kernel's storage precision, because later integer decisions (routing,
+argmax, re-noise set) depend on it and both sides must take them at the same
+precision.  The fp32 model computes everything in float64 here.  A bf16 model
+stores its weights, its KV cache and the attention query operand in bf16 and hands
+every other activation to its GEMMs at fp32 precision (the CUDA path carries it as
+two bf16 terms, ~16 significant bits, which this float64 reference treats as
+exact); the input of the vocabulary projection is a single bf16 term.  So
+`Precision('bf16')` rounds (round-to-nearest-even) exactly at post-RoPE q/k, v,
+and the final normed hidden state.  Everything else stays float64.
 """
 from __future__ import annotations
 
@@ -64,8 +68,8 @@ class Precision:
         assert dtype in ("bf16", "f32")
         self.dtype = dtype
 
-    def act(self, x: np.ndarray) -> np.ndarray:
-        """An activation stored in the model's activation dtype."""
+    def store(self, x: np.ndarray) -> np.ndarray:
+        """A value stored in the model's storage dtype (KV cache, query operand, vocabulary input)."""
         return round_bf16(x) if self.dtype == "bf16" else x
 
 
@@ -191,20 +195,20 @@ def _qkv(model, l: int, x: np.ndarray, positions: np.ndarray, prec: Precision):
     cfg = model.cfg
     nq, nkv, d = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
     L = model.layers[l]
-    xn = prec.act(rms_norm(x, cfg["rms_eps"]))
+    xn = rms_norm(x, cfg["rms_eps"])
     T = x.shape[0]
     q = (xn @ widen(L["w_q"]).T).reshape(T, nq, d).transpose(1, 0, 2)
     k = (xn @ widen(L["w_k"]).T).reshape(T, nkv, d).transpose(1, 0, 2)
     v = (xn @ widen(L["w_v"]).T).reshape(T, nkv, d).transpose(1, 0, 2)
-    q = prec.act(rope(q, positions, cfg["rope_theta"]))
-    k = prec.act(rope(k, positions, cfg["rope_theta"]))
-    v = prec.act(v)
+    q = prec.store(rope(q, positions, cfg["rope_theta"]))
+    k = prec.store(rope(k, positions, cfg["rope_theta"]))
+    v = prec.store(v)
     return q, k, v
 
 
 def _attn_out(model, l: int, o: np.ndarray, prec: Precision) -> np.ndarray:
     T = o.shape[1]
-    o = prec.act(o.transpose(1, 0, 2).reshape(T, -1))
+    o = o.transpose(1, 0, 2).reshape(T, -1)
     return o @ widen(model.layers[l]["w_o"]).T
 
 
@@ -222,7 +226,7 @@ def moe(model, l: int, x: np.ndarray, prec: Precision, tap: dict | None = None) 
     logits = xn @ widen(L["w_router"]).T
     idx, w, margin = router_topk(logits, k)
     counts, offsets, perm, inv, union = expert_permutation(idx, E)
-    xs = prec.act(xn)
+    xs = xn
     T, H = x.shape
     ys = np.zeros((T * k, H))
     for e in range(E):
@@ -232,7 +236,7 @@ def moe(model, l: int, x: np.ndarray, prec: Precision, tap: dict | None = None) 
         xe = xs[rows // k]
         g = xe @ widen(L["w_gate"][e]).T
         u = xe @ widen(L["w_up"][e]).T
-        h = prec.act(silu(g) * u)
+        h = silu(g) * u
         ys[offsets[e]:offsets[e + 1]] = h @ widen(L["w_down"][e]).T
     out = np.zeros((T, H))
     for j in range(k):
@@ -255,7 +259,7 @@ def vocab_logits(model, x: np.ndarray, prec: Precision, rows=None, chunk: int = 
     parallel, so every row gets a full distribution over the vocabulary.
     """
     cfg = model.cfg
-    xn = prec.act(rms_norm(x, cfg["rms_eps"]))
+    xn = prec.store(rms_norm(x, cfg["rms_eps"]))
     if rows is not None:
         xn = xn[np.asarray(rows)]
     V = cfg["vocab"]
@@ -315,7 +319,7 @@ def denoise_pass(model, cache: Cache, canvas: np.ndarray, prec: Precision, logit
         kk = np.concatenate([cache.k[l], k], axis=1)
         vv = np.concatenate([cache.v[l], v], axis=1)
         o = attention(q, kk, vv, mask)
-        tap["attn_o"] = prec.act(o.transpose(1, 0, 2).reshape(C, -1))
+        tap["attn_o"] = o.transpose(1, 0, 2).reshape(C, -1)
         x = x + _attn_out(model, l, o, prec)
         tap["x_attn"] = x.copy()
         x = x + moe(model, l, x, prec, tap)

@@ -92,12 +92,11 @@ def test_prefill_append_matches_oracle(dg):
             near_tie |= {P0 + int(i) for i in np.nonzero(t["router_margin"] < PL.ROUTE_MARGIN)[0]}
     dg.device_status(ws)
     assert st.cache.len == 227 == st.ocache.len
-    keep = [p for p in range(227) if p not in near_tie]
     for l in range(cfg["n_layers"]):
         k, v = st.cache.logical(l)
-        ok, ov = st.ocache.k[l], st.ocache.v[l]
-        assert PL.rel_err(k[:, keep].reshape(-1, 128), ok[:, keep].reshape(-1, 128)) < 2e-2, l
-        assert PL.rel_err(v[:, keep].reshape(-1, 128), ov[:, keep].reshape(-1, 128)) < 2e-2, l
+        for name, g, o in (("K", k, st.ocache.k[l]), ("V", v, st.ocache.v[l])):
+            ok, frac, dmax = PL.kv_close(g, o, near_tie)
+            assert ok, f"layer {l} {name}: {frac:.2%} of elements differ, max {dmax:.3e}"
 
 
 def test_mask_worked_example_on_gpu(dg):
@@ -118,7 +117,10 @@ def test_mask_worked_example_on_gpu(dg):
 
 
 def test_chained_canvases_small(dg):
-    """prompt prefill -> (S denoising steps with re-noising -> append) x 2, step by step."""
+    """prompt prefill -> (S denoising steps with re-noising -> append) x 2, step by step.
+
+    Positions whose tokens came out different (only allowed where the oracle's margin
+    exempts them) stay exempt in later steps and canvases of the comparison."""
     cfg = dict(SMALL_BF16, n_layers=2)
     C, S, n_can = 64, 3, 2
     st = PL.Setup(cfg, 0, capacity=512, with_prefix=False)
@@ -126,32 +128,31 @@ def test_chained_canvases_small(dg):
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 96, cfg["vocab"])
     dg.prefill_append(st.model, st.cache, torch.from_numpy(prompt).cuda(), ws)
     oc = O.prefill_append(st.host, st.ocache, prompt, st.prec)
-    tainted = set()
     for c in range(n_can):
         cur_g = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])
         cur_o = cur_g.copy()
+        tainted = set()
         for s in range(S):
             n = O.renoise_count(C, S, s, 0.5, 0.0)
-            taps, logits, nxt_g, conf = _gpu_pass(dg, st, cur_g, n, step=s, taps=False)
-            logits_o, _ = O.denoise_pass(st.host, oc, cur_o, st.prec)
+            taps, logits, nxt_g, conf = _gpu_pass(dg, st, cur_g, n, step=s)
+            logits_o, taps_o = O.denoise_pass(st.host, oc, cur_o, st.prec)
             upd = O.canvas_update(logits_o, n, synth.SEED_RENOISE, s)
-            assert PL.rel_err(logits, logits_o, tainted) < 2e-2
-            for i in range(C):
-                if i in tainted or nxt_g[i] == upd["canvas"][i]:
-                    continue
-                ok = upd["cut_margin"][i] < PL.CUT_MARGIN or (i not in set(upd["renoised"].tolist())
-                                                             and upd["top_margin"][i] <= PL.TOKEN_MARGIN)
-                assert ok, f"canvas {c} step {s} position {i}: {nxt_g[i]} vs {upd['canvas'][i]}"
-                tainted.add(i)
+            exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, exempt=tainted)
+            PL.compare_update(nxt_g, conf, upd, exempt, n)
+            tainted = exempt | {i for i in range(C) if nxt_g[i] != upd["canvas"][i]}
             cur_g, cur_o = nxt_g, upd["canvas"]
+        print(f"canvas {c}: positions exempt at the end {sorted(tainted)}")
+        if tainted:
+            return   # the two runs now append different canvases; the rest is not comparable
         dg.prefill_append(st.model, st.cache, torch.from_numpy(cur_g.astype(np.int32)).cuda(), ws)
         oc = O.prefill_append(st.host, oc, cur_o, st.prec)
-        print(f"canvas {c}: tainted {sorted(tainted)}")
     dg.device_status(ws)
     assert st.cache.len == oc.len == 96 + n_can * C
     for l in range(cfg["n_layers"]):
-        k, _ = st.cache.logical(l, upto=96)
-        assert PL.rel_err(k.reshape(-1, 128), oc.k[l][:, :96].reshape(-1, 128)) < 2e-2
+        k, v = st.cache.logical(l)
+        for name, g, o in (("K", k, oc.k[l]), ("V", v, oc.v[l])):
+            ok, frac, dmax = PL.kv_close(g, o)
+            assert ok, f"layer {l} {name}: {frac:.2%} of elements differ, max {dmax:.3e}"
 
 
 def test_generate_canvas_equals_step_loop(dg):
