@@ -49,11 +49,17 @@ __global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, const T* _
   }
   const T* e = embed + (size_t)tok * H;
   float* xr = x + (size_t)t * H;
+  constexpr int VE = 16 / sizeof(T);  // elements per 16-byte vector
   float ss = 0.0f;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    const float v = to_f32(e[h]);
-    xr[h] = v;
-    ss += v * v;
+  for (int v = threadIdx.x; v < H / VE; v += blockDim.x) {
+    const uint4 raw = reinterpret_cast<const uint4*>(e)[v];
+    const T* el = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+    for (int j = 0; j < VE; ++j) {
+      const float f = to_f32(el[j]);
+      xr[v * VE + j] = f;
+      ss += f * f;
+    }
   }
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / (float)H + eps);
@@ -89,10 +95,16 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, 
   }
   const int W = (nq + 2 * nkv) * d;
   float* row = cs + d;  // qkv row = sum of the split-K partials, in a fixed order
-  for (int i = threadIdx.x; i < W; i += blockDim.x) {
-    float v = 0.0f;
-    for (int s = 0; s < n_parts; ++s) v += qkv[s * part_stride + (size_t)t * W + i];
-    row[i] = v;
+  for (int i = threadIdx.x; i < W / 4; i += blockDim.x) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_parts; ++s) {
+      const float4 a = reinterpret_cast<const float4*>(qkv + s * part_stride + (size_t)t * W)[i];
+      v.x += a.x;
+      v.y += a.y;
+      v.z += a.z;
+      v.w += a.w;
+    }
+    reinterpret_cast<float4*>(row)[i] = v;
   }
   __syncthreads();
   // q and k heads: pairs (i, i + d/2)
@@ -259,10 +271,12 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
 // Per token: x += sum of the output-projection partials (fixed order); xn = x / rms(x)
 // in fp32; router logits l[e] = xn . w_router[e] (fp32); the k largest (ties to the
 // lower expert id) and their softmax weights.  xn is also stored (hi/lo) as the expert
-// input.  CTA = RTF_TOK tokens, 256 threads; warp w handles experts w, w + 8, ...
+// input.  CTA = RTF_TOK tokens, RTF_THREADS threads; each warp takes two experts at a
+// time and keeps eight float4 loads of router weights in flight.
 constexpr int RTF_TOK = 4;
+constexpr int RTF_THREADS = 512;
 template <typename T>
-__global__ void __launch_bounds__(256) router_fused_kernel(
+__global__ void __launch_bounds__(RTF_THREADS) router_fused_kernel(
     float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
     const float* __restrict__ wr, int n, int H, int E, int k, float eps, float* __restrict__ logits_out,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, T* __restrict__ xn, T* __restrict__ xn_lo) {
@@ -271,16 +285,29 @@ __global__ void __launch_bounds__(256) router_fused_kernel(
   float* lg = sm + RTF_TOK * H;
   __shared__ float inv_s[RTF_TOK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = RTF_THREADS / 32;
   const int t0 = blockIdx.x * RTF_TOK;
   const int nt = min(RTF_TOK, n - t0);
-  // residual add of the partials
-  for (int i = threadIdx.x; i < nt * H; i += blockDim.x) {
-    const int a = i / H, h = i % H;
-    const size_t o = (size_t)(t0 + a) * H + h;
-    float v = x[o];
-    for (int s = 0; s < n_parts; ++s) v += parts[s * part_stride + o];
-    x[o] = v;
-    xs[a * H + h] = v;
+  const int H4 = H / 4;
+  // residual add of the partials (float4, all loads of an element issued together)
+  {
+    float4* x4 = reinterpret_cast<float4*>(x + (size_t)t0 * H);
+    const float4* p4 = reinterpret_cast<const float4*>(parts + (size_t)t0 * H);
+    const size_t ps4 = part_stride / 4;
+    float4* xs4 = reinterpret_cast<float4*>(xs);
+#pragma unroll 2
+    for (int i = threadIdx.x; i < nt * H4; i += RTF_THREADS) {
+      float4 v = x4[i];
+      for (int s = 0; s < n_parts; ++s) {
+        const float4 a = p4[s * ps4 + i];
+        v.x += a.x;
+        v.y += a.y;
+        v.z += a.z;
+        v.w += a.w;
+      }
+      x4[i] = v;
+      xs4[i] = v;
+    }
   }
   __syncthreads();
   if (warp < RTF_TOK) {
@@ -291,34 +318,53 @@ __global__ void __launch_bounds__(256) router_fused_kernel(
     if (lane == 0) inv_s[warp] = 1.0f / sqrtf(ss / (float)H + eps);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < nt * H; i += blockDim.x) {
-    const int a = i / H;
-    const float v = xs[i] * inv_s[a];
+  for (int i = threadIdx.x; i < nt * H; i += RTF_THREADS) {
+    const float v = xs[i] * inv_s[i / H];
     xs[i] = v;
     store_act(xn, xn_lo, (size_t)t0 * H + i, v);
   }
   __syncthreads();
-  // logits: one expert row per warp iteration, float4 over H, all tokens of the CTA at once
-  for (int e = warp; e < E; e += 8) {
-    const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)e * H);
-    float acc[RTF_TOK] = {};
-    for (int i = lane; i < H / 4; i += 32) {
-      const float4 w = w4[i];
+  const float4* xs4 = reinterpret_cast<const float4*>(xs);
+  for (int e0 = 2 * warp; e0 < E; e0 += 2 * NW) {
+    const int e1 = min(e0 + 1, E - 1);
+    const float4* w0 = reinterpret_cast<const float4*>(wr + (size_t)e0 * H);
+    const float4* w1 = reinterpret_cast<const float4*>(wr + (size_t)e1 * H);
+    float a0[RTF_TOK] = {}, a1[RTF_TOK] = {};
+    for (int i0 = lane; i0 < H4; i0 += 32 * 4) {
+      float4 u0[4], u1[4];
 #pragma unroll
-      for (int a = 0; a < RTF_TOK; ++a) {
-        const float4 v = reinterpret_cast<const float4*>(xs + a * H)[i];
-        acc[a] = fmaf(w.x, v.x, fmaf(w.y, v.y, fmaf(w.z, v.z, fmaf(w.w, v.w, acc[a]))));
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 32 * u;
+        const bool in = i < H4;
+        u0[u] = in ? w0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        u1[u] = in ? w1[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < H4) {
+#pragma unroll
+          for (int a = 0; a < RTF_TOK; ++a) {
+            const float4 v = xs4[a * H4 + i];
+            a0[a] = fmaf(u0[u].x, v.x, fmaf(u0[u].y, v.y, fmaf(u0[u].z, v.z, fmaf(u0[u].w, v.w, a0[a]))));
+            a1[a] = fmaf(u1[u].x, v.x, fmaf(u1[u].y, v.y, fmaf(u1[u].z, v.z, fmaf(u1[u].w, v.w, a1[a]))));
+          }
+        }
       }
     }
 #pragma unroll
     for (int a = 0; a < RTF_TOK; ++a) {
-      const float r = warp_sum(acc[a]);
-      if (lane == 0) lg[a * E + e] = r;
+      const float r0 = warp_sum(a0[a]);
+      const float r1 = warp_sum(a1[a]);
+      if (lane == 0) {
+        lg[a * E + e0] = r0;
+        if (e0 + 1 < E) lg[a * E + e0 + 1] = r1;
+      }
     }
   }
   __syncthreads();
   if (logits_out)
-    for (int i = threadIdx.x; i < nt * E; i += blockDim.x) logits_out[(size_t)t0 * E + i] = lg[i];
+    for (int i = threadIdx.x; i < nt * E; i += RTF_THREADS) logits_out[(size_t)t0 * E + i] = lg[i];
   // top-k: warp a < nt selects for token a
   if (warp < nt) {
     const float* l = lg + warp * E;
@@ -368,9 +414,8 @@ cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_
   const size_t smem = (size_t)RTF_TOK * (H + E) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  router_fused_kernel<T><<<(n + RTF_TOK - 1) / RTF_TOK, 256, smem, st>>>(x, parts, n_parts, part_stride, w_router, n,
-                                                                          H, E, k, eps, logits, topk_idx, topk_w, xn,
-                                                                          xn_lo);
+  router_fused_kernel<T><<<(n + RTF_TOK - 1) / RTF_TOK, RTF_THREADS, smem, st>>>(
+      x, parts, n_parts, part_stride, w_router, n, H, E, k, eps, logits, topk_idx, topk_w, xn, xn_lo);
   return cudaGetLastError();
 }
 
@@ -598,18 +643,28 @@ __global__ void update_partial_kernel(const float* __restrict__ logits, int V, i
   const float* lg = logits + (size_t)row * V;
   float m = -INFINITY, s = 0.0f;
   int a = 0x7fffffff;
-  for (int i = lo + threadIdx.x * 4; i < hi; i += blockDim.x * 4) {
-    const float4 v4 = *reinterpret_cast<const float4*>(lg + i);
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+  const int stride = blockDim.x * 4;
+  for (int i0 = lo + threadIdx.x * 4; i0 < hi; i0 += 4 * stride) {
+    float4 v4[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float x = v[u];
-      if (x > m) {
-        s = s * __expf(m - x) + 1.0f;
-        m = x;
-        a = i + u;
-      } else {
-        s += __expf(x - m);
+      const int i = i0 + u * stride;
+      v4[u] = (i < hi) ? *reinterpret_cast<const float4*>(lg + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * stride;
+      const float v[4] = {v4[u].x, v4[u].y, v4[u].z, v4[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float xv = v[q];
+        if (xv > m) {
+          s = s * __expf(m - xv) + 1.0f;
+          m = xv;
+          a = i + q;
+        } else if (xv != -INFINITY) {
+          s += __expf(xv - m);
+        }
       }
     }
   }

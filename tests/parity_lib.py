@@ -131,18 +131,31 @@ def compare_pass(cfg, taps_gpu, logits_gpu, taps_o, logits_o, report=None, exemp
     return exempt
 
 
+def bf16_spacing(x):
+    """Distance between consecutive bf16 values around |x| (8 significant bits)."""
+    _, e = np.frexp(np.abs(np.asarray(x, np.float64)))
+    return np.ldexp(1.0, e - 8)
+
+
 def kv_close(gpu, ref, skip_positions=()):
     """bf16-stored K/V against the oracle's rounded values: every element equal or one
     rounding step apart (the two sides round values that differ in the last fp32 bits),
-    and only a small fraction of elements apart at all.  Arrays [nkv][len][d]."""
+    and only a small fraction of elements apart at all.  Arrays [nkv][len][d].
+    Returns (ok, fraction differing, description of the worst element)."""
     g = np.asarray(gpu, np.float64)
     r = np.asarray(ref, np.float64)
-    keep = [p for p in range(r.shape[1]) if p not in set(skip_positions)]
+    skip = set(skip_positions)
+    keep = [p for p in range(r.shape[1]) if p not in skip]
     g, r = g[:, keep], r[:, keep]
     d = np.abs(g - r)
-    ok = d <= 2.0 ** -7 * np.abs(r) + 1e-30
+    step = bf16_spacing(np.maximum(np.abs(g), np.abs(r)))
+    bad = d > step * 1.0001
     frac = float((d > 0).mean())
-    return bool(ok.all()) and frac < 0.01, frac, float(d.max())
+    worst = ""
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(bad, d / step, 0)), d.shape)
+        worst = f"gpu {g[i]!r} oracle {r[i]!r} at {i}"
+    return (not bad.any()) and frac < 0.01, frac, worst
 
 
 def compare_update(canvas_gpu, conf_gpu, upd_o, exempt, n):
