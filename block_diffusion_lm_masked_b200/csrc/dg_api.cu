@@ -130,10 +130,18 @@ static dg_status map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint6
   const uint32_t box[2] = {64, box_rows};
   return encode_bf16(m, base, 2, dims, strides, box);
 }
+// weights [groups][rows][cols] bf16 as a 3-D map with box (64 cols, 128 rows, 1 group);
+// rows past the end of a group read as zeros instead of the next group's rows
+static dg_status map_weights(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const uint64_t dims[3] = {cols, rows, groups};
+  const uint64_t strides[2] = {cols * 2, rows * cols * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_bf16(m, base, 3, dims, strides, box);
+}
 
 // ---------------------------------------------------------------- model
 struct LayerMaps {
-  CUtensorMap qkv, o, gate_up, down;
+  CUtensorMap qkv, o, gate, up, down;
 };
 struct dg_model {
   dg_config cfg;
@@ -179,7 +187,7 @@ extern "C" dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, 
   DG_CHECK_ARG(w && out && w->embed && w->w_out && w->layers, "weights / out pointer is NULL");
   for (int l = 0; l < cfg->n_layers; ++l) {
     const dg_layer_weights& L = w->layers[l];
-    DG_CHECK_ARG(L.w_qkv && L.w_o && L.w_router && L.w_gate_up && L.w_down, "layer %d has a NULL weight", l);
+    DG_CHECK_ARG(L.w_qkv && L.w_o && L.w_router && L.w_gate && L.w_up && L.w_down, "layer %d has a NULL weight", l);
   }
   dg_model* m = new dg_model();
   m->cfg = *cfg;
@@ -192,15 +200,17 @@ extern "C" dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, 
     for (int l = 0; l < c.n_layers; ++l) {
       const dg_layer_weights& L = m->layers[l];
       LayerMaps& M = m->maps[l];
-      if ((s = map_rows(&M.qkv, L.w_qkv, qkv_rows(c), c.hidden, 128)) != DG_OK ||
-          (s = map_rows(&M.o, L.w_o, c.hidden, (uint64_t)c.n_q_heads * c.head_dim, 128)) != DG_OK ||
-          (s = map_rows(&M.gate_up, L.w_gate_up, (uint64_t)c.n_experts * 2 * c.expert_ffn, c.hidden, 128)) != DG_OK ||
-          (s = map_rows(&M.down, L.w_down, (uint64_t)c.n_experts * c.hidden, c.expert_ffn, 128)) != DG_OK) {
+      const uint64_t E = c.n_experts, F = c.expert_ffn, H = c.hidden;
+      if ((s = map_weights(&M.qkv, L.w_qkv, 1, qkv_rows(c), H)) != DG_OK ||
+          (s = map_weights(&M.o, L.w_o, 1, H, (uint64_t)c.n_q_heads * c.head_dim)) != DG_OK ||
+          (s = map_weights(&M.gate, L.w_gate, E, F, H)) != DG_OK ||
+          (s = map_weights(&M.up, L.w_up, E, F, H)) != DG_OK ||
+          (s = map_weights(&M.down, L.w_down, E, H, F)) != DG_OK) {
         delete m;
         return s;
       }
     }
-    if ((s = map_rows(&m->out_map, m->w_out, c.vocab, c.hidden, 128)) != DG_OK) {
+    if ((s = map_weights(&m->out_map, m->w_out, 1, c.vocab, c.hidden)) != DG_OK) {
       delete m;
       return s;
     }
@@ -216,13 +226,14 @@ namespace {
 constexpr int kMaxAttnSplits = 16;
 constexpr int kMaxKsQkv = 4;   // split-K of the QKV projection
 constexpr int kMaxKsO = 8;     // split-K of the output projection
-constexpr int kSmemShared = 100 * 1024;  // GEMM stage budget when two CTAs share an SM
-constexpr int kSmemSolo = 200 * 1024;    // ... when one CTA owns the SM
+constexpr int kSmemGemm = 200 * 1024;    // stage budget of the persistent GEMM (one CTA per SM)
 inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+
+constexpr int kItemRows = 64;            // rows per work item of the grouped expert GEMMs
 
 struct WsLayout {
   size_t err, upd, x, xn, xn_lo, qkv, q, o, o_lo, part_o, part_lse, opart, topk_idx, topk_w, counts, offsets, perm,
-      inv, uni, xs, xs_lo, h, h_lo, gu, ys, total;
+      inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, total;
 };
 
 size_t upd_bytes(int C, int V) { return al((size_t)C * dg::update_splits(C, V) * sizeof(dg::UpdPart)); }
@@ -259,6 +270,8 @@ WsLayout layout(const dg_config& c, int T) {
   L.perm = take((size_t)T * k * 4);
   L.inv = take((size_t)T * k * 4);
   L.uni = take(4);
+  L.items = take(((size_t)T * k / kItemRows + E + 1) * sizeof(dg::TcWorkItem));
+  L.n_items = take(4);
   L.xs = take((size_t)T * k * H * ab);
   L.xs_lo = take(bf ? (size_t)T * k * H * 2 : 0);
   L.h = take((size_t)T * k * F * ab);
@@ -282,11 +295,11 @@ struct Ws {
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // split-K factor: a divisor of the k-block count, at most max_ks, keeping >= 2 k-blocks
-// per CTA and about two CTAs per SM at most
+// per tile and the tile count within one wave of the persistent GEMM
 int pick_ksplit(int m_tiles, int token_chunks, int nkb, int max_ks) {
   int best = 1;
   for (int ks = 1; ks <= max_ks; ++ks)
-    if (nkb % ks == 0 && nkb / ks >= 2 && m_tiles * token_chunks * ks <= 2 * 148) best = ks;
+    if (nkb % ks == 0 && nkb / ks >= 2 && m_tiles * token_chunks * ks <= dg::num_sms()) best = ks;
   return best;
 }
 }  // namespace
@@ -306,11 +319,15 @@ namespace {
 struct GemmCall {
   int kind, epi;
   const CUtensorMap* A;
+  const CUtensorMap* A2;  // dual_a (gate / up) or null
   const void* X;
-  const void* X_lo;  // null: single term
-  int x_rows, K, a_rows_per_group, n_groups;
-  const int* group_off;
-  int max_rows_per_group;
+  const void* X_lo;       // null: single term
+  int x_rows, K;
+  int a_rows_per_group;   // output features per group
+  const dg::TcWorkItem* items;  // grouped work list or null (dense)
+  const int* n_items;
+  int max_items;          // upper bound of the work-item count (sizes the grid)
+  int n_max;              // token rows per tile
   void* out;
   void* out_lo;
   int ld_out;
@@ -328,21 +345,26 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   } else {
     B2 = B;
   }
-  dg::TcGemmParams p;
+  dg::TcGemmParams p{};
   p.K = g.K;
   p.a_rows_per_group = g.a_rows_per_group;
-  p.group_off = g.group_off;
+  p.m_tiles = ceil_div(g.a_rows_per_group, 128);
+  p.n_max = g.n_max;
   p.n_tokens = g.x_rows;
+  p.k_splits = g.k_splits;
+  p.split_stride = g.split_stride;
+  p.items = g.items;
+  p.n_items = g.n_items;
+  p.dual_a = g.A2 != nullptr;
+  p.two_terms = g.X_lo != nullptr;
   p.out = g.out;
   p.out_lo = g.out_lo;
   p.ld_out = g.ld_out;
-  p.two_terms = g.X_lo != nullptr;
-  p.k_splits = g.k_splits;
-  p.split_stride = g.split_stride;
   p.smem_budget = g.smem_budget;
   p.err = err;
+  const int items = g.items ? g.max_items : ceil_div(g.x_rows, g.n_max) * g.k_splits;
   LAUNCH(g.kind, st,
-         dg::launch_tc_gemm(g.epi, *g.A, B, B2, p, g.a_rows_per_group / 128, g.n_groups, g.max_rows_per_group, st));
+         dg::launch_tc_gemm(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, B, B2, p, items * p.m_tiles, st));
   return DG_OK;
 }
 
@@ -425,13 +447,12 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   int* err = ws.err();
   T* xn_lo = bf ? ws.at<T>(ws.L.xn_lo) : nullptr;
   dg_status s;
-  const int chunks = ceil_div(n, 256);
   // ---- attention block: QKV (split-K partials) -> RoPE + K/V into the cache -> attention -> output projection
   int ks_qkv = 1, ks_o = 1;
   if (bf) {
-    ks_qkv = pick_ksplit(QR / 128, chunks, H / 64, kMaxKsQkv);
-    GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, ws.at<void>(ws.L.xn), xn_lo, n, H, QR, 1,
-               nullptr, n, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemSolo};
+    ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
+    GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
+               nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_QKV, st,
@@ -444,9 +465,10 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
-    ks_o = pick_ksplit(H / 128, chunks, nq * d / 64, kMaxKsO);
-    GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo), n,
-               nq * d, H, 1, nullptr, n, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H, kSmemSolo};
+    ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
+    GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
+               n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
+               kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_O, st,
@@ -465,24 +487,35 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   LAUNCH(DG_K_PERMUTE, st,
          dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
                             ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
-                            ws.at<int32_t>(ws.L.uni), st));
+                            ws.at<int32_t>(ws.L.uni), kItemRows, ws.at<dg::TcWorkItem>(ws.L.items),
+                            ws.at<int>(ws.L.n_items), st));
   T* xs_lo = bf ? ws.at<T>(ws.L.xs_lo) : nullptr;
   LAUNCH(DG_K_GATHER, st,
          dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), xn_lo, ws.at<int32_t>(ws.L.perm), n * k, k, H,
                                    ws.at<T>(ws.L.xs), xs_lo, st));
   const int* off = ws.at<int>(ws.L.offsets);
   if (bf) {
-    GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate_up, ws.at<void>(ws.L.xs), xs_lo, n * k, H,
-                2 * F, E, off, n, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0, kSmemShared};
+    const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
+    const int* n_items = ws.at<int>(ws.L.n_items);
+    const int max_items = n * k / kItemRows + E;
+    GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate, &m->maps[l].up, ws.at<void>(ws.L.xs), xs_lo,
+                n * k, H, F, items, n_items, max_items, kItemRows, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
+                kSmemGemm};
     if ((s = gemm_bf16(gu, err, st)) != DG_OK) return s;
-    GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo),
-                n * k, F, H, E, off, n, ws.at<float>(ws.L.ys), nullptr, H, 1, 0, kSmemShared};
+    GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, nullptr, ws.at<void>(ws.L.h),
+                ws.at<void>(ws.L.h_lo), n * k, F, H, items, n_items, max_items, kItemRows, ws.at<float>(ws.L.ys),
+                nullptr, H, 1, 0, kSmemGemm};
     if ((s = gemm_bf16(dn, err, st)) != DG_OK) return s;
   } else {
+    float* g = ws.at<float>(ws.L.gu);
+    float* u = g + (size_t)n * k * F;
     LAUNCH(DG_K_GEMM_GATE_UP, st,
-           dg::launch_simt_gemm_f32(0, (const float*)W.w_gate_up, ws.at<float>(ws.L.xs), off, E, n, n * k, 2 * F, H,
-                                    ws.at<float>(ws.L.gu), 2 * F, st));
-    LAUNCH(DG_K_SWIGLU, st, dg::launch_swiglu_packed_f32(ws.at<float>(ws.L.gu), n * k, F, ws.at<float>(ws.L.h), st));
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_gate, ws.at<float>(ws.L.xs), off, E, n, n * k, F, H, g, F,
+                                    st));
+    LAUNCH(DG_K_GEMM_GATE_UP, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_up, ws.at<float>(ws.L.xs), off, E, n, n * k, F, H, u, F,
+                                    st));
+    LAUNCH(DG_K_SWIGLU, st, dg::launch_swiglu_f32(g, u, n * k, F, ws.at<float>(ws.L.h), st));
     LAUNCH(DG_K_GEMM_DOWN, st,
            dg::launch_simt_gemm_f32(0, (const float*)W.w_down, ws.at<float>(ws.L.h), off, E, n, n * k, H, F,
                                     ws.at<float>(ws.L.ys), H, st));
@@ -594,8 +627,8 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
   if (s != DG_OK) return s;
   // vocabulary projection of the final RMSNorm (left in ws.xn by the last layer) to fp32 logits
   if (is_bf16(c)) {
-    GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, ws.at<void>(ws.L.xn), nullptr, C, c.hidden, c.vocab,
-               1, nullptr, C, d_logits, nullptr, c.vocab, 1, 0, kSmemShared};
+    GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, C, c.hidden,
+               c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm};
     if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_VOCAB, st,
@@ -655,22 +688,6 @@ extern "C" dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t
       return s;
   }
   if (append) return dg_prefill_append(m, cache, d_canvas, C, d_ws, ws_bytes, stream);
-  return DG_OK;
-}
-
-extern "C" dg_status dg_pack_gate_up(const void* d_gate, const void* d_up, void* d_out, int32_t E, int32_t F,
-                                     int32_t H, int32_t elem_bytes, dg_stream stream) {
-  DG_CHECK_ARG(d_gate && d_up && d_out, "NULL pointer");
-  DG_CHECK_ARG(E > 0 && F > 0 && H > 0 && F % 64 == 0, "E, F, H must be positive and F a multiple of 64");
-  DG_CHECK_ARG(elem_bytes == 2 || elem_bytes == 4, "elem_bytes must be 2 or 4");
-  DG_CHECK_ARG(((size_t)H * elem_bytes) % 16 == 0, "rows must be a multiple of 16 bytes");
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = dg::launch_pack_gate_up(d_gate, d_up, d_out, E, F, H, elem_bytes, st);
-  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "pack_gate_up: %s", cudaGetErrorString(e));
-  {
-    std::lock_guard<std::mutex> lk(g_prof_mu);
-    g_launches++;
-  }
   return DG_OK;
 }
 
@@ -745,22 +762,32 @@ extern "C" int64_t dg_launch_count(void) {
   return g_launches;
 }
 
-extern "C" dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups,
+extern "C" dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_t n_groups,
                                         const void* X, const void* X_lo, int32_t x_rows, int32_t K,
-                                        const int32_t* group_off, int32_t max_rows_per_group, void* out,
-                                        void* out_lo, int32_t ld_out, int32_t* d_err, dg_stream stream) {
-  DG_CHECK_ARG(W && X && out && d_err, "NULL pointer");
-  DG_CHECK_ARG(epi >= 0 && epi <= 2, "epi must be 0, 1 or 2");
-  DG_CHECK_ARG(K > 0 && K % 64 == 0 && a_rows_per_group > 0 && a_rows_per_group % 128 == 0 && n_groups > 0 &&
-                   x_rows > 0 && max_rows_per_group > 0,
-               "bad GEMM shape");
+                                        const int32_t* group_off, void* out, void* out_lo, int32_t ld_out,
+                                        void* d_scratch, int32_t* d_err, dg_stream stream) {
+  DG_CHECK_ARG(W && X && out && d_err && d_scratch, "NULL pointer");
+  DG_CHECK_ARG(K > 0 && K % 64 == 0 && rows > 0 && n_groups > 0 && x_rows > 0, "bad GEMM shape");
   DG_CHECK_ARG(group_off || n_groups == 1, "several groups need group_off");
-  CUtensorMap A;
-  dg_status s = map_rows(&A, W, (uint64_t)n_groups * a_rows_per_group, (uint64_t)K, 128);
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_scratch) & 15) == 0, "scratch must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap A, A2;
+  dg_status s = map_weights(&A, W, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K);
   if (s != DG_OK) return s;
-  GemmCall g{DG_K_GEMM_QKV, epi, &A, X, X_lo, x_rows, K, a_rows_per_group, n_groups, group_off, max_rows_per_group,
-             out, out_lo, ld_out, 1, 0, kSmemShared};
-  return gemm_bf16(g, d_err, reinterpret_cast<cudaStream_t>(stream));
+  if (W2 && (s = map_weights(&A2, W2, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  dg::TcWorkItem* items = nullptr;
+  int* n_items = nullptr;
+  int max_items = 0;
+  if (group_off) {
+    items = static_cast<dg::TcWorkItem*>(d_scratch);
+    n_items = reinterpret_cast<int*>(items + x_rows + n_groups);
+    max_items = x_rows / kItemRows + n_groups;
+    LAUNCH(DG_K_PERMUTE, st, dg::launch_build_items(group_off, n_groups, kItemRows, items, n_items, st));
+  }
+  GemmCall g{DG_K_GEMM_QKV, W2 ? dg::EPI_SWIGLU_BF16 : dg::EPI_STORE_F32, &A, W2 ? &A2 : nullptr, X, X_lo, x_rows,
+             K, rows, items, n_items, max_items, group_off ? kItemRows : (x_rows < 256 ? ((x_rows + 15) & ~15) : 256),
+             out, out_lo, ld_out, 1, 0, kSmemGemm};
+  return gemm_bf16(g, d_err, st);
 }
 
 extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,

@@ -8,32 +8,45 @@
 namespace dg {
 
 // ---------------------------------------------------------------- tcgen05 GEMM
-// out[token][feature] (op)= sum_k W[feature][k] * X[token][k]
-// W rows come from tensor map A (bf16, K-major, box 64 x 128), X rows from tensor map
-// B (bf16, K-major, box 64 x 16).  With two_terms, X = X_hi + X_lo is given as two
-// bf16 tensors (maps B and B2) and both products accumulate into the same fp32 tile.
-// Group g (an expert) owns token rows [group_off[g], group_off[g+1]) of X and W rows
-// [g * a_rows_per_group, ...).  With k_splits > 1 (one group only), split s reduces
-// K range [s K/k_splits, (s+1) K/k_splits) and stores to out + s * split_stride.
-enum TcEpilogue { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_SWIGLU_BF16 = 2 };
+// out[row][feature] (op)= sum_k W[g][feature][k] * X[row][k]
+// W comes from a 3-D tensor map (K, rows per group, groups), box 64 x 128 x 1; X from
+// a 2-D map (K, rows), box 64 x 16.  With two_terms, X = X_hi + X_lo (maps B and B2);
+// with dual_a, a second weight tensor (map A2, same shape) accumulates into a second
+// TMEM region and the epilogue writes silu(W x) * (W2 x) as bf16 hi (+ lo).
+// Work: dense -- rows [0, n_tokens) in chunks of n_max, times k_splits (split s reduces
+// K range [s K/k_splits, (s+1) K/k_splits) into out + s * split_stride); grouped -- the
+// device list items[0 .. *n_items).
+enum TcEpilogue { EPI_STORE_F32 = 0, EPI_SWIGLU_BF16 = 2 };
+
+struct TcWorkItem {
+  int group, row0, rows, pad;
+};
 
 struct TcGemmParams {
   int K;                 // reduction length, multiple of 64 * k_splits
-  int a_rows_per_group;  // W rows per group, multiple of 128
-  const int* group_off;  // device [n_groups + 1], or nullptr for one group of n_tokens rows
-  int n_tokens;
-  void* out;             // EPI_SWIGLU_BF16: bf16 h_hi; h_lo follows at out_lo
+  int a_rows_per_group;  // output features per group (rows of W[g])
+  int m_tiles;           // ceil(a_rows_per_group / 128)
+  int n_max;             // token rows per tile, multiple of 16, <= 256
+  int n_tokens;          // dense: token rows
+  int k_splits;          // dense only
+  size_t split_stride;   // elements between split outputs
+  const TcWorkItem* items;  // grouped: device work list (null: dense)
+  const int* n_items;       // grouped: device count
+  int dual_a;
+  int two_terms;
+  void* out;
   void* out_lo;
   int ld_out;            // elements per output row
-  int two_terms;         // X given as hi + lo
-  int k_splits;
-  size_t split_stride;   // elements between split outputs
   int smem_budget;       // bytes for pipeline stages
   int* err;              // device error word
 };
 
-cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
-                           const TcGemmParams& p, int m_tiles, int n_groups, int max_rows_per_group, cudaStream_t st);
+// grid = min(max_tiles, SMs); max_tiles bounds the tile count (exact for dense GEMMs)
+cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
+                           const CUtensorMap& B2, const TcGemmParams& p, int max_tiles, cudaStream_t st);
+cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
+                               cudaStream_t st);
+int num_sms();
 
 // ---------------------------------------------------------------- tcgen05 attention
 // Q [nq][n_q][128] bf16, K cache [nkv][cap][128] bf16, V^T cache [nkv][128][cap] bf16.
@@ -78,16 +91,15 @@ cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_
                                 int n, int H, int E, int k, float eps, float* logits, int32_t* topk_idx, float* topk_w,
                                 T* xn, T* xn_lo, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int n, int k, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* perm, int32_t* inv, int32_t* union_out, cudaStream_t st);
+                           int32_t* perm, int32_t* inv, int32_t* union_out, int item_rows, TcWorkItem* items,
+                           int* n_items, cudaStream_t st);
 template <typename T>
 cudaError_t launch_gather_rows(const T* xn, const T* xn_lo, const int32_t* perm, int rows, int k, int H, T* xs,
                                T* xs_lo, cudaStream_t st);
-cudaError_t launch_swiglu_packed_f32(const float* gu, int rows, int F, float* h, cudaStream_t st);
+cudaError_t launch_swiglu_f32(const float* g, const float* u, int rows, int F, float* h, cudaStream_t st);
 template <typename T>
 cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float* w, int n, int k, int H, float eps,
                                 float* x, T* xn, T* xn_lo, cudaStream_t st);
-cudaError_t launch_pack_gate_up(const void* gate, const void* up, void* out, int E, int F, int H, int elem_bytes,
-                                cudaStream_t st);
 
 // ---------------------------------------------------------------- canvas update
 struct UpdPart {

@@ -427,7 +427,8 @@ constexpr int PM_EMAX = 256;
 __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int total, int E,
                                                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                       int32_t* __restrict__ union_out) {
+                                                       int32_t* __restrict__ union_out, int item_rows,
+                                                       TcWorkItem* __restrict__ items, int* __restrict__ n_items) {
   __shared__ int cnt[PM_EMAX], base[PM_EMAX], run[PM_EMAX];
   __shared__ int wcnt[32][PM_EMAX];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -449,6 +450,18 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
     }
     offsets[E] = acc;
     *union_out = u;
+    // work list of the grouped expert GEMMs: each expert's rows in items of <= item_rows
+    int ni = 0;
+    for (int e = 0; e < E; ++e)
+      for (int r = 0; r < cnt[e]; r += item_rows) {
+        TcWorkItem it;
+        it.group = e;
+        it.row0 = base[e] + r;
+        it.rows = min(item_rows, cnt[e] - r);
+        it.pad = 0;
+        items[ni++] = it;
+      }
+    *n_items = ni;
   }
   __syncthreads();
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -479,9 +492,10 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
 }
 
 cudaError_t launch_permute(const int32_t* idx, int n, int k, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* perm, int32_t* inv, int32_t* union_out, cudaStream_t st) {
-  if (E > PM_EMAX) return cudaErrorInvalidValue;
-  permute_kernel<<<1, 1024, 0, st>>>(idx, n * k, E, counts, offsets, perm, inv, union_out);
+                           int32_t* perm, int32_t* inv, int32_t* union_out, int item_rows, TcWorkItem* items,
+                           int* n_items, cudaStream_t st) {
+  if (E > PM_EMAX || item_rows < 1) return cudaErrorInvalidValue;
+  permute_kernel<<<1, 1024, 0, st>>>(idx, n * k, E, counts, offsets, perm, inv, union_out, item_rows, items, n_items);
   return cudaGetLastError();
 }
 
@@ -513,19 +527,18 @@ cudaError_t launch_gather_rows(const T* xn, const T* xn_lo, const int32_t* perm,
   return cudaGetLastError();
 }
 
-// fp32 model: gu rows in the packed gate/up order -> h = silu(gate) * up
-__global__ void swiglu_packed_f32_kernel(const float* __restrict__ gu, int F, float* __restrict__ h) {
-  const int p = blockIdx.x;
-  const float* r = gu + (size_t)p * 2 * F;
+// fp32 model: h = silu(g) * u
+__global__ void swiglu_f32_kernel(const float* __restrict__ g, const float* __restrict__ u, int F,
+                                  float* __restrict__ h) {
+  const size_t base = (size_t)blockIdx.x * F;
   for (int f = threadIdx.x; f < F; f += blockDim.x) {
-    const int blk = f / 64, i = f % 64;
-    const float g = r[blk * 128 + i], u = r[blk * 128 + 64 + i];
-    h[(size_t)p * F + f] = g / (1.0f + expf(-g)) * u;
+    const float a = g[base + f];
+    h[base + f] = a / (1.0f + expf(-a)) * u[base + f];
   }
 }
-cudaError_t launch_swiglu_packed_f32(const float* gu, int rows, int F, float* h, cudaStream_t st) {
+cudaError_t launch_swiglu_f32(const float* g, const float* u, int rows, int F, float* h, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  swiglu_packed_f32_kernel<<<rows, 256, 0, st>>>(gu, F, h);
+  swiglu_f32_kernel<<<rows, 256, 0, st>>>(g, u, F, h);
   return cudaGetLastError();
 }
 
@@ -581,27 +594,6 @@ cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float
   if (n <= 0) return cudaSuccess;
   if (k > 16 || (H % 4) != 0) return cudaErrorInvalidValue;
   combine_norm_kernel<T><<<n, 256, 0, st>>>(ys, inv, w, k, H, eps, x, xn, xn_lo);
-  return cudaGetLastError();
-}
-
-// packed[e][b*128 + r] = r < 64 ? gate[e][b*64 + r] : up[e][b*64 + r - 64]  (rows of H elements)
-__global__ void pack_gate_up_kernel(const uint8_t* __restrict__ gate, const uint8_t* __restrict__ up,
-                                    uint8_t* __restrict__ out, int F, size_t row_bytes) {
-  const int prow = blockIdx.x;  // over E * 2F
-  const int e = prow / (2 * F), r2 = prow % (2 * F);
-  const int blk = r2 / 128, r = r2 % 128;
-  const uint8_t* src = (r < 64) ? gate + ((size_t)e * F + blk * 64 + r) * row_bytes
-                                : up + ((size_t)e * F + blk * 64 + r - 64) * row_bytes;
-  uint8_t* dst = out + (size_t)prow * row_bytes;
-  for (size_t i = threadIdx.x * 16; i < row_bytes; i += blockDim.x * 16)
-    *reinterpret_cast<uint4*>(dst + i) = *reinterpret_cast<const uint4*>(src + i);
-}
-cudaError_t launch_pack_gate_up(const void* gate, const void* up, void* out, int E, int F, int H, int elem_bytes,
-                                cudaStream_t st) {
-  const size_t row_bytes = (size_t)H * elem_bytes;
-  if ((row_bytes % 16) != 0 || (F % 64) != 0) return cudaErrorInvalidValue;
-  pack_gate_up_kernel<<<E * 2 * F, 128, 0, st>>>((const uint8_t*)gate, (const uint8_t*)up, (uint8_t*)out, F,
-                                                  row_bytes);
   return cudaGetLastError();
 }
 

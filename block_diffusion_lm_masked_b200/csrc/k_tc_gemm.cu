@@ -1,14 +1,18 @@
-// tcgen05 / TMEM / TMA GEMM for every dense contraction of the bf16 pass:
-// QKV and output projections, the two grouped expert GEMMs and the vocabulary
-// projection.  All of them stream a weight matrix once while the token operand
-// (at most 256 rows per tile) is small, so weights sit on the 128-row M side of
-// the MMA and tokens on N ("swap-AB"): one CTA owns a 128-row weight tile and
-// all tokens of its group (an expert's routed rows, or the whole canvas).
+// Persistent tcgen05 / TMEM / TMA GEMM for every dense contraction of the bf16 pass:
+// the QKV and output projections, the two grouped expert GEMMs and the vocabulary
+// projection.  All of them stream a weight matrix once while the token operand is
+// small, so weights sit on the 128-row M side of the MMA and tokens on N: a tile is
+// 128 weight rows x (up to n_max) token rows.
 //
-// Roles (128 threads): thread 0 issues TMA loads into a ring of smem stages,
-// thread 32 issues tcgen05.mma into a TMEM accumulator and frees stages with
-// tcgen05.commit, then all four warps drain TMEM (warp w owns lanes 32w..32w+31)
-// through the epilogue.  Stage count adapts to the token count at run time.
+// One CTA per SM walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Roles
+// (192 threads): warp 0 issues TMA loads into a ring of smem stages; warp 1 owns
+// the TMEM allocation and issues tcgen05.mma into one of two accumulator buffers;
+// warps 2-5 drain the other buffer through the epilogue, so the loads and MMAs of
+// tile i+1 overlap the epilogue of tile i.  Every wait is bounded.
+//
+// Options: two_terms (tokens given as bf16 hi + lo, both accumulated: fp32-precision
+// activations against bf16 weights); dual_a (gate and up weight tiles accumulated
+// into two TMEM regions, SwiGLU epilogue); k_splits (split-K, one output slab per split).
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -16,55 +20,81 @@ namespace dg {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
-constexpr int TC_MAX_N = 256;
 constexpr int TC_B_BOX = 16;
-constexpr int TC_MAX_STAGES = 24;
+constexpr int TC_MAX_STAGES = 16;
+constexpr int TC_THREADS = 192;
+
+struct TileInfo {
+  int g, row0, rows, split, m;
+};
+
+__device__ __forceinline__ int total_items(const TcGemmParams& p) {
+  if (p.items) return *p.n_items;
+  const int chunks = (p.n_tokens + p.n_max - 1) / p.n_max;
+  return chunks * p.k_splits;
+}
+
+// tile t -> (work item t / m_tiles, weight tile t % m_tiles)
+__device__ __forceinline__ TileInfo decode_tile(const TcGemmParams& p, int t) {
+  TileInfo ti;
+  const int item = t / p.m_tiles;
+  ti.m = t % p.m_tiles;
+  if (p.items) {
+    const TcWorkItem it = p.items[item];
+    ti.g = it.group;
+    ti.row0 = it.row0;
+    ti.rows = it.rows;
+    ti.split = 0;
+  } else {
+    const int chunk = item / p.k_splits;
+    ti.split = item % p.k_splits;
+    ti.g = 0;
+    ti.row0 = chunk * p.n_max;
+    ti.rows = min(p.n_max, p.n_tokens - ti.row0);
+  }
+  return ti;
+}
 
 template <int EPI>
-__global__ void __launch_bounds__(128, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const TcGemmParams p) {
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                   const TcGemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_MAX_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[TC_MAX_STAGES];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
+  __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ int n_issued_s, n_consumed_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.y;
-  int tok_begin = 0, tok_end = p.n_tokens;
-  if (p.group_off) {
-    tok_begin = p.group_off[g];
-    tok_end = p.group_off[g + 1];
-  }
-  const int split = (int)blockIdx.z % p.k_splits;
-  const int chunk = (int)blockIdx.z / p.k_splits;
-  const int t0 = tok_begin + chunk * TC_MAX_N;
-  if (t0 >= tok_end) return;  // uniform across the CTA, before any allocation
-  const int n = min(TC_MAX_N, tok_end - t0);
-  const int n_pad = (n + 15) & ~15;
   const int terms = p.two_terms ? 2 : 1;
-  const uint32_t a_bytes = TC_BM * TC_BK * 2;
-  const uint32_t b_bytes = (uint32_t)n_pad * TC_BK * 2;  // one term
-  const uint32_t stage_bytes = a_bytes + terms * b_bytes;
+  const int n_a = p.dual_a ? 2 : 1;
+  const uint32_t a_bytes = TC_BM * TC_BK * 2;           // one weight tile per k-block
+  const uint32_t bmax_bytes = (uint32_t)p.n_max * 128;  // one token term per k-block, n_max rows
+  const uint32_t stage_bytes = n_a * a_bytes + terms * bmax_bytes;
   int stages = p.smem_budget / (int)stage_bytes;
   if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int a_row0 = g * p.a_rows_per_group + (int)blockIdx.x * TC_BM;
-  const int nkb = p.K / TC_BK / p.k_splits;
-  const int kb0 = split * nkb;
+  const int acc_cols = p.n_max * n_a;  // one accumulator buffer
   uint32_t tmem_cols = 32;
-  while (tmem_cols < (uint32_t)n_pad) tmem_cols <<= 1;
+  while (tmem_cols < (uint32_t)(2 * acc_cols)) tmem_cols <<= 1;
+  const int nkb = p.K / TC_BK / p.k_splits;
 
-  if (warp == 0) tmem_alloc(&tmem_base_s, tmem_cols);
-  if (tid == 32) {
+  if (warp == 1) tmem_alloc(&tmem_base_s, tmem_cols);
+  if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&accum_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(&drain_bar, 1);
     abort_s = 0;
     n_issued_s = 0;
     n_consumed_s = 0;
@@ -74,142 +104,220 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  const int n_tiles = total_items(p) * p.m_tiles;
 
-  if (tid == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    if (terms == 2) prefetch_tmap(&tmB2);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % stages;
-      const uint32_t ph = (uint32_t)(kb / stages) & 1u;
-      if (!mbar_wait(&empty_bar[s], ph ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_EMPTY)) break;
-      uint8_t* sa = smem + (size_t)s * stage_bytes;
-      uint8_t* sb = sa + a_bytes;
-      const int kx = (kb0 + kb) * TC_BK;
-      mbar_arrive_expect_tx(&full_bar[s], stage_bytes);
-      tma_load_2d(sa, &tmA, kx, a_row0, &full_bar[s]);
-      for (int r = 0; r < n_pad; r += TC_B_BOX) tma_load_2d(sb + r * 128, &tmB, kx, t0 + r, &full_bar[s]);
-      if (terms == 2)
-        for (int r = 0; r < n_pad; r += TC_B_BOX)
-          tma_load_2d(sb + b_bytes + r * 128, &tmB2, kx, t0 + r, &full_bar[s]);
-      n_issued_s = kb + 1;
-    }
-  } else if (tid == 32) {
-    const uint32_t idesc = idesc_bf16_f32(TC_BM, n_pad);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % stages;
-      const uint32_t ph = (uint32_t)(kb / stages) & 1u;
-      if (!mbar_wait(&full_bar[s], ph, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) break;
-      tc_fence_after();
-      const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
-      const uint32_t sb = sa + a_bytes;
-#pragma unroll
-      for (int kk = 0; kk < TC_BK / 16; ++kk) {
-        const uint64_t ad = sw128_kmajor_desc(sa + kk * 32);
-        tc_mma(tmem, ad, sw128_kmajor_desc(sb + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
-        if (terms == 2) tc_mma(tmem, ad, sw128_kmajor_desc(sb + b_bytes + kk * 32), idesc, 1u);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      prefetch_tmap(&tmA);
+      if (p.dual_a) prefetch_tmap(&tmA2);
+      prefetch_tmap(&tmB);
+      if (terms == 2) prefetch_tmap(&tmB2);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(p, t);
+        const int n_pad = (ti.rows + 15) & ~15;
+        const uint32_t tx = n_a * a_bytes + terms * (uint32_t)n_pad * 128;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % stages;
+          if (!mbar_wait(&empty_bar[s], ((uint32_t)(it / stages) & 1u) ^ 1u, &abort_s, p.err,
+                         DG_DEVERR_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + (size_t)s * stage_bytes;
+          uint8_t* sb = sa + n_a * a_bytes;
+          const int kx = (ti.split * nkb + kb) * TC_BK;
+          mbar_arrive_expect_tx(&full_bar[s], tx);
+          tma_load_3d(sa, &tmA, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
+          if (p.dual_a) tma_load_3d(sa + a_bytes, &tmA2, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
+          for (int r = 0; r < n_pad; r += TC_B_BOX) {
+            tma_load_2d(sb + r * 128, &tmB, kx, ti.row0 + r, &full_bar[s]);
+            if (terms == 2) tma_load_2d(sb + bmax_bytes + r * 128, &tmB2, kx, ti.row0 + r, &full_bar[s]);
+          }
+          n_issued_s = it + 1;
+        }
       }
-      tc_commit(&empty_bar[s]);
-      n_consumed_s = kb + 1;
     }
-    tc_commit(&accum_bar);
-  }
-  __syncwarp();
-
-  mbar_wait(&accum_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM);
-  __syncthreads();
-  const bool run = (abort_s == 0);  // uniform across the CTA
-  tc_fence_after();
-  const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
-  if (run) {
-    if (EPI == EPI_STORE_F32 || EPI == EPI_ADD_F32) {
-      float* out = reinterpret_cast<float*>(p.out) + (size_t)split * p.split_stride;
-      const int feat = (int)blockIdx.x * TC_BM + warp * 32 + lane;
-      for (int c0 = 0; c0 < n_pad; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(t_lane + c0, r);
-        tc_wait_ld();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++j) {
+        const TileInfo ti = decode_tile(p, t);
+        const int n_pad = (ti.rows + 15) & ~15;
+        const int buf = j & 1;
+        if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
+          break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
+        const uint32_t d1 = d0 + (uint32_t)p.n_max;
+        const uint32_t idesc = idesc_bf16_f32(TC_BM, n_pad);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % stages;
+          if (!mbar_wait(&full_bar[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+          const uint32_t sb = sa + n_a * a_bytes;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (c0 + j < n) {
-            float* dst = out + (size_t)(t0 + c0 + j) * p.ld_out + feat;
-            const float v = __uint_as_float(r[j]);
-            if (EPI == EPI_ADD_F32)
-              *dst += v;
-            else
-              *dst = v;
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint64_t ad = sw128_kmajor_desc(sa + kk * 32);
+            const uint64_t bd = sw128_kmajor_desc(sb + kk * 32);
+            const uint64_t bd2 = sw128_kmajor_desc(sb + bmax_bytes + kk * 32);
+            tc_mma(d0, ad, bd, idesc, acc);
+            if (terms == 2) tc_mma(d0, ad, bd2, idesc, 1u);
+            if (p.dual_a) {
+              const uint64_t ad2 = sw128_kmajor_desc(sa + a_bytes + kk * 32);
+              tc_mma(d1, ad2, bd, idesc, acc);
+              if (terms == 2) tc_mma(d1, ad2, bd2, idesc, 1u);
+            }
+          }
+          tc_commit(&empty_bar[s]);
+          n_consumed_s = it + 1;
+        }
+        if (ok) tc_commit(&acc_full[buf]);
+      }
+      tc_commit(&drain_bar);  // completes once every MMA issued above has landed
+    }
+  } else {
+    // ---------------- epilogue warps 2..5: TMEM lanes (warp % 4) * 32 .. + 31
+    const int lg = warp & 3;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    int j = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++j) {
+      const TileInfo ti = decode_tile(p, t);
+      const int n_pad = (ti.rows + 15) & ~15;
+      const int buf = j & 1;
+      if (!mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)) break;
+      tc_fence_after();
+      const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
+      const int f = ti.m * TC_BM + lg * 32 + lane;  // weight row = output feature
+      const bool fvalid = f < p.a_rows_per_group;
+      if (EPI == EPI_STORE_F32) {
+        float* out = reinterpret_cast<float*>(p.out) + (size_t)ti.split * p.split_stride;
+        for (int c0 = 0; c0 < n_pad; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(t0 + c0, r);
+          tc_wait_ld();
+          if (fvalid) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              if (c0 + q < ti.rows) out[(size_t)(ti.row0 + c0 + q) * p.ld_out + f] = __uint_as_float(r[q]);
           }
         }
-      }
-    } else {
-      // packed gate/up tile: lanes 0..63 hold gate rows f0..f0+63, lanes 64..127 the up rows
-      float* xch = reinterpret_cast<float*>(smem);  // [n_pad][64]; all loads were consumed
-      if (warp >= 2) {
-        for (int c0 = 0; c0 < n_pad; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(t_lane + c0, r);
-          tc_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) xch[(c0 + j) * 64 + (warp - 2) * 32 + lane] = __uint_as_float(r[j]);
-        }
-      }
-      __syncthreads();
-      if (warp < 2) {
+      } else {
         bf16* out = reinterpret_cast<bf16*>(p.out);
         bf16* out_lo = reinterpret_cast<bf16*>(p.out_lo);
-        const int f = (int)blockIdx.x * 64 + warp * 32 + lane;
         for (int c0 = 0; c0 < n_pad; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(t_lane + c0, r);
+          uint32_t rg[16], ru[16];
+          tmem_ld16(t0 + c0, rg);
+          tmem_ld16(t0 + p.n_max + c0, ru);
           tc_wait_ld();
+          if (fvalid) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c0 + j < n) {
-              const float gte = __uint_as_float(r[j]);
-              const float up = xch[(c0 + j) * 64 + warp * 32 + lane];
-              const float hv = gte / (1.0f + expf(-gte)) * up;
-              const bf16 hi = __float2bfloat16_rn(hv);
-              out[(size_t)(t0 + c0 + j) * p.ld_out + f] = hi;
-              if (out_lo) out_lo[(size_t)(t0 + c0 + j) * p.ld_out + f] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+            for (int q = 0; q < 16; ++q) {
+              if (c0 + q < ti.rows) {
+                const float gte = __uint_as_float(rg[q]);
+                const float hv = gte / (1.0f + expf(-gte)) * __uint_as_float(ru[q]);
+                const bf16 hi = __float2bfloat16_rn(hv);
+                const size_t o = (size_t)(ti.row0 + c0 + q) * p.ld_out + f;
+                out[o] = hi;
+                if (out_lo) out_lo[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+              }
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
-  } else if (tid == 0) {
-    // wind down: let issued loads and MMAs land before the smem / TMEM go away
-    for (int kb = n_consumed_s; kb < n_issued_s; ++kb)
-      mbar_wait_drain(&full_bar[kb % stages], (uint32_t)(kb / stages) & 1u);
-    mbar_wait_drain(&accum_bar, 0);
   }
+
+  __syncthreads();
+  if (abort_s && tid == 0) {
+    // wind down: let issued loads land before the smem goes away
+    for (int i = n_consumed_s; i < n_issued_s; ++i)
+      mbar_wait_drain(&full_bar[i % stages], (uint32_t)(i / stages) & 1u);
+  }
+  if (tid == 32) mbar_wait_drain(&drain_bar, 0);  // every issued MMA has landed
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 }
 
-cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& B2,
-                           const TcGemmParams& p, int m_tiles, int n_groups, int max_rows_per_group, cudaStream_t st) {
-  if (m_tiles <= 0 || n_groups <= 0 || max_rows_per_group <= 0) return cudaSuccess;
-  if (p.k_splits < 1 || (p.K / TC_BK) % p.k_splits != 0 || (p.k_splits > 1 && n_groups != 1))
+// ---------------------------------------------------------------- work items of a grouped GEMM
+// For each group g with rows [off[g], off[g+1]): items of at most n_max rows, in group
+// order.  Written by one thread (E is small).
+static __device__ void emit_work_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items) {
+  int ni = 0;
+  for (int e = 0; e < E; ++e) {
+    const int c = off[e + 1] - off[e];
+    for (int r = 0; r < c; r += n_max) {
+      TcWorkItem it;
+      it.group = e;
+      it.row0 = off[e] + r;
+      it.rows = min(n_max, c - r);
+      it.pad = 0;
+      items[ni++] = it;
+    }
+  }
+  *n_items = ni;
+}
+
+__global__ void build_items_kernel(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) emit_work_items(off, E, n_max, items, n_items);
+}
+
+cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
+                               cudaStream_t st) {
+  build_items_kernel<<<1, 32, 0, st>>>(off, E, n_max, items, n_items);
+  return cudaGetLastError();
+}
+
+static int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
+                           const CUtensorMap& B2, const TcGemmParams& p, int max_tiles, cudaStream_t st) {
+  if (max_tiles <= 0) return cudaSuccess;
+  if (p.k_splits < 1 || (p.K / TC_BK) % p.k_splits != 0 || (p.k_splits > 1 && p.items) || p.n_max < 16 ||
+      p.n_max > 256 || (p.n_max % 16) != 0 || p.m_tiles < 1)
+    return cudaErrorInvalidValue;
+  const int n_a = p.dual_a ? 2 : 1;
+  const int stage = n_a * TC_BM * TC_BK * 2 + (p.two_terms ? 2 : 1) * p.n_max * 128;
+  if (p.smem_budget < stage || 2 * p.n_max * n_a > 512 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
     return cudaErrorInvalidValue;
   const int smem = p.smem_budget + 1024;
-  dim3 grid(m_tiles, n_groups, ((max_rows_per_group + TC_MAX_N - 1) / TC_MAX_N) * p.k_splits);
+  const int sms = num_sms();
+  const int grid = max_tiles < sms ? max_tiles : sms;
   cudaError_t e;
   switch (epi) {
     case EPI_STORE_F32:
       e = cudaFuncSetAttribute(tc_gemm_kernel<EPI_STORE_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
-      tc_gemm_kernel<EPI_STORE_F32><<<grid, 128, smem, st>>>(A, B, B2, p);
-      break;
-    case EPI_ADD_F32:
-      e = cudaFuncSetAttribute(tc_gemm_kernel<EPI_ADD_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      tc_gemm_kernel<EPI_ADD_F32><<<grid, 128, smem, st>>>(A, B, B2, p);
+      tc_gemm_kernel<EPI_STORE_F32><<<grid, TC_THREADS, smem, st>>>(A, A2, B, B2, p);
       break;
     case EPI_SWIGLU_BF16:
       e = cudaFuncSetAttribute(tc_gemm_kernel<EPI_SWIGLU_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
-      tc_gemm_kernel<EPI_SWIGLU_BF16><<<grid, 128, smem, st>>>(A, B, B2, p);
+      tc_gemm_kernel<EPI_SWIGLU_BF16><<<grid, TC_THREADS, smem, st>>>(A, A2, B, B2, p);
       break;
     default:
       return cudaErrorInvalidValue;

@@ -39,7 +39,7 @@ class Config(ctypes.Structure):
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p), ("w_router", ctypes.c_void_p),
-                ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+                ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
 
 
 class Weights(ctypes.Structure):
@@ -73,7 +73,6 @@ def _load():
         "dg_denoise_pass": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, P, SZ, P]),
         "dg_canvas_update": (I32, [P, I32, I32, I32, U64, U32, P, P, P, SZ, P]),
         "dg_generate_canvas": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, U64, I32, P, P, SZ, P]),
-        "dg_pack_gate_up": (I32, [P, P, P, I32, I32, I32, I32, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
         "dg_set_taps": (I32, [P, ctypes.POINTER(Taps)]),
@@ -84,7 +83,7 @@ def _load():
         "dg_launch_count": (ctypes.c_int64, []),
         "dg_renoise_count": (I32, [I32, I32, I32, F32, F32]),
         "dg_debug_bounded_wait": (I32, [P, I32, P]),
-        "dg_debug_gemm_bf16": (I32, [I32, P, I32, I32, P, P, I32, I32, P, I32, P, P, I32, P, P]),
+        "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, P, P]),
         "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -138,22 +137,15 @@ class Model:
         self.embed = _upload(host_model.embed, device)
         self.w_out = _upload(host_model.w_out, device)
         self.layers = []
-        eb = 2 if cfg["dtype"] == "bf16" else 4
         for L in host_model.layers:
             wqkv = _upload(np.concatenate([L["w_q"], L["w_k"], L["w_v"]], axis=0), device)
-            gate = _upload(L["w_gate"], device)
-            up = _upload(L["w_up"], device)
-            E, F, H = L["w_gate"].shape
-            gu = torch.empty((E, 2 * F, H), dtype=gate.dtype, device=device)
-            _check(lib.dg_pack_gate_up(_ptr(gate), _ptr(up), _ptr(gu), E, F, H, eb, _stream()))
-            torch.cuda.current_stream().synchronize()
-            del gate, up
             self.layers.append(dict(w_qkv=wqkv, w_o=_upload(L["w_o"], device),
                                     w_router=torch.from_numpy(np.ascontiguousarray(L["w_router"], np.float32)).to(device),
-                                    w_gate_up=gu, w_down=_upload(L["w_down"], device)))
+                                    w_gate=_upload(L["w_gate"], device), w_up=_upload(L["w_up"], device),
+                                    w_down=_upload(L["w_down"], device)))
         self._lw = (LayerWeights * len(self.layers))(*[
             LayerWeights(L["w_qkv"].data_ptr(), L["w_o"].data_ptr(), L["w_router"].data_ptr(),
-                         L["w_gate_up"].data_ptr(), L["w_down"].data_ptr()) for L in self.layers])
+                         L["w_gate"].data_ptr(), L["w_up"].data_ptr(), L["w_down"].data_ptr()) for L in self.layers])
         self._w = Weights(self.embed.data_ptr(), self.w_out.data_ptr(), self._lw)
         self._cfg = make_config(cfg)
         h = ctypes.c_void_p()
@@ -309,12 +301,12 @@ def launch_count() -> int:
     return int(lib.dg_launch_count())
 
 
-def debug_gemm_bf16(epi, W, a_rows_per_group, n_groups, X, group_off, max_rows_per_group, out, ld_out, err,
-                    X_lo=None, out_lo=None, stream=None):
-    """One tcgen05 GEMM launch (see include/dg_debug.h)."""
-    _check(lib.dg_debug_gemm_bf16(epi, _ptr(W), a_rows_per_group, n_groups, _ptr(X), _ptr(X_lo), X.shape[0],
-                                  X.shape[1], _ptr(group_off), max_rows_per_group, _ptr(out), _ptr(out_lo), ld_out,
-                                  _ptr(err), _stream(stream)))
+def debug_gemm_bf16(W, X, out, ld_out, err, scratch, W2=None, X_lo=None, group_off=None, out_lo=None,
+                    stream=None):
+    """One persistent tcgen05 GEMM launch (see include/dg_debug.h). W [groups][rows][K]."""
+    G, rows, K = W.shape
+    _check(lib.dg_debug_gemm_bf16(_ptr(W), _ptr(W2), rows, G, _ptr(X), _ptr(X_lo), X.shape[0], K, _ptr(group_off),
+                                  _ptr(out), _ptr(out_lo), ld_out, _ptr(scratch), _ptr(err), _stream(stream)))
 
 
 def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out_lo=None, stream=None):

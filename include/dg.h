@@ -36,9 +36,7 @@
  *     w_qkv          [(nq + 2 nkv) d][H]    rows of W_q, then W_k, then W_v
  *     w_o            [H][nq d]
  *     w_router       [E][H]                 always fp32
- *     w_gate_up      [E][2F][H]             packed: for b = 0..F/64-1, rows 128b..128b+63
- *                                            are gate rows 64b..64b+63, rows 128b+64..128b+127
- *                                            the up rows 64b..64b+63 (see dg_pack_gate_up)
+ *     w_gate, w_up   [E][F][H]              SwiGLU expert: h = silu(x W_gate^T) * (x W_up^T)
  *     w_down         [E][H][F]
  *   KV cache, per layer:  K [nkv][capacity][d],  V transposed: Vt [nkv][d][capacity]
  *   canvas / tokens int32 [n];  logits fp32 [C][V]
@@ -74,15 +72,15 @@ typedef struct dg_config {
   int32_t dtype;    /* dg_dtype of weights, activations and KV cache                 */
 } dg_config;
 /* Shape rules.  Both dtypes: n_q_heads % n_kv_heads == 0, top_k <= min(16, n_experts),
- * n_experts <= 256, hidden % 64 == 0, expert_ffn % 64 == 0.  bf16 additionally:
- * head_dim == 128, vocab % 128 == 0, (n_q_heads + 2 n_kv_heads) * 128 % 128 == 0.
- * fp32: head_dim <= 128. */
+ * n_experts <= 256, hidden % 64 == 0, expert_ffn % 64 == 0, vocab % 4 == 0,
+ * head_dim even and <= 128.  bf16 additionally: head_dim == 128, hidden % 128 == 0. */
 
 typedef struct dg_layer_weights {
   const void* w_qkv;
   const void* w_o;
   const float* w_router;
-  const void* w_gate_up;
+  const void* w_gate;
+  const void* w_up;
   const void* w_down;
 } dg_layer_weights;
 
@@ -150,11 +148,6 @@ dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas,
 
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
-
-/* Lay out separate gate and up weights ([E][F][H] each) in the packed w_gate_up layout.
- * elem_bytes: 2 (bf16) or 4 (fp32).  Pure data movement on the stream. */
-dg_status dg_pack_gate_up(const void* d_gate, const void* d_up, void* d_out, int32_t E, int32_t F, int32_t H,
-                          int32_t elem_bytes, dg_stream stream);
 
 /* Synchronize the stream, read and clear the workspace error word.  DG_OK or
  * DG_ERR_TIMEOUT (a kernel's bounded wait gave up; its outputs are not valid). */

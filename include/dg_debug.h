@@ -66,18 +66,17 @@ dg_status dg_profile_read(int32_t kind, double* total_ms, int32_t* launches);
 void dg_profile_reset(void);
 const char* dg_kernel_name(int32_t kind);
 
-/* One launch of the tcgen05 GEMM alone (bf16):
- *   out[r][f] (op)= sum_k W[g * a_rows_per_group + f][k] * (X[r][k] + X_lo[r][k])
+/* One launch of the persistent tcgen05 GEMM alone (bf16):
+ *   acc[r][f] = sum_k W[g][f][k] * (X[r][k] + X_lo[r][k])   (X_lo NULL: X alone)
  * for rows r of group g = [group_off[g], group_off[g+1]) (group_off: device int32
- * [n_groups + 1], or NULL for one group of x_rows rows; X_lo NULL: X alone).  epi 0:
- * store fp32 out, 1: add into fp32 out, 2: packed gate/up rows -> silu(gate) * up with
- * a_rows_per_group / 2 output columns, written as bf16 hi (out) and lo (out_lo, or
- * NULL).  W [n_groups * a_rows_per_group][K], X [x_rows][K] bf16; K % 64 == 0,
- * a_rows_per_group % 128 == 0.  d_err: device int32 error word. */
-dg_status dg_debug_gemm_bf16(int32_t epi, const void* W, int32_t a_rows_per_group, int32_t n_groups, const void* X,
-                             const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off,
-                             int32_t max_rows_per_group, void* out, void* out_lo, int32_t ld_out, int32_t* d_err,
-                             dg_stream stream);
+ * [n_groups + 1], or NULL for one group of x_rows rows).  W is [n_groups][rows][K].
+ * W2 NULL: out (fp32, row stride ld_out) = acc.  W2 given (same shape as W): out / out_lo
+ * (bf16 hi / lo, out_lo nullable) = silu(acc) * acc2, acc2 the same sum over W2.
+ * K % 64 == 0, rows >= 1.  d_scratch: >= 16 * (x_rows + n_groups + 1) device bytes
+ * (work list); d_err: device int32 error word. */
+dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_t n_groups, const void* X,
+                             const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off, void* out,
+                             void* out_lo, int32_t ld_out, void* d_scratch, int32_t* d_err, dg_stream stream);
 
 /* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
  * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
