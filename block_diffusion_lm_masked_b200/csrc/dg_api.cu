@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -17,6 +18,11 @@
 #include "dg_kernels.h"
 
 using dg::bf16;
+
+bool dg::pdl_enabled() {
+  static const bool on = getenv("DG_NO_PDL") == nullptr;
+  return on;
+}
 
 // ---------------------------------------------------------------- errors
 static thread_local std::string g_err;
@@ -337,13 +343,16 @@ struct GemmCall {
 };
 
 dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
-  CUtensorMap B, B2;
-  dg_status s = map_rows(&B, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 16);
-  if (s != DG_OK) return s;
+  CUtensorMap B, B2, Bb, B2b;
+  dg_status s;
+  if ((s = map_rows(&B, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
+  if ((s = map_rows(&Bb, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 64)) != DG_OK) return s;
   if (g.X_lo) {
     if ((s = map_rows(&B2, g.X_lo, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
+    if ((s = map_rows(&B2b, g.X_lo, (uint64_t)g.x_rows, (uint64_t)g.K, 64)) != DG_OK) return s;
   } else {
     B2 = B;
+    B2b = Bb;
   }
   dg::TcGemmParams p{};
   p.K = g.K;
@@ -364,7 +373,7 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   p.err = err;
   const int items = g.items ? g.max_items : ceil_div(g.x_rows, g.n_max) * g.k_splits;
   LAUNCH(g.kind, st,
-         dg::launch_tc_gemm(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, B, B2, p, items * p.m_tiles, st));
+         dg::launch_tc_gemm(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, B, B2, Bb, B2b, p, items * p.m_tiles, st));
   return DG_OK;
 }
 

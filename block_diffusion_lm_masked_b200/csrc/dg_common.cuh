@@ -5,6 +5,8 @@
 // time it records an error code in the caller's device error word, raises the
 // CTA's abort flag and returns false, and the kernel winds down (no trap).
 #pragma once
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -23,6 +25,41 @@
 namespace dg {
 
 typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: its
+// CTAs may become resident while the previous kernel on the stream still runs.  Each
+// kernel therefore waits (griddepcontrol.wait: the previous grid has completed and its
+// memory is visible) before it reads or writes global memory, then lets the next kernel
+// launch.  Work before the wait touches only registers, shared memory and TMEM.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_sync() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
+
+bool pdl_enabled();  // false if DG_NO_PDL is set in the environment
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }

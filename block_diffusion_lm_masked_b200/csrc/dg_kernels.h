@@ -10,7 +10,7 @@ namespace dg {
 // ---------------------------------------------------------------- tcgen05 GEMM
 // out[row][feature] (op)= sum_k W[g][feature][k] * X[row][k]
 // W comes from a 3-D tensor map (K, rows per group, groups), box 64 x 128 x 1; X from
-// a 2-D map (K, rows), box 64 x 16.  With two_terms, X = X_hi + X_lo (maps B and B2);
+// 2-D maps (K, rows) with boxes of 64 x 16 and 64 x 64 rows.  With two_terms, X = X_hi + X_lo (maps B and B2);
 // with dual_a, a second weight tensor (map A2, same shape) accumulates into a second
 // TMEM region and the epilogue writes silu(W x) * (W2 x) as bf16 hi (+ lo).
 // Work: dense -- rows [0, n_tokens) in chunks of n_max, times k_splits (split s reduces
@@ -42,8 +42,10 @@ struct TcGemmParams {
 };
 
 // grid = min(max_tiles, SMs); max_tiles bounds the tile count (exact for dense GEMMs)
+// B / B2: token maps with 16-row boxes; Bb / B2b: the same tensors with 64-row boxes
 cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
-                           const CUtensorMap& B2, const TcGemmParams& p, int max_tiles, cudaStream_t st);
+                           const CUtensorMap& B2, const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p,
+                           int max_tiles, cudaStream_t st);
 cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
                                cudaStream_t st);
 int num_sms();

@@ -40,6 +40,7 @@ template <typename T>
 __global__ void embed_norm_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ embed, int V, int H,
                                   float eps, float* __restrict__ x, T* __restrict__ xn, T* __restrict__ xn_lo,
                                   int* __restrict__ err) {
+  griddep_sync();
   __shared__ float red[32];
   const int t = blockIdx.x;
   int tok = tokens[t];
@@ -70,8 +71,7 @@ template <typename T>
 cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int V, int H, float eps, float* x, T* xn,
                               T* xn_lo, int* err, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  embed_norm_kernel<T><<<n, 256, 0, st>>>(tokens, embed, V, H, eps, x, xn, xn_lo, err);
-  return cudaGetLastError();
+  return launch_k(embed_norm_kernel<T>, dim3(n), dim3(256), 0, st, tokens, embed, V, H, eps, x, xn, xn_lo, err);
 }
 
 // ---------------------------------------------------------------- RoPE + KV cache write
@@ -82,6 +82,7 @@ template <typename T>
 __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, size_t part_stride, int nq, int nkv,
                                     int d, int pos0, float theta, int n, T* __restrict__ q, T* __restrict__ kc,
                                     T* __restrict__ vtc, int cap) {
+  griddep_sync();
   extern __shared__ float cs[];  // [d/2] cos, [d/2] sin, then the summed qkv row
   const int t = blockIdx.x;
   const int half = d / 2;
@@ -134,9 +135,7 @@ cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_strid
                                 int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const size_t smem = (size_t)(d + (nq + 2 * nkv) * d) * sizeof(float);
-  rope_scatter_kernel<T><<<n, 256, smem, st>>>(qkv, n_parts, part_stride, nq, nkv, d, pos0, theta, n, q, kcache,
-                                                vtcache, cap);
-  return cudaGetLastError();
+  return launch_k(rope_scatter_kernel<T>, dim3(n), dim3(256), smem, st, qkv, n_parts, part_stride, nq, nkv, d, pos0, theta, n, q, kcache, vtcache, cap);
 }
 
 // ---------------------------------------------------------------- fp32 GEMM (fp32 model)
@@ -145,6 +144,7 @@ constexpr int SG_BT = 32, SG_BF = 64, SG_BK = 32;
 __global__ void simt_gemm_f32_kernel(int epi_add, const float* __restrict__ W, const float* __restrict__ X,
                                      const int* __restrict__ group_off, int n_tokens, int M, int K,
                                      float* __restrict__ out, int ld_out) {
+  griddep_sync();
   __shared__ float sx[SG_BT][SG_BK + 1];
   __shared__ float sw[SG_BF][SG_BK + 1];
   const int g = blockIdx.y;
@@ -205,8 +205,7 @@ cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, co
                                  cudaStream_t st) {
   if (max_rows_per_group <= 0 || n_groups <= 0) return cudaSuccess;
   dim3 grid((M + SG_BF - 1) / SG_BF, n_groups, (max_rows_per_group + SG_BT - 1) / SG_BT);
-  simt_gemm_f32_kernel<<<grid, 256, 0, st>>>(epi_add, W, X, group_off, n_tokens, M, K, out, ld_out);
-  return cudaGetLastError();
+  return launch_k(simt_gemm_f32_kernel, dim3(grid), dim3(256), 0, st, epi_add, W, X, group_off, n_tokens, M, K, out, ld_out);
 }
 
 // ---------------------------------------------------------------- fp32 attention (fp32 model)
@@ -214,6 +213,7 @@ cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, co
 __global__ void simt_attention_f32_kernel(const float* __restrict__ q, const float* __restrict__ kc,
                                           const float* __restrict__ vtc, int cap, int n_q, int q_pos0, int n_keys,
                                           int causal, int nq, int nkv, int d, float* __restrict__ out) {
+  griddep_sync();
   __shared__ float sq[128];
   const int qrow = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
   const int kvh = h / (nq / nkv);
@@ -262,9 +262,8 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
                                       int q_pos0, int n_keys, int causal, int nq, int nkv, int d, float* out,
                                       cudaStream_t st) {
   if (n_q <= 0) return cudaSuccess;
-  simt_attention_f32_kernel<<<dim3(n_q, nq), 32, 0, st>>>(q, kcache, vtcache, cap, n_q, q_pos0, n_keys, causal, nq,
-                                                          nkv, d, out);
-  return cudaGetLastError();
+  return launch_k(simt_attention_f32_kernel, dim3(n_q, nq), dim3(32), 0, st, q, kcache, vtcache, cap, n_q, q_pos0, n_keys,
+           causal, nq, nkv, d, out);
 }
 
 // ---------------------------------------------------------------- residual + RMSNorm + router + top-k
@@ -280,6 +279,7 @@ __global__ void __launch_bounds__(RTF_THREADS) router_fused_kernel(
     float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
     const float* __restrict__ wr, int n, int H, int E, int k, float eps, float* __restrict__ logits_out,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, T* __restrict__ xn, T* __restrict__ xn_lo) {
+  griddep_sync();
   extern __shared__ float sm[];  // xs[RTF_TOK][H], lg[RTF_TOK][E]
   float* xs = sm;
   float* lg = sm + RTF_TOK * H;
@@ -414,9 +414,7 @@ cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_
   const size_t smem = (size_t)RTF_TOK * (H + E) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  router_fused_kernel<T><<<(n + RTF_TOK - 1) / RTF_TOK, RTF_THREADS, smem, st>>>(
-      x, parts, n_parts, part_stride, w_router, n, H, E, k, eps, logits, topk_idx, topk_w, xn, xn_lo);
-  return cudaGetLastError();
+  return launch_k(router_fused_kernel<T>, dim3((n + RTF_TOK - 1) / RTF_TOK), dim3(RTF_THREADS), smem, st, x, parts, n_parts, part_stride, w_router, n, H, E, k, eps, logits, topk_idx, topk_w, xn, xn_lo);
 }
 
 // ---------------------------------------------------------------- expert histogram + stable permutation
@@ -429,6 +427,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
                                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                                        int32_t* __restrict__ union_out, int item_rows,
                                                        TcWorkItem* __restrict__ items, int* __restrict__ n_items) {
+  griddep_sync();
   __shared__ int cnt[PM_EMAX], base[PM_EMAX], run[PM_EMAX];
   __shared__ int wcnt[32][PM_EMAX];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -495,8 +494,7 @@ cudaError_t launch_permute(const int32_t* idx, int n, int k, int E, int32_t* cou
                            int32_t* perm, int32_t* inv, int32_t* union_out, int item_rows, TcWorkItem* items,
                            int* n_items, cudaStream_t st) {
   if (E > PM_EMAX || item_rows < 1) return cudaErrorInvalidValue;
-  permute_kernel<<<1, 1024, 0, st>>>(idx, n * k, E, counts, offsets, perm, inv, union_out, item_rows, items, n_items);
-  return cudaGetLastError();
+  return launch_k(permute_kernel, dim3(1), dim3(1024), 0, st, idx, n * k, E, counts, offsets, perm, inv, union_out, item_rows, items, n_items);
 }
 
 // xs[p] = xn[perm[p] / k] for the hi and (if present) lo parts; 16-byte vector copies
@@ -504,6 +502,7 @@ template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ xn, const T* __restrict__ xn_lo,
                                    const int32_t* __restrict__ perm, int k, int H, T* __restrict__ xs,
                                    T* __restrict__ xs_lo) {
+  griddep_sync();
   const int p = blockIdx.x;
   const int t = perm[p] / k;
   const int nv = H * (int)sizeof(T) / 16;
@@ -523,13 +522,13 @@ template <typename T>
 cudaError_t launch_gather_rows(const T* xn, const T* xn_lo, const int32_t* perm, int rows, int k, int H, T* xs,
                                T* xs_lo, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  gather_rows_kernel<T><<<rows, 128, 0, st>>>(xn, xn_lo, perm, k, H, xs, xs_lo);
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel<T>, dim3(rows), dim3(128), 0, st, xn, xn_lo, perm, k, H, xs, xs_lo);
 }
 
 // fp32 model: h = silu(g) * u
 __global__ void swiglu_f32_kernel(const float* __restrict__ g, const float* __restrict__ u, int F,
                                   float* __restrict__ h) {
+  griddep_sync();
   const size_t base = (size_t)blockIdx.x * F;
   for (int f = threadIdx.x; f < F; f += blockDim.x) {
     const float a = g[base + f];
@@ -538,8 +537,7 @@ __global__ void swiglu_f32_kernel(const float* __restrict__ g, const float* __re
 }
 cudaError_t launch_swiglu_f32(const float* g, const float* u, int rows, int F, float* h, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  swiglu_f32_kernel<<<rows, 256, 0, st>>>(g, u, F, h);
-  return cudaGetLastError();
+  return launch_k(swiglu_f32_kernel, dim3(rows), dim3(256), 0, st, g, u, F, h);
 }
 
 // x[t] += sum_j w[t][j] * ys[inv[t*k + j]] (slots in order j = 0..k-1), then
@@ -549,6 +547,7 @@ template <typename T>
 __global__ void combine_norm_kernel(const float* __restrict__ ys, const int32_t* __restrict__ inv,
                                     const float* __restrict__ w, int k, int H, float eps, float* __restrict__ x,
                                     T* __restrict__ xn, T* __restrict__ xn_lo) {
+  griddep_sync();
   const int t = blockIdx.x;
   __shared__ int rows[16];
   __shared__ float ws[16];
@@ -593,8 +592,7 @@ cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float
                                 float* x, T* xn, T* xn_lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   if (k > 16 || (H % 4) != 0) return cudaErrorInvalidValue;
-  combine_norm_kernel<T><<<n, 256, 0, st>>>(ys, inv, w, k, H, eps, x, xn, xn_lo);
-  return cudaGetLastError();
+  return launch_k(combine_norm_kernel<T>, dim3(n), dim3(256), 0, st, ys, inv, w, k, H, eps, x, xn, xn_lo);
 }
 
 // ---------------------------------------------------------------- canvas update
@@ -627,6 +625,7 @@ int update_splits(int C, int V) {
 
 // per (row, slice): max, first argmax and sum exp(l - max), one streaming pass
 __global__ void update_partial_kernel(const float* __restrict__ logits, int V, int splits, UpdPart* __restrict__ part) {
+  griddep_sync();
   __shared__ float sm[32], ss[32];
   __shared__ int sa[32];
   const int row = blockIdx.x, sp = blockIdx.y;
@@ -694,6 +693,7 @@ __device__ __forceinline__ uint64_t splitmix64_out(uint64_t seed, uint64_t n) {
 __global__ void update_select_kernel(const UpdPart* __restrict__ part, int C, int V, int splits, int n_renoise,
                                      uint64_t seed, uint32_t step, int32_t* __restrict__ canvas,
                                      float* __restrict__ conf) {
+  griddep_sync();
   extern __shared__ float den[];  // [C]
   const int i = threadIdx.x;
   float m = -INFINITY, s = 0.0f;
@@ -724,23 +724,21 @@ __global__ void update_select_kernel(const UpdPart* __restrict__ part, int C, in
 
 cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, UpdPart* part, cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
-  update_partial_kernel<<<dim3(C, splits), 256, 0, st>>>(logits, V, splits, part);
-  return cudaGetLastError();
+  return launch_k(update_partial_kernel, dim3(C, splits), dim3(256), 0, st, logits, V, splits, part);
 }
 cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
                                  uint32_t step, int32_t* canvas, float* conf, cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
   if (C > 1024) return cudaErrorInvalidValue;
   const int threads = (C + 31) & ~31;
-  update_select_kernel<<<1, threads, C * sizeof(float), st>>>(part, C, V, splits, n_renoise, seed, step, canvas,
-                                                              conf);
-  return cudaGetLastError();
+  return launch_k(update_select_kernel, dim3(1), dim3(threads), C * sizeof(float), st, part, C, V, splits, n_renoise, seed, step, canvas, conf);
 }
 
 // ---------------------------------------------------------------- timeout self-test
 // One thread waits on an mbarrier that nothing will complete; the bounded wait gives
 // up after limit_ns, records the error code and the kernel returns normally.
 __global__ void bounded_wait_selftest_kernel(int* err, uint64_t limit_ns) {
+  griddep_sync();
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
@@ -749,8 +747,7 @@ __global__ void bounded_wait_selftest_kernel(int* err, uint64_t limit_ns) {
   }
 }
 cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
-  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit_ns);
-  return cudaGetLastError();
+  return launch_k(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0, st, err, limit_ns);
 }
 
 // ---------------------------------------------------------------- explicit instantiations

@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(128, 1)
 
   if (nck <= 0) {
     // this split sees no key of the tile: an empty partial (weight 0 in the merge)
+    griddep_sync();
     if (qrow < p.n_q) {
       float* po = p.part_o + (((size_t)sp * p.nq + h) * p.n_q + qrow) * AT_D;
       for (int i = 0; i < AT_D; ++i) po[i] = 0.0f;
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_sync();  // the previous kernel wrote q and this layer's canvas K/V
   const uint32_t tmem_S = tmem_base_s;
   const uint32_t tmem_O = tmem_base_s + 128;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(128, 1)
 
 __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_splits,
                                   int nq, int n_q, int d, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
+  griddep_sync();
   const int qrow = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
   float mx = -INFINITY;
   for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, part_lse[((size_t)s * nq + h) * n_q + qrow]);
@@ -323,14 +326,12 @@ cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& K, cons
   cudaError_t e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((p.n_q + AT_BQ - 1) / AT_BQ, p.nq, p.n_splits);
-  tc_attn_kernel<<<grid, 128, AT_SMEM, st>>>(Q, K, Vt, p);
-  return cudaGetLastError();
+  return launch_k(tc_attn_kernel, dim3(grid), dim3(128), AT_SMEM, st, Q, K, Vt, p);
 }
 
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
-  attn_merge_kernel<<<dim3(n_q, nq), 128, 0, st>>>(part_o, part_lse, n_splits, nq, n_q, d, out, out_lo);
-  return cudaGetLastError();
+  return launch_k(attn_merge_kernel, dim3(n_q, nq), dim3(128), 0, st, part_o, part_lse, n_splits, nq, n_q, d, out, out_lo);
 }
 
 }  // namespace dg

@@ -13,6 +13,10 @@
 // Options: two_terms (tokens given as bf16 hi + lo, both accumulated: fp32-precision
 // activations against bf16 weights); dual_a (gate and up weight tiles accumulated
 // into two TMEM regions, SwiGLU epilogue); k_splits (split-K, one output slab per split).
+//
+// Each tile starts its K walk at a different k-block (tile index mod k-blocks): tiles
+// that run at the same time then read different k-blocks of the token operand, which
+// all of them share, instead of hammering the same L2 lines in lockstep.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -20,7 +24,8 @@ namespace dg {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
-constexpr int TC_B_BOX = 16;
+constexpr int TC_B_BOX = 16;      // token rows per small TMA box
+constexpr int TC_B_BOX_BIG = 64;  // token rows per large TMA box
 constexpr int TC_MAX_STAGES = 16;
 constexpr int TC_THREADS = 192;
 
@@ -59,6 +64,7 @@ template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmBb, const __grid_constant__ CUtensorMap tmB2b,
                    const TcGemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_MAX_STAGES];
@@ -104,6 +110,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  griddep_sync();  // the work list and the token operand come from the previous kernels
   const int n_tiles = total_items(p) * p.m_tiles;
 
   if (warp == 0) {
@@ -112,7 +119,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       prefetch_tmap(&tmA);
       if (p.dual_a) prefetch_tmap(&tmA2);
       prefetch_tmap(&tmB);
-      if (terms == 2) prefetch_tmap(&tmB2);
+      prefetch_tmap(&tmBb);
+      if (terms == 2) {
+        prefetch_tmap(&tmB2);
+        prefetch_tmap(&tmB2b);
+      }
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
@@ -128,11 +139,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           uint8_t* sa = smem + (size_t)s * stage_bytes;
           uint8_t* sb = sa + n_a * a_bytes;
-          const int kx = (ti.split * nkb + kb) * TC_BK;
+          const int kx = (ti.split * nkb + (kb + t) % nkb) * TC_BK;
           mbar_arrive_expect_tx(&full_bar[s], tx);
           tma_load_3d(sa, &tmA, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
           if (p.dual_a) tma_load_3d(sa + a_bytes, &tmA2, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
-          for (int r = 0; r < n_pad; r += TC_B_BOX) {
+          int r = 0;
+          for (; r + TC_B_BOX_BIG <= n_pad; r += TC_B_BOX_BIG) {
+            tma_load_2d(sb + r * 128, &tmBb, kx, ti.row0 + r, &full_bar[s]);
+            if (terms == 2) tma_load_2d(sb + bmax_bytes + r * 128, &tmB2b, kx, ti.row0 + r, &full_bar[s]);
+          }
+          for (; r < n_pad; r += TC_B_BOX) {
             tma_load_2d(sb + r * 128, &tmB, kx, ti.row0 + r, &full_bar[s]);
             if (terms == 2) tma_load_2d(sb + bmax_bytes + r * 128, &tmB2, kx, ti.row0 + r, &full_bar[s]);
           }
@@ -273,13 +289,13 @@ static __device__ void emit_work_items(const int32_t* off, int E, int n_max, TcW
 }
 
 __global__ void build_items_kernel(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items) {
+  griddep_sync();
   if (threadIdx.x == 0 && blockIdx.x == 0) emit_work_items(off, E, n_max, items, n_items);
 }
 
 cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
                                cudaStream_t st) {
-  build_items_kernel<<<1, 32, 0, st>>>(off, E, n_max, items, n_items);
-  return cudaGetLastError();
+  return launch_k(build_items_kernel, dim3(1), dim3(32), 0, st, off, E, n_max, items, n_items);
 }
 
 static int g_num_sms = 0;
@@ -295,7 +311,8 @@ int num_sms() {
 }
 
 cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
-                           const CUtensorMap& B2, const TcGemmParams& p, int max_tiles, cudaStream_t st) {
+                           const CUtensorMap& B2, const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p,
+                           int max_tiles, cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
   if (p.k_splits < 1 || (p.K / TC_BK) % p.k_splits != 0 || (p.k_splits > 1 && p.items) || p.n_max < 16 ||
       p.n_max > 256 || (p.n_max % 16) != 0 || p.m_tiles < 1)
@@ -312,13 +329,13 @@ cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2,
     case EPI_STORE_F32:
       e = cudaFuncSetAttribute(tc_gemm_kernel<EPI_STORE_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
-      tc_gemm_kernel<EPI_STORE_F32><<<grid, TC_THREADS, smem, st>>>(A, A2, B, B2, p);
-      break;
+      return launch_k(tc_gemm_kernel<EPI_STORE_F32>, dim3(grid), dim3(TC_THREADS), smem, st, A, A2, B, B2, Bb,
+                      B2b, p);
     case EPI_SWIGLU_BF16:
       e = cudaFuncSetAttribute(tc_gemm_kernel<EPI_SWIGLU_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
-      tc_gemm_kernel<EPI_SWIGLU_BF16><<<grid, TC_THREADS, smem, st>>>(A, A2, B, B2, p);
-      break;
+      return launch_k(tc_gemm_kernel<EPI_SWIGLU_BF16>, dim3(grid), dim3(TC_THREADS), smem, st, A, A2, B, B2, Bb,
+                      B2b, p);
     default:
       return cudaErrorInvalidValue;
   }
