@@ -377,12 +377,14 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   return DG_OK;
 }
 
+// split-KV factor: one wave of CTAs (the attention kernel holds a whole SM), at least two
+// 128-key chunks per CTA
 int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
   const int nch = ceil_div(n_keys, 128);
   const int base = ceil_div(n_q, 128) * nq;
-  int splits = ceil_div(2 * 148, base);
+  int splits = dg::num_sms() / base;
   if (splits > kMaxAttnSplits) splits = kMaxAttnSplits;
-  if (splits > ceil_div(nch, 2)) splits = ceil_div(nch, 2);
+  if (splits > nch / 2) splits = nch / 2;
   if (splits < 1) splits = 1;
   *chunks_per_split = ceil_div(nch, splits);
   splits = ceil_div(nch, *chunks_per_split);
