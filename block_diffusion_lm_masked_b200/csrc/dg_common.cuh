@@ -21,6 +21,7 @@
 #define DG_DEVERR_TIMEOUT_ATTN 4
 #define DG_DEVERR_BAD_COUNT 5
 #define DG_DEVERR_BAD_TOKEN 6
+#define DG_DEVERR_TIMEOUT_PART 7
 
 namespace dg {
 

@@ -39,6 +39,12 @@ struct TcGemmParams {
   int ld_out;            // elements per output row
   int smem_budget;       // bytes for pipeline stages
   int* err;              // device error word
+  // stream-K scratch (null: one tile per CTA and turn): one parked fp32 partial of
+  // 128 x n_max (x2 with dual_a) floats and one flag per CTA; flags hold the epoch of the
+  // launch that last raised them (zero-initialised once, epochs increase per launch)
+  float* sk_part;
+  int* sk_flag;
+  int sk_epoch;
 };
 
 // grid = min(max_tiles, SMs); max_tiles bounds the tile count (exact for dense GEMMs)

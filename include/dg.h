@@ -105,8 +105,9 @@ dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** 
 void dg_model_destroy(dg_model* m);
 
 /* Bytes of device workspace for calls on up to max_tokens tokens per call (canvas or
- * prefill length).  The caller allocates it (256-byte aligned) and passes it to every
- * call; its first 4 bytes are the device error word (zero it once after allocating). */
+ * prefill length).  The caller allocates it (256-byte aligned), zero-fills it once, and
+ * passes it to every call; its first 4 bytes are the device error word.  Calls that
+ * share a workspace must be ordered on one stream (they reuse its buffers). */
 size_t dg_workspace_bytes(const dg_config* cfg, int32_t max_tokens);
 /* Workspace bytes dg_canvas_update needs on its own for a C x V logits matrix. */
 size_t dg_update_workspace_bytes(int32_t C, int32_t V);

@@ -35,11 +35,13 @@ Precision model.  The pages fix no precision beyond bf16 weights, so the oracle
 follows the kernel's storage precision, because later integer decisions (routing,
 argmax, re-noise set) depend on it and both sides must take them at the same
 precision.  The fp32 model computes everything in float64 here.  A bf16 model
-stores its weights, its KV cache and the attention query operand in bf16 and hands
-every other activation to its GEMMs at fp32 precision (the CUDA path carries it as
-two bf16 terms, ~16 significant bits, which this float64 reference treats as
-exact); the input of the vocabulary projection is a single bf16 term.  So
-`Precision('bf16')` rounds (round-to-nearest-even) exactly at post-RoPE q/k, v,
+stores its weights and its KV cache in bf16; everything in flight -- the
+activations handed to GEMMs, the query, and the K/V of the tokens the call itself
+processes (the canvas in a denoising pass, the new tokens in a prefill) -- stays at
+fp32 precision (the CUDA path carries such values as two bf16 terms, ~16
+significant bits, which this float64 reference treats as exact); the input of the
+vocabulary projection is a single bf16 term.  So `Precision('bf16')` rounds
+(round-to-nearest-even) exactly where a value is stored: K/V written to the cache,
 and the final normed hidden state.  Everything else stays float64.
 """
 from __future__ import annotations
@@ -69,7 +71,7 @@ class Precision:
         self.dtype = dtype
 
     def store(self, x: np.ndarray) -> np.ndarray:
-        """A value stored in the model's storage dtype (KV cache, query operand, vocabulary input)."""
+        """A value stored in the model's storage dtype (KV cache entries, vocabulary input)."""
         return round_bf16(x) if self.dtype == "bf16" else x
 
 
@@ -200,9 +202,8 @@ def _qkv(model, l: int, x: np.ndarray, positions: np.ndarray, prec: Precision):
     q = (xn @ widen(L["w_q"]).T).reshape(T, nq, d).transpose(1, 0, 2)
     k = (xn @ widen(L["w_k"]).T).reshape(T, nkv, d).transpose(1, 0, 2)
     v = (xn @ widen(L["w_v"]).T).reshape(T, nkv, d).transpose(1, 0, 2)
-    q = prec.store(rope(q, positions, cfg["rope_theta"]))
-    k = prec.store(rope(k, positions, cfg["rope_theta"]))
-    v = prec.store(v)
+    q = rope(q, positions, cfg["rope_theta"])
+    k = rope(k, positions, cfg["rope_theta"])
     return q, k, v
 
 
@@ -316,7 +317,7 @@ def denoise_pass(model, cache: Cache, canvas: np.ndarray, prec: Precision, logit
     for l in range(cfg["n_layers"]):
         tap = {"x_in": x.copy()}
         q, k, v = _qkv(model, l, x, pos, prec)
-        kk = np.concatenate([cache.k[l], k], axis=1)
+        kk = np.concatenate([cache.k[l], k], axis=1)   # cached prefix (stored) + canvas (in flight)
         vv = np.concatenate([cache.v[l], v], axis=1)
         o = attention(q, kk, vv, mask)
         tap["attn_o"] = o.transpose(1, 0, 2).reshape(C, -1)
@@ -345,11 +346,11 @@ def prefill_append(model, cache: Cache, tokens: np.ndarray, prec: Precision, tap
     mask = causal_rows(P, T)
     for l in range(cfg["n_layers"]):
         q, k, v = _qkv(model, l, x, pos, prec)
-        out.k[l] = np.concatenate([cache.k[l], k], axis=1)
-        out.v[l] = np.concatenate([cache.v[l], v], axis=1)
+        out.k[l] = np.concatenate([cache.k[l], prec.store(k)], axis=1)   # what later calls read
+        out.v[l] = np.concatenate([cache.v[l], prec.store(v)], axis=1)
         if l == cfg["n_layers"] - 1:
             break
-        o = attention(q, out.k[l], out.v[l], mask)
+        o = attention(q, np.concatenate([cache.k[l], k], axis=1), np.concatenate([cache.v[l], v], axis=1), mask)
         x = x + _attn_out(model, l, o, prec)
         tap = {} if taps is not None else None
         x = x + moe(model, l, x, prec, tap)
@@ -374,9 +375,12 @@ def full_sequence_states(model, prefix_tokens: np.ndarray, canvas: np.ndarray, p
     ks, vs = [], []
     for l in range(cfg["n_layers"]):
         q, k, v = _qkv(model, l, x, pos, prec)
-        ks.append(k)
-        vs.append(v)
-        o = attention(q, k, v, mask)
+        ks.append(prec.store(k))
+        vs.append(prec.store(v))
+        # prefix keys as the cache holds them; block keys in flight
+        kk = np.concatenate([prec.store(k[:, :P]), k[:, P:]], axis=1)
+        vv = np.concatenate([prec.store(v[:, :P]), v[:, P:]], axis=1)
+        o = attention(q, kk, vv, mask)
         x = x + _attn_out(model, l, o, prec)
         x = x + moe(model, l, x, prec)
     return ks, vs, vocab_logits(model, x[P:], prec)

@@ -20,8 +20,8 @@ def _bf(*shape, scale=1.0, gen=None):
     return (torch.randn(*shape, generator=gen, device="cuda") * scale).to(torch.bfloat16)
 
 
-def _scratch(rows, groups):
-    return torch.zeros(16 * (rows + groups + 1) + 64, dtype=torch.uint8, device="cuda")
+def _scratch(dg, rows, groups):
+    return dg.debug_gemm_scratch(rows, groups)
 
 
 @pytest.mark.parametrize("M,K,n", [(128, 64, 1), (256, 128, 16), (384, 512, 100), (128, 2048, 256), (256, 256, 300),
@@ -31,7 +31,7 @@ def test_dense_gemm_store(dg, M, K, n):
     W, X = _bf(1, M, K, gen=g), _bf(n, K, gen=g)
     out = torch.full((n, M), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dg.debug_gemm_bf16(W, X, out, M, err, _scratch(n, 1))
+    dg.debug_gemm_bf16(W, X, out, M, err, _scratch(dg, n, 1))
     torch.cuda.synchronize()
     ref = X.float() @ W[0].float().T
     assert err.item() == 0
@@ -48,7 +48,7 @@ def test_two_term_gemm_is_fp32_accurate(dg):
     lo = (Xf - hi.float()).to(torch.bfloat16)
     out = torch.full((n, M), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dg.debug_gemm_bf16(W, hi, out, M, err, _scratch(n, 1), X_lo=lo)
+    dg.debug_gemm_bf16(W, hi, out, M, err, _scratch(dg, n, 1), X_lo=lo)
     torch.cuda.synchronize()
     ref = (Xf.double() @ W[0].double().T).float()
     single = hi.float() @ W[0].float().T
@@ -71,7 +71,7 @@ def test_grouped_gemm(dg, counts, M):
     W, X = _bf(E, M, K, gen=g), _bf(rows, K, gen=g)
     out = torch.full((rows, M), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dg.debug_gemm_bf16(W, X, out, M, err, _scratch(rows, E), group_off=off)
+    dg.debug_gemm_bf16(W, X, out, M, err, _scratch(dg, rows, E), group_off=off)
     torch.cuda.synchronize()
     assert err.item() == 0
     ref = torch.empty_like(out)
@@ -79,6 +79,39 @@ def test_grouped_gemm(dg, counts, M):
     for e in range(E):
         ref[o[e]:o[e + 1]] = X[o[e]:o[e + 1]].float() @ W[e].float().T
     torch.testing.assert_close(out, ref, rtol=1e-4, atol=1e-3 * ref.abs().max().item())
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_stream_k_matches_one_tile_per_cta(dg, swiglu):
+    """Enough tiles for the stream-K split (cut tiles finished from a parked partial):
+    the result equals the one-tile-per-CTA schedule to fp32 rounding, and both match torch."""
+    g = torch.Generator(device="cuda").manual_seed(21)
+    counts = [37, 0, 64, 5, 90, 130, 16, 1] * 8
+    E, F, K = len(counts), 704, 512
+    off, rows = _groups(counts)
+    W = _bf(E, F, K, scale=0.1, gen=g)
+    W2 = _bf(E, F, K, scale=0.1, gen=g) if swiglu else None
+    X = _bf(rows, K, gen=g)
+    outs = []
+    for sk in (True, False):
+        if swiglu:
+            o = torch.zeros(rows, F, dtype=torch.bfloat16, device="cuda")
+            olo = torch.zeros(rows, F, dtype=torch.bfloat16, device="cuda")
+        else:
+            o, olo = torch.zeros(rows, F, device="cuda"), None
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        dg.debug_gemm_bf16(W, X, o, F, err, _scratch(dg, rows, E), W2=W2, group_off=off, out_lo=olo, streamk=sk)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        outs.append(o.double() + (olo.double() if olo is not None else 0))
+    ref = torch.empty(rows, F, dtype=torch.float64, device="cuda")
+    o = off.cpu().numpy()
+    for e in range(E):
+        a = X[o[e]:o[e + 1]].double() @ W[e].double().T
+        ref[o[e]:o[e + 1]] = torch.nn.functional.silu(a) * (X[o[e]:o[e + 1]].double() @ W2[e].double().T) if swiglu else a
+    scale = ref.abs().max().item()
+    torch.testing.assert_close(outs[0], outs[1], rtol=1e-5, atol=1e-6 * scale)
+    torch.testing.assert_close(outs[0], ref, rtol=1e-4, atol=1e-5 * scale)
 
 
 @pytest.mark.parametrize("F", [128, 704])
@@ -93,7 +126,7 @@ def test_gate_up_swiglu_epilogue(dg, F):
     h = torch.zeros(rows, F, dtype=torch.bfloat16, device="cuda")
     h_lo = torch.zeros(rows, F, dtype=torch.bfloat16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dg.debug_gemm_bf16(gate, X, h, F, err, _scratch(rows, E), W2=up, X_lo=X_lo, group_off=off, out_lo=h_lo)
+    dg.debug_gemm_bf16(gate, X, h, F, err, _scratch(dg, rows, E), W2=up, X_lo=X_lo, group_off=off, out_lo=h_lo)
     torch.cuda.synchronize()
     assert err.item() == 0
     o = off.cpu().numpy()
