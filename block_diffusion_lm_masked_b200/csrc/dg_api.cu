@@ -242,8 +242,9 @@ constexpr int kSkFlagBytes = 4096;                 // stream-K flags (one int pe
 constexpr size_t kSkSlotFloats = 128 * 256;        // largest parked partial: 128 x n_max (x2 dual)
 
 struct WsLayout {
-  size_t err, sk_flag, upd, x, xn, xn_lo, qkv, q, o, o_lo, part_o, part_lse, opart, topk_idx, topk_w, counts, offsets,
-      perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, sk_part, total;
+  size_t err, sk_flag, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
+      topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, sk_part, total;
+  int lo_rows;  // rows of the current-token K/V low-term window
 };
 
 size_t upd_bytes(int C, int V) { return al((size_t)C * dg::update_splits(C, V) * sizeof(dg::UpdPart)); }
@@ -269,6 +270,10 @@ WsLayout layout(const dg_config& c, int T) {
   L.xn_lo = take(bf ? (size_t)T * H * 2 : 0);
   L.qkv = take((size_t)(bf ? kMaxKsQkv : 1) * T * qkv_rows(c) * 4);
   L.q = take((size_t)c.n_q_heads * T * d * ab);
+  L.lo_rows = ((T + 127) / 128) * 128 + 128;
+  L.q_lo = take(bf ? (size_t)c.n_q_heads * T * d * 2 : 0);
+  L.k_lo = take(bf ? (size_t)c.n_kv_heads * L.lo_rows * d * 2 : 0);
+  L.vt_lo = take(bf ? (size_t)c.n_kv_heads * L.lo_rows * d * 2 : 0);
   L.o = take((size_t)T * c.n_q_heads * d * ab);
   L.o_lo = take(bf ? (size_t)T * c.n_q_heads * d * 2 : 0);
   L.part_o = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
@@ -417,13 +422,16 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
                                          n_keys, causal, nq, nkv, d, ws.at<float>(ws.L.o), st));
     return DG_OK;
   }
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mql, mk, mv, mkl, mvl;
   dg_status s;
+  const int base = (pos0 / 128) * 128;  // the low-term window starts at this chunk
+  const int Lc = ws.L.lo_rows;
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)n_q * d * 2};
     const uint32_t box[3] = {64, 128, 1};
     if ((s = encode_bf16(&mq, ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&mql, ws.at<void>(ws.L.q_lo), 3, dims, str, box)) != DG_OK) return s;
   }
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
@@ -437,6 +445,18 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
     const uint32_t box[3] = {64, 128, 1};
     if ((s = encode_bf16(&mv, vtc, 3, dims, str, box)) != DG_OK) return s;
   }
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)(n_keys - base), (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)Lc * d * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mkl, ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)(n_keys - base), (uint64_t)d, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)Lc * 2, (uint64_t)d * Lc * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mvl, ws.at<void>(ws.L.vt_lo), 3, dims, str, box)) != DG_OK) return s;
+  }
   dg::TcAttnParams p;
   p.n_q = n_q;
   p.q_pos0 = pos0;
@@ -446,12 +466,14 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
   p.nq = nq;
   p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  p.has_lo = 1;
+  p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
   p.part_o = ws.at<float>(ws.L.part_o);
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
-  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mq, mk, mv, p, st));
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mq, mql, mk, mv, mkl, mvl, p, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
            dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),
@@ -489,7 +511,9 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   }
   LAUNCH(DG_K_ROPE_KV, st,
          dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), ks_qkv, (size_t)n * QR, n, nq, nkv, d, pos0, c.rope_theta,
-                                    ws.at<T>(ws.L.q), (T*)kc, (T*)vtc, cap, st));
+                                    ws.at<T>(ws.L.q), (T*)kc, (T*)vtc, cap, bf ? ws.at<T>(ws.L.q_lo) : nullptr,
+                                    bf ? ws.at<T>(ws.L.k_lo) : nullptr, bf ? ws.at<T>(ws.L.vt_lo) : nullptr,
+                                    (pos0 / 128) * 128, ws.L.lo_rows, st));
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
@@ -856,8 +880,12 @@ extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const
   dg_status s = check_ws(c, d_ws, ws_bytes, n_q, &ws);
   if (s != DG_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // the pass reads q from the workspace's q buffer and writes o to its o buffer
+  // the pass reads q from the workspace's q buffer and writes o to its o buffer; the low
+  // terms of q and of the current K/V are zero here (all inputs are bf16 already)
   cudaError_t e = cudaMemcpyAsync(ws.at<void>(ws.L.q), q, (size_t)nq * n_q * 128 * 2, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.q_lo), 0, (size_t)nq * n_q * 128 * 2, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.k_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.vt_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy q: %s", cudaGetErrorString(e));
   if ((s = attention(c, ws, const_cast<void*>(k), const_cast<void*>(vt), cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
     return s;

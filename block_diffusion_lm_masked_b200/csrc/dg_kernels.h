@@ -68,13 +68,18 @@ struct TcAttnParams {
   int chunks_per_split;
   int n_splits;
   float scale_log2;    // log2(e) / sqrt(d)
+  int has_lo;          // query and current K/V carry low terms (bf16 model)
+  int base;            // 128-aligned start of the low-term window (<= q_pos0)
   __nv_bfloat16* out;     // [n_q][nq * 128] when n_splits == 1 (hi part)
   __nv_bfloat16* out_lo;  // lo part, or null
   float* part_o;       // [n_splits][nq][n_q][128]
   float* part_lse;     // [n_splits][nq][n_q], log2 domain
   int* err;
 };
-cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& K, const CUtensorMap& Vt,
+// Q / Ql: query hi / lo [nq][n_q][128]; K / Vt: the cache; Kl / Vtl: low terms of the
+// current K/V, rows (keys) counted from `base`
+cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
+                                const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
                                 const TcAttnParams& p, cudaStream_t st);
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
@@ -85,9 +90,13 @@ cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_
 template <typename T>
 cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int V, int H, float eps, float* x, T* xn,
                               T* xn_lo, int* err, cudaStream_t st);
+// q / K / V^T hi parts (the cache holds K and V^T); with q_lo set (bf16 model) also the
+// low parts: q_lo like q, k_lo [nkv][lo_rows][d] and vt_lo [nkv][d][lo_rows] at row
+// (position - lo_base), rows [0, pos0 - lo_base) zeroed
 template <typename T>
 cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
-                                int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, cudaStream_t st);
+                                int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
+                                T* vt_lo, int lo_base, int lo_rows, cudaStream_t st);
 cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, const int* group_off, int n_groups,
                                  int max_rows_per_group, int n_tokens, int M, int K, float* out, int ld_out,
                                  cudaStream_t st);

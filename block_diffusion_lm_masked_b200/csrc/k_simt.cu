@@ -81,7 +81,8 @@ cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int 
 template <typename T>
 __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, size_t part_stride, int nq, int nkv,
                                     int d, int pos0, float theta, int n, T* __restrict__ q, T* __restrict__ kc,
-                                    T* __restrict__ vtc, int cap) {
+                                    T* __restrict__ vtc, int cap, T* __restrict__ q_lo, T* __restrict__ k_lo,
+                                    T* __restrict__ vt_lo, int lo_base, int lo_rows) {
   griddep_sync();
   extern __shared__ float cs[];  // [d/2] cos, [d/2] sin, then the summed qkv row
   const int t = blockIdx.x;
@@ -115,27 +116,48 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, 
     const float c = cs[i], s = cs[half + i];
     const float o1 = x1 * c - x2 * s, o2 = x2 * c + x1 * s;
     if (hh < nq) {
-      T* dst = q + ((size_t)hh * n + t) * d;
-      dst[i] = from_f32<T>(o1);
-      dst[i + half] = from_f32<T>(o2);
+      const size_t o = ((size_t)hh * n + t) * d;
+      store_act(q, q_lo, o + i, o1);
+      store_act(q, q_lo, o + i + half, o2);
     } else {
-      T* dst = kc + ((size_t)(hh - nq) * cap + pos) * d;
-      dst[i] = from_f32<T>(o1);
-      dst[i + half] = from_f32<T>(o2);
+      const int kh = hh - nq;
+      T* dst = kc + ((size_t)kh * cap + pos) * d;
+      const T a = from_f32<T>(o1), b = from_f32<T>(o2);
+      dst[i] = a;
+      dst[i + half] = b;
+      if (k_lo) {
+        T* dl = k_lo + ((size_t)kh * lo_rows + (pos - lo_base)) * d;
+        dl[i] = from_f32<T>(o1 - to_f32(a));
+        dl[i + half] = from_f32<T>(o2 - to_f32(b));
+      }
     }
   }
   for (int idx = threadIdx.x; idx < nkv * d; idx += blockDim.x) {
     const int hh = idx / d, dd = idx % d;
-    vtc[((size_t)hh * d + dd) * cap + pos] = from_f32<T>(row[(nq + nkv) * d + idx]);
+    const float v = row[(nq + nkv) * d + idx];
+    const T a = from_f32<T>(v);
+    vtc[((size_t)hh * d + dd) * cap + pos] = a;
+    if (vt_lo) vt_lo[((size_t)hh * d + dd) * lo_rows + (pos - lo_base)] = from_f32<T>(v - to_f32(a));
+  }
+  // the window rows before the first current position hold cached keys: no low part
+  if (k_lo) {
+    for (int r = t; r < pos0 - lo_base; r += n)
+      for (int idx = threadIdx.x; idx < nkv * d; idx += blockDim.x) {
+        const int hh = idx / d, dd = idx % d;
+        k_lo[((size_t)hh * lo_rows + r) * d + dd] = from_f32<T>(0.0f);
+        vt_lo[((size_t)hh * d + dd) * lo_rows + r] = from_f32<T>(0.0f);
+      }
   }
 }
 
 template <typename T>
 cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
-                                int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, cudaStream_t st) {
+                                int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
+                                T* vt_lo, int lo_base, int lo_rows, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const size_t smem = (size_t)(d + (nq + 2 * nkv) * d) * sizeof(float);
-  return launch_k(rope_scatter_kernel<T>, dim3(n), dim3(256), smem, st, qkv, n_parts, part_stride, nq, nkv, d, pos0, theta, n, q, kcache, vtcache, cap);
+  return launch_k(rope_scatter_kernel<T>, dim3(n), dim3(256), smem, st, qkv, n_parts, part_stride, nq, nkv, d, pos0,
+                  theta, n, q, kcache, vtcache, cap, q_lo, k_lo, vt_lo, lo_base, lo_rows);
 }
 
 // ---------------------------------------------------------------- fp32 GEMM (fp32 model)
@@ -755,7 +777,7 @@ cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream
   template cudaError_t launch_embed_norm<T>(const int32_t*, const T*, int, int, int, float, float*, T*, T*, int*, \
                                             cudaStream_t);                                                        \
   template cudaError_t launch_rope_scatter<T>(const float*, int, size_t, int, int, int, int, int, float, T*, T*,  \
-                                              T*, int, cudaStream_t);                                             \
+                                              T*, int, T*, T*, T*, int, int, cudaStream_t);                       \
   template cudaError_t launch_router_fused<T>(float*, const float*, int, size_t, const float*, int, int, int, int, \
                                               float, float*, int32_t*, float*, T*, T*, cudaStream_t);             \
   template cudaError_t launch_gather_rows<T>(const T*, const T*, const int32_t*, int, int, int, T*, T*,          \

@@ -3,16 +3,23 @@
 //                   keys (bidirectional block rows of the prefix/block mask);
 //   prefill mode:   new tokens see keys up to their own position (causal rows).
 // One CTA = one query head x 128 query rows x a contiguous range of 128-key chunks
-// (split-KV; partial results merged by attn_merge_kernel).  S = Q K^T and
-// O += P V both run on the tensor core with fp32 accumulators in TMEM (S: columns
-// 0..127, O: columns 128..255); softmax runs one query row per thread.  V is kept
-// transposed in the cache ([d][position]) so both MMAs read K-major operands.
-// The running max is only raised when it grows by more than 2^8 (log2 domain), so
-// O in TMEM is rescaled rarely; P and l use the same (possibly stale) max, which
-// leaves O / l exact.  P is carried as two bf16 terms, hi = bf16(p) and
-// lo = bf16(p - hi), and O accumulates hi V + lo V: the probabilities keep about 16
-// significant bits instead of 8, which keeps the attention output within a few
-// fp32-accumulation ulps of exact softmax attention.
+// (split-KV; partial results merged by attn_merge_kernel).  V is kept transposed in the
+// cache ([d][position]) so the B operands of both MMAs are K-major in shared memory.
+//
+// Precision.  Cached keys/values are bf16 (the cache's storage format).  The query and
+// the keys/values of the tokens the call itself processes are in flight at fp32
+// precision, carried as bf16 hi + lo terms: S = Q_hi K^T + Q_lo K^T (+ Q_hi K_lo^T on
+// the chunks holding current tokens), O += P_hi V + P_lo V (+ P_hi V_lo on those
+// chunks).  The low parts of the current K/V live in a workspace window whose row 0 is
+// the 128-aligned chunk start `base` at or below the first current position; rows
+// before the first current position are zero there.
+//
+// Pipeline.  S (fp32) sits in TMEM columns 0..127; the softmax (one query row per
+// thread, max raised lazily by more than 2^8 so O is rescaled rarely) writes P as
+// packed bf16 pairs into TMEM columns 128..191 (hi) and 192..255 (lo), and the PV MMAs
+// read P from TMEM; O accumulates in columns 256..383.  Chunks of cached keys alternate
+// between two 64 KB smem slots (the next one loads while this one is used); a chunk of
+// current tokens takes both slots (hi K/V in one, lo in the other).
 #include <math.h>
 
 #include "dg_common.cuh"
@@ -23,12 +30,27 @@ namespace dg {
 constexpr int AT_BQ = 128;
 constexpr int AT_BKEYS = 128;
 constexpr int AT_D = 128;
-constexpr uint32_t AT_HALF = 128 * 128;  // one [128 rows][64 bf16] swizzled block: 16 KB
-constexpr int AT_SMEM = 1024 + 14 * AT_HALF;  // Q (2 blocks), K[2] (4), Vt[2] (4), P hi (2), P lo (2)
+constexpr uint32_t AT_HALF = 128 * 128;                   // one [128 rows][64 bf16] swizzled block
+constexpr uint32_t AT_SLOT = 4 * AT_HALF;                 // K (2 blocks) + V^T (2 blocks)
+constexpr int AT_SMEM = 1024 + 4 * AT_HALF + 2 * AT_SLOT;  // Q hi, Q lo, two slots
+constexpr uint32_t TM_S = 0, TM_PHI = 128, TM_PLO = 192, TM_O = 256;
+
+// A operand from TMEM (P), B from shared memory (V^T), fp32 accumulate in TMEM
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 __global__ void __launch_bounds__(128, 1)
-    tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmVt, const TcAttnParams p) {
+    tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
+                   const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
+                   const TcAttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_bar;
   __shared__ __align__(8) uint64_t kv_bar[2];
@@ -37,7 +59,6 @@ __global__ void __launch_bounds__(128, 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
-  __shared__ int kv_issued_s, kv_consumed_s, q_consumed_s;
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int qt = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
@@ -64,13 +85,11 @@ __global__ void __launch_bounds__(128, 1)
   }
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                    // 2 blocks: d 0..63, d 64..127
-  uint8_t* sK = smem + 2 * AT_HALF;      // [buf][2 blocks]
-  uint8_t* sV = smem + 6 * AT_HALF;      // [buf][2 blocks]: V^T rows = d, K = keys 0..63 / 64..127
-  uint8_t* sP = smem + 10 * AT_HALF;     // P hi, 2 blocks: keys 0..63, 64..127
-  uint8_t* sPl = smem + 12 * AT_HALF;    // P lo, same layout
+  uint8_t* sQ = smem;                   // 2 blocks: d 0..63, 64..127
+  uint8_t* sQl = smem + 2 * AT_HALF;    // low terms
+  uint8_t* sSlot = smem + 4 * AT_HALF;  // [2 slots][K blk0, K blk1, Vt blk0, Vt blk1]
 
-  if (warp == 0) tmem_alloc(&tmem_base_s, 256);
+  if (warp == 0) tmem_alloc(&tmem_base_s, 512);
   if (tid == 32) {
     mbar_init(&q_bar, 1);
     mbar_init(&kv_bar[0], 1);
@@ -79,39 +98,63 @@ __global__ void __launch_bounds__(128, 1)
     mbar_init(&pv_bar, 1);
     mbar_init(&drain_bar, 1);
     abort_s = 0;
-    kv_issued_s = 0;
-    kv_consumed_s = 0;
-    q_consumed_s = 0;
     fence_barrier_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_sync();  // the previous kernel wrote q and this layer's canvas K/V
-  const uint32_t tmem_S = tmem_base_s;
-  const uint32_t tmem_O = tmem_base_s + 128;
+  griddep_sync();  // the previous kernel wrote q and this layer's current K/V
+  const uint32_t tmem = tmem_base_s;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  auto load_kv = [&](int buf, int chunk) {
-    const int key0 = chunk * AT_BKEYS;
-    uint8_t* k = sK + buf * 2 * AT_HALF;
-    uint8_t* v = sV + buf * 2 * AT_HALF;
-    mbar_arrive_expect_tx(&kv_bar[buf], 4 * AT_HALF);
-    tma_load_3d(k, &tmK, 0, key0, kvh, &kv_bar[buf]);
-    tma_load_3d(k + AT_HALF, &tmK, 64, key0, kvh, &kv_bar[buf]);
-    tma_load_3d(v, &tmVt, key0, 0, kvh, &kv_bar[buf]);
-    tma_load_3d(v + AT_HALF, &tmVt, key0 + 64, 0, kvh, &kv_bar[buf]);
+  // chunk j (0-based within this CTA) holds keys [key0, key0 + 128); "current" chunks
+  // (key0 >= base) also carry low parts; cached-key chunks alternate slots j & 1
+  auto is_cur = [&](int j) { return p.has_lo && (c_begin + j) * AT_BKEYS >= p.base; };
+
+  // ---- TMA issue bookkeeping (thread 0 only)
+  int slot_loads[2] = {0, 0};  // loads issued into each slot so far
+  int par_ring[2][2] = {{0, 0}, {0, 0}};  // [j & 1][slot]: parity of chunk j's load in that slot
+  int issued = 0;                         // chunks issued so far (in order)
+  auto load_slot = [&](int slot, const CUtensorMap* mk, const CUtensorMap* mv, int krow, int vx) {
+    uint8_t* k = sSlot + slot * AT_SLOT;
+    uint8_t* v = k + 2 * AT_HALF;
+    mbar_arrive_expect_tx(&kv_bar[slot], AT_SLOT);
+    tma_load_3d(k, mk, 0, krow, kvh, &kv_bar[slot]);
+    tma_load_3d(k + AT_HALF, mk, 64, krow, kvh, &kv_bar[slot]);
+    tma_load_3d(v, mv, vx, 0, kvh, &kv_bar[slot]);
+    tma_load_3d(v + AT_HALF, mv, vx + 64, 0, kvh, &kv_bar[slot]);
+  };
+  auto issue = [&](int j) {
+    const int key0 = (c_begin + j) * AT_BKEYS;
+    if (is_cur(j)) {
+      par_ring[j & 1][0] = slot_loads[0]++ & 1;
+      par_ring[j & 1][1] = slot_loads[1]++ & 1;
+      load_slot(0, &tmK, &tmVt, key0, key0);
+      load_slot(1, &tmKl, &tmVtl, key0 - p.base, key0 - p.base);
+    } else {
+      const int s = j & 1;
+      par_ring[j & 1][s] = slot_loads[s]++ & 1;
+      load_slot(s, &tmK, &tmVt, key0, key0);
+    }
+    issued = j + 1;
   };
 
   if (tid == 0) {
     prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmQl);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmVt);
-    mbar_arrive_expect_tx(&q_bar, 2 * AT_HALF);
+    if (p.has_lo) {
+      prefetch_tmap(&tmKl);
+      prefetch_tmap(&tmVtl);
+    }
+    mbar_arrive_expect_tx(&q_bar, 4 * AT_HALF);
     tma_load_3d(sQ, &tmQ, 0, q_row0, h, &q_bar);
     tma_load_3d(sQ + AT_HALF, &tmQ, 64, q_row0, h, &q_bar);
-    for (int i = 0; i < 2 && i < nck; ++i) load_kv(i, c_begin + i);
-    kv_issued_s = min(2, nck);
+    tma_load_3d(sQl, &tmQl, 0, q_row0, h, &q_bar);
+    tma_load_3d(sQl + AT_HALF, &tmQl, 64, q_row0, h, &q_bar);
+    issue(0);
+    if (nck > 1 && !is_cur(0) && !is_cur(1)) issue(1);
   }
 
   const uint32_t idesc = idesc_bf16_f32(AT_BQ, AT_BKEYS);
@@ -119,24 +162,33 @@ __global__ void __launch_bounds__(128, 1)
   const int key_lim = p.causal ? min(p.n_keys, qpos + 1) : p.n_keys;
 
   for (int j = 0; j < nck; ++j) {
-    const int buf = j & 1;
+    const bool cur = is_cur(j);
+    const int s_hi = cur ? 0 : (j & 1);
     if (tid == 0) {
       bool ok = true;
-      if (j == 0) {
-        ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-        if (ok) q_consumed_s = 1;
+      if (issued <= j) {
+        // this chunk needs a slot the previous chunk still used: wait for its PV first
+        if (j > 0) ok = mbar_wait(&pv_bar, (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        if (ok) issue(j);
       }
-      ok = ok && mbar_wait(&kv_bar[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      if (ok && j == 0) ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      if (ok)
+        ok = mbar_wait(&kv_bar[s_hi], (uint32_t)par_ring[j & 1][s_hi], &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      if (ok && cur) ok = mbar_wait(&kv_bar[1], (uint32_t)par_ring[j & 1][1], &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
       if (ok) {
-        kv_consumed_s = j + 1;
         tc_fence_after();
-        const uint32_t q = smem_u32(sQ), k = smem_u32(sK + buf * 2 * AT_HALF);
+        const uint32_t q = smem_u32(sQ), ql = smem_u32(sQl);
+        const uint32_t k = smem_u32(sSlot + s_hi * AT_SLOT), kl = smem_u32(sSlot + AT_SLOT);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma(tmem_S, sw128_kmajor_desc(q + kb * AT_HALF + kk * 32),
-                   sw128_kmajor_desc(k + kb * AT_HALF + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t off = kb * AT_HALF + kk * 32;
+            const uint64_t kd = sw128_kmajor_desc(k + off);
+            tc_mma(tmem + TM_S, sw128_kmajor_desc(q + off), kd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma(tmem + TM_S, sw128_kmajor_desc(ql + off), kd, idesc, 1u);
+            if (cur) tc_mma(tmem + TM_S, sw128_kmajor_desc(q + off), sw128_kmajor_desc(kl + off), idesc, 1u);
+          }
       }
       tc_commit(&s_bar);
     }
@@ -148,7 +200,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
     for (int c = 0; c < AT_BKEYS / 16; ++c) {
       uint32_t r[16];
-      tmem_ld16(tmem_S + lane_off + c * 16, r);
+      tmem_ld16(tmem + TM_S + lane_off + c * 16, r);
       tc_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[i]) * p.scale_log2;
@@ -161,72 +213,66 @@ __global__ void __launch_bounds__(128, 1)
       rmax = fmaxf(rmax, s[i]);
     }
 
-    // PV of the previous chunk done: O is stable, P smem and the other KV buffer are free
+    // PV of the previous chunk done: O is stable, P in TMEM and the previous slot are free
     if (j > 0) mbar_wait(&pv_bar, (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-    if (tid == 0 && j >= 1 && j + 1 < nck && !abort_s) {
-      load_kv((j + 1) & 1, c_begin + j + 1);
-      kv_issued_s = j + 2;
-    }
+    if (tid == 0 && issued == j + 1 && j + 1 < nck && !cur && !is_cur(j + 1) && !abort_s) issue(j + 1);
+
     const bool upd = rmax > m_used + 8.0f;
     const float alpha = upd ? exp2f(m_used - rmax) : 1.0f;  // 0 while nothing was visible yet
     // tcgen05.ld/st are warp-collective: the whole warp rescales if any of its rows must
     if (__any_sync(0xffffffffu, upd && j > 0)) {
-      {
-        tc_fence_after();
+      tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < AT_D / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(tmem_O + lane_off + c * 16, r);
-          tc_wait_ld();
+      for (int c = 0; c < AT_D / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem + TM_O + lane_off + c * 16, r);
+        tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st16(tmem_O + lane_off + c * 16, r);
-        }
-        tc_wait_st();
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        tmem_st16(tmem + TM_O + lane_off + c * 16, r);
       }
     }
     if (upd) {
       l *= alpha;
       m_used = rmax;
     }
-    // P = exp2(s - m_used) as hi + lo bf16 terms, written as K-major A operands of the PV MMAs
+    // P = exp2(s - m_used) as packed bf16 pairs, hi and lo, into TMEM
 #pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      uint8_t* pb = sP + blk * AT_HALF;
-      uint8_t* pl = sPl + blk * AT_HALF;
+    for (int c = 0; c < 4; ++c) {  // 32 keys -> 16 packed columns per store
+      uint32_t wh[16], wl[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t wh[4], wl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = blk * 64 + c * 8 + 2 * e;
-          const float p0 = (s[i0] == -INFINITY) ? 0.0f : exp2f(s[i0] - m_used);
-          const float p1 = (s[i0 + 1] == -INFINITY) ? 0.0f : exp2f(s[i0 + 1] - m_used);
-          l += p0 + p1;
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-          const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
-          wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
-          wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
-        }
-        *reinterpret_cast<uint4*>(pb + sw128_offset(tid, c)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-        *reinterpret_cast<uint4*>(pl + sw128_offset(tid, c)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      for (int e = 0; e < 16; ++e) {
+        const int i0 = c * 32 + 2 * e;
+        const float p0 = (s[i0] == -INFINITY) ? 0.0f : exp2f(s[i0] - m_used);
+        const float p1 = (s[i0 + 1] == -INFINITY) ? 0.0f : exp2f(s[i0 + 1] - m_used);
+        l += p0 + p1;
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
+        wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
+        wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
       }
+      tmem_st16(tmem + TM_PHI + lane_off + c * 16, wh);
+      tmem_st16(tmem + TM_PLO + lane_off + c * 16, wl);
     }
-    fence_proxy_async_smem();
+    tc_wait_st();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       if (!abort_s) {
         tc_fence_after();
-        const uint32_t pp = smem_u32(sP), pl = smem_u32(sPl), v = smem_u32(sV + buf * 2 * AT_HALF);
+        const uint32_t v = smem_u32(sSlot + s_hi * AT_SLOT + 2 * AT_HALF);
+        const uint32_t vl = smem_u32(sSlot + AT_SLOT + 2 * AT_HALF);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t pcol = kb * 32 + kk * 8;  // 16 keys = 8 packed columns
             const uint64_t vd = sw128_kmajor_desc(v + kb * AT_HALF + kk * 32);
-            tc_mma(tmem_O, sw128_kmajor_desc(pp + kb * AT_HALF + kk * 32), vd, idesc,
-                   (j > 0 || (kb | kk) != 0) ? 1u : 0u);
-            tc_mma(tmem_O, sw128_kmajor_desc(pl + kb * AT_HALF + kk * 32), vd, idesc, 1u);
+            tc_mma_ts(tmem + TM_O, tmem + TM_PHI + pcol, vd, idesc, (j > 0 || (kb | kk) != 0) ? 1u : 0u);
+            tc_mma_ts(tmem + TM_O, tmem + TM_PLO + pcol, vd, idesc, 1u);
+            if (cur)
+              tc_mma_ts(tmem + TM_O, tmem + TM_PHI + pcol, sw128_kmajor_desc(vl + kb * AT_HALF + kk * 32), idesc,
+                        1u);
           }
       }
       tc_commit(&pv_bar);
@@ -245,7 +291,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int c = 0; c < AT_D / 16; ++c) {
         uint32_t r[16];
-        tmem_ld16(tmem_O + lane_off + c * 16, r);
+        tmem_ld16(tmem + TM_O + lane_off + c * 16, r);
         tc_wait_ld();
         if (valid) {
           uint32_t w[8], wl[8];
@@ -272,7 +318,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int c = 0; c < AT_D / 16; ++c) {
         uint32_t r[16];
-        tmem_ld16(tmem_O + lane_off + c * 16, r);
+        tmem_ld16(tmem + TM_O + lane_off + c * 16, r);
         tc_wait_ld();
         if (valid) {
           float4* dst = reinterpret_cast<float4*>(po + c * 16);
@@ -286,14 +332,16 @@ __global__ void __launch_bounds__(128, 1)
         p.part_lse[((size_t)sp * p.nq + h) * p.n_q + qrow] = (l > 0.0f) ? m_used + log2f(l) : -INFINITY;
     }
   } else if (tid == 0) {
-    if (!q_consumed_s) mbar_wait_drain(&q_bar, 0);
-    for (int c = kv_consumed_s; c < kv_issued_s; ++c) mbar_wait_drain(&kv_bar[c & 1], (uint32_t)(c >> 1) & 1u);
+    // wind down: let issued loads and MMAs land before the smem / TMEM go away
+    mbar_wait_drain(&q_bar, 0);
+    for (int s2 = 0; s2 < 2; ++s2)
+      if (slot_loads[s2] > 0) mbar_wait_drain(&kv_bar[s2], (uint32_t)(slot_loads[s2] - 1) & 1u);
     tc_commit(&drain_bar);
     mbar_wait_drain(&drain_bar, 0);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem_base_s, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_splits,
@@ -321,17 +369,19 @@ __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float*
   }
 }
 
-cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& K, const CUtensorMap& Vt,
+cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
+                                const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
                                 const TcAttnParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((p.n_q + AT_BQ - 1) / AT_BQ, p.nq, p.n_splits);
-  return launch_k(tc_attn_kernel, dim3(grid), dim3(128), AT_SMEM, st, Q, K, Vt, p);
+  return launch_k(tc_attn_kernel, grid, dim3(128), AT_SMEM, st, Q, Ql, K, Vt, Kl, Vtl, p);
 }
 
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
-  return launch_k(attn_merge_kernel, dim3(n_q, nq), dim3(128), 0, st, part_o, part_lse, n_splits, nq, n_q, d, out, out_lo);
+  return launch_k(attn_merge_kernel, dim3(n_q, nq), dim3(128), 0, st, part_o, part_lse, n_splits, nq, n_q, d, out,
+                  out_lo);
 }
 
 }  // namespace dg
