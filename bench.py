@@ -208,7 +208,7 @@ def main():
 
     # expert union per layer of this input (read once, outside the timed region)
     unions = torch.zeros(cfg["n_layers"], dtype=torch.int32, device=dev)
-    model.set_taps({"unions": unions})
+    model.set_taps({"unions": unions, "rows": C})
     step(0)
     model.set_taps(None)
     torch.cuda.synchronize(dev)

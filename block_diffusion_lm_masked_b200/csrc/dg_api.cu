@@ -161,6 +161,7 @@ struct dg_model {
   std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
   std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
   int32_t* tap_unions = nullptr;
+  int tap_rows = 0;
 };
 
 static bool is_bf16(const dg_config& c) { return c.dtype == DG_DTYPE_BF16; }
@@ -242,8 +243,8 @@ constexpr int kSkFlagBytes = 4096;                 // stream-K flags (one int pe
 constexpr size_t kSkSlotFloats = 128 * 256;        // largest parked partial: 128 x n_max (x2 dual)
 
 struct WsLayout {
-  size_t err, sk_flag, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
-      topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, sk_part, total;
+  size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
+      topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, total;
   int lo_rows;  // rows of the current-token K/V low-term window
 };
 
@@ -261,7 +262,6 @@ WsLayout layout(const dg_config& c, int T) {
   const size_t ab = act_bytes(c);
   const size_t H = c.hidden, k = c.top_k, F = c.expert_ffn, d = c.head_dim, E = c.n_experts;
   L.err = take(256);
-  L.sk_flag = take(kSkFlagBytes);
   size_t upd_max = 0;
   for (int C = 1; C <= T; ++C) upd_max = upd_max > upd_bytes(C, c.vocab) ? upd_max : upd_bytes(C, c.vocab);
   L.upd = take(upd_max);
@@ -294,7 +294,6 @@ WsLayout layout(const dg_config& c, int T) {
   L.h_lo = take(bf ? (size_t)T * k * F * 2 : 0);
   L.gu = take(bf ? 0 : (size_t)T * k * 2 * F * 4);
   L.ys = take((size_t)T * k * H * 4);
-  L.sk_part = take(bf ? (size_t)dg::num_sms() * kSkSlotFloats * 4 : 0);
   L.total = o;
   return L;
 }
@@ -351,7 +350,7 @@ struct GemmCall {
   int k_splits;
   size_t split_stride;
   int smem_budget;
-  float* sk_part;  // stream-K scratch (null: classic schedule)
+  float* sk_part;  // stream-K scratch; null (every pass GEMM): one tile per CTA per turn
   int* sk_flag;
 };
 
@@ -502,7 +501,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
     ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
     GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
                nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm,
-               ws.at<float>(ws.L.sk_part), ws.at<int>(ws.L.sk_flag)};
+               nullptr, nullptr};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_QKV, st,
@@ -520,7 +519,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
     ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
     GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
                n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
-               kSmemGemm, ws.at<float>(ws.L.sk_part), ws.at<int>(ws.L.sk_flag)};
+               kSmemGemm, nullptr, nullptr};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_O, st,
@@ -532,7 +531,8 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
          dg::launch_router_fused<T>(ws.at<float>(ws.L.x), ws.at<float>(ws.L.opart), ks_o, (size_t)n * H, W.w_router,
                                     n, H, E, k, c.rms_eps, nullptr, ws.at<int32_t>(ws.L.topk_idx),
                                     ws.at<float>(ws.L.topk_w), ws.at<T>(ws.L.xn), xn_lo, st));
-  if (m->taps_on && !m->tap_x_attn.empty() && m->tap_x_attn[l])
+  const bool taps = m->taps_on && n <= m->tap_rows;
+  if (taps && !m->tap_x_attn.empty() && m->tap_x_attn[l])
     if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
         cudaSuccess)
       return fail(DG_ERR_CUDA, "tap copy failed");
@@ -552,11 +552,11 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
     const int max_items = n * k / kItemRows + E;
     GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate, &m->maps[l].up, ws.at<void>(ws.L.xs), xs_lo,
                 n * k, H, F, items, n_items, max_items, kItemRows, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
-                kSmemGemm, ws.at<float>(ws.L.sk_part), ws.at<int>(ws.L.sk_flag)};
+                kSmemGemm, nullptr, nullptr};
     if ((s = gemm_bf16(gu, err, st)) != DG_OK) return s;
     GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, nullptr, ws.at<void>(ws.L.h),
                 ws.at<void>(ws.L.h_lo), n * k, F, H, items, n_items, max_items, kItemRows, ws.at<float>(ws.L.ys),
-                nullptr, H, 1, 0, kSmemGemm, ws.at<float>(ws.L.sk_part), ws.at<int>(ws.L.sk_flag)};
+                nullptr, H, 1, 0, kSmemGemm, nullptr, nullptr};
     if ((s = gemm_bf16(dn, err, st)) != DG_OK) return s;
   } else {
     float* g = ws.at<float>(ws.L.gu);
@@ -576,7 +576,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
          dg::launch_combine_norm<T>(ws.at<float>(ws.L.ys), ws.at<int32_t>(ws.L.inv), ws.at<float>(ws.L.topk_w), n, k,
                                     H, c.rms_eps, ws.at<float>(ws.L.x), ws.at<T>(ws.L.xn),
                                     final_layer ? nullptr : xn_lo, st));
-  if (m->taps_on) {
+  if (taps) {
     auto cp = [&](void* dst, const void* src, size_t bytes) {
       return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
     };
@@ -651,11 +651,8 @@ extern "C" dg_status dg_prefill_append(dg_model* m, dg_kv_cache* cache, const in
   Ws ws;
   if ((s = check_ws(m->cfg, d_ws, ws_bytes, T, &ws)) != DG_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool saved = m->taps_on;
-  m->taps_on = false;
   s = is_bf16(m->cfg) ? run_stack<bf16>(m, cache, d_tokens, T, true, ws, st)
                       : run_stack<float>(m, cache, d_tokens, T, true, ws, st);
-  m->taps_on = saved;
   if (s != DG_OK) return s;
   cache->len += T;
   return DG_OK;
@@ -681,7 +678,7 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
   if (is_bf16(c)) {
     GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, C, c.hidden,
                c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm,
-               ws.at<float>(ws.L.sk_part), ws.at<int>(ws.L.sk_flag)};
+               nullptr, nullptr};
     if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_VOCAB, st,
@@ -774,6 +771,7 @@ extern "C" dg_status dg_set_taps(dg_model* m, const dg_taps* t) {
     m->taps_on = false;
     return DG_OK;
   }
+  DG_CHECK_ARG(t->rows >= 0, "taps rows must be >= 0");
   grab(t->x_attn, m->tap_x_attn);
   grab(t->x_out, m->tap_x_out);
   grab(t->topk_w, m->tap_topk_w);
@@ -781,6 +779,7 @@ extern "C" dg_status dg_set_taps(dg_model* m, const dg_taps* t) {
   grab(t->counts, m->tap_counts);
   grab(t->perm, m->tap_perm);
   m->tap_unions = t->unions;
+  m->tap_rows = t->rows;
   m->taps_on = true;
   return DG_OK;
 }

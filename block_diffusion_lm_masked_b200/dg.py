@@ -55,7 +55,7 @@ class Taps(ctypes.Structure):
     _fields_ = [("x_attn", ctypes.POINTER(ctypes.c_void_p)), ("x_out", ctypes.POINTER(ctypes.c_void_p)),
                 ("topk_idx", ctypes.POINTER(ctypes.c_void_p)), ("topk_w", ctypes.POINTER(ctypes.c_void_p)),
                 ("counts", ctypes.POINTER(ctypes.c_void_p)), ("perm", ctypes.POINTER(ctypes.c_void_p)),
-                ("unions", ctypes.c_void_p)]
+                ("unions", ctypes.c_void_p), ("rows", ctypes.c_int32)]
 
 
 def _load():
@@ -160,7 +160,8 @@ class Model:
             self.handle = None
 
     def set_taps(self, taps: dict | None):
-        """taps: name -> list (per layer) of device tensors, 'unions' -> int32 tensor [L]; None turns off."""
+        """taps: name -> list (per layer) of device tensors sized for taps['rows'] tokens,
+        'unions' -> int32 tensor [L]; None turns off.  Calls of more tokens take no taps."""
         if taps is None:
             _check(lib.dg_set_taps(self.handle, None))
             self._taps = None
@@ -176,7 +177,7 @@ class Model:
             return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
 
         t = Taps(arr("x_attn"), arr("x_out"), arr("topk_idx"), arr("topk_w"), arr("counts"), arr("perm"),
-                 taps["unions"].data_ptr() if "unions" in taps else None)
+                 taps["unions"].data_ptr() if "unions" in taps else None, int(taps["rows"]))
         _check(lib.dg_set_taps(self.handle, ctypes.byref(t)))
         self._taps = (taps, keep)
 

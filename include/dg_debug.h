@@ -12,8 +12,10 @@
 extern "C" {
 #endif
 
-/* Per-layer copies taken during dg_denoise_pass.  Each member is a host array of
- * n_layers device pointers (the array itself or any entry may be NULL = not taken).
+/* Per-layer copies taken during dg_denoise_pass and dg_prefill_append, for calls of at
+ * most `rows` tokens (a call with more tokens takes none; C below is the call's token
+ * count).  Each member is a host array of n_layers device pointers (the array itself or
+ * any entry may be NULL = not taken), each sized for `rows` tokens.
  *   x_attn   fp32 [C][H]   residual after the attention block
  *   x_out    fp32 [C][H]   residual after the MoE block
  *   topk_idx int32 [C][k]  routed experts, descending router logit
@@ -29,6 +31,7 @@ typedef struct dg_taps {
   int32_t* const* counts;
   int32_t* const* perm;
   int32_t* unions;
+  int32_t rows;
 } dg_taps;
 
 /* Copy the tap pointers into the model (NULL turns taps off). */

@@ -8,6 +8,8 @@ design notes):
     logit; re-noise: log-confidence distance to the cut);
   * a position exempted that way, and which then actually differs, stays exempt in
     every later comparison of the same pass (its hidden state, logits and token);
+    after a routing difference at a layer before the last, the rest of the pass is
+    checked for structure only (the row's K/V reach every other row);
   * hidden states and logits: max |gpu - oracle| / rms(oracle) <= 2e-2 (bf16) or 1e-4
     (fp32) over the non-exempt rows;
   * canvas tokens: identical wherever the oracle's top-1/top-2 logit margin exceeds 1e-2.
@@ -75,7 +77,7 @@ class Setup:
                  topk_w=[torch.zeros(C, k, device=dev) for _ in range(L)],
                  counts=[torch.zeros(E, dtype=torch.int32, device=dev) for _ in range(L)],
                  perm=[torch.zeros(C * k, dtype=torch.int32, device=dev) for _ in range(L)],
-                 unions=torch.zeros(L, dtype=torch.int32, device=dev))
+                 unions=torch.zeros(L, dtype=torch.int32, device=dev), rows=C)
         self.model.set_taps(t)
         return t
 
@@ -83,29 +85,21 @@ class Setup:
 def compare_pass(cfg, taps_gpu, logits_gpu, taps_o, logits_o, report=None, exempt=None):
     """Layer-by-layer comparison of one pass; returns the set of exempt rows.
 
-    `exempt`: rows already exempt on entry (positions whose input token differs)."""
+    `exempt`: rows already exempt on entry (positions whose input token differs).
+
+    A routing difference allowed at layer l (a near tie) gives that row a different MoE
+    output, and from layer l + 1 on its K/V reach every other row through block
+    attention: the two sides then solve different problems.  The layers after the first
+    such difference are checked for structure only (the GPU's permutation, counts and
+    union consistent with its own routing), and every row of the pass is returned
+    exempt, so that the update is checked for structure only as well."""
     t = tol(cfg)
     k, E = cfg["top_k"], cfg["n_experts"]
     exempt = set() if exempt is None else set(exempt)
+    C = logits_gpu.shape[0]
+    diverged = None   # layer of the first allowed routing difference
     for l, to in enumerate(taps_o):
-        xa = taps_gpu["x_attn"][l].cpu().numpy()
-        e_attn = rel_err(xa, to["x_attn"], exempt)
-        assert e_attn <= t, f"layer {l} attention residual: rel err {e_attn:.3e} > {t}"
         gi = taps_gpu["topk_idx"][l].cpu().numpy()
-        gw = taps_gpu["topk_w"][l].cpu().numpy()
-        oi, ow, om = to["topk_idx"], to["topk_w"], to["router_margin"]
-        for row in range(gi.shape[0]):
-            if row in exempt:
-                continue
-            if set(gi[row].tolist()) != set(oi[row].tolist()):
-                assert om[row] < ROUTE_MARGIN, (
-                    f"layer {l} row {row}: routing {sorted(gi[row])} vs oracle {sorted(oi[row])}, margin {om[row]:.3e}")
-                exempt.add(row)
-                continue
-            # weights per expert
-            gmap = dict(zip(gi[row].tolist(), gw[row].tolist()))
-            for e, w in zip(oi[row].tolist(), ow[row].tolist()):
-                assert abs(gmap[e] - w) <= 10 * t, (l, row, e, gmap[e], w)
         counts = taps_gpu["counts"][l].cpu().numpy()
         assert counts.sum() == gi.shape[0] * k
         np.testing.assert_array_equal(counts, np.bincount(gi.reshape(-1), minlength=E))
@@ -115,6 +109,29 @@ def compare_pass(cfg, taps_gpu, logits_gpu, taps_o, logits_o, report=None, exemp
         want = sorted(range(flat.size), key=lambda a: (int(flat[a]), a))
         np.testing.assert_array_equal(perm, want)
         assert int(taps_gpu["unions"][l].item()) == int((counts > 0).sum())
+        for row in range(gi.shape[0]):
+            assert len(set(gi[row].tolist())) == k and gi[row].min() >= 0 and gi[row].max() < E
+        if diverged is not None:
+            continue
+        xa = taps_gpu["x_attn"][l].cpu().numpy()
+        e_attn = rel_err(xa, to["x_attn"], exempt)
+        assert e_attn <= t, f"layer {l} attention residual: rel err {e_attn:.3e} > {t}"
+        gw = taps_gpu["topk_w"][l].cpu().numpy()
+        oi, ow, om = to["topk_idx"], to["topk_w"], to["router_margin"]
+        flipped = False
+        for row in range(gi.shape[0]):
+            if row in exempt:
+                continue
+            if set(gi[row].tolist()) != set(oi[row].tolist()):
+                assert om[row] < ROUTE_MARGIN, (
+                    f"layer {l} row {row}: routing {sorted(gi[row])} vs oracle {sorted(oi[row])}, margin {om[row]:.3e}")
+                exempt.add(row)
+                flipped = True
+                continue
+            # weights per expert
+            gmap = dict(zip(gi[row].tolist(), gw[row].tolist()))
+            for e, w in zip(oi[row].tolist(), ow[row].tolist()):
+                assert abs(gmap[e] - w) <= 10 * t, (l, row, e, gmap[e], w)
         if not exempt:
             np.testing.assert_array_equal(counts, to["counts"])
             # tokens of each expert segment, in order (independent of the slot order)
@@ -124,11 +141,83 @@ def compare_pass(cfg, taps_gpu, logits_gpu, taps_o, logits_o, report=None, exemp
         assert e_out <= t, f"layer {l} MoE residual: rel err {e_out:.3e} > {t}"
         if report is not None:
             report.append(dict(layer=l, attn=e_attn, out=e_out, exempt=len(exempt)))
+        if flipped and l + 1 < len(taps_o):
+            diverged = l
+    if diverged is not None:
+        if report is not None:
+            report.append(dict(logits=None, diverged_after_layer=diverged))
+        return set(range(C))
     e_log = rel_err(logits_gpu, logits_o, exempt)
     assert e_log <= t, f"logits rel err {e_log:.3e} > {t}"
     if report is not None:
         report.append(dict(logits=e_log))
     return exempt
+
+
+def causal_reach(runs, n_layers):
+    """For each layer l, the first cache position whose K/V may legitimately differ.
+
+    `runs`: (position offset, GPU top-k per layer [T][k], oracle taps per layer) for each
+    prefill call, in order.  A row routed differently at layer l (allowed only at a near
+    tie, which is asserted for every row not already reached) has a different hidden
+    state from layer l + 1 on, and through causal attention so has every later position
+    in the layers above."""
+    reach = [None] * n_layers
+    for off, gpu_topk, taps in runs:
+        for l, t in enumerate(taps):
+            gi = np.asarray(gpu_topk[l])
+            oi, om = t["topk_idx"], np.asarray(t["router_margin"])
+            for r in range(gi.shape[0]):
+                if reach[l] is not None and off + r >= reach[l]:
+                    break
+                if set(gi[r].tolist()) != set(np.asarray(oi[r]).tolist()):
+                    assert om[r] < ROUTE_MARGIN, (
+                        f"prefill layer {l} position {off + r}: routing {sorted(gi[r])} vs oracle "
+                        f"{sorted(oi[r])}, margin {om[r]:.3e}")
+                    for l2 in range(l + 1, n_layers):
+                        reach[l2] = off + r if reach[l2] is None else min(reach[l2], off + r)
+                    break
+    return reach
+
+
+def prefill_topk(st, T):
+    """Taps sized for a T-token prefill; returns the per-layer top-k device tensors."""
+    return st.taps(T)["topk_idx"]
+
+
+def stored_kv(oc, cfg):
+    """The oracle cache's (already stored-precision) K/V as arrays dg.KVCache.load_prefix
+    takes: bf16 bit patterns (exact: every value is a bf16 value) or float32."""
+    out = []
+    for k, v in zip(oc.k, oc.v):
+        pair = []
+        for a in (k, v):
+            f = np.ascontiguousarray(a.astype(np.float32))
+            assert np.array_equal(f.astype(np.float64), a)
+            if cfg["dtype"] == "bf16":
+                bits = f.view(np.uint32)
+                assert not (bits & 0xFFFF).any()
+                pair.append((bits >> 16).astype(np.uint16))
+            else:
+                pair.append(f)
+        out.append(tuple(pair))
+    return out
+
+
+def kv_close_causal(cache, oc, reach, label):
+    """Every layer's K and V against the oracle's, up to that layer's causal reach of a
+    near-tie routing row; returns the fraction of positions compared."""
+    total, seen = 0, 0
+    for l in range(len(reach)):
+        k, v = cache.logical(l)
+        n = oc.k[l].shape[1]
+        stop = n if reach[l] is None else reach[l]
+        for name, a, b in (("K", k, oc.k[l]), ("V", v, oc.v[l])):
+            ok, frac, worst = kv_close(np.asarray(a)[:, :stop], np.asarray(b)[:, :stop])
+            assert ok, f"{label} layer {l} {name}: {frac:.2%} differ; {worst}"
+        total += n
+        seen += stop
+    return seen / max(total, 1)
 
 
 def bf16_spacing(x):

@@ -1,11 +1,17 @@
 """The multi-layer workloads at their full sizes, through the C-ABI, against the oracle.
 
 - 8-layer denoise (prefix 2048, canvas 256, 16 passes, re-noise 50% -> 0%): every pass
-  compared with the oracle, free running, exemptions carried from pass to pass.
+  compared with the oracle from the oracle's canvas; the GPU's own 16-pass loop for the
+  properties that hold at any size (dg_generate_canvas equal to it, untouched prefix).
 - chained canvases (8 layers, 512-token prompt, 4 canvases x 16 passes + append): the
   prompt's K/V and the first canvas's 16 passes and append against the oracle; all four
   canvases for the properties that hold at any size (cache length, untouched prefix,
   bit-identical repeat run).
+
+Each compared pass starts both sides from the oracle's canvas.  A token that comes out
+different at a near tie (allowed by the tolerance) reaches every row of the next pass
+through block attention, so once the two canvases part, later passes are different
+problems; the GPU's free-running canvas is checked only for properties.
 - large pass (4 layers, H2816, E128 top-8, F704, V262144, prefix 32768): the first pass
   layer by layer and its update against the oracle; the 8-pass run for its properties.
 """
@@ -46,44 +52,66 @@ def _pass(dg, st, canvas_np, n, step, seed=synth.SEED_RENOISE, taps=True):
     return tp, logits.cpu().numpy(), canvas.cpu().numpy(), conf.cpu().numpy()
 
 
-def _free_run(dg, st, oc, noise, S, r0, r1, label):
-    """S passes on both sides from the same noise; returns (gpu canvas, oracle canvas, exempt)."""
+def _forced_run(dg, st, oc, noise, S, r0, r1, label):
+    """S passes, each started on both sides from the oracle's canvas; returns the oracle's
+    final canvas."""
     C = len(noise)
-    cur_g, cur_o = noise.copy(), noise.copy()
-    tainted = set()
+    cur = noise.copy()
+    diverged = 0
     for s in range(S):
         n = O.renoise_count(C, S, s, r0, r1)
-        taps, logits, nxt_g, conf = _pass(dg, st, cur_g, n, s)
-        logits_o, taps_o = O.denoise_pass(st.host, oc, cur_o, st.prec)
+        taps, logits, nxt_g, conf = _pass(dg, st, cur, n, s)
+        logits_o, taps_o = O.denoise_pass(st.host, oc, cur, st.prec)
         upd = O.canvas_update(logits_o, n, synth.SEED_RENOISE, s)
         report = []
-        exempt = PL.compare_pass(st.cfg, taps, logits, taps_o, logits_o, report, exempt=tainted)
+        exempt = PL.compare_pass(st.cfg, taps, logits, taps_o, logits_o, report)
         PL.compare_update(nxt_g, conf, upd, exempt, n)
-        tainted = exempt | {i for i in range(C) if nxt_g[i] != upd["canvas"][i]}
-        print(f"{label} pass {s}: n={n} logits err {report[-1]['logits']:.2e} exempt {len(tainted)}", flush=True)
-        cur_g, cur_o = nxt_g, upd["canvas"]
-    return cur_g, cur_o, tainted
+        diff = int((nxt_g != upd["canvas"]).sum())
+        end = report[-1]
+        if end["logits"] is None:
+            diverged += 1
+            state = f"structure only after layer {end['diverged_after_layer']}"
+        else:
+            state = f"logits err {end['logits']:.2e} exempt {len(exempt)}"
+        print(f"{label} pass {s}: n={n} {state} tokens differing {diff}", flush=True)
+        cur = upd["canvas"]
+    # most passes must be compared in full
+    assert diverged <= S // 4, f"{diverged} of {S} passes compared for structure only"
+    return cur
+
+
+def _gpu_loop(dg, st, noise, S, r0, r1):
+    """The GPU's own S passes (pass + update), no taps."""
+    C, V = len(noise), st.cfg["vocab"]
+    st.model.set_taps(None)
+    can = torch.from_numpy(np.asarray(noise, dtype=np.int32)).cuda()
+    lg = torch.empty(C, V, device="cuda")
+    for s in range(S):
+        dg.denoise_pass(st.model, st.cache, can, lg, st.ws)
+        dg.canvas_update(lg, dg.renoise_count(C, S, s, r0, r1), synth.SEED_RENOISE, s, can, st.ws)
+    dg.device_status(st.ws)
+    return can.cpu().numpy()
 
 
 def test_denoise8_full_size(dg):
     cfg = CF.CONFIGS["denoise8_bf16"]
     P, C, S = cfg["prefix"], cfg["canvas"], cfg["steps"]
+    r0, r1 = cfg["renoise_start"], cfg["renoise_end"]
     st = PL.Setup(cfg, P, capacity=P + C)
     st.ws = st.workspace(C)
     before = [(k[:, :P].clone(), v[:, :, :P].clone()) for k, v in zip(st.cache.k, st.cache.vt)]
     noise = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
-    g, o, exempt = _free_run(dg, st, st.ocache, noise, S, cfg["renoise_start"], cfg["renoise_end"], "denoise8")
-    assert len(exempt) <= C // 8, f"too many exempt positions: {len(exempt)}"
+    _forced_run(dg, st, st.ocache, noise, S, r0, r1, "denoise8")
+    g = _gpu_loop(dg, st, noise, S, r0, r1)
+    assert g.min() >= 0 and g.max() < cfg["vocab"]
     # the prefix K/V were reused untouched across all passes
     for (k0, v0), k, v in zip(before, st.cache.k, st.cache.vt):
         assert torch.equal(k[:, :P], k0) and torch.equal(v[:, :, :P], v0)
     assert st.cache.len == P
-    # dg_generate_canvas gives the same canvas, bit for bit
+    # dg_generate_canvas gives the same canvas as the pass / update loop, bit for bit
     can = torch.from_numpy(noise).cuda()
     lg = torch.empty(C, cfg["vocab"], device="cuda")
-    st.model.set_taps(None)
-    dg.generate_canvas(st.model, st.cache, can, S, cfg["renoise_start"], cfg["renoise_end"], synth.SEED_RENOISE,
-                       False, lg, st.ws)
+    dg.generate_canvas(st.model, st.cache, can, S, r0, r1, synth.SEED_RENOISE, False, lg, st.ws)
     dg.device_status(st.ws)
     np.testing.assert_array_equal(can.cpu().numpy(), g)
 
@@ -91,55 +119,68 @@ def test_denoise8_full_size(dg):
 def test_chained8_full_size(dg):
     cfg = CF.CONFIGS["chained8_bf16"]
     T0, C, S, n_can = cfg["prompt"], cfg["canvas"], cfg["steps"], cfg["n_canvases"]
+    r0, r1 = cfg["renoise_start"], cfg["renoise_end"]
+    L = cfg["n_layers"]
     cap = T0 + n_can * C
     st = PL.Setup(cfg, 0, capacity=cap, with_prefix=False)
     st.ws = st.workspace(max(T0, C))
+    # the prompt's prefill against the oracle, up to the causal reach of a near-tie flip
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, T0, cfg["vocab"])
+    topk = PL.prefill_topk(st, T0)
     dg.prefill_append(st.model, st.cache, torch.from_numpy(prompt).cuda(), st.ws)
     taps = []
     oc = O.prefill_append(st.host, st.ocache, prompt, st.prec, taps)
-    near_tie = {int(i) for t in taps for i in np.nonzero(t["router_margin"] < PL.ROUTE_MARGIN)[0]}
-    for l in range(cfg["n_layers"]):
-        k, v = st.cache.logical(l)
-        for name, a, b in (("K", k, oc.k[l]), ("V", v, oc.v[l])):
-            ok, frac, worst = PL.kv_close(a, b, near_tie)
-            assert ok, f"prompt layer {l} {name}: {frac:.2%} differ; {worst}"
-    prompt_kv = [(k[:, :T0].clone(), v[:, :, :T0].clone()) for k, v in zip(st.cache.k, st.cache.vt)]
-    # first canvas: 16 passes free running against the oracle, then its append
+    seen = PL.kv_close_causal(st.cache, oc, PL.causal_reach([(0, [t.cpu().numpy() for t in topk], taps)], L),
+                              "prompt")
+    print(f"prompt K/V: {seen:.1%} of layer positions compared", flush=True)
+    assert seen >= 0.5
+    gpu_prompt_kv = [(k[:, :T0].clone(), v[:, :, :T0].clone()) for k, v in zip(st.cache.k, st.cache.vt)]
+    # the canvases continue from the oracle's prompt K/V on both sides
+    prompt_stored = PL.stored_kv(oc, cfg)
+
+    def oracle_prompt_cache():
+        cache = dg.KVCache(cfg, cap)
+        cache.load_prefix(prompt_stored)
+        return cache
+    st.cache = oracle_prompt_cache()
     noise0 = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
-    g, o, exempt = _free_run(dg, st, oc, noise0, S, cfg["renoise_start"], cfg["renoise_end"], "chained canvas 0")
-    assert len(exempt) <= C // 8
-    dg.prefill_append(st.model, st.cache, torch.from_numpy(g.astype(np.int32)).cuda(), st.ws)
-    if not exempt:
-        oc = O.prefill_append(st.host, oc, o, st.prec)
-        for l in range(cfg["n_layers"]):
-            k, v = st.cache.logical(l)
-            ok, frac, worst = PL.kv_close(k, oc.k[l], near_tie)
-            assert ok, f"after append layer {l} K: {frac:.2%} differ; {worst}"
+    first = _forced_run(dg, st, oc, noise0, S, r0, r1, "chained canvas 0").astype(np.int32)
+    topk = PL.prefill_topk(st, C)
+    dg.prefill_append(st.model, st.cache, torch.from_numpy(first).cuda(), st.ws)
+    taps = []
+    oc = O.prefill_append(st.host, oc, first, st.prec, taps)
+    seen = PL.kv_close_causal(st.cache, oc, PL.causal_reach([(T0, [t.cpu().numpy() for t in topk], taps)], L),
+                              "after append")
+    print(f"after append K/V: {seen:.1%} of layer positions compared", flush=True)
+    assert seen >= 0.5
     # the remaining canvases through dg_generate_canvas (append included)
-    canvases = [g]
+    canvases = []
     st.model.set_taps(None)
     lg = torch.empty(C, cfg["vocab"], device="cuda")
     for c in range(1, n_can):
         can = torch.from_numpy(synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])).cuda()
-        dg.generate_canvas(st.model, st.cache, can, S, cfg["renoise_start"], cfg["renoise_end"], synth.SEED_RENOISE,
-                           True, lg, st.ws)
+        dg.generate_canvas(st.model, st.cache, can, S, r0, r1, synth.SEED_RENOISE, True, lg, st.ws)
         canvases.append(can.cpu().numpy())
     dg.device_status(st.ws)
     assert st.cache.len == cap
-    for (k0, v0), k, v in zip(prompt_kv, st.cache.k, st.cache.vt):
-        assert torch.equal(k[:, :T0], k0) and torch.equal(v[:, :, :T0], v0)
+    k0 = oracle_prompt_cache()
+    for a, b, va, vb in zip(st.cache.k, k0.k, st.cache.vt, k0.vt):
+        assert torch.equal(a[:, :T0], b[:, :T0]) and torch.equal(va[:, :, :T0], vb[:, :, :T0])
     for c in canvases:
         assert c.min() >= 0 and c.max() < cfg["vocab"]
-    # a second, independent run of the whole chain is bit-identical
+    # a second, independent run is bit-identical: the prompt's prefill, and the chain
     st2 = PL.Setup(cfg, 0, capacity=cap, with_prefix=False)
     st2.ws = st2.workspace(max(T0, C))
     dg.prefill_append(st2.model, st2.cache, torch.from_numpy(prompt).cuda(), st2.ws)
-    for c in range(n_can):
+    for (k, v), k2, v2 in zip(gpu_prompt_kv, st2.cache.k, st2.cache.vt):
+        assert torch.equal(k, k2[:, :T0]) and torch.equal(v, v2[:, :, :T0])
+    st2.cache = oracle_prompt_cache()
+    dg.prefill_append(st2.model, st2.cache, torch.from_numpy(first).cuda(), st2.ws)
+    for c in range(1, n_can):
         can = torch.from_numpy(synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])).cuda()
-        dg.generate_canvas(st2.model, st2.cache, can, S, cfg["renoise_start"], cfg["renoise_end"],
-                           synth.SEED_RENOISE, True, lg, st2.ws)
-        np.testing.assert_array_equal(can.cpu().numpy(), canvases[c])
+        dg.generate_canvas(st2.model, st2.cache, can, S, r0, r1, synth.SEED_RENOISE, True, lg, st2.ws)
+        np.testing.assert_array_equal(can.cpu().numpy(), canvases[c - 1])
+    dg.device_status(st2.ws)
     for a, b in zip(st.cache.k, st2.cache.k):
         assert torch.equal(a, b)
 
@@ -157,7 +198,7 @@ def test_large4_full_size(dg):
     report = []
     exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, report)
     PL.compare_update(nxt, conf, upd, exempt, n0)
-    print("large4 first pass:", report, "exempt", sorted(exempt))
+    print("large4 first pass:", report, "exempt", len(exempt))
     unions = taps["unions"].cpu().numpy()
     assert (unions >= cfg["top_k"]).all() and (unions <= cfg["n_experts"]).all()
     assert [t["union"] for t in taps_o] == list(unions) or exempt

@@ -84,7 +84,9 @@ def test_grouped_gemm(dg, counts, M):
 @pytest.mark.parametrize("swiglu", [False, True])
 def test_stream_k_matches_one_tile_per_cta(dg, swiglu):
     """Enough tiles for the stream-K split (cut tiles finished from a parked partial):
-    the result equals the one-tile-per-CTA schedule to fp32 rounding, and both match torch."""
+    the result equals the one-tile-per-CTA schedule, and both match torch, to the
+    rounding of fp32 sums in another order (the SwiGLU output as hi + lo bf16 carries
+    about 16 significant bits)."""
     g = torch.Generator(device="cuda").manual_seed(21)
     counts = [37, 0, 64, 5, 90, 130, 16, 1] * 8
     E, F, K = len(counts), 704, 512
@@ -110,7 +112,7 @@ def test_stream_k_matches_one_tile_per_cta(dg, swiglu):
         a = X[o[e]:o[e + 1]].double() @ W[e].double().T
         ref[o[e]:o[e + 1]] = torch.nn.functional.silu(a) * (X[o[e]:o[e + 1]].double() @ W2[e].double().T) if swiglu else a
     scale = ref.abs().max().item()
-    torch.testing.assert_close(outs[0], outs[1], rtol=1e-5, atol=1e-6 * scale)
+    torch.testing.assert_close(outs[0], outs[1], rtol=1e-4, atol=1e-5 * scale)
     torch.testing.assert_close(outs[0], ref, rtol=1e-4, atol=1e-5 * scale)
 
 

@@ -82,21 +82,18 @@ def test_prefill_append_matches_oracle(dg):
     ws = st.workspace(300)
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 77, cfg["vocab"])
     more = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(9), 150, cfg["vocab"])
-    near_tie = set()   # positions whose oracle routing margin is below 1e-3 in some layer
+    runs = []
     for toks in (prompt, more):
         P0 = st.ocache.len
+        topk = PL.prefill_topk(st, len(toks))
         dg.prefill_append(st.model, st.cache, torch.from_numpy(toks).cuda(), ws)
         taps = []
         st.ocache = O.prefill_append(st.host, st.ocache, toks, st.prec, taps)
-        for t in taps:
-            near_tie |= {P0 + int(i) for i in np.nonzero(t["router_margin"] < PL.ROUTE_MARGIN)[0]}
+        runs.append((P0, [t.cpu().numpy() for t in topk], taps))
     dg.device_status(ws)
     assert st.cache.len == 227 == st.ocache.len
-    for l in range(cfg["n_layers"]):
-        k, v = st.cache.logical(l)
-        for name, g, o in (("K", k, st.ocache.k[l]), ("V", v, st.ocache.v[l])):
-            ok, frac, worst = PL.kv_close(g, o, near_tie)
-            assert ok, f"layer {l} {name}: {frac:.2%} of elements differ; {worst}"
+    seen = PL.kv_close_causal(st.cache, st.ocache, PL.causal_reach(runs, cfg["n_layers"]), "prefill")
+    assert seen >= 0.5
 
 
 def test_mask_worked_example_on_gpu(dg):
@@ -119,40 +116,39 @@ def test_mask_worked_example_on_gpu(dg):
 def test_chained_canvases_small(dg):
     """prompt prefill -> (S denoising steps with re-noising -> append) x 2, step by step.
 
-    Positions whose tokens came out different (only allowed where the oracle's margin
-    exempts them) stay exempt in later steps and canvases of the comparison."""
+    Every pass starts both sides from the oracle's canvas: one token that legitimately
+    comes out different (a near-tie top-1/top-2 margin) changes every row of the next
+    pass through block attention, so a free-running comparison would compare different
+    problems.  The appended canvas is the oracle's as well."""
     cfg = dict(SMALL_BF16, n_layers=2)
     C, S, n_can = 64, 3, 2
     st = PL.Setup(cfg, 0, capacity=512, with_prefix=False)
     ws = st.workspace(96)
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 96, cfg["vocab"])
+    topk = PL.prefill_topk(st, 96)
     dg.prefill_append(st.model, st.cache, torch.from_numpy(prompt).cuda(), ws)
-    oc = O.prefill_append(st.host, st.ocache, prompt, st.prec)
+    taps = []
+    oc = O.prefill_append(st.host, st.ocache, prompt, st.prec, taps)
+    runs = [(0, [t.cpu().numpy() for t in topk], taps)]
     for c in range(n_can):
-        cur_g = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])
-        cur_o = cur_g.copy()
-        tainted = set()
+        cur = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])
         for s in range(S):
             n = O.renoise_count(C, S, s, 0.5, 0.0)
-            taps, logits, nxt_g, conf = _gpu_pass(dg, st, cur_g, n, step=s)
-            logits_o, taps_o = O.denoise_pass(st.host, oc, cur_o, st.prec)
+            taps, logits, nxt_g, conf = _gpu_pass(dg, st, cur, n, step=s)
+            logits_o, taps_o = O.denoise_pass(st.host, oc, cur, st.prec)
             upd = O.canvas_update(logits_o, n, synth.SEED_RENOISE, s)
-            exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, exempt=tainted)
+            exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o)
             PL.compare_update(nxt_g, conf, upd, exempt, n)
-            tainted = exempt | {i for i in range(C) if nxt_g[i] != upd["canvas"][i]}
-            cur_g, cur_o = nxt_g, upd["canvas"]
-        print(f"canvas {c}: positions exempt at the end {sorted(tainted)}")
-        if tainted:
-            return   # the two runs now append different canvases; the rest is not comparable
-        dg.prefill_append(st.model, st.cache, torch.from_numpy(cur_g.astype(np.int32)).cuda(), ws)
-        oc = O.prefill_append(st.host, oc, cur_o, st.prec)
+            cur = upd["canvas"]
+        topk = PL.prefill_topk(st, C)
+        dg.prefill_append(st.model, st.cache, torch.from_numpy(cur.astype(np.int32)).cuda(), ws)
+        taps = []
+        runs.append((oc.len, [t.cpu().numpy() for t in topk], taps))
+        oc = O.prefill_append(st.host, oc, cur, st.prec, taps)
     dg.device_status(ws)
     assert st.cache.len == oc.len == 96 + n_can * C
-    for l in range(cfg["n_layers"]):
-        k, v = st.cache.logical(l)
-        for name, g, o in (("K", k, oc.k[l]), ("V", v, oc.v[l])):
-            ok, frac, worst = PL.kv_close(g, o)
-            assert ok, f"layer {l} {name}: {frac:.2%} of elements differ; {worst}"
+    seen = PL.kv_close_causal(st.cache, oc, PL.causal_reach(runs, cfg["n_layers"]), "chained")
+    assert seen >= 0.5
 
 
 def test_generate_canvas_equals_step_loop(dg):
