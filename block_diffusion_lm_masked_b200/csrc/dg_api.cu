@@ -36,6 +36,11 @@ static dg_status fail(dg_status s, const char* fmt, ...) {
   g_err = buf;
   return s;
 }
+namespace dg {
+// for entry points defined in other translation units
+dg_status set_error(dg_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace dg
+
 #define DG_CHECK_ARG(cond, ...) \
   do {                          \
     if (!(cond)) return fail(DG_ERR_INVALID_ARG, __VA_ARGS__); \

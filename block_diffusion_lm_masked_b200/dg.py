@@ -72,6 +72,7 @@ def _load():
         "dg_prefill_append": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, SZ, P]),
         "dg_denoise_pass": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, P, SZ, P]),
         "dg_canvas_update": (I32, [P, I32, I32, I32, U64, U32, P, P, P, SZ, P]),
+        "dg_canvas_update_noalloc": (I32, [P, I32, I32, I32, U64, U32, P, P, P]),
         "dg_generate_canvas": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, U64, I32, P, P, SZ, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
@@ -265,6 +266,15 @@ def canvas_update(logits: torch.Tensor, n_renoise: int, seed: int, step: int, ca
     nb = ws.nbytes if isinstance(ws, Workspace) else ws.numel()
     _check(lib.dg_canvas_update(_ptr(logits), C, V, n_renoise, seed & 0xFFFFFFFFFFFFFFFF, step, _ptr(canvas),
                                 _ptr(conf), ptr, nb, _stream(stream)))
+
+
+def canvas_update_noalloc(logits: torch.Tensor, n_renoise: int, seed: int, step: int, canvas: torch.Tensor,
+                          conf: torch.Tensor | None = None, stream=None):
+    """dg_canvas_update without a workspace: the scratch is libdg's fixed per-device array
+    (calls on one device must be ordered; see include/dg_noalloc.h)."""
+    C, V = logits.shape
+    _check(lib.dg_canvas_update_noalloc(_ptr(logits), C, V, n_renoise, seed & 0xFFFFFFFFFFFFFFFF, step,
+                                        _ptr(canvas), _ptr(conf), _stream(stream)))
 
 
 def generate_canvas(model: Model, cache: KVCache, canvas: torch.Tensor, S: int, r_start: float, r_end: float,
