@@ -19,7 +19,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
+import threading
 import sys
 import time
 
@@ -53,41 +53,69 @@ def _workload_desc(name, cfg):
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled through NVML (the counters nvidia-smi
+    reads) every ~10 ms in a background thread during the timed region; read-only."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.p = None
+    def __init__(self, device):
+        self.dev = device
+        self.samples = []
+        self.thread = None
+        self.stop_flag = threading.Event()
+        self.nv = None
+
+    def _handle(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        self.nv = nv
+        p = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _run(self, h):
+        nv = self.nv
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                self.samples.append((sm, reasons(h)))
+            except Exception as e:   # keep sampling; report the first failure
+                self.error = self.error or repr(e)
+            time.sleep(0.01)
 
     def start(self):
+        self.error = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
-                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.p = None
+            h = self._handle()
+            self.max_mhz = self.nv.nvmlDeviceGetMaxClockInfo(h, self.nv.NVML_CLOCK_SM)
+        except Exception as e:
+            self.error = repr(e)
+            self.thread = None
+            return
+        self.thread = threading.Thread(target=self._run, args=(h,), daemon=True)
+        self.thread.start()
+        time.sleep(0.05)   # the sampler runs before the timed region starts
 
     def stop(self):
-        if self.p is None:
-            return None
-        self.p.terminate()
-        try:
-            out, _ = self.p.communicate(timeout=5)
-        except Exception:
-            self.p.kill()
-            out, _ = self.p.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self.thread is None:
+            return {"unavailable": self.error}
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return {"unavailable": self.error or "no sample in the timed region"}
+        nv = self.nv
+        reasons = sorted({name for _, r in self.samples for name, attr in self.REASONS
+                          if hasattr(nv, attr) and r & getattr(nv, attr)})
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "NVML, 10 ms"}
 
 
 def _oracle_step(host, ocache, canvas, n, prec, step):
@@ -104,6 +132,27 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+REF_BUDGET_S = 90.0
+
+# DRAM bytes (read + write) of one gate/up GEMM launch from an ncu capture of this
+# workload, valid only for the kernel source it was taken on (sha256 prefix of
+# k_tc_gemm.cu); any other source reports null.
+NCU_TRAFFIC = {"layer1_bf16": ("47b56d50d45be312", 467.090688e6 + 6.504448e6)}
+
+
+def _ncu_traffic(workload):
+    import hashlib
+    entry = NCU_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    src = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", "k_tc_gemm.cu")
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return entry[1] if digest == entry[0] else None
+
+
 def run_reference(args, cfg, name):
     """The CPU oracle on the host cores, one oracle step per timed step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -116,16 +165,21 @@ def run_reference(args, cfg, name):
     canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
     prec = O.Precision(cfg["dtype"])
     n = O.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
-    for w in range(args.warmup):
+    # a bounded sample: at most one warm-up step, then whole steps until K are done or
+    # REF_BUDGET_S seconds have passed (at least one)
+    for w in range(min(args.warmup, 1)):
         _oracle_step(host, ocache, canvas, n, prec, 0)
     t0 = time.perf_counter()
-    for s in range(args.steps):
+    done = 0
+    while done < args.steps and (done == 0 or time.perf_counter() - t0 < REF_BUDGET_S):
         _oracle_step(host, ocache, canvas, n, prec, 0)
+        done += 1
     dt = time.perf_counter() - t0
-    ms = dt * 1e3 / max(1, args.steps)
+    ms = dt * 1e3 / done
     value = C / (ms / 1e3)
     cores = _blas_threads()
-    sample = f"{args.steps} full oracle steps (pass + update) of the workload, fp64 numpy"
+    sample = (f"{done} of {args.steps} requested whole oracle steps (pass + update, fp64 numpy) of the workload, "
+              f"{REF_BUDGET_S:.0f} s budget")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
@@ -160,7 +214,7 @@ def cpu_baseline(cfg, budget_s=30.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--workload", default="layer1_bf16", choices=[n for n in CF.ORDER if n != "chained8_bf16"])
@@ -237,7 +291,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clk = Clocks(local)
+    clk = Clocks(dev)
     clk.start()
     total_ms, launches = timed(args.steps, profile=False)
     clocks = clk.stop()
@@ -248,8 +302,9 @@ def main():
         total_ms = float(t.item())
         dist.barrier()
 
-    # per-kernel breakdown with CUDA events on the launching stream (separate timed run)
-    prof_ms, _ = timed(args.steps, profile=True)
+    # per-kernel breakdown with CUDA events on the launching stream (separate timed run,
+    # at most 200 steps: it records an event pair around every launch)
+    prof_ms, _ = timed(min(args.steps, 200), profile=True)
     kern = {}
     for kname in dg.KERNEL_KINDS:
         ms, n = dg.profile_read(kname)
@@ -293,7 +348,7 @@ def main():
         per_launch = RF.gate_up_bytes(cfg, unions_h[0], C * cfg["top_k"])
         achieved = per_launch / (gu["avg_us"] * 1e-6) / 1e9
         roof = {"kernel": "gemm_gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                "frac": achieved / hbm, "traffic": _ncu_traffic(name), "peak_source": f"{peak_src} hbm_gbs",
                 "bytes_per_launch": per_launch}
 
     line = {
