@@ -70,6 +70,7 @@ class Clocks:
 
     def _handle(self):
         import pynvml as nv
+        import torch
         nv.nvmlInit()
         self.nv = nv
         p = torch.cuda.get_device_properties(self.dev)

@@ -242,10 +242,8 @@ constexpr int kMaxKsO = 8;     // split-K of the output projection
 constexpr int kSmemGemm = 200 * 1024;    // stage budget of the persistent GEMM (one CTA per SM)
 inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kItemRows = 64;            // rows per work item of the grouped expert GEMMs
+constexpr int kItemRows = 128;           // rows per work item of the grouped expert GEMMs
 
-constexpr int kSkFlagBytes = 4096;                 // stream-K flags (one int per CTA, <= 1024 SMs)
-constexpr size_t kSkSlotFloats = 128 * 256;        // largest parked partial: 128 x n_max (x2 dual)
 
 struct WsLayout {
   size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
@@ -355,14 +353,7 @@ struct GemmCall {
   int k_splits;
   size_t split_stride;
   int smem_budget;
-  float* sk_part;  // stream-K scratch; null (every pass GEMM): one tile per CTA per turn
-  int* sk_flag;
 };
-
-int next_epoch() {
-  static std::atomic<int> epoch{0};
-  return ++epoch;
-}
 
 dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   CUtensorMap B, B2, Bb, B2b;
@@ -393,9 +384,6 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   p.ld_out = g.ld_out;
   p.smem_budget = g.smem_budget;
   p.err = err;
-  p.sk_part = g.sk_part;
-  p.sk_flag = g.sk_flag;
-  p.sk_epoch = next_epoch();
   const int items = g.items ? g.max_items : ceil_div(g.x_rows, g.n_max) * g.k_splits;
   LAUNCH(g.kind, st,
          dg::launch_tc_gemm(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, B, B2, Bb, B2b, p, items * p.m_tiles, st));
@@ -505,8 +493,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   if (bf) {
     ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
     GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
-               nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm,
-               nullptr, nullptr};
+               nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_QKV, st,
@@ -524,7 +511,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
     ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
     GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
                n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
-               kSmemGemm, nullptr, nullptr};
+               kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_O, st,
@@ -557,11 +544,11 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
     const int max_items = n * k / kItemRows + E;
     GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate, &m->maps[l].up, ws.at<void>(ws.L.xs), xs_lo,
                 n * k, H, F, items, n_items, max_items, kItemRows, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
-                kSmemGemm, nullptr, nullptr};
+                kSmemGemm};
     if ((s = gemm_bf16(gu, err, st)) != DG_OK) return s;
     GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, nullptr, ws.at<void>(ws.L.h),
                 ws.at<void>(ws.L.h_lo), n * k, F, H, items, n_items, max_items, kItemRows, ws.at<float>(ws.L.ys),
-                nullptr, H, 1, 0, kSmemGemm, nullptr, nullptr};
+                nullptr, H, 1, 0, kSmemGemm};
     if ((s = gemm_bf16(dn, err, st)) != DG_OK) return s;
   } else {
     float* g = ws.at<float>(ws.L.gu);
@@ -682,8 +669,7 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
   // vocabulary projection of the final RMSNorm (left in ws.xn by the last layer) to fp32 logits
   if (is_bf16(c)) {
     GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, C, c.hidden,
-               c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm,
-               nullptr, nullptr};
+               c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm};
     if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
   } else {
     LAUNCH(DG_K_GEMM_VOCAB, st,
@@ -821,14 +807,13 @@ extern "C" int64_t dg_launch_count(void) {
 
 extern "C" size_t dg_debug_gemm_scratch_bytes(int32_t x_rows, int32_t n_groups) {
   if (x_rows <= 0 || n_groups <= 0) return 0;
-  return kSkFlagBytes + al(sizeof(dg::TcWorkItem) * ((size_t)x_rows + n_groups + 1) + 16) +
-         (size_t)dg::num_sms() * kSkSlotFloats * 4;
+  return al(sizeof(dg::TcWorkItem) * ((size_t)x_rows + n_groups + 1) + 16);
 }
 
 extern "C" dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_t n_groups,
                                         const void* X, const void* X_lo, int32_t x_rows, int32_t K,
                                         const int32_t* group_off, void* out, void* out_lo, int32_t ld_out,
-                                        int32_t streamk, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
+                                        void* d_scratch, size_t scratch_bytes, int32_t* d_err,
                                         dg_stream stream) {
   DG_CHECK_ARG(W && X && out && d_err && d_scratch, "NULL pointer");
   DG_CHECK_ARG(K > 0 && K % 64 == 0 && rows > 0 && n_groups > 0 && x_rows > 0, "bad GEMM shape");
@@ -842,21 +827,17 @@ extern "C" dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t r
   dg_status s = map_weights(&A, W, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K);
   if (s != DG_OK) return s;
   if (W2 && (s = map_weights(&A2, W2, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
-  char* sc = static_cast<char*>(d_scratch);
-  int* sk_flag = reinterpret_cast<int*>(sc);
-  dg::TcWorkItem* items = reinterpret_cast<dg::TcWorkItem*>(sc + kSkFlagBytes);
+  dg::TcWorkItem* items = static_cast<dg::TcWorkItem*>(d_scratch);
   int* n_items = reinterpret_cast<int*>(items + x_rows + n_groups);
-  float* sk_part = reinterpret_cast<float*>(sc + kSkFlagBytes +
-                                            al(sizeof(dg::TcWorkItem) * ((size_t)x_rows + n_groups + 1) + 16));
   int max_items = 0;
   if (group_off) {
     max_items = x_rows / kItemRows + n_groups;
-    LAUNCH(DG_K_PERMUTE, st, dg::launch_build_items(group_off, n_groups, kItemRows, items, n_items, st));
+    LAUNCH(DG_K_PERMUTE, st, dg::launch_build_items(group_off, n_groups, kItemRows, x_rows, items, n_items, d_err, st));
   }
+  const int n_max = group_off ? kItemRows : (x_rows < 256 ? ((x_rows + 15) & ~15) : 256);
   GemmCall g{DG_K_GEMM_QKV, W2 ? dg::EPI_SWIGLU_BF16 : dg::EPI_STORE_F32, &A, W2 ? &A2 : nullptr, X, X_lo, x_rows,
-             K, rows, group_off ? items : nullptr, group_off ? n_items : nullptr, max_items,
-             group_off ? kItemRows : (x_rows < 256 ? ((x_rows + 15) & ~15) : 256), out, out_lo, ld_out, 1, 0,
-             kSmemGemm, streamk ? sk_part : nullptr, streamk ? sk_flag : nullptr};
+             K, rows, group_off ? items : nullptr, group_off ? n_items : nullptr, max_items, n_max, out, out_lo,
+             ld_out, 1, 0, kSmemGemm};
   return gemm_bf16(g, d_err, st);
 }
 

@@ -39,12 +39,6 @@ struct TcGemmParams {
   int ld_out;            // elements per output row
   int smem_budget;       // bytes for pipeline stages
   int* err;              // device error word
-  // stream-K scratch (null: one tile per CTA and turn): one parked fp32 partial of
-  // 128 x n_max (x2 with dual_a) floats and one flag per CTA; flags hold the epoch of the
-  // launch that last raised them (zero-initialised once, epochs increase per launch)
-  float* sk_part;
-  int* sk_flag;
-  int sk_epoch;
 };
 
 // grid = min(max_tiles, SMs); max_tiles bounds the tile count (exact for dense GEMMs)
@@ -52,8 +46,10 @@ struct TcGemmParams {
 cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
                            const CUtensorMap& B2, const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p,
                            int max_tiles, cudaStream_t st);
-cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
-                               cudaStream_t st);
+// grouped work list from group offsets off[E + 1] over `rows` token rows (checked on the
+// device: bad offsets give no items and DG_DEVERR_BAD_COUNT in *err)
+cudaError_t launch_build_items(const int32_t* off, int E, int n_max, int rows, TcWorkItem* items, int* n_items,
+                               int* err, cudaStream_t st);
 int num_sms();
 
 // ---------------------------------------------------------------- tcgen05 attention

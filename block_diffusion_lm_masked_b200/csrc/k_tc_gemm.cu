@@ -18,13 +18,6 @@
 // that run at the same time then read different k-blocks of the token operand, which
 // all of them share, instead of hammering the same L2 lines in lockstep.
 //
-// Scheduling: with at least as many tiles as CTAs the launch is split "stream-K": CTA c
-// owns iterations [c T / G, (c+1) T / G) of the T = tiles x k-blocks iteration space, so
-// every CTA streams the same number of weight bytes however the tile count falls
-// against the SM count.  A tile cut between CTAs c and c+1 is finished by c, which
-// reaches its first k-blocks at the end of its range: c+1 walks the rest at the start
-// of its range, parks the fp32 partial in the workspace and raises a flag; c adds it
-// before the epilogue (the wait is bounded and, in practice, already satisfied).
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -68,47 +61,17 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmParams& p, int t) {
   return ti;
 }
 
-// A contiguous run of k-blocks [kb0, kb1) of tile t.
-struct Seg {
-  int t, kb0, kb1;
-};
-
-// Walks this CTA's segments: tiles blockIdx.x, + gridDim.x, ... or, stream-K, its share
-// of the iteration space.
-struct SegWalk {
-  long long it, end;  // stream-K iteration cursor and end
-  int t;              // tile cursor (classic)
-  int n_tiles, nkb;
-  bool streamk;
-  __device__ SegWalk(int n_tiles_, int nkb_, bool sk) : n_tiles(n_tiles_), nkb(nkb_), streamk(sk) {
-    const long long total = (long long)n_tiles * nkb;
-    it = total * blockIdx.x / gridDim.x;
-    end = total * (blockIdx.x + 1) / gridDim.x;
-    t = blockIdx.x;
-  }
-  __device__ bool next(Seg& s) {
-    if (streamk) {
-      if (it >= end) return false;
-      s.t = (int)(it / nkb);
-      s.kb0 = (int)(it % nkb);
-      s.kb1 = (int)min((long long)nkb, s.kb0 + (end - it));
-      it += s.kb1 - s.kb0;
-      return true;
-    }
+// This CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+struct TileWalk {
+  int t, n_tiles;
+  __device__ TileWalk(int n_tiles_) : t(blockIdx.x), n_tiles(n_tiles_) {}
+  __device__ bool next(int& tile) {
     if (t >= n_tiles) return false;
-    s.t = t;
-    s.kb0 = 0;
-    s.kb1 = nkb;
+    tile = t;
     t += gridDim.x;
     return true;
   }
 };
-
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -122,7 +85,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __shared__ __align__(8) uint64_t acc_full[2];
   __shared__ __align__(8) uint64_t acc_empty[2];
   __shared__ __align__(8) uint64_t drain_bar;
-  __shared__ __align__(8) uint64_t part_bar;  // the four epilogue warps parked their partial
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ int n_issued_s, n_consumed_s;
@@ -152,7 +114,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(&drain_bar, 1);
-    mbar_init(&part_bar, 4);
     abort_s = 0;
     n_issued_s = 0;
     n_consumed_s = 0;
@@ -164,7 +125,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = tmem_base_s;
   griddep_sync();  // the work list and the token operand come from the previous kernels
   const int n_tiles = total_items(p) * p.m_tiles;
-  const bool streamk = p.sk_part != nullptr && n_tiles >= (int)gridDim.x;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -177,16 +137,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prefetch_tmap(&tmB2);
         prefetch_tmap(&tmB2b);
       }
-      int it = 0;
+      int it = 0, t;
       bool ok = true;
-      SegWalk walk(n_tiles, nkb, streamk);
-      Seg sg;
-      while (ok && walk.next(sg)) {
-        const int t = sg.t;
+      TileWalk walk(n_tiles);
+      while (ok && walk.next(t)) {
         const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
         const uint32_t tx = n_a * a_bytes + terms * (uint32_t)n_pad * 128;
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % stages;
           if (!mbar_wait(&empty_bar[s], ((uint32_t)(it / stages) & 1u) ^ 1u, &abort_s, p.err,
                          DG_DEVERR_TIMEOUT_EMPTY)) {
@@ -215,12 +173,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      int it = 0, j = 0;
+      int it = 0, j = 0, t;
       bool ok = true;
-      SegWalk walk(n_tiles, nkb, streamk);
-      Seg sg;
-      for (; ok && walk.next(sg); ++j) {
-        const TileInfo ti = decode_tile(p, sg.t);
+      TileWalk walk(n_tiles);
+      for (; ok && walk.next(t); ++j) {
+        const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
         const int buf = j & 1;
         if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
@@ -229,7 +186,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
         const uint32_t d1 = d0 + (uint32_t)p.n_max;
         const uint32_t idesc = idesc_bf16_f32(TC_BM, n_pad);
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % stages;
           if (!mbar_wait(&full_bar[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
             ok = false;
@@ -240,7 +197,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t sb = sa + n_a * a_bytes;
 #pragma unroll
           for (int kk = 0; kk < TC_BK / 16; ++kk) {
-            const uint32_t acc = (kb != sg.kb0 || kk != 0) ? 1u : 0u;
+            const uint32_t acc = (kb != 0 || kk != 0) ? 1u : 0u;
             const uint64_t ad = sw128_kmajor_desc(sa + kk * 32);
             const uint64_t bd = sw128_kmajor_desc(sb + kk * 32);
             const uint64_t bd2 = sw128_kmajor_desc(sb + bmax_bytes + kk * 32);
@@ -264,36 +221,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int lg = warp & 3;
     const int row = lg * 32 + lane;  // row of the 128-row tile this thread drains
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
-    const size_t slot = (size_t)TC_BM * p.n_max * n_a;  // floats of one parked partial
-    int j = 0;
-    SegWalk walk(n_tiles, nkb, streamk);
-    Seg sg;
-    for (; walk.next(sg); ++j) {
-      const TileInfo ti = decode_tile(p, sg.t);
+    int j = 0, t;
+    TileWalk walk(n_tiles);
+    for (; walk.next(t); ++j) {
+      const TileInfo ti = decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;
       const int buf = j & 1;
       if (!mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)) break;
       tc_fence_after();
       const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
-      const bool park = sg.kb0 > 0;                       // later k-blocks of a cut tile
-      const bool fold = sg.kb0 == 0 && sg.kb1 < nkb;      // first k-blocks: add the parked part
-      float* mine = p.sk_part + (size_t)blockIdx.x * slot;
-      const float* theirs = p.sk_part + (size_t)(blockIdx.x + 1) * slot;
-      if (fold) {
-        bool ready = false;
-        if (lane == 0) {
-          const uint64_t w0 = globaltimer();
-          while (!(ready = ld_acquire_gpu(p.sk_flag + blockIdx.x + 1) == p.sk_epoch)) {
-            if (abort_s || globaltimer() - w0 > DG_WAIT_NS) {
-              abort_s = 1;
-              atomicCAS(p.err, 0, DG_DEVERR_TIMEOUT_PART);
-              break;
-            }
-          }
-        }
-        ready = __shfl_sync(0xffffffffu, ready, 0);
-        if (!ready) break;
-      }
       const int f = ti.m * TC_BM + row;  // weight row = output feature
       const bool fvalid = f < p.a_rows_per_group;
       for (int c0 = 0; c0 < n_pad; c0 += 16) {
@@ -304,17 +240,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int col = c0 + q;
-          float a = __uint_as_float(ra[q]);
-          float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
-          if (park) {
-            mine[(size_t)col * TC_BM + row] = a;
-            if (EPI == EPI_SWIGLU_BF16) mine[(size_t)(p.n_max + col) * TC_BM + row] = b;
-            continue;
-          }
-          if (fold) {
-            a += theirs[(size_t)col * TC_BM + row];
-            if (EPI == EPI_SWIGLU_BF16) b += theirs[(size_t)(p.n_max + col) * TC_BM + row];
-          }
+          const float a = __uint_as_float(ra[q]);
+          const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
           if (!fvalid || col >= ti.rows) continue;
           const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
           if (EPI == EPI_STORE_F32) {
@@ -328,17 +255,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       tc_fence_before();
-      if (park) {
-        __threadfence();  // this thread's partial is visible GPU-wide before the flag goes up
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&part_bar);
-        if (warp == 2 && lane == 0) {
-          if (mbar_wait(&part_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_PART)) {
-            __threadfence();
-            atomicExch(p.sk_flag + blockIdx.x, p.sk_epoch);
-          }
-        }
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
@@ -359,8 +275,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
 // ---------------------------------------------------------------- work items of a grouped GEMM
 // For each group g with rows [off[g], off[g+1]): items of at most n_max rows, in group
-// order.  Written by one thread (E is small).
-static __device__ void emit_work_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items) {
+// order.  Written by one thread (E is small).  Offsets that decrease or leave [0, rows]
+// are an input error: no item is emitted and the error word records DG_DEVERR_BAD_COUNT.
+static __device__ void emit_work_items(const int32_t* off, int E, int n_max, int rows, TcWorkItem* items,
+                                       int* n_items, int* err) {
+  for (int e = 0; e < E; ++e) {
+    if (off[e] < 0 || off[e + 1] < off[e] || off[e + 1] > rows) {
+      atomicCAS(err, 0, DG_DEVERR_BAD_COUNT);
+      *n_items = 0;
+      return;
+    }
+  }
   int ni = 0;
   for (int e = 0; e < E; ++e) {
     const int c = off[e + 1] - off[e];
@@ -376,14 +301,15 @@ static __device__ void emit_work_items(const int32_t* off, int E, int n_max, TcW
   *n_items = ni;
 }
 
-__global__ void build_items_kernel(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items) {
+__global__ void build_items_kernel(const int32_t* off, int E, int n_max, int rows, TcWorkItem* items, int* n_items,
+                                   int* err) {
   griddep_sync();
-  if (threadIdx.x == 0 && blockIdx.x == 0) emit_work_items(off, E, n_max, items, n_items);
+  if (threadIdx.x == 0 && blockIdx.x == 0) emit_work_items(off, E, n_max, rows, items, n_items, err);
 }
 
-cudaError_t launch_build_items(const int32_t* off, int E, int n_max, TcWorkItem* items, int* n_items,
-                               cudaStream_t st) {
-  return launch_k(build_items_kernel, dim3(1), dim3(32), 0, st, off, E, n_max, items, n_items);
+cudaError_t launch_build_items(const int32_t* off, int E, int n_max, int rows, TcWorkItem* items, int* n_items,
+                               int* err, cudaStream_t st) {
+  return launch_k(build_items_kernel, dim3(1), dim3(32), 0, st, off, E, n_max, rows, items, n_items, err);
 }
 
 static int g_num_sms = 0;

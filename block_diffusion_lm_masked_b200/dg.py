@@ -84,7 +84,7 @@ def _load():
         "dg_launch_count": (ctypes.c_int64, []),
         "dg_renoise_count": (I32, [I32, I32, I32, F32, F32]),
         "dg_debug_bounded_wait": (I32, [P, I32, P]),
-        "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, I32, P, SZ, P, P]),
+        "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_scratch_bytes": (SZ, [I32, I32]),
         "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
@@ -318,12 +318,12 @@ def debug_gemm_scratch(x_rows, n_groups, device="cuda"):
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def debug_gemm_bf16(W, X, out, ld_out, err, scratch, W2=None, X_lo=None, group_off=None, out_lo=None, streamk=True,
+def debug_gemm_bf16(W, X, out, ld_out, err, scratch, W2=None, X_lo=None, group_off=None, out_lo=None,
                     stream=None):
     """One persistent tcgen05 GEMM launch (see include/dg_debug.h). W [groups][rows][K]."""
     G, rows, K = W.shape
     _check(lib.dg_debug_gemm_bf16(_ptr(W), _ptr(W2), rows, G, _ptr(X), _ptr(X_lo), X.shape[0], K, _ptr(group_off),
-                                  _ptr(out), _ptr(out_lo), ld_out, 1 if streamk else 0, _ptr(scratch),
+                                  _ptr(out), _ptr(out_lo), ld_out, _ptr(scratch),
                                   scratch.numel(), _ptr(err), _stream(stream)))
 
 

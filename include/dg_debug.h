@@ -75,14 +75,15 @@ const char* dg_kernel_name(int32_t kind);
  * [n_groups + 1], or NULL for one group of x_rows rows).  W is [n_groups][rows][K].
  * W2 NULL: out (fp32, row stride ld_out) = acc.  W2 given (same shape as W): out / out_lo
  * (bf16 hi / lo, out_lo nullable) = silu(acc) * acc2, acc2 the same sum over W2.
- * streamk: 1 lets the launch split tiles across CTAs (when there are at least as many
- * tiles as SMs), 0 keeps one tile per CTA and turn.  K % 64 == 0, rows >= 1.
- * d_scratch: 256-byte aligned, dg_debug_gemm_scratch_bytes(x_rows, n_groups) bytes,
- * zero-filled once before its first use.  d_err: device int32 error word. */
+ * Groups are cut into work items of at most 128 rows, as in the pass's expert GEMMs;
+ * offsets that decrease or leave [0, x_rows] launch no tile and set the error word to 5.
+ * K % 64 == 0, rows >= 1.  d_scratch: 256-byte aligned,
+ * dg_debug_gemm_scratch_bytes(x_rows, n_groups) bytes (the work list).  d_err: device
+ * int32 error word. */
 size_t dg_debug_gemm_scratch_bytes(int32_t x_rows, int32_t n_groups);
 dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_t n_groups, const void* X,
                              const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off, void* out,
-                             void* out_lo, int32_t ld_out, int32_t streamk, void* d_scratch, size_t scratch_bytes,
+                             void* out_lo, int32_t ld_out, void* d_scratch, size_t scratch_bytes,
                              int32_t* d_err, dg_stream stream);
 
 /* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
