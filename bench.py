@@ -138,7 +138,7 @@ REF_BUDGET_S = 90.0
 # DRAM bytes (read + write) of one gate/up GEMM launch from an ncu capture of this
 # workload, valid only for the kernel source it was taken on (sha256 prefix of
 # k_tc_gemm.cu); any other source reports null.
-NCU_TRAFFIC = {"layer1_bf16": ("47b56d50d45be312", 467.090688e6 + 6.504448e6)}
+NCU_TRAFFIC = {"layer1_bf16": ("8f9740b8fc51d669", 457.380608e6 + 6.031104e6)}
 
 
 def _ncu_traffic(workload):
