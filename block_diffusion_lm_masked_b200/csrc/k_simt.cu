@@ -5,8 +5,12 @@
 // fp32 model (tcgen05 has no fp32 operand kind).
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include "dg_common.cuh"
 #include "dg_kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace dg {
 
@@ -292,33 +296,47 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
 // Per token: x += sum of the output-projection partials (fixed order); xn = x / rms(x)
 // in fp32; router logits l[e] = xn . w_router[e] (fp32); the k largest (ties to the
 // lower expert id) and their softmax weights.  xn is also stored (hi/lo) as the expert
-// input.  CTA = RTF_TOK tokens, RTF_THREADS threads; each warp takes two experts at a
-// time and keeps eight float4 loads of router weights in flight.
-constexpr int RTF_TOK = 4;
-constexpr int RTF_THREADS = 512;
+// input.
+//
+// A cluster of RT_G CTAs takes RT_TOK tokens and splits the experts among its CTAs, so
+// each CTA streams only E / RT_G rows of the router matrix: CTA r adds the residual and
+// normalises its own RT_TOK / RT_G tokens, the normalised rows are shared through
+// distributed shared memory, every CTA computes its experts' logits for all RT_TOK
+// tokens (one expert per warp, eight float4 loads per lane in flight), and CTA r runs
+// the top-k of its own tokens over the logits of all CTAs.  Each logit is one lane-
+// strided fp32 dot product followed by a warp sum, as in a single-CTA version.
+constexpr int RT_G = 4;
+constexpr int RT_TOK = 8;
+constexpr int RT_OWN = RT_TOK / RT_G;
+constexpr int RT_THREADS = 512;
 template <typename T>
-__global__ void __launch_bounds__(RTF_THREADS) router_fused_kernel(
+__global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
     const float* __restrict__ wr, int n, int H, int E, int k, float eps, float* __restrict__ logits_out,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, T* __restrict__ xn, T* __restrict__ xn_lo) {
   griddep_sync();
-  extern __shared__ float sm[];  // xs[RTF_TOK][H], lg[RTF_TOK][E]
-  float* xs = sm;
-  float* lg = sm + RTF_TOK * H;
-  __shared__ float inv_s[RTF_TOK];
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int Eg = E / RT_G;
+  extern __shared__ float sm[];
+  float* own = sm;                  // [RT_OWN][H] this CTA's normalised rows
+  float* xs = own + RT_OWN * H;     // [RT_TOK][H] the cluster's normalised rows
+  float* lg = xs + RT_TOK * H;      // [RT_TOK][Eg] this CTA's experts' logits
+  __shared__ float inv_s[RT_OWN];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NW = RTF_THREADS / 32;
-  const int t0 = blockIdx.x * RTF_TOK;
-  const int nt = min(RTF_TOK, n - t0);
+  constexpr int NW = RT_THREADS / 32;
+  const int t0 = (int)(blockIdx.x / RT_G) * RT_TOK;
+  const int nt = min(RT_TOK, n - t0);
+  const int o0 = t0 + rank * RT_OWN;
+  const int no = max(0, min(RT_OWN, n - o0));
   const int H4 = H / 4;
-  // residual add of the partials (float4, all loads of an element issued together)
+  // residual add of the partials for the owned tokens
   {
-    float4* x4 = reinterpret_cast<float4*>(x + (size_t)t0 * H);
-    const float4* p4 = reinterpret_cast<const float4*>(parts + (size_t)t0 * H);
+    float4* x4 = reinterpret_cast<float4*>(x + (size_t)o0 * H);
+    const float4* p4 = reinterpret_cast<const float4*>(parts + (size_t)o0 * H);
     const size_t ps4 = part_stride / 4;
-    float4* xs4 = reinterpret_cast<float4*>(xs);
-#pragma unroll 2
-    for (int i = threadIdx.x; i < nt * H4; i += RTF_THREADS) {
+    float4* own4 = reinterpret_cast<float4*>(own);
+    for (int i = threadIdx.x; i < no * H4; i += RT_THREADS) {
       float4 v = x4[i];
       for (int s = 0; s < n_parts; ++s) {
         const float4 a = p4[s * ps4 + i];
@@ -328,78 +346,86 @@ __global__ void __launch_bounds__(RTF_THREADS) router_fused_kernel(
         v.w += a.w;
       }
       x4[i] = v;
-      xs4[i] = v;
+      own4[i] = v;
     }
   }
   __syncthreads();
-  if (warp < RTF_TOK) {
+  if (warp < no) {
     float ss = 0.0f;
-    if (warp < nt)
-      for (int h = lane; h < H; h += 32) ss += xs[warp * H + h] * xs[warp * H + h];
+    for (int h = lane; h < H; h += 32) ss += own[warp * H + h] * own[warp * H + h];
     ss = warp_sum(ss);
     if (lane == 0) inv_s[warp] = 1.0f / sqrtf(ss / (float)H + eps);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < nt * H; i += RTF_THREADS) {
-    const float v = xs[i] * inv_s[i / H];
-    xs[i] = v;
-    store_act(xn, xn_lo, (size_t)t0 * H + i, v);
+  for (int i = threadIdx.x; i < no * H; i += RT_THREADS) {
+    const float v = own[i] * inv_s[i / H];
+    own[i] = v;
+    store_act(xn, xn_lo, (size_t)o0 * H + i, v);
+  }
+  cl.sync();  // every CTA's rows are normalised
+  for (int r = 0; r < RT_G; ++r) {
+    const int nr = max(0, min(RT_OWN, nt - r * RT_OWN));
+    const float4* src = reinterpret_cast<const float4*>(cl.map_shared_rank(own, r));
+    float4* dst = reinterpret_cast<float4*>(xs + (size_t)r * RT_OWN * H);
+    for (int i = threadIdx.x; i < nr * H4; i += RT_THREADS) dst[i] = src[i];
   }
   __syncthreads();
   const float4* xs4 = reinterpret_cast<const float4*>(xs);
-  for (int e0 = 2 * warp; e0 < E; e0 += 2 * NW) {
-    const int e1 = min(e0 + 1, E - 1);
-    const float4* w0 = reinterpret_cast<const float4*>(wr + (size_t)e0 * H);
-    const float4* w1 = reinterpret_cast<const float4*>(wr + (size_t)e1 * H);
-    float a0[RTF_TOK] = {}, a1[RTF_TOK] = {};
-    for (int i0 = lane; i0 < H4; i0 += 32 * 4) {
-      float4 u0[4], u1[4];
+  for (int j = warp; j < Eg; j += NW) {
+    const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)(rank * Eg + j) * H);
+    float acc[RT_TOK] = {};
+    for (int i0 = lane; i0 < H4; i0 += 32 * 8) {
+      float4 u[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + 32 * u;
-        const bool in = i < H4;
-        u0[u] = in ? w0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        u1[u] = in ? w1[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < 8; ++q) {
+        const int i = i0 + 32 * q;
+        u[q] = i < H4 ? w4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + 32 * u;
+      for (int q = 0; q < 8; ++q) {
+        const int i = i0 + 32 * q;
         if (i < H4) {
 #pragma unroll
-          for (int a = 0; a < RTF_TOK; ++a) {
-            const float4 v = xs4[a * H4 + i];
-            a0[a] = fmaf(u0[u].x, v.x, fmaf(u0[u].y, v.y, fmaf(u0[u].z, v.z, fmaf(u0[u].w, v.w, a0[a]))));
-            a1[a] = fmaf(u1[u].x, v.x, fmaf(u1[u].y, v.y, fmaf(u1[u].z, v.z, fmaf(u1[u].w, v.w, a1[a]))));
+          for (int a = 0; a < RT_TOK; ++a) {
+            if (a < nt) {
+              const float4 v = xs4[a * H4 + i];
+              acc[a] = fmaf(u[q].x, v.x, fmaf(u[q].y, v.y, fmaf(u[q].z, v.z, fmaf(u[q].w, v.w, acc[a]))));
+            }
           }
         }
       }
     }
 #pragma unroll
-    for (int a = 0; a < RTF_TOK; ++a) {
-      const float r0 = warp_sum(a0[a]);
-      const float r1 = warp_sum(a1[a]);
-      if (lane == 0) {
-        lg[a * E + e0] = r0;
-        if (e0 + 1 < E) lg[a * E + e0 + 1] = r1;
-      }
+    for (int a = 0; a < RT_TOK; ++a) {
+      const float r = warp_sum(acc[a]);
+      if (lane == 0) lg[a * Eg + j] = r;
     }
   }
-  __syncthreads();
-  if (logits_out)
-    for (int i = threadIdx.x; i < nt * E; i += RTF_THREADS) logits_out[(size_t)t0 * E + i] = lg[i];
-  // top-k: warp a < nt selects for token a
-  if (warp < nt) {
-    const float* l = lg + warp * E;
+  cl.sync();  // every CTA's logits are in place
+  // top-k: warp w < no selects for owned token w; lane takes experts lane + 32 i
+  if (warp < no) {
+    const int a = rank * RT_OWN + warp;  // token within the cluster
+    float l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = -INFINITY;
+      if (e < E) l[i] = cl.map_shared_rank(lg, e / Eg)[a * Eg + e % Eg];
+    }
+    if (logits_out)
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) logits_out[(size_t)(t0 + a) * E + lane + 32 * i] = l[i];
     float chosen[16];
     int chosen_id[16];
     unsigned taken = 0u;  // bit i: entry lane + 32 i already chosen
     for (int j = 0; j < k; ++j) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
+#pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || l[e] > bv || (l[e] == bv && e < bi))) {
-          bv = l[e];
+        if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || l[i] > bv || (l[i] == bv && e < bi))) {
+          bv = l[i];
           bi = e;
         }
       }
@@ -420,11 +446,12 @@ __global__ void __launch_bounds__(RTF_THREADS) router_fused_kernel(
       float den = 0.0f;
       for (int j = 0; j < k; ++j) den += expf(chosen[j] - chosen[0]);
       for (int j = 0; j < k; ++j) {
-        topk_idx[(size_t)(t0 + warp) * k + j] = chosen_id[j];
-        topk_w[(size_t)(t0 + warp) * k + j] = expf(chosen[j] - chosen[0]) / den;
+        topk_idx[(size_t)(t0 + a) * k + j] = chosen_id[j];
+        topk_w[(size_t)(t0 + a) * k + j] = expf(chosen[j] - chosen[0]) / den;
       }
     }
   }
+  cl.sync();  // no CTA leaves while another still reads its shared memory
 }
 
 template <typename T>
@@ -432,11 +459,13 @@ cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_
                                 int n, int H, int E, int k, float eps, float* logits, int32_t* topk_idx, float* topk_w,
                                 T* xn, T* xn_lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  if (E > 256 || k > 16 || k > E || (H % 4) != 0) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)RTF_TOK * (H + E) * sizeof(float);
+  if (E > 256 || E % RT_G != 0 || k > 16 || k > E || (H % 4) != 0) return cudaErrorInvalidValue;
+  const size_t smem = ((size_t)(RT_OWN + RT_TOK) * H + (size_t)RT_TOK * (E / RT_G)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_k(router_fused_kernel<T>, dim3((n + RTF_TOK - 1) / RTF_TOK), dim3(RTF_THREADS), smem, st, x, parts, n_parts, part_stride, w_router, n, H, E, k, eps, logits, topk_idx, topk_w, xn, xn_lo);
+  const int clusters = (n + RT_TOK - 1) / RT_TOK;
+  return launch_k_cluster(router_fused_kernel<T>, dim3(clusters * RT_G), dim3(RT_THREADS), smem, st, RT_G, x, parts,
+                          n_parts, part_stride, w_router, n, H, E, k, eps, logits, topk_idx, topk_w, xn, xn_lo);
 }
 
 // ---------------------------------------------------------------- expert histogram + stable permutation
@@ -657,29 +686,35 @@ __global__ void update_partial_kernel(const float* __restrict__ logits, int V, i
   float m = -INFINITY, s = 0.0f;
   int a = 0x7fffffff;
   const int stride = blockDim.x * 4;
-  for (int i0 = lo + threadIdx.x * 4; i0 < hi; i0 += 4 * stride) {
-    float4 v4[4];
+  constexpr int VEC = 8;  // float4 loads in flight per thread
+  for (int i0 = lo + threadIdx.x * 4; i0 < hi; i0 += VEC * stride) {
+    float4 v4[VEC];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < VEC; ++u) {
       const int i = i0 + u * stride;
       v4[u] = (i < hi) ? *reinterpret_cast<const float4*>(lg + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
+    // this chunk's max and first argmax (elements in index order), then its sum of exp
+    float cm = -INFINITY;
+    int ca = 0x7fffffff;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * stride;
+    for (int u = 0; u < VEC; ++u) {
       const float v[4] = {v4[u].x, v4[u].y, v4[u].z, v4[u].w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float xv = v[q];
-        if (xv > m) {
-          s = s * __expf(m - xv) + 1.0f;
-          m = xv;
-          a = i + q;
-        } else if (xv != -INFINITY) {
-          s += __expf(xv - m);
+      for (int q = 0; q < 4; ++q)
+        if (v[q] > cm) {
+          cm = v[q];
+          ca = i0 + u * stride + q;
         }
-      }
     }
+    if (cm == -INFINITY) continue;
+    float cs = 0.0f;
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) {
+      cs += __expf(v4[u].x - cm) + __expf(v4[u].y - cm);
+      cs += __expf(v4[u].z - cm) + __expf(v4[u].w - cm);
+    }
+    upd_merge(m, s, a, cm, cs, ca);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
