@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
                                                        int32_t* __restrict__ union_out, int item_rows,
                                                        TcWorkItem* __restrict__ items, int* __restrict__ n_items) {
   griddep_sync();
-  __shared__ int cnt[PM_EMAX], base[PM_EMAX], run[PM_EMAX];
+  __shared__ int cnt[PM_EMAX], base[PM_EMAX], run[PM_EMAX], ibase[PM_EMAX];
   __shared__ int wcnt[32][PM_EMAX];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0, run[e] = 0;
@@ -489,31 +489,57 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
     if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0, u = 0;
-    for (int e = 0; e < E; ++e) {
-      base[e] = acc;
-      offsets[e] = acc;
-      counts[e] = cnt[e];
-      acc += cnt[e];
-      u += cnt[e] > 0;
+  if (warp == 0) {
+    // exclusive scans of the counts and of the work items per expert: lane l holds
+    // experts 8l .. 8l + 7
+    constexpr int PER = PM_EMAX / 32;
+    int c[PER], rows_l = 0, items_l = 0, used_l = 0;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int e = lane * PER + q;
+      c[q] = e < E ? cnt[e] : 0;
+      rows_l += c[q];
+      items_l += (c[q] + item_rows - 1) / item_rows;
+      used_l += c[q] > 0;
     }
-    offsets[E] = acc;
-    *union_out = u;
-    // work list of the grouped expert GEMMs: each expert's rows in items of <= item_rows
-    int ni = 0;
-    for (int e = 0; e < E; ++e)
-      for (int r = 0; r < cnt[e]; r += item_rows) {
-        TcWorkItem it;
-        it.group = e;
-        it.row0 = base[e] + r;
-        it.rows = min(item_rows, cnt[e] - r);
-        it.pad = 0;
-        items[ni++] = it;
+    int rows_x = rows_l, items_x = items_l;  // inclusive scans over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int r2 = __shfl_up_sync(0xffffffffu, rows_x, o);
+      const int i2 = __shfl_up_sync(0xffffffffu, items_x, o);
+      if (lane >= o) rows_x += r2, items_x += i2;
+    }
+    int acc = rows_x - rows_l, iacc = items_x - items_l;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int e = lane * PER + q;
+      if (e < E) {
+        base[e] = acc;
+        ibase[e] = iacc;
+        offsets[e] = acc;
+        counts[e] = c[q];
       }
-    *n_items = ni;
+      acc += c[q];
+      iacc += (c[q] + item_rows - 1) / item_rows;
+    }
+    const int used = warp_sum((float)used_l) + 0.5f;
+    if (lane == 31) {
+      offsets[E] = rows_x;
+      *n_items = items_x;
+    }
+    if (lane == 0) *union_out = used;
   }
   __syncthreads();
+  // work list of the grouped expert GEMMs: each expert's rows in items of <= item_rows
+  for (int e = tid; e < E; e += blockDim.x)
+    for (int r = 0, i = ibase[e]; r < cnt[e]; r += item_rows, ++i) {
+      TcWorkItem it;
+      it.group = e;
+      it.row0 = base[e] + r;
+      it.rows = min(item_rows, cnt[e] - r);
+      it.pad = 0;
+      items[i] = it;
+    }
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int c0 = 0; c0 < total; c0 += blockDim.x) {
     const int a = c0 + tid;
