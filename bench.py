@@ -287,7 +287,9 @@ def main():
         torch.cuda.synchronize(dev)
         if profile:
             dg.profile_enable(False)
-        return sum(a.elapsed_time(b) for a, b in ev), dg.launch_count() - l0
+        per = [a.elapsed_time(b) for a, b in ev]
+        timed.last = per
+        return sum(per), dg.launch_count() - l0
 
     if world > 1:
         dist.barrier()
@@ -302,6 +304,50 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
         dist.barrier()
+
+    step_median_us = statistics.median(timed.last) * 1e3
+
+    # the pass alone (no update), same timing rules
+    def pass_only(s):
+        dg.denoise_pass(model, cache, canvas_in, logits, ws)
+    k2 = min(args.steps, 500)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k2)]
+    for s_ in range(k2):
+        flush.zero_()
+        ev2[s_][0].record(stream)
+        pass_only(s_)
+        ev2[s_][1].record(stream)
+    torch.cuda.synchronize(dev)
+    pass_us = [a.elapsed_time(b) * 1e3 for a, b in ev2]
+
+    # the step replayed from a CUDA graph (host launch cost removed), same flush rule
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step(0)  # warm the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g):
+            step(0)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k2)]
+        for s_ in range(k2):
+            flush.zero_()
+            ev3[s_][0].record(stream)
+            g.replay()
+            ev3[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+        dg.device_status(ws)
+        gus = [a.elapsed_time(b) * 1e3 for a, b in ev3]
+        graph = {"median_us": statistics.median(gus), "mean_us": sum(gus) / len(gus), "replays": k2}
+        del g
+    except Exception as e:  # report, do not fail the bench line
+        graph = {"unavailable": repr(e)[:200]}
 
     # per-kernel breakdown with CUDA events on the launching stream (separate timed run,
     # at most 200 steps: it records an event pair around every launch)
@@ -352,6 +398,25 @@ def main():
                 "frac": achieved / hbm, "traffic": _ncu_traffic(name), "peak_source": f"{peak_src} hbm_gbs",
                 "bytes_per_launch": per_launch}
 
+    # the other big kernels against their own bounds (algorithmic units per launch / average time)
+    kroof = {}
+    def _hbm(kname, nbytes_launch):
+        if kname in kern:
+            a = nbytes_launch / (kern[kname]["avg_us"] * 1e-6) / 1e9
+            kroof[kname] = {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+                            "bytes_per_launch": nbytes_launch}
+    if len(set(unions_h)) == 1:
+        _hbm("gemm_down", RF.down_bytes(cfg, unions_h[0], C * cfg["top_k"]))
+    _hbm("gemm_vocab", RF.vocab_bytes(cfg, C))
+    _hbm("update_partial", RF.update_bytes(cfg, C))
+    if "attention" in kern:
+        fl = 4.0 * C * cfg["n_q_heads"] * cfg["head_dim"] * (P + C)
+        a = fl / (kern["attention"]["avg_us"] * 1e-6) / 1e12
+        kroof["attention"] = {"bound": "tensor", "achieved": a, "peak": tf_burst, "unit": "TFLOP/s",
+                              "frac": a / tf_burst, "flops_per_launch": fl,
+                              "note": "algorithmic QK^T and PV FLOPs; the kernel issues about twice as many "
+                                      "(query and probabilities as bf16 hi + lo terms)"}
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "pass_latency_us": ms_step * 1e3,
@@ -364,6 +429,10 @@ def main():
                           "bytes": nbytes, "bound": "hbm" if nbytes / (hbm * 1e9) > flops / (tf_burst * 1e12)
                           else "tensor", "peak_source": peak_src},
         "kernels": kern,
+        "kernel_rooflines": kroof,
+        "step_median_us": step_median_us,
+        "pass_only_us": {"median": statistics.median(pass_us), "mean": sum(pass_us) / len(pass_us), "steps": k2},
+        "graph_step_us": graph,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": C * 4, "d2h_bytes_per_step": C * 4},
         "gpu_launches": launches,
         "clocks": clocks,

@@ -186,22 +186,32 @@ def test_chained8_full_size(dg):
 
 
 def test_large4_full_size(dg):
+    """First passes layer by layer and their updates against the oracle, on up to three
+    noise canvases until one is compared in full (with 8 of 128 experts per token a
+    near-tie routing difference in the first layers is common, and it turns the rest
+    of that pass into a structure-only check); then the 8-pass run for its properties."""
     cfg = CF.CONFIGS["large4_bf16"]
     P, C, S = cfg["prefix"], cfg["canvas"], cfg["steps"]
     st = PL.Setup(cfg, P, capacity=P + C)
     st.ws = st.workspace(C)
-    noise = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
     n0 = O.renoise_count(C, S, 0, cfg["renoise_start"], cfg["renoise_end"])
-    taps, logits, nxt, conf = _pass(dg, st, noise, n0, 0)
-    logits_o, taps_o = O.denoise_pass(st.host, st.ocache, noise, st.prec)
-    upd = O.canvas_update(logits_o, n0, synth.SEED_RENOISE, 0)
-    report = []
-    exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, report)
-    PL.compare_update(nxt, conf, upd, exempt, n0)
-    print("large4 first pass:", report, "exempt", len(exempt))
-    unions = taps["unions"].cpu().numpy()
-    assert (unions >= cfg["top_k"]).all() and (unions <= cfg["n_experts"]).all()
-    assert [t["union"] for t in taps_o] == list(unions) or exempt
+    full = False
+    for c in range(3):
+        canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])
+        taps, logits, nxt, conf = _pass(dg, st, canvas, n0, 0)
+        logits_o, taps_o = O.denoise_pass(st.host, st.ocache, canvas, st.prec)
+        upd = O.canvas_update(logits_o, n0, synth.SEED_RENOISE, 0)
+        report = []
+        exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, report)
+        PL.compare_update(nxt, conf, upd, exempt, n0)
+        print(f"large4 canvas {c}:", report, "exempt", len(exempt), flush=True)
+        unions = taps["unions"].cpu().numpy()
+        assert (unions >= cfg["top_k"]).all() and (unions <= cfg["n_experts"]).all()
+        if report[-1]["logits"] is not None:
+            full = True
+            break
+    assert full, "no pass of three compared in full"
+    noise = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
     # the 8-pass run: untouched prefix, tokens in range, bit-identical repeat
     before = [(k[:, :P].clone(), v[:, :, :P].clone()) for k, v in zip(st.cache.k, st.cache.vt)]
     st.model.set_taps(None)
