@@ -29,7 +29,8 @@ Readings where the pages are silent (each one listed in the design notes):
   k chosen logits; SwiGLU experts; untied embedding / output matrices;
   confidence = largest softmax probability (temperature 1); every position
   takes its argmax (ties to the lowest id), then the n lowest-confidence
-  positions (ties to the lower position) get a fresh random token.
+  positions (ties to the lower position) get a fresh random token.  The
+  masked-diffusion variant (canvas_update_masked) states its own readings.
 
 Precision model.  The pages fix no precision beyond bf16 weights, so the oracle
 follows the kernel's storage precision, because later integer decisions (routing,
@@ -454,6 +455,73 @@ def canvas_update(logits: np.ndarray, n_renoise: int, seed: int, step: int) -> d
         cut_margin = np.where(sel, lo_out - lc, lc - hi_in)
     return dict(canvas=canvas.astype(np.int32), argmax=argmax.astype(np.int32), conf=conf,
                 top_margin=top_margin, renoised=chosen, cut_margin=cut_margin)
+
+
+def canvas_update_masked(logits: np.ndarray, canvas: np.ndarray, n_keep: int, mask_id: int) -> dict:
+    """Masked-diffusion update: fill [MASK] positions, which then stay fixed.
+
+    [DG-explainer] "First attempt: masked diffusion": noise is a [MASK] placeholder; the
+    model predicts the word and fills it in, and a filled position is locked from then on.
+    Readings (the page gives no more): a position holding any token other than
+    `mask_id` is locked and keeps it; a masked position's candidate is its argmax over
+    every token except `mask_id` (ties to the lowest id), its confidence that token's
+    softmax probability over all V logits; of the M masked positions the
+    min(n_keep, M) least confident stay masked (ties to the lower position) and the
+    others take their candidates.
+
+    Returns the canvas, the candidates, the confidences, each position's top-1/top-2
+    margin among the candidate logits, the positions kept masked (sorted) and each masked
+    position's log-confidence distance to the cut (inf elsewhere).
+    """
+    C, V = logits.shape
+    canvas = np.asarray(canvas).astype(np.int64)
+    m = logits.max(axis=1)
+    denom = np.exp(logits - m[:, None]).sum(axis=1)
+    cand_logits = logits.copy()
+    cand_logits[:, mask_id] = -np.inf
+    cand = np.argmax(cand_logits, axis=1).astype(np.int64)      # first (lowest) id on ties
+    conf = np.exp(cand_logits[np.arange(C), cand] - m) / denom
+    srt = np.sort(cand_logits, axis=1)
+    top_margin = srt[:, -1] - srt[:, -2] if V > 2 else np.full(C, np.inf)
+    masked = np.nonzero(canvas == mask_id)[0]                    # ascending positions
+    keep = min(int(n_keep), len(masked))
+    order = masked[np.argsort(conf[masked], kind="stable")]      # ties: lower position first
+    kept = np.sort(order[:keep])
+    out = canvas.copy()
+    out[masked] = cand[masked]
+    out[kept] = mask_id
+    lc = np.log(conf)
+    cut_margin = np.full(C, np.inf)
+    if 0 < keep < len(masked):
+        lo_out = lc[order[keep]]        # least confident filled position
+        hi_in = lc[order[keep - 1]]     # most confident position kept masked
+        sel = np.zeros(C, dtype=bool)
+        sel[kept] = True
+        cut_margin[masked] = np.where(sel[masked], lo_out - lc[masked], lc[masked] - hi_in)
+    return dict(canvas=out.astype(np.int32), argmax=cand.astype(np.int32), conf=conf, top_margin=top_margin,
+                kept=kept, cut_margin=cut_margin)
+
+
+def generate_canvas_masked(model, cache: Cache, C: int, S: int, keep_start: float, keep_end: float, mask_id: int,
+                           prec: Precision, append: bool, record=None):
+    """S passes of masked diffusion from an all-[MASK] canvas, then (optionally) append.
+
+    [DG-explainer] "First attempt: masked diffusion" with the pass loop and the append of
+    "Uniform State Diffusion" / "Long-form text: chaining canvases".  After pass s the
+    number of positions that stay masked is at most renoise_count(C, S, s, keep_start,
+    keep_end).  Returns (canvas, cache).
+    """
+    cur = np.full(C, mask_id, dtype=np.int32)
+    for s in range(S):
+        logits, taps = denoise_pass(model, cache, cur, prec)
+        n = renoise_count(C, S, s, keep_start, keep_end)
+        upd = canvas_update_masked(logits, cur, n, mask_id)
+        if record is not None:
+            record.append(dict(step=s, canvas_in=cur.copy(), logits=logits, taps=taps, update=upd, n=n))
+        cur = upd["canvas"]
+    if append:
+        cache = prefill_append(model, cache, cur, prec)
+    return cur, cache
 
 
 def generate_canvas(model, cache: Cache, canvas: np.ndarray, S: int, r_start: float, r_end: float,

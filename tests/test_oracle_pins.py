@@ -393,6 +393,70 @@ def test_canvas_update_renoise_set_brute_force():
     assert all(u["cut_margin"] >= 0)
 
 
+def _masked_example():
+    rec = {}
+    with open(golden_path("masked_update_example.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, _, rest = line.partition(" ")
+            rec[key] = rest.strip()
+    logits = np.array([[float(v) for v in row.split()] for row in rec["logits"].split("|")])
+    return (logits, np.array(rec["canvas_in"].split(), dtype=np.int64), int(rec["mask_id"]), int(rec["n_keep"]),
+            np.array(rec["canvas_out"].split(), dtype=np.int64), rec["conf"].split())
+
+
+def test_masked_update_worked_example():
+    logits, cin, mask_id, n_keep, cout, conf = _masked_example()
+    got = O.canvas_update_masked(logits, cin, n_keep, mask_id)
+    np.testing.assert_array_equal(got["canvas"], cout)
+    for i, c in enumerate(conf):
+        if c != "-":
+            assert abs(got["conf"][i] - float(c)) < 5e-7
+    np.testing.assert_array_equal(got["kept"], [0])
+
+
+def test_masked_update_special_cases():
+    rng = np.random.default_rng(31)
+    C, V, mask_id = 40, 97, 96
+    logits = rng.standard_normal((C, V)) * 3.0
+    canvas = np.where(rng.random(C) < 0.6, mask_id, rng.integers(0, mask_id, C))
+    masked = canvas == mask_id
+    # n_keep = 0: every masked position takes its best non-mask token; locked ones keep theirs
+    got = O.canvas_update_masked(logits, canvas, 0, mask_id)
+    want = np.where(masked, np.argmax(logits[:, :mask_id], axis=1), canvas)
+    np.testing.assert_array_equal(got["canvas"], want)
+    # n_keep >= M: nothing changes
+    np.testing.assert_array_equal(O.canvas_update_masked(logits, canvas, C, mask_id)["canvas"], canvas)
+    # the mask id is never a fill value, even where it has the largest logit
+    big = logits.copy()
+    big[:, mask_id] = 50.0
+    g2 = O.canvas_update_masked(big, canvas, 0, mask_id)
+    np.testing.assert_array_equal(g2["canvas"], want)
+    assert np.all(g2["conf"] < 1e-15)
+    # a single dominant logit: confidence 1
+    one = np.full((C, V), -1e4)
+    one[np.arange(C), np.arange(C) % mask_id] = 0.0
+    assert np.allclose(O.canvas_update_masked(one, canvas, 0, mask_id)["conf"], 1.0)
+
+
+def test_masked_schedule_unmasks_to_zero_and_locks():
+    """From an all-[MASK] canvas, the keep counts renoise_count(C, S, s, (S-1)/S, 0) leave
+    exactly that many positions masked after pass s (C/S fewer per pass), none at the
+    end, and a filled position never changes again."""
+    rng = np.random.default_rng(32)
+    C, V, S, mask_id = 64, 50, 8, 49
+    cur = np.full(C, mask_id)
+    for s in range(S):
+        n = O.renoise_count(C, S, s, (S - 1) / S, 0.0)
+        nxt = O.canvas_update_masked(rng.standard_normal((C, V)), cur, n, mask_id)["canvas"]
+        filled = cur != mask_id
+        np.testing.assert_array_equal(nxt[filled], cur[filled])
+        assert int((nxt == mask_id).sum()) == n == C * (S - 1 - s) // S
+        cur = nxt
+    assert not np.any(cur == mask_id)
+
+
 def test_renoise_schedule_golden():
     g = {r[0]: [int(v) for v in r[1:]] for r in _read_golden("renoise_schedule.txt")}
     assert [O.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]
