@@ -694,9 +694,31 @@ extern "C" dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dg::UpdPart* part = reinterpret_cast<dg::UpdPart*>(static_cast<char*>(d_ws) + 256);
   const int splits = dg::update_splits(C, V);
-  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, part, st));
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, -1, part, st));
   LAUNCH(DG_K_UPDATE_SELECT, st,
-         dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, st));
+         dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, -1, st));
+  return DG_OK;
+}
+
+extern "C" dg_status dg_canvas_update_masked(const float* d_logits, int32_t C, int32_t V, int32_t n_keep,
+                                             int32_t mask_id, int32_t* d_canvas, float* d_conf, void* d_ws,
+                                             size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(d_logits && d_canvas && d_ws, "logits / canvas / workspace is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(V > 1 && V % 4 == 0, "V must be a multiple of 4 and > 1");
+  DG_CHECK_ARG(mask_id >= 0 && mask_id < V, "mask_id must be in [0, V)");
+  DG_CHECK_ARG(n_keep >= 0 && n_keep <= C, "n_keep must be in [0, C]");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_logits) & 15) == 0, "logits must be 16-byte aligned");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_ws) & 255) == 0, "workspace must be 256-byte aligned");
+  if (ws_bytes < dg_update_workspace_bytes(C, V))
+    return fail(DG_ERR_CAPACITY, "workspace too small for the update: %zu < %zu", ws_bytes,
+                dg_update_workspace_bytes(C, V));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dg::UpdPart* part = reinterpret_cast<dg::UpdPart*>(static_cast<char*>(d_ws) + 256);
+  const int splits = dg::update_splits(C, V);
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, mask_id, part, st));
+  LAUNCH(DG_K_UPDATE_SELECT, st,
+         dg::launch_update_select(part, C, V, splits, n_keep, 0, 0, d_canvas, d_conf, mask_id, st));
   return DG_OK;
 }
 
@@ -726,6 +748,35 @@ extern "C" dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t
     const int n = renoise_count(C, S, step, r_start, r_end);
     if ((s = dg_canvas_update(d_logits, C, m->cfg.vocab, n, seed, (uint32_t)step, d_canvas, nullptr, d_ws, ws_bytes,
                               stream)) != DG_OK)
+      return s;
+  }
+  if (append) return dg_prefill_append(m, cache, d_canvas, C, d_ws, ws_bytes, stream);
+  return DG_OK;
+}
+
+extern "C" dg_status dg_generate_canvas_masked(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas, int32_t C,
+                                               int32_t S, float keep_start, float keep_end, int32_t mask_id,
+                                               int32_t append, float* d_logits, void* d_ws, size_t ws_bytes,
+                                               dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(d_canvas, "canvas is NULL");
+  DG_CHECK_ARG(S >= 1, "S must be >= 1");
+  DG_CHECK_ARG(keep_start >= 0.f && keep_start <= 1.f && keep_end >= 0.f && keep_end <= 1.f,
+               "keep fractions must be in [0,1]");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(mask_id >= 0 && mask_id < m->cfg.vocab, "mask_id must be in [0, vocab)");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  if ((int64_t)cache->len + C > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
+                cache->capacity);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LAUNCH(DG_K_UPDATE_SELECT, st, dg::launch_fill_i32(d_canvas, C, mask_id, st));
+  for (int step = 0; step < S; ++step) {
+    if ((s = dg_denoise_pass(m, cache, d_canvas, C, d_logits, d_ws, ws_bytes, stream)) != DG_OK) return s;
+    const int n = renoise_count(C, S, step, keep_start, keep_end);
+    if ((s = dg_canvas_update_masked(d_logits, C, m->cfg.vocab, n, mask_id, d_canvas, nullptr, d_ws, ws_bytes,
+                                     stream)) != DG_OK)
       return s;
   }
   if (append) return dg_prefill_append(m, cache, d_canvas, C, d_ws, ws_bytes, stream);

@@ -118,13 +118,17 @@ cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float
 struct UpdPart {
   float m;    // row max over the slice
   float s;    // sum of exp(l - m) over the slice
-  int a;      // first index attaining m
-  int pad;
+  int a;      // first index of the largest logit among the candidate ids
+  float m2;   // that logit (the ids other than an excluded one; m when nothing is excluded)
 };
 int update_splits(int C, int V);
-cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, UpdPart* part, cudaStream_t st);
+// excl >= 0: the candidate skips that id
+cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, int excl, UpdPart* part,
+                                  cudaStream_t st);
+// mask_id < 0: the re-noising update; mask_id >= 0: the masked-diffusion update
 cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
-                                 uint32_t step, int32_t* canvas, float* conf, cudaStream_t st);
+                                 uint32_t step, int32_t* canvas, float* conf, int mask_id, cudaStream_t st);
+cudaError_t launch_fill_i32(int32_t* p, int n, int32_t v, cudaStream_t st);
 
 cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 

@@ -84,8 +84,9 @@ extern "C" dg_status dg_canvas_update_noalloc(const float* d_logits, int32_t C, 
   dg_status s = scratch_for_current_device(&part);
   if (s != DG_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = dg::launch_update_partial(d_logits, C, V, splits, part, st);
-  if (e == cudaSuccess) e = dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, st);
+  cudaError_t e = dg::launch_update_partial(d_logits, C, V, splits, -1, part, st);
+  if (e == cudaSuccess)
+    e = dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, -1, st);
   if (e != cudaSuccess) {
     snprintf(msg, sizeof msg, "canvas update launch: %s", cudaGetErrorString(e));
     return dg::set_error(DG_ERR_CUDA, msg);

@@ -673,21 +673,28 @@ cudaError_t launch_combine_norm(const float* ys, const int32_t* inv, const float
 }
 
 // ---------------------------------------------------------------- canvas update
-__device__ __forceinline__ void upd_merge(float& m, float& s, int& a, float m2, float s2, int a2) {
-  if (m2 == -INFINITY) return;
+// (m, s): the largest logit and the sum of exp(l - m) over the ids seen
+__device__ __forceinline__ void ms_merge(float& m, float& s, float om, float os) {
+  if (om == -INFINITY) return;
   if (m == -INFINITY) {
-    m = m2, s = s2, a = a2;
+    m = om, s = os;
     return;
   }
-  if (m2 > m) {
-    s = s * expf(m - m2) + s2;
-    m = m2;
-    a = a2;
-  } else if (m2 < m) {
-    s += s2 * expf(m2 - m);
+  if (om > m) {
+    s = s * expf(m - om) + os;
+    m = om;
+  } else if (om < m) {
+    s += os * expf(om - m);
   } else {
-    s += s2;
-    a = min(a, a2);
+    s += os;
+  }
+}
+// (m2, a): the largest logit among the ids other than an excluded one and its first
+// index; merged by value, ties to the lower index
+__device__ __forceinline__ void cand_merge(float& m2, int& a, float om2, int oa) {
+  if (om2 > m2 || (om2 == m2 && oa < a)) {
+    m2 = om2;
+    a = oa;
   }
 }
 
@@ -701,15 +708,18 @@ int update_splits(int C, int V) {
 }
 
 // per (row, slice): max, first argmax and sum exp(l - max), one streaming pass
-__global__ void update_partial_kernel(const float* __restrict__ logits, int V, int splits, UpdPart* __restrict__ part) {
+// excl >= 0: the candidate (a, m2) skips that id (the masked-diffusion update never fills
+// with the mask token); excl < 0: the candidate is the plain first argmax (m2 = m)
+__global__ void update_partial_kernel(const float* __restrict__ logits, int V, int splits, int excl,
+                                      UpdPart* __restrict__ part) {
   griddep_sync();
-  __shared__ float sm[32], ss[32];
+  __shared__ float sm[32], ss[32], sm2[32];
   __shared__ int sa[32];
   const int row = blockIdx.x, sp = blockIdx.y;
   const int slice = ((V + splits - 1) / splits + 3) & ~3;
   const int lo = sp * slice, hi = min(V, lo + slice);
   const float* lg = logits + (size_t)row * V;
-  float m = -INFINITY, s = 0.0f;
+  float m = -INFINITY, s = 0.0f, m2 = -INFINITY;
   int a = 0x7fffffff;
   const int stride = blockDim.x * 4;
   constexpr int VEC = 8;  // float4 loads in flight per thread
@@ -740,25 +750,50 @@ __global__ void update_partial_kernel(const float* __restrict__ logits, int V, i
       cs += __expf(v4[u].x - cm) + __expf(v4[u].y - cm);
       cs += __expf(v4[u].z - cm) + __expf(v4[u].w - cm);
     }
-    upd_merge(m, s, a, cm, cs, ca);
+    float cm2 = cm;
+    int ca2 = ca;
+    if (excl >= 0 && excl >= i0 && excl < i0 + VEC * stride && (excl - i0) % stride < 4) {
+      // the excluded id lies in this chunk: its best other element, in index order
+      cm2 = -INFINITY;
+      ca2 = 0x7fffffff;
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) {
+        const float v[4] = {v4[u].x, v4[u].y, v4[u].z, v4[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int id = i0 + u * stride + q;
+          if (id != excl && v[q] > cm2) {
+            cm2 = v[q];
+            ca2 = id;
+          }
+        }
+      }
+    }
+    ms_merge(m, s, cm, cs);  // over every id
+    cand_merge(m2, a, cm2, ca2);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
-    upd_merge(m, s, a, m2, s2, a2);
+    const float om = __shfl_xor_sync(0xffffffffu, m, o);
+    const float os = __shfl_xor_sync(0xffffffffu, s, o);
+    const float om2 = __shfl_xor_sync(0xffffffffu, m2, o);
+    const int oa = __shfl_xor_sync(0xffffffffu, a, o);
+    ms_merge(m, s, om, os);
+    cand_merge(m2, a, om2, oa);
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) sm[warp] = m, ss[warp] = s, sa[warp] = a;
+  if (lane == 0) sm[warp] = m, ss[warp] = s, sm2[warp] = m2, sa[warp] = a;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w2 = 1; w2 < (int)(blockDim.x >> 5); ++w2) upd_merge(m, s, a, sm[w2], ss[w2], sa[w2]);
+    for (int w2 = 1; w2 < (int)(blockDim.x >> 5); ++w2) {
+      ms_merge(m, s, sm[w2], ss[w2]);
+      cand_merge(m2, a, sm2[w2], sa[w2]);
+    }
     UpdPart r;
     r.m = m;
     r.s = s;
     r.a = a;
-    r.pad = 0;
+    r.m2 = m2;
     part[(size_t)row * splits + sp] = r;
   }
 }
@@ -773,48 +808,94 @@ __device__ __forceinline__ uint64_t splitmix64_out(uint64_t seed, uint64_t n) {
 // merge slices, confidence = 1 / sum exp(l - max); every position takes its argmax, then
 // the n_renoise lowest-confidence positions (ties: lower position first) take a fresh
 // token: SplitMix64(seed) draw number (step << 32 | position), multiply-shift onto [0, V).
+// Masked mode (mask_id >= 0): positions holding a token other than mask_id keep it; a
+// masked position's candidate is its best token other than mask_id, with confidence
+// exp(m2 - m) / sum; of the M masked positions the min(n_renoise, M) least confident
+// (ties: lower position first) stay mask_id and the others take their candidates.
 __global__ void update_select_kernel(const UpdPart* __restrict__ part, int C, int V, int splits, int n_renoise,
                                      uint64_t seed, uint32_t step, int32_t* __restrict__ canvas,
-                                     float* __restrict__ conf) {
+                                     float* __restrict__ conf, int mask_id) {
   griddep_sync();
-  extern __shared__ float den[];  // [C]
+  extern __shared__ float den[];  // [C] sums (uniform) or confidences (masked), then [C] masked flags
+  int* is_m = reinterpret_cast<int*>(den + C);
+  __shared__ int n_masked;
   const int i = threadIdx.x;
-  float m = -INFINITY, s = 0.0f;
+  float m = -INFINITY, s = 0.0f, m2 = -INFINITY;
   int a = 0x7fffffff;
+  if (i == 0) n_masked = 0;
+  __syncthreads();
   if (i < C) {
-    for (int sp = 0; sp < splits; ++sp) {
-      const UpdPart q = part[(size_t)i * splits + sp];
-      upd_merge(m, s, a, q.m, q.s, q.a);
+    for (int sp0 = 0; sp0 < splits; sp0 += 8) {  // eight slices' partials in flight, merged in order
+      UpdPart q[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < splits) q[u] = part[(size_t)i * splits + sp0 + u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < splits) {
+          ms_merge(m, s, q[u].m, q[u].s);
+          cand_merge(m2, a, q[u].m2, q[u].a);
+        }
     }
-    den[i] = s;
+    if (mask_id < 0) {
+      den[i] = s;
+    } else {
+      den[i] = expf(m2 - m) / s;
+      is_m[i] = canvas[i] == mask_id;
+      if (is_m[i]) atomicAdd(&n_masked, 1);
+    }
   }
   __syncthreads();
   if (i < C) {
-    int rank = 0;
-    for (int j = 0; j < C; ++j) {
-      const float dj = den[j];
-      rank += (dj > s) || (dj == s && j < i);
+    if (mask_id < 0) {
+      int rank = 0;
+      for (int j = 0; j < C; ++j) {
+        const float dj = den[j];
+        rank += (dj > s) || (dj == s && j < i);
+      }
+      int tok = a;
+      if (rank < n_renoise) {
+        const uint64_t x = splitmix64_out(seed, ((uint64_t)step << 32) | (uint64_t)i);
+        tok = (int)(((x >> 32) * (uint64_t)V) >> 32);
+      }
+      canvas[i] = tok;
+      if (conf) conf[i] = 1.0f / s;
+    } else {
+      const float ci = den[i];
+      if (is_m[i]) {
+        int rank = 0;  // among the masked positions, by confidence, ties to the lower position
+        for (int j = 0; j < C; ++j) rank += is_m[j] && (den[j] < ci || (den[j] == ci && j < i));
+        const int keep = min(n_renoise, n_masked);
+        canvas[i] = rank < keep ? mask_id : a;
+      }
+      if (conf) conf[i] = ci;
     }
-    int tok = a;
-    if (rank < n_renoise) {
-      const uint64_t x = splitmix64_out(seed, ((uint64_t)step << 32) | (uint64_t)i);
-      tok = (int)(((x >> 32) * (uint64_t)V) >> 32);
-    }
-    canvas[i] = tok;
-    if (conf) conf[i] = 1.0f / s;
   }
 }
 
-cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, UpdPart* part, cudaStream_t st) {
+cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, int excl, UpdPart* part,
+                                  cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
-  return launch_k(update_partial_kernel, dim3(C, splits), dim3(256), 0, st, logits, V, splits, part);
+  return launch_k(update_partial_kernel, dim3(C, splits), dim3(256), 0, st, logits, V, splits, excl, part);
 }
 cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
-                                 uint32_t step, int32_t* canvas, float* conf, cudaStream_t st) {
+                                 uint32_t step, int32_t* canvas, float* conf, int mask_id, cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
   if (C > 1024) return cudaErrorInvalidValue;
   const int threads = (C + 31) & ~31;
-  return launch_k(update_select_kernel, dim3(1), dim3(threads), C * sizeof(float), st, part, C, V, splits, n_renoise, seed, step, canvas, conf);
+  return launch_k(update_select_kernel, dim3(1), dim3(threads), 2 * C * sizeof(float), st, part, C, V, splits,
+                  n_renoise, seed, step, canvas, conf, mask_id);
+}
+
+// ---------------------------------------------------------------- int32 fill
+__global__ void fill_i32_kernel(int32_t* p, int n, int32_t v) {
+  griddep_sync();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
+}
+cudaError_t launch_fill_i32(int32_t* p, int n, int32_t v, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  return launch_k(fill_i32_kernel, dim3((n + 255) / 256), dim3(256), 0, st, p, n, v);
 }
 
 // ---------------------------------------------------------------- timeout self-test

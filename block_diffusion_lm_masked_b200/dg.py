@@ -73,6 +73,9 @@ def _load():
         "dg_denoise_pass": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, P, SZ, P]),
         "dg_canvas_update": (I32, [P, I32, I32, I32, U64, U32, P, P, P, SZ, P]),
         "dg_canvas_update_noalloc": (I32, [P, I32, I32, I32, U64, U32, P, P, P]),
+        "dg_canvas_update_masked": (I32, [P, I32, I32, I32, I32, P, P, P, SZ, P]),
+        "dg_generate_canvas_masked": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, I32, I32, P, P, SZ,
+                                            P]),
         "dg_generate_canvas": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, U64, I32, P, P, SZ, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
@@ -282,6 +285,23 @@ def generate_canvas(model: Model, cache: KVCache, canvas: torch.Tensor, S: int, 
     _check(lib.dg_generate_canvas(model.handle, ctypes.byref(cache.s), _ptr(canvas), canvas.numel(), S, r_start,
                                   r_end, seed & 0xFFFFFFFFFFFFFFFF, 1 if append else 0, _ptr(logits), ws.ptr,
                                   ws.nbytes, _stream(stream)))
+
+
+def canvas_update_masked(logits: torch.Tensor, n_keep: int, mask_id: int, canvas: torch.Tensor, ws,
+                         conf: torch.Tensor | None = None, stream=None):
+    C, V = logits.shape
+    ptr = ws.ptr if isinstance(ws, Workspace) else ctypes.c_void_p(ws.data_ptr())
+    nb = ws.nbytes if isinstance(ws, Workspace) else ws.numel()
+    _check(lib.dg_canvas_update_masked(_ptr(logits), C, V, n_keep, mask_id, _ptr(canvas), _ptr(conf), ptr, nb,
+                                       _stream(stream)))
+
+
+def generate_canvas_masked(model: Model, cache: KVCache, canvas: torch.Tensor, S: int, keep_start: float,
+                           keep_end: float, mask_id: int, append: bool, logits: torch.Tensor, ws: Workspace,
+                           stream=None):
+    _check(lib.dg_generate_canvas_masked(model.handle, ctypes.byref(cache.s), _ptr(canvas), canvas.numel(), S,
+                                         keep_start, keep_end, mask_id, 1 if append else 0, _ptr(logits), ws.ptr,
+                                         ws.nbytes, _stream(stream)))
 
 
 def device_status(ws, stream=None):

@@ -147,6 +147,28 @@ dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas,
                              float r_start, float r_end, uint64_t seed, int32_t append, float* d_logits,
                              void* d_ws, size_t ws_bytes, dg_stream stream);
 
+/* Masked-diffusion variant of the update ("DiffusionGemma" video explainer -- "First
+ * attempt: masked diffusion": noise is a [MASK] placeholder that the model fills in,
+ * and a filled position stays fixed).  For each row i of d_logits[C][V]: a position
+ * holding any token other than mask_id is locked and keeps it; a masked position's
+ * candidate is its argmax over every token except mask_id (lowest id on ties), its
+ * confidence that token's softmax probability over all V logits.  Of the M masked
+ * positions the min(n_keep, M) least confident (lower position first on ties) keep
+ * mask_id; the others take their candidates.  Writes d_canvas[C] in place; d_conf[C]
+ * (every position's candidate confidence) if not NULL.  Workspace as for
+ * dg_canvas_update.  C <= 1024, V % 4 == 0, 0 <= mask_id < V, 0 <= n_keep <= C. */
+dg_status dg_canvas_update_masked(const float* d_logits, int32_t C, int32_t V, int32_t n_keep, int32_t mask_id,
+                                  int32_t* d_canvas, float* d_conf, void* d_ws, size_t ws_bytes, dg_stream stream);
+
+/* S masked-diffusion passes from an all-mask_id canvas (written by this call into
+ * d_canvas[C]): pass s keeps n_s = dg_renoise_count(C, S, s, keep_start, keep_end)
+ * positions masked at most (keep_start = (S-1)/S, keep_end = 0 unmasks C/S per pass and
+ * ends with none), then appends the canvas by prefill if `append`.  Same workspace,
+ * logits buffer and errors as dg_generate_canvas. */
+dg_status dg_generate_canvas_masked(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t S,
+                                    float keep_start, float keep_end, int32_t mask_id, int32_t append,
+                                    float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream);
+
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
 

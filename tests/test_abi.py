@@ -56,6 +56,9 @@ def test_null_arguments_rejected_on_host():
     assert dg.lib.dg_prefill_append(None, None, None, 4, None, 0, None) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_device_status(None, None) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_canvas_update_noalloc(None, 4, 8, 1, 0, 0, None, None, None) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_canvas_update_masked(None, 4, 8, 1, 7, None, None, None, 0, None) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_generate_canvas_masked(None, None, None, 4, 2, 0.5, 0.0, 7, 0, None, None, 0,
+                                            None) == dg.DG_ERR_INVALID_ARG
 
 
 def test_renoise_schedule_matches_golden():
