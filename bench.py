@@ -212,6 +212,54 @@ def cpu_baseline(cfg, budget_s=30.0):
                       f"median {ms:.0f} ms per step"}
 
 
+class Ranks:
+    """One process per GPU (torchrun sets WORLD_SIZE / RANK / LOCAL_RANK): the process
+    group, barriers, and the max over ranks of a device-timed quantity.  With one rank
+    every call is a no-op."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=120):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self.dist = None
+        if self.world > 1:
+            import torch.distributed as dist
+            from datetime import timedelta
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    @property
+    def is_root(self):
+        return self.rank == 0
+
+    def barrier(self):
+        if self.dist:
+            self.dist.barrier()
+
+    def max(self, x):
+        """The largest x over the ranks (every rank gets it)."""
+        if not self.dist:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def job_value(world, C, steps, max_ms):
+    """Whole-job canvas tokens per second: every rank processed C * steps tokens; the job
+    took as long as its slowest rank."""
+    return world * C * steps / (max_ms / 1e3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -227,16 +275,12 @@ def main():
         return run_reference(args, cfg, name)
 
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
 
     from block_diffusion_lm_masked_b200 import dg
 
@@ -291,19 +335,15 @@ def main():
         timed.last = per
         return sum(per), dg.launch_count() - l0
 
-    if world > 1:
-        dist.barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     clk = Clocks(dev)
     clk.start()
     total_ms, launches = timed(args.steps, profile=False)
     clocks = clk.stop()
     dg.device_status(ws)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
+    total_ms = ranks.max(total_ms)
+    ranks.barrier()
 
     step_median_us = statistics.median(timed.last) * 1e3
 
@@ -373,15 +413,11 @@ def main():
         b.synchronize()
         if s >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = ranks.max(sum(e2e_ms))
 
     ms_step = total_ms / args.steps
-    value = world * C * args.steps / (total_ms / 1e3)
-    e2e_value = world * C * args.steps / (e2e_total / 1e3)
+    value = job_value(world, C, args.steps, total_ms)
+    e2e_value = job_value(world, C, args.steps, e2e_total)
     hbm, tf_burst, tf_sust, peak_src = _peaks()
 
     # whole-pass roofline (slower of FLOPs at the bf16 peak and bytes at HBM bandwidth)
@@ -439,9 +475,7 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
