@@ -11,6 +11,11 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+    # the C-ABI library is a build artefact: compile it (sm_100a, nvcc cross-compiles
+    # without a GPU) when a checkout does not have it yet; an existing one is used as is
+    from block_diffusion_lm_masked_b200 import build as B
+    if not os.path.exists(B.LIB):
+        B.build()
 
 
 def golden_path(name):

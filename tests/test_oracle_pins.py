@@ -457,6 +457,26 @@ def test_masked_schedule_unmasks_to_zero_and_locks():
     assert not np.any(cur == mask_id)
 
 
+def test_generate_masked_loop_properties():
+    """The masked generation loop on a tiny model: it starts from an all-[MASK] canvas,
+    leaves exactly the scheduled number masked after each pass, never changes a filled
+    position, ends with none masked, and appends the final canvas."""
+    cfg = _tiny_cfg(n_layers=1)
+    m = _M(cfg)
+    C, S, mask_id = 12, 4, cfg["vocab"] - 1
+    rec = []
+    cache0 = O.Cache.empty(cfg)
+    out, cache = O.generate_canvas_masked(m, cache0, C, S, (S - 1) / S, 0.0, mask_id, O.Precision("f32"), True, rec)
+    assert len(rec) == S and np.all(rec[0]["canvas_in"] == mask_id)
+    for r in rec:
+        cin, cout = r["canvas_in"], r["update"]["canvas"]
+        assert int((cout == mask_id).sum()) == r["n"] == C * (S - 1 - r["step"]) // S
+        filled = cin != mask_id
+        np.testing.assert_array_equal(cout[filled], cin[filled])
+    assert not np.any(out == mask_id)
+    assert cache.len == C
+
+
 def test_renoise_schedule_golden():
     g = {r[0]: [int(v) for v in r[1:]] for r in _read_golden("renoise_schedule.txt")}
     assert [O.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]

@@ -1,0 +1,107 @@
+"""The comparison rules of the GPU parity tests, checked on planted CPU data (no GPU):
+an allowed routing difference switches the rest of a pass to structure-only checks, a
+routing difference at a clear margin fails, and the causal reach of a prefill starts at
+the first position whose routing actually differs."""
+import numpy as np
+import pytest
+import torch
+
+import parity_lib as PL
+
+CFG = dict(top_k=2, n_experts=4, dtype="bf16")
+
+
+def _taps(topk, x_attn, x_out, counts=None, device="cpu"):
+    L = len(topk)
+    t = dict(topk_idx=[torch.tensor(a, dtype=torch.int32) for a in topk],
+             topk_w=[torch.full(np.asarray(a).shape, 0.5) for a in topk],
+             x_attn=[torch.tensor(a, dtype=torch.float32) for a in x_attn],
+             x_out=[torch.tensor(a, dtype=torch.float32) for a in x_out])
+    cnt, perm, uni = [], [], []
+    for a in topk:
+        a = np.asarray(a)
+        c = np.bincount(a.reshape(-1), minlength=CFG["n_experts"])
+        cnt.append(torch.tensor(c, dtype=torch.int32))
+        flat = a.reshape(-1)
+        perm.append(torch.tensor(sorted(range(flat.size), key=lambda i: (int(flat[i]), i)), dtype=torch.int32))
+        uni.append(int((c > 0).sum()))
+    t.update(counts=cnt, perm=perm, unions=torch.tensor(uni, dtype=torch.int32))
+    return t
+
+
+def _oracle_taps(topk, margins, x_attn, x_out):
+    out = []
+    for a, m, xa, xo in zip(topk, margins, x_attn, x_out):
+        a = np.asarray(a)
+        flat = a.reshape(-1)
+        out.append(dict(topk_idx=a, topk_w=np.full(a.shape, 0.5), router_margin=np.asarray(m, dtype=float),
+                        counts=np.bincount(flat, minlength=CFG["n_experts"]),
+                        perm=sorted(range(flat.size), key=lambda i: (int(flat[i]), i)),
+                        x_attn=np.asarray(xa, dtype=float), x_out=np.asarray(xo, dtype=float)))
+    return out
+
+
+def _pass(rows=3, layers=3, seed=0):
+    rng = np.random.default_rng(seed)
+    topk = [np.array([[0, 1], [2, 3], [1, 2]])[:rows] for _ in range(layers)]
+    xa = [rng.standard_normal((rows, 4)) for _ in range(layers)]
+    xo = [rng.standard_normal((rows, 4)) for _ in range(layers)]
+    return topk, xa, xo
+
+
+def test_identical_pass_compares_in_full():
+    topk, xa, xo = _pass()
+    logits = np.random.default_rng(1).standard_normal((3, 5))
+    report = []
+    ex = PL.compare_pass(CFG, _taps(topk, xa, xo), logits, _oracle_taps(topk, [[1, 1, 1]] * 3, xa, xo), logits, report)
+    assert ex == set() and report[-1]["logits"] == 0.0
+
+
+def test_near_tie_flip_turns_rest_of_pass_structure_only():
+    topk, xa, xo = _pass()
+    g_topk = [t.copy() for t in topk]
+    g_topk[0][1] = [2, 0]                           # row 1 routes differently at layer 0 ...
+    margins = [[1, 5e-4, 1], [1, 1, 1], [1, 1, 1]]   # ... where the oracle's margin is a near tie
+    g_xa = [a.copy() for a in xa]
+    g_xa[1] = g_xa[1] + 10.0                         # later layers may then differ arbitrarily
+    logits = np.zeros((3, 5))
+    report = []
+    ex = PL.compare_pass(CFG, _taps(g_topk, g_xa, xo), logits + 7.0, _oracle_taps(topk, margins, xa, xo), logits,
+                         report)
+    assert ex == {0, 1, 2}
+    assert report[-1] == dict(logits=None, diverged_after_layer=0)
+
+
+def test_flip_at_clear_margin_fails():
+    topk, xa, xo = _pass()
+    g_topk = [t.copy() for t in topk]
+    g_topk[1][2] = [0, 2]
+    with pytest.raises(AssertionError, match="routing"):
+        PL.compare_pass(CFG, _taps(g_topk, xa, xo), np.zeros((3, 5)),
+                        _oracle_taps(topk, [[1, 1, 1]] * 3, xa, xo), np.zeros((3, 5)))
+
+
+def test_hidden_state_outside_tolerance_fails():
+    topk, xa, xo = _pass()
+    g_xo = [a.copy() for a in xo]
+    g_xo[2][0, 0] += 0.5                             # ~0.5 RMS at the last layer
+    with pytest.raises(AssertionError, match="MoE residual"):
+        PL.compare_pass(CFG, _taps(topk, xa, g_xo), np.zeros((3, 5)),
+                        _oracle_taps(topk, [[1, 1, 1]] * 3, xa, xo), np.zeros((3, 5)))
+
+
+def test_causal_reach_from_actual_flips():
+    # two layers' taps of a 6-token prefill at offset 10; the GPU differs at position 3 of layer 0
+    o_topk = [np.tile([[0, 1]], (6, 1)), np.tile([[2, 3]], (6, 1))]
+    g_topk = [t.copy() for t in o_topk]
+    g_topk[0][3] = [1, 2]
+    taps = [dict(topk_idx=o_topk[0], router_margin=np.array([1, 1, 1, 5e-4, 1, 1])),
+            dict(topk_idx=o_topk[1], router_margin=np.ones(6))]
+    reach = PL.causal_reach([(10, g_topk, taps)], 3)
+    assert reach == [None, 13, 13]
+    # near ties that did not flip reach nothing
+    assert PL.causal_reach([(10, o_topk, taps)], 3) == [None, None, None]
+    # a flip at a clear margin before any reach is an error
+    taps[0]["router_margin"][3] = 1.0
+    with pytest.raises(AssertionError, match="prefill layer 0 position 13"):
+        PL.causal_reach([(10, g_topk, taps)], 3)
