@@ -679,10 +679,6 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
   return DG_OK;
 }
 
-// the update's completion ticket: a counter in the workspace's reserved head (after the
-// device error word), zero while no update runs
-constexpr size_t kUpdTicketOffset = 128;
-
 extern "C" dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t V, int32_t n_renoise, uint64_t seed,
                                       uint32_t step, int32_t* d_canvas, float* d_conf, void* d_ws, size_t ws_bytes,
                                       dg_stream stream) {
@@ -698,9 +694,9 @@ extern "C" dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dg::UpdPart* part = reinterpret_cast<dg::UpdPart*>(static_cast<char*>(d_ws) + 256);
   const int splits = dg::update_splits(C, V);
-  unsigned* ticket = reinterpret_cast<unsigned*>(static_cast<char*>(d_ws) + kUpdTicketOffset);
-  LAUNCH(DG_K_UPDATE_PARTIAL, st,
-         dg::launch_update(d_logits, C, V, splits, -1, part, ticket, n_renoise, seed, step, d_canvas, d_conf, -1, st));
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, -1, part, st));
+  LAUNCH(DG_K_UPDATE_SELECT, st,
+         dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, -1, st));
   return DG_OK;
 }
 
@@ -720,9 +716,9 @@ extern "C" dg_status dg_canvas_update_masked(const float* d_logits, int32_t C, i
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dg::UpdPart* part = reinterpret_cast<dg::UpdPart*>(static_cast<char*>(d_ws) + 256);
   const int splits = dg::update_splits(C, V);
-  unsigned* ticket = reinterpret_cast<unsigned*>(static_cast<char*>(d_ws) + kUpdTicketOffset);
-  LAUNCH(DG_K_UPDATE_PARTIAL, st,
-         dg::launch_update(d_logits, C, V, splits, mask_id, part, ticket, n_keep, 0, 0, d_canvas, d_conf, mask_id, st));
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, C, V, splits, mask_id, part, st));
+  LAUNCH(DG_K_UPDATE_SELECT, st,
+         dg::launch_update_select(part, C, V, splits, n_keep, 0, 0, d_canvas, d_conf, mask_id, st));
   return DG_OK;
 }
 

@@ -122,12 +122,12 @@ struct UpdPart {
   float m2;   // that logit (the ids other than an excluded one; m when nothing is excluded)
 };
 int update_splits(int C, int V);
-// the canvas update in one launch: per-slice partials, then the last CTA selects.
-// excl >= 0: the candidate skips that id; mask_id < 0: the re-noising update, mask_id >= 0:
-// the masked-diffusion update.  ticket: a zero-initialised counter the launch leaves zero.
-cudaError_t launch_update(const float* logits, int C, int V, int splits, int excl, UpdPart* part, unsigned* ticket,
-                          int n_renoise, uint64_t seed, uint32_t step, int32_t* canvas, float* conf, int mask_id,
-                          cudaStream_t st);
+// excl >= 0: the candidate skips that id
+cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, int excl, UpdPart* part,
+                                  cudaStream_t st);
+// mask_id < 0: the re-noising update; mask_id >= 0: the masked-diffusion update
+cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
+                                 uint32_t step, int32_t* canvas, float* conf, int mask_id, cudaStream_t st);
 cudaError_t launch_fill_i32(int32_t* p, int n, int32_t v, cudaStream_t st);
 
 cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);

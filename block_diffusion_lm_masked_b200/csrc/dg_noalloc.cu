@@ -27,16 +27,13 @@ constexpr int kMaxDevices = 64;
 
 std::mutex g_setup_mu;
 std::atomic<dg::UpdPart*> g_scratch[kMaxDevices];
-std::atomic<unsigned*> g_ticket[kMaxDevices];
 
 }  // namespace
 
 static __device__ __align__(256) dg::UpdPart g_upd_scratch[kScratchParts];
-static __device__ unsigned g_upd_ticket;  // the update's completion counter, zero between calls
 
-// device addresses of g_upd_scratch and g_upd_ticket on the current device, looked up on
-// first use
-static dg_status scratch_for_current_device(dg::UpdPart** out, unsigned** ticket) {
+// device address of g_upd_scratch on the current device, looked up on first use
+static dg_status scratch_for_current_device(dg::UpdPart** out) {
   char msg[160];
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -54,20 +51,16 @@ static dg_status scratch_for_current_device(dg::UpdPart** out, unsigned** ticket
     p = g_scratch[dev].load(std::memory_order_relaxed);
     if (!p) {
       void* a = nullptr;
-      void* t = nullptr;
       e = cudaGetSymbolAddress(&a, g_upd_scratch);
-      if (e == cudaSuccess) e = cudaGetSymbolAddress(&t, g_upd_ticket);
       if (e != cudaSuccess) {
         snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the update scratch: %s", cudaGetErrorString(e));
         return dg::set_error(DG_ERR_CUDA, msg);
       }
       p = static_cast<dg::UpdPart*>(a);
-      g_ticket[dev].store(static_cast<unsigned*>(t), std::memory_order_relaxed);
       g_scratch[dev].store(p, std::memory_order_release);
     }
   }
   *out = p;
-  *ticket = g_ticket[dev].load(std::memory_order_relaxed);
   return DG_OK;
 }
 
@@ -88,12 +81,12 @@ extern "C" dg_status dg_canvas_update_noalloc(const float* d_logits, int32_t C, 
     return dg::set_error(DG_ERR_CAPACITY, msg);
   }
   dg::UpdPart* part = nullptr;
-  unsigned* ticket = nullptr;
-  dg_status s = scratch_for_current_device(&part, &ticket);
+  dg_status s = scratch_for_current_device(&part);
   if (s != DG_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      dg::launch_update(d_logits, C, V, splits, -1, part, ticket, n_renoise, seed, step, d_canvas, d_conf, -1, st);
+  cudaError_t e = dg::launch_update_partial(d_logits, C, V, splits, -1, part, st);
+  if (e == cudaSuccess)
+    e = dg::launch_update_select(part, C, V, splits, n_renoise, seed, step, d_canvas, d_conf, -1, st);
   if (e != cudaSuccess) {
     snprintf(msg, sizeof msg, "canvas update launch: %s", cudaGetErrorString(e));
     return dg::set_error(DG_ERR_CUDA, msg);

@@ -707,38 +707,14 @@ int update_splits(int C, int V) {
   return s;
 }
 
-// The canvas update in one launch.  CTA (row, slice) streams its slice of the row's
-// logits once: max, sum of exp(l - max), and the candidate (the largest logit among the
-// ids other than `excl`, first index on ties; the plain argmax when excl < 0), and parks
-// them.  The last CTA to finish (an atomic ticket, reset by it for the next call) merges
-// every row's slices in slice order and selects:
-//   re-noising (mask_id < 0): every position takes its argmax, then the n lowest-
-//     confidence positions (confidence 1 / sum; ties: lower position first) take a fresh
-//     token, SplitMix64(seed) draw number (step << 32 | position), multiply-shift onto [0, V);
-//   masked (mask_id >= 0): positions holding a token other than mask_id keep it; a masked
-//     position's candidate confidence is exp(m2 - m) / sum; of the M masked positions the
-//     min(n, M) least confident (ties: lower position first) stay mask_id, the others take
-//     their candidates.
-constexpr int UPD_THREADS = 256;
-constexpr int UPD_MAX_C = 1024;
-
-__device__ __forceinline__ uint64_t splitmix64_out(uint64_t seed, uint64_t n) {
-  uint64_t z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
-}
-
-__global__ void __launch_bounds__(UPD_THREADS, 3) update_kernel(
-    const float* __restrict__ logits, int C, int V, int splits, int excl, UpdPart* __restrict__ part,
-    unsigned* __restrict__ ticket, int n_renoise, uint64_t seed, uint32_t step, int32_t* __restrict__ canvas,
-    float* __restrict__ conf, int mask_id) {
+// per (row, slice): max, first argmax and sum exp(l - max), one streaming pass
+// excl >= 0: the candidate (a, m2) skips that id (the masked-diffusion update never fills
+// with the mask token); excl < 0: the candidate is the plain first argmax (m2 = m)
+__global__ void update_partial_kernel(const float* __restrict__ logits, int V, int splits, int excl,
+                                      UpdPart* __restrict__ part) {
   griddep_sync();
   __shared__ float sm[32], ss[32], sm2[32];
   __shared__ int sa[32];
-  __shared__ float den[UPD_MAX_C];  // per position: sum (re-noising) or confidence (masked)
-  __shared__ int cand[UPD_MAX_C], is_m[UPD_MAX_C];
-  __shared__ int last_s, n_masked;
   const int row = blockIdx.x, sp = blockIdx.y;
   const int slice = ((V + splits - 1) / splits + 3) & ~3;
   const int lo = sp * slice, hi = min(V, lo + slice);
@@ -819,76 +795,95 @@ __global__ void __launch_bounds__(UPD_THREADS, 3) update_kernel(
     r.a = a;
     r.m2 = m2;
     part[(size_t)row * splits + sp] = r;
-    __threadfence();  // the partial is visible GPU-wide before the ticket
-    const unsigned total = (unsigned)C * (unsigned)splits;
-    last_s = atomicAdd(ticket, 1u) == total - 1u;
   }
+}
+
+__device__ __forceinline__ uint64_t splitmix64_out(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// merge slices, confidence = 1 / sum exp(l - max); every position takes its argmax, then
+// the n_renoise lowest-confidence positions (ties: lower position first) take a fresh
+// token: SplitMix64(seed) draw number (step << 32 | position), multiply-shift onto [0, V).
+// Masked mode (mask_id >= 0): positions holding a token other than mask_id keep it; a
+// masked position's candidate is its best token other than mask_id, with confidence
+// exp(m2 - m) / sum; of the M masked positions the min(n_renoise, M) least confident
+// (ties: lower position first) stay mask_id and the others take their candidates.
+__global__ void update_select_kernel(const UpdPart* __restrict__ part, int C, int V, int splits, int n_renoise,
+                                     uint64_t seed, uint32_t step, int32_t* __restrict__ canvas,
+                                     float* __restrict__ conf, int mask_id) {
+  griddep_sync();
+  extern __shared__ float den[];  // [C] sums (uniform) or confidences (masked), then [C] masked flags
+  int* is_m = reinterpret_cast<int*>(den + C);
+  __shared__ int n_masked;
+  const int i = threadIdx.x;
+  float m = -INFINITY, s = 0.0f, m2 = -INFINITY;
+  int a = 0x7fffffff;
+  if (i == 0) n_masked = 0;
   __syncthreads();
-  if (!last_s) return;
-  // ---- the last CTA: merge every row's slices, then select
-  __threadfence();
-  if (threadIdx.x == 0) {
-    n_masked = 0;
-    *ticket = 0u;  // every CTA of this launch has taken its ticket
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < C; i += blockDim.x) {
-    float pm = -INFINITY, ps = 0.0f, pm2 = -INFINITY;
-    int pa = 0x7fffffff;
-    for (int sp0 = 0; sp0 < splits; sp0 += 4) {  // four slices' partials in flight, merged in order
-      float4 q[4];
+  if (i < C) {
+    for (int sp0 = 0; sp0 < splits; sp0 += 8) {  // eight slices' partials in flight, merged in order
+      UpdPart q[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (sp0 + u < splits) q[u] = __ldcg(reinterpret_cast<const float4*>(part + (size_t)i * splits + sp0 + u));
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < splits) q[u] = part[(size_t)i * splits + sp0 + u];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
         if (sp0 + u < splits) {
-          ms_merge(pm, ps, q[u].x, q[u].y);
-          cand_merge(pm2, pa, q[u].w, __float_as_int(q[u].z));
+          ms_merge(m, s, q[u].m, q[u].s);
+          cand_merge(m2, a, q[u].m2, q[u].a);
         }
     }
-    cand[i] = pa;
     if (mask_id < 0) {
-      den[i] = ps;
+      den[i] = s;
     } else {
-      den[i] = expf(pm2 - pm) / ps;
+      den[i] = expf(m2 - m) / s;
       is_m[i] = canvas[i] == mask_id;
       if (is_m[i]) atomicAdd(&n_masked, 1);
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < C; i += blockDim.x) {
-    const float di = den[i];
+  if (i < C) {
     if (mask_id < 0) {
       int rank = 0;
       for (int j = 0; j < C; ++j) {
         const float dj = den[j];
-        rank += (dj > di) || (dj == di && j < i);
+        rank += (dj > s) || (dj == s && j < i);
       }
-      int tok = cand[i];
+      int tok = a;
       if (rank < n_renoise) {
         const uint64_t x = splitmix64_out(seed, ((uint64_t)step << 32) | (uint64_t)i);
         tok = (int)(((x >> 32) * (uint64_t)V) >> 32);
       }
       canvas[i] = tok;
-      if (conf) conf[i] = 1.0f / di;
+      if (conf) conf[i] = 1.0f / s;
     } else {
+      const float ci = den[i];
       if (is_m[i]) {
         int rank = 0;  // among the masked positions, by confidence, ties to the lower position
-        for (int j = 0; j < C; ++j) rank += is_m[j] && (den[j] < di || (den[j] == di && j < i));
-        canvas[i] = rank < min(n_renoise, n_masked) ? mask_id : cand[i];
+        for (int j = 0; j < C; ++j) rank += is_m[j] && (den[j] < ci || (den[j] == ci && j < i));
+        const int keep = min(n_renoise, n_masked);
+        canvas[i] = rank < keep ? mask_id : a;
       }
-      if (conf) conf[i] = di;
+      if (conf) conf[i] = ci;
     }
   }
 }
 
-cudaError_t launch_update(const float* logits, int C, int V, int splits, int excl, UpdPart* part, unsigned* ticket,
-                          int n_renoise, uint64_t seed, uint32_t step, int32_t* canvas, float* conf, int mask_id,
-                          cudaStream_t st) {
+cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, int excl, UpdPart* part,
+                                  cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
-  if (C > UPD_MAX_C) return cudaErrorInvalidValue;
-  return launch_k(update_kernel, dim3(C, splits), dim3(UPD_THREADS), 0, st, logits, C, V, splits, excl, part, ticket,
+  return launch_k(update_partial_kernel, dim3(C, splits), dim3(256), 0, st, logits, V, splits, excl, part);
+}
+cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, int n_renoise, uint64_t seed,
+                                 uint32_t step, int32_t* canvas, float* conf, int mask_id, cudaStream_t st) {
+  if (C <= 0) return cudaSuccess;
+  if (C > 1024) return cudaErrorInvalidValue;
+  const int threads = (C + 31) & ~31;
+  return launch_k(update_select_kernel, dim3(1), dim3(threads), 2 * C * sizeof(float), st, part, C, V, splits,
                   n_renoise, seed, step, canvas, conf, mask_id);
 }
 
