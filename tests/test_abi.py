@@ -61,6 +61,25 @@ def test_null_arguments_rejected_on_host():
                                             None) == dg.DG_ERR_INVALID_ARG
 
 
+def test_masked_update_validation_on_host():
+    """Every bad argument of the masked entry points is rejected before any CUDA call
+    (the placeholder pointers below are never dereferenced)."""
+    p = ctypes.c_void_p(4096)
+    L = dg.lib
+
+    def upd(C, V, n_keep, mask_id, ws_bytes=1 << 20):
+        return L.dg_canvas_update_masked(p, C, V, n_keep, mask_id, p, None, p, ws_bytes, None)
+
+    for args in ((0, 8, 0, 1), (1025, 8, 0, 1), (4, 6, 0, 1), (4, 8, 0, 8), (4, 8, 0, -1), (4, 8, 5, 1),
+                 (4, 8, -1, 1)):
+        assert upd(*args) == dg.DG_ERR_INVALID_ARG, args
+    assert upd(4, 8, 0, 1, ws_bytes=16) == dg.DG_ERR_CAPACITY
+    assert L.dg_canvas_update_masked(ctypes.c_void_p(4100), 4, 8, 0, 1, p, None, p, 1 << 20,
+                                     None) == dg.DG_ERR_INVALID_ARG        # logits not 16-byte aligned
+    assert L.dg_generate_canvas_masked(None, None, p, 4, 2, 0.5, 0.0, 1, 0, p, p, 1 << 20,
+                                       None) == dg.DG_ERR_INVALID_ARG     # no model
+
+
 def test_renoise_schedule_matches_golden():
     g = {}
     for line in open(golden_path("renoise_schedule.txt")):
