@@ -346,6 +346,7 @@ def main():
     ranks.barrier()
 
     step_median_us = statistics.median(timed.last) * 1e3
+    step_p10_us, step_p90_us = (float(v) * 1e3 for v in np.percentile(timed.last, [10, 90]))
 
     # the pass alone (no update), same timing rules
     def pass_only(s):
@@ -467,6 +468,7 @@ def main():
         "kernels": kern,
         "kernel_rooflines": kroof,
         "step_median_us": step_median_us,
+        "step_p10_p90_us": [step_p10_us, step_p90_us],
         "pass_only_us": {"median": statistics.median(pass_us), "mean": sum(pass_us) / len(pass_us), "steps": k2},
         "graph_step_us": graph,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": C * 4, "d2h_bytes_per_step": C * 4},

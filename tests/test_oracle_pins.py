@@ -477,6 +477,25 @@ def test_generate_masked_loop_properties():
     assert cache.len == C
 
 
+def test_resume_from_a_middle_pass_reproduces_the_run():
+    """The generation state is (cache, canvas, pass index, seed): the re-noise draws are
+    counter-based on (seed, pass, position), so restarting at pass s from the canvas the
+    run had there gives the same final canvas."""
+    cfg = _tiny_cfg(n_layers=1)
+    m = _M(cfg)
+    S, prec, seed = 5, O.Precision("f32"), 99
+    cache = O.Cache.empty(cfg)
+    start = np.random.default_rng(3).integers(0, cfg["vocab"], 10).astype(np.int32)
+    rec = []
+    full, _ = O.generate_canvas(m, cache, start, S, 0.5, 0.0, seed, prec, False, rec)
+    for s0 in (1, 3):
+        cur = rec[s0]["canvas_in"].copy()
+        for s in range(s0, S):
+            logits, _ = O.denoise_pass(m, cache, cur, prec)
+            cur = O.canvas_update(logits, O.renoise_count(len(cur), S, s, 0.5, 0.0), seed, s)["canvas"]
+        np.testing.assert_array_equal(cur, full)
+
+
 def test_renoise_schedule_golden():
     g = {r[0]: [int(v) for v in r[1:]] for r in _read_golden("renoise_schedule.txt")}
     assert [O.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]
