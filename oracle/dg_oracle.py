@@ -544,3 +544,66 @@ def generate_canvas(model, cache: Cache, canvas: np.ndarray, S: int, r_start: fl
     if append:
         cache = prefill_append(model, cache, cur, prec)
     return cur, cache
+
+
+# ----------------------------------------------------------------------------
+# 8-bit expert weights (groundwork for the FP8 deployment the pages mention): the OCP
+# "E4M3" element format and MX block scaling, written from the published definitions.
+# Nothing in the pass uses these yet.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an 8-bit E4M3 code: sign, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent 0 is subnormal (m * 2^-9); 0x7F / 0xFF are NaN; no infinities."""
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return s * m * 2.0 ** -9
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+_E4M3_POS = np.array([e4m3_decode(c) for c in range(0x7F)])  # codes 0x00 .. 0x7E, increasing
+
+
+def e4m3_encode(x: float) -> int:
+    """Nearest E4M3 code (ties to the even code, i.e. even mantissa); magnitudes beyond
+    448 saturate to 448."""
+    neg = np.signbit(x)
+    a = min(abs(float(x)), E4M3_MAX)
+    i = int(np.searchsorted(_E4M3_POS, a))  # first value >= a
+    if i < len(_E4M3_POS) and _E4M3_POS[i] == a:
+        c = i
+    else:
+        lo, hi = i - 1, i
+        dlo, dhi = a - _E4M3_POS[lo], _E4M3_POS[hi] - a
+        c = lo if (dlo < dhi or (dlo == dhi and lo % 2 == 0)) else hi
+    return c | (0x80 if neg else 0)
+
+
+def mx_e4m3_quantize(w: np.ndarray, block: int = 32):
+    """MX block scaling along the last axis: each block of `block` consecutive values
+    shares the power-of-two scale X = 2^(floor(log2(max |v|)) - 8) (8 = the largest
+    E4M3 exponent), and each value is stored as e4m3_encode(v / X).  Returns (codes
+    uint8 [..., n], scale exponents int32 [..., n / block]); an all-zero block gets
+    exponent -127."""
+    w = np.asarray(w, dtype=np.float64)
+    assert w.shape[-1] % block == 0
+    blocks = w.reshape(*w.shape[:-1], w.shape[-1] // block, block)
+    amax = np.abs(blocks).max(axis=-1)
+    exp = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127).astype(np.int32)
+    exp = np.clip(exp, -127, 127)
+    scaled = blocks / np.ldexp(1.0, exp)[..., None]
+    codes = np.vectorize(e4m3_encode, otypes=[np.uint8])(scaled)
+    return codes.reshape(w.shape), exp
+
+
+def mx_e4m3_dequantize(codes: np.ndarray, exp: np.ndarray, block: int = 32) -> np.ndarray:
+    """X * e4m3_decode(code) for every element."""
+    vals = np.vectorize(e4m3_decode, otypes=[np.float64])(np.asarray(codes))
+    blocks = vals.reshape(*vals.shape[:-1], vals.shape[-1] // block, block)
+    return (blocks * np.ldexp(1.0, exp)[..., None]).reshape(vals.shape)

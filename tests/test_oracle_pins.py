@@ -496,6 +496,61 @@ def test_resume_from_a_middle_pass_reproduces_the_run():
         np.testing.assert_array_equal(cur, full)
 
 
+def test_e4m3_decode_closed_forms():
+    d = O.e4m3_decode
+    assert d(0x00) == 0.0 and np.signbit(d(0x80)) and d(0x80) == 0.0
+    assert d(0x01) == 2.0 ** -9 and d(0x07) == 7 * 2.0 ** -9       # subnormals
+    assert d(0x08) == 2.0 ** -6 and d(0x0F) == 1.875 * 2.0 ** -6   # smallest binade of normals
+    assert d(0x38) == 1.0 and d(0x39) == 1.125 and d(0x7E) == 448.0
+    assert np.isnan(d(0x7F)) and np.isnan(d(0xFF))
+    pos = [d(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(pos, pos[1:]))
+    for c in range(0x7F):
+        assert d(c | 0x80) == -d(c)
+    # within a binade the spacing is 2^(e-7) / 8
+    for e in range(1, 15):
+        vals = [d((e << 3) | m) for m in range(8)]
+        assert np.allclose(np.diff(vals), 2.0 ** (e - 7) / 8, rtol=0, atol=0)
+
+
+def test_e4m3_encode_round_trip_rounding_saturation():
+    for c in range(256):
+        if c in (0x7F, 0xFF):
+            continue
+        assert O.e4m3_encode(O.e4m3_decode(c)) == c
+    enc = O.e4m3_encode
+    assert enc(1.0625) == 0x38 and enc(1.1875) == 0x3A              # ties go to the even mantissa
+    assert enc(1.07) == 0x39 and enc(-1.07) == 0xB9
+    assert enc(2.0 ** -10) == 0x00 and enc(1.5 * 2.0 ** -10) == 0x01  # around the smallest subnormal
+    assert enc(464.0) == 0x7E and enc(1000.0) == 0x7E and enc(-1e6) == 0xFE   # saturation
+
+
+def test_mx_e4m3_block_scaling():
+    rng = np.random.default_rng(41)
+    w = rng.standard_normal((6, 128)) * np.array([1e-3, 0.02, 1.0, 7.0, 300.0, 1e4])[:, None]
+    w[2, 32:64] = 0.0                                                   # one all-zero block
+    codes, exp = O.mx_e4m3_quantize(w)
+    dq = O.mx_e4m3_dequantize(codes, exp)
+    blocks = w.reshape(6, 4, 32)
+    amax = np.abs(blocks).max(axis=-1)
+    nz = amax > 0
+    # the block's largest magnitude lands in [256, 512) after scaling
+    r = amax[nz] / np.ldexp(1.0, exp[nz])
+    assert np.all((r >= 256) & (r < 512))
+    assert np.all(dq.reshape(6, 4, 32)[~nz] == 0)
+    # relative error of a 3-bit mantissa (half a unit in the last place) for values in the
+    # normal range that did not saturate
+    X = np.repeat(np.ldexp(1.0, exp), 32, axis=-1).reshape(w.shape)
+    sc = np.abs(w) / X
+    ok = (sc >= 2.0 ** -6) & (sc <= 448.0)
+    assert np.all(np.abs(dq - w)[ok] <= 2.0 ** -4 * np.abs(w)[ok] + 1e-300)
+    sat = sc > 464.0
+    assert np.all(np.abs(dq[sat]) == 448.0 * X[sat])
+    # a hand example: [3, 0, ...]: X = 2^(1 - 8), 3 / X = 384 = 1.5 * 2^8, exact
+    c1, e1 = O.mx_e4m3_quantize(np.array([3.0] + [0.0] * 31))
+    assert e1[0] == -7 and c1[0] == 0x7C and O.mx_e4m3_dequantize(c1, e1)[0] == 3.0
+
+
 def test_renoise_schedule_golden():
     g = {r[0]: [int(v) for v in r[1:]] for r in _read_golden("renoise_schedule.txt")}
     assert [O.renoise_count(256, 16, s, 0.5, 0.0) for s in range(16)] == g["S16"]
