@@ -557,6 +557,7 @@ E4M3_MAX = 448.0
 def e4m3_decode(code: int) -> float:
     """Value of an 8-bit E4M3 code: sign, 4 exponent bits (bias 7), 3 mantissa bits;
     exponent 0 is subnormal (m * 2^-9); 0x7F / 0xFF are NaN; no infinities."""
+    code = int(code)  # numpy uint8 arithmetic would wrap in e - 7
     s = -1.0 if code & 0x80 else 1.0
     e = (code >> 3) & 0xF
     m = code & 0x7
@@ -607,3 +608,59 @@ def mx_e4m3_dequantize(codes: np.ndarray, exp: np.ndarray, block: int = 32) -> n
     vals = np.vectorize(e4m3_decode, otypes=[np.float64])(np.asarray(codes))
     blocks = vals.reshape(*vals.shape[:-1], vals.shape[-1] // block, block)
     return (blocks * np.ldexp(1.0, exp)[..., None]).reshape(vals.shape)
+
+
+# 4-bit elements (E2M1: sign, 2 exponent bits with bias 1, 1 mantissa bit; no inf/NaN)
+# scaled per 16-element block by an E4M3 value and per tensor by an fp32 value.
+
+
+def e2m1_decode(code: int) -> float:
+    code = int(code)
+    s = -1.0 if code & 0x8 else 1.0
+    e = (code >> 1) & 0x3
+    m = code & 0x1
+    if e == 0:
+        return s * 0.5 * m
+    return s * (1.0 + 0.5 * m) * 2.0 ** (e - 1)
+
+
+_E2M1_POS = np.array([e2m1_decode(c) for c in range(8)])  # 0, 0.5, 1, 1.5, 2, 3, 4, 6
+
+
+def e2m1_encode(x: float) -> int:
+    """Nearest E2M1 code (ties to the even code); magnitudes beyond 6 saturate to 6."""
+    neg = np.signbit(x)
+    a = min(abs(float(x)), 6.0)
+    i = int(np.searchsorted(_E2M1_POS, a))
+    if i < 8 and _E2M1_POS[i] == a:
+        c = i
+    else:
+        lo, hi = i - 1, i
+        dlo, dhi = a - _E2M1_POS[lo], _E2M1_POS[hi] - a
+        c = lo if (dlo < dhi or (dlo == dhi and lo % 2 == 0)) else hi
+    return c | (0x8 if neg else 0)
+
+
+def nvfp4_quantize(w: np.ndarray, block: int = 16):
+    """Two-level scaling along the last axis: a tensor scale g = max |w| / (448 * 6); per
+    block of `block` values an E4M3 scale code for max |v| / (6 g); each value stored as
+    e2m1_encode(v / (s_b g)) with s_b the decoded block scale.  Returns (codes uint8
+    [..., n], block scale codes uint8 [..., n / block], g)."""
+    w = np.asarray(w, dtype=np.float64)
+    assert w.shape[-1] % block == 0
+    amax_t = float(np.abs(w).max())
+    g = amax_t / (E4M3_MAX * 6.0) if amax_t > 0 else 1.0
+    blocks = w.reshape(*w.shape[:-1], w.shape[-1] // block, block)
+    amax = np.abs(blocks).max(axis=-1)
+    sc = np.vectorize(e4m3_encode, otypes=[np.uint8])(amax / (6.0 * g))
+    sb = np.vectorize(e4m3_decode, otypes=[np.float64])(sc)
+    denom = np.where(sb > 0, sb * g, 1.0)[..., None]
+    codes = np.vectorize(e2m1_encode, otypes=[np.uint8])(blocks / denom)
+    return codes.reshape(w.shape), sc, g
+
+
+def nvfp4_dequantize(codes: np.ndarray, scale_codes: np.ndarray, g: float, block: int = 16) -> np.ndarray:
+    vals = np.vectorize(e2m1_decode, otypes=[np.float64])(np.asarray(codes))
+    sb = np.vectorize(e4m3_decode, otypes=[np.float64])(np.asarray(scale_codes))
+    blocks = vals.reshape(*vals.shape[:-1], vals.shape[-1] // block, block)
+    return (blocks * (sb * g)[..., None]).reshape(vals.shape)

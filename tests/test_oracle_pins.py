@@ -503,6 +503,7 @@ def test_e4m3_decode_closed_forms():
     assert d(0x08) == 2.0 ** -6 and d(0x0F) == 1.875 * 2.0 ** -6   # smallest binade of normals
     assert d(0x38) == 1.0 and d(0x39) == 1.125 and d(0x7E) == 448.0
     assert np.isnan(d(0x7F)) and np.isnan(d(0xFF))
+    assert d(np.uint8(0x30)) == 0.5                                # numpy integer codes decode the same
     pos = [d(c) for c in range(0x7F)]
     assert all(a < b for a, b in zip(pos, pos[1:]))
     for c in range(0x7F):
@@ -549,6 +550,38 @@ def test_mx_e4m3_block_scaling():
     # a hand example: [3, 0, ...]: X = 2^(1 - 8), 3 / X = 384 = 1.5 * 2^8, exact
     c1, e1 = O.mx_e4m3_quantize(np.array([3.0] + [0.0] * 31))
     assert e1[0] == -7 and c1[0] == 0x7C and O.mx_e4m3_dequantize(c1, e1)[0] == 3.0
+
+
+def test_e2m1_codes_rounding_saturation():
+    assert [O.e2m1_decode(c) for c in range(8)] == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(8):
+        assert O.e2m1_decode(c | 0x8) == -O.e2m1_decode(c)
+        assert O.e2m1_encode(O.e2m1_decode(c)) == c
+    enc = O.e2m1_encode
+    assert enc(0.25) == 0 and enc(0.75) == 2 and enc(1.25) == 2 and enc(1.75) == 4   # ties to even
+    assert enc(2.5) == 4 and enc(3.5) == 6 and enc(5.0) == 6                          # ties to even
+    assert enc(2.4) == 4 and enc(5.1) == 7 and enc(100.0) == 7 and enc(-100.0) == 0xF
+
+
+def test_nvfp4_block_scaling():
+    rng = np.random.default_rng(43)
+    w = rng.standard_normal((4, 64)) * np.array([0.01, 0.2, 1.0, 5.0])[:, None]
+    codes, sc, g = O.nvfp4_quantize(w)
+    dq = O.nvfp4_dequantize(codes, sc, g)
+    assert g == np.abs(w).max() / (448.0 * 6.0)
+    # the tensor's largest value: block scale 448 exactly, element code 6, reproduced
+    i = np.unravel_index(np.argmax(np.abs(w)), w.shape)
+    assert O.e4m3_decode(int(sc[i[0], i[1] // 16])) == 448.0 and abs(dq[i]) == pytest.approx(abs(w[i]))
+    # every element within half an E2M1 step of its scaled value (the step is at most 2 at
+    # the top of the range) after the block scale's own rounding
+    sb = np.vectorize(O.e4m3_decode)(sc)
+    X = np.repeat(sb * g, 16, axis=-1).reshape(w.shape)
+    sc_v = np.abs(w) / X
+    assert np.all(np.abs(dq - w) <= np.where(sc_v <= 2, 0.25, np.where(sc_v <= 4, 0.5, 1.0)) * X + 1e-15)
+    # values that are E2M1 grid points of an exactly representable scale come back exactly
+    exact = np.array([[6.0, -4.0, 3.0, 0.5] * 4]) * 2.0
+    c2, s2, g2 = O.nvfp4_quantize(exact)
+    np.testing.assert_array_equal(O.nvfp4_dequantize(c2, s2, g2), exact)
 
 
 def test_renoise_schedule_golden():
