@@ -51,6 +51,17 @@ def test_splitmix64_known_answers():
     assert [int(v) for v in got] == want
 
 
+def test_renoise_token_is_the_top_bits_of_the_published_draw():
+    """At step 0, position p uses draw number p of SplitMix64(seed); the token is the
+    multiply-shift of that draw's top 32 bits, so for V = 2^b it is the top b bits."""
+    pub = [int(r[0], 16) for r in _read_golden("splitmix64_seed0.txt")]
+    for p, x in enumerate(pub):
+        assert O.renoise_token(0, 0, p, 1 << 32) == x >> 32
+        assert O.renoise_token(0, 0, p, 2) == x >> 63
+        assert O.renoise_token(0, 0, p, 1 << 10) == x >> 54
+        assert O.renoise_token(0, 0, p, 1000) == (x >> 32) * 1000 // (1 << 32)
+
+
 def test_renoise_tokens_uniform_chi2():
     V, n = 64, 64 * 400
     draws = [O.renoise_token(1236, s, p, V) for s in range(4) for p in range(n // 4)]
@@ -281,6 +292,28 @@ def test_moe_k1_routes_each_token_to_its_argmax_expert():
         np.testing.assert_allclose(got[t], want, rtol=1e-12, atol=1e-13)
 
 
+def test_moe_combine_pairs_each_weight_with_its_expert():
+    """Experts that differ only by a scale c_e of their down projection: the MoE output of
+    token t is (sum_j w[t,j] c_{e_j}) times one SwiGLU, with the top-k and the weights
+    found here by brute force over each token's router logits."""
+    cfg = _tiny_cfg(n_experts=5, top_k=3)
+    m = _M(cfg)
+    L = m.layers[0]
+    c = np.array([1.0, 2.0, 4.0, 8.0, 16.0])
+    for e in range(5):
+        L["w_gate"][e] = L["w_gate"][0]; L["w_up"][e] = L["w_up"][0]; L["w_down"][e] = c[e] * L["w_down"][0]
+    x = np.random.default_rng(12).standard_normal((11, cfg["hidden"]))
+    xn = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + cfg["rms_eps"])
+    got = O.moe(m, 0, x, O.Precision("f32"))
+    base = _swiglu(xn, L["w_gate"][0], L["w_up"][0], L["w_down"][0])
+    for t in range(11):
+        r = (xn[t] @ L["w_router"].T).tolist()
+        top = sorted(range(5), key=lambda e: (-r[e], e))[:3]
+        z = [math.exp(r[e] - r[top[0]]) for e in top]
+        scale = sum(zi / sum(z) * c[e] for zi, e in zip(z, top))
+        np.testing.assert_allclose(got[t], scale * base[t], rtol=1e-12, atol=1e-13)
+
+
 # ---------------------------------------------------------------- whole pass
 
 def test_single_token_pass_closed_form():
@@ -346,6 +379,43 @@ def test_chunked_prefill_equals_single_prefill():
         for l in range(2):
             np.testing.assert_allclose(two.k[l], one.k[l], rtol=tol, atol=tol)
             np.testing.assert_allclose(two.v[l], one.v[l], rtol=tol, atol=tol)
+
+
+def _is_nearest_bf16(stored, exact):
+    """Each stored value has 8 significant bits and lies within half a bf16 step of the exact one."""
+    st = np.asarray(stored, dtype=np.float64)
+    bits = st.astype(np.float32).view(np.uint32)
+    representable = np.all(st.astype(np.float32).astype(np.float64) == st) and np.all((bits & 0xFFFF) == 0)
+    _, e = np.frexp(exact)
+    half_step = np.ldexp(1.0, e - 9)
+    return representable and bool(np.all(np.abs(st - exact) <= half_step))
+
+
+def test_bf16_storage_rounds_what_prefill_writes_and_nothing_in_flight():
+    """The storage rule in a bf16 model: prefill rounds the K/V it writes to the nearest
+    bf16 value and nothing else, so its residual stream matches the f32 model's; a
+    denoising pass rounds only the vocabulary input, never the canvas K/V it computes."""
+    cfg = _tiny_cfg(n_layers=2)
+    m = _M(cfg)
+    toks = np.array([4, 8, 15, 16, 23, 2])
+    f32, b16 = O.Precision("f32"), O.Precision("bf16")
+    exact = O.prefill_append(m, O.Cache.empty(cfg), toks, f32)
+    stored = O.prefill_append(m, O.Cache.empty(cfg), toks, b16)
+    for l in range(2):
+        for a, b in ((stored.k[l], exact.k[l]), (stored.v[l], exact.v[l])):
+            assert _is_nearest_bf16(a, b)
+            assert np.abs(a - b).max() > 0
+    # a pass against a given cache: identical residual streams, logits differ only by the
+    # rounding of the final normed state
+    can = np.array([7, 30, 1])
+    lf, tf = O.denoise_pass(m, stored, can, f32)
+    lb, tb = O.denoise_pass(m, stored, can, b16)
+    for a, b in zip(tf, tb):
+        for key in ("attn_o", "x_attn", "x_out"):
+            np.testing.assert_array_equal(a[key], b[key])
+    xn = O.rms_norm(tf[-1]["x_out"], cfg["rms_eps"])
+    np.testing.assert_allclose(lb, O.round_bf16(xn) @ m.w_out.T, rtol=1e-12, atol=1e-13)
+    assert np.abs(lb - lf).max() > 0
 
 
 def test_denoise_pass_leaves_cache_untouched():
