@@ -10,6 +10,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <new>
 #include <string>
 #include <vector>
 
@@ -109,15 +110,18 @@ struct ProfScope {
   } while (0)
 
 // ---------------------------------------------------------------- tensor maps
-static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode{nullptr};
+static std::mutex g_encode_mu;
 static dg_status get_encoder() {
-  if (g_encode) return DG_OK;
+  if (g_encode.load(std::memory_order_acquire)) return DG_OK;
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (g_encode.load(std::memory_order_relaxed)) return DG_OK;
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
   cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
   if (e != cudaSuccess || fn == nullptr || q != cudaDriverEntryPointSuccess)
     return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(e));
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  g_encode.store(reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn), std::memory_order_release);
   return DG_OK;
 }
 
@@ -129,7 +133,7 @@ static dg_status encode_bf16(CUtensorMap* map, const void* base, int rank, const
   cuuint32_t bx[3], es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) gd[i] = dims[i], bx[i] = box[i];
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx,
+  CUresult r = g_encode.load(std::memory_order_acquire)(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx,
                         es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -198,18 +202,28 @@ extern "C" dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, 
   dg_status s = validate_config(cfg);
   if (s != DG_OK) return s;
   DG_CHECK_ARG(w && out && w->embed && w->w_out && w->layers, "weights / out pointer is NULL");
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  DG_CHECK_ARG(a16(w->embed) && a16(w->w_out), "embed / w_out must be 16-byte aligned");
   for (int l = 0; l < cfg->n_layers; ++l) {
     const dg_layer_weights& L = w->layers[l];
     DG_CHECK_ARG(L.w_qkv && L.w_o && L.w_router && L.w_gate && L.w_up && L.w_down, "layer %d has a NULL weight", l);
+    DG_CHECK_ARG(a16(L.w_qkv) && a16(L.w_o) && a16(L.w_router) && a16(L.w_gate) && a16(L.w_up) && a16(L.w_down),
+                 "layer %d: weights must be 16-byte aligned", l);
   }
-  dg_model* m = new dg_model();
+  dg_model* m = new (std::nothrow) dg_model();
+  if (!m) return fail(DG_ERR_CUDA, "out of host memory");
   m->cfg = *cfg;
   m->embed = w->embed;
   m->w_out = w->w_out;
-  m->layers.assign(w->layers, w->layers + cfg->n_layers);
+  try {
+    m->layers.assign(w->layers, w->layers + cfg->n_layers);
+    if (is_bf16(*cfg)) m->maps.resize(cfg->n_layers);
+  } catch (...) {
+    delete m;
+    return fail(DG_ERR_CUDA, "out of host memory");
+  }
   if (is_bf16(*cfg)) {
     const dg_config& c = *cfg;
-    m->maps.resize(c.n_layers);
     for (int l = 0; l < c.n_layers; ++l) {
       const dg_layer_weights& L = m->layers[l];
       LayerMaps& M = m->maps[l];
@@ -722,6 +736,22 @@ extern "C" dg_status dg_canvas_update_masked(const float* d_logits, int32_t C, i
   return DG_OK;
 }
 
+// Everything the passes, updates and the append of a generation call check, checked
+// before the first launch so that a rejected call launches nothing.
+static dg_status check_generate_args(dg_model* m, const dg_kv_cache* cache, const int32_t* d_canvas, int32_t C,
+                                     const float* d_logits, void* d_ws, size_t ws_bytes) {
+  DG_CHECK_ARG(d_canvas && d_logits, "canvas / logits is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_logits) & 15) == 0, "logits must be 16-byte aligned");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  if ((int64_t)cache->len + C > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
+                cache->capacity);
+  Ws ws;
+  return check_ws(m->cfg, d_ws, ws_bytes, C, &ws);
+}
+
 static int renoise_count(int C, int S, int s, double r0, double r1) {
   const double f = (S == 1) ? r0 : (r0 * (S - 1 - s) + r1 * s) / (double)(S - 1);
   return (int)floor((double)C * f + 1e-9);
@@ -737,12 +767,8 @@ extern "C" dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t
   DG_CHECK_ARG(m, "model is NULL");
   DG_CHECK_ARG(S >= 1, "S must be >= 1");
   DG_CHECK_ARG(r_start >= 0.f && r_start <= 1.f && r_end >= 0.f && r_end <= 1.f, "re-noise fractions must be in [0,1]");
-  DG_CHECK_ARG(C <= 1024, "C must be <= 1024");
-  dg_status s = check_cache(m->cfg, cache);
+  dg_status s = check_generate_args(m, cache, d_canvas, C, d_logits, d_ws, ws_bytes);
   if (s != DG_OK) return s;
-  if ((int64_t)cache->len + C > cache->capacity)
-    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
-                cache->capacity);
   for (int step = 0; step < S; ++step) {
     if ((s = dg_denoise_pass(m, cache, d_canvas, C, d_logits, d_ws, ws_bytes, stream)) != DG_OK) return s;
     const int n = renoise_count(C, S, step, r_start, r_end);
@@ -759,17 +785,12 @@ extern "C" dg_status dg_generate_canvas_masked(dg_model* m, dg_kv_cache* cache, 
                                                int32_t append, float* d_logits, void* d_ws, size_t ws_bytes,
                                                dg_stream stream) {
   DG_CHECK_ARG(m, "model is NULL");
-  DG_CHECK_ARG(d_canvas, "canvas is NULL");
   DG_CHECK_ARG(S >= 1, "S must be >= 1");
   DG_CHECK_ARG(keep_start >= 0.f && keep_start <= 1.f && keep_end >= 0.f && keep_end <= 1.f,
                "keep fractions must be in [0,1]");
-  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
   DG_CHECK_ARG(mask_id >= 0 && mask_id < m->cfg.vocab, "mask_id must be in [0, vocab)");
-  dg_status s = check_cache(m->cfg, cache);
+  dg_status s = check_generate_args(m, cache, d_canvas, C, d_logits, d_ws, ws_bytes);
   if (s != DG_OK) return s;
-  if ((int64_t)cache->len + C > cache->capacity)
-    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
-                cache->capacity);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   LAUNCH(DG_K_UPDATE_SELECT, st, dg::launch_fill_i32(d_canvas, C, mask_id, st));
   for (int step = 0; step < S; ++step) {

@@ -100,7 +100,9 @@ typedef struct dg_kv_cache {
 typedef struct dg_model dg_model;
 
 /* Validate the config, copy it and the weight pointers, and pre-encode the weight
- * tensor maps.  The weights must stay alive and unchanged while the model exists. */
+ * tensor maps.  The weights must stay alive and unchanged while the model exists.
+ * Every weight pointer must be 16-byte aligned (DG_ERR_INVALID_ARG otherwise): the
+ * kernels read embedding and router rows with 16-byte loads and TMA needs aligned bases. */
 dg_status dg_model_create(const dg_config* cfg, const dg_weights* w, dg_model** out);
 void dg_model_destroy(dg_model* m);
 
@@ -141,8 +143,9 @@ dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t V, int32_t 
  * cache by dg_prefill_append.  After pass s (0-based) the number of re-noised
  * positions is floor(C * f_s + 1e-9), f_s = (r_start (S-1-s) + r_end s) / (S-1)
  * (f_0 = r_start when S == 1); the update of pass s uses step = s.  d_canvas holds
- * the initial noise on entry and the result on return.  d_logits ([C][V]) receives
- * the last pass's logits. */
+ * the initial noise on entry and the result on return.  d_logits ([C][V], 16-byte
+ * aligned) receives the last pass's logits.  C <= 1024.  Every argument the passes,
+ * updates and append would check is checked before the first launch. */
 dg_status dg_generate_canvas(dg_model* m, dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t S,
                              float r_start, float r_end, uint64_t seed, int32_t append, float* d_logits,
                              void* d_ws, size_t ws_bytes, dg_stream stream);

@@ -91,3 +91,72 @@ def test_renoise_schedule_matches_golden():
     assert dg.renoise_count(256, 1, 0, 0.25, 0.25) == g["S1_C256_q25"][0]
     assert dg.renoise_count(32, 1, 0, 0.25, 0.25) == g["S1_C32_q25"][0]
     assert dg.renoise_count(256, 4, 4, 0.5, 0.0) == -1
+
+
+def _fake_model(cfg, misalign=None):
+    """A model over placeholder device addresses (never dereferenced).  fp32 models encode
+    no tensor maps, so dg_model_create needs no GPU for them."""
+    base = [1 << 20]
+
+    def addr(name):
+        base[0] += 1 << 16
+        return base[0] + (8 if name == misalign else 0)
+
+    L = cfg["n_layers"]
+    lw = (dg.LayerWeights * L)(*[dg.LayerWeights(*[addr(n) for n in ("w_qkv", "w_o", "w_router", "w_gate", "w_up",
+                                                                      "w_down")]) for _ in range(L)])
+    w = dg.Weights(addr("embed"), addr("w_out"), lw)
+    c = dg.make_config(cfg)
+    h = ctypes.c_void_p()
+    st = dg.lib.dg_model_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h))
+    return st, h
+
+
+@pytest.mark.parametrize("name", ["embed", "w_out", "w_qkv", "w_o", "w_router", "w_gate", "w_up", "w_down"])
+def test_misaligned_weights_rejected_on_host(name):
+    """Kernels read the embedding and router rows with 16-byte vector loads and TMA needs
+    16-byte aligned bases, so a weight that is not 16-byte aligned is refused at creation."""
+    st, h = _fake_model(CF.CONFIGS["tiny_fp32"], misalign=name)
+    assert st == dg.DG_ERR_INVALID_ARG and not h.value
+    assert "aligned" in dg.lib.dg_last_error().decode()
+
+
+def test_generation_rejects_bad_arguments_before_any_launch():
+    """The generation calls check what their passes, updates and append would check
+    before the first launch, so a rejected call launches nothing (the model and cache
+    here are placeholders that a launch would fault on)."""
+    cfg = CF.CONFIGS["tiny_fp32"]
+    st, h = _fake_model(cfg)
+    assert st == dg.DG_OK and h.value
+    try:
+        L = cfg["n_layers"]
+        ka = (ctypes.c_void_p * L)(*[(1 << 30) + (i << 16) for i in range(L)])
+        va = (ctypes.c_void_p * L)(*[(1 << 31) + (i << 16) for i in range(L)])
+        cache = dg.KVCacheS(ka, va, 256, 64)
+        C, S = 32, 2
+        ws_need = dg.workspace_bytes(cfg, C)
+        p, ws = ctypes.c_void_p(1 << 24), ctypes.c_void_p(1 << 25)
+        G, GM = dg.lib.dg_generate_canvas, dg.lib.dg_generate_canvas_masked
+
+        def gen(canvas=p, C=C, logits=p, ws=ws, ws_bytes=ws_need, S=S):
+            return G(h, ctypes.byref(cache), canvas, C, S, 0.5, 0.0, 7, 1, logits, ws, ws_bytes, None)
+
+        def genm(canvas=p, C=C, logits=p, ws=ws, ws_bytes=ws_need):
+            return GM(h, ctypes.byref(cache), canvas, C, S, 0.5, 0.0, 3, 1, logits, ws, ws_bytes, None)
+
+        launches = dg.lib.dg_launch_count()
+        for f in (gen, genm):
+            assert f(logits=ctypes.c_void_p((1 << 24) + 4)) == dg.DG_ERR_INVALID_ARG      # misaligned logits
+            assert "aligned" in dg.lib.dg_last_error().decode()
+            assert f(logits=None) == dg.DG_ERR_INVALID_ARG
+            assert f(canvas=None) == dg.DG_ERR_INVALID_ARG
+            assert f(C=0) == dg.DG_ERR_INVALID_ARG
+            assert f(C=1025) == dg.DG_ERR_INVALID_ARG
+            assert f(ws=None) == dg.DG_ERR_INVALID_ARG
+            assert f(ws=ctypes.c_void_p((1 << 25) + 128)) == dg.DG_ERR_INVALID_ARG     # workspace alignment
+            assert f(ws_bytes=ws_need - 256) == dg.DG_ERR_CAPACITY
+            assert f(C=256 - 64 + 8) == dg.DG_ERR_CAPACITY                              # no room in the cache
+        assert gen(S=0) == dg.DG_ERR_INVALID_ARG
+        assert dg.lib.dg_launch_count() == launches          # no launch was even attempted
+    finally:
+        dg.lib.dg_model_destroy(h)
