@@ -644,6 +644,183 @@ dg_status run_stack(dg_model* m, const dg_kv_cache* cache, const int32_t* tokens
   return DG_OK;
 }
 
+// ---- several canvases in one pass
+// Canvas b occupies rows [b C, (b + 1) C) of every row-wise buffer and reads and writes
+// only its own cache; all rows share one router / permutation / expert GEMM / vocabulary
+// projection, so an expert's weights are read once for the whole batch.
+struct Seg {
+  void* kc;
+  void* vtc;
+  int cap;
+  int pos0;  // the canvas's cache length
+};
+
+// A view of the workspace whose q / o buffers start at canvas b's slice: q is head-major
+// [nq][C][d] per canvas, o row-major [C][nq d], so both slices are contiguous.
+Ws canvas_view(const dg_config& c, const Ws& ws, int b, int C) {
+  Ws wb = ws;
+  const size_t qo = (size_t)b * c.n_q_heads * C * c.head_dim;  // elements before canvas b (q and o alike)
+  wb.L.q += qo * act_bytes(c);
+  wb.L.o += qo * act_bytes(c);
+  if (is_bf16(c)) {
+    wb.L.q_lo += qo * 2;
+    wb.L.o_lo += qo * 2;
+  }
+  return wb;
+}
+
+template <typename T>
+dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>& segs, int C, int causal,
+                        bool stop_after_kv, bool final_layer, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const dg_layer_weights& W = m->layers[l];
+  const int H = c.hidden, nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
+  const int E = c.n_experts, k = c.top_k, F = c.expert_ffn, QR = qkv_rows(c);
+  const int n = (int)segs.size() * C;
+  const bool bf = is_bf16(c);
+  int* err = ws.err();
+  T* xn_lo = bf ? ws.at<T>(ws.L.xn_lo) : nullptr;
+  dg_status s;
+  int ks_qkv = 1, ks_o = 1;
+  if (bf) {
+    ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
+    GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
+               nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm};
+    if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
+  } else {
+    LAUNCH(DG_K_GEMM_QKV, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_qkv, ws.at<float>(ws.L.xn), nullptr, 1, n, n, QR, H,
+                                    ws.at<float>(ws.L.qkv), QR, st));
+  }
+  // per canvas: RoPE at its own positions, K/V into its own cache, attention over its own
+  // keys (the low-term window and the split-KV partials are reused canvas after canvas)
+  for (int b = 0; b < (int)segs.size(); ++b) {
+    const Seg& g = segs[b];
+    const Ws wb = canvas_view(c, ws, b, C);
+    LAUNCH(DG_K_ROPE_KV, st,
+           dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv) + (size_t)b * C * QR, ks_qkv, (size_t)n * QR, C, nq, nkv,
+                                      d, g.pos0, c.rope_theta, wb.at<T>(wb.L.q), (T*)g.kc, (T*)g.vtc, g.cap,
+                                      bf ? wb.at<T>(wb.L.q_lo) : nullptr, bf ? ws.at<T>(ws.L.k_lo) : nullptr,
+                                      bf ? ws.at<T>(ws.L.vt_lo) : nullptr, (g.pos0 / 128) * 128, ws.L.lo_rows, st));
+    if (stop_after_kv) continue;
+    if ((s = attention(c, wb, g.kc, g.vtc, g.cap, C, g.pos0, g.pos0 + C, causal, st)) != DG_OK) return s;
+  }
+  if (stop_after_kv) return DG_OK;
+  if (bf) {
+    ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
+    GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
+               n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
+               kSmemGemm};
+    if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
+  } else {
+    LAUNCH(DG_K_GEMM_O, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_o, ws.at<float>(ws.L.o), nullptr, 1, n, n, H, nq * d,
+                                    ws.at<float>(ws.L.opart), H, st));
+  }
+  LAUNCH(DG_K_ROUTER, st,
+         dg::launch_router_fused<T>(ws.at<float>(ws.L.x), ws.at<float>(ws.L.opart), ks_o, (size_t)n * H, W.w_router,
+                                    n, H, E, k, c.rms_eps, nullptr, ws.at<int32_t>(ws.L.topk_idx),
+                                    ws.at<float>(ws.L.topk_w), ws.at<T>(ws.L.xn), xn_lo, st));
+  const bool taps = m->taps_on && n <= m->tap_rows;
+  if (taps && !m->tap_x_attn.empty() && m->tap_x_attn[l])
+    if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return fail(DG_ERR_CUDA, "tap copy failed");
+  LAUNCH(DG_K_PERMUTE, st,
+         dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
+                            ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
+                            ws.at<int32_t>(ws.L.uni), kItemRows, ws.at<dg::TcWorkItem>(ws.L.items),
+                            ws.at<int>(ws.L.n_items), st));
+  T* xs_lo = bf ? ws.at<T>(ws.L.xs_lo) : nullptr;
+  LAUNCH(DG_K_GATHER, st,
+         dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), xn_lo, ws.at<int32_t>(ws.L.perm), n * k, k, H,
+                                   ws.at<T>(ws.L.xs), xs_lo, st));
+  const int* off = ws.at<int>(ws.L.offsets);
+  if (bf) {
+    const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
+    const int* n_items = ws.at<int>(ws.L.n_items);
+    const int max_items = n * k / kItemRows + E;
+    GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &m->maps[l].gate, &m->maps[l].up, ws.at<void>(ws.L.xs), xs_lo,
+                n * k, H, F, items, n_items, max_items, kItemRows, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
+                kSmemGemm};
+    if ((s = gemm_bf16(gu, err, st)) != DG_OK) return s;
+    GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &m->maps[l].down, nullptr, ws.at<void>(ws.L.h),
+                ws.at<void>(ws.L.h_lo), n * k, F, H, items, n_items, max_items, kItemRows, ws.at<float>(ws.L.ys),
+                nullptr, H, 1, 0, kSmemGemm};
+    if ((s = gemm_bf16(dn, err, st)) != DG_OK) return s;
+  } else {
+    float* g = ws.at<float>(ws.L.gu);
+    float* u = g + (size_t)n * k * F;
+    LAUNCH(DG_K_GEMM_GATE_UP, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_gate, ws.at<float>(ws.L.xs), off, E, n, n * k, F, H, g, F,
+                                    st));
+    LAUNCH(DG_K_GEMM_GATE_UP, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_up, ws.at<float>(ws.L.xs), off, E, n, n * k, F, H, u, F,
+                                    st));
+    LAUNCH(DG_K_SWIGLU, st, dg::launch_swiglu_f32(g, u, n * k, F, ws.at<float>(ws.L.h), st));
+    LAUNCH(DG_K_GEMM_DOWN, st,
+           dg::launch_simt_gemm_f32(0, (const float*)W.w_down, ws.at<float>(ws.L.h), off, E, n, n * k, H, F,
+                                    ws.at<float>(ws.L.ys), H, st));
+  }
+  LAUNCH(DG_K_COMBINE, st,
+         dg::launch_combine_norm<T>(ws.at<float>(ws.L.ys), ws.at<int32_t>(ws.L.inv), ws.at<float>(ws.L.topk_w), n, k,
+                                    H, c.rms_eps, ws.at<float>(ws.L.x), ws.at<T>(ws.L.xn),
+                                    final_layer ? nullptr : xn_lo, st));
+  if (taps) {
+    auto cp = [&](void* dst, const void* src, size_t bytes) {
+      return dst ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
+    };
+    cudaError_t e = cudaSuccess;
+    if (!m->tap_x_out.empty()) e = cp(m->tap_x_out[l], ws.at<float>(ws.L.x), (size_t)n * H * 4);
+    if (e == cudaSuccess && !m->tap_topk_idx.empty())
+      e = cp(m->tap_topk_idx[l], ws.at<int32_t>(ws.L.topk_idx), (size_t)n * k * 4);
+    if (e == cudaSuccess && !m->tap_topk_w.empty())
+      e = cp(m->tap_topk_w[l], ws.at<float>(ws.L.topk_w), (size_t)n * k * 4);
+    if (e == cudaSuccess && !m->tap_counts.empty()) e = cp(m->tap_counts[l], ws.at<int32_t>(ws.L.counts), E * 4);
+    if (e == cudaSuccess && !m->tap_perm.empty())
+      e = cp(m->tap_perm[l], ws.at<int32_t>(ws.L.perm), (size_t)n * k * 4);
+    if (e == cudaSuccess && m->tap_unions) e = cp(m->tap_unions + l, ws.at<int32_t>(ws.L.uni), 4);
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "tap copy failed: %s", cudaGetErrorString(e));
+  }
+  return DG_OK;
+}
+
+template <typename T>
+dg_status run_stack_batched(dg_model* m, const dg_kv_cache* caches, int B, const int32_t* tokens, int C, bool prefill,
+                            const Ws& ws, cudaStream_t st) {
+  const dg_config& c = m->cfg;
+  const int n = B * C;
+  T* xn_lo = is_bf16(c) ? ws.at<T>(ws.L.xn_lo) : nullptr;
+  LAUNCH(DG_K_EMBED_NORM, st,
+         dg::launch_embed_norm<T>(tokens, (const T*)m->embed, n, c.vocab, c.hidden, c.rms_eps, ws.at<float>(ws.L.x),
+                                  ws.at<T>(ws.L.xn), xn_lo, ws.err(), st));
+  std::vector<Seg> segs(B);
+  for (int l = 0; l < c.n_layers; ++l) {
+    for (int b = 0; b < B; ++b) segs[b] = Seg{caches[b].k[l], caches[b].vt[l], caches[b].capacity, caches[b].len};
+    const bool last = l == c.n_layers - 1;
+    dg_status s = layer_batched<T>(m, l, ws, segs, C, prefill ? 1 : 0, last && prefill, last && !prefill, st);
+    if (s != DG_OK) return s;
+  }
+  return DG_OK;
+}
+
+// the caches of a batch: each valid, with room for C more positions, none shared
+dg_status check_caches(const dg_config& c, const dg_kv_cache* caches, int B, int C) {
+  DG_CHECK_ARG(caches && B >= 1, "caches NULL or B < 1");
+  for (int b = 0; b < B; ++b) {
+    dg_status s = check_cache(c, &caches[b]);
+    if (s != DG_OK) return s;
+    if ((int64_t)caches[b].len + C > caches[b].capacity)
+      return fail(DG_ERR_CAPACITY, "cache %d has no room for the canvas: len %d + C %d > capacity %d", b,
+                  caches[b].len, C, caches[b].capacity);
+    for (int b2 = 0; b2 < b; ++b2)
+      for (int l = 0; l < c.n_layers; ++l)
+        DG_CHECK_ARG(caches[b].k[l] != caches[b2].k[l] && caches[b].vt[l] != caches[b2].vt[l],
+                     "caches %d and %d share layer %d's buffers", b2, b, l);
+  }
+  return DG_OK;
+}
+
 }  // namespace
 
 extern "C" dg_status dg_prefill_append(dg_model* m, dg_kv_cache* cache, const int32_t* d_tokens, int32_t T,
@@ -801,6 +978,86 @@ extern "C" dg_status dg_generate_canvas_masked(dg_model* m, dg_kv_cache* cache, 
       return s;
   }
   if (append) return dg_prefill_append(m, cache, d_canvas, C, d_ws, ws_bytes, stream);
+  return DG_OK;
+}
+
+extern "C" dg_status dg_prefill_append_batched(dg_model* m, dg_kv_cache* caches, int32_t B, const int32_t* d_tokens,
+                                               int32_t T, void* d_ws, size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(d_tokens && T > 0, "tokens NULL or T <= 0");
+  DG_CHECK_ARG(B >= 1 && (int64_t)B * T <= (1 << 20), "B must be >= 1 and B * T <= 2^20");
+  dg_status s = check_caches(m->cfg, caches, B, T);
+  if (s != DG_OK) return s;
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, B * T, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = is_bf16(m->cfg) ? run_stack_batched<bf16>(m, caches, B, d_tokens, T, true, ws, st)
+                      : run_stack_batched<float>(m, caches, B, d_tokens, T, true, ws, st);
+  if (s != DG_OK) return s;
+  for (int b = 0; b < B; ++b) caches[b].len += T;
+  return DG_OK;
+}
+
+extern "C" dg_status dg_denoise_pass_batched(dg_model* m, const dg_kv_cache* caches, int32_t B,
+                                             const int32_t* d_canvases, int32_t C, float* d_logits, void* d_ws,
+                                             size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(d_canvases && d_logits && C > 0, "canvases / logits NULL or C <= 0");
+  DG_CHECK_ARG(B >= 1 && (int64_t)B * C <= (1 << 20), "B must be >= 1 and B * C <= 2^20");
+  dg_status s = check_caches(m->cfg, caches, B, C);
+  if (s != DG_OK) return s;
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, B * C, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dg_config& c = m->cfg;
+  const int n = B * C;
+  s = is_bf16(c) ? run_stack_batched<bf16>(m, caches, B, d_canvases, C, false, ws, st)
+                 : run_stack_batched<float>(m, caches, B, d_canvases, C, false, ws, st);
+  if (s != DG_OK) return s;
+  if (is_bf16(c)) {
+    GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, n, c.hidden,
+               c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm};
+    if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
+  } else {
+    LAUNCH(DG_K_GEMM_VOCAB, st,
+           dg::launch_simt_gemm_f32(0, (const float*)m->w_out, ws.at<float>(ws.L.xn), nullptr, 1, n, n, c.vocab,
+                                    c.hidden, d_logits, c.vocab, st));
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases, int32_t C,
+                                          int32_t S, float r_start, float r_end, const uint64_t* seeds,
+                                          int32_t append, float* d_logits, void* d_ws, size_t ws_bytes,
+                                          dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(S >= 1, "S must be >= 1");
+  DG_CHECK_ARG(r_start >= 0.f && r_start <= 1.f && r_end >= 0.f && r_end <= 1.f, "re-noise fractions must be in [0,1]");
+  DG_CHECK_ARG(seeds, "seeds is NULL");
+  DG_CHECK_ARG(d_canvases && d_logits, "canvases / logits is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(B >= 1 && (int64_t)B * C <= (1 << 20), "B must be >= 1 and B * C <= 2^20");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_logits) & 15) == 0, "logits must be 16-byte aligned");
+  dg_status s = check_caches(m->cfg, caches, B, C);
+  if (s != DG_OK) return s;
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, B * C, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int V = m->cfg.vocab, n = B * C;
+  const int splits = dg::update_splits(n, V);
+  dg::UpdPart* part = ws.at<dg::UpdPart>(ws.L.upd);
+  for (int step = 0; step < S; ++step) {
+    if ((s = dg_denoise_pass_batched(m, caches, B, d_canvases, C, d_logits, d_ws, ws_bytes, stream)) != DG_OK)
+      return s;
+    const int nr = renoise_count(C, S, step, r_start, r_end);
+    // row statistics of all B C rows at once, then each canvas's own re-noise set
+    LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, n, V, splits, -1, part, st));
+    for (int b = 0; b < B; ++b)
+      LAUNCH(DG_K_UPDATE_SELECT, st,
+             dg::launch_update_select(part + (size_t)b * C * splits, C, V, splits, nr, seeds[b], (uint32_t)step,
+                                      d_canvases + (size_t)b * C, nullptr, -1, st));
+  }
+  if (append) return dg_prefill_append_batched(m, caches, B, d_canvases, C, d_ws, ws_bytes, stream);
   return DG_OK;
 }
 

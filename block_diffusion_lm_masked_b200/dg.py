@@ -77,6 +77,9 @@ def _load():
         "dg_generate_canvas_masked": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, I32, I32, P, P, SZ,
                                             P]),
         "dg_generate_canvas": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, U64, I32, P, P, SZ, P]),
+        "dg_prefill_append_batched": (I32, [P, P, I32, P, I32, P, SZ, P]),
+        "dg_denoise_pass_batched": (I32, [P, P, I32, P, I32, P, P, SZ, P]),
+        "dg_generate_canvases": (I32, [P, P, I32, P, I32, I32, F32, F32, P, I32, P, P, SZ, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
         "dg_set_taps": (I32, [P, ctypes.POINTER(Taps)]),
@@ -302,6 +305,40 @@ def generate_canvas_masked(model: Model, cache: KVCache, canvas: torch.Tensor, S
     _check(lib.dg_generate_canvas_masked(model.handle, ctypes.byref(cache.s), _ptr(canvas), canvas.numel(), S,
                                          keep_start, keep_end, mask_id, 1 if append else 0, _ptr(logits), ws.ptr,
                                          ws.nbytes, _stream(stream)))
+
+
+def _caches(caches):
+    """Host array of the caches' C structs (copies; lens are copied back after a call that advances them)."""
+    return (KVCacheS * len(caches))(*[c.s for c in caches])
+
+
+def prefill_append_batched(model: Model, caches: list, tokens: torch.Tensor, ws: Workspace, stream=None):
+    """tokens int32 [B][T]: row b is appended to caches[b]."""
+    B, T = tokens.shape
+    arr = _caches(caches)
+    _check(lib.dg_prefill_append_batched(model.handle, arr, B, _ptr(tokens), T, ws.ptr, ws.nbytes, _stream(stream)))
+    for c, s in zip(caches, arr):
+        c.len = s.len
+
+
+def denoise_pass_batched(model: Model, caches: list, canvases: torch.Tensor, logits: torch.Tensor, ws: Workspace,
+                         stream=None):
+    """canvases int32 [B][C], logits fp32 [B][C][V]; canvas b attends to caches[b] only."""
+    B, C = canvases.shape
+    _check(lib.dg_denoise_pass_batched(model.handle, _caches(caches), B, _ptr(canvases), C, _ptr(logits), ws.ptr,
+                                       ws.nbytes, _stream(stream)))
+
+
+def generate_canvases(model: Model, caches: list, canvases: torch.Tensor, S: int, r_start: float, r_end: float,
+                      seeds, append: bool, logits: torch.Tensor, ws: Workspace, stream=None):
+    """generate_canvas for B canvases at once; canvas b re-noised from seeds[b]."""
+    B, C = canvases.shape
+    arr = _caches(caches)
+    sd = (ctypes.c_uint64 * B)(*[int(x) & 0xFFFFFFFFFFFFFFFF for x in seeds])
+    _check(lib.dg_generate_canvases(model.handle, arr, B, _ptr(canvases), C, S, r_start, r_end, sd,
+                                    1 if append else 0, _ptr(logits), ws.ptr, ws.nbytes, _stream(stream)))
+    for c, s in zip(caches, arr):
+        c.len = s.len
 
 
 def device_status(ws, stream=None):

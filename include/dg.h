@@ -172,6 +172,29 @@ dg_status dg_generate_canvas_masked(dg_model* m, dg_kv_cache* cache, int32_t* d_
                                     float keep_start, float keep_end, int32_t mask_id, int32_t append,
                                     float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream);
 
+/* Several canvases in one call.  Canvas b (0 <= b < B) is a separate request with its
+ * own KV cache caches[b] (host array of B caches that share no buffers; each must have
+ * room for C more positions) and its own positions caches[b].len ..; it attends only to
+ * its own cache and its own canvas.  Row-wise buffers hold the canvases one after
+ * another: tokens / canvases int32 [B][C], logits fp32 [B][C][V].  Each canvas's result
+ * is the one the single-canvas call gives it (up to fp32 summation order: split-K factors
+ * follow the row count); the router, the expert GEMMs and the vocabulary projection run
+ * once over all B C rows, so each used expert's weights are read once per batch instead
+ * of once per canvas (Hacker News discussion of DiffusionGemma, the comment on batching:
+ * batched requests share the reads of common weights).  Workspace:
+ * dg_workspace_bytes(cfg, B * C).  B * C <= 2^20. */
+dg_status dg_prefill_append_batched(dg_model* m, dg_kv_cache* caches, int32_t B, const int32_t* d_tokens, int32_t T,
+                                    void* d_ws, size_t ws_bytes, dg_stream stream);
+dg_status dg_denoise_pass_batched(dg_model* m, const dg_kv_cache* caches, int32_t B, const int32_t* d_canvases,
+                                  int32_t C, float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream);
+/* dg_generate_canvas for B canvases at once: the same schedule for all, canvas b
+ * re-noised from the stream seeded with seeds[b] (host array [B]); the append (if any)
+ * writes canvas b into caches[b].  C <= 1024; every argument is checked before the first
+ * launch. */
+dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases, int32_t C, int32_t S,
+                               float r_start, float r_end, const uint64_t* seeds, int32_t append, float* d_logits,
+                               void* d_ws, size_t ws_bytes, dg_stream stream);
+
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
 

@@ -547,6 +547,44 @@ def generate_canvas(model, cache: Cache, canvas: np.ndarray, S: int, r_start: fl
 
 
 # ----------------------------------------------------------------------------
+# several canvases at once
+
+
+def denoise_pass_batched(model, caches: list, canvases, prec: Precision):
+    """Denoising passes of B independent canvases, canvas b against its own cache.
+
+    Batching shares weight reads, not arithmetic: each canvas attends only to its own
+    cache and its own canvas (one request each), and every per-token step (routing,
+    experts, vocabulary projection) is row-wise, so canvas b's result is its
+    single-canvas pass.  Returns [(logits, taps)] per canvas.
+    """
+    return [denoise_pass(model, c, np.asarray(x), prec) for c, x in zip(caches, canvases)]
+
+
+def merge_batch_taps(per_canvas_taps: list, n_experts: int) -> list:
+    """Per-layer taps of a batch from the canvases' own taps: row-wise entries stacked in
+    canvas order; the expert histogram, stable permutation and union taken over all rows
+    together, as one pass over the batch groups them."""
+    out = []
+    for layer_taps in zip(*per_canvas_taps):
+        m = {key: np.concatenate([t[key] for t in layer_taps], axis=0)
+             for key in ("x_in", "attn_o", "x_attn", "x_out", "router_logits", "topk_idx", "topk_w", "router_margin")}
+        counts, offsets, perm, inv, union = expert_permutation(m["topk_idx"], n_experts)
+        m.update(counts=counts, offsets=offsets, perm=perm, union=union)
+        out.append(m)
+    return out
+
+
+def generate_canvases(model, caches: list, canvases, S: int, r_start: float, r_end: float, seeds, prec: Precision,
+                      append: bool):
+    """generate_canvas for each canvas with its own cache and re-noise seed.  Returns
+    ([canvas], [cache])."""
+    res = [generate_canvas(model, c, x, S, r_start, r_end, sd, prec, append)
+           for c, x, sd in zip(caches, canvases, seeds)]
+    return [r[0] for r in res], [r[1] for r in res]
+
+
+# ----------------------------------------------------------------------------
 # 8-bit expert weights (groundwork for the FP8 deployment the pages mention): the OCP
 # "E4M3" element format and MX block scaling, written from the published definitions.
 # Nothing in the pass uses these yet.

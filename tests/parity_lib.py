@@ -68,18 +68,21 @@ class Setup:
         return dg.Workspace(self.cfg, max_tokens, self.device)
 
     def taps(self, C):
-        cfg = self.cfg
-        L, H, k, E = cfg["n_layers"], cfg["hidden"], cfg["top_k"], cfg["n_experts"]
-        dev = self.device
-        t = dict(x_attn=[torch.zeros(C, H, device=dev) for _ in range(L)],
-                 x_out=[torch.zeros(C, H, device=dev) for _ in range(L)],
-                 topk_idx=[torch.zeros(C, k, dtype=torch.int32, device=dev) for _ in range(L)],
-                 topk_w=[torch.zeros(C, k, device=dev) for _ in range(L)],
-                 counts=[torch.zeros(E, dtype=torch.int32, device=dev) for _ in range(L)],
-                 perm=[torch.zeros(C * k, dtype=torch.int32, device=dev) for _ in range(L)],
-                 unions=torch.zeros(L, dtype=torch.int32, device=dev), rows=C)
-        self.model.set_taps(t)
-        return t
+        return make_taps(self.model, self.cfg, C, self.device)
+
+
+def make_taps(model, cfg, C, device="cuda"):
+    """Per-layer tap buffers for calls of up to C rows, installed on the model."""
+    L, H, k, E = cfg["n_layers"], cfg["hidden"], cfg["top_k"], cfg["n_experts"]
+    t = dict(x_attn=[torch.zeros(C, H, device=device) for _ in range(L)],
+             x_out=[torch.zeros(C, H, device=device) for _ in range(L)],
+             topk_idx=[torch.zeros(C, k, dtype=torch.int32, device=device) for _ in range(L)],
+             topk_w=[torch.zeros(C, k, device=device) for _ in range(L)],
+             counts=[torch.zeros(E, dtype=torch.int32, device=device) for _ in range(L)],
+             perm=[torch.zeros(C * k, dtype=torch.int32, device=device) for _ in range(L)],
+             unions=torch.zeros(L, dtype=torch.int32, device=device), rows=C)
+    model.set_taps(t)
+    return t
 
 
 def compare_pass(cfg, taps_gpu, logits_gpu, taps_o, logits_o, report=None, exempt=None):

@@ -160,3 +160,59 @@ def test_generation_rejects_bad_arguments_before_any_launch():
         assert dg.lib.dg_launch_count() == launches          # no launch was even attempted
     finally:
         dg.lib.dg_model_destroy(h)
+
+
+def test_batched_calls_reject_bad_arguments_before_any_launch():
+    """The batched entry points check every cache (valid, room for the canvas, no buffer
+    shared with another canvas of the batch) and the workspace for B * C rows before the
+    first launch."""
+    cfg = CF.CONFIGS["tiny_fp32"]
+    st, h = _fake_model(cfg)
+    assert st == dg.DG_OK
+    try:
+        L, C, B = cfg["n_layers"], 16, 3
+
+        def cache(i, length=8, cap=64, share_with=None):
+            j = i if share_with is None else share_with
+            ka = (ctypes.c_void_p * L)(*[(1 << 32) + (j << 24) + (l << 16) for l in range(L)])
+            va = (ctypes.c_void_p * L)(*[(1 << 33) + (j << 24) + (l << 16) for l in range(L)])
+            return dg.KVCacheS(ka, va, cap, length), (ka, va)
+
+        def batch(*specs):
+            made = [cache(i, **kw) for i, kw in enumerate(specs)]
+            return (dg.KVCacheS * len(made))(*[m[0] for m in made]), made
+
+        good, keep = batch({}, {}, {})
+        ws_need = dg.workspace_bytes(cfg, B * C)
+        p, ws = ctypes.c_void_p(1 << 24), ctypes.c_void_p(1 << 25)
+        seeds = (ctypes.c_uint64 * B)(1, 2, 3)
+        lib = dg.lib
+        launches = lib.dg_launch_count()
+
+        def den(caches=good, B=B, C=C, ws_bytes=ws_need, logits=p):
+            return lib.dg_denoise_pass_batched(h, caches, B, p, C, logits, ws, ws_bytes, None)
+
+        def pre(caches=good, B=B, C=C, ws_bytes=ws_need):
+            return lib.dg_prefill_append_batched(h, caches, B, p, C, ws, ws_bytes, None)
+
+        def gen(caches=good, B=B, C=C, ws_bytes=ws_need, logits=p, sd=seeds):
+            return lib.dg_generate_canvases(h, caches, B, p, C, 2, 0.5, 0.0, sd, 1, logits, ws, ws_bytes, None)
+
+        shared, k2 = batch({}, {"share_with": 0}, {})
+        full, k3 = batch({}, {}, {"length": 60})
+        for f in (den, pre, gen):
+            assert f(caches=None) == dg.DG_ERR_INVALID_ARG
+            assert f(B=0) == dg.DG_ERR_INVALID_ARG
+            assert f(C=0) == dg.DG_ERR_INVALID_ARG
+            assert f(caches=shared) == dg.DG_ERR_INVALID_ARG
+            assert "share" in lib.dg_last_error().decode()
+            assert f(caches=full) == dg.DG_ERR_CAPACITY
+            assert "cache 2" in lib.dg_last_error().decode()
+            assert f(ws_bytes=dg.workspace_bytes(cfg, C)) == dg.DG_ERR_CAPACITY     # sized for one canvas
+        assert gen(logits=ctypes.c_void_p((1 << 24) + 8)) == dg.DG_ERR_INVALID_ARG
+        assert gen(sd=None) == dg.DG_ERR_INVALID_ARG
+        assert gen(C=1025) == dg.DG_ERR_INVALID_ARG
+        assert lib.dg_launch_count() == launches
+        assert [good[i].len for i in range(B)] == [8, 8, 8]                        # nothing advanced
+    finally:
+        dg.lib.dg_model_destroy(h)

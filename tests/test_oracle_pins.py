@@ -429,6 +429,53 @@ def test_denoise_pass_leaves_cache_untouched():
         np.testing.assert_array_equal(cache.v[l], before.v[l])
 
 
+# ---------------------------------------------------------------- several canvases
+
+def test_batch_reads_the_union_of_the_canvases_experts():
+    """A batch of canvases groups all rows by expert at once: its histogram is the sum of
+    the canvases' histograms and the experts it reads are the set union of theirs, never
+    more than the sum of the per-canvas unions (the bytes a batch saves)."""
+    cfg = _tiny_cfg(n_layers=2, n_experts=8, top_k=2)
+    m = _M(cfg)
+    prec = O.Precision("f32")
+    rng = np.random.default_rng(21)
+    caches = [O.prefill_append(m, O.Cache.empty(cfg), rng.integers(0, 40, P), prec) if P else O.Cache.empty(cfg)
+              for P in (3, 0, 7)]
+    canvases = [rng.integers(0, 40, 5) for _ in range(3)]
+    res = O.denoise_pass_batched(m, caches, canvases, prec)
+    merged = O.merge_batch_taps([t for _, t in res], cfg["n_experts"])
+    for l in range(2):
+        sets = [set(t[l]["topk_idx"].reshape(-1).tolist()) for _, t in res]
+        assert merged[l]["union"] == len(set().union(*sets)) <= sum(len(x) for x in sets)
+        np.testing.assert_array_equal(merged[l]["counts"], sum(t[l]["counts"] for _, t in res))
+        assert merged[l]["counts"].sum() == 3 * 5 * 2
+        # the batch permutation is the stable grouping of the stacked routing
+        flat = merged[l]["topk_idx"].reshape(-1)
+        assert list(merged[l]["perm"]) == sorted(range(flat.size), key=lambda a: (int(flat[a]), a))
+
+
+def test_batched_canvases_do_not_see_each_other():
+    """Each canvas of a batch is its own request: replacing another canvas's tokens or
+    cache leaves its logits exactly unchanged, and a batch of one is the single pass."""
+    cfg = _tiny_cfg(n_layers=2)
+    m = _M(cfg)
+    prec = O.Precision("f32")
+    rng = np.random.default_rng(22)
+    c0 = O.prefill_append(m, O.Cache.empty(cfg), rng.integers(0, 40, 4), prec)
+    c1 = O.prefill_append(m, O.Cache.empty(cfg), rng.integers(0, 40, 6), prec)
+    x0, x1 = rng.integers(0, 40, 5), rng.integers(0, 40, 5)
+    a = O.denoise_pass_batched(m, [c0, c1], [x0, x1], prec)
+    b = O.denoise_pass_batched(m, [c0, O.Cache.empty(cfg)], [x0, rng.integers(0, 40, 5)], prec)
+    np.testing.assert_array_equal(a[0][0], b[0][0])
+    single, _ = O.denoise_pass(m, c0, x0, prec)
+    np.testing.assert_array_equal(a[0][0], single)
+    outs, caches = O.generate_canvases(m, [c0, c1], [x0, x1], 3, 0.5, 0.0, [5, 6], prec, True)
+    one, cache_one = O.generate_canvas(m, c1, x1, 3, 0.5, 0.0, 6, prec, True)
+    np.testing.assert_array_equal(outs[1], one)
+    assert caches[0].len == c0.len + 5 and caches[1].len == cache_one.len
+
+
+# ---------------------------------------------------------------- canvas update
 # ---------------------------------------------------------------- canvas update
 
 def test_canvas_update_special_cases():
