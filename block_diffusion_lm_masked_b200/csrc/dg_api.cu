@@ -139,6 +139,35 @@ static dg_status encode_bf16(CUtensorMap* map, const void* base, int rank, const
   if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return DG_OK;
 }
+// byte tensor (8-bit weight codes or their scales), up to 3 dims (dims[0] innermost)
+static dg_status encode_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  if (get_encoder() != DG_OK) return DG_ERR_CUDA;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) gd[i] = dims[i], bx[i] = box[i];
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = g_encode.load(std::memory_order_acquire)(
+      map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", (int)r);
+  return DG_OK;
+}
+// 8-bit weight codes [groups][rows][cols] as a 3-D map, box (64 cols, 128 rows, 1 group),
+// 64-byte swizzle; rows past a group's end read as zero codes
+static dg_status map_codes(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const uint64_t dims[3] = {cols, rows, groups};
+  const uint64_t strides[2] = {cols, rows * cols};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+// their scales [groups][cols / 64][rows][2] as a 3-D map, box (256 bytes = 128 rows, 1, 1)
+static dg_status map_scales(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const uint64_t dims[3] = {rows * 2, cols / 64, groups};
+  const uint64_t strides[2] = {rows * 2, (cols / 64) * rows * 2};
+  const uint32_t box[3] = {256, 1, 1};
+  return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
 // row-major [rows][cols] bf16 matrix as a 2-D map with box (64 cols, box_rows rows)
 static dg_status map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   const uint64_t dims[2] = {cols, rows};
@@ -1168,6 +1197,76 @@ extern "C" dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t r
              K, rows, group_off ? items : nullptr, group_off ? n_items : nullptr, max_items, n_max, out, out_lo,
              ld_out, 1, 0, kSmemGemm};
   return gemm_bf16(g, d_err, st);
+}
+
+extern "C" dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, const void* W2, const void* W2_scales,
+                                       int32_t rows, int32_t n_groups, const void* X, const void* X_lo,
+                                       int32_t x_rows, int32_t K, const int32_t* group_off, void* out, void* out_lo,
+                                       int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
+                                       dg_stream stream) {
+  DG_CHECK_ARG(W && W_scales && X && out && d_err && d_scratch, "NULL pointer");
+  DG_CHECK_ARG(!W2 == !W2_scales, "W2 and its scales come together");
+  DG_CHECK_ARG(K > 0 && K % 64 == 0 && rows > 0 && rows % 8 == 0 && n_groups > 0 && x_rows > 0, "bad GEMM shape");
+  DG_CHECK_ARG(ld_out >= rows, "ld_out < rows");
+  DG_CHECK_ARG(group_off || n_groups == 1, "several groups need group_off");
+  auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  DG_CHECK_ARG(a16(W) && a16(W_scales) && a16(X) && (!X_lo || a16(X_lo)) && (!W2 || (a16(W2) && a16(W2_scales))),
+               "operands must be 16-byte aligned");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_scratch) & 255) == 0, "scratch must be 256-byte aligned");
+  if (scratch_bytes < dg_debug_gemm_scratch_bytes(x_rows, n_groups))
+    return fail(DG_ERR_CAPACITY, "scratch too small: %zu < %zu", scratch_bytes,
+                dg_debug_gemm_scratch_bytes(x_rows, n_groups));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  constexpr int kRows = 64;  // token rows per tile of the 8-bit GEMM
+  CUtensorMap A, A2, S, S2, B, B2, Bb, B2b;
+  dg_status s;
+  if ((s = map_codes(&A, W, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  if ((s = map_scales(&S, W_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  if (W2) {
+    if ((s = map_codes(&A2, W2, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+    if ((s = map_scales(&S2, W2_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  } else {
+    A2 = A;
+    S2 = S;
+  }
+  if ((s = map_rows(&B, X, (uint64_t)x_rows, (uint64_t)K, 16)) != DG_OK) return s;
+  if ((s = map_rows(&Bb, X, (uint64_t)x_rows, (uint64_t)K, 64)) != DG_OK) return s;
+  if (X_lo) {
+    if ((s = map_rows(&B2, X_lo, (uint64_t)x_rows, (uint64_t)K, 16)) != DG_OK) return s;
+    if ((s = map_rows(&B2b, X_lo, (uint64_t)x_rows, (uint64_t)K, 64)) != DG_OK) return s;
+  } else {
+    B2 = B;
+    B2b = Bb;
+  }
+  dg::TcWorkItem* items = static_cast<dg::TcWorkItem*>(d_scratch);
+  int* n_items = reinterpret_cast<int*>(items + x_rows + n_groups);
+  int max_items = 0;
+  if (group_off) {
+    max_items = x_rows / kRows + n_groups;
+    LAUNCH(DG_K_PERMUTE, st, dg::launch_build_items(group_off, n_groups, kRows, x_rows, items, n_items, d_err, st));
+  }
+  dg::TcGemmParams p{};
+  p.K = K;
+  p.a_rows_per_group = rows;
+  p.m_tiles = ceil_div(rows, 128);
+  p.n_max = group_off ? kRows : (x_rows < kRows ? ((x_rows + 15) & ~15) : kRows);
+  p.n_tokens = x_rows;
+  p.k_splits = 1;
+  p.split_stride = 0;
+  p.items = group_off ? items : nullptr;
+  p.n_items = group_off ? n_items : nullptr;
+  p.dual_a = W2 != nullptr;
+  p.two_terms = X_lo != nullptr;
+  p.out = out;
+  p.out_lo = out_lo;
+  p.ld_out = ld_out;
+  p.smem_budget = kSmemGemm;
+  p.err = d_err;
+  const int tiles = (group_off ? max_items : ceil_div(x_rows, p.n_max)) * p.m_tiles;
+  LAUNCH(DG_K_GEMM_GATE_UP, st,
+         dg::launch_tc_gemm_mx8(W2 ? dg::EPI_SWIGLU_BF16 : dg::EPI_STORE_F32, A, A2, S, S2, B, B2, Bb, B2b, p, tiles,
+                                st));
+  return DG_OK;
 }
 
 extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,

@@ -1,0 +1,414 @@
+// Persistent tcgen05 GEMM with 8-bit weights for the expert contractions: the same
+// weights-on-M / tokens-on-N tiling as the bf16 GEMM, but each weight row is stored as
+// E4M3 codes with one power-of-two scale per 32 consecutive K elements (the OCP MX
+// block format: E8M0 scale 2^(s - 127)).  The weight stream, which bounds these GEMMs,
+// is half the bytes of bf16.
+//
+// Decoding is exact: an E4M3 value times a power of two has at most 4 significant bits,
+// which bf16 holds, so the MMAs see exactly the weights the codes define and the pass
+// keeps the precision model of the bf16 path (activations in one or two bf16 terms,
+// fp32 accumulation).  Decoded tiles never touch shared memory: decoder warps read the
+// 8-bit tile and its scales from shared memory, build the bf16 values in registers and
+// store them to TMEM, and the MMA takes its A operand (the weights) from TMEM.
+//
+// Roles (448 threads, one CTA per SM, tiles blockIdx.x, blockIdx.x + gridDim.x, ...):
+//   warp 0      TMA: 8-bit weight tiles (64-byte swizzle), scale tiles and token tiles
+//               into a ring of shared-memory stages;
+//   warp 1      TMEM allocation and tcgen05.mma (A from TMEM, B = tokens from smem) into
+//               one of two accumulator buffers;
+//   warps 2-5   epilogue of the other accumulator buffer (as the bf16 GEMM);
+//   warps 6-13  decoders: shared-memory stage -> bf16 weights in a ring of TMEM stages.
+//               Warp w covers TMEM lanes 32 (w % 4) .. + 31 (its weight rows) and one
+//               32-element half of each 64-element k-block.
+// Every wait is bounded; on a timeout the CTA winds down and the error word says which
+// wait gave up.
+//
+// Decoding one code c (sign, 4 exponent bits e with bias 7, 3 mantissa bits m): the bf16
+// bit pattern sign << 15 | (c & 0x7F) << 4 has exponent field e and mantissa m << 4, so it
+// is value(c) * 2^-120 for normal codes (e > 0) and, as a bf16 subnormal, for the
+// subnormal codes too (m * 2^-9 * 2^-120).  One bf16 multiply by 2^(s - 7) (exact: a
+// power of two) gives value(c) * 2^(s - 127).  Preconditions: s <= 134 (block scale
+// <= 2^7, so the multiplier is a finite bf16), and codes 0x7F / 0xFF (NaN in E4M3) do
+// not occur (they would decode as 480 times the scale).
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+constexpr int MX_BM = 128;                    // weight rows per tile
+constexpr int MX_BK = 64;                     // K elements per k-block (two scale blocks)
+constexpr uint32_t MX_A_BYTES = MX_BM * MX_BK;  // one 8-bit weight tile
+constexpr uint32_t MX_S_BYTES = MX_BM * 2;      // its scales: two per row
+constexpr int MX_T_STAGES = 4;                // TMEM stages of decoded weights
+constexpr int MX_F_STAGES_MAX = 8;
+constexpr int MX_DEC_WARPS = 8;
+constexpr int MX_DEC_WARP0 = 6;
+constexpr int MX_THREADS = 32 * (MX_DEC_WARP0 + MX_DEC_WARPS);
+constexpr int MX_B_BOX = 16;
+constexpr int MX_B_BOX_BIG = 64;
+
+struct MxTile {
+  int g, row0, rows, m;
+};
+
+__device__ __forceinline__ int mx_total_items(const TcGemmParams& p) {
+  if (p.items) return *p.n_items;
+  return (p.n_tokens + p.n_max - 1) / p.n_max;
+}
+
+// tile t -> (work item t / m_tiles, weight tile t % m_tiles)
+__device__ __forceinline__ MxTile mx_decode_tile(const TcGemmParams& p, int t) {
+  MxTile ti;
+  const int item = t / p.m_tiles;
+  ti.m = t % p.m_tiles;
+  if (p.items) {
+    const TcWorkItem it = p.items[item];
+    ti.g = it.group;
+    ti.row0 = it.row0;
+    ti.rows = it.rows;
+  } else {
+    ti.g = 0;
+    ti.row0 = item * p.n_max;
+    ti.rows = min(p.n_max, p.n_tokens - ti.row0);
+  }
+  return ti;
+}
+
+struct MxWalk {
+  int t, n_tiles;
+  __device__ MxWalk(int n) : t(blockIdx.x), n_tiles(n) {}
+  __device__ bool next(int& tile) {
+    if (t >= n_tiles) return false;
+    tile = t;
+    t += gridDim.x;
+    return true;
+  }
+};
+
+__device__ __forceinline__ void mx_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// four codes (code i in byte i) -> two bf16x2 words (codes 0, 1 and codes 2, 3; the
+// lower-indexed code in the low half), each value times the multiplier pair mm
+__device__ __forceinline__ void mx8_decode4(uint32_t x, uint32_t mm, uint32_t& p01, uint32_t& p23) {
+  const uint32_t mag = x & 0x7F7F7F7Fu;
+  // bytes 0 and 1 to bits 8..15 and 24..31 (the sign lands on bits 15 and 31)
+  const uint32_t s01 = __byte_perm(x, 0u, 0x1404), s23 = __byte_perm(x, 0u, 0x3424);
+  const uint32_t m01 = __byte_perm(mag, 0u, 0x1404) >> 4, m23 = __byte_perm(mag, 0u, 0x3424) >> 4;
+  p01 = bf16x2_mul((s01 & 0x80008000u) | m01, mm);
+  p23 = bf16x2_mul((s23 & 0x80008000u) | m23, mm);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(MX_THREADS, 1)
+    tc_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                       const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmS2,
+                       const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                       const __grid_constant__ CUtensorMap tmBb, const __grid_constant__ CUtensorMap tmB2b,
+                       const TcGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t f_full[MX_F_STAGES_MAX];   // a stage's TMA loads landed
+  __shared__ __align__(8) uint64_t f_empty[MX_F_STAGES_MAX];  // decoders and MMAs are done with it
+  __shared__ __align__(8) uint64_t t_full[MX_T_STAGES];       // decoded weights are in TMEM
+  __shared__ __align__(8) uint64_t t_empty[MX_T_STAGES];      // the MMAs reading them completed
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ int n_issued_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int terms = p.two_terms ? 2 : 1;
+  const int n_a = p.dual_a ? 2 : 1;
+  // stage: token tiles (terms x n_max rows x 128 B, 1024-aligned for the 128-byte
+  // swizzle), then the 8-bit weight tiles, then their scales
+  const uint32_t b_bytes = (uint32_t)p.n_max * 128;
+  const uint32_t a_off = (uint32_t)terms * b_bytes;
+  const uint32_t s_off = a_off + (uint32_t)n_a * MX_A_BYTES;
+  const uint32_t stage_bytes = (s_off + (uint32_t)n_a * MX_S_BYTES + 1023u) & ~1023u;
+  int stages = p.smem_budget / (int)stage_bytes;
+  if (stages > MX_F_STAGES_MAX) stages = MX_F_STAGES_MAX;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int acc_cols = p.n_max * n_a;
+  const uint32_t a_col0 = 2u * (uint32_t)acc_cols;
+  const uint32_t a_stage_cols = 32u * (uint32_t)n_a;  // 64 K elements = 32 packed columns per weight tile
+  uint32_t tmem_cols = 32;
+  while (tmem_cols < a_col0 + MX_T_STAGES * a_stage_cols) tmem_cols <<= 1;
+  const int nkb = p.K / MX_BK;
+
+  if (warp == 1) tmem_alloc(&tmem_base_s, tmem_cols);
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&f_full[s], 1);
+      mbar_init(&f_empty[s], MX_DEC_WARPS + 1);
+    }
+    for (int s = 0; s < MX_T_STAGES; ++s) {
+      mbar_init(&t_full[s], MX_DEC_WARPS);
+      mbar_init(&t_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    n_issued_s = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  griddep_sync();  // the work list and the token operand come from the previous kernels
+  const int n_tiles = mx_total_items(p) * p.m_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmS);
+      if (p.dual_a) {
+        prefetch_tmap(&tmA2);
+        prefetch_tmap(&tmS2);
+      }
+      prefetch_tmap(&tmB);
+      prefetch_tmap(&tmBb);
+      if (terms == 2) {
+        prefetch_tmap(&tmB2);
+        prefetch_tmap(&tmB2b);
+      }
+      int it = 0, t;
+      bool ok = true;
+      MxWalk walk(n_tiles);
+      while (ok && walk.next(t)) {
+        const MxTile ti = mx_decode_tile(p, t);
+        const int n_pad = (ti.rows + 15) & ~15;
+        const uint32_t tx = (uint32_t)terms * (uint32_t)n_pad * 128u + (uint32_t)n_a * (MX_A_BYTES + MX_S_BYTES);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % stages;
+          if (!mbar_wait(&f_empty[s], ((uint32_t)(it / stages) & 1u) ^ 1u, &abort_s, p.err,
+                         DG_DEVERR_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + (size_t)s * stage_bytes;
+          const int kbx = (kb + t) % nkb;  // tiles running together start at different k-blocks
+          const int kx = kbx * MX_BK;
+          mbar_arrive_expect_tx(&f_full[s], tx);
+          tma_load_3d(st + a_off, &tmA, kx, ti.m * MX_BM, ti.g, &f_full[s]);
+          tma_load_3d(st + s_off, &tmS, ti.m * MX_BM * 2, kbx, ti.g, &f_full[s]);
+          if (p.dual_a) {
+            tma_load_3d(st + a_off + MX_A_BYTES, &tmA2, kx, ti.m * MX_BM, ti.g, &f_full[s]);
+            tma_load_3d(st + s_off + MX_S_BYTES, &tmS2, ti.m * MX_BM * 2, kbx, ti.g, &f_full[s]);
+          }
+          int r = 0;
+          for (; r + MX_B_BOX_BIG <= n_pad; r += MX_B_BOX_BIG) {
+            tma_load_2d(st + r * 128, &tmBb, kx, ti.row0 + r, &f_full[s]);
+            if (terms == 2) tma_load_2d(st + b_bytes + r * 128, &tmB2b, kx, ti.row0 + r, &f_full[s]);
+          }
+          for (; r < n_pad; r += MX_B_BOX) {
+            tma_load_2d(st + r * 128, &tmB, kx, ti.row0 + r, &f_full[s]);
+            if (terms == 2) tma_load_2d(st + b_bytes + r * 128, &tmB2, kx, ti.row0 + r, &f_full[s]);
+          }
+          n_issued_s = it + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: A (decoded weights) from TMEM, B (tokens) from smem
+      int it = 0, j = 0, t;
+      bool ok = true;
+      MxWalk walk(n_tiles);
+      for (; ok && walk.next(t); ++j) {
+        const MxTile ti = mx_decode_tile(p, t);
+        const int n_pad = (ti.rows + 15) & ~15;
+        const int buf = j & 1;
+        if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
+          break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
+        const uint32_t d1 = d0 + (uint32_t)p.n_max;
+        const uint32_t idesc = idesc_bf16_f32(MX_BM, n_pad);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % stages, ts = it % MX_T_STAGES;
+          if (!mbar_wait(&t_full[ts], (uint32_t)(it / MX_T_STAGES) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL) ||
+              !mbar_wait(&f_full[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + (size_t)s * stage_bytes);
+          const uint32_t a0 = tmem + a_col0 + (uint32_t)ts * a_stage_cols;
+#pragma unroll
+          for (int kk = 0; kk < MX_BK / 16; ++kk) {
+            const uint32_t acc = (kb != 0 || kk != 0) ? 1u : 0u;
+            const uint64_t bd = sw128_kmajor_desc(sb + kk * 32);
+            const uint64_t bd2 = sw128_kmajor_desc(sb + b_bytes + kk * 32);
+            const uint32_t ak = a0 + (uint32_t)kk * 8u;  // 16 K elements = 8 packed columns
+            mx_mma_ts(d0, ak, bd, idesc, acc);
+            if (terms == 2) mx_mma_ts(d0, ak, bd2, idesc, 1u);
+            if (p.dual_a) {
+              mx_mma_ts(d1, ak + 32u, bd, idesc, acc);
+              if (terms == 2) mx_mma_ts(d1, ak + 32u, bd2, idesc, 1u);
+            }
+          }
+          tc_commit(&t_empty[ts]);
+          tc_commit(&f_empty[s]);
+        }
+        if (ok) tc_commit(&acc_full[buf]);
+      }
+      tc_commit(&drain_bar);  // completes once every MMA issued above has landed
+    }
+  } else if (warp < MX_DEC_WARP0) {
+    // ---------------- epilogue warps 2..5: TMEM lanes (warp % 4) * 32 .. + 31
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
+    int j = 0, t;
+    MxWalk walk(n_tiles);
+    for (; walk.next(t); ++j) {
+      const MxTile ti = mx_decode_tile(p, t);
+      const int n_pad = (ti.rows + 15) & ~15;
+      const int buf = j & 1;
+      if (!mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)) break;
+      tc_fence_after();
+      const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
+      const int f = ti.m * MX_BM + row;  // weight row = output feature
+      const bool fvalid = f < p.a_rows_per_group;
+      for (int c0 = 0; c0 < n_pad; c0 += 16) {
+        uint32_t ra[16], rb[16];
+        tmem_ld16(t0 + c0, ra);
+        if (EPI == EPI_SWIGLU_BF16) tmem_ld16(t0 + p.n_max + c0, rb);
+        tc_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int col = c0 + q;
+          const float a = __uint_as_float(ra[q]);
+          const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
+          if (!fvalid || col >= ti.rows) continue;
+          const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
+          if (EPI == EPI_STORE_F32) {
+            reinterpret_cast<float*>(p.out)[o] = a;
+          } else {
+            const float hv = a / (1.0f + expf(-a)) * b;
+            const bf16 hi = __float2bfloat16_rn(hv);
+            reinterpret_cast<bf16*>(p.out)[o] = hi;
+            if (p.out_lo) reinterpret_cast<bf16*>(p.out_lo)[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  } else {
+    // ---------------- decoders: rows 32 (warp % 4) + lane, K half (warp - 6) / 4 of each k-block
+    const int lq = warp & 3;
+    const int half = (warp - MX_DEC_WARP0) >> 2;
+    const int row = lq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(lq * 32) << 16;
+    const int swz = (row >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of the row sits at c ^ swz
+    int it = 0, t;
+    bool ok = true;
+    MxWalk walk(n_tiles);
+    while (ok && walk.next(t)) {
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % stages, ts = it % MX_T_STAGES;
+        if (!mbar_wait(&f_full[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL) ||
+            !mbar_wait(&t_empty[ts], ((uint32_t)(it / MX_T_STAGES) & 1u) ^ 1u, &abort_s, p.err,
+                       DG_DEVERR_TIMEOUT_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* st = smem + (size_t)s * stage_bytes;
+        for (int a = 0; a < n_a; ++a) {
+          const uint8_t* codes = st + a_off + (uint32_t)a * MX_A_BYTES + row * MX_BK;
+          const uint32_t e8 = st[s_off + (uint32_t)a * MX_S_BYTES + row * 2 + half];
+          const uint32_t mh = (e8 + 120u) << 7;  // bf16 bits of 2^(e8 - 7)
+          const uint32_t mm = mh | (mh << 16);
+          uint32_t w[16];
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c = 2 * half + c2;
+            const uint4 v = *reinterpret_cast<const uint4*>(codes + ((c ^ swz) << 4));
+            mx8_decode4(v.x, mm, w[c2 * 8 + 0], w[c2 * 8 + 1]);
+            mx8_decode4(v.y, mm, w[c2 * 8 + 2], w[c2 * 8 + 3]);
+            mx8_decode4(v.z, mm, w[c2 * 8 + 4], w[c2 * 8 + 5]);
+            mx8_decode4(v.w, mm, w[c2 * 8 + 6], w[c2 * 8 + 7]);
+          }
+          tmem_st16(tmem + lane_off + a_col0 + (uint32_t)ts * a_stage_cols + (uint32_t)a * 32u + (uint32_t)half * 16u,
+                    w);
+        }
+        tc_wait_st();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&f_empty[s]);  // this warp's reads of the stage are done
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&t_full[ts]);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (abort_s && tid == 0) {
+    // wind down: let the most recent load of every stage land before the smem goes away
+    const int first = n_issued_s > stages ? n_issued_s - stages : 0;
+    for (int i = first; i < n_issued_s; ++i) mbar_wait_drain(&f_full[i % stages], (uint32_t)(i / stages) & 1u);
+  }
+  if (tid == 32) mbar_wait_drain(&drain_bar, 0);  // every issued MMA has landed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, tmem_cols);
+}
+
+cudaError_t launch_tc_gemm_mx8(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
+                               const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
+                               const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, int max_tiles,
+                               cudaStream_t st) {
+  if (max_tiles <= 0) return cudaSuccess;
+  if (p.k_splits != 1 || p.K % MX_BK != 0 || p.K <= 0 || p.n_max < 16 || p.n_max > 64 || (p.n_max % 16) != 0 ||
+      p.m_tiles < 1 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
+    return cudaErrorInvalidValue;
+  const int n_a = p.dual_a ? 2 : 1;
+  const int terms = p.two_terms ? 2 : 1;
+  const int stage = ((terms * p.n_max * 128 + n_a * (int)(MX_A_BYTES + MX_S_BYTES)) + 1023) & ~1023;
+  if (p.smem_budget < 2 * stage) return cudaErrorInvalidValue;
+  const int smem = p.smem_budget + 1024;
+  const int sms = num_sms();
+  const int grid = max_tiles < sms ? max_tiles : sms;
+  cudaError_t e;
+  switch (epi) {
+    case EPI_STORE_F32:
+      e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_STORE_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      return launch_k(tc_gemm_mx8_kernel<EPI_STORE_F32>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B, B2,
+                      Bb, B2b, p);
+    case EPI_SWIGLU_BF16:
+      e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem);
+      if (e != cudaSuccess) return e;
+      return launch_k(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B,
+                      B2, Bb, B2b, p);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dg

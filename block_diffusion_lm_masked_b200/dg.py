@@ -92,6 +92,7 @@ def _load():
         "dg_debug_bounded_wait": (I32, [P, I32, P]),
         "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_scratch_bytes": (SZ, [I32, I32]),
+        "dg_debug_gemm_mx8": (I32, [P, P, P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -382,6 +383,27 @@ def debug_gemm_bf16(W, X, out, ld_out, err, scratch, W2=None, X_lo=None, group_o
     _check(lib.dg_debug_gemm_bf16(_ptr(W), _ptr(W2), rows, G, _ptr(X), _ptr(X_lo), X.shape[0], K, _ptr(group_off),
                                   _ptr(out), _ptr(out_lo), ld_out, _ptr(scratch),
                                   scratch.numel(), _ptr(err), _stream(stream)))
+
+
+def pack_mx8_scales(exponents: np.ndarray) -> np.ndarray:
+    """Block exponents x of weights [groups][rows][K] (one per 32 consecutive K elements,
+    array [groups][rows][K / 32], block scale 2^x) -> the library's scale bytes
+    [groups][K / 64][rows][2] (E8M0: x + 127)."""
+    e = np.asarray(exponents, dtype=np.int64)
+    G, R, nb = e.shape
+    if nb % 2 or e.min() < -127 or e.max() > 7:
+        raise ValueError("block exponents must come in pairs per 64 K elements and lie in [-127, 7]")
+    return np.ascontiguousarray((e + 127).astype(np.uint8).reshape(G, R, nb // 2, 2).transpose(0, 2, 1, 3))
+
+
+def debug_gemm_mx8(W, W_scales, X, out, ld_out, err, scratch, W2=None, W2_scales=None, X_lo=None, group_off=None,
+                   out_lo=None, stream=None):
+    """One launch of the 8-bit-weight GEMM (see include/dg_debug.h): W uint8 codes
+    [groups][rows][K], W_scales uint8 [groups][K / 64][rows][2]."""
+    G, rows, K = W.shape
+    _check(lib.dg_debug_gemm_mx8(_ptr(W), _ptr(W_scales), _ptr(W2), _ptr(W2_scales), rows, G, _ptr(X), _ptr(X_lo),
+                                 X.shape[0], K, _ptr(group_off), _ptr(out), _ptr(out_lo), ld_out, _ptr(scratch),
+                                 scratch.numel(), _ptr(err), _stream(stream)))
 
 
 def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out_lo=None, stream=None):

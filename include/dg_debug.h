@@ -86,6 +86,22 @@ dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_
                              void* out_lo, int32_t ld_out, void* d_scratch, size_t scratch_bytes,
                              int32_t* d_err, dg_stream stream);
 
+/* The same GEMM over 8-bit weights (MX-FP8 storage: OCP E4M3 elements with one E8M0
+ * power-of-two scale per 32 consecutive K elements of a row): every weight is
+ * value(code) * 2^(scale - 127), decoded exactly to bf16 in the kernel, so
+ *   acc[r][f] = sum_k dec(W)[g][f][k] * (X[r][k] + X_lo[r][k])
+ * with everything else (groups, W2 / SwiGLU epilogue, outputs, errors, scratch) as
+ * dg_debug_gemm_bf16, except that groups are cut into work items of at most 64 rows.
+ * W (and W2): codes uint8 [n_groups][rows][K] (E4M3: sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits; codes 0x7F and 0xFF must not occur).  W_scales (and W2_scales): uint8
+ * [n_groups][K / 64][rows][2], entry [g][j][f][h] the E8M0 scale of elements
+ * 64 j + 32 h .. + 31 of row f; every scale <= 134 (block scale <= 2^7).  rows % 8 == 0,
+ * K % 64 == 0; every pointer 16-byte aligned. */
+dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, const void* W2, const void* W2_scales, int32_t rows,
+                            int32_t n_groups, const void* X, const void* X_lo, int32_t x_rows, int32_t K,
+                            const int32_t* group_off, void* out, void* out_lo, int32_t ld_out, void* d_scratch,
+                            size_t scratch_bytes, int32_t* d_err, dg_stream stream);
+
 /* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
  * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
  * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128] (hi part); out_lo (nullable)

@@ -1,10 +1,12 @@
 """The C-ABI library: it loads, exports every symbol the headers declare, and its
 host-side validation and arithmetic work without a GPU (no compute calls here)."""
 import ctypes
+import itertools
 import glob
 import os
 import re
 
+import numpy as np
 import pytest
 
 from conftest import ROOT, golden_path
@@ -216,3 +218,40 @@ def test_batched_calls_reject_bad_arguments_before_any_launch():
         assert [good[i].len for i in range(B)] == [8, 8, 8]                        # nothing advanced
     finally:
         dg.lib.dg_model_destroy(h)
+
+
+def test_mx8_scale_packing_layout():
+    """The binding's scale packing puts the exponent of elements 64 j + 32 h .. + 31 of row
+    f in group g at [g][j][f][h], biased by 127 (E8M0), as include/dg_debug.h states."""
+    rng = np.random.default_rng(3)
+    e = rng.integers(-127, 8, size=(3, 16, 8))
+    p = dg.pack_mx8_scales(e)
+    assert p.dtype == np.uint8 and p.shape == (3, 4, 16, 2) and p.flags["C_CONTIGUOUS"]
+    for g, j, f, h in itertools.product(range(3), range(4), range(16), range(2)):
+        assert p[g, j, f, h] == e[g, f, 2 * j + h] + 127
+    with pytest.raises(ValueError):
+        dg.pack_mx8_scales(np.full((1, 2, 2), 8))
+    with pytest.raises(ValueError):
+        dg.pack_mx8_scales(np.zeros((1, 2, 3), dtype=int))
+
+
+def test_mx8_gemm_validation_on_host():
+    """Every bad argument of dg_debug_gemm_mx8 is rejected before any CUDA call (the
+    placeholder addresses are never dereferenced)."""
+    p = ctypes.c_void_p(1 << 24)
+    err = ctypes.c_void_p(1 << 25)
+    sc = ctypes.c_void_p(1 << 26)
+    L = dg.lib
+    launches = L.dg_launch_count()
+
+    def call(W=p, S=p, W2=None, S2=None, rows=128, G=1, X=p, X_lo=None, n=16, K=128, off=None, ld=128,
+             scratch=sc, sbytes=1 << 20):
+        return L.dg_debug_gemm_mx8(W, S, W2, S2, rows, G, X, X_lo, n, K, off, p, None, ld, scratch, sbytes, err, None)
+
+    for kw in (dict(W=None), dict(S=None), dict(X=None), dict(scratch=None), dict(W2=p), dict(S2=p),
+               dict(K=96), dict(K=0), dict(rows=100), dict(rows=0), dict(n=0), dict(G=2), dict(ld=64),
+               dict(W=ctypes.c_void_p((1 << 24) + 8)), dict(X_lo=ctypes.c_void_p((1 << 24) + 4)),
+               dict(scratch=ctypes.c_void_p((1 << 26) + 16))):
+        assert call(**kw) == dg.DG_ERR_INVALID_ARG, kw
+    assert call(sbytes=8) == dg.DG_ERR_CAPACITY
+    assert L.dg_launch_count() == launches
