@@ -27,7 +27,8 @@
 // bit pattern sign << 15 | (c & 0x7F) << 4 has exponent field e and mantissa m << 4, so it
 // is value(c) * 2^-120 for normal codes (e > 0) and, as a bf16 subnormal, for the
 // subnormal codes too (m * 2^-9 * 2^-120).  One bf16 multiply by 2^(s - 7) (exact: a
-// power of two) gives value(c) * 2^(s - 127).  Preconditions: s <= 134 (block scale
+// power of two) gives value(c) * 2^(s - 127), exactly for every code when s >= 9 (below,
+// subnormal codes round to bf16's subnormal grid).  Preconditions: s <= 134 (block scale
 // <= 2^7, so the multiplier is a finite bf16), and codes 0x7F / 0xFF (NaN in E4M3) do
 // not occur (they would decode as 480 times the scale).
 #include "dg_common.cuh"

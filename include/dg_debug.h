@@ -95,7 +95,8 @@ dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t rows, int32_
  * W (and W2): codes uint8 [n_groups][rows][K] (E4M3: sign, 4 exponent bits with bias 7,
  * 3 mantissa bits; codes 0x7F and 0xFF must not occur).  W_scales (and W2_scales): uint8
  * [n_groups][K / 64][rows][2], entry [g][j][f][h] the E8M0 scale of elements
- * 64 j + 32 h .. + 31 of row f; every scale <= 134 (block scale <= 2^7).  rows % 8 == 0,
+ * 64 j + 32 h .. + 31 of row f; every scale <= 134 (block scale <= 2^7); decoding is exact
+ * for scales >= 9 (below, subnormal codes round to bf16's subnormals).  rows % 8 == 0,
  * K % 64 == 0; every pointer 16-byte aligned. */
 dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, const void* W2, const void* W2_scales, int32_t rows,
                             int32_t n_groups, const void* X, const void* X_lo, int32_t x_rows, int32_t K,
