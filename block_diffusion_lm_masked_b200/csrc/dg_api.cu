@@ -188,6 +188,10 @@ static dg_status map_weights(CUtensorMap* m, const void* base, uint64_t groups, 
 struct LayerMaps {
   CUtensorMap qkv, o, gate, up, down;
 };
+// 8-bit experts of one layer: codes and block scales of gate, up and down
+struct Mx8Maps {
+  CUtensorMap gate, gate_s, up, up_s, down, down_s;
+};
 struct dg_model {
   dg_config cfg;
   const void* embed;
@@ -195,6 +199,7 @@ struct dg_model {
   std::vector<dg_layer_weights> layers;
   std::vector<LayerMaps> maps;
   CUtensorMap out_map;
+  std::vector<Mx8Maps> mx8;  // non-empty: the batched calls run the experts from 8-bit weights
   bool taps_on = false;
   std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
   std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
@@ -286,6 +291,7 @@ constexpr int kSmemGemm = 200 * 1024;    // stage budget of the persistent GEMM 
 inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr int kItemRows = 128;           // rows per work item of the grouped expert GEMMs
+constexpr int kItemRowsMx8 = 64;         // the same for the 8-bit-weight expert GEMMs
 
 
 struct WsLayout {
@@ -332,7 +338,7 @@ WsLayout layout(const dg_config& c, int T) {
   L.perm = take((size_t)T * k * 4);
   L.inv = take((size_t)T * k * 4);
   L.uni = take(4);
-  L.items = take(((size_t)T * k / kItemRows + E + 1) * sizeof(dg::TcWorkItem));
+  L.items = take(((size_t)T * k / kItemRowsMx8 + E + 1) * sizeof(dg::TcWorkItem));
   L.n_items = take(4);
   L.xs = take((size_t)T * k * H * ab);
   L.xs_lo = take(bf ? (size_t)T * k * H * 2 : 0);
@@ -430,6 +436,41 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   const int items = g.items ? g.max_items : ceil_div(g.x_rows, g.n_max) * g.k_splits;
   LAUNCH(g.kind, st,
          dg::launch_tc_gemm(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, B, B2, Bb, B2b, p, items * p.m_tiles, st));
+  return DG_OK;
+}
+
+// a grouped expert GEMM over 8-bit weights (A, S: codes and scales; A2, S2 for gate / up)
+dg_status gemm_mx8(const GemmCall& g, const CUtensorMap* S, const CUtensorMap* S2, int* err, cudaStream_t st) {
+  CUtensorMap B, B2, Bb, B2b;
+  dg_status s;
+  if ((s = map_rows(&B, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
+  if ((s = map_rows(&Bb, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 64)) != DG_OK) return s;
+  if (g.X_lo) {
+    if ((s = map_rows(&B2, g.X_lo, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
+    if ((s = map_rows(&B2b, g.X_lo, (uint64_t)g.x_rows, (uint64_t)g.K, 64)) != DG_OK) return s;
+  } else {
+    B2 = B;
+    B2b = Bb;
+  }
+  dg::TcGemmParams p{};
+  p.K = g.K;
+  p.a_rows_per_group = g.a_rows_per_group;
+  p.m_tiles = ceil_div(g.a_rows_per_group, 128);
+  p.n_max = g.n_max;
+  p.n_tokens = g.x_rows;
+  p.k_splits = 1;
+  p.items = g.items;
+  p.n_items = g.n_items;
+  p.dual_a = g.A2 != nullptr;
+  p.two_terms = g.X_lo != nullptr;
+  p.out = g.out;
+  p.out_lo = g.out_lo;
+  p.ld_out = g.ld_out;
+  p.smem_budget = g.smem_budget;
+  p.err = err;
+  LAUNCH(g.kind, st,
+         dg::launch_tc_gemm_mx8(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, *S, S2 ? *S2 : *S, B, B2, Bb, B2b, p,
+                                g.max_items * p.m_tiles, st));
   return DG_OK;
 }
 
@@ -755,17 +796,32 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
     if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
         cudaSuccess)
       return fail(DG_ERR_CUDA, "tap copy failed");
+  const bool mx8 = bf && !m->mx8.empty();
+  const int item_rows = mx8 ? kItemRowsMx8 : kItemRows;
   LAUNCH(DG_K_PERMUTE, st,
          dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
                             ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
-                            ws.at<int32_t>(ws.L.uni), kItemRows, ws.at<dg::TcWorkItem>(ws.L.items),
+                            ws.at<int32_t>(ws.L.uni), item_rows, ws.at<dg::TcWorkItem>(ws.L.items),
                             ws.at<int>(ws.L.n_items), st));
   T* xs_lo = bf ? ws.at<T>(ws.L.xs_lo) : nullptr;
   LAUNCH(DG_K_GATHER, st,
          dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), xn_lo, ws.at<int32_t>(ws.L.perm), n * k, k, H,
                                    ws.at<T>(ws.L.xs), xs_lo, st));
   const int* off = ws.at<int>(ws.L.offsets);
-  if (bf) {
+  if (mx8) {
+    const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
+    const int* n_items = ws.at<int>(ws.L.n_items);
+    const int max_items = n * k / kItemRowsMx8 + E;
+    const Mx8Maps& X8 = m->mx8[l];
+    GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &X8.gate, &X8.up, ws.at<void>(ws.L.xs), xs_lo, n * k, H, F,
+                items, n_items, max_items, kItemRowsMx8, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
+                kSmemGemm};
+    if ((s = gemm_mx8(gu, &X8.gate_s, &X8.up_s, err, st)) != DG_OK) return s;
+    GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &X8.down, nullptr, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo),
+                n * k, F, H, items, n_items, max_items, kItemRowsMx8, ws.at<float>(ws.L.ys), nullptr, H, 1, 0,
+                kSmemGemm};
+    if ((s = gemm_mx8(dn, &X8.down_s, nullptr, err, st)) != DG_OK) return s;
+  } else if (bf) {
     const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
     const int* n_items = ws.at<int>(ws.L.n_items);
     const int max_items = n * k / kItemRows + E;
@@ -1087,6 +1143,42 @@ extern "C" dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int3
                                       d_canvases + (size_t)b * C, nullptr, -1, st));
   }
   if (append) return dg_prefill_append_batched(m, caches, B, d_canvases, C, d_ws, ws_bytes, stream);
+  return DG_OK;
+}
+
+extern "C" dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* layers) {
+  DG_CHECK_ARG(m, "model is NULL");
+  if (!layers) {
+    m->mx8.clear();
+    return DG_OK;
+  }
+  const dg_config& c = m->cfg;
+  DG_CHECK_ARG(is_bf16(c), "8-bit experts need a bf16 model");
+  auto a16 = [](const void* q) { return q && (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_expert_weights_mx8& X = layers[l];
+    DG_CHECK_ARG(a16(X.gate) && a16(X.gate_scales) && a16(X.up) && a16(X.up_scales) && a16(X.down) &&
+                     a16(X.down_scales),
+                 "layer %d: 8-bit expert pointers must be non-NULL and 16-byte aligned", l);
+  }
+  std::vector<Mx8Maps> maps;
+  try {
+    maps.resize(c.n_layers);
+  } catch (...) {
+    return fail(DG_ERR_CUDA, "out of host memory");
+  }
+  const uint64_t E = c.n_experts, F = c.expert_ffn, H = c.hidden;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_expert_weights_mx8& X = layers[l];
+    Mx8Maps& M = maps[l];
+    dg_status s;
+    if ((s = map_codes(&M.gate, X.gate, E, F, H)) != DG_OK || (s = map_scales(&M.gate_s, X.gate_scales, E, F, H)) != DG_OK ||
+        (s = map_codes(&M.up, X.up, E, F, H)) != DG_OK || (s = map_scales(&M.up_s, X.up_scales, E, F, H)) != DG_OK ||
+        (s = map_codes(&M.down, X.down, E, H, F)) != DG_OK ||
+        (s = map_scales(&M.down_s, X.down_scales, E, H, F)) != DG_OK)
+      return s;
+  }
+  m->mx8.swap(maps);
   return DG_OK;
 }
 

@@ -51,6 +51,11 @@ class KVCacheS(ctypes.Structure):
                 ("capacity", ctypes.c_int32), ("len", ctypes.c_int32)]
 
 
+class ExpertsMx8(ctypes.Structure):
+    _fields_ = [("gate", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p), ("up", ctypes.c_void_p),
+                ("up_scales", ctypes.c_void_p), ("down", ctypes.c_void_p), ("down_scales", ctypes.c_void_p)]
+
+
 class Taps(ctypes.Structure):
     _fields_ = [("x_attn", ctypes.POINTER(ctypes.c_void_p)), ("x_out", ctypes.POINTER(ctypes.c_void_p)),
                 ("topk_idx", ctypes.POINTER(ctypes.c_void_p)), ("topk_w", ctypes.POINTER(ctypes.c_void_p)),
@@ -80,6 +85,7 @@ def _load():
         "dg_prefill_append_batched": (I32, [P, P, I32, P, I32, P, SZ, P]),
         "dg_denoise_pass_batched": (I32, [P, P, I32, P, I32, P, P, SZ, P]),
         "dg_generate_canvases": (I32, [P, P, I32, P, I32, I32, F32, F32, P, I32, P, P, SZ, P]),
+        "dg_model_set_experts_mx8": (I32, [P, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
         "dg_set_taps": (I32, [P, ctypes.POINTER(Taps)]),
@@ -166,6 +172,28 @@ class Model:
         if getattr(self, "handle", None):
             lib.dg_model_destroy(self.handle)
             self.handle = None
+
+    def set_experts_mx8(self, layers: list | None):
+        """layers: per layer dict(gate=(codes, exps), up=(codes, exps), down=(codes, exps)) with
+        codes uint8 [E][rows][K] and block exponents [E][rows][K / 32] (scale 2^x); None
+        returns to the bf16 experts.  Used by the batched calls."""
+        if layers is None:
+            _check(lib.dg_model_set_experts_mx8(self.handle, None))
+            self._mx8 = None
+            return
+        dev, keep, structs = self.device, [], []
+        for L in layers:
+            ptrs = []
+            for name in ("gate", "up", "down"):
+                codes, exps = L[name]
+                c = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).to(dev)
+                sc = torch.from_numpy(pack_mx8_scales(exps)).to(dev)
+                keep += [c, sc]
+                ptrs += [c.data_ptr(), sc.data_ptr()]
+            structs.append(ExpertsMx8(*ptrs))
+        arr = (ExpertsMx8 * len(structs))(*structs)
+        _check(lib.dg_model_set_experts_mx8(self.handle, arr))
+        self._mx8 = keep
 
     def set_taps(self, taps: dict | None):
         """taps: name -> list (per layer) of device tensors sized for taps['rows'] tokens,

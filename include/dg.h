@@ -195,6 +195,30 @@ dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int32_t B, int3
                                float r_start, float r_end, const uint64_t* seeds, int32_t append, float* d_logits,
                                void* d_ws, size_t ws_bytes, dg_stream stream);
 
+/* 8-bit expert weights (MX-FP8 storage: E4M3 codes with one E8M0 power-of-two scale per
+ * 32 consecutive K elements of a row; see dg_debug_gemm_mx8 in dg_debug.h for the byte
+ * layouts and limits).  Per layer:
+ *   gate, up     codes [E][F][H],  scales [E][H / 64][F][2]
+ *   down         codes [E][H][F],  scales [E][F / 64][H][2]
+ * all device pointers, 16-byte aligned, alive and unchanged while set.  Each weight is
+ * value(code) * 2^(scale - 127), decoded exactly to bf16 inside the expert GEMMs, so the
+ * model computes with exactly those weights at the bf16 path's precision; the expert
+ * weight stream is half the bytes of bf16. */
+typedef struct dg_expert_weights_mx8 {
+  const void* gate;
+  const void* gate_scales;
+  const void* up;
+  const void* up_scales;
+  const void* down;
+  const void* down_scales;
+} dg_expert_weights_mx8;
+/* Run the experts of every layer from these 8-bit weights (host array [n_layers]; NULL
+ * returns to the bf16 experts given at creation).  bf16 models only.  Applies to the
+ * batched calls (dg_denoise_pass_batched, dg_prefill_append_batched,
+ * dg_generate_canvases; B = 1 is one canvas); the single-canvas calls keep the bf16
+ * experts. */
+dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* layers);
+
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
 

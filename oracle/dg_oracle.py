@@ -624,6 +624,20 @@ def e4m3_encode(x: float) -> int:
     return c | (0x80 if neg else 0)
 
 
+def e4m3_encode_array(x) -> np.ndarray:
+    """e4m3_encode element by element on an array (the same rule: nearest code, ties to
+    the even code, magnitudes beyond 448 saturate), as uint8 codes."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    i = np.searchsorted(_E4M3_POS, a)  # first value >= a (a <= 448, the last value)
+    hit = _E4M3_POS[i] == a
+    lo = np.maximum(i - 1, 0)
+    dlo, dhi = a - _E4M3_POS[lo], _E4M3_POS[i] - a
+    pick_lo = (dlo < dhi) | ((dlo == dhi) & (lo % 2 == 0))
+    c = np.where(hit, i, np.where(pick_lo, lo, i))
+    return (c | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
 def mx_e4m3_quantize(w: np.ndarray, block: int = 32):
     """MX block scaling along the last axis: each block of `block` consecutive values
     shares the power-of-two scale X = 2^(floor(log2(max |v|)) - 8) (8 = the largest
@@ -637,13 +651,16 @@ def mx_e4m3_quantize(w: np.ndarray, block: int = 32):
     exp = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127).astype(np.int32)
     exp = np.clip(exp, -127, 127)
     scaled = blocks / np.ldexp(1.0, exp)[..., None]
-    codes = np.vectorize(e4m3_encode, otypes=[np.uint8])(scaled)
+    codes = e4m3_encode_array(scaled)
     return codes.reshape(w.shape), exp
+
+
+_E4M3_ALL = np.array([e4m3_decode(c) for c in range(256)])  # value of every code (NaN at 0x7F, 0xFF)
 
 
 def mx_e4m3_dequantize(codes: np.ndarray, exp: np.ndarray, block: int = 32) -> np.ndarray:
     """X * e4m3_decode(code) for every element."""
-    vals = np.vectorize(e4m3_decode, otypes=[np.float64])(np.asarray(codes))
+    vals = _E4M3_ALL[np.asarray(codes, dtype=np.int64)]
     blocks = vals.reshape(*vals.shape[:-1], vals.shape[-1] // block, block)
     return (blocks * np.ldexp(1.0, exp)[..., None]).reshape(vals.shape)
 

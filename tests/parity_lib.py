@@ -275,3 +275,70 @@ def compare_update(canvas_gpu, conf_gpu, upd_o, exempt, n):
                 f"re-noise set differs at {i}: cut margin {upd_o['cut_margin'][i]:.3e}")
         keep = [i for i in range(C) if i not in exempt]
         np.testing.assert_allclose(c[keep], upd_o["conf"][keep], rtol=5e-2)
+
+
+# ---------------------------------------------------------------- several canvases
+
+class BatchSetup:
+    """One model, B caches with prefixes of the given lengths (each its own seeded K/V)."""
+
+    def __init__(self, dg, cfg, prefixes, capacity):
+        self.cfg = cfg
+        self.host = synth.Model(cfg)
+        self.model = dg.Model(self.host)
+        self.prec = O.Precision(cfg["dtype"])
+        self.caches, self.ocaches = [], []
+        for b, P in enumerate(prefixes):
+            c = dg.KVCache(cfg, capacity)
+            if P > 0:
+                kv = synth.prefix_cache(cfg, P, seed=synth.SEED_WEIGHTS + 100 + b)
+                c.load_prefix(kv)
+                self.ocaches.append(O.Cache(kv))
+            else:
+                self.ocaches.append(O.Cache.empty(cfg))
+            self.caches.append(c)
+
+    def taps(self, rows):
+        return make_taps(self.model, self.cfg, rows)
+
+
+def batch_canvases(cfg, B, C, first=0):
+    return np.stack([synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(first + b), C, cfg["vocab"])
+                     for b in range(B)]).astype(np.int32)
+
+
+def check_batched_pass(dg, cfg, prefixes, C, prepare=None):
+    """One batched pass (each canvas with its own prefix) and each canvas's update against
+    the oracle; `prepare(setup)` may change the model first (e.g. 8-bit experts)."""
+    B = len(prefixes)
+    bt = BatchSetup(dg, cfg, prefixes, round_up(max(prefixes) + C + 8, 8))
+    if prepare is not None:
+        prepare(bt)
+    V = cfg["vocab"]
+    canv = batch_canvases(cfg, B, C)
+    taps = bt.taps(B * C)
+    ws = dg.Workspace(cfg, B * C)
+    logits = torch.empty(B, C, V, device="cuda")
+    dg.denoise_pass_batched(bt.model, bt.caches, torch.from_numpy(canv).cuda(), logits, ws)
+    # each canvas's own update from its slice of the logits
+    n = O.renoise_count(C, 1, 0, 0.25, 0.25)
+    out = torch.from_numpy(canv).cuda()
+    conf = torch.empty(B, C, device="cuda")
+    for b in range(B):
+        dg.canvas_update(logits[b], n, synth.SEED_RENOISE + b, 0, out[b], ws, conf[b])
+    dg.device_status(ws)
+    res = O.denoise_pass_batched(bt.host, bt.ocaches, list(canv), bt.prec)
+    merged = O.merge_batch_taps([t for _, t in res], cfg["n_experts"])
+    logits_o = np.concatenate([lg for lg, _ in res], axis=0)
+    report = []
+    exempt = compare_pass(cfg, taps, logits.reshape(B * C, V).cpu().numpy(), merged, logits_o, report)
+    out_np, conf_np = out.cpu().numpy(), conf.cpu().numpy()
+    for b in range(B):
+        upd_o = O.canvas_update(res[b][0], n, synth.SEED_RENOISE + b, 0)
+        ex_b = {r - b * C for r in exempt if b * C <= r < (b + 1) * C}
+        compare_update(out_np[b], conf_np[b], upd_o, ex_b, n)
+    print(report, "exempt rows:", len(exempt))
+    # the caches' committed prefixes are untouched and their lengths unchanged
+    for c, P in zip(bt.caches, prefixes):
+        assert c.len == P
+    return bt, canv, logits

@@ -255,3 +255,21 @@ def test_mx8_gemm_validation_on_host():
         assert call(**kw) == dg.DG_ERR_INVALID_ARG, kw
     assert call(sbytes=8) == dg.DG_ERR_CAPACITY
     assert L.dg_launch_count() == launches
+
+
+def test_set_experts_mx8_validation_on_host():
+    """dg_model_set_experts_mx8 refuses an fp32 model, NULL or misaligned pointers before
+    encoding anything; NULL layers turns the 8-bit experts off."""
+    cfg = CF.CONFIGS["tiny_fp32"]
+    st, h = _fake_model(cfg)
+    assert st == dg.DG_OK
+    try:
+        L = cfg["n_layers"]
+        good = (dg.ExpertsMx8 * L)(*[dg.ExpertsMx8(*[(1 << 28) + (l << 20) + (i << 16) for i in range(6)])
+                                     for l in range(L)])
+        assert dg.lib.dg_model_set_experts_mx8(h, good) == dg.DG_ERR_INVALID_ARG      # fp32 model
+        assert "bf16" in dg.lib.dg_last_error().decode()
+        assert dg.lib.dg_model_set_experts_mx8(h, None) == dg.DG_OK
+        assert dg.lib.dg_model_set_experts_mx8(None, good) == dg.DG_ERR_INVALID_ARG
+    finally:
+        dg.lib.dg_model_destroy(h)

@@ -32,81 +32,19 @@ def dg():
     return _dg
 
 
-class Batch:
-    """One model, B caches with prefixes of the given lengths (each its own seeded K/V)."""
-
-    def __init__(self, dg, cfg, prefixes, capacity):
-        self.cfg = cfg
-        self.host = synth.Model(cfg)
-        self.model = dg.Model(self.host)
-        self.prec = O.Precision(cfg["dtype"])
-        self.caches, self.ocaches = [], []
-        for b, P in enumerate(prefixes):
-            c = dg.KVCache(cfg, capacity)
-            if P > 0:
-                kv = synth.prefix_cache(cfg, P, seed=synth.SEED_WEIGHTS + 100 + b)
-                c.load_prefix(kv)
-                self.ocaches.append(O.Cache(kv))
-            else:
-                self.ocaches.append(O.Cache.empty(cfg))
-            self.caches.append(c)
-        self.dg = dg
-
-    def taps(self, rows):
-        return PL.make_taps(self.model, self.cfg, rows)
-
-
-def _canvases(cfg, B, C, first=0):
-    return np.stack([synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(first + b), C, cfg["vocab"])
-                     for b in range(B)]).astype(np.int32)
-
-
-def _check_batched_pass(dg, cfg, prefixes, C):
-    B = len(prefixes)
-    bt = Batch(dg, cfg, prefixes, PL.round_up(max(prefixes) + C + 8, 8))
-    V = cfg["vocab"]
-    canv = _canvases(cfg, B, C)
-    taps = bt.taps(B * C)
-    ws = dg.Workspace(cfg, B * C)
-    logits = torch.empty(B, C, V, device="cuda")
-    dg.denoise_pass_batched(bt.model, bt.caches, torch.from_numpy(canv).cuda(), logits, ws)
-    # each canvas's own update from its slice of the logits
-    n = O.renoise_count(C, 1, 0, 0.25, 0.25)
-    out = torch.from_numpy(canv).cuda()
-    conf = torch.empty(B, C, device="cuda")
-    for b in range(B):
-        dg.canvas_update(logits[b], n, synth.SEED_RENOISE + b, 0, out[b], ws, conf[b])
-    dg.device_status(ws)
-    res = O.denoise_pass_batched(bt.host, bt.ocaches, list(canv), bt.prec)
-    merged = O.merge_batch_taps([t for _, t in res], cfg["n_experts"])
-    logits_o = np.concatenate([lg for lg, _ in res], axis=0)
-    report = []
-    exempt = PL.compare_pass(cfg, taps, logits.reshape(B * C, V).cpu().numpy(), merged, logits_o, report)
-    out_np, conf_np = out.cpu().numpy(), conf.cpu().numpy()
-    for b in range(B):
-        upd_o = O.canvas_update(res[b][0], n, synth.SEED_RENOISE + b, 0)
-        ex_b = {r - b * C for r in exempt if b * C <= r < (b + 1) * C}
-        PL.compare_update(out_np[b], conf_np[b], upd_o, ex_b, n)
-    print(report, "exempt rows:", len(exempt))
-    # the caches' committed prefixes are untouched and their lengths unchanged
-    for c, P in zip(bt.caches, prefixes):
-        assert c.len == P
-    return bt, canv, logits
-
-
 def test_tiny_fp32_batched_pass(dg):
     cfg = CF.CONFIGS["tiny_fp32"]
-    _check_batched_pass(dg, cfg, [cfg["prefix"], 0, 17], cfg["canvas"])
+    PL.check_batched_pass(dg, cfg, [cfg["prefix"], 0, 17], cfg["canvas"])
 
 
 def test_small_bf16_batched_pass_ragged(dg):
     # ragged prefixes (one empty) and a canvas that is not a multiple of the 128-row tiles
-    _check_batched_pass(dg, SMALL_BF16, [200, 0, 131, 64], 100)
+    PL.check_batched_pass(dg, SMALL_BF16, [200, 0, 131, 64], 100)
 
 
 def test_layer1_bf16_batched_full_size(dg):
     cfg = CF.CONFIGS["layer1_bf16"]
-    _check_batched_pass(dg, cfg, [cfg["prefix"], cfg["prefix"] // 2], cfg["canvas"])
+    PL.check_batched_pass(dg, cfg, [cfg["prefix"], cfg["prefix"] // 2], cfg["canvas"])
 
 
 def test_batched_pass_equals_single_passes(dg):
@@ -116,9 +54,9 @@ def test_batched_pass_equals_single_passes(dg):
     hidden-state tolerance."""
     for cfg, prefixes, C in ((CF.CONFIGS["tiny_fp32"], [64, 0, 9], 32), (SMALL_BF16, [150, 0], 70)):
         B = len(prefixes)
-        bt = Batch(dg, cfg, prefixes, PL.round_up(max(prefixes) + C + 8, 8))
+        bt = PL.BatchSetup(dg, cfg, prefixes, PL.round_up(max(prefixes) + C + 8, 8))
         V = cfg["vocab"]
-        canv = _canvases(cfg, B, C, first=5)
+        canv = PL.batch_canvases(cfg, B, C, first=5)
         ws = dg.Workspace(cfg, B * C)
         lb = torch.empty(B, C, V, device="cuda")
         dg.denoise_pass_batched(bt.model, bt.caches, torch.from_numpy(canv).cuda(), lb, ws)
@@ -134,7 +72,7 @@ def test_prefill_append_batched_matches_oracle(dg):
     cfg = SMALL_BF16
     prefixes = [0, 40, 0]
     B, T = len(prefixes), 77
-    bt = Batch(dg, cfg, prefixes, 256)
+    bt = PL.BatchSetup(dg, cfg, prefixes, 256)
     prompts = np.stack([synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS + 50 + b, T, cfg["vocab"])
                         for b in range(B)]).astype(np.int32)
     topk = bt.taps(B * T)["topk_idx"]
@@ -159,9 +97,9 @@ def test_generate_canvases_equals_single_generation_fp32(dg):
     prefixes, C, S = [64, 0], 32, 4
     B = len(prefixes)
     seeds = [synth.SEED_RENOISE, synth.SEED_RENOISE + 7]
-    a = Batch(dg, cfg, prefixes, 256)
-    s = Batch(dg, cfg, prefixes, 256)
-    canv = _canvases(cfg, B, C, first=11)
+    a = PL.BatchSetup(dg, cfg, prefixes, 256)
+    s = PL.BatchSetup(dg, cfg, prefixes, 256)
+    canv = PL.batch_canvases(cfg, B, C, first=11)
     ws = dg.Workspace(cfg, B * C)
     lb = torch.empty(B, C, cfg["vocab"], device="cuda")
     out = torch.from_numpy(canv).cuda()

@@ -7,7 +7,10 @@ import numpy as np
 import pytest
 import torch
 
+from block_diffusion_lm_masked_b200 import configs as CF
 from oracle import dg_oracle as O
+
+import parity_lib as PL
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skip(reason="the 8-bit-weight GEMM has not yet run on a B200; enabled after its first run")]
@@ -116,3 +119,31 @@ def test_gate_up_swiglu_mx8(dg):
         g, u = xe @ wg[e].T, xe @ wu[e].T
         ref = O.silu(g) * u
         assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-4, e
+
+
+# ---------------------------------------------------------------- a whole pass with 8-bit experts
+
+SMALL_BF16 = dict(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=128, n_experts=8, top_k=2,
+                  expert_ffn=192, vocab=2048, rope_theta=10000.0, rms_eps=1e-6, dtype="bf16")
+
+
+def _experts_to_mx8(setup):
+    """Quantise the model's bf16 experts with the oracle's MX-E4M3 quantiser: the GPU model
+    gets the codes, the oracle model the decoded values (the weights the codes define)."""
+    layers = []
+    for L in setup.host.layers:
+        d = {}
+        for name, key in (("gate", "w_gate"), ("up", "w_up"), ("down", "w_down")):
+            codes, exps = O.mx_e4m3_quantize(O.widen(L[key]))
+            d[name] = (codes, exps)
+            L[key] = O.mx_e4m3_dequantize(codes, exps)
+        layers.append(d)
+    setup.model.set_experts_mx8(layers)
+
+
+@pytest.mark.parametrize("cfg,prefixes,C", [(SMALL_BF16, [200], 100), (SMALL_BF16, [64, 0, 131], 37),
+                                            (CF.CONFIGS["layer1_bf16"], [1024], 256)])
+def test_pass_with_mx8_experts_matches_oracle(dg, cfg, prefixes, C):
+    """The pass with 8-bit experts against the oracle pass over the decoded weights, under
+    the bf16 path's parity rules (the decode is exact, so nothing else changes)."""
+    PL.check_batched_pass(dg, cfg, prefixes, C, prepare=_experts_to_mx8)

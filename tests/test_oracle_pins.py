@@ -643,6 +643,21 @@ def test_e4m3_encode_round_trip_rounding_saturation():
     assert enc(464.0) == 0x7E and enc(1000.0) == 0x7E and enc(-1e6) == 0xFE   # saturation
 
 
+def test_e4m3_array_encoder_is_the_scalar_rule():
+    """The array form of the encoder agrees with e4m3_encode on every code value, every
+    midpoint between neighbours (the ties), values just beside them, saturation, signed
+    zeros and random values across the whole range."""
+    pos = np.array([O.e4m3_decode(c) for c in range(0x7F)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(41)
+    xs = np.concatenate([pos, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9), [448.0, 449.0, 464.0, 1e6],
+                         [0.0, -0.0], rng.standard_normal(4000) * np.exp(rng.uniform(-12, 7, 4000))])
+    xs = np.concatenate([xs, -xs])
+    got = O.e4m3_encode_array(xs)
+    assert got.dtype == np.uint8
+    assert list(got) == [O.e4m3_encode(v) for v in xs]
+
+
 def test_mx_e4m3_block_scaling():
     rng = np.random.default_rng(41)
     w = rng.standard_normal((6, 128)) * np.array([1e-3, 0.02, 1.0, 7.0, 300.0, 1e4])[:, None]
