@@ -260,6 +260,140 @@ def job_value(world, C, steps, max_ms):
     return world * C * steps / (max_ms / 1e3)
 
 
+def run_variant(args, cfg, name):
+    """B canvases per pass through the batched calls (each with its own cache and prefix),
+    optionally with the experts in 8-bit (MX-FP8) storage; the same metric, timing rules
+    and JSON keys as the default line, whose CPU baseline it does not repeat.  A step is
+    one batched pass plus each canvas's update."""
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    from block_diffusion_lm_masked_b200 import dg
+
+    B, mx8 = args.canvases, args.experts == "mx8"
+    P, C, V, k = cfg["prefix"], cfg["canvas"], cfg["vocab"], cfg["top_k"]
+    model = dg.Model(synth.Model(cfg), dev)
+    if mx8:
+        model.set_experts_mx8(synth.mx8_experts(cfg))
+    caches = []
+    for b in range(B):
+        c = dg.KVCache(cfg, ((P + C + 7) // 8) * 8, dev)
+        c.load_prefix(synth.prefix_cache(cfg, P, seed=synth.SEED_WEIGHTS + 100 + b))
+        caches.append(c)
+    ws = dg.Workspace(cfg, B * C, dev)
+    noise = torch.from_numpy(np.stack([synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(rank * B + b), C, V)
+                                       for b in range(B)]))
+    canv_in = noise.to(dev)
+    canv_out = torch.empty_like(canv_in)
+    logits = torch.empty(B, C, V, device=dev)
+    n_ren = dg.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step(s):
+        dg.denoise_pass_batched(model, caches, canv_in, logits, ws)
+        for b in range(B):
+            dg.canvas_update(logits[b], n_ren, synth.SEED_RENOISE + b, s, canv_out[b], ws)
+
+    unions = torch.zeros(cfg["n_layers"], dtype=torch.int32, device=dev)
+    model.set_taps({"unions": unions, "rows": B * C})
+    step(0)
+    model.set_taps(None)
+    torch.cuda.synchronize(dev)
+    unions_h = [int(u) for u in unions.cpu()]
+    for w in range(args.warmup):
+        step(w)
+    dg.device_status(ws)
+
+    def timed(K, profile):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if profile:
+            dg.profile_reset()
+            dg.profile_enable(True)
+        l0 = dg.launch_count()
+        for s_ in range(K):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            step(s_)
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if profile:
+            dg.profile_enable(False)
+        return sum(a.elapsed_time(b) for a, b in ev), dg.launch_count() - l0
+
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    clk = Clocks(dev)
+    clk.start()
+    total_ms, launches = timed(args.steps, profile=False)
+    clocks = clk.stop()
+    dg.device_status(ws)
+    total_ms = ranks.max(total_ms)
+    ranks.barrier()
+    prof_ms, _ = timed(min(args.steps, 200), profile=True)
+    kern = {}
+    for kname in dg.KERNEL_KINDS:
+        ms, n = dg.profile_read(kname)
+        if n:
+            kern[kname] = {"launches": n, "avg_us": ms * 1e3 / n, "share": ms / max(prof_ms, 1e-9)}
+
+    h_in, h_out = noise.clone().pin_memory(), torch.empty_like(noise).pin_memory()
+    e2e_ms = []
+    for s_ in range(args.steps + args.warmup):
+        flush.zero_()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        canv_in.copy_(h_in, non_blocking=True)
+        step(s_)
+        h_out.copy_(canv_out, non_blocking=True)
+        b_.record(stream)
+        b_.synchronize()
+        if s_ >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b_))
+    e2e_total = ranks.max(sum(e2e_ms))
+    dg.device_status(ws)
+
+    hbm, tf_burst, _, peak_src = _peaks()
+    ew = RF.MX8_WBYTES if mx8 else None
+    flops = B * RF.pass_flops(cfg, P, C)
+    nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew) + B * RF.update_bytes(cfg, C)
+    t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
+    ms_step = total_ms / args.steps
+    roof = None
+    gu = kern.get("gemm_gate_up")
+    if gu:
+        per_launch = RF.gate_up_bytes(cfg, unions_h[0], B * C * k, ew)
+        achieved = per_launch / (gu["avg_us"] * 1e-6) / 1e9
+        roof = {"kernel": "gemm_gate_up" + ("_mx8" if mx8 else ""), "bound": "hbm", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": per_launch}
+    line = {
+        "metric": METRIC, "value": job_value(world, B * C, args.steps, total_ms), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": _workload_desc(name, cfg), "canvases_per_pass": B,
+                   "experts": "mx8 (E4M3 + E8M0 per 32, synthetic codes)" if mx8 else "bf16",
+                   "l2": "flushed between steps (256 MB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "expert_union": unions_h},
+        "roofline": roof,
+        "pass_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof * 1e3 / ms_step, "flops": flops,
+                          "bytes": nbytes, "peak_source": peak_src},
+        "kernels": kern,
+        "e2e": {"value": job_value(world, B * C, args.steps, e2e_total), "unit": UNIT,
+                "h2d_bytes_per_step": B * C * 4, "d2h_bytes_per_step": B * C * 4},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    ranks.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -268,11 +402,19 @@ def main():
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--workload", default="layer1_bf16", choices=[n for n in CF.ORDER if n != "chained8_bf16"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--canvases", type=int, default=1,
+                    help="canvases per pass (each its own request and cache) through the batched calls")
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8"],
+                    help="expert weight storage; mx8 runs through the batched calls")
     args = ap.parse_args()
     name = args.workload
     cfg = CF.CONFIGS[name]
     if args.impl == "reference":
         return run_reference(args, cfg, name)
+    if args.canvases < 1:
+        ap.error("--canvases must be >= 1")
+    if args.canvases > 1 or args.experts != "bf16":
+        return run_variant(args, cfg, name)
 
     import torch
 

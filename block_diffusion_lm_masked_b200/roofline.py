@@ -27,20 +27,25 @@ def layer_attn_weight_bytes(cfg: dict) -> int:
     return wbytes(cfg) * H * (nq * d + 2 * nkv * d) + wbytes(cfg) * nq * d * H
 
 
-def expert_bytes(cfg: dict, union: int) -> int:
-    """Weights of `union` experts (gate, up and down matrices)."""
-    return wbytes(cfg) * 3 * cfg["hidden"] * cfg["expert_ffn"] * union
+# bytes per expert weight of the 8-bit format: one E4M3 code plus one E8M0 scale per 32
+MX8_WBYTES = 1.0 + 1.0 / 32.0
 
 
-def gate_up_bytes(cfg: dict, union: int, rows: int) -> int:
+def expert_bytes(cfg: dict, union: int, ew: float | None = None) -> float:
+    """Weights of `union` experts (gate, up and down matrices); `ew` bytes per expert
+    weight (default: the model dtype's)."""
+    return (wbytes(cfg) if ew is None else ew) * 3 * cfg["hidden"] * cfg["expert_ffn"] * union
+
+
+def gate_up_bytes(cfg: dict, union: int, rows: int, ew: float | None = None) -> float:
     """Gate/up grouped GEMM: its weights for the touched experts, its gathered input rows, its output."""
     H, F, b = cfg["hidden"], cfg["expert_ffn"], wbytes(cfg)
-    return b * 2 * H * F * union + b * rows * H + b * rows * F
+    return (b if ew is None else ew) * 2 * H * F * union + b * rows * H + b * rows * F
 
 
-def down_bytes(cfg: dict, union: int, rows: int) -> int:
+def down_bytes(cfg: dict, union: int, rows: int, ew: float | None = None) -> float:
     H, F, b = cfg["hidden"], cfg["expert_ffn"], wbytes(cfg)
-    return b * H * F * union + b * rows * F + 4 * rows * H
+    return (b if ew is None else ew) * H * F * union + b * rows * F + 4 * rows * H
 
 
 def vocab_bytes(cfg: dict, C: int) -> int:
@@ -65,16 +70,24 @@ def pass_flops(cfg: dict, P: int, C: int) -> float:
     return cfg["n_layers"] * per_layer + 2.0 * C * H * V
 
 
-def pass_bytes(cfg: dict, P: int, C: int, unions) -> float:
+def pass_bytes(cfg: dict, P: int, C: int, unions, ew: float | None = None) -> float:
     """`unions`: the expert union size of each layer (one int per layer)."""
+    return pass_bytes_batched(cfg, [P], C, unions, ew)
+
+
+def pass_bytes_batched(cfg: dict, prefixes, C: int, unions, ew: float | None = None) -> float:
+    """A pass over one canvas of C positions per cache prefix in `prefixes`: every weight
+    once (the experts of the batch's union), each canvas's K/V and logits traffic."""
     H, nkv, d, E, V = cfg["hidden"], cfg["n_kv_heads"], cfg["head_dim"], cfg["n_experts"], cfg["vocab"]
     b = wbytes(cfg)
+    B = len(prefixes)
     total = 0.0
     for l in range(cfg["n_layers"]):
-        total += layer_attn_weight_bytes(cfg) + 4 * H * E + expert_bytes(cfg, unions[l])
-        total += b * 2 * nkv * d * (P + C)        # K/V read (cached prefix + canvas)
-        total += b * 2 * nkv * d * C              # canvas K/V written
-    total += b * V * H + 4 * C * V + 4 * C * V    # output matrix, logits write + read
+        total += layer_attn_weight_bytes(cfg) + 4 * H * E + expert_bytes(cfg, unions[l], ew)
+        for P in prefixes:
+            total += b * 2 * nkv * d * (P + C)    # K/V read (cached prefix + canvas)
+            total += b * 2 * nkv * d * C          # canvas K/V written
+    total += b * V * H + B * (4 * C * V + 4 * C * V)   # output matrix, logits write + read
     return total
 
 

@@ -117,7 +117,8 @@ def tid_canvas_noise(canvas_index: int) -> int:
 
 
 def tid_layer(layer: int, j: int) -> int:
-    """j: 0 w_q, 1 w_k, 2 w_v, 3 w_o, 4 w_router, 5 w_gate, 6 w_up, 7 w_down, 8 cache K, 9 cache V"""
+    """j: 0 w_q, 1 w_k, 2 w_v, 3 w_o, 4 w_router, 5 w_gate, 6 w_up, 7 w_down, 8 cache K, 9 cache V,
+    10-12 8-bit gate / up / down codes"""
     return 1024 + 16 * layer + j
 
 
@@ -153,6 +154,38 @@ class Model:
                 w_up=normal(seed, tid_layer(l, 6), (E, F, H), std, dt),
                 w_down=normal(seed, tid_layer(l, 7), (E, H, F), std, dt),
             ))
+
+
+def _codes8(seed, tensor_id, shape, n_mag):
+    """Bytes: a random sign (bit 7) over a magnitude uniform over [0, n_mag)."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+
+    def fill(lo, hi):
+        x = splitmix64(seed, _tensor_base(tensor_id) | np.arange(lo, hi, dtype=np.uint64))
+        with np.errstate(over="ignore"):
+            mag = ((x >> np.uint64(32)) * np.uint64(n_mag)) >> np.uint64(32)
+        out[lo:hi] = (mag | (((x >> np.uint64(31)) & np.uint64(1)) << np.uint64(7))).astype(np.uint8)
+
+    _parallel(n, fill)
+    return out.reshape(shape)
+
+
+def mx8_experts(cfg: dict, seed: int = SEED_WEIGHTS):
+    """Synthetic 8-bit expert weights drawn directly as MX-FP8 data (random bytes, no
+    quantiser): per layer dict(gate=(codes, exps), up=..., down=...) with codes uint8
+    [E][F][H] (down [E][H][F]) -- a random sign over an E4M3 magnitude code uniform over
+    0x00..0x6F -- and every block exponent -12 (one per 32 elements), so weights are
+    E4M3 values up to 120 times 2^-12 (magnitudes up to about 0.03)."""
+    E, F, H = cfg["n_experts"], cfg["expert_ffn"], cfg["hidden"]
+    out = []
+    for l in range(cfg["n_layers"]):
+        d = {}
+        for j, (name, shape) in enumerate((("gate", (E, F, H)), ("up", (E, F, H)), ("down", (E, H, F)))):
+            codes = _codes8(seed, tid_layer(l, 10 + j), shape, 0x70)
+            d[name] = (codes, np.full(shape[:-1] + (shape[-1] // 32,), -12, dtype=np.int32))
+        out.append(d)
+    return out
 
 
 def prefix_cache(cfg: dict, P: int, seed: int = SEED_WEIGHTS):

@@ -726,6 +726,21 @@ def test_renoise_schedule_golden():
 
 # ---------------------------------------------------------------- roofline calculator
 
+def test_roofline_batch_and_8bit_accounting():
+    """A batch of one is the single pass; a batch of B counts the weights once and each
+    canvas's K/V and logits B times; 8-bit experts count 1 + 1/32 bytes per weight."""
+    from block_diffusion_lm_masked_b200 import configs as CF
+    cfg = CF.CONFIGS["layer1_bf16"]
+    P, C, U = 1024, 256, [52]
+    one = R.pass_bytes(cfg, P, C, U)
+    assert R.pass_bytes_batched(cfg, [P], C, U) == one
+    H, nkv, d, V, F = cfg["hidden"], cfg["n_kv_heads"], cfg["head_dim"], cfg["vocab"], cfg["expert_ffn"]
+    per_canvas = 2 * 2 * nkv * d * (P + C) + 2 * 2 * nkv * d * C + 8 * C * V
+    assert R.pass_bytes_batched(cfg, [P] * 4, C, U) == one + 3 * per_canvas
+    assert one - R.pass_bytes(cfg, P, C, U, ew=R.MX8_WBYTES) == (2 - 1 - 1 / 32) * 3 * H * F * 52
+    assert R.gate_up_bytes(cfg, 52, 1024, ew=1.0) == 2 * H * F * 52 + 2 * 1024 * (H + F)
+
+
 def test_roofline_reproduces_exercise_arithmetic():
     g = {r[0]: float(r[1]) for r in _read_golden("roofline_h100_model.txt")}
     bw, peak = 3.35e12, 990e12

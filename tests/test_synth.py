@@ -29,3 +29,19 @@ def test_tokens_uniform_in_range():
     assert t.min() >= 0 and t.max() < 1000
     cnt = np.bincount(t, minlength=1000)
     assert cnt.min() > 40 and cnt.max() < 170
+
+
+def test_mx8_experts_are_valid_deterministic_codes(monkeypatch):
+    cfg = dict(n_layers=1, hidden=128, n_experts=2, expert_ffn=64)
+    a = synth.mx8_experts(cfg)
+    monkeypatch.setattr(synth, "_CHUNK", 1000)
+    b = synth.mx8_experts(cfg)
+    for name, shape in (("gate", (2, 64, 128)), ("up", (2, 64, 128)), ("down", (2, 128, 64))):
+        codes, exps = a[0][name]
+        assert codes.shape == shape and codes.dtype == np.uint8
+        np.testing.assert_array_equal(codes, b[0][name][0])
+        assert not np.isin(codes, [0x7F, 0xFF]).any()            # no NaN codes
+        mag = codes & 0x7F
+        assert mag.max() == 0x6F and 0.4 < (codes >> 7).mean() < 0.6
+        assert exps.shape == shape[:-1] + (shape[-1] // 32,) and (exps == -12).all()
+    assert (a[0]["gate"][0] != a[0]["up"][0]).mean() > 0.9
