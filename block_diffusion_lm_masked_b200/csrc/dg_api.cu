@@ -168,6 +168,22 @@ static dg_status map_scales(CUtensorMap* m, const void* base, uint64_t groups, u
   const uint32_t box[3] = {256, 1, 1};
   return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
+// 4-bit weight codes [groups][rows][cols / 2] (two per byte) as a 3-D map, box (32 bytes =
+// 64 cols, 128 rows, 1 group), 32-byte swizzle
+static dg_status map_codes4(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const uint64_t dims[3] = {cols / 2, rows, groups};
+  const uint64_t strides[2] = {cols / 2, rows * cols / 2};
+  const uint32_t box[3] = {32, 128, 1};
+  return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B);
+}
+// their E4M3 scales [groups][cols / 64][rows][4], viewed as 16-byte rows of 4 weight rows:
+// dims (16, rows / 4, groups * cols / 64), box (16, 32, 1) = one 128-row tile's scales
+static dg_status map_scales4(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const uint64_t dims[3] = {16, rows / 4, groups * (cols / 64)};
+  const uint64_t strides[2] = {16, rows * 4};
+  const uint32_t box[3] = {16, 32, 1};
+  return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
 // row-major [rows][cols] bf16 matrix as a 2-D map with box (64 cols, box_rows rows)
 static dg_status map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   const uint64_t dims[2] = {cols, rows};
@@ -469,8 +485,8 @@ dg_status gemm_mx8(const GemmCall& g, const CUtensorMap* S, const CUtensorMap* S
   p.smem_budget = g.smem_budget;
   p.err = err;
   LAUNCH(g.kind, st,
-         dg::launch_tc_gemm_mx8(g.epi, *g.A, g.A2 ? *g.A2 : *g.A, *S, S2 ? *S2 : *S, B, B2, Bb, B2b, p,
-                                g.max_items * p.m_tiles, st));
+         dg::launch_tc_gemm_lowp(dg::FMT_MX8, g.epi, *g.A, g.A2 ? *g.A2 : *g.A, *S, S2 ? *S2 : *S, B, B2, Bb, B2b,
+                                 p, 1.0f, 1.0f, g.max_items * p.m_tiles, st));
   return DG_OK;
 }
 
@@ -1291,11 +1307,36 @@ extern "C" dg_status dg_debug_gemm_bf16(const void* W, const void* W2, int32_t r
   return gemm_bf16(g, d_err, st);
 }
 
+static dg_status debug_gemm_lowp(int fmt, const void* W, const void* W_scales, float g, const void* W2,
+                                 const void* W2_scales, float g2, int32_t rows, int32_t n_groups, const void* X,
+                                 const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off, void* out,
+                                 void* out_lo, int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
+                                 dg_stream stream);
+
 extern "C" dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, const void* W2, const void* W2_scales,
                                        int32_t rows, int32_t n_groups, const void* X, const void* X_lo,
                                        int32_t x_rows, int32_t K, const int32_t* group_off, void* out, void* out_lo,
                                        int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
                                        dg_stream stream) {
+  return debug_gemm_lowp(dg::FMT_MX8, W, W_scales, 1.0f, W2, W2_scales, 1.0f, rows, n_groups, X, X_lo, x_rows, K,
+                         group_off, out, out_lo, ld_out, d_scratch, scratch_bytes, d_err, stream);
+}
+
+extern "C" dg_status dg_debug_gemm_nv4(const void* W, const void* W_scales, float g, const void* W2,
+                                       const void* W2_scales, float g2, int32_t rows, int32_t n_groups, const void* X,
+                                       const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off,
+                                       void* out, void* out_lo, int32_t ld_out, void* d_scratch,
+                                       size_t scratch_bytes, int32_t* d_err, dg_stream stream) {
+  DG_CHECK_ARG(isfinite(g) && (!W2 || isfinite(g2)), "tensor scales must be finite");
+  return debug_gemm_lowp(dg::FMT_NV4, W, W_scales, g, W2, W2_scales, g2, rows, n_groups, X, X_lo, x_rows, K,
+                         group_off, out, out_lo, ld_out, d_scratch, scratch_bytes, d_err, stream);
+}
+
+static dg_status debug_gemm_lowp(int fmt, const void* W, const void* W_scales, float g, const void* W2,
+                                 const void* W2_scales, float g2, int32_t rows, int32_t n_groups, const void* X,
+                                 const void* X_lo, int32_t x_rows, int32_t K, const int32_t* group_off, void* out,
+                                 void* out_lo, int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
+                                 dg_stream stream) {
   DG_CHECK_ARG(W && W_scales && X && out && d_err && d_scratch, "NULL pointer");
   DG_CHECK_ARG(!W2 == !W2_scales, "W2 and its scales come together");
   DG_CHECK_ARG(K > 0 && K % 64 == 0 && rows > 0 && rows % 8 == 0 && n_groups > 0 && x_rows > 0, "bad GEMM shape");
@@ -1312,11 +1353,13 @@ extern "C" dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, cons
   constexpr int kRows = 64;  // token rows per tile of the 8-bit GEMM
   CUtensorMap A, A2, S, S2, B, B2, Bb, B2b;
   dg_status s;
-  if ((s = map_codes(&A, W, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
-  if ((s = map_scales(&S, W_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  auto codes = fmt == dg::FMT_NV4 ? map_codes4 : map_codes;
+  auto scales = fmt == dg::FMT_NV4 ? map_scales4 : map_scales;
+  if ((s = codes(&A, W, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+  if ((s = scales(&S, W_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
   if (W2) {
-    if ((s = map_codes(&A2, W2, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
-    if ((s = map_scales(&S2, W2_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+    if ((s = codes(&A2, W2, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
+    if ((s = scales(&S2, W2_scales, (uint64_t)n_groups, (uint64_t)rows, (uint64_t)K)) != DG_OK) return s;
   } else {
     A2 = A;
     S2 = S;
@@ -1356,8 +1399,8 @@ extern "C" dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, cons
   p.err = d_err;
   const int tiles = (group_off ? max_items : ceil_div(x_rows, p.n_max)) * p.m_tiles;
   LAUNCH(DG_K_GEMM_GATE_UP, st,
-         dg::launch_tc_gemm_mx8(W2 ? dg::EPI_SWIGLU_BF16 : dg::EPI_STORE_F32, A, A2, S, S2, B, B2, Bb, B2b, p, tiles,
-                                st));
+         dg::launch_tc_gemm_lowp(fmt, W2 ? dg::EPI_SWIGLU_BF16 : dg::EPI_STORE_F32, A, A2, S, S2, B, B2, Bb, B2b,
+                                 p, g, g2, tiles, st));
   return DG_OK;
 }
 

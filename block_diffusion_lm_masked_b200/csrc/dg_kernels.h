@@ -46,14 +46,20 @@ struct TcGemmParams {
 cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& B,
                            const CUtensorMap& B2, const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p,
                            int max_tiles, cudaStream_t st);
-// The same GEMM over 8-bit weights: A / A2 are E4M3 codes (3-D maps (K, rows, groups) of
-// bytes, box 64 x 128 x 1, 64-byte swizzle), S / S2 their E8M0 block scales laid out
-// [groups][K / 64][rows][2] (3-D maps (2 rows, K / 64, groups), box 256 x 1 x 1).  Token
-// maps, work list and epilogues as launch_tc_gemm; n_max <= 64, k_splits == 1.
-cudaError_t launch_tc_gemm_mx8(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
-                               const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
-                               const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, int max_tiles,
-                               cudaStream_t st);
+// The same GEMM over low-precision weights decoded exactly to bf16 (token maps, work list
+// and epilogues as launch_tc_gemm; n_max <= 64, k_splits == 1).  A / A2: weight codes,
+// S / S2: their block scales, as byte tensors.
+//   FMT_MX8: E4M3 codes, 3-D maps (K bytes, rows, groups), box 64 x 128 x 1, 64-byte swizzle;
+//            E8M0 scales [groups][K / 64][rows][2], 3-D maps (2 rows, K / 64, groups), box 256 x 1 x 1.
+//   FMT_NV4: E2M1 codes two per byte, 3-D maps (K / 2 bytes, rows, groups), box 32 x 128 x 1,
+//            32-byte swizzle; E4M3 scales [groups][K / 64][rows][4] as 3-D maps
+//            (16 bytes = 4 rows, rows / 4, groups * K / 64), box 16 x 32 x 1; the epilogue
+//            multiplies the accumulators by the tensor scales g_a (and g_a2 for A2).
+enum LowpFormat { FMT_MX8 = 0, FMT_NV4 = 1 };
+cudaError_t launch_tc_gemm_lowp(int fmt, int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
+                                const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
+                                const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, float g_a,
+                                float g_a2, int max_tiles, cudaStream_t st);
 // grouped work list from group offsets off[E + 1] over `rows` token rows (checked on the
 // device: bad offsets give no items and DG_DEVERR_BAD_COUNT in *err)
 cudaError_t launch_build_items(const int32_t* off, int E, int n_max, int rows, TcWorkItem* items, int* n_items,

@@ -31,15 +31,24 @@
 // subnormal codes round to bf16's subnormal grid).  Preconditions: s <= 134 (block scale
 // <= 2^7, so the multiplier is a finite bf16), and codes 0x7F / 0xFF (NaN in E4M3) do
 // not occur (they would decode as 480 times the scale).
+//
+// The 4-bit format (FMT_NV4) runs through the same kernel: E2M1 codes (sign, 2 exponent
+// bits with bias 1, 1 mantissa bit; two per byte, the lower-indexed element in the low
+// nibble), one E4M3 scale per 16 consecutive K elements, and one fp32 scale per weight
+// tensor.  Code value times block scale has at most 6 significant bits, so the decoded
+// bf16 weight is exact; the tensor scale multiplies the fp32 accumulator in the
+// epilogue.  A code's bf16 bytes come from two 8-entry tables by byte permutes, its sign
+// is merged with one select, and one bf16 multiply applies the block scale.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
 namespace dg {
 
 constexpr int MX_BM = 128;                    // weight rows per tile
-constexpr int MX_BK = 64;                     // K elements per k-block (two scale blocks)
-constexpr uint32_t MX_A_BYTES = MX_BM * MX_BK;  // one 8-bit weight tile
-constexpr uint32_t MX_S_BYTES = MX_BM * 2;      // its scales: two per row
+constexpr int MX_BK = 64;                     // K elements per k-block
+// per format: bytes of one weight tile (128 rows x 64 K) and of its scales
+__host__ __device__ constexpr uint32_t mx_a_bytes(int fmt) { return fmt == FMT_NV4 ? MX_BM * MX_BK / 2 : MX_BM * MX_BK; }
+__host__ __device__ constexpr uint32_t mx_s_bytes(int fmt) { return fmt == FMT_NV4 ? MX_BM * 4 : MX_BM * 2; }
 constexpr int MX_T_STAGES = 4;                // TMEM stages of decoded weights
 constexpr int MX_F_STAGES_MAX = 8;
 constexpr int MX_DEC_WARPS = 8;
@@ -113,13 +122,40 @@ __device__ __forceinline__ void mx8_decode4(uint32_t x, uint32_t mm, uint32_t& p
   p23 = bf16x2_mul((s23 & 0x80008000u) | m23, mm);
 }
 
-template <int EPI>
+// bf16 bytes of the E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (high bytes, then low bytes)
+constexpr uint32_t NV4_HI_A = 0x3F3F3F00u, NV4_HI_B = 0x40404040u;
+constexpr uint32_t NV4_LO_A = 0xC0800000u, NV4_LO_B = 0xC0804000u;
+
+// eight 4-bit codes (code i in bits 4i .. 4i+3) -> four bf16x2 words (codes 2j, 2j+1 in
+// word j, the lower-indexed code in the low half), each value times the multiplier pair mm
+__device__ __forceinline__ void nv4_decode8(uint32_t x, uint32_t mm, uint32_t (&w)[4]) {
+  const uint32_t mags = x & 0x77777777u;  // table indices (the selector's replicate bits clear)
+  const uint32_t h0 = __byte_perm(NV4_HI_A, NV4_HI_B, mags), h1 = __byte_perm(NV4_HI_A, NV4_HI_B, mags >> 16);
+  const uint32_t l0 = __byte_perm(NV4_LO_A, NV4_LO_B, mags), l1 = __byte_perm(NV4_LO_A, NV4_LO_B, mags >> 16);
+  const uint32_t xs = x << 4;  // byte j of xs carries code 2j's sign in bit 7; byte j of x, code 2j+1's
+  const uint32_t m0 = __byte_perm(l0, h0, 0x5140), m1 = __byte_perm(l0, h0, 0x7362);
+  const uint32_t m2 = __byte_perm(l1, h1, 0x5140), m3 = __byte_perm(l1, h1, 0x7362);
+  w[0] = bf16x2_mul(m0 | (__byte_perm(xs, x, 0x4000) & 0x80008000u), mm);
+  w[1] = bf16x2_mul(m1 | (__byte_perm(xs, x, 0x5010) & 0x80008000u), mm);
+  w[2] = bf16x2_mul(m2 | (__byte_perm(xs, x, 0x6020) & 0x80008000u), mm);
+  w[3] = bf16x2_mul(m3 | (__byte_perm(xs, x, 0x7030) & 0x80008000u), mm);
+}
+
+// bf16x2 pair of an E4M3 block scale (non-negative; exact: 4 significant bits, 2^-9..448)
+__device__ __forceinline__ uint32_t e4m3_scale_pair(uint32_t sc) {
+  const float f = __uint_as_float((sc & 0x7Fu) << 20) * 0x1p120f;  // the f32 bit trick, subnormal codes included
+  const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+  return h | (h << 16);
+}
+
+template <int EPI, int FMT>
 __global__ void __launch_bounds__(MX_THREADS, 1)
     tc_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                        const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmS2,
                        const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                        const __grid_constant__ CUtensorMap tmBb, const __grid_constant__ CUtensorMap tmB2b,
-                       const TcGemmParams p) {
+                       const TcGemmParams p, const float g_a, const float g_a2) {
+  constexpr uint32_t MX_A_BYTES = mx_a_bytes(FMT), MX_S_BYTES = mx_s_bytes(FMT);
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t f_full[MX_F_STAGES_MAX];   // a stage's TMA loads landed
   __shared__ __align__(8) uint64_t f_empty[MX_F_STAGES_MAX];  // decoders and MMAs are done with it
@@ -210,11 +246,17 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
           const int kbx = (kb + t) % nkb;  // tiles running together start at different k-blocks
           const int kx = kbx * MX_BK;
           mbar_arrive_expect_tx(&f_full[s], tx);
-          tma_load_3d(st + a_off, &tmA, kx, ti.m * MX_BM, ti.g, &f_full[s]);
-          tma_load_3d(st + s_off, &tmS, ti.m * MX_BM * 2, kbx, ti.g, &f_full[s]);
+          // codes: x in bytes along K; scales: MX8 (2 rows' bytes, k-block, group),
+          // NV4 (16 bytes = 4 rows, rows / 4, group * k-blocks + k-block)
+          const int ax = FMT == FMT_NV4 ? kx / 2 : kx;
+          const int s0 = FMT == FMT_NV4 ? 0 : ti.m * MX_BM * 2;
+          const int s1 = FMT == FMT_NV4 ? ti.m * (MX_BM / 4) : kbx;
+          const int s2 = FMT == FMT_NV4 ? ti.g * nkb + kbx : ti.g;
+          tma_load_3d(st + a_off, &tmA, ax, ti.m * MX_BM, ti.g, &f_full[s]);
+          tma_load_3d(st + s_off, &tmS, s0, s1, s2, &f_full[s]);
           if (p.dual_a) {
-            tma_load_3d(st + a_off + MX_A_BYTES, &tmA2, kx, ti.m * MX_BM, ti.g, &f_full[s]);
-            tma_load_3d(st + s_off + MX_S_BYTES, &tmS2, ti.m * MX_BM * 2, kbx, ti.g, &f_full[s]);
+            tma_load_3d(st + a_off + MX_A_BYTES, &tmA2, ax, ti.m * MX_BM, ti.g, &f_full[s]);
+            tma_load_3d(st + s_off + MX_S_BYTES, &tmS2, s0, s1, s2, &f_full[s]);
           }
           int r = 0;
           for (; r + MX_B_BOX_BIG <= n_pad; r += MX_B_BOX_BIG) {
@@ -299,8 +341,12 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int col = c0 + q;
-          const float a = __uint_as_float(ra[q]);
-          const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
+          float a = __uint_as_float(ra[q]);
+          float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
+          if (FMT == FMT_NV4) {  // the tensor scales
+            a *= g_a;
+            b *= g_a2;
+          }
           if (!fvalid || col >= ti.rows) continue;
           const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
           if (EPI == EPI_STORE_F32) {
@@ -323,7 +369,10 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
     const int half = (warp - MX_DEC_WARP0) >> 2;
     const int row = lq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(lq * 32) << 16;
-    const int swz = (row >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of the row sits at c ^ swz
+    // 16-byte chunk c of the row sits at c ^ swz: MX8 rows of 64 bytes, 64-byte swizzle;
+    // NV4 rows of 32 bytes, 32-byte swizzle
+    const int swz = FMT == FMT_NV4 ? (row >> 2) & 1 : (row >> 1) & 3;
+    constexpr int row_bytes = FMT == FMT_NV4 ? MX_BK / 2 : MX_BK;
     int it = 0, t;
     bool ok = true;
     MxWalk walk(n_tiles);
@@ -339,19 +388,35 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
         tc_fence_after();
         const uint8_t* st = smem + (size_t)s * stage_bytes;
         for (int a = 0; a < n_a; ++a) {
-          const uint8_t* codes = st + a_off + (uint32_t)a * MX_A_BYTES + row * MX_BK;
-          const uint32_t e8 = st[s_off + (uint32_t)a * MX_S_BYTES + row * 2 + half];
-          const uint32_t mh = (e8 + 120u) << 7;  // bf16 bits of 2^(e8 - 7)
-          const uint32_t mm = mh | (mh << 16);
+          const uint8_t* codes = st + a_off + (uint32_t)a * MX_A_BYTES + row * row_bytes;
           uint32_t w[16];
+          if (FMT == FMT_NV4) {
+            // 32 codes = one 16-byte chunk; block scales 2 half and 2 half + 1 (16 elements each)
+            const uint8_t* sc = st + s_off + (uint32_t)a * MX_S_BYTES + row * 4 + 2 * half;
+            const uint32_t mm0 = e4m3_scale_pair(sc[0]), mm1 = e4m3_scale_pair(sc[1]);
+            const uint4 v = *reinterpret_cast<const uint4*>(codes + ((half ^ swz) << 4));
+            uint32_t q[4];
+            nv4_decode8(v.x, mm0, q);
+            w[0] = q[0], w[1] = q[1], w[2] = q[2], w[3] = q[3];
+            nv4_decode8(v.y, mm0, q);
+            w[4] = q[0], w[5] = q[1], w[6] = q[2], w[7] = q[3];
+            nv4_decode8(v.z, mm1, q);
+            w[8] = q[0], w[9] = q[1], w[10] = q[2], w[11] = q[3];
+            nv4_decode8(v.w, mm1, q);
+            w[12] = q[0], w[13] = q[1], w[14] = q[2], w[15] = q[3];
+          } else {
+            const uint32_t e8 = st[s_off + (uint32_t)a * MX_S_BYTES + row * 2 + half];
+            const uint32_t mh = (e8 + 120u) << 7;  // bf16 bits of 2^(e8 - 7)
+            const uint32_t mm = mh | (mh << 16);
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const int c = 2 * half + c2;
-            const uint4 v = *reinterpret_cast<const uint4*>(codes + ((c ^ swz) << 4));
-            mx8_decode4(v.x, mm, w[c2 * 8 + 0], w[c2 * 8 + 1]);
-            mx8_decode4(v.y, mm, w[c2 * 8 + 2], w[c2 * 8 + 3]);
-            mx8_decode4(v.z, mm, w[c2 * 8 + 4], w[c2 * 8 + 5]);
-            mx8_decode4(v.w, mm, w[c2 * 8 + 6], w[c2 * 8 + 7]);
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int c = 2 * half + c2;
+              const uint4 v = *reinterpret_cast<const uint4*>(codes + ((c ^ swz) << 4));
+              mx8_decode4(v.x, mm, w[c2 * 8 + 0], w[c2 * 8 + 1]);
+              mx8_decode4(v.y, mm, w[c2 * 8 + 2], w[c2 * 8 + 3]);
+              mx8_decode4(v.z, mm, w[c2 * 8 + 4], w[c2 * 8 + 5]);
+              mx8_decode4(v.w, mm, w[c2 * 8 + 6], w[c2 * 8 + 7]);
+            }
           }
           tmem_st16(tmem + lane_off + a_col0 + (uint32_t)ts * a_stage_cols + (uint32_t)a * 32u + (uint32_t)half * 16u,
                     w);
@@ -379,37 +444,46 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 }
 
-cudaError_t launch_tc_gemm_mx8(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
-                               const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
-                               const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, int max_tiles,
-                               cudaStream_t st) {
+template <int FMT>
+static cudaError_t launch_fmt(int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
+                              const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
+                              const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, float g_a,
+                              float g_a2, int grid, int smem, cudaStream_t st) {
+  cudaError_t e;
+  if (epi == EPI_STORE_F32) {
+    e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_STORE_F32, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(tc_gemm_mx8_kernel<EPI_STORE_F32, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B,
+                    B2, Bb, B2b, p, g_a, g_a2);
+  }
+  if (epi == EPI_SWIGLU_BF16) {
+    e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2,
+                    B, B2, Bb, B2b, p, g_a, g_a2);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc_gemm_lowp(int fmt, int epi, const CUtensorMap& A, const CUtensorMap& A2, const CUtensorMap& S,
+                                const CUtensorMap& S2, const CUtensorMap& B, const CUtensorMap& B2,
+                                const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, float g_a,
+                                float g_a2, int max_tiles, cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
-  if (p.k_splits != 1 || p.K % MX_BK != 0 || p.K <= 0 || p.n_max < 16 || p.n_max > 64 || (p.n_max % 16) != 0 ||
-      p.m_tiles < 1 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
+  if ((fmt != FMT_MX8 && fmt != FMT_NV4) || p.k_splits != 1 || p.K % MX_BK != 0 || p.K <= 0 || p.n_max < 16 ||
+      p.n_max > 64 || (p.n_max % 16) != 0 || p.m_tiles < 1 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
     return cudaErrorInvalidValue;
   const int n_a = p.dual_a ? 2 : 1;
   const int terms = p.two_terms ? 2 : 1;
-  const int stage = ((terms * p.n_max * 128 + n_a * (int)(MX_A_BYTES + MX_S_BYTES)) + 1023) & ~1023;
+  const int stage = ((terms * p.n_max * 128 + n_a * (int)(mx_a_bytes(fmt) + mx_s_bytes(fmt))) + 1023) & ~1023;
   if (p.smem_budget < 2 * stage) return cudaErrorInvalidValue;
   const int smem = p.smem_budget + 1024;
   const int sms = num_sms();
   const int grid = max_tiles < sms ? max_tiles : sms;
-  cudaError_t e;
-  switch (epi) {
-    case EPI_STORE_F32:
-      e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_STORE_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      return launch_k(tc_gemm_mx8_kernel<EPI_STORE_F32>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B, B2,
-                      Bb, B2b, p);
-    case EPI_SWIGLU_BF16:
-      e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               smem);
-      if (e != cudaSuccess) return e;
-      return launch_k(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B,
-                      B2, Bb, B2b, p);
-    default:
-      return cudaErrorInvalidValue;
-  }
+  return fmt == FMT_NV4 ? launch_fmt<FMT_NV4>(epi, A, A2, S, S2, B, B2, Bb, B2b, p, g_a, g_a2, grid, smem, st)
+                        : launch_fmt<FMT_MX8>(epi, A, A2, S, S2, B, B2, Bb, B2b, p, g_a, g_a2, grid, smem, st);
 }
 
 }  // namespace dg

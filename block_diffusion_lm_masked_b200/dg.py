@@ -99,6 +99,7 @@ def _load():
         "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_scratch_bytes": (SZ, [I32, I32]),
         "dg_debug_gemm_mx8": (I32, [P, P, P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
+        "dg_debug_gemm_nv4": (I32, [P, P, F32, P, P, F32, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -432,6 +433,34 @@ def debug_gemm_mx8(W, W_scales, X, out, ld_out, err, scratch, W2=None, W2_scales
     _check(lib.dg_debug_gemm_mx8(_ptr(W), _ptr(W_scales), _ptr(W2), _ptr(W2_scales), rows, G, _ptr(X), _ptr(X_lo),
                                  X.shape[0], K, _ptr(group_off), _ptr(out), _ptr(out_lo), ld_out, _ptr(scratch),
                                  scratch.numel(), _ptr(err), _stream(stream)))
+
+
+def pack_nv4_codes(codes: np.ndarray) -> np.ndarray:
+    """4-bit codes, one per byte [groups][rows][K] -> two per byte [groups][rows][K / 2]
+    (element 2 i in the low nibble of byte i)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    if c.shape[-1] % 2 or (c > 0xF).any():
+        raise ValueError("4-bit codes in [0, 16) with an even row length")
+    return np.ascontiguousarray(c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def pack_nv4_scales(scale_codes: np.ndarray) -> np.ndarray:
+    """E4M3 block-scale codes [groups][rows][K / 16] -> the library's [groups][K / 64][rows][4]."""
+    sc = np.asarray(scale_codes, dtype=np.uint8)
+    G, R, nb = sc.shape
+    if nb % 4:
+        raise ValueError("four block scales per 64 K elements")
+    return np.ascontiguousarray(sc.reshape(G, R, nb // 4, 4).transpose(0, 2, 1, 3))
+
+
+def debug_gemm_nv4(W, W_scales, g, X, out, ld_out, err, scratch, W2=None, W2_scales=None, g2=1.0, X_lo=None,
+                   group_off=None, out_lo=None, stream=None):
+    """One launch of the 4-bit-weight GEMM (see include/dg_debug.h): W uint8 packed codes
+    [groups][rows][K / 2], W_scales uint8 [groups][K / 64][rows][4], g the tensor scale."""
+    G, rows, K2 = W.shape
+    _check(lib.dg_debug_gemm_nv4(_ptr(W), _ptr(W_scales), float(g), _ptr(W2), _ptr(W2_scales), float(g2), rows, G,
+                                 _ptr(X), _ptr(X_lo), X.shape[0], 2 * K2, _ptr(group_off), _ptr(out), _ptr(out_lo),
+                                 ld_out, _ptr(scratch), scratch.numel(), _ptr(err), _stream(stream)))
 
 
 def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out_lo=None, stream=None):

@@ -103,6 +103,21 @@ dg_status dg_debug_gemm_mx8(const void* W, const void* W_scales, const void* W2,
                             const int32_t* group_off, void* out, void* out_lo, int32_t ld_out, void* d_scratch,
                             size_t scratch_bytes, int32_t* d_err, dg_stream stream);
 
+/* The same GEMM over 4-bit weights (NVFP4-style storage: E2M1 elements -- sign, 2 exponent
+ * bits with bias 1, 1 mantissa bit -- with one E4M3 scale per 16 consecutive K elements of
+ * a row and one fp32 scale g per weight tensor): every weight is
+ * e2m1(code) * e4m3(block scale) * g.  Code times block scale is decoded exactly to bf16
+ * in the kernel and g multiplies the fp32 accumulator, so
+ *   acc[r][f] = g * sum_k dec(W)[g][f][k] * (X[r][k] + X_lo[r][k]).
+ * W (and W2): uint8 [n_groups][rows][K / 2], element 2 i of a row in the low nibble of
+ * byte i.  W_scales (and W2_scales): E4M3 codes uint8 [n_groups][K / 64][rows][4], entry
+ * [g][j][f][b] the scale of elements 64 j + 16 b .. + 15 of row f (non-negative, not NaN).
+ * g (and g2 for W2): finite.  Everything else as dg_debug_gemm_mx8. */
+dg_status dg_debug_gemm_nv4(const void* W, const void* W_scales, float g, const void* W2, const void* W2_scales,
+                            float g2, int32_t rows, int32_t n_groups, const void* X, const void* X_lo,
+                            int32_t x_rows, int32_t K, const int32_t* group_off, void* out, void* out_lo,
+                            int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err, dg_stream stream);
+
 /* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
  * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
  * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128] (hi part); out_lo (nullable)

@@ -273,3 +273,19 @@ def test_set_experts_mx8_validation_on_host():
         assert dg.lib.dg_model_set_experts_mx8(None, good) == dg.DG_ERR_INVALID_ARG
     finally:
         dg.lib.dg_model_destroy(h)
+
+
+def test_nv4_gemm_validation_on_host():
+    p = ctypes.c_void_p(1 << 24)
+    err, sc = ctypes.c_void_p(1 << 25), ctypes.c_void_p(1 << 26)
+    L = dg.lib
+    launches = L.dg_launch_count()
+
+    def call(g=1.0, W2=None, S2=None, g2=1.0, K=128, rows=128):
+        return L.dg_debug_gemm_nv4(p, p, g, W2, S2, g2, rows, 1, p, None, 16, K, None, p, None, rows, sc, 1 << 20,
+                                   err, None)
+
+    for kw in (dict(g=float("nan")), dict(g=float("inf")), dict(W2=p, S2=p, g2=float("nan")), dict(W2=p),
+               dict(K=96), dict(rows=12)):
+        assert call(**kw) == dg.DG_ERR_INVALID_ARG, kw
+    assert L.dg_launch_count() == launches

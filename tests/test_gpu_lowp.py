@@ -1,8 +1,9 @@
-"""The 8-bit-weight GEMM (dg_debug_gemm_mx8) against the oracle: weights quantised by
-the oracle's MX-E4M3 quantiser, the expected products computed in fp64 from the
-oracle's decoding of the same codes.  Exact where the arithmetic allows it (decoding:
-identity activations give the decoded weights themselves), fp32-accumulation close
-elsewhere."""
+"""The low-precision-weight GEMMs (dg_debug_gemm_mx8: MX-FP8; dg_debug_gemm_nv4: 4-bit
+E2M1 with E4M3 block scales and a tensor scale) against the oracle: weights quantised by
+the oracle's quantisers, the expected products computed in fp64 from the oracle's
+decoding of the same codes.  Exact where the arithmetic allows it (decoding: identity
+activations give the decoded weights themselves), fp32-accumulation close elsewhere;
+and whole passes with 8-bit experts."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +14,8 @@ from oracle import dg_oracle as O
 import parity_lib as PL
 
 pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="the 8-bit-weight GEMM has not yet run on a B200; enabled after its first run")]
+              pytest.mark.skip(reason="the low-precision-weight GEMMs have not yet run on a B200; enabled after their "
+                                      "first run")]
 
 
 @pytest.fixture(scope="module")
@@ -147,3 +149,72 @@ def test_pass_with_mx8_experts_matches_oracle(dg, cfg, prefixes, C):
     """The pass with 8-bit experts against the oracle pass over the decoded weights, under
     the bf16 path's parity rules (the decode is exact, so nothing else changes)."""
     PL.check_batched_pass(dg, cfg, prefixes, C, prepare=_experts_to_mx8)
+
+
+# ---------------------------------------------------------------- 4-bit weights
+
+def _nv4(rng, G, rows, K, std=0.02):
+    w = rng.standard_normal((G, rows, K)) * std
+    codes, sc, g = O.nvfp4_quantize(w)
+    return codes, sc, g, O.nvfp4_dequantize(codes, sc, g)
+
+
+def _run_nv4(dg, codes, sc, g, X, out_cols, X_lo=None, group_off=None, c2=None, sc2=None, g2=1.0, out_lo=None):
+    W = torch.from_numpy(dg.pack_nv4_codes(codes)).cuda()
+    S = torch.from_numpy(dg.pack_nv4_scales(sc)).cuda()
+    W2 = torch.from_numpy(dg.pack_nv4_codes(c2)).cuda() if c2 is not None else None
+    S2 = torch.from_numpy(dg.pack_nv4_scales(sc2)).cuda() if c2 is not None else None
+    n = X.shape[0]
+    dt = torch.bfloat16 if c2 is not None else torch.float32
+    out = torch.full((n, out_cols), float("nan"), device="cuda", dtype=dt)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dg.debug_gemm_nv4(W, S, g, X, out, out_cols, err, dg.debug_gemm_scratch(n, codes.shape[0]), W2=W2, W2_scales=S2,
+                      g2=g2, X_lo=X_lo, group_off=group_off, out_lo=out_lo)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    return out
+
+
+def test_nv4_decoding_is_exact_for_every_code_and_scale(dg):
+    """Every 4-bit code under block scales across the E4M3 range, tensor scale 1: with X = I
+    the output is the decoded weight matrix, bit for bit the oracle's."""
+    K, rows = 256, 128
+    codes = np.array([[(r + 7 * k) % 16 for k in range(K)] for r in range(rows)], dtype=np.uint8)[None]
+    sc = np.array([[[(3 + 11 * r + 5 * b) % 0x7F for b in range(K // 16)] for r in range(rows)]], dtype=np.uint8)
+    want = O.nvfp4_dequantize(codes, sc, 1.0)[0]
+    X = torch.eye(K, dtype=torch.bfloat16, device="cuda")
+    out = _run_nv4(dg, codes, sc, 1.0, X, rows)
+    np.testing.assert_array_equal(out.double().cpu().numpy(), want.T)
+
+
+@pytest.mark.parametrize("counts,M", [([0, 3, 17, 40, 1], 256), ([64, 65, 0, 129], 2048), ([300, 2], 704)])
+def test_grouped_two_term_nv4_gemm(dg, counts, M):
+    rng = np.random.default_rng(sum(counts) + M + 1)
+    E, K = len(counts), 1024
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    codes, sc, g, wq = _nv4(rng, E, M, K)
+    x, hi, lo = _bf16_pair(rng, int(off[-1]), K)
+    out = _run_nv4(dg, codes, sc, g, hi, M, X_lo=lo, group_off=torch.from_numpy(off).cuda())
+    got = out.double().cpu().numpy()
+    for e in range(E):
+        ref = x[off[e]:off[e + 1]] @ wq[e].T
+        if ref.size:
+            assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 2e-5, e
+
+
+def test_gate_up_swiglu_nv4(dg):
+    rng = np.random.default_rng(6)
+    counts, F, K = [20, 0, 64, 7], 512, 1024
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    cg, sg, gg, wg = _nv4(rng, 4, F, K)
+    cu, su, gu, wu = _nv4(rng, 4, F, K)
+    x, hi, lo = _bf16_pair(rng, int(off[-1]), K)
+    out_lo = torch.zeros(int(off[-1]), F, dtype=torch.bfloat16, device="cuda")
+    out = _run_nv4(dg, cg, sg, gg, hi, F, X_lo=lo, group_off=torch.from_numpy(off).cuda(), c2=cu, sc2=su, g2=gu,
+                   out_lo=out_lo)
+    got = out.double().cpu().numpy() + out_lo.double().cpu().numpy()
+    for e in range(4):
+        xe = x[off[e]:off[e + 1]]
+        if len(xe):
+            ref = O.silu(xe @ wg[e].T) * (xe @ wu[e].T)
+            assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-4, e
