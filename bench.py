@@ -274,11 +274,13 @@ def run_variant(args, cfg, name):
     world, rank = ranks.world, ranks.rank
     from block_diffusion_lm_masked_b200 import dg
 
-    B, mx8 = args.canvases, args.experts == "mx8"
+    B, lowp = args.canvases, args.experts
     P, C, V, k = cfg["prefix"], cfg["canvas"], cfg["vocab"], cfg["top_k"]
     model = dg.Model(synth.Model(cfg), dev)
-    if mx8:
+    if lowp == "mx8":
         model.set_experts_mx8(synth.mx8_experts(cfg))
+    elif lowp == "nv4":
+        model.set_experts_nv4(synth.nv4_experts(cfg))
     caches = []
     for b in range(B):
         c = dg.KVCache(cfg, ((P + C + 7) // 8) * 8, dev)
@@ -358,7 +360,7 @@ def run_variant(args, cfg, name):
     dg.device_status(ws)
 
     hbm, tf_burst, _, peak_src = _peaks()
-    ew = RF.MX8_WBYTES if mx8 else None
+    ew = {"mx8": RF.MX8_WBYTES, "nv4": RF.NV4_WBYTES}.get(lowp)
     flops = B * RF.pass_flops(cfg, P, C)
     nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew) + B * RF.update_bytes(cfg, C)
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
@@ -368,7 +370,8 @@ def run_variant(args, cfg, name):
     if gu:
         per_launch = RF.gate_up_bytes(cfg, unions_h[0], B * C * k, ew)
         achieved = per_launch / (gu["avg_us"] * 1e-6) / 1e9
-        roof = {"kernel": "gemm_gate_up" + ("_mx8" if mx8 else ""), "bound": "hbm", "achieved": achieved,
+        roof = {"kernel": "gemm_gate_up" + ("" if lowp == "bf16" else "_" + lowp), "bound": "hbm",
+                "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
                 "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": per_launch}
     line = {
@@ -376,7 +379,8 @@ def run_variant(args, cfg, name):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": _workload_desc(name, cfg), "canvases_per_pass": B,
-                   "experts": "mx8 (E4M3 + E8M0 per 32, synthetic codes)" if mx8 else "bf16",
+                   "experts": {"bf16": "bf16", "mx8": "mx8 (E4M3 + E8M0 per 32, synthetic codes)",
+                               "nv4": "nv4 (E2M1 + E4M3 per 16 + fp32 tensor scale, synthetic codes)"}[lowp],
                    "l2": "flushed between steps (256 MB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "expert_union": unions_h},
         "roofline": roof,
@@ -404,8 +408,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per pass (each its own request and cache) through the batched calls")
-    ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8"],
-                    help="expert weight storage; mx8 runs through the batched calls")
+    ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8", "nv4"],
+                    help="expert weight storage; mx8 and nv4 run through the batched calls")
     args = ap.parse_args()
     name = args.workload
     cfg = CF.CONFIGS[name]

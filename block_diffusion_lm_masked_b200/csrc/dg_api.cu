@@ -204,9 +204,12 @@ static dg_status map_weights(CUtensorMap* m, const void* base, uint64_t groups, 
 struct LayerMaps {
   CUtensorMap qkv, o, gate, up, down;
 };
-// 8-bit experts of one layer: codes and block scales of gate, up and down
+// low-precision experts of one layer: codes and block scales of gate, up and down, the
+// format (dg::FMT_MX8 / dg::FMT_NV4) and the 4-bit tensor scales
 struct Mx8Maps {
   CUtensorMap gate, gate_s, up, up_s, down, down_s;
+  int fmt;
+  float g_gate, g_up, g_down;
 };
 struct dg_model {
   dg_config cfg;
@@ -215,7 +218,7 @@ struct dg_model {
   std::vector<dg_layer_weights> layers;
   std::vector<LayerMaps> maps;
   CUtensorMap out_map;
-  std::vector<Mx8Maps> mx8;  // non-empty: the batched calls run the experts from 8-bit weights
+  std::vector<Mx8Maps> mx8;  // non-empty: the batched calls run the experts from low-precision weights
   bool taps_on = false;
   std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
   std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
@@ -455,8 +458,10 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   return DG_OK;
 }
 
-// a grouped expert GEMM over 8-bit weights (A, S: codes and scales; A2, S2 for gate / up)
-dg_status gemm_mx8(const GemmCall& g, const CUtensorMap* S, const CUtensorMap* S2, int* err, cudaStream_t st) {
+// a grouped expert GEMM over low-precision weights (A, S: codes and scales; A2, S2 for gate
+// / up; g_a, g_a2: the 4-bit tensor scales)
+dg_status gemm_mx8(const GemmCall& g, int fmt, const CUtensorMap* S, const CUtensorMap* S2, float g_a, float g_a2,
+                   int* err, cudaStream_t st) {
   CUtensorMap B, B2, Bb, B2b;
   dg_status s;
   if ((s = map_rows(&B, g.X, (uint64_t)g.x_rows, (uint64_t)g.K, 16)) != DG_OK) return s;
@@ -485,8 +490,8 @@ dg_status gemm_mx8(const GemmCall& g, const CUtensorMap* S, const CUtensorMap* S
   p.smem_budget = g.smem_budget;
   p.err = err;
   LAUNCH(g.kind, st,
-         dg::launch_tc_gemm_lowp(dg::FMT_MX8, g.epi, *g.A, g.A2 ? *g.A2 : *g.A, *S, S2 ? *S2 : *S, B, B2, Bb, B2b,
-                                 p, 1.0f, 1.0f, g.max_items * p.m_tiles, st));
+         dg::launch_tc_gemm_lowp(fmt, g.epi, *g.A, g.A2 ? *g.A2 : *g.A, *S, S2 ? *S2 : *S, B, B2, Bb, B2b, p, g_a,
+                                 g_a2, g.max_items * p.m_tiles, st));
   return DG_OK;
 }
 
@@ -832,11 +837,11 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
     GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &X8.gate, &X8.up, ws.at<void>(ws.L.xs), xs_lo, n * k, H, F,
                 items, n_items, max_items, kItemRowsMx8, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
                 kSmemGemm};
-    if ((s = gemm_mx8(gu, &X8.gate_s, &X8.up_s, err, st)) != DG_OK) return s;
+    if ((s = gemm_mx8(gu, X8.fmt, &X8.gate_s, &X8.up_s, X8.g_gate, X8.g_up, err, st)) != DG_OK) return s;
     GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &X8.down, nullptr, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo),
                 n * k, F, H, items, n_items, max_items, kItemRowsMx8, ws.at<float>(ws.L.ys), nullptr, H, 1, 0,
                 kSmemGemm};
-    if ((s = gemm_mx8(dn, &X8.down_s, nullptr, err, st)) != DG_OK) return s;
+    if ((s = gemm_mx8(dn, X8.fmt, &X8.down_s, nullptr, X8.g_down, 1.0f, err, st)) != DG_OK) return s;
   } else if (bf) {
     const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
     const int* n_items = ws.at<int>(ws.L.n_items);
@@ -1162,20 +1167,23 @@ extern "C" dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int3
   return DG_OK;
 }
 
-extern "C" dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* layers) {
+static dg_status set_experts_lowp(dg_model* m, int fmt, const dg_expert_weights_mx8* layers, const float* g3) {
   DG_CHECK_ARG(m, "model is NULL");
   if (!layers) {
     m->mx8.clear();
     return DG_OK;
   }
   const dg_config& c = m->cfg;
-  DG_CHECK_ARG(is_bf16(c), "8-bit experts need a bf16 model");
+  DG_CHECK_ARG(is_bf16(c), "low-precision experts need a bf16 model");
   auto a16 = [](const void* q) { return q && (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_expert_weights_mx8& X = layers[l];
     DG_CHECK_ARG(a16(X.gate) && a16(X.gate_scales) && a16(X.up) && a16(X.up_scales) && a16(X.down) &&
                      a16(X.down_scales),
-                 "layer %d: 8-bit expert pointers must be non-NULL and 16-byte aligned", l);
+                 "layer %d: expert pointers must be non-NULL and 16-byte aligned", l);
+    if (g3)
+      DG_CHECK_ARG(isfinite(g3[3 * l]) && isfinite(g3[3 * l + 1]) && isfinite(g3[3 * l + 2]),
+                   "layer %d: tensor scales must be finite", l);
   }
   std::vector<Mx8Maps> maps;
   try {
@@ -1184,18 +1192,33 @@ extern "C" dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weigh
     return fail(DG_ERR_CUDA, "out of host memory");
   }
   const uint64_t E = c.n_experts, F = c.expert_ffn, H = c.hidden;
+  auto codes = fmt == dg::FMT_NV4 ? map_codes4 : map_codes;
+  auto scales = fmt == dg::FMT_NV4 ? map_scales4 : map_scales;
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_expert_weights_mx8& X = layers[l];
     Mx8Maps& M = maps[l];
     dg_status s;
-    if ((s = map_codes(&M.gate, X.gate, E, F, H)) != DG_OK || (s = map_scales(&M.gate_s, X.gate_scales, E, F, H)) != DG_OK ||
-        (s = map_codes(&M.up, X.up, E, F, H)) != DG_OK || (s = map_scales(&M.up_s, X.up_scales, E, F, H)) != DG_OK ||
-        (s = map_codes(&M.down, X.down, E, H, F)) != DG_OK ||
-        (s = map_scales(&M.down_s, X.down_scales, E, H, F)) != DG_OK)
+    if ((s = codes(&M.gate, X.gate, E, F, H)) != DG_OK || (s = scales(&M.gate_s, X.gate_scales, E, F, H)) != DG_OK ||
+        (s = codes(&M.up, X.up, E, F, H)) != DG_OK || (s = scales(&M.up_s, X.up_scales, E, F, H)) != DG_OK ||
+        (s = codes(&M.down, X.down, E, H, F)) != DG_OK || (s = scales(&M.down_s, X.down_scales, E, H, F)) != DG_OK)
       return s;
+    M.fmt = fmt;
+    M.g_gate = g3 ? g3[3 * l] : 1.0f;
+    M.g_up = g3 ? g3[3 * l + 1] : 1.0f;
+    M.g_down = g3 ? g3[3 * l + 2] : 1.0f;
   }
   m->mx8.swap(maps);
   return DG_OK;
+}
+
+extern "C" dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* layers) {
+  return set_experts_lowp(m, dg::FMT_MX8, layers, nullptr);
+}
+
+extern "C" dg_status dg_model_set_experts_nv4(dg_model* m, const dg_expert_weights_mx8* layers,
+                                              const float* tensor_scales) {
+  DG_CHECK_ARG(!layers || tensor_scales, "4-bit experts need their tensor scales");
+  return set_experts_lowp(m, dg::FMT_NV4, layers, tensor_scales);
 }
 
 extern "C" dg_status dg_device_status(void* d_ws, dg_stream stream) {

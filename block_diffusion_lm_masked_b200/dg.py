@@ -86,6 +86,7 @@ def _load():
         "dg_denoise_pass_batched": (I32, [P, P, I32, P, I32, P, P, SZ, P]),
         "dg_generate_canvases": (I32, [P, P, I32, P, I32, I32, F32, F32, P, I32, P, P, SZ, P]),
         "dg_model_set_experts_mx8": (I32, [P, P]),
+        "dg_model_set_experts_nv4": (I32, [P, P, P]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
         "dg_set_taps": (I32, [P, ctypes.POINTER(Taps)]),
@@ -194,6 +195,30 @@ class Model:
             structs.append(ExpertsMx8(*ptrs))
         arr = (ExpertsMx8 * len(structs))(*structs)
         _check(lib.dg_model_set_experts_mx8(self.handle, arr))
+        self._mx8 = keep
+
+    def set_experts_nv4(self, layers: list | None):
+        """layers: per layer dict(gate=(codes, scale_codes, g), up=..., down=...) with codes
+        uint8 [E][rows][K] (one 4-bit code per byte), E4M3 block-scale codes
+        [E][rows][K / 16] and the tensor scale g; None returns to the bf16 experts."""
+        if layers is None:
+            _check(lib.dg_model_set_experts_nv4(self.handle, None, None))
+            self._mx8 = None
+            return
+        dev, keep, structs, gs = self.device, [], [], []
+        for L in layers:
+            ptrs = []
+            for name in ("gate", "up", "down"):
+                codes, sc, g = L[name]
+                c = torch.from_numpy(pack_nv4_codes(codes)).to(dev)
+                s_ = torch.from_numpy(pack_nv4_scales(sc)).to(dev)
+                keep += [c, s_]
+                ptrs += [c.data_ptr(), s_.data_ptr()]
+                gs.append(float(g))
+            structs.append(ExpertsMx8(*ptrs))
+        arr = (ExpertsMx8 * len(structs))(*structs)
+        g_arr = (ctypes.c_float * len(gs))(*gs)
+        _check(lib.dg_model_set_experts_nv4(self.handle, arr, g_arr))
         self._mx8 = keep
 
     def set_taps(self, taps: dict | None):

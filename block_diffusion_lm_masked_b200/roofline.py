@@ -29,6 +29,8 @@ def layer_attn_weight_bytes(cfg: dict) -> int:
 
 # bytes per expert weight of the 8-bit format: one E4M3 code plus one E8M0 scale per 32
 MX8_WBYTES = 1.0 + 1.0 / 32.0
+# and of the 4-bit format: half a byte per E2M1 code plus one E4M3 scale per 16
+NV4_WBYTES = 0.5 + 1.0 / 16.0
 
 
 def expert_bytes(cfg: dict, union: int, ew: float | None = None) -> float:

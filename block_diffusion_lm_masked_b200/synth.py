@@ -118,7 +118,7 @@ def tid_canvas_noise(canvas_index: int) -> int:
 
 def tid_layer(layer: int, j: int) -> int:
     """j: 0 w_q, 1 w_k, 2 w_v, 3 w_o, 4 w_router, 5 w_gate, 6 w_up, 7 w_down, 8 cache K, 9 cache V,
-    10-12 8-bit gate / up / down codes"""
+    10-12 8-bit gate / up / down codes, 13-15 4-bit gate / up / down codes"""
     return 1024 + 16 * layer + j
 
 
@@ -184,6 +184,25 @@ def mx8_experts(cfg: dict, seed: int = SEED_WEIGHTS):
         for j, (name, shape) in enumerate((("gate", (E, F, H)), ("up", (E, F, H)), ("down", (E, H, F)))):
             codes = _codes8(seed, tid_layer(l, 10 + j), shape, 0x70)
             d[name] = (codes, np.full(shape[:-1] + (shape[-1] // 32,), -12, dtype=np.int32))
+        out.append(d)
+    return out
+
+
+def nv4_experts(cfg: dict, seed: int = SEED_WEIGHTS):
+    """Synthetic 4-bit expert weights drawn directly as NVFP4-style data (random nibbles, no
+    quantiser): per layer dict(gate=(codes, scale_codes, g), up=..., down=...) with one
+    uniformly random E2M1 code per byte [E][F][H] (down [E][H][F]), every E4M3 block
+    scale 0.25 (code 0x28, one per 16 elements) and tensor scale 2^-6, so weights are
+    E2M1 values times 2^-8 (magnitudes up to about 0.023)."""
+    E, F, H = cfg["n_experts"], cfg["expert_ffn"], cfg["hidden"]
+    out = []
+    for l in range(cfg["n_layers"]):
+        d = {}
+        for j, (name, shape) in enumerate((("gate", (E, F, H)), ("up", (E, F, H)), ("down", (E, H, F)))):
+            b = _codes8(seed, tid_layer(l, 13 + j), shape, 8)  # sign in bit 7 over a magnitude in [0, 8)
+            codes = ((b >> 4) & 0x8) | (b & 0x7)
+            d[name] = (codes.astype(np.uint8), np.full(shape[:-1] + (shape[-1] // 16,), 0x28, dtype=np.uint8),
+                       2.0 ** -6)
         out.append(d)
     return out
 

@@ -218,6 +218,15 @@ typedef struct dg_expert_weights_mx8 {
  * dg_generate_canvases; B = 1 is one canvas); the single-canvas calls keep the bf16
  * experts. */
 dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* layers);
+/* The same with 4-bit expert weights (E2M1 codes two per byte with one E4M3 scale per 16
+ * consecutive K elements and an fp32 scale per weight tensor; see dg_debug_gemm_nv4 in
+ * dg_debug.h for the byte layouts).  Per layer, in the same struct:
+ *   gate, up     codes [E][F][H / 2],  scales [E][H / 64][F][4]
+ *   down         codes [E][H][F / 2],  scales [E][F / 64][H][4]
+ * tensor_scales: host array [n_layers][3] (gate, up, down), finite.  Each weight is
+ * e2m1(code) * e4m3(block scale) * tensor scale; the expert weight stream is about a
+ * quarter of bf16's. */
+dg_status dg_model_set_experts_nv4(dg_model* m, const dg_expert_weights_mx8* layers, const float* tensor_scales);
 
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);

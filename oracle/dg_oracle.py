@@ -696,6 +696,22 @@ def e2m1_encode(x: float) -> int:
     return c | (0x8 if neg else 0)
 
 
+def e2m1_encode_array(x) -> np.ndarray:
+    """e2m1_encode element by element on an array (nearest code, ties to the even code,
+    saturation at 6), as uint8 codes."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 6.0)
+    i = np.searchsorted(_E2M1_POS, a)
+    hit = _E2M1_POS[i] == a
+    lo = np.maximum(i - 1, 0)
+    dlo, dhi = a - _E2M1_POS[lo], _E2M1_POS[i] - a
+    c = np.where(hit, i, np.where((dlo < dhi) | ((dlo == dhi) & (lo % 2 == 0)), lo, i))
+    return (c | np.where(np.signbit(x), 0x8, 0)).astype(np.uint8)
+
+
+_E2M1_ALL = np.array([e2m1_decode(c) for c in range(16)])
+
+
 def nvfp4_quantize(w: np.ndarray, block: int = 16):
     """Two-level scaling along the last axis: a tensor scale g = max |w| / (448 * 6); per
     block of `block` values an E4M3 scale code for max |v| / (6 g); each value stored as
@@ -707,15 +723,15 @@ def nvfp4_quantize(w: np.ndarray, block: int = 16):
     g = amax_t / (E4M3_MAX * 6.0) if amax_t > 0 else 1.0
     blocks = w.reshape(*w.shape[:-1], w.shape[-1] // block, block)
     amax = np.abs(blocks).max(axis=-1)
-    sc = np.vectorize(e4m3_encode, otypes=[np.uint8])(amax / (6.0 * g))
-    sb = np.vectorize(e4m3_decode, otypes=[np.float64])(sc)
+    sc = e4m3_encode_array(amax / (6.0 * g))
+    sb = _E4M3_ALL[sc.astype(np.int64)]
     denom = np.where(sb > 0, sb * g, 1.0)[..., None]
-    codes = np.vectorize(e2m1_encode, otypes=[np.uint8])(blocks / denom)
+    codes = e2m1_encode_array(blocks / denom)
     return codes.reshape(w.shape), sc, g
 
 
 def nvfp4_dequantize(codes: np.ndarray, scale_codes: np.ndarray, g: float, block: int = 16) -> np.ndarray:
-    vals = np.vectorize(e2m1_decode, otypes=[np.float64])(np.asarray(codes))
-    sb = np.vectorize(e4m3_decode, otypes=[np.float64])(np.asarray(scale_codes))
+    vals = _E2M1_ALL[np.asarray(codes, dtype=np.int64)]
+    sb = _E4M3_ALL[np.asarray(scale_codes, dtype=np.int64)]
     blocks = vals.reshape(*vals.shape[:-1], vals.shape[-1] // block, block)
     return (blocks * (sb * g)[..., None]).reshape(vals.shape)

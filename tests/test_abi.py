@@ -289,3 +289,19 @@ def test_nv4_gemm_validation_on_host():
                dict(K=96), dict(rows=12)):
         assert call(**kw) == dg.DG_ERR_INVALID_ARG, kw
     assert L.dg_launch_count() == launches
+
+
+def test_set_experts_nv4_validation_on_host():
+    cfg = CF.CONFIGS["tiny_fp32"]
+    st, h = _fake_model(cfg)
+    assert st == dg.DG_OK
+    try:
+        L = cfg["n_layers"]
+        good = (dg.ExpertsMx8 * L)(*[dg.ExpertsMx8(*[(1 << 28) + (l << 20) + (i << 16) for i in range(6)])
+                                     for l in range(L)])
+        gs = (ctypes.c_float * (3 * L))(*([0.01] * (3 * L)))
+        assert dg.lib.dg_model_set_experts_nv4(h, good, None) == dg.DG_ERR_INVALID_ARG       # no tensor scales
+        assert dg.lib.dg_model_set_experts_nv4(h, good, gs) == dg.DG_ERR_INVALID_ARG         # fp32 model
+        assert dg.lib.dg_model_set_experts_nv4(h, None, None) == dg.DG_OK
+    finally:
+        dg.lib.dg_model_destroy(h)

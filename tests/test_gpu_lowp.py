@@ -218,3 +218,27 @@ def test_gate_up_swiglu_nv4(dg):
         if len(xe):
             ref = O.silu(xe @ wg[e].T) * (xe @ wu[e].T)
             assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-4, e
+
+
+def _experts_to_nv4(setup):
+    """Quantise the model's bf16 experts with the oracle's NVFP4 quantiser (one tensor
+    scale per expert tensor of a layer): codes to the GPU model, decoded weights to the
+    oracle model."""
+    layers = []
+    for L in setup.host.layers:
+        d = {}
+        for name, key in (("gate", "w_gate"), ("up", "w_up"), ("down", "w_down")):
+            codes, sc, g = O.nvfp4_quantize(O.widen(L[key]))
+            d[name] = (codes, sc, g)
+            L[key] = O.nvfp4_dequantize(codes, sc, g)
+        layers.append(d)
+    setup.model.set_experts_nv4(layers)
+
+
+@pytest.mark.parametrize("cfg,prefixes,C", [(SMALL_BF16, [200], 100), (SMALL_BF16, [64, 0, 131], 37),
+                                            (CF.CONFIGS["layer1_bf16"], [1024], 256)])
+def test_pass_with_nv4_experts_matches_oracle(dg, cfg, prefixes, C):
+    """The pass with 4-bit experts against the oracle pass over the decoded weights (the
+    tensor scale applied once to the accumulator on the GPU, to every weight in the oracle:
+    rounding differences only)."""
+    PL.check_batched_pass(dg, cfg, prefixes, C, prepare=_experts_to_nv4)

@@ -347,6 +347,17 @@ def _e2m1_encode_ties_up(x):
     return c | (0x8 if neg else 0)
 
 
+def _array_ties_away(table, top, sign_bit):
+    def enc(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.minimum(np.abs(x), top)
+        i = np.searchsorted(table, a)
+        lo = np.maximum(i - 1, 0)
+        c = np.where(table[i] == a, i, np.where(a - table[lo] < table[i] - a, lo, i))
+        return (c | np.where(np.signbit(x), sign_bit, 0)).astype(np.uint8)
+    return enc
+
+
 def _widen_shift8(a):
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << np.uint32(8)).view(np.float32).astype(np.float64)
@@ -446,6 +457,10 @@ MUTANTS = {
     "e2m1 subnormal value": ("e2m1_decode", _e2m1_subnormal, ["test_e2m1_codes_rounding_saturation"]),
     "e2m1 ties away from even": ("e2m1_encode", _e2m1_encode_ties_up, ["test_e2m1_codes_rounding_saturation"]),
     "nvfp4 tensor scale without the 6": ("nvfp4_quantize", _nvfp4_no_six, ["test_nvfp4_block_scaling"]),
+    "array e4m3 encoder ties away from even": ("e4m3_encode_array", _array_ties_away(O._E4M3_POS, 448.0, 0x80),
+                                               ["test_e4m3_array_encoder_is_the_scalar_rule"]),
+    "array e2m1 encoder ties away from even": ("e2m1_encode_array", _array_ties_away(O._E2M1_POS, 6.0, 0x8),
+                                               ["test_e2m1_array_encoder_is_the_scalar_rule"]),
 }
 
 

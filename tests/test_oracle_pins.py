@@ -695,6 +695,18 @@ def test_e2m1_codes_rounding_saturation():
     assert enc(2.4) == 4 and enc(5.1) == 7 and enc(100.0) == 7 and enc(-100.0) == 0xF
 
 
+def test_e2m1_array_encoder_is_the_scalar_rule():
+    pos = np.array([O.e2m1_decode(c) for c in range(8)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(43)
+    xs = np.concatenate([pos, mids, np.nextafter(mids, 0), np.nextafter(mids, 9), [6.0, 6.5, 7.0, 100.0], [0.0, -0.0],
+                         rng.standard_normal(3000) * 3])
+    xs = np.concatenate([xs, -xs])
+    got = O.e2m1_encode_array(xs)
+    assert got.dtype == np.uint8
+    assert list(got) == [O.e2m1_encode(v) for v in xs]
+
+
 def test_nvfp4_block_scaling():
     rng = np.random.default_rng(43)
     w = rng.standard_normal((4, 64)) * np.array([0.01, 0.2, 1.0, 5.0])[:, None]

@@ -45,3 +45,15 @@ def test_mx8_experts_are_valid_deterministic_codes(monkeypatch):
         assert mag.max() == 0x6F and 0.4 < (codes >> 7).mean() < 0.6
         assert exps.shape == shape[:-1] + (shape[-1] // 32,) and (exps == -12).all()
     assert (a[0]["gate"][0] != a[0]["up"][0]).mean() > 0.9
+
+
+def test_nv4_experts_are_uniform_4bit_codes():
+    cfg = dict(n_layers=1, hidden=128, n_experts=2, expert_ffn=64)
+    a = synth.nv4_experts(cfg)
+    for name, shape in (("gate", (2, 64, 128)), ("up", (2, 64, 128)), ("down", (2, 128, 64))):
+        codes, sc, g = a[0][name]
+        assert codes.shape == shape and codes.dtype == np.uint8 and codes.max() < 16
+        cnt = np.bincount(codes.ravel(), minlength=16)
+        assert cnt.min() > 0.8 * codes.size / 16 and cnt.max() < 1.2 * codes.size / 16
+        assert sc.shape == shape[:-1] + (shape[-1] // 16,) and (sc == 0x28).all() and g == 2.0 ** -6
+    np.testing.assert_array_equal(a[0]["gate"][0], synth.nv4_experts(cfg)[0]["gate"][0])
