@@ -1221,6 +1221,42 @@ extern "C" dg_status dg_model_set_experts_nv4(dg_model* m, const dg_expert_weigh
   return set_experts_lowp(m, dg::FMT_NV4, layers, tensor_scales);
 }
 
+extern "C" dg_status dg_generate_canvases_masked(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases,
+                                                 int32_t C, int32_t S, float keep_start, float keep_end,
+                                                 int32_t mask_id, int32_t append, float* d_logits, void* d_ws,
+                                                 size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  DG_CHECK_ARG(S >= 1, "S must be >= 1");
+  DG_CHECK_ARG(keep_start >= 0.f && keep_start <= 1.f && keep_end >= 0.f && keep_end <= 1.f,
+               "keep fractions must be in [0,1]");
+  DG_CHECK_ARG(mask_id >= 0 && mask_id < m->cfg.vocab, "mask_id must be in [0, vocab)");
+  DG_CHECK_ARG(d_canvases && d_logits, "canvases / logits is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(B >= 1 && (int64_t)B * C <= (1 << 20), "B must be >= 1 and B * C <= 2^20");
+  DG_CHECK_ARG((reinterpret_cast<uintptr_t>(d_logits) & 15) == 0, "logits must be 16-byte aligned");
+  dg_status s = check_caches(m->cfg, caches, B, C);
+  if (s != DG_OK) return s;
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, B * C, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int V = m->cfg.vocab, n = B * C;
+  const int splits = dg::update_splits(n, V);
+  dg::UpdPart* part = ws.at<dg::UpdPart>(ws.L.upd);
+  LAUNCH(DG_K_UPDATE_SELECT, st, dg::launch_fill_i32(d_canvases, n, mask_id, st));
+  for (int step = 0; step < S; ++step) {
+    if ((s = dg_denoise_pass_batched(m, caches, B, d_canvases, C, d_logits, d_ws, ws_bytes, stream)) != DG_OK)
+      return s;
+    const int nk = renoise_count(C, S, step, keep_start, keep_end);
+    LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_update_partial(d_logits, n, V, splits, mask_id, part, st));
+    for (int b = 0; b < B; ++b)
+      LAUNCH(DG_K_UPDATE_SELECT, st,
+             dg::launch_update_select(part + (size_t)b * C * splits, C, V, splits, nk, 0, 0,
+                                      d_canvases + (size_t)b * C, nullptr, mask_id, st));
+  }
+  if (append) return dg_prefill_append_batched(m, caches, B, d_canvases, C, d_ws, ws_bytes, stream);
+  return DG_OK;
+}
+
 extern "C" dg_status dg_device_status(void* d_ws, dg_stream stream) {
   DG_CHECK_ARG(d_ws, "workspace is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

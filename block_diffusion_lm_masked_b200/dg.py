@@ -85,6 +85,7 @@ def _load():
         "dg_prefill_append_batched": (I32, [P, P, I32, P, I32, P, SZ, P]),
         "dg_denoise_pass_batched": (I32, [P, P, I32, P, I32, P, P, SZ, P]),
         "dg_generate_canvases": (I32, [P, P, I32, P, I32, I32, F32, F32, P, I32, P, P, SZ, P]),
+        "dg_generate_canvases_masked": (I32, [P, P, I32, P, I32, I32, F32, F32, I32, I32, P, P, SZ, P]),
         "dg_model_set_experts_mx8": (I32, [P, P]),
         "dg_model_set_experts_nv4": (I32, [P, P, P]),
         "dg_device_status": (I32, [P, P]),
@@ -392,6 +393,18 @@ def generate_canvases(model: Model, caches: list, canvases: torch.Tensor, S: int
     sd = (ctypes.c_uint64 * B)(*[int(x) & 0xFFFFFFFFFFFFFFFF for x in seeds])
     _check(lib.dg_generate_canvases(model.handle, arr, B, _ptr(canvases), C, S, r_start, r_end, sd,
                                     1 if append else 0, _ptr(logits), ws.ptr, ws.nbytes, _stream(stream)))
+    for c, s in zip(caches, arr):
+        c.len = s.len
+
+
+def generate_canvases_masked(model: Model, caches: list, canvases: torch.Tensor, S: int, keep_start: float,
+                             keep_end: float, mask_id: int, append: bool, logits: torch.Tensor, ws: Workspace,
+                             stream=None):
+    """generate_canvas_masked for B canvases at once (canvases int32 [B][C], written by the call)."""
+    B, C = canvases.shape
+    arr = _caches(caches)
+    _check(lib.dg_generate_canvases_masked(model.handle, arr, B, _ptr(canvases), C, S, keep_start, keep_end, mask_id,
+                                           1 if append else 0, _ptr(logits), ws.ptr, ws.nbytes, _stream(stream)))
     for c, s in zip(caches, arr):
         c.len = s.len
 

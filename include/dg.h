@@ -194,6 +194,11 @@ dg_status dg_denoise_pass_batched(dg_model* m, const dg_kv_cache* caches, int32_
 dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases, int32_t C, int32_t S,
                                float r_start, float r_end, const uint64_t* seeds, int32_t append, float* d_logits,
                                void* d_ws, size_t ws_bytes, dg_stream stream);
+/* dg_generate_canvas_masked for B canvases at once (each from an all-mask_id canvas,
+ * written by this call into d_canvases[B][C]; the same keep schedule for all). */
+dg_status dg_generate_canvases_masked(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases, int32_t C,
+                                      int32_t S, float keep_start, float keep_end, int32_t mask_id, int32_t append,
+                                      float* d_logits, void* d_ws, size_t ws_bytes, dg_stream stream);
 
 /* 8-bit expert weights (MX-FP8 storage: E4M3 codes with one E8M0 power-of-two scale per
  * 32 consecutive K elements of a row; see dg_debug_gemm_mx8 in dg_debug.h for the byte

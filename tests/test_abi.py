@@ -200,9 +200,12 @@ def test_batched_calls_reject_bad_arguments_before_any_launch():
         def gen(caches=good, B=B, C=C, ws_bytes=ws_need, logits=p, sd=seeds):
             return lib.dg_generate_canvases(h, caches, B, p, C, 2, 0.5, 0.0, sd, 1, logits, ws, ws_bytes, None)
 
+        def genm(caches=good, B=B, C=C, ws_bytes=ws_need, logits=p):
+            return lib.dg_generate_canvases_masked(h, caches, B, p, C, 2, 0.5, 0.0, 7, 1, logits, ws, ws_bytes, None)
+
         shared, k2 = batch({}, {"share_with": 0}, {})
         full, k3 = batch({}, {}, {"length": 60})
-        for f in (den, pre, gen):
+        for f in (den, pre, gen, genm):
             assert f(caches=None) == dg.DG_ERR_INVALID_ARG
             assert f(B=0) == dg.DG_ERR_INVALID_ARG
             assert f(C=0) == dg.DG_ERR_INVALID_ARG
@@ -212,6 +215,9 @@ def test_batched_calls_reject_bad_arguments_before_any_launch():
             assert "cache 2" in lib.dg_last_error().decode()
             assert f(ws_bytes=dg.workspace_bytes(cfg, C)) == dg.DG_ERR_CAPACITY     # sized for one canvas
         assert gen(logits=ctypes.c_void_p((1 << 24) + 8)) == dg.DG_ERR_INVALID_ARG
+        assert genm(logits=ctypes.c_void_p((1 << 24) + 8)) == dg.DG_ERR_INVALID_ARG
+        assert lib.dg_generate_canvases_masked(h, good, B, p, C, 2, 0.5, 0.0, cfg["vocab"], 1, p, ws, ws_need,
+                                               None) == dg.DG_ERR_INVALID_ARG     # mask id outside the vocabulary
         assert gen(sd=None) == dg.DG_ERR_INVALID_ARG
         assert gen(C=1025) == dg.DG_ERR_INVALID_ARG
         assert lib.dg_launch_count() == launches

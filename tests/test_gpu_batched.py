@@ -116,3 +116,24 @@ def test_generate_canvases_equals_single_generation_fp32(dg):
             np.testing.assert_allclose(ka, ks, rtol=1e-5, atol=1e-6)
             np.testing.assert_allclose(va, vs, rtol=1e-5, atol=1e-6)
     dg.device_status(ws)
+
+
+def test_generate_canvases_masked_equals_single_generation_fp32(dg):
+    """The masked batched generation against the single-canvas masked generation on the
+    fp32 model: each canvas ends fully unmasked with the tokens of its own run."""
+    cfg = CF.CONFIGS["tiny_fp32"]
+    prefixes, C, S, mask_id = [64, 0], 32, 4, cfg["vocab"] - 1
+    a = PL.BatchSetup(dg, cfg, prefixes, 256)
+    s = PL.BatchSetup(dg, cfg, prefixes, 256)
+    ws = dg.Workspace(cfg, len(prefixes) * C)
+    lb = torch.empty(len(prefixes), C, cfg["vocab"], device="cuda")
+    out = torch.empty(len(prefixes), C, dtype=torch.int32, device="cuda")
+    dg.generate_canvases_masked(a.model, a.caches, out, S, (S - 1) / S, 0.0, mask_id, True, lb, ws)
+    for b in range(len(prefixes)):
+        one = torch.empty(C, dtype=torch.int32, device="cuda")
+        ls = torch.empty(C, cfg["vocab"], device="cuda")
+        dg.generate_canvas_masked(s.model, s.caches[b], one, S, (S - 1) / S, 0.0, mask_id, True, ls, ws)
+        np.testing.assert_array_equal(out[b].cpu().numpy(), one.cpu().numpy())
+        assert not (out[b] == mask_id).any()
+        assert a.caches[b].len == s.caches[b].len == prefixes[b] + C
+    dg.device_status(ws)
