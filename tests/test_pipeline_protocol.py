@@ -45,7 +45,7 @@ class Barrier:
     def passes(self, parity, want_phase):
         """try_wait.parity: the phase in progress has parity completed % 2."""
         ok = (self.completed % 2) != parity
-        if ok:
+        if ok and want_phase is not None:
             assert self.completed <= want_phase + 1, f"{self.name}: ran past phase {want_phase}"
         return ok
 
@@ -297,3 +297,150 @@ def test_the_checker_catches_a_wrong_count():
     assert caught > 0
     for seed in range(20):       # and the kernel's count passes the same interleavings
         _lowp_with_count(9, seed)
+
+
+# ---------------------------------------------------------------- the attention kernel (k_tc_attn.cu)
+
+def attention(nck, cur_from, seed, n_warps=8):
+    """Chunks [cur_from, nck) are the call's own keys ("current": hi and lo parts, both
+    smem slots); earlier chunks are cached keys alternating the two slots."""
+    rng = random.Random(seed * 7919 + nck)
+    q_bar = Barrier("q_bar", 1)
+    kv = [Barrier(f"kv{s}", 1) for s in range(2)]
+    s_full, s_free = Barrier("s_full", 1), Barrier("s_free", n_warps)
+    p_ready = [Barrier(f"p_ready{b}", n_warps) for b in range(2)]
+    pv_done = [Barrier(f"pv_done{b}", 1) for b in range(2)]
+    x_bar = [Barrier(f"x_bar{b}", n_warps) for b in range(2)]
+    l_bar = Barrier("l_bar", n_warps)
+    bufs, q = Buffers(), Async()
+    st = dict(pv_issued=0, pv_completed=0, s_issued=0, s_completed=0)
+    p_writes, x_writes = {}, {}
+
+    def is_cur(j):
+        return j >= cur_from
+
+    def control():
+        slot_loads = [0, 0]
+        par = {}
+        issued = 0
+        pv_next = 0
+
+        def issue(j):
+            nonlocal issued
+            slots = (0, 1) if is_cur(j) else (j & 1,)
+            for s_ in slots:
+                par[(j & 1, s_)] = slot_loads[s_] & 1
+                slot_loads[s_] += 1
+                bufs.fill(("slot", s_), 2)     # read by the S MMA and the PV MMA of chunk j
+                kv[s_].arrive_expect_tx(32)
+                q.loads.append(lambda s_=s_: kv[s_].complete_tx(32))
+            issued = j + 1
+
+        def issue_pv(k):
+            assert st["pv_issued"] == k and st["s_completed"] >= k + 1
+            st["pv_issued"] += 1
+            assert p_writes.get(k & 1) == (k, n_warps), "PV read a P buffer not fully written"
+            slots = (0, 1) if is_cur(k) else (k & 1,)
+
+            def done(k=k, slots=slots):
+                st["pv_completed"] += 1
+                bufs.release(("p", k & 1))
+                for s_ in slots:
+                    bufs.release(("slot", s_))
+                pv_done[k & 1].arrive()
+            q.mma.append(done)
+
+        def do_pv(k):
+            nonlocal pv_next
+            yield wait(p_ready[k & 1], (k >> 1) & 1, k >> 1)
+            issue_pv(k)
+            pv_next = k + 1
+            yield wait(pv_done[k & 1], (k >> 1) & 1, k >> 1)
+
+        q_bar.arrive_expect_tx(16)
+        q.loads.append(lambda: q_bar.complete_tx(16))
+        issue(0)
+        if nck > 1 and not is_cur(0) and not is_cur(1):
+            issue(1)
+        for j in range(nck):
+            cur = is_cur(j)
+            s_hi = 0 if cur else (j & 1)
+            if issued <= j:
+                if j >= 1 and pv_next == j - 1:
+                    yield from do_pv(j - 1)
+                issue(j)
+            if j == 0:
+                yield wait(q_bar, 0, 0)
+            yield wait(kv[s_hi], par[(j & 1, s_hi)], None)
+            if cur:
+                yield wait(kv[1], par[(j & 1, 1)], None)
+            if j >= 1:
+                yield wait(s_free, (j - 1) & 1, j - 1)
+            bufs.fill(("S",), n_warps)
+            st["s_issued"] += 1
+
+            def s_done(j=j, cur=cur, s_hi=s_hi):
+                st["s_completed"] += 1
+                for s_ in ((0, 1) if cur else (s_hi,)):
+                    bufs.release(("slot", s_))
+                s_full.arrive()
+            q.mma.append(s_done)
+            if j >= 1 and pv_next == j - 1:
+                yield from do_pv(j - 1)
+            if issued == j + 1 and j + 1 < nck and not cur and not is_cur(j + 1):
+                issue(j + 1)
+        if pv_next == nck - 1:
+            yield wait(p_ready[(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
+            issue_pv(nck - 1)
+
+    def softmax(w):
+        for j in range(nck):
+            yield wait(s_full, j & 1, j)
+            assert st["s_completed"] == j + 1
+            bufs.release(("S",))
+            s_free.arrive()
+            # the row max exchange through x_max[j & 1]
+            last, n = x_writes.get(j & 1, (None, 0))
+            if last != j:
+                bufs.fill(("x", j & 1), n_warps)
+                x_writes[j & 1] = (j, 1)
+            else:
+                x_writes[j & 1] = (j, n + 1)
+            x_bar[j & 1].arrive()
+            yield wait(x_bar[j & 1], (j >> 1) & 1, j >> 1)
+            assert x_writes[j & 1] == (j, n_warps), "a row max read before both halves posted"
+            bufs.release(("x", j & 1))
+            if j > 0 and rng.random() < 0.5:   # some row of this warp needs O rescaled
+                yield wait(pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                assert st["pv_completed"] >= j and st["pv_issued"] <= j, "O rescaled while a PV may write it"
+            if j >= 2:
+                yield wait(pv_done[j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
+            last, n = p_writes.get(j & 1, (None, 0))
+            if last != j:
+                bufs.fill(("p", j & 1), 1)     # read by the PV of chunk j
+                p_writes[j & 1] = (j, 1)
+            else:
+                p_writes[j & 1] = (j, n + 1)
+            p_ready[j & 1].arrive()
+        yield wait(pv_done[(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
+        assert st["pv_completed"] == nck
+        l_bar.arrive()
+        yield wait(l_bar, 0, 0)
+
+    roles = {"ctrl": control()}
+    roles.update({f"sm{w}": softmax(w) for w in range(n_warps)})
+    return roles, q
+
+
+# What the simulation shows about this protocol: dropping the softmax's wait for the S
+# buffer or for a finished PV before rescaling O is caught; dropping its wait for the PV
+# two chunks back (before reusing that P buffer) is not, because the control warp waits
+# for every PV to complete before issuing the next S, which the softmax waits for first.
+# That wait is therefore redundant, and the control warp's wait is what serialises a PV's
+# completion against the next S on the tensor pipe.
+@pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (2, 1), (2, 0), (3, 3), (5, 3), (6, 0), (7, 5),
+                                          (9, 9), (12, 10)])
+def test_attention_protocol(nck, cur_from):
+    for seed in range(25):
+        roles, q = attention(nck, cur_from, seed)
+        run(roles, q, seed)
