@@ -290,13 +290,16 @@ def run_variant(args, cfg, name):
     noise = torch.from_numpy(np.stack([synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(rank * B + b), C, V)
                                        for b in range(B)]))
     canv_in = noise.to(dev)
-    canv_out = torch.empty_like(canv_in)
+    canv_out = canv_in.clone()
     logits = torch.empty(B, C, V, device=dev)
     n_ren = dg.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
     def step(s):
+        if args.fused_update:  # the canvas is the call's input and output: each step denoises the last result
+            dg.denoise_update(model, caches[0], canv_out[0], n_ren, ws, seed=synth.SEED_RENOISE, step=s)
+            return
         dg.denoise_pass_batched(model, caches, canv_in, logits, ws)
         for b in range(B):
             dg.canvas_update(logits[b], n_ren, synth.SEED_RENOISE + b, s, canv_out[b], ws)
@@ -362,7 +365,9 @@ def run_variant(args, cfg, name):
     hbm, tf_burst, _, peak_src = _peaks()
     ew = {"mx8": RF.MX8_WBYTES, "nv4": RF.NV4_WBYTES}.get(lowp)
     flops = B * RF.pass_flops(cfg, P, C)
-    nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew) + B * RF.update_bytes(cfg, C)
+    nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew) + B * 8 * C
+    if args.fused_update:  # no logits written or read back: the tile records instead
+        nbytes += 2 * 16 * C * ((V + 127) // 128) - 2 * 4 * C * V
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
     ms_step = total_ms / args.steps
     roof = None
@@ -379,6 +384,7 @@ def run_variant(args, cfg, name):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": _workload_desc(name, cfg), "canvases_per_pass": B,
+                   "update": "fused into the vocabulary projection" if args.fused_update else "two kernels on logits",
                    "experts": {"bf16": "bf16", "mx8": "mx8 (E4M3 + E8M0 per 32, synthetic codes)",
                                "nv4": "nv4 (E2M1 + E4M3 per 16 + fp32 tensor scale, synthetic codes)"}[lowp],
                    "l2": "flushed between steps (256 MB write)",
@@ -408,6 +414,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per pass (each its own request and cache) through the batched calls")
+    ap.add_argument("--fused-update", action="store_true",
+                    help="one call per step: the pass with the update's statistics as the vocabulary "
+                         "projection's epilogue (no logits)")
     ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8", "nv4"],
                     help="expert weight storage; mx8 and nv4 run through the batched calls")
     args = ap.parse_args()
@@ -417,7 +426,9 @@ def main():
         return run_reference(args, cfg, name)
     if args.canvases < 1:
         ap.error("--canvases must be >= 1")
-    if args.canvases > 1 or args.experts != "bf16":
+    if args.fused_update and (args.canvases > 1 or args.experts != "bf16"):
+        ap.error("--fused-update runs one canvas with bf16 experts")
+    if args.canvases > 1 or args.experts != "bf16" or args.fused_update:
         return run_variant(args, cfg, name)
 
     import torch
@@ -569,7 +580,9 @@ def main():
 
     # whole-pass roofline (slower of FLOPs at the bf16 peak and bytes at HBM bandwidth)
     flops = RF.pass_flops(cfg, P, C)
-    nbytes = RF.pass_bytes(cfg, P, C, unions_h) + RF.update_bytes(cfg, C)
+    # the pass's bytes already hold the logits' write and the update's read of them; the
+    # update adds its canvas in / out
+    nbytes = RF.pass_bytes(cfg, P, C, unions_h) + 8 * C
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
     # dominant kernel: the gate/up grouped GEMM, HBM-bound on the union of expert weights
     gu = kern.get("gemm_gate_up")

@@ -315,7 +315,7 @@ constexpr int kItemRowsMx8 = 64;         // the same for the 8-bit-weight expert
 
 struct WsLayout {
   size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
-      topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, total;
+      topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, vtiles, total;
   int lo_rows;  // rows of the current-token K/V low-term window
 };
 
@@ -365,6 +365,8 @@ WsLayout layout(const dg_config& c, int T) {
   L.h_lo = take(bf ? (size_t)T * k * F * 2 : 0);
   L.gu = take(bf ? 0 : (size_t)T * k * 2 * F * 4);
   L.ys = take((size_t)T * k * H * 4);
+  // the fused vocabulary/update path: one statistics record per (token, 128-id tile)
+  L.vtiles = take((size_t)(T < 1024 ? T : 1024) * ((c.vocab + 127) / 128) * sizeof(dg::UpdPart));
   L.total = o;
   return L;
 }
@@ -973,6 +975,47 @@ extern "C" dg_status dg_denoise_pass(dg_model* m, const dg_kv_cache* cache, cons
            dg::launch_simt_gemm_f32(0, (const float*)m->w_out, ws.at<float>(ws.L.xn), nullptr, 1, C, C, c.vocab,
                                     c.hidden, d_logits, c.vocab, st));
   }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_denoise_update(dg_model* m, const dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t n,
+                                       uint64_t seed, uint32_t step, int32_t mask_id, float* d_conf, void* d_ws,
+                                       size_t ws_bytes, dg_stream stream) {
+  DG_CHECK_ARG(m, "model is NULL");
+  if (!is_bf16(m->cfg)) return fail(DG_ERR_UNSUPPORTED, "the fused update runs on the tcgen05 path (bf16 models)");
+  dg_status s = check_cache(m->cfg, cache);
+  if (s != DG_OK) return s;
+  DG_CHECK_ARG(d_canvas, "canvas is NULL");
+  DG_CHECK_ARG(C > 0 && C <= 1024, "C must be in [1, 1024]");
+  DG_CHECK_ARG(n >= 0 && n <= C, "n must be in [0, C]");
+  DG_CHECK_ARG(mask_id < m->cfg.vocab, "mask_id must be < vocab (negative: the re-noising update)");
+  if ((int64_t)cache->len + C > cache->capacity)
+    return fail(DG_ERR_CAPACITY, "cache has no room for the canvas: len %d + C %d > capacity %d", cache->len, C,
+                cache->capacity);
+  Ws ws;
+  if ((s = check_ws(m->cfg, d_ws, ws_bytes, C, &ws)) != DG_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dg_config& c = m->cfg;
+  if ((s = run_stack<bf16>(m, cache, d_canvas, C, false, ws, st)) != DG_OK) return s;
+  CUtensorMap B, Bb;
+  if ((s = map_rows(&B, ws.at<void>(ws.L.xn), (uint64_t)C, (uint64_t)c.hidden, 16)) != DG_OK) return s;
+  if ((s = map_rows(&Bb, ws.at<void>(ws.L.xn), (uint64_t)C, (uint64_t)c.hidden, 64)) != DG_OK) return s;
+  dg::VuParams p{};
+  p.K = c.hidden;
+  p.V = c.vocab;
+  p.m_tiles = ceil_div(c.vocab, 128);
+  p.n_max = C < 256 ? ((C + 15) & ~15) : 256;
+  p.n_tokens = C;
+  p.excl = mask_id < 0 ? -1 : mask_id;
+  p.part = ws.at<dg::UpdPart>(ws.L.vtiles);
+  p.smem_budget = kSmemGemm;
+  p.err = ws.err();
+  dg::UpdPart* rows = ws.at<dg::UpdPart>(ws.L.upd);
+  LAUNCH(DG_K_GEMM_VOCAB, st, dg::launch_vocab_update(m->out_map, B, Bb, p, st));
+  LAUNCH(DG_K_UPDATE_PARTIAL, st, dg::launch_upd_merge_rows(p.part, C, p.m_tiles, rows, st));
+  LAUNCH(DG_K_UPDATE_SELECT, st,
+         dg::launch_update_select(rows, C, c.vocab, 1, n, seed, step, d_canvas, d_conf, mask_id < 0 ? -1 : mask_id,
+                                  st));
   return DG_OK;
 }
 

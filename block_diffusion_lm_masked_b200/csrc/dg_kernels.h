@@ -136,6 +136,26 @@ struct UpdPart {
   float m2;   // that logit (the ids other than an excluded one; m when nothing is excluded)
 };
 int update_splits(int C, int V);
+
+// The vocabulary projection with the update's statistics as its epilogue (no logits):
+// part[token][tile] for tokens [0, n_tokens) and 128-id tiles [0, m_tiles) of the output
+// matrix (A: 3-D map (K, V, 1), box 64 x 128 x 1; B / Bb: the final normed state, 2-D maps
+// with 16- and 64-row boxes); excl >= 0 makes every record's candidate skip that id.
+struct VuParams {
+  int K;            // hidden size
+  int V;            // vocabulary
+  int m_tiles;      // ceil(V / 128)
+  int n_max;        // tokens per tile, multiple of 16, <= 256
+  int n_tokens;
+  int excl;
+  UpdPart* part;    // [n_tokens][m_tiles]
+  int smem_budget;
+  int* err;
+};
+cudaError_t launch_vocab_update(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& Bb, const VuParams& p,
+                                cudaStream_t st);
+// each token's tile records merged in id order into out[token]
+cudaError_t launch_upd_merge_rows(const UpdPart* part, int C, int tiles, UpdPart* out, cudaStream_t st);
 // excl >= 0: the candidate skips that id
 cudaError_t launch_update_partial(const float* logits, int C, int V, int splits, int excl, UpdPart* part,
                                   cudaStream_t st);

@@ -77,6 +77,7 @@ def _load():
         "dg_prefill_append": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, SZ, P]),
         "dg_denoise_pass": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, P, P, SZ, P]),
         "dg_canvas_update": (I32, [P, I32, I32, I32, U64, U32, P, P, P, SZ, P]),
+        "dg_denoise_update": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, U64, U32, I32, P, P, SZ, P]),
         "dg_canvas_update_noalloc": (I32, [P, I32, I32, I32, U64, U32, P, P, P]),
         "dg_canvas_update_masked": (I32, [P, I32, I32, I32, I32, P, P, P, SZ, P]),
         "dg_generate_canvas_masked": (I32, [P, ctypes.POINTER(KVCacheS), P, I32, I32, F32, F32, I32, I32, P, P, SZ,
@@ -319,6 +320,14 @@ def denoise_pass(model: Model, cache: KVCache, canvas: torch.Tensor, logits: tor
                  stream=None):
     _check(lib.dg_denoise_pass(model.handle, ctypes.byref(cache.s), _ptr(canvas), canvas.numel(), _ptr(logits),
                                ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def denoise_update(model: Model, cache: KVCache, canvas: torch.Tensor, n: int, ws: Workspace, seed: int = 0,
+                   step: int = 0, mask_id: int = -1, conf: torch.Tensor | None = None, stream=None):
+    """One pass and its update without logits (include/dg.h); canvas int32 [C] in/out."""
+    _check(lib.dg_denoise_update(model.handle, ctypes.byref(cache.s), _ptr(canvas), canvas.numel(), n,
+                                 seed & 0xFFFFFFFFFFFFFFFF, step, mask_id, _ptr(conf), ws.ptr, ws.nbytes,
+                                 _stream(stream)))
 
 
 def canvas_update(logits: torch.Tensor, n_renoise: int, seed: int, step: int, canvas: torch.Tensor, ws,

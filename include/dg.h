@@ -139,6 +139,19 @@ dg_status dg_canvas_update(const float* d_logits, int32_t C, int32_t V, int32_t 
                            uint32_t step, int32_t* d_canvas, float* d_conf, void* d_ws, size_t ws_bytes,
                            dg_stream stream);
 
+/* One denoising pass and its canvas update without materialising the logits (bf16
+ * models; DG_ERR_UNSUPPORTED for fp32): the vocabulary projection's epilogue emits the
+ * update's statistics per (token, 128-id tile) -- the largest logit, the sum of exp(l -
+ * max), the candidate id and its logit -- which are merged per token in id order and
+ * selected as dg_canvas_update (mask_id < 0: n = n_renoise, with seed and step) or
+ * dg_canvas_update_masked (mask_id >= 0: n = n_keep; seed and step unused) would on the
+ * logits.  d_canvas[C] is the pass's input and receives the update; d_conf[C] as those
+ * calls (nullable).  The 4 C V bytes of logits are neither written nor read.  Results
+ * equal the two-call path's up to fp32 summation order.  C <= 1024, 0 <= n <= C. */
+dg_status dg_denoise_update(dg_model* m, const dg_kv_cache* cache, int32_t* d_canvas, int32_t C, int32_t n,
+                            uint64_t seed, uint32_t step, int32_t mask_id, float* d_conf, void* d_ws, size_t ws_bytes,
+                            dg_stream stream);
+
 /* S denoising passes with re-noising, then (if append) the canvas is appended to the
  * cache by dg_prefill_append.  After pass s (0-based) the number of re-noised
  * positions is floor(C * f_s + 1e-9), f_s = (r_start (S-1-s) + r_end s) / (S-1)
