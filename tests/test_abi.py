@@ -311,3 +311,25 @@ def test_set_experts_nv4_validation_on_host():
         assert dg.lib.dg_model_set_experts_nv4(h, None, None) == dg.DG_OK
     finally:
         dg.lib.dg_model_destroy(h)
+
+
+def test_denoise_update_validation_on_host():
+    """dg_denoise_update: an fp32 model is unsupported (the fused epilogue is a tcgen05
+    kernel); bad sizes and a missing canvas are rejected before any launch."""
+    cfg = CF.CONFIGS["tiny_fp32"]
+    st, h = _fake_model(cfg)
+    assert st == dg.DG_OK
+    try:
+        L = cfg["n_layers"]
+        ka = (ctypes.c_void_p * L)(*[(1 << 30) + (i << 16) for i in range(L)])
+        va = (ctypes.c_void_p * L)(*[(1 << 31) + (i << 16) for i in range(L)])
+        cs = dg.KVCacheS(ka, va, 256, 64)
+        p, ws = ctypes.c_void_p(1 << 24), ctypes.c_void_p(1 << 25)
+        launches = dg.lib.dg_launch_count()
+        assert dg.lib.dg_denoise_update(h, ctypes.byref(cs), p, 32, 8, 1, 0, -1, None, ws, 1 << 30,
+                                        None) == dg.DG_ERR_UNSUPPORTED
+        assert dg.lib.dg_denoise_update(None, ctypes.byref(cs), p, 32, 8, 1, 0, -1, None, ws, 1 << 30,
+                                        None) == dg.DG_ERR_INVALID_ARG
+        assert dg.lib.dg_launch_count() == launches
+    finally:
+        dg.lib.dg_model_destroy(h)
