@@ -444,3 +444,73 @@ def test_attention_protocol(nck, cur_from):
     for seed in range(25):
         roles, q = attention(nck, cur_from, seed)
         run(roles, q, seed)
+
+
+# ---------------------------------------------------------------- the fused vocabulary/update GEMM (k_tc_vocab_update.cu)
+
+def test_fused_vocab_epilogue_barriers():
+    """Four warps meeting at a named barrier 2 + 2 * chunks times per tile, interleaved with
+    the accumulator hand-offs: no deadlock and no phase overrun."""
+    for n_tiles, nkb, stages, chunks in ((1, 2, 2, 1), (3, 4, 3, 16), (5, 2, 4, 3)):
+        for seed in range(20):
+            full = [Barrier(f"full{s}", 1) for s in range(stages)]
+            empty = [Barrier(f"empty{s}", 1) for s in range(stages)]
+            acc_full = [Barrier(f"acc_full{b}", 1) for b in range(2)]
+            acc_empty = [Barrier(f"acc_empty{b}", 4) for b in range(2)]
+            named = Barrier("bar1", 4)
+            bufs, q = Buffers(), Async()
+            acc_done = {}
+
+            def producer():
+                it = 0
+                for t in range(n_tiles):
+                    for kb in range(nkb):
+                        s = it % stages
+                        yield wait(empty[s], ((it // stages) & 1) ^ 1, it // stages - 1)
+                        bufs.fill(("smem", s), 1)
+                        full[s].arrive_expect_tx(64)
+                        q.loads.append(lambda s=s: full[s].complete_tx(64))
+                        it += 1
+
+            def mma():
+                it = 0
+                for j in range(n_tiles):
+                    buf = j & 1
+                    yield wait(acc_empty[buf], ((j >> 1) & 1) ^ 1, (j >> 1) - 1)
+                    bufs.fill(("acc", buf), 4)
+                    acc_done[buf] = 0
+                    for kb in range(nkb):
+                        s = it % stages
+                        yield wait(full[s], (it // stages) & 1, it // stages)
+
+                        def done(s=s, buf=buf):
+                            acc_done[buf] += 1
+                            bufs.release(("smem", s))
+                            empty[s].arrive()
+                        q.mma.append(done)
+                        it += 1
+                    q.mma.append(lambda b=buf: acc_full[b].arrive())
+
+            def epilogue(w):
+                k = 0  # named-barrier phases this warp has passed
+
+                def meet():
+                    nonlocal k
+                    named.arrive()
+                    yield wait(named, k & 1, k)
+                    k += 1
+                for j in range(n_tiles):
+                    buf = j & 1
+                    yield wait(acc_full[buf], (j >> 1) & 1, j >> 1)
+                    yield from meet()          # post the wait result
+                    yield from meet()          # the vote is read; the flags may be rewritten
+                    assert acc_done[buf] == nkb
+                    for c in range(chunks):
+                        yield from meet()      # the four warps' records are in shared memory
+                        yield from meet()      # merged and stored; the next chunk may write
+                    bufs.release(("acc", buf))
+                    acc_empty[buf].arrive()
+
+            roles = {"tma": producer(), "mma": mma()}
+            roles.update({f"epi{w}": epilogue(w) for w in range(4)})
+            run(roles, q, seed)
