@@ -1,0 +1,94 @@
+"""bench.py's host-side helpers on the CPU: the NVML clock sampler (against a fake NVML
+module: it only reads), the hash guard that reports ncu traffic only for the kernel
+source it was captured on, the peak-file fallback and the whole-job value."""
+import os
+import shutil
+import sys
+import time
+import types
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _fake_nvml(clock_seq, reason_bits):
+    nv = types.SimpleNamespace()
+    nv.NVML_CLOCK_SM = 1
+    nv.nvmlClocksEventReasonHwSlowdown = 0x8
+    nv.nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nv.nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nv.nvmlClocksEventReasonSwPowerCap = 0x4
+    nv.nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+    it = iter(clock_seq)
+    last = [clock_seq[0]]
+
+    def clock(h, which):
+        assert h == "gpu0" and which == 1
+        try:
+            last[0] = next(it)
+        except StopIteration:
+            pass
+        return last[0]
+    nv.nvmlDeviceGetClockInfo = clock
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, which: 1965
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: reason_bits
+    return nv
+
+
+def test_clock_sampler_reports_median_and_reasons(monkeypatch):
+    nv = _fake_nvml([1965, 1950, 1965, 1900, 1965], 0x4)
+    c = bench.Clocks(device=None)
+
+    def handle(self):
+        self.nv = nv
+        return "gpu0"
+    monkeypatch.setattr(bench.Clocks, "_handle", handle)
+    c.start()
+    time.sleep(0.1)
+    r = c.stop()
+    assert r["sm_max_mhz"] == 1965 and r["samples"] >= 3
+    assert r["sm_mhz"] in (1950, 1965)
+    assert r["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_reports_why_it_is_unavailable(monkeypatch):
+    def handle(self):
+        raise RuntimeError("no NVML here")
+    monkeypatch.setattr(bench.Clocks, "_handle", handle)
+    c = bench.Clocks(device=None)
+    c.start()
+    r = c.stop()
+    assert "unavailable" in r and "no NVML" in r["unavailable"]
+
+
+def test_ncu_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
+    assert bench._ncu_traffic("layer1_bf16") == pytest.approx(457.380608e6 + 6.031104e6)
+    assert bench._ncu_traffic("large4_bf16") is None                   # no capture for it
+    src = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", "k_tc_gemm.cu")
+    fake = tmp_path / "block_diffusion_lm_masked_b200" / "csrc"
+    fake.mkdir(parents=True)
+    shutil.copy(src, fake / "k_tc_gemm.cu")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._ncu_traffic("layer1_bf16") is not None              # same bytes, same hash
+    with open(fake / "k_tc_gemm.cu", "a") as f:
+        f.write("\n// changed\n")
+    assert bench._ncu_traffic("layer1_bf16") is None                   # the kernel changed since
+
+
+def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    hbm, tf, tfs, src = bench._peaks()
+    assert src == "fallback" and hbm == 6650.0 and tf == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6554.6, "bf16_tflops": 1591.5}')
+    hbm, tf, tfs, src = bench._peaks()
+    assert src == "measured" and hbm == 6554.6 and tf == tfs == 1591.5
+
+
+def test_job_value_counts_every_rank_over_the_slowest():
+    assert bench.job_value(1, 256, 1000, 347.6) == pytest.approx(256 * 1000 / 0.3476)
+    assert bench.job_value(8, 256, 1000, 400.0) == pytest.approx(8 * 256 * 1000 / 0.4)
