@@ -1311,6 +1311,8 @@ extern "C" dg_status dg_device_status(void* d_ws, dg_stream stream) {
     const int zero = 0;
     cudaMemcpy(d_ws, &zero, sizeof(int), cudaMemcpyHostToDevice);
     if (v == DG_DEVERR_BAD_TOKEN) return fail(DG_ERR_INVALID_ARG, "a token id was outside [0, vocab)");
+    if (v == DG_DEVERR_CHECK)
+      return fail(DG_ERR_CUDA, "a kernel access failed its bounds or alignment check (checked build); it was skipped");
     return fail(DG_ERR_TIMEOUT, "device error word %d (a bounded wait gave up)", v);
   }
   return DG_OK;

@@ -22,6 +22,20 @@
 #define DG_DEVERR_BAD_COUNT 5
 #define DG_DEVERR_BAD_TOKEN 6
 #define DG_DEVERR_TIMEOUT_PART 7
+#define DG_DEVERR_CHECK 8  // checked build only: an access failed its bounds or alignment check
+
+// Checked build (compiled with DG_CHECKED): DG_GUARD(cond, err) records DG_DEVERR_CHECK in
+// the error word and yields false when cond does not hold, so that the caller skips the
+// access; the product build compiles it to true.
+#ifdef DG_CHECKED
+__device__ __forceinline__ bool dg_guard(bool ok, int* err) {
+  if (!ok && err) atomicCAS(err, 0, DG_DEVERR_CHECK);
+  return ok;
+}
+#define DG_GUARD(cond, err) dg_guard((cond), (err))
+#else
+#define DG_GUARD(cond, err) true
+#endif
 
 namespace dg {
 

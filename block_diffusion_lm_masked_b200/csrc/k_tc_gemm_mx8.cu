@@ -245,6 +245,17 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
           uint8_t* st = smem + (size_t)s * stage_bytes;
           const int kbx = (kb + t) % nkb;  // tiles running together start at different k-blocks
           const int kx = kbx * MX_BK;
+          // the stage's TMA rules: x coordinates on 16-byte boundaries, every box inside the
+          // stage, token rows within the ring's reservation, TMEM stages within the allocation
+          if (!DG_GUARD(((FMT == FMT_NV4 ? kx / 2 : kx) % 16 == 0) && ((kx * 2) % 16 == 0) && n_pad <= p.n_max &&
+                            s_off + (uint32_t)n_a * MX_S_BYTES <= stage_bytes &&
+                            (uint32_t)(s + 1) * stage_bytes <= (uint32_t)p.smem_budget &&
+                            a_col0 + MX_T_STAGES * a_stage_cols <= tmem_cols,
+                        p.err)) {
+            abort_s = 1;
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(&f_full[s], tx);
           // codes: x in bytes along K; scales: MX8 (2 rows' bytes, k-block, group),
           // NV4 (16 bytes = 4 rows, rows / 4, group * k-blocks + k-block)
@@ -349,6 +360,7 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
           }
           if (!fvalid || col >= ti.rows) continue;
           const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
+          if (!DG_GUARD(ti.row0 + col < p.n_tokens && f < p.ld_out && c0 + q < n_pad, p.err)) continue;
           if (EPI == EPI_STORE_F32) {
             reinterpret_cast<float*>(p.out)[o] = a;
           } else {
@@ -387,7 +399,11 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
         }
         tc_fence_after();
         const uint8_t* st = smem + (size_t)s * stage_bytes;
-        for (int a = 0; a < n_a; ++a) {
+        const bool in_bounds = DG_GUARD(
+            (uint32_t)row * row_bytes + row_bytes <= MX_A_BYTES / MX_BM * MX_BM && row < MX_BM &&
+                a_col0 + (uint32_t)(ts + 1) * a_stage_cols <= tmem_cols,
+            p.err);
+        for (int a = 0; a < n_a && in_bounds; ++a) {
           const uint8_t* codes = st + a_off + (uint32_t)a * MX_A_BYTES + row * row_bytes;
           uint32_t w[16];
           if (FMT == FMT_NV4) {

@@ -134,6 +134,14 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
           uint8_t* sa = smem + (size_t)s * stage_bytes;
           uint8_t* sb = sa + a_bytes;
           const int kx = ((kb + t) % nkb) * VU_BK;  // tiles running together start at different k-blocks
+          if (!DG_GUARD((kx * 2) % 16 == 0 && n_pad <= p.n_max &&
+                            (uint32_t)(s + 1) * stage_bytes <= (uint32_t)p.smem_budget &&
+                            (uint32_t)(2 * acc_cols) <= tmem_cols,
+                        p.err)) {
+            abort_s = 1;
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(&full_bar[s], tx);
           tma_load_3d(sa, &tmA, kx, m * VU_BM, 0, &full_bar[s]);
           int r = 0;
@@ -227,7 +235,8 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
         }
         if (lane < 16) red[lg][lane] = mine;
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
-        if (lg == 0 && lane < 16 && c0 + lane < rows) {
+        if (lg == 0 && lane < 16 && c0 + lane < rows &&
+            DG_GUARD(row0 + c0 + lane < p.n_tokens && m < p.m_tiles && c0 + lane < n_pad, p.err)) {
           UpdPart o = red[0][lane];
 #pragma unroll
           for (int w2 = 1; w2 < 4; ++w2) {  // warps in id order

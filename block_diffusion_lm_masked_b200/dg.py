@@ -15,7 +15,9 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdg.so")
+# DG_CHECKED=1 loads the build with the kernels' bounds and alignment checks compiled in
+# (python -m block_diffusion_lm_masked_b200.build --checked)
+LIB_PATH = os.path.join(_HERE, "libdg_checked.so" if os.environ.get("DG_CHECKED") == "1" else "libdg.so")
 
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_CAPACITY, DG_ERR_CUDA, DG_ERR_TIMEOUT, DG_ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
 DTYPE = {"bf16": 0, "f32": 1}

@@ -333,3 +333,22 @@ def test_denoise_update_validation_on_host():
         assert dg.lib.dg_launch_count() == launches
     finally:
         dg.lib.dg_model_destroy(h)
+
+
+def test_checked_build_is_selected_by_the_environment():
+    """DG_CHECKED=1 makes the binding load libdg_checked.so (the kernels' bounds and
+    alignment checks compiled in); without it the product library loads."""
+    import subprocess
+    import sys
+    code = "from block_diffusion_lm_masked_b200 import dg; print(dg.LIB_PATH)"
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    env.pop("DG_CHECKED", None)
+    plain = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, cwd=ROOT)
+    assert plain.returncode == 0 and plain.stdout.strip().endswith("libdg.so")
+    checked_path = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "libdg_checked.so")
+    if not os.path.exists(checked_path):
+        pytest.skip("the checked build is made on demand (build --checked)")
+    env["DG_CHECKED"] = "1"
+    chk = subprocess.run([sys.executable, "-c", code + "; print(dg.lib.dg_launch_count())"], env=env,
+                         capture_output=True, text=True, cwd=ROOT)
+    assert chk.returncode == 0 and chk.stdout.split()[0].endswith("libdg_checked.so"), chk.stderr
