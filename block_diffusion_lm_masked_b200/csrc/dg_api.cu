@@ -206,7 +206,7 @@ struct LayerMaps {
 };
 // low-precision experts of one layer: codes and block scales of gate, up and down, the
 // format (dg::FMT_MX8 / dg::FMT_NV4) and the 4-bit tensor scales
-struct Mx8Maps {
+struct LowpMaps {
   CUtensorMap gate, gate_s, up, up_s, down, down_s;
   int fmt;
   float g_gate, g_up, g_down;
@@ -218,7 +218,7 @@ struct dg_model {
   std::vector<dg_layer_weights> layers;
   std::vector<LayerMaps> maps;
   CUtensorMap out_map;
-  std::vector<Mx8Maps> mx8;  // non-empty: the batched calls run the experts from low-precision weights
+  std::vector<LowpMaps> lowp;  // non-empty: the batched calls run the experts from low-precision weights
   bool taps_on = false;
   std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
   std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
@@ -462,7 +462,7 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
 
 // a grouped expert GEMM over low-precision weights (A, S: codes and scales; A2, S2 for gate
 // / up; g_a, g_a2: the 4-bit tensor scales)
-dg_status gemm_mx8(const GemmCall& g, int fmt, const CUtensorMap* S, const CUtensorMap* S2, float g_a, float g_a2,
+dg_status gemm_lowp(const GemmCall& g, int fmt, const CUtensorMap* S, const CUtensorMap* S2, float g_a, float g_a2,
                    int* err, cudaStream_t st) {
   CUtensorMap B, B2, Bb, B2b;
   dg_status s;
@@ -819,8 +819,8 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
     if (cudaMemcpyAsync(m->tap_x_attn[l], ws.at<float>(ws.L.x), (size_t)n * H * 4, cudaMemcpyDeviceToDevice, st) !=
         cudaSuccess)
       return fail(DG_ERR_CUDA, "tap copy failed");
-  const bool mx8 = bf && !m->mx8.empty();
-  const int item_rows = mx8 ? kItemRowsMx8 : kItemRows;
+  const bool lowp = bf && !m->lowp.empty();
+  const int item_rows = lowp ? kItemRowsMx8 : kItemRows;
   LAUNCH(DG_K_PERMUTE, st,
          dg::launch_permute(ws.at<int32_t>(ws.L.topk_idx), n, k, E, ws.at<int32_t>(ws.L.counts),
                             ws.at<int32_t>(ws.L.offsets), ws.at<int32_t>(ws.L.perm), ws.at<int32_t>(ws.L.inv),
@@ -831,19 +831,19 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
          dg::launch_gather_rows<T>(ws.at<T>(ws.L.xn), xn_lo, ws.at<int32_t>(ws.L.perm), n * k, k, H,
                                    ws.at<T>(ws.L.xs), xs_lo, st));
   const int* off = ws.at<int>(ws.L.offsets);
-  if (mx8) {
+  if (lowp) {
     const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
     const int* n_items = ws.at<int>(ws.L.n_items);
     const int max_items = n * k / kItemRowsMx8 + E;
-    const Mx8Maps& X8 = m->mx8[l];
+    const LowpMaps& X8 = m->lowp[l];
     GemmCall gu{DG_K_GEMM_GATE_UP, dg::EPI_SWIGLU_BF16, &X8.gate, &X8.up, ws.at<void>(ws.L.xs), xs_lo, n * k, H, F,
                 items, n_items, max_items, kItemRowsMx8, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo), F, 1, 0,
                 kSmemGemm};
-    if ((s = gemm_mx8(gu, X8.fmt, &X8.gate_s, &X8.up_s, X8.g_gate, X8.g_up, err, st)) != DG_OK) return s;
+    if ((s = gemm_lowp(gu, X8.fmt, &X8.gate_s, &X8.up_s, X8.g_gate, X8.g_up, err, st)) != DG_OK) return s;
     GemmCall dn{DG_K_GEMM_DOWN, dg::EPI_STORE_F32, &X8.down, nullptr, ws.at<void>(ws.L.h), ws.at<void>(ws.L.h_lo),
                 n * k, F, H, items, n_items, max_items, kItemRowsMx8, ws.at<float>(ws.L.ys), nullptr, H, 1, 0,
                 kSmemGemm};
-    if ((s = gemm_mx8(dn, X8.fmt, &X8.down_s, nullptr, X8.g_down, 1.0f, err, st)) != DG_OK) return s;
+    if ((s = gemm_lowp(dn, X8.fmt, &X8.down_s, nullptr, X8.g_down, 1.0f, err, st)) != DG_OK) return s;
   } else if (bf) {
     const dg::TcWorkItem* items = ws.at<dg::TcWorkItem>(ws.L.items);
     const int* n_items = ws.at<int>(ws.L.n_items);
@@ -1213,7 +1213,7 @@ extern "C" dg_status dg_generate_canvases(dg_model* m, dg_kv_cache* caches, int3
 static dg_status set_experts_lowp(dg_model* m, int fmt, const dg_expert_weights_mx8* layers, const float* g3) {
   DG_CHECK_ARG(m, "model is NULL");
   if (!layers) {
-    m->mx8.clear();
+    m->lowp.clear();
     return DG_OK;
   }
   const dg_config& c = m->cfg;
@@ -1228,7 +1228,7 @@ static dg_status set_experts_lowp(dg_model* m, int fmt, const dg_expert_weights_
       DG_CHECK_ARG(isfinite(g3[3 * l]) && isfinite(g3[3 * l + 1]) && isfinite(g3[3 * l + 2]),
                    "layer %d: tensor scales must be finite", l);
   }
-  std::vector<Mx8Maps> maps;
+  std::vector<LowpMaps> maps;
   try {
     maps.resize(c.n_layers);
   } catch (...) {
@@ -1239,7 +1239,7 @@ static dg_status set_experts_lowp(dg_model* m, int fmt, const dg_expert_weights_
   auto scales = fmt == dg::FMT_NV4 ? map_scales4 : map_scales;
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_expert_weights_mx8& X = layers[l];
-    Mx8Maps& M = maps[l];
+    LowpMaps& M = maps[l];
     dg_status s;
     if ((s = codes(&M.gate, X.gate, E, F, H)) != DG_OK || (s = scales(&M.gate_s, X.gate_scales, E, F, H)) != DG_OK ||
         (s = codes(&M.up, X.up, E, F, H)) != DG_OK || (s = scales(&M.up_s, X.up_scales, E, F, H)) != DG_OK ||
@@ -1250,7 +1250,7 @@ static dg_status set_experts_lowp(dg_model* m, int fmt, const dg_expert_weights_
     M.g_up = g3 ? g3[3 * l + 1] : 1.0f;
     M.g_down = g3 ? g3[3 * l + 2] : 1.0f;
   }
-  m->mx8.swap(maps);
+  m->lowp.swap(maps);
   return DG_OK;
 }
 

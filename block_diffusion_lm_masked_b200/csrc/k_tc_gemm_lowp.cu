@@ -150,7 +150,7 @@ __device__ __forceinline__ uint32_t e4m3_scale_pair(uint32_t sc) {
 
 template <int EPI, int FMT>
 __global__ void __launch_bounds__(MX_THREADS, 1)
-    tc_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+    tc_gemm_lowp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                        const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmS2,
                        const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                        const __grid_constant__ CUtensorMap tmBb, const __grid_constant__ CUtensorMap tmB2b,
@@ -467,17 +467,17 @@ static cudaError_t launch_fmt(int epi, const CUtensorMap& A, const CUtensorMap& 
                               float g_a2, int grid, int smem, cudaStream_t st) {
   cudaError_t e;
   if (epi == EPI_STORE_F32) {
-    e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_STORE_F32, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc_gemm_lowp_kernel<EPI_STORE_F32, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
     if (e != cudaSuccess) return e;
-    return launch_k(tc_gemm_mx8_kernel<EPI_STORE_F32, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B,
+    return launch_k(tc_gemm_lowp_kernel<EPI_STORE_F32, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2, B,
                     B2, Bb, B2b, p, g_a, g_a2);
   }
   if (epi == EPI_SWIGLU_BF16) {
-    e = cudaFuncSetAttribute(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc_gemm_lowp_kernel<EPI_SWIGLU_BF16, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
     if (e != cudaSuccess) return e;
-    return launch_k(tc_gemm_mx8_kernel<EPI_SWIGLU_BF16, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2,
+    return launch_k(tc_gemm_lowp_kernel<EPI_SWIGLU_BF16, FMT>, dim3(grid), dim3(MX_THREADS), smem, st, A, A2, S, S2,
                     B, B2, Bb, B2b, p, g_a, g_a2);
   }
   return cudaErrorInvalidValue;

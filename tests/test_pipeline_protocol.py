@@ -2,7 +2,7 @@
 
 Each role of a kernel (TMA producer, MMA issuer, decoder warps, epilogue warps) is
 written here as a sequence of the waits and arrivals it performs, with the counts,
-parities and ring sizes of the kernel source (k_tc_gemm.cu, k_tc_gemm_mx8.cu).  A
+parities and ring sizes of the kernel source (k_tc_gemm.cu, k_tc_gemm_lowp.cu).  A
 scheduler runs the roles in random interleavings under mbarrier semantics (a phase
 completes when its pending arrivals and transaction bytes reach zero; a parity wait on
 phase parity P passes once the phase in progress has the other parity), and checks:
@@ -171,7 +171,7 @@ def bf16_gemm(n_tiles, nkb, stages):
     return roles, q
 
 
-# ---------------------------------------------------------------- the 8-bit GEMM (k_tc_gemm_mx8.cu)
+# ---------------------------------------------------------------- the 8-bit GEMM (k_tc_gemm_lowp.cu)
 
 def lowp_gemm(n_tiles, nkb, stages, t_stages=4, dec_warps=8):
     f_full = [Barrier(f"f_full{s}", 1) for s in range(stages)]
