@@ -514,3 +514,148 @@ def test_fused_vocab_epilogue_barriers():
             roles = {"tma": producer(), "mma": mma()}
             roles.update({f"epi{w}": epilogue(w) for w in range(4)})
             run(roles, q, seed)
+
+
+# ---------------------------------------------------------------- leaving on a timeout
+
+def fused_epilogue_with_abort(n_tiles, nkb, stages, chunks, rng, vote=True):
+    """The fused vocabulary/update kernel's roles where some wait gives up: a bounded
+    mbarrier wait returns (false) once the CTA's abort flag is set, a named barrier does
+    not.  With the vote, the four epilogue warps agree before every named barrier on
+    whether to go on; without it, each warp leaves alone."""
+    full = [Barrier(f"full{s}", 1) for s in range(stages)]
+    empty = [Barrier(f"empty{s}", 1) for s in range(stages)]
+    acc_full = [Barrier(f"acc_full{b}", 1) for b in range(2)]
+    acc_empty = [Barrier(f"acc_empty{b}", 4) for b in range(2)]
+    named = Barrier("bar1", 4)
+    q = Async()
+    flags = {"abort": False}
+    epi_ok = [True] * 4
+    give_up_at = rng.randrange(1, 2 * n_tiles * nkb + 2)   # the step at which some wait times out
+    steps = [0]
+
+    def wait_ab(bar, parity, phase):
+        # a bounded wait: passes on the phase, or gives up once the abort flag is set (or
+        # when this wait is the one chosen to time out, which raises the flag)
+        steps[0] += 1
+        if steps[0] == give_up_at:
+            flags["abort"] = True
+        return ("waitab", bar, parity, phase)
+
+    def ok_after(bar, parity):
+        return (bar.completed % 2) != parity
+
+    def producer():
+        it = 0
+        for t in range(n_tiles):
+            for kb in range(nkb):
+                s = it % stages
+                par = ((it // stages) & 1) ^ 1
+                yield wait_ab(empty[s], par, None)
+                if not ok_after(empty[s], par):
+                    return
+                full[s].arrive_expect_tx(64)
+                q.loads.append(lambda s=s: full[s].complete_tx(64))
+                it += 1
+
+    def mma():
+        it = 0
+        for j in range(n_tiles):
+            buf = j & 1
+            par = ((j >> 1) & 1) ^ 1
+            yield wait_ab(acc_empty[buf], par, None)
+            if not ok_after(acc_empty[buf], par):
+                return
+            for kb in range(nkb):
+                s = it % stages
+                par2 = (it // stages) & 1
+                yield wait_ab(full[s], par2, None)
+                if not ok_after(full[s], par2):
+                    return
+                q.mma.append(lambda s=s: empty[s].arrive())
+                it += 1
+            q.mma.append(lambda b=buf: acc_full[b].arrive())
+
+    def epilogue(w):
+        k = 0
+
+        def meet():
+            nonlocal k
+            named.arrive()
+            yield wait(named, k & 1, k)
+            k += 1
+        for j in range(n_tiles):
+            buf = j & 1
+            par = (j >> 1) & 1
+            yield wait_ab(acc_full[buf], par, None)
+            ok = ok_after(acc_full[buf], par)
+            if vote:
+                epi_ok[w] = ok
+                yield from meet()
+                all_ok = all(epi_ok)
+                yield from meet()
+                if not all_ok:
+                    return
+            elif not ok:
+                return
+            for c in range(chunks):
+                yield from meet()
+                yield from meet()
+            acc_empty[buf].arrive()
+
+    roles = {"tma": producer(), "mma": mma()}
+    roles.update({f"epi{w}": epilogue(w) for w in range(4)})
+    return roles, q, flags
+
+
+def run_ab(roles, q, flags, seed, max_steps=200000):
+    """run() where an abort-aware wait also passes once the abort flag is set."""
+    rng = random.Random(seed)
+    blocked = {}
+    live = dict(roles)
+    for _ in range(max_steps):
+        if not live:
+            return
+        ready = []
+        for name in live:
+            b = blocked.get(name)
+            if b is None:
+                ready.append(name)
+            elif b[0] == "waitab" and (flags["abort"] or (b[1].completed % 2) != b[2]):
+                ready.append(name)
+            elif b[0] == "wait" and b[1].passes(b[2], b[3]):
+                ready.append(name)
+        choices = ready + (["<async>"] if q else [])
+        assert choices, f"deadlock: blocked {sorted((n, b[1].name) for n, b in blocked.items())}"
+        pick = rng.choice(choices)
+        if pick == "<async>":
+            q.step(rng)
+            continue
+        blocked.pop(pick, None)
+        try:
+            step = next(live[pick])
+        except StopIteration:
+            del live[pick]
+            continue
+        if step is not None:
+            blocked[pick] = step
+    raise AssertionError("no progress")
+
+
+def test_fused_epilogue_warps_leave_together_on_a_timeout():
+    """With the vote every role of the fused kernel finishes whichever wait gives up (the
+    final __syncthreads is reached); without it some interleaving leaves warps blocked at
+    the named barrier for good -- the hang the vote prevents."""
+    for seed in range(300):
+        rng = random.Random(seed)
+        roles, q, flags = fused_epilogue_with_abort(3, 3, 2, 2, rng, vote=True)
+        run_ab(roles, q, flags, seed)
+    hung = 0
+    for seed in range(300):
+        rng = random.Random(seed)
+        roles, q, flags = fused_epilogue_with_abort(3, 3, 2, 2, rng, vote=False)
+        try:
+            run_ab(roles, q, flags, seed)
+        except AssertionError as e:
+            hung += "deadlock" in str(e)
+    assert hung > 0
