@@ -14,6 +14,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>  // header-only; ranges reach a profiler only when one is attached
+
 #include "../../include/dg.h"
 #include "../../include/dg_debug.h"
 #include "dg_common.cuh"
@@ -48,6 +50,7 @@ dg_status set_error(dg_status s, const char* msg) { return fail(s, "%s", msg); }
   } while (0)
 
 // ---------------------------------------------------------------- profiling
+extern "C" const char* dg_kernel_name(int32_t kind);
 namespace {
 struct ProfPair {
   cudaEvent_t a, b;
@@ -73,11 +76,23 @@ void prof_flush_locked() {
   g_prof_pending.clear();
 }
 
+// DG_NVTX set in the environment: every launch sits in an NVTX range named after its kind
+// (for filtering ncu / nsys captures)
+bool nvtx_on() {
+  static const bool on = getenv("DG_NVTX") != nullptr;
+  return on;
+}
+
 struct ProfScope {
   ProfPair pair{};
   bool on = false;
+  bool nvtx = false;
   cudaStream_t st;
   ProfScope(int kind, cudaStream_t s) : st(s) {
+    if (nvtx_on()) {
+      nvtxRangePushA(dg_kernel_name(kind));
+      nvtx = true;
+    }
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_launches++;
     if (!g_prof_on) return;
@@ -92,6 +107,7 @@ struct ProfScope {
     on = cudaEventRecord(pair.a, st) == cudaSuccess;
   }
   ~ProfScope() {
+    if (nvtx) nvtxRangePop();
     if (!on) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
     if (cudaEventRecord(pair.b, st) == cudaSuccess) g_prof_pending.push_back(pair);
