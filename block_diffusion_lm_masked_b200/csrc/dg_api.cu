@@ -115,8 +115,29 @@ struct ProfScope {
 };
 }  // namespace
 
+// Host-side fault injection: DG_FAULT_INJECT=launch:N makes the N-th kernel launch of the
+// process (1-based, every kind) fail on the host without launching, as a failed launch
+// would, so that the error paths can be exercised without faulting a GPU.
+namespace {
+long long fault_launch_index() {
+  static const long long n = [] {
+    const char* v = getenv("DG_FAULT_INJECT");
+    long long k = 0;
+    if (v && sscanf(v, "launch:%lld", &k) == 1 && k > 0) return k;
+    return 0LL;
+  }();
+  return n;
+}
+std::atomic<long long> g_launch_seq{0};
+bool inject_launch_fault() {
+  const long long n = fault_launch_index();
+  return n > 0 && g_launch_seq.fetch_add(1) + 1 == n;
+}
+}  // namespace
+
 #define LAUNCH(kind, st, call)                                                                          \
   do {                                                                                                  \
+    if (inject_launch_fault()) return fail(DG_ERR_CUDA, "%s: injected launch failure", #call);        \
     cudaError_t _e;                                                                                     \
     {                                                                                                   \
       ProfScope _ps((kind), (st));                                                                      \

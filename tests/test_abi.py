@@ -352,3 +352,38 @@ def test_checked_build_is_selected_by_the_environment():
     chk = subprocess.run([sys.executable, "-c", code + "; print(dg.lib.dg_launch_count())"], env=env,
                          capture_output=True, text=True, cwd=ROOT)
     assert chk.returncode == 0 and chk.stdout.split()[0].endswith("libdg_checked.so"), chk.stderr
+
+
+_INJECT = r"""
+import ctypes, sys
+sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+from block_diffusion_lm_masked_b200 import configs as CF, dg
+import test_abi as T
+cfg = CF.CONFIGS["tiny_fp32"]
+st, h = T._fake_model(cfg)
+L = cfg["n_layers"]
+ka = (ctypes.c_void_p * L)(*[(1 << 30) + (i << 16) for i in range(L)])
+va = (ctypes.c_void_p * L)(*[(1 << 31) + (i << 16) for i in range(L)])
+cache = dg.KVCacheS(ka, va, 256, 64)
+n = dg.workspace_bytes(cfg, 32)
+r = dg.lib.dg_prefill_append(h, ctypes.byref(cache), ctypes.c_void_p(1 << 24), 32, ctypes.c_void_p(1 << 25), n, None)
+print(r, cache.len, dg.lib.dg_launch_count(), dg.lib.dg_last_error().decode(), sep="|")
+"""
+
+
+def test_injected_launch_failure_is_a_clean_error_with_the_cache_unchanged():
+    """DG_FAULT_INJECT=launch:1: the first launch of a prefill fails on the host (no kernel
+    runs, no GPU is involved); the call returns DG_ERR_CUDA with the injected message and
+    the cache length does not advance."""
+    import subprocess
+    import sys
+    code = _INJECT.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
+    env = dict(os.environ, DG_FAULT_INJECT="launch:1")
+    env.pop("DG_CHECKED", None)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    status, length, launches, msg = r.stdout.strip().split("|", 3)
+    assert int(status) == dg.DG_ERR_CUDA
+    assert int(length) == 64
+    assert "injected launch failure" in msg
+    assert int(launches) == 0                          # failed before any launch was attempted
