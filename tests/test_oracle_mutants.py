@@ -358,6 +358,28 @@ def _array_ties_away(table, top, sign_bit):
     return enc
 
 
+def _merge_taps_per_canvas(per_canvas_taps, n_experts):
+    """Rows stacked, but the permutation kept per canvas (offset) instead of grouped over the batch."""
+    out = []
+    for layer_taps in zip(*per_canvas_taps):
+        m = {key: np.concatenate([t[key] for t in layer_taps], axis=0)
+             for key in ("x_in", "attn_o", "x_attn", "x_out", "router_logits", "topk_idx", "topk_w", "router_margin")}
+        perms, base = [], 0
+        for t in layer_taps:
+            perms.append(np.asarray(t["perm"]) + base)
+            base += t["topk_idx"].size
+        counts = sum(t["counts"] for t in layer_taps)
+        m.update(counts=counts, offsets=np.concatenate([[0], np.cumsum(counts)]), perm=np.concatenate(perms),
+                 union=int((counts > 0).sum()))
+        out.append(m)
+    return out
+
+
+def _batched_shared_cache(model, caches, canvases, prec):
+    """Every canvas attends to the first canvas's cache."""
+    return [_orig["denoise_pass"](model, caches[0], np.asarray(x), prec) for x in canvases]
+
+
 def _widen_shift8(a):
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << np.uint32(8)).view(np.float32).astype(np.float64)
@@ -457,6 +479,10 @@ MUTANTS = {
     "e2m1 subnormal value": ("e2m1_decode", _e2m1_subnormal, ["test_e2m1_codes_rounding_saturation"]),
     "e2m1 ties away from even": ("e2m1_encode", _e2m1_encode_ties_up, ["test_e2m1_codes_rounding_saturation"]),
     "nvfp4 tensor scale without the 6": ("nvfp4_quantize", _nvfp4_no_six, ["test_nvfp4_block_scaling"]),
+    "batch permutation kept per canvas": ("merge_batch_taps", _merge_taps_per_canvas,
+                                          ["test_batch_reads_the_union_of_the_canvases_experts"]),
+    "batched canvases share a cache": ("denoise_pass_batched", _batched_shared_cache,
+                                       ["test_batched_canvases_do_not_see_each_other"]),
     "array e4m3 encoder ties away from even": ("e4m3_encode_array", _array_ties_away(O._E4M3_POS, 448.0, 0x80),
                                                ["test_e4m3_array_encoder_is_the_scalar_rule"]),
     "array e2m1 encoder ties away from even": ("e2m1_encode_array", _array_ties_away(O._E2M1_POS, 6.0, 0x8),

@@ -467,8 +467,9 @@ def test_batched_canvases_do_not_see_each_other():
     a = O.denoise_pass_batched(m, [c0, c1], [x0, x1], prec)
     b = O.denoise_pass_batched(m, [c0, O.Cache.empty(cfg)], [x0, rng.integers(0, 40, 5)], prec)
     np.testing.assert_array_equal(a[0][0], b[0][0])
-    single, _ = O.denoise_pass(m, c0, x0, prec)
-    np.testing.assert_array_equal(a[0][0], single)
+    for (lg, _), c, x in zip(a, (c0, c1), (x0, x1)):     # every canvas is its own single pass
+        single, _ = O.denoise_pass(m, c, x, prec)
+        np.testing.assert_array_equal(lg, single)
     outs, caches = O.generate_canvases(m, [c0, c1], [x0, x1], 3, 0.5, 0.0, [5, 6], prec, True)
     one, cache_one = O.generate_canvas(m, c1, x1, 3, 0.5, 0.0, 6, prec, True)
     np.testing.assert_array_equal(outs[1], one)
