@@ -380,6 +380,18 @@ def _batched_shared_cache(model, caches, canvases, prec):
     return [_orig["denoise_pass"](model, caches[0], np.asarray(x), prec) for x in canvases]
 
 
+def _generate_first_seed(model, caches, canvases, S, r_start, r_end, seeds, prec, append):
+    res = [_orig["generate_canvas"](model, c, x, S, r_start, r_end, seeds[0], prec, append)
+           for c, x in zip(caches, canvases)]
+    return [r[0] for r in res], [r[1] for r in res]
+
+
+def _generate_no_append(model, caches, canvases, S, r_start, r_end, seeds, prec, append):
+    res = [_orig["generate_canvas"](model, c, x, S, r_start, r_end, sd, prec, False)
+           for c, x, sd in zip(caches, canvases, seeds)]
+    return [r[0] for r in res], [r[1] for r in res]
+
+
 def _widen_shift8(a):
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << np.uint32(8)).view(np.float32).astype(np.float64)
@@ -483,6 +495,10 @@ MUTANTS = {
                                           ["test_batch_reads_the_union_of_the_canvases_experts"]),
     "batched canvases share a cache": ("denoise_pass_batched", _batched_shared_cache,
                                        ["test_batched_canvases_do_not_see_each_other"]),
+    "batched generation with one seed": ("generate_canvases", _generate_first_seed,
+                                         ["test_batched_canvases_do_not_see_each_other"]),
+    "batched generation skips the append": ("generate_canvases", _generate_no_append,
+                                            ["test_batched_canvases_do_not_see_each_other"]),
     "array e4m3 encoder ties away from even": ("e4m3_encode_array", _array_ties_away(O._E4M3_POS, 448.0, 0x80),
                                                ["test_e4m3_array_encoder_is_the_scalar_rule"]),
     "array e2m1 encoder ties away from even": ("e2m1_encode_array", _array_ties_away(O._E2M1_POS, 6.0, 0x8),
