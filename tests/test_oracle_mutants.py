@@ -392,6 +392,35 @@ def _generate_no_append(model, caches, canvases, S, r_start, r_end, seeds, prec,
     return [r[0] for r in res], [r[1] for r in res]
 
 
+def _generate_step_plus_one(model, cache, canvas, S, r_start, r_end, seed, prec, append, record=None):
+    C = len(canvas)
+    cur = np.asarray(canvas, dtype=np.int32).copy()
+    for s in range(S):
+        logits, taps = O.denoise_pass(model, cache, cur, prec)
+        n = O.renoise_count(C, S, s, r_start, r_end)
+        upd = O.canvas_update(logits, n, seed, s + 1)
+        if record is not None:
+            record.append(dict(step=s, canvas_in=cur.copy(), logits=logits, taps=taps, update=upd, n=n))
+        cur = upd["canvas"]
+    if append:
+        cache = O.prefill_append(model, cache, cur, prec)
+    return cur, cache
+
+
+def _masked_generation_from_noise(model, cache, C, S, keep_start, keep_end, mask_id, prec, append, record=None):
+    cur = np.arange(C, dtype=np.int32) % mask_id            # not an all-[MASK] canvas
+    for s in range(S):
+        logits, taps = O.denoise_pass(model, cache, cur, prec)
+        n = O.renoise_count(C, S, s, keep_start, keep_end)
+        upd = O.canvas_update_masked(logits, cur, n, mask_id)
+        if record is not None:
+            record.append(dict(step=s, canvas_in=cur.copy(), logits=logits, taps=taps, update=upd, n=n))
+        cur = upd["canvas"]
+    if append:
+        cache = O.prefill_append(model, cache, cur, prec)
+    return cur, cache
+
+
 def _widen_shift8(a):
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << np.uint32(8)).view(np.float32).astype(np.float64)
@@ -499,6 +528,10 @@ MUTANTS = {
                                          ["test_batched_canvases_do_not_see_each_other"]),
     "batched generation skips the append": ("generate_canvases", _generate_no_append,
                                             ["test_batched_canvases_do_not_see_each_other"]),
+    "generation re-noises with the next step's draws": ("generate_canvas", _generate_step_plus_one,
+                                                        ["test_resume_from_a_middle_pass_reproduces_the_run"]),
+    "masked generation starts from noise": ("generate_canvas_masked", _masked_generation_from_noise,
+                                            ["test_generate_masked_loop_properties"]),
     "array e4m3 encoder ties away from even": ("e4m3_encode_array", _array_ties_away(O._E4M3_POS, 448.0, 0x80),
                                                ["test_e4m3_array_encoder_is_the_scalar_rule"]),
     "array e2m1 encoder ties away from even": ("e2m1_encode_array", _array_ties_away(O._E2M1_POS, 6.0, 0x8),
