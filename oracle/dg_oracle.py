@@ -553,6 +553,9 @@ def generate_canvas(model, cache: Cache, canvas: np.ndarray, S: int, r_start: fl
 def denoise_pass_batched(model, caches: list, canvases, prec: Precision):
     """Denoising passes of B independent canvases, canvas b against its own cache.
 
+    Hacker News discussion of DiffusionGemma, the comment on batching: batched requests
+    share the reads of common weights -- which is all batching changes.
+
     Batching shares weight reads, not arithmetic: each canvas attends only to its own
     cache and its own canvas (one request each), and every per-token step (routing,
     experts, vocabulary projection) is row-wise, so canvas b's result is its
