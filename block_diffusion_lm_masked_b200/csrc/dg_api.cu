@@ -778,6 +778,11 @@ dg_status run_stack(dg_model* m, const dg_kv_cache* cache, const int32_t* tokens
 // Canvas b occupies rows [b C, (b + 1) C) of every row-wise buffer and reads and writes
 // only its own cache; all rows share one router / permutation / expert GEMM / vocabulary
 // projection, so an expert's weights are read once for the whole batch.
+//
+// layer_batched repeats layer()'s sequence with a loop over canvases around RoPE and
+// attention, and the low-precision experts.  The copy is deliberate: the single-canvas
+// sequence stays exactly as measured and validated until this one has run on a GPU;
+// then layer() becomes layer_batched with one canvas and the copy goes.
 struct Seg {
   void* kc;
   void* vtc;
