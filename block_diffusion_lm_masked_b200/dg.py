@@ -185,7 +185,7 @@ class Model:
         returns to the bf16 experts.  Used by the batched calls."""
         if layers is None:
             _check(lib.dg_model_set_experts_mx8(self.handle, None))
-            self._mx8 = None
+            self._lowp = None
             return
         dev, keep, structs = self.device, [], []
         for L in layers:
@@ -199,7 +199,7 @@ class Model:
             structs.append(ExpertsMx8(*ptrs))
         arr = (ExpertsMx8 * len(structs))(*structs)
         _check(lib.dg_model_set_experts_mx8(self.handle, arr))
-        self._mx8 = keep
+        self._lowp = keep
 
     def set_experts_nv4(self, layers: list | None):
         """layers: per layer dict(gate=(codes, scale_codes, g), up=..., down=...) with codes
@@ -207,7 +207,7 @@ class Model:
         [E][rows][K / 16] and the tensor scale g; None returns to the bf16 experts."""
         if layers is None:
             _check(lib.dg_model_set_experts_nv4(self.handle, None, None))
-            self._mx8 = None
+            self._lowp = None
             return
         dev, keep, structs, gs = self.device, [], [], []
         for L in layers:
@@ -223,7 +223,7 @@ class Model:
         arr = (ExpertsMx8 * len(structs))(*structs)
         g_arr = (ctypes.c_float * len(gs))(*gs)
         _check(lib.dg_model_set_experts_nv4(self.handle, arr, g_arr))
-        self._mx8 = keep
+        self._lowp = keep
 
     def set_taps(self, taps: dict | None):
         """taps: name -> list (per layer) of device tensors sized for taps['rows'] tokens,
