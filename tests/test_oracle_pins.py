@@ -132,6 +132,31 @@ def test_rope_closed_form_and_relative_position():
     np.testing.assert_allclose(np.linalg.norm(O.rope(q, np.array([12345]), 1e4)), np.linalg.norm(q), rtol=1e-12)
 
 
+def test_rope_composes_as_a_rotation_and_norm_is_scale_free():
+    """RoPE at p1 then at p2 is RoPE at p1 + p2 (each pair turns by an angle linear in the
+    position); RMSNorm without eps ignores the scale of its input."""
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((2, 3, 16))
+    for p1, p2 in ((0, 5), (7, 11), (1000, 24)):
+        a = O.rope(O.rope(x, np.array([p1] * 3), 1e4), np.array([p2] * 3), 1e4)
+        np.testing.assert_allclose(a, O.rope(x, np.array([p1 + p2] * 3), 1e4), rtol=1e-9, atol=1e-12)
+    y = rng.standard_normal((4, 32))
+    np.testing.assert_allclose(O.rms_norm(7.5 * y, 0.0), O.rms_norm(y, 0.0), rtol=1e-13)
+
+
+def test_attention_ignores_an_equal_shift_of_a_rows_scores():
+    """Adding c q / |q|^2 to every key raises each of that query's scores by the same
+    c / sqrt(d): the softmax, hence the output row, does not change."""
+    rng = np.random.default_rng(13)
+    d = 16
+    q = rng.standard_normal((1, 1, d))
+    k = rng.standard_normal((1, 7, d))
+    v = rng.standard_normal((1, 7, d))
+    allowed = np.ones((1, 7), dtype=bool)
+    shifted = k + 3.0 * q[0, 0] / np.dot(q[0, 0], q[0, 0])
+    np.testing.assert_allclose(O.attention(q, shifted, v, allowed), O.attention(q, k, v, allowed), rtol=1e-12)
+
+
 def test_silu_closed_forms():
     np.testing.assert_allclose(O.silu(np.array([0.0, 50.0, -50.0, 1.0])),
                                [0.0, 50.0, -50.0 * math.exp(-50.0) / (1 + math.exp(-50.0)), 1 / (1 + math.exp(-1))],
@@ -496,6 +521,15 @@ def test_canvas_update_special_cases():
     # ties: argmax takes the lowest id; equal confidences re-noise lower positions first
     u3 = O.canvas_update(np.zeros((4, 6)), 2, 1, 0)
     assert list(u3["argmax"]) == [0, 0, 0, 0] and list(u3["renoised"]) == [0, 1]
+
+
+def test_canvas_update_ignores_a_constant_added_to_a_row():
+    rng = np.random.default_rng(14)
+    lg = rng.standard_normal((9, 33)) * 3
+    shift = rng.standard_normal((9, 1)) * 100
+    a, b = O.canvas_update(lg, 4, 3, 1), O.canvas_update(lg + shift, 4, 3, 1)
+    np.testing.assert_array_equal(a["canvas"], b["canvas"])
+    np.testing.assert_allclose(a["conf"], b["conf"], rtol=1e-10)
 
 
 def test_canvas_update_renoise_set_brute_force():
