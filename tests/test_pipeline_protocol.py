@@ -659,3 +659,95 @@ def test_fused_epilogue_warps_leave_together_on_a_timeout():
         except AssertionError as e:
             hung += "deadlock" in str(e)
     assert hung > 0
+
+
+# ---------------------------------------------------------------- the attention redesign (on paper)
+
+def attention_two_heads(nck, seed, slots=3, warps_per_head=4):
+    """The redesigned attention's hand-offs: a load warp fills `slots` K/V slots; the MMA
+    warp issues S_A(j), S_B(j) into S/P buffer j & 1 of each head, then PV_A(j-1),
+    PV_B(j-1), then frees chunk j-1's slot with a commit; each head's softmax warps read
+    S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  Before S_h(j)
+    reuses buffer j & 1, the MMA warp waits for PV_h(j-2), the last reader of that P."""
+    rng = random.Random(seed * 104729 + nck)
+    kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
+    kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
+    H = 2
+    s_full = [[Barrier(f"s_full{h}{b}", 1) for b in range(2)] for h in range(H)]
+    p_ready = [[Barrier(f"p_ready{h}{b}", warps_per_head) for b in range(2)] for h in range(H)]
+    pv_done = [[Barrier(f"pv_done{h}{b}", 1) for b in range(2)] for h in range(H)]
+    bufs, q = Buffers(), Async()
+    st = {"pv_done": [0, 0], "pv_issued": [0, 0], "s_done": [0, 0]}
+    p_writes = {}
+
+    def load():
+        for j in range(nck):
+            s = j % slots
+            yield wait(kv_free[s], ((j // slots) & 1) ^ 1, j // slots - 1)
+            bufs.fill(("slot", s), 2 * H)             # S_A, S_B, PV_A, PV_B of chunk j read it
+            kv_full[s].arrive_expect_tx(32)
+            q.loads.append(lambda s=s: kv_full[s].complete_tx(32))
+
+    def mma():
+        def issue_pv(h, k):
+            assert p_writes.get((h, k & 1)) == (k, warps_per_head), "PV read a P not fully written"
+            st["pv_issued"][h] += 1
+
+            def done(h=h, k=k):
+                st["pv_done"][h] += 1
+                for w in range(warps_per_head):       # every warp's lanes of P(k) were read
+                    bufs.release(("sp", h, k & 1, w))
+                bufs.release(("slot", k % slots))
+                pv_done[h][k & 1].arrive()
+            q.mma.append(done)
+
+        for j in range(nck):
+            s = j % slots
+            yield wait(kv_full[s], (j // slots) & 1, j // slots)
+            for h in range(H):
+                if j >= 2:
+                    yield wait(pv_done[h][j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
+                for w in range(warps_per_head):       # S: each warp reads its own 32 lanes
+                    bufs.fill(("sp", h, j & 1, w), 1)
+
+                def s_done(h=h, j=j, s=s):
+                    st["s_done"][h] += 1
+                    bufs.release(("slot", s))
+                    s_full[h][j & 1].arrive()
+                q.mma.append(s_done)
+            if j >= 1:
+                for h in range(H):
+                    yield wait(p_ready[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                    issue_pv(h, j - 1)
+                q.mma.append(lambda k=j - 1: kv_free[k % slots].arrive())
+        for h in range(H):
+            yield wait(p_ready[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
+            issue_pv(h, nck - 1)
+
+    def softmax(h, w):
+        for j in range(nck):
+            yield wait(s_full[h][j & 1], (j >> 1) & 1, j >> 1)
+            bufs.release(("sp", h, j & 1, w))          # this warp's lanes of S read into registers
+            if j > 0 and rng.random() < 0.4:           # the row max grew: rescale O after PV(j-1)
+                yield wait(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                assert st["pv_done"][h] >= j and st["pv_issued"][h] <= j, "O rescaled while a PV may write it"
+            bufs.fill(("sp", h, j & 1, w), 1)         # P over this warp's lanes of S, read by PV(j)
+            last, n = p_writes.get((h, j & 1), (None, 0))
+            p_writes[(h, j & 1)] = (j, 1) if last != j else (j, n + 1)
+            p_ready[h][j & 1].arrive()
+        yield wait(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
+        assert st["pv_done"][h] == nck
+
+    roles = {"load": load(), "mma": mma()}
+    for h in range(H):
+        roles.update({f"sm{h}{w}": softmax(h, w) for w in range(warps_per_head)})
+    return roles, q
+
+
+@pytest.mark.parametrize("nck", [1, 2, 3, 4, 7, 12])
+def test_attention_redesign_protocol(nck):
+    """The protocol planned for the attention redesign: no deadlock, no overrun, no
+    buffer refilled while read, no P read before all its writers, no O rescaled under a PV."""
+    for seed in range(40):
+        roles, q = attention_two_heads(nck, seed)
+        run(roles, q, seed)
