@@ -663,13 +663,31 @@ def test_fused_epilogue_warps_leave_together_on_a_timeout():
 
 # ---------------------------------------------------------------- the attention redesign (on paper)
 
-def attention_two_heads(nck, seed, slots=3, warps_per_head=4):
+def slot_plan(nck, cur_from, slots):
+    """Slots of each chunk: a cached chunk takes the next slot, a current chunk (the call's
+    own keys: hi and lo parts) the next two; returns [(slots of chunk j, use index of each)]."""
+    nxt, uses, plan = 0, [0] * slots, []
+    for j in range(nck):
+        k = 2 if j >= cur_from else 1
+        ss = [(nxt + i) % slots for i in range(k)]
+        plan.append([(x, uses[x]) for x in ss])
+        for x in ss:
+            uses[x] += 1
+        nxt = (nxt + k) % slots
+    return plan
+
+
+def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_first_rule=True):
     """The redesigned attention's hand-offs: a load warp fills `slots` K/V slots; the MMA
     warp issues S_A(j), S_B(j) into S/P buffer j & 1 of each head, then PV_A(j-1),
-    PV_B(j-1), then frees chunk j-1's slot with a commit; each head's softmax warps read
+    PV_B(j-1), then frees chunk j-1's slots with a commit; each head's softmax warps read
     S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  Before S_h(j)
-    reuses buffer j & 1, the MMA warp waits for PV_h(j-2), the last reader of that P."""
+    reuses buffer j & 1, the MMA warp waits for PV_h(j-2), the last reader of that P.
+    When chunks j-1 and j together need more slots than the ring has (two current chunks
+    in three slots), chunk j cannot load before chunk j-1's slots are free, so the MMA
+    warp issues PV(j-1) before S(j) (`pv_first_rule`; without it that case deadlocks)."""
     rng = random.Random(seed * 104729 + nck)
+    plan = slot_plan(nck, nck if cur_from is None else cur_from, slots)
     kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
     kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
     H = 2
@@ -682,11 +700,11 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4):
 
     def load():
         for j in range(nck):
-            s = j % slots
-            yield wait(kv_free[s], ((j // slots) & 1) ^ 1, j // slots - 1)
-            bufs.fill(("slot", s), 2 * H)             # S_A, S_B, PV_A, PV_B of chunk j read it
-            kv_full[s].arrive_expect_tx(32)
-            q.loads.append(lambda s=s: kv_full[s].complete_tx(32))
+            for s, u in plan[j]:
+                yield wait(kv_free[s], (u & 1) ^ 1, u - 1)
+                bufs.fill(("slot", s), 2 * H)         # S_A, S_B, PV_A, PV_B of chunk j read it
+                kv_full[s].arrive_expect_tx(32)
+                q.loads.append(lambda s=s: kv_full[s].complete_tx(32))
 
     def mma():
         def issue_pv(h, k):
@@ -697,29 +715,38 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4):
                 st["pv_done"][h] += 1
                 for w in range(warps_per_head):       # every warp's lanes of P(k) were read
                     bufs.release(("sp", h, k & 1, w))
-                bufs.release(("slot", k % slots))
+                for x, _ in plan[k]:
+                    bufs.release(("slot", x))
                 pv_done[h][k & 1].arrive()
             q.mma.append(done)
 
+        def pv_prev(j):
+            for h in range(H):
+                yield wait(p_ready[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                issue_pv(h, j - 1)
+            for x, _ in plan[j - 1]:                   # one commit per slot of chunk j-1
+                q.mma.append(lambda x=x: kv_free[x].arrive())
+
         for j in range(nck):
-            s = j % slots
-            yield wait(kv_full[s], (j // slots) & 1, j // slots)
+            pv_first = pv_first_rule and j >= 1 and len(plan[j - 1]) + len(plan[j]) > slots
+            if pv_first:
+                yield from pv_prev(j)
+            for x, u in plan[j]:
+                yield wait(kv_full[x], u & 1, u)
             for h in range(H):
                 if j >= 2:
                     yield wait(pv_done[h][j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
                 for w in range(warps_per_head):       # S: each warp reads its own 32 lanes
                     bufs.fill(("sp", h, j & 1, w), 1)
 
-                def s_done(h=h, j=j, s=s):
+                def s_done(h=h, j=j):
                     st["s_done"][h] += 1
-                    bufs.release(("slot", s))
+                    for x, _ in plan[j]:
+                        bufs.release(("slot", x))
                     s_full[h][j & 1].arrive()
                 q.mma.append(s_done)
-            if j >= 1:
-                for h in range(H):
-                    yield wait(p_ready[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
-                    issue_pv(h, j - 1)
-                q.mma.append(lambda k=j - 1: kv_free[k % slots].arrive())
+            if j >= 1 and not pv_first:
+                yield from pv_prev(j)
         for h in range(H):
             yield wait(p_ready[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
             issue_pv(h, nck - 1)
@@ -744,10 +771,23 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4):
     return roles, q
 
 
-@pytest.mark.parametrize("nck", [1, 2, 3, 4, 7, 12])
-def test_attention_redesign_protocol(nck):
-    """The protocol planned for the attention redesign: no deadlock, no overrun, no
-    buffer refilled while read, no P read before all its writers, no O rescaled under a PV."""
+@pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (3, 3), (4, 2), (7, 7), (7, 4), (12, 8), (6, 0)])
+def test_attention_redesign_protocol(nck, cur_from):
+    """The protocol planned for the attention redesign, cached chunks in one slot and the
+    call's own (current) chunks in two: no deadlock, no overrun, no buffer refilled while
+    read, no P read before all its writers, no O rescaled under a PV."""
     for seed in range(40):
-        roles, q = attention_two_heads(nck, seed)
+        roles, q = attention_two_heads(nck, seed, cur_from=cur_from)
+        run(roles, q, seed)
+
+
+def test_attention_redesign_needs_pv_first_for_two_current_chunks():
+    """Two current chunks in a row hold four slots of three if S(j) runs before PV(j-1):
+    the simulator finds the deadlock the issue-order rule avoids."""
+    with pytest.raises(AssertionError, match="deadlock"):
+        roles, q = attention_two_heads(4, 0, cur_from=2, pv_first_rule=False)
+        run(roles, q, 0)
+    # one current chunk after cached ones fits: the rule never fires there
+    for seed in range(20):
+        roles, q = attention_two_heads(5, seed, cur_from=4, pv_first_rule=False)
         run(roles, q, seed)
