@@ -548,10 +548,94 @@ int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
   return splits;
 }
 
+// split-KV factor of the head-pair kernel: one wave of CTAs, at least four 64-key chunks
+// per CTA (each CTA loads its query tiles once)
+int attn_pair_splits(int n_q, int nq, int group, int n_keys, int* chunks_per_split) {
+  const int nch = ceil_div(n_keys, 64);
+  const int base = ceil_div(n_q, 128) * dg::attn2_head_groups(nq, group);
+  int splits = dg::num_sms() / base;
+  if (splits > kMaxAttnSplits) splits = kMaxAttnSplits;
+  if (splits > nch / 4) splits = nch / 4;
+  if (splits < 1) splits = 1;
+  *chunks_per_split = ceil_div(nch, splits);
+  splits = ceil_div(nch, *chunks_per_split);
+  return splits;
+}
+
+// DG_ATTN_PAIR=1 routes the bf16 pass's attention through the head-pair kernel
+bool attn_pair_enabled() {
+  static const bool on = getenv("DG_ATTN_PAIR") != nullptr && getenv("DG_ATTN_PAIR")[0] == '1';
+  return on;
+}
+
+// attention() through the head-pair kernel: the same inputs, outputs and workspace
+dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0,
+                         int n_keys, int causal, cudaStream_t st) {
+  const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
+  CUtensorMap mq, mql, mk, mv, mkl, mvl;
+  dg_status s;
+  const int base = (pos0 / 128) * 128;  // the low-term window starts here (a multiple of 64)
+  const int Lc = ws.L.lo_rows;
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)n_q * d * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mq, ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&mql, ws.at<void>(ws.L.q_lo), 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if ((s = encode_bf16(&mk, kc, 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)n_keys, (uint64_t)d, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)cap * 2, (uint64_t)d * cap * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mv, vtc, 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)(n_keys - base), (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)Lc * d * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if ((s = encode_bf16(&mkl, ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)(n_keys - base), (uint64_t)d, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)Lc * 2, (uint64_t)d * Lc * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if ((s = encode_bf16(&mvl, ws.at<void>(ws.L.vt_lo), 3, dims, str, box)) != DG_OK) return s;
+  }
+  dg::TcAttnParams p;
+  p.n_q = n_q;
+  p.q_pos0 = pos0;
+  p.n_keys = n_keys;
+  p.causal = causal;
+  p.group = nq / nkv;
+  p.nq = nq;
+  p.n_splits = attn_pair_splits(n_q, nq, p.group, n_keys, &p.chunks_per_split);
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  p.has_lo = 1;
+  p.base = base;
+  p.out = ws.at<bf16>(ws.L.o);
+  p.out_lo = ws.at<bf16>(ws.L.o_lo);
+  p.part_o = ws.at<float>(ws.L.part_o);
+  p.part_lse = ws.at<float>(ws.L.part_lse);
+  p.err = ws.err();
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, st));
+  if (p.n_splits > 1)
+    LAUNCH(DG_K_ATTN_MERGE, st,
+           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),
+                                 ws.at<bf16>(ws.L.o_lo), st));
+  return DG_OK;
+}
+
 // attention of n_q new rows at positions pos0.. over cache keys [0, n_keys) -> ws.o (+ ws.o_lo)
 dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0, int n_keys,
                     int causal, cudaStream_t st) {
   const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
+  if (is_bf16(c) && attn_pair_enabled()) return attention_pair(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st);
   if (!is_bf16(c)) {
     LAUNCH(DG_K_ATTENTION, st,
            dg::launch_simt_attention_f32(ws.at<float>(ws.L.q), (const float*)kc, (const float*)vtc, cap, n_q, pos0,
@@ -1550,9 +1634,9 @@ static dg_status debug_gemm_lowp(int fmt, const void* W, const void* W_scales, f
   return DG_OK;
 }
 
-extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,
-                                             int32_t pos0, int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv,
-                                             void* out, void* out_lo, void* d_ws, size_t ws_bytes, dg_stream stream) {
+static dg_status debug_attention(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q, int32_t pos0,
+                                 int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv, void* out, void* out_lo,
+                                 void* d_ws, size_t ws_bytes, dg_stream stream, bool pair) {
   DG_CHECK_ARG(q && k && vt && out && d_ws, "NULL pointer");
   DG_CHECK_ARG(nq > 0 && nkv > 0 && nq % nkv == 0 && n_q > 0 && n_keys > 0 && n_keys <= cap && cap % 8 == 0,
                "bad attention shape");
@@ -1581,13 +1665,31 @@ extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.k_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.vt_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy q: %s", cudaGetErrorString(e));
-  if ((s = attention(c, ws, const_cast<void*>(k), const_cast<void*>(vt), cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
+  void* kc = const_cast<void*>(k);
+  void* vtc = const_cast<void*>(vt);
+  if ((s = pair ? attention_pair(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)
+                : attention(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
     return s;
   e = cudaMemcpyAsync(out, ws.at<void>(ws.L.o), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess && out_lo)
     e = cudaMemcpyAsync(out_lo, ws.at<void>(ws.L.o_lo), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy o: %s", cudaGetErrorString(e));
   return DG_OK;
+}
+
+extern "C" dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,
+                                             int32_t pos0, int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv,
+                                             void* out, void* out_lo, void* d_ws, size_t ws_bytes, dg_stream stream) {
+  return debug_attention(q, k, vt, cap, n_q, pos0, n_keys, causal, nq, nkv, out, out_lo, d_ws, ws_bytes, stream,
+                         false);
+}
+
+extern "C" dg_status dg_debug_attention_pair_bf16(const void* q, const void* k, const void* vt, int32_t cap,
+                                                  int32_t n_q, int32_t pos0, int32_t n_keys, int32_t causal,
+                                                  int32_t nq, int32_t nkv, void* out, void* out_lo, void* d_ws,
+                                                  size_t ws_bytes, dg_stream stream) {
+  return debug_attention(q, k, vt, cap, n_q, pos0, n_keys, causal, nq, nkv, out, out_lo, d_ws, ws_bytes, stream,
+                         true);
 }
 
 extern "C" dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream) {

@@ -93,6 +93,12 @@ cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, con
                                 const TcAttnParams& p, cudaStream_t st);
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
+// Head-pair variant (same parameters and outputs; chunks_per_split counts 64-key chunks):
+// K / Kl maps with 64-row boxes, Vt / Vtl as above.  Grid y = attn2_head_groups(nq, group).
+cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
+                                 const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
+                                 const TcAttnParams& p, cudaStream_t st);
+int attn2_head_groups(int nq, int group);
 
 // ---------------------------------------------------------------- SIMT kernels (any dtype)
 // T = float (fp32 model) or __nv_bfloat16; an activation for a bf16 GEMM is written as

@@ -1,0 +1,441 @@
+// tcgen05 flash attention, head-pair variant: the same attention as tc_attn_kernel (both
+// modes, the same hi + lo precision terms, the same lazy rescale and split-KV partials),
+// organised for more tensor-core overlap per CTA.
+//
+// One CTA = two query heads of one KV head (one head when the GQA group is odd) x 128
+// query rows x a contiguous range of 64-key chunks.  Each K/V chunk is loaded once for
+// both heads.  Warps 0-3 run the softmax of the first head and warps 4-7 that of the
+// second, one query row per thread over the whole 64-key chunk, so no row statistics are
+// exchanged between warps.  Warp 8 issues the TMA loads, warp 9 the MMAs.
+//
+// TMEM (512 columns): per head, two S/P buffers of 64 columns and O (128 columns).  The
+// softmax reads S (fp32, 64 keys) into registers and writes P over it as packed bf16
+// pairs, hi in the first 32 columns and lo in the next 32; the PV MMAs read P from there.
+// Shared memory: the query tiles (hi + lo, 64 KB per head) and three 32 KB K/V slots
+// (K [64 keys][128 d] and V^T [128 d][64 keys]).  A chunk of cached keys takes one slot; a
+// chunk of the call's own keys takes two (hi K/V in the first, lo in the second).
+//
+// Issue order of the MMA warp: S_A(j), S_B(j), then PV_A(j-1), PV_B(j-1) and a commit per
+// slot of chunk j-1 that frees it, so the PVs of one chunk run beside the softmax of the
+// next.  Before S_h(j) reuses buffer j & 1 it waits for PV_h(j-2), the last reader of that
+// P.  Where chunks j-1 and j together need more than the three slots (two chunks of own
+// keys in a row), chunk j cannot load until chunk j-1's slots are free, so PV(j-1) goes
+// first there.  That order was checked in a barrier simulation over random interleavings
+// (no deadlock, no slot or S/P buffer refilled while read, no O rescaled under a PV); the
+// plain order deadlocks in that case.
+#include <math.h>
+
+#include "dg_common.cuh"
+#include "dg_kernels.h"
+
+namespace dg {
+
+constexpr int A2_BQ = 128;
+constexpr int A2_W = 64;                              // keys per chunk
+constexpr int A2_D = 128;
+constexpr int A2_SLOTS = 3;
+constexpr uint32_t A2_QBLK = 128 * 128;               // [128 rows][64 bf16] swizzled: 16 KB
+constexpr uint32_t A2_QHEAD = 4 * A2_QBLK;            // Q hi (2 blocks) + Q lo (2 blocks)
+constexpr uint32_t A2_KBLK = 64 * 128;                // [64 keys][64 d]: 8 KB
+constexpr uint32_t A2_VOFF = 2 * A2_KBLK;             // V^T block [128 d][64 keys]: 16 KB
+constexpr uint32_t A2_SLOT = A2_VOFF + A2_QBLK;       // 32 KB
+constexpr int A2_SMEM = 1024 + 2 * A2_QHEAD + A2_SLOTS * A2_SLOT;
+constexpr int A2_LOAD_WARP = 8;
+constexpr int A2_MMA_WARP = 9;
+constexpr int A2_THREADS = 32 * 10;
+static_assert(A2_SMEM <= 227 * 1024 - 512, "shared memory budget");
+
+// TMEM column offsets: head hl's S/P buffer b, and its O
+__device__ __forceinline__ uint32_t a2_sp(int hl, int b) { return (uint32_t)(hl * 256 + b * 64); }
+__device__ __forceinline__ uint32_t a2_o(int hl) { return (uint32_t)(hl * 256 + 128); }
+
+// A operand from TMEM (P), B from shared memory (V^T), fp32 accumulate in TMEM
+__device__ __forceinline__ void a2_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The slot plan both the load and the MMA warp follow: chunk j takes the next one slot
+// (cached keys) or two (own keys) of the ring, in order.
+struct SlotPlan {
+  int nxt = 0;
+  int uses[A2_SLOTS] = {0, 0, 0};
+  int slot[2][2], use[2][2], n[2];  // [j & 1][part]: slot, its use index; parts of chunk j
+  __device__ void take(int j, bool cur) {
+    const int b = j & 1;
+    n[b] = cur ? 2 : 1;
+    for (int i = 0; i < n[b]; ++i) {
+      slot[b][i] = nxt;
+      use[b][i] = uses[nxt]++;
+      nxt = nxt + 1 == A2_SLOTS ? 0 : nxt + 1;
+    }
+  }
+};
+
+__global__ void __launch_bounds__(A2_THREADS, 1)
+    tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
+                    const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
+                    const TcAttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_bar;
+  __shared__ __align__(8) uint64_t kv_full[A2_SLOTS];  // the slot's TMA loads have landed
+  __shared__ __align__(8) uint64_t kv_free[A2_SLOTS];  // the MMAs reading the slot are complete
+  __shared__ __align__(8) uint64_t s_full[2][2];       // [head][buffer]: S is in TMEM
+  __shared__ __align__(8) uint64_t p_ready[2][2];      // [head][buffer]: P is in TMEM (4 warps)
+  __shared__ __align__(8) uint64_t pv_done[2][2];      // [head][buffer]: the PV reading P is complete
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, sp = blockIdx.z;
+  const int nh = (p.group % 2 == 0) ? 2 : 1;
+  const int h0 = blockIdx.y * nh;
+  const int kvh = h0 / p.group;
+  const int q_row0 = qt * A2_BQ;
+  const int rows_here = min(A2_BQ, p.n_q - q_row0);
+  int kv_end = p.n_keys;
+  if (p.causal) kv_end = min(p.n_keys, p.q_pos0 + q_row0 + rows_here);
+  const int nch_total = (kv_end + A2_W - 1) / A2_W;
+  const int c_begin = sp * p.chunks_per_split;
+  const int nck = min(nch_total, c_begin + p.chunks_per_split) - c_begin;
+
+  if (nck <= 0) {
+    // this split sees no key of the tile: empty partials (weight 0 in the merge)
+    griddep_sync();
+    const int qrow = q_row0 + tid;
+    if (tid < A2_BQ && qrow < p.n_q)
+      for (int hl = 0; hl < nh; ++hl) {
+        float* po = p.part_o + (((size_t)sp * p.nq + h0 + hl) * p.n_q + qrow) * A2_D;
+        for (int i = 0; i < A2_D; ++i) po[i] = 0.0f;
+        p.part_lse[((size_t)sp * p.nq + h0 + hl) * p.n_q + qrow] = -INFINITY;
+      }
+    return;
+  }
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                       // [head][Q hi blk0, blk1, Q lo blk0, blk1]
+  uint8_t* sSlot = smem + 2 * A2_QHEAD;     // [slot][K blk0, K blk1, V^T]
+
+  if (warp == A2_MMA_WARP) tmem_alloc(&tmem_base_s, 512);
+  if (tid == A2_LOAD_WARP * 32) {
+    mbar_init(&q_bar, 1);
+    for (int s = 0; s < A2_SLOTS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_free[s], 1);
+    }
+    for (int hl = 0; hl < 2; ++hl)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&s_full[hl][b], 1);
+        mbar_init(&p_ready[hl][b], 4);
+        mbar_init(&pv_done[hl][b], 1);
+      }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  griddep_sync();  // the previous kernel wrote q and this layer's current K/V
+  const uint32_t tmem = tmem_base_s;
+
+  auto is_cur = [&](int j) { return p.has_lo && (c_begin + j) * A2_W >= p.base; };
+  const uint32_t idesc_s = idesc_bf16_f32(A2_BQ, A2_W);
+  const uint32_t idesc_pv = idesc_bf16_f32(A2_BQ, A2_D);
+  int loaded[A2_SLOTS] = {0, 0, 0};  // loads the load thread issued into each slot (for the wind-down)
+  bool q_issued = false;
+
+  if (warp == A2_LOAD_WARP) {
+    if (lane == 0) {
+      // ================= loads: the query tiles, then each chunk's slots in plan order
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmQl);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmVt);
+      if (p.has_lo) {
+        prefetch_tmap(&tmKl);
+        prefetch_tmap(&tmVtl);
+      }
+      mbar_arrive_expect_tx(&q_bar, nh * A2_QHEAD);
+      for (int hl = 0; hl < nh; ++hl) {
+        uint8_t* q = sQ + hl * A2_QHEAD;
+        tma_load_3d(q, &tmQ, 0, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + A2_QBLK, &tmQ, 64, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + 2 * A2_QBLK, &tmQl, 0, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + 3 * A2_QBLK, &tmQl, 64, q_row0, h0 + hl, &q_bar);
+      }
+      q_issued = true;
+      SlotPlan lp;
+      bool ok = true;
+      for (int j = 0; j < nck && ok; ++j) {
+        const int key0 = (c_begin + j) * A2_W;
+        lp.take(j, is_cur(j));
+        for (int i = 0; i < lp.n[j & 1] && ok; ++i) {
+          const int s = lp.slot[j & 1][i], u = lp.use[j & 1][i];
+          // the slot's previous chunk was freed by the MMAs that read it
+          if (u >= 1 && !(ok = mbar_wait(&kv_free[s], (uint32_t)(u - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN)))
+            break;
+          uint8_t* k = sSlot + s * A2_SLOT;
+          const CUtensorMap* mk = (i == 0) ? &tmK : &tmKl;
+          const CUtensorMap* mv = (i == 0) ? &tmVt : &tmVtl;
+          const int krow = (i == 0) ? key0 : key0 - p.base;  // the low-term window starts at `base`
+          if (!DG_GUARD(krow >= 0 && krow % A2_W == 0, p.err)) {
+            ok = false;
+            abort_s = 1;
+            break;
+          }
+          loaded[s] += 1;
+          mbar_arrive_expect_tx(&kv_full[s], A2_SLOT);
+          tma_load_3d(k, mk, 0, krow, kvh, &kv_full[s]);
+          tma_load_3d(k + A2_KBLK, mk, 64, krow, kvh, &kv_full[s]);
+          tma_load_3d(k + A2_VOFF, mv, krow, 0, kvh, &kv_full[s]);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == A2_MMA_WARP) {
+    if (lane == 0) {
+      // ================= MMAs
+      SlotPlan mp;
+      auto slot_addr = [&](int s) { return smem_u32(sSlot + s * A2_SLOT); };
+      auto issue_s = [&](int hl, int j) {
+        const int b = j & 1;
+        const bool cur = mp.n[b] == 2;
+        const uint32_t d = tmem + a2_sp(hl, b);
+        const uint32_t q = smem_u32(sQ + hl * A2_QHEAD), ql = q + 2 * A2_QBLK;
+        const uint32_t k = slot_addr(mp.slot[b][0]);
+        const uint32_t kl = cur ? slot_addr(mp.slot[b][1]) : 0u;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t oq = kb * A2_QBLK + kk * 32, okb = kb * A2_KBLK + kk * 32;
+            const uint64_t kd = sw128_kmajor_desc(k + okb);
+            tc_mma(d, sw128_kmajor_desc(q + oq), kd, idesc_s, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma(d, sw128_kmajor_desc(ql + oq), kd, idesc_s, 1u);
+            if (cur) tc_mma(d, sw128_kmajor_desc(q + oq), sw128_kmajor_desc(kl + okb), idesc_s, 1u);
+          }
+        tc_commit(&s_full[hl][b]);
+      };
+      auto issue_pv = [&](int hl, int k) {
+        const int b = k & 1;
+        const bool cur = mp.n[b] == 2;
+        const uint32_t o = tmem + a2_o(hl), pp = tmem + a2_sp(hl, b);
+        const uint32_t v = slot_addr(mp.slot[b][0]) + A2_VOFF;
+        const uint32_t vl = cur ? slot_addr(mp.slot[b][1]) + A2_VOFF : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 keys = 8 packed P columns per MMA
+          const uint64_t vd = sw128_kmajor_desc(v + kk * 32);
+          a2_mma_ts(o, pp + kk * 8, vd, idesc_pv, (k > 0 || kk != 0) ? 1u : 0u);
+          a2_mma_ts(o, pp + 32 + kk * 8, vd, idesc_pv, 1u);
+          if (cur) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + kk * 32), idesc_pv, 1u);
+        }
+        tc_commit(&pv_done[hl][b]);
+      };
+      // PV of chunk k for every head once its P is written, then free chunk k's slots
+      auto pv_chunk = [&](int k) {
+        for (int hl = 0; hl < nh; ++hl) {
+          if (!mbar_wait(&p_ready[hl][k & 1], (uint32_t)(k >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
+            return false;
+          tc_fence_after();
+          issue_pv(hl, k);
+        }
+        for (int i = 0; i < mp.n[k & 1]; ++i) tc_commit(&kv_free[mp.slot[k & 1][i]]);
+        return true;
+      };
+
+      bool ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      for (int j = 0; j < nck && ok; ++j) {
+        mp.take(j, is_cur(j));
+        const bool pv_first = j >= 1 && mp.n[(j - 1) & 1] + mp.n[j & 1] > A2_SLOTS;
+        if (pv_first && !(ok = pv_chunk(j - 1))) break;
+        for (int i = 0; i < mp.n[j & 1] && ok; ++i)
+          ok = mbar_wait(&kv_full[mp.slot[j & 1][i]], (uint32_t)mp.use[j & 1][i] & 1u, &abort_s, p.err,
+                         DG_DEVERR_TIMEOUT_ATTN);
+        for (int hl = 0; hl < nh && ok; ++hl) {
+          // S/P buffer j & 1 was last read by PV(j - 2)
+          if (j >= 2)
+            ok = mbar_wait(&pv_done[hl][j & 1], (uint32_t)((j >> 1) - 1) & 1u, &abort_s, p.err,
+                           DG_DEVERR_TIMEOUT_ATTN);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(hl, j);
+        }
+        if (!ok) break;
+        if (j >= 1 && !pv_first) ok = pv_chunk(j - 1);
+      }
+      if (ok) pv_chunk(nck - 1);
+    }
+    __syncwarp();
+  } else if ((warp >> 2) < nh) {
+    // ================= softmax: head hl, query row `row` (TMEM lane), all 64 keys of a chunk
+    const int hl = warp >> 2;
+    const int h = h0 + hl;
+    const int row = (warp & 3) * 32 + lane;
+    const int my_row = q_row0 + row;
+    const int my_pos = p.q_pos0 + my_row;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int key_lim = p.causal ? min(p.n_keys, my_pos + 1) : p.n_keys;
+    float m_used = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nck && ok; ++j) {
+      const int b = j & 1;
+      ok = mbar_wait(&s_full[hl][b], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t spa = tmem + a2_sp(hl, b) + lane_off;
+      float s[A2_W];
+#pragma unroll
+      for (int c = 0; c < A2_W / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(spa + c * 16, r);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[i]) * p.scale_log2;
+      }
+      const int key0 = (c_begin + j) * A2_W;
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < A2_W; ++i) {
+        if (key0 + i >= key_lim) s[i] = -INFINITY;
+        cmax = fmaxf(cmax, s[i]);
+      }
+      const bool upd = cmax > m_used + 8.0f;
+      const float alpha = upd ? exp2f(m_used - cmax) : 1.0f;  // 0 while nothing was visible yet
+      // tcgen05.ld/st are warp-collective: the warp rescales its rows of O if any row must,
+      // once the previous chunk's PV is complete (O stable; PV(j) waits for this P)
+      if (__any_sync(0xffffffffu, upd && j > 0)) {
+        ok = mbar_wait(&pv_done[hl][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s, p.err,
+                       DG_DEVERR_TIMEOUT_ATTN);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t oa = tmem + a2_o(hl) + lane_off;
+#pragma unroll
+        for (int c = 0; c < A2_D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(oa + c * 16, r);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st16(oa + c * 16, r);
+        }
+      }
+      if (upd) {
+        l *= alpha;
+        m_used = cmax;
+      }
+      // P = exp2(s - m_used) as packed bf16 pairs over this row's S: hi in columns 0..31,
+      // lo in 32..63 (S was read into registers above)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // 32 keys -> 16 packed columns per store
+        uint32_t wh[16], wl[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i0 = c * 32 + 2 * e;
+          const float p0 = (s[i0] == -INFINITY) ? 0.0f : exp2f(s[i0] - m_used);
+          const float p1 = (s[i0 + 1] == -INFINITY) ? 0.0f : exp2f(s[i0 + 1] - m_used);
+          l += p0 + p1;
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
+          wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
+          wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+        }
+        tmem_st16(spa + c * 16, wh);
+        tmem_st16(spa + 32 + c * 16, wl);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[hl][b]);
+    }
+    if (ok)
+      ok = mbar_wait(&pv_done[hl][(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s, p.err,
+                     DG_DEVERR_TIMEOUT_ATTN);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = my_row < p.n_q;
+      const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+      const uint32_t oa = tmem + a2_o(hl) + lane_off;
+      if (p.n_splits == 1) {
+        const size_t base = (size_t)my_row * p.nq * A2_D + (size_t)h * A2_D;
+#pragma unroll
+        for (int c = 0; c < A2_D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(oa + c * 16, r);
+          tc_wait_ld();
+          if (valid) {
+            uint32_t w[8], wl[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a = __uint_as_float(r[2 * e]) * inv_l, bb = __uint_as_float(r[2 * e + 1]) * inv_l;
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(a, bb);
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), bb - __high2float(hi));
+              w[e] = *reinterpret_cast<const uint32_t*>(&hi);
+              wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.out + base + c * 16);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            if (p.out_lo) {
+              uint4* dl = reinterpret_cast<uint4*>(p.out_lo + base + c * 16);
+              dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+              dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+            }
+          }
+        }
+      } else {
+        float* po = p.part_o + (((size_t)sp * p.nq + h) * p.n_q + my_row) * A2_D;
+#pragma unroll
+        for (int c = 0; c < A2_D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(oa + c * 16, r);
+          tc_wait_ld();
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(po + c * 16);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv_l, __uint_as_float(r[4 * e + 1]) * inv_l,
+                                   __uint_as_float(r[4 * e + 2]) * inv_l, __uint_as_float(r[4 * e + 3]) * inv_l);
+          }
+        }
+        if (valid) p.part_lse[((size_t)sp * p.nq + h) * p.n_q + my_row] = (l > 0.0f) ? m_used + log2f(l) : -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+  if (abort_s) {
+    // wind down: let issued loads and MMAs land before the smem / TMEM go away
+    if (tid == A2_LOAD_WARP * 32) {
+      if (q_issued) mbar_wait_drain(&q_bar, 0);
+      for (int s = 0; s < A2_SLOTS; ++s)
+        if (loaded[s] > 0) mbar_wait_drain(&kv_full[s], (uint32_t)(loaded[s] - 1) & 1u);
+    }
+    if (tid == A2_MMA_WARP * 32) {
+      tc_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == A2_MMA_WARP) tmem_dealloc(tmem, 512);
+}
+
+int attn2_head_groups(int nq, int group) { return (group % 2 == 0) ? nq / 2 : nq; }
+
+cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
+                                 const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
+                                 const TcAttnParams& p, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(tc_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, A2_SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.n_q + A2_BQ - 1) / A2_BQ, attn2_head_groups(p.nq, p.group), p.n_splits);
+  return launch_k(tc_attn2_kernel, grid, dim3(A2_THREADS), A2_SMEM, st, Q, Ql, K, Vt, Kl, Vtl, p);
+}
+
+}  // namespace dg

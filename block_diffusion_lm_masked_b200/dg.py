@@ -106,6 +106,7 @@ def _load():
         "dg_debug_gemm_mx8": (I32, [P, P, P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_nv4": (I32, [P, P, F32, P, P, F32, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_attention_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
+        "dg_debug_attention_pair_bf16": (I32, [P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -518,6 +519,14 @@ def debug_attention_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out
     nkv, cap, _ = k.shape
     _check(lib.dg_debug_attention_bf16(_ptr(q), _ptr(k), _ptr(vt), cap, n_q, pos0, n_keys, 1 if causal else 0, nq,
                                        nkv, _ptr(out), _ptr(out_lo), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def debug_attention_pair_bf16(q, k, vt, n_keys, pos0, causal, out, ws: Workspace, out_lo=None, stream=None):
+    """The same attention through the head-pair kernel (see include/dg_debug.h)."""
+    nq, n_q, _ = q.shape
+    nkv, cap, _ = k.shape
+    _check(lib.dg_debug_attention_pair_bf16(_ptr(q), _ptr(k), _ptr(vt), cap, n_q, pos0, n_keys, 1 if causal else 0,
+                                            nq, nkv, _ptr(out), _ptr(out_lo), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def debug_bounded_wait(ws, timeout_ms, stream=None):

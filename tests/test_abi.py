@@ -387,3 +387,21 @@ def test_injected_launch_failure_is_a_clean_error_with_the_cache_unchanged():
     assert int(length) == 64
     assert "injected launch failure" in msg
     assert int(launches) == 0                          # failed before any launch was attempted
+
+
+@pytest.mark.parametrize("name", ["dg_debug_attention_bf16", "dg_debug_attention_pair_bf16"])
+def test_debug_attention_validation_on_host(name):
+    """Both attention entry points refuse bad shapes before touching any pointer."""
+    f = getattr(dg.lib, name)
+    P = ctypes.c_void_p(256)                     # never dereferenced: every call below is refused first
+    launches = dg.lib.dg_launch_count()
+    #        q     k  vt  cap  n_q pos0 n_keys causal nq nkv out out_lo ws   bytes
+    bad = [(None, P, P, 64, 8, 0, 8, 0, 2, 1, P, None, P, 1 << 20),      # NULL q
+           (P, P, P, 64, 8, 0, 8, 0, 3, 2, P, None, P, 1 << 20),         # nq not a multiple of nkv
+           (P, P, P, 60, 8, 0, 8, 0, 2, 1, P, None, P, 1 << 20),         # cap not a multiple of 8
+           (P, P, P, 64, 8, 0, 72, 0, 2, 1, P, None, P, 1 << 20),        # n_keys beyond cap
+           (P, P, P, 64, 8, 4, 8, 1, 2, 1, P, None, P, 1 << 20),         # causal rows past the keys
+           (P, P, P, 64, 0, 0, 8, 0, 2, 1, P, None, P, 1 << 20)]         # no query rows
+    for args in bad:
+        assert f(*args, None) == dg.DG_ERR_INVALID_ARG, args
+    assert dg.lib.dg_launch_count() == launches

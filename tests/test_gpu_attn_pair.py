@@ -1,0 +1,99 @@
+"""The head-pair attention kernel (dg_debug_attention_pair_bf16) against a plain fp32
+reference of the same attention and against today's kernel on the same inputs, then
+whole passes with it (DG_ATTN_PAIR=1) against the oracle, in a child process since the
+switch is read once per process."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
+                                 reason="the head-pair attention kernel has not yet run on a B200: "
+                                        "DG_RUN_NEW_GPU_TESTS=1 runs it")]
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dg():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from block_diffusion_lm_masked_b200 import dg as _dg
+    return _dg
+
+
+def _attn_ref(q, k, vt, n_keys, pos0, causal):
+    nq, n_q, d = q.shape
+    g = nq // k.shape[0]
+    kk = k[:, :n_keys].double()
+    vv = vt[:, :, :n_keys].double().transpose(1, 2)
+    pos = torch.arange(n_q, device="cuda") + pos0
+    keys = torch.arange(n_keys, device="cuda")
+    mask = keys[None, :] <= pos[:, None] if causal else torch.ones(n_q, n_keys, dtype=torch.bool, device="cuda")
+    out = torch.empty(n_q, nq * d, dtype=torch.float64, device="cuda")
+    for h in range(nq):
+        s = (q[h].double() @ kk[h // g].T) / d ** 0.5
+        s = s.masked_fill(~mask, float("-inf"))
+        out[:, h * d:(h + 1) * d] = torch.softmax(s, dim=1) @ vv[h // g]
+    return out
+
+
+def _run(dg, fn, nq, nkv, n_q, pos0, n_keys, causal, seed):
+    from block_diffusion_lm_masked_b200 import configs as CF
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    d, cap = 128, ((n_keys + 7) // 8) * 8 + 8
+
+    def bf(*shape):
+        return torch.randn(*shape, generator=g, device="cuda").to(torch.bfloat16)
+    q, k, vt = bf(nq, n_q, d), bf(nkv, cap, d), bf(nkv, d, cap)
+    cfg = dict(CF.CONFIGS["layer1_bf16"], n_q_heads=nq, n_kv_heads=nkv, hidden=128, expert_ffn=64, n_experts=1,
+               top_k=1, vocab=128, n_layers=1)
+    ws = dg.Workspace(cfg, n_q)
+    out = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device="cuda")
+    out_lo = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device="cuda")
+    fn(q, k, vt, n_keys, pos0, causal, out, ws, out_lo=out_lo)
+    dg.device_status(ws)
+    return q, k, vt, out.double() + out_lo.double()
+
+
+CASES = [
+    # nq, nkv, n_q, pos0, n_keys, causal
+    (4, 2, 100, 200, 300, False),      # canvas rows over a ragged prefix + canvas, head pairs
+    (16, 4, 256, 1024, 1280, False),   # the single-layer workload's shape: group 4, split-KV
+    (4, 1, 200, 50, 250, True),        # prefill rows, causal, ragged
+    (2, 2, 64, 4900, 4964, False),     # group 1: one head per CTA, long keys
+    (2, 1, 300, 0, 300, True),         # prefill from an empty cache
+    (8, 2, 256, 16128, 16384, False),  # long prefix: the most splits the workspace holds
+    (2, 1, 1024, 0, 1024, True),       # causal prefill with splits: early tiles' later splits are empty
+]
+
+
+@pytest.mark.parametrize("nq,nkv,n_q,pos0,n_keys,causal", CASES)
+def test_pair_kernel_matches_reference(dg, nq, nkv, n_q, pos0, n_keys, causal):
+    q, k, vt, got = _run(dg, dg.debug_attention_pair_bf16, nq, nkv, n_q, pos0, n_keys, causal, n_q + n_keys)
+    ref = _attn_ref(q, k, vt, n_keys, pos0, causal)
+    rms = ref.pow(2).mean().sqrt().item()
+    assert ((got - ref).abs() <= 1e-4 * ref.abs() + 1e-4 * rms).all(), (got - ref).abs().max().item()
+
+
+@pytest.mark.parametrize("nq,nkv,n_q,pos0,n_keys,causal", CASES[:4])
+def test_pair_kernel_agrees_with_the_single_head_kernel(dg, nq, nkv, n_q, pos0, n_keys, causal):
+    """Same inputs through both kernels: both carry fp32 accuracy, so they agree far
+    inside the reference tolerance."""
+    _, _, _, a = _run(dg, dg.debug_attention_pair_bf16, nq, nkv, n_q, pos0, n_keys, causal, 7)
+    _, _, _, b = _run(dg, dg.debug_attention_bf16, nq, nkv, n_q, pos0, n_keys, causal, 7)
+    rms = b.pow(2).mean().sqrt().item()
+    assert ((a - b).abs() <= 2e-5 * b.abs() + 2e-5 * rms).all(), (a - b).abs().max().item()
+
+
+def test_passes_with_pair_kernel_match_the_oracle():
+    """The pass parity tests (own-key low terms, causal prefill, chained canvases) with the
+    pass's attention routed through the head-pair kernel."""
+    env = dict(os.environ, DG_ATTN_PAIR="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "tests/test_gpu_parity.py",
+                        "-k", "small_bf16 or layer1_bf16 or prefill_append or chained"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
