@@ -1657,6 +1657,11 @@ static dg_status debug_attention(const void* q, const void* k, const void* vt, i
   Ws ws;
   dg_status s = check_ws(c, d_ws, ws_bytes, n_q, &ws);
   if (s != DG_OK) return s;
+  // the kernels read the low terms of the keys from the 128-aligned start at or below pos0
+  // up to n_keys out of the workspace's window (sized for n_q rows): that range must fit it
+  DG_CHECK_ARG(pos0 >= 0 && pos0 <= n_keys, "pos0 must lie in [0, n_keys]");
+  DG_CHECK_ARG(n_keys - (pos0 / 128) * 128 <= ws.L.lo_rows,
+               "keys from the 128-aligned start at or below pos0 exceed the workspace's low-term window");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // the pass reads q from the workspace's q buffer and writes o to its o buffer; the low
   // terms of q and of the current K/V are zero here (all inputs are bf16 already)

@@ -123,7 +123,10 @@ dg_status dg_debug_gemm_nv4(const void* W, const void* W_scales, float g, const 
  * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128] (hi part); out_lo (nullable)
  * receives the lo part, out + out_lo = the fp32 attention output to ~16 bits.  d_ws: a
  * workspace sized by dg_workspace_bytes for a config with these heads, hidden 128 and
- * >= n_q tokens. */
+ * >= n_q tokens.  As in the pass, the keys from the multiple of 128 at or below pos0 up
+ * to n_keys are read as the call's own (with zero low terms here); they must fit the
+ * workspace's window of ceil(n_q / 128) * 128 + 128 rows, which pos0 + n_q == n_keys
+ * always does.  0 <= pos0 <= n_keys.  Violations: DG_ERR_INVALID_ARG, nothing launched. */
 dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q, int32_t pos0,
                                   int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv, void* out, void* out_lo,
                                   void* d_ws, size_t ws_bytes, dg_stream stream);
