@@ -1,0 +1,521 @@
+"""Both attention kernels replayed at the address level on the CPU (tests/tc_emu.py): every
+TMA box, shared-memory offset, descriptor start, TMEM column, packed-P layout and output
+index as the kernel source computes it, in an order the kernel's barriers allow, against
+the oracle's attention at the GPU test's tolerance.
+
+tc_attn_kernel (validated on a B200) is the control: its transcription passing shows the
+hardware model is right.  The head-pair kernel (tc_attn2_kernel, not yet run) is replayed
+with its load warp running as far ahead as its slot plan lets it, so a slot reused too
+early, an S/P buffer overwritten before its PV, or a wrong column or offset changes the
+result.  Planted mistakes in the transcription are caught, which shows the replay is
+sharp enough to see them.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import tc_emu as T
+from oracle import dg_oracle as O
+from test_attn_geometry import lo_rows, splits_pair, splits_single
+
+D = 128
+NEG = np.float32(-np.inf)
+
+
+# ---------------------------------------------------------------- inputs
+def build(seed, nq, nkv, n_q, pos0, n_keys, causal):
+    """The attention of one pass: query (fp32 as bf16 hi + lo), the cache's bf16 K and V^T,
+    and the low terms of the call's own K/V (positions pos0 .. n_keys - 1) in a window of
+    rows counted from base = the multiple of 128 at or below pos0, zero before pos0."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((nq, n_q, D)).astype(np.float32)
+    q_hi = T.bf16_bits(q)
+    q_lo = T.bf16_bits(q - T.bf16_value(q_hi))
+    cap = -(-n_keys // 8) * 8 + 8
+    Kc = T.bf16_bits(rng.standard_normal((nkv, cap, D)).astype(np.float32))
+    Vc = T.bf16_bits(rng.standard_normal((nkv, cap, D)).astype(np.float32))
+    base = (pos0 // 128) * 128
+    Lc = lo_rows(n_q)
+    K_lo = np.zeros((nkv, Lc, D), np.uint16)
+    V_lo = np.zeros((nkv, Lc, D), np.uint16)
+    own = n_keys - pos0
+    K_lo[:, pos0 - base:n_keys - base] = T.bf16_bits(rng.standard_normal((nkv, own, D)).astype(np.float32) * 2 ** -9)
+    V_lo[:, pos0 - base:n_keys - base] = T.bf16_bits(rng.standard_normal((nkv, own, D)).astype(np.float32) * 2 ** -9)
+    pos = pos0 + np.arange(n_q)
+    key_lim = np.minimum(pos + 1, n_keys) if causal else np.full(n_q, n_keys)
+    return dict(nq=nq, nkv=nkv, n_q=n_q, pos0=pos0, n_keys=n_keys, causal=causal, base=base,
+                q_hi=q_hi, q_lo=q_lo, Kc=Kc, Vt=np.ascontiguousarray(Vc.transpose(0, 2, 1)), K_lo=K_lo,
+                Vt_lo=np.ascontiguousarray(V_lo.transpose(0, 2, 1)), key_lim=key_lim)
+
+
+def maps(c):
+    """The tensors the kernels' tensor maps cover (extents as the host encodes them)."""
+    nk, b = c["n_keys"], c["base"]
+    return dict(Q=c["q_hi"], Ql=c["q_lo"], K=c["Kc"][:, :nk, :], Vt=c["Vt"][:, :, :nk],
+                Kl=c["K_lo"][:, :nk - b, :], Vtl=c["Vt_lo"][:, :, :nk - b])
+
+
+def oracle(c):
+    nk, b = c["n_keys"], c["base"]
+    q = T.bf16_value(c["q_hi"]).astype(np.float64) + T.bf16_value(c["q_lo"])
+    K = T.bf16_value(c["Kc"][:, :nk]).astype(np.float64)
+    V = T.bf16_value(c["Vt"][:, :, :nk]).transpose(0, 2, 1).astype(np.float64)
+    K[:, b:] += T.bf16_value(c["K_lo"][:, :nk - b])
+    V[:, b:] += T.bf16_value(c["Vt_lo"][:, :, :nk - b]).transpose(0, 2, 1)
+    allowed = np.arange(nk)[None, :] < c["key_lim"][:, None]
+    out = O.attention(q, K, V, allowed)                       # [nq][n_q][d]
+    return out.transpose(1, 0, 2).reshape(c["n_q"], -1)
+
+
+def within(got, ref):
+    rms = math.sqrt(float(np.mean(ref * ref)))
+    return bool((np.abs(got - ref) <= 1e-4 * np.abs(ref) + 1e-4 * rms).all())
+
+
+# ---------------------------------------------------------------- shared pieces
+def softmax_chunk(s_raw, key0, key_lim, scale_log2, m_used, l):
+    """One chunk of a thread's row: scale, mask, lazy max; returns (s, rmax-applied state)."""
+    s = (s_raw.view(np.float32) * scale_log2).astype(np.float32)
+    keys = key0 + np.arange(s.shape[1])
+    s = np.where(keys[None, :] >= key_lim[:, None], NEG, s).astype(np.float32)
+    return s
+
+
+def p_words(s, m_used, l):
+    """P = exp2(s - m) for 2 x 16 keys at a time, packed hi / lo (as the kernels), and the
+    row sums accumulated pair by pair in fp32."""
+    n = s.shape[1]
+    with np.errstate(invalid="ignore", over="ignore"):
+        p = np.where(np.isneginf(s), np.float32(0), np.exp2((s - m_used[:, None]).astype(np.float32)))
+    p = p.astype(np.float32)
+    for e in range(0, n, 2):
+        l = (l + (p[:, e] + p[:, e + 1]).astype(np.float32)).astype(np.float32)
+    hi = T.bf16_value(T.bf16_bits(p))
+    lo = (p - hi).astype(np.float32)
+    wh = T.pack_bf16x2(p[:, 0::2], p[:, 1::2])
+    wl = T.pack_bf16x2(lo[:, 0::2], lo[:, 1::2])
+    return wh, wl, l
+
+
+def lazy_update(rmax, m_used, l, warp_rescale):
+    upd = rmax > m_used + np.float32(8.0)
+    with np.errstate(invalid="ignore"):
+        alpha = np.where(upd, np.exp2((m_used - rmax).astype(np.float32)), np.float32(1.0)).astype(np.float32)
+    any_w = np.repeat(np.array([upd[w * 32:(w + 1) * 32].any() for w in range(4)]), 32)
+    warp_rescale(any_w, alpha)
+    l = np.where(upd, (l * alpha).astype(np.float32), l).astype(np.float32)
+    m_used = np.where(upd, rmax, m_used).astype(np.float32)
+    return m_used, l
+
+
+def epilogue(tm, o_cols, l, m_used, rows, out, out_lo, part_o, part_lse, sp, h, n_splits, nq, n_q, col0=0, ncols=128):
+    inv = np.where(l > 0, (np.float32(1.0) / np.where(l > 0, l, 1)).astype(np.float32), np.float32(0)).astype(np.float32)
+    o = (tm.f32(o_cols, ncols) * inv[:, None]).astype(np.float32)
+    valid = rows < n_q
+    if n_splits == 1:
+        hi = T.bf16_value(T.bf16_bits(o))
+        lo = T.bf16_value(T.bf16_bits((o - hi).astype(np.float32)))
+        out[rows[valid], h * D + col0:h * D + col0 + ncols] = hi[valid]
+        out_lo[rows[valid], h * D + col0:h * D + col0 + ncols] = lo[valid]
+    else:
+        part_o[sp, h, rows[valid], col0:col0 + ncols] = o[valid]
+        if part_lse is not None:
+            with np.errstate(divide="ignore"):
+                lse = np.where(l > 0, m_used + np.log2(np.where(l > 0, l, 1)).astype(np.float32), NEG)
+            part_lse[sp, h, rows[valid]] = lse[valid]
+
+
+def merge(part_o, part_lse, n_splits):
+    mx = part_lse[:n_splits].max(axis=0)                        # [nq][n_q]
+    num = np.zeros(part_o.shape[1:], np.float32)
+    den = np.zeros(part_lse.shape[1:], np.float32)
+    for s in range(n_splits):
+        lse = part_lse[s]
+        with np.errstate(invalid="ignore"):
+            w = np.where(np.isneginf(lse), np.float32(0), np.exp2((lse - mx).astype(np.float32))).astype(np.float32)
+        num = (num + w[..., None] * part_o[s]).astype(np.float32)
+        den = (den + w).astype(np.float32)
+    v = np.where(den[..., None] > 0, num / np.where(den > 0, den, 1)[..., None], 0).astype(np.float32)
+    hi = T.bf16_value(T.bf16_bits(v))
+    lo = T.bf16_value(T.bf16_bits((v - hi).astype(np.float32)))
+    nq, n_q = v.shape[0], v.shape[1]
+    return (hi + lo).transpose(1, 0, 2).reshape(n_q, nq * D)
+
+
+# ---------------------------------------------------------------- tc_attn_kernel
+def run_single(c, bug=None):
+    """tc_attn_kernel: one head x 128 rows x 128-key chunks, two 64 KB slots (a current
+    chunk takes both), S in TMEM 0..127, P in 128.. / 384.. (hi, lo + 64), O in 256."""
+    nq, nkv, n_q, pos0, n_keys, causal = (c[k] for k in ("nq", "nkv", "n_q", "pos0", "n_keys", "causal"))
+    m = maps(c)
+    group = nq // nkv
+    n_splits, cps = splits_single(n_q, nq, n_keys)
+    HALF, SLOT = 128 * 128, 4 * 128 * 128
+    sQ, sQl, sSlot = 0, 2 * HALF, 4 * HALF
+    TM_S, TM_O = 0, 256
+    tm_phi = (lambda j: 128) if bug == "one_p_buffer" else (lambda j: 384 if j & 1 else 128)
+    scale = np.float32(1.4426950408889634 / math.sqrt(D))
+    out = np.zeros((n_q, nq * D), np.float32)
+    out_lo = np.zeros_like(out)
+    part_o = np.zeros((n_splits, nq, n_q, D), np.float32)
+    part_lse = np.full((n_splits, nq, n_q), NEG, np.float32)
+    for qt in range(-(-n_q // 128)):
+        for h in range(nq):
+            for sp in range(n_splits):
+                kvh = h // group
+                q_row0 = qt * 128
+                rows_here = min(128, n_q - q_row0)
+                kv_end = min(n_keys, pos0 + q_row0 + rows_here) if causal else n_keys
+                nch_total = -(-kv_end // 128)
+                c_begin = sp * cps
+                nck = min(nch_total, c_begin + cps) - c_begin
+                rows = q_row0 + np.arange(128)
+                if nck <= 0:
+                    continue                                  # empty partial: zeros, lse -inf
+                sm, tm = T.Smem(4 * HALF + 2 * SLOT), T.Tmem()
+                is_cur = lambda j: (c_begin + j) * 128 >= c["base"]
+                for off, mp, x in ((sQ, "Q", 0), (sQ + HALF, "Q", 64), (sQl, "Ql", 0), (sQl + HALF, "Ql", 64)):
+                    sm.tma_load_3d(off, m[mp], x, q_row0, h, 64, 128)
+
+                def load_slot(slot, mk, mv, krow, vx):
+                    k = sSlot + slot * SLOT
+                    v = k + 2 * HALF
+                    sm.tma_load_3d(k, m[mk], 0, krow, kvh, 64, 128)
+                    sm.tma_load_3d(k + HALF, m[mk], 64, krow, kvh, 64, 128)
+                    sm.tma_load_3d(v, m[mv], vx, 0, kvh, 64, 128)
+                    sm.tma_load_3d(v + HALF, m[mv], vx + 64, 0, kvh, 64, 128)
+
+                issued = [0]
+
+                def issue(j):
+                    key0 = (c_begin + j) * 128
+                    if is_cur(j):
+                        load_slot(0, "K", "Vt", key0, key0)
+                        load_slot(1, "Kl", "Vtl", key0 - c["base"], key0 - c["base"])
+                    else:
+                        load_slot(j & 1, "K", "Vt", key0, key0)
+                    issued[0] = j + 1
+
+                def issue_s(j):
+                    cur = is_cur(j)
+                    s_hi = 0 if cur else (j & 1)
+                    k, kl = sSlot + s_hi * SLOT, sSlot + SLOT
+                    for kb in range(2):
+                        for kk in range(4):
+                            off = kb * HALF + kk * 32
+                            T.mma_ss(tm, sm, TM_S, sQ + off, k + off, 128, 128, (kb | kk) != 0)
+                            T.mma_ss(tm, sm, TM_S, sQl + off, k + off, 128, 128, True)
+                            if cur:
+                                T.mma_ss(tm, sm, TM_S, sQ + off, kl + off, 128, 128, True)
+
+                def issue_pv(j):
+                    cur = is_cur(j)
+                    s_hi = 0 if cur else (j & 1)
+                    v = sSlot + s_hi * SLOT + 2 * HALF
+                    vl = sSlot + SLOT + 2 * HALF
+                    for kb in range(2):
+                        for kk in range(4):
+                            pcol = kb * 32 + kk * 8
+                            vd = v + kb * HALF + kk * 32
+                            T.mma_ts(tm, sm, TM_O, tm_phi(j) + pcol, vd, 128, 128, j > 0 or (kb | kk) != 0)
+                            T.mma_ts(tm, sm, TM_O, tm_phi(j) + 64 + pcol, vd, 128, 128, True)
+                            if cur:
+                                T.mma_ts(tm, sm, TM_O, tm_phi(j) + pcol, vl + kb * HALF + kk * 32, 128, 128, True)
+
+                # a PV issued by the control warp runs on the tensor pipe later: it is deferred
+                # until the next MMA issue (in-order pipe), an O rescale or the end, so the
+                # softmax of the next chunk writes its P while the PV is still pending
+                pending = []
+
+                def flush():
+                    while pending:
+                        issue_pv(pending.pop(0))
+
+                def mma_s(j):
+                    flush()
+                    issue_s(j)
+
+                m_used = np.full(128, NEG, np.float32)
+                lsum = [np.zeros(128, np.float32), np.zeros(128, np.float32)]
+                key_lim = np.array([c["key_lim"][r] if r < n_q else n_keys for r in rows])
+
+                def softmax(j):
+                    nonlocal m_used
+                    s_h, hmax = [], []
+                    for hf in range(2):
+                        raw = np.concatenate([tm.t[:, TM_S + hf * 64 + cc * 16:TM_S + hf * 64 + cc * 16 + 16]
+                                              for cc in range(4)], axis=1)
+                        s = softmax_chunk(raw, (c_begin + j) * 128 + hf * 64, key_lim, scale, None, None)
+                        s_h.append(s)
+                        hmax.append(s.max(axis=1))
+                    rmax = np.maximum(hmax[0], hmax[1])
+                    for hf in range(2):
+                        def rescale(any_w, alpha, hf=hf):
+                            if j > 0 and any_w.any():
+                                flush()                       # waits for PV(j - 1)
+                                sel = any_w
+                                blk = tm.f32(TM_O + hf * 64, 64)
+                                blk[sel] = (blk[sel] * alpha[sel, None]).astype(np.float32)
+                        mu, lsum[hf] = lazy_update(rmax, m_used, lsum[hf], rescale)
+                    m_used = mu
+                    for hf in range(2):
+                        wh, wl, lsum[hf] = p_words(s_h[hf], m_used, lsum[hf])
+                        tm.t[:, tm_phi(j) + hf * 32:tm_phi(j) + hf * 32 + 32] = wh
+                        tm.t[:, tm_phi(j) + 64 + hf * 32:tm_phi(j) + 64 + hf * 32 + 32] = wl
+
+                issue(0)
+                if nck > 1 and not is_cur(0) and not is_cur(1):
+                    issue(1)
+                pv_next = 0
+                for j in range(nck):
+                    cur = is_cur(j)
+                    if issued[0] <= j:
+                        if j >= 1 and pv_next == j - 1:
+                            pending.append(j - 1)             # do_pv waits for its completion
+                            flush()
+                            pv_next = j
+                        issue(j)
+                    mma_s(j)
+                    # the softmax warps need only S(j): they may write P(j) before PV(j - 1),
+                    # which the control warp issues after S(j), has run
+                    softmax(j)
+                    if j >= 1 and pv_next == j - 1:
+                        pending.append(j - 1)
+                        flush()                               # do_pv waits for it before any load
+                        pv_next = j
+                    if issued[0] == j + 1 and j + 1 < nck and not cur and not is_cur(j + 1):
+                        issue(j + 1)
+                if pv_next == nck - 1:
+                    pending.append(nck - 1)
+                flush()
+                l = (lsum[0] + lsum[1]).astype(np.float32)
+                for hf in range(2):
+                    epilogue(tm, TM_O + hf * 64, l, m_used, rows, out, out_lo, part_o,
+                             part_lse if hf == 0 else None, sp, h, n_splits, nq, n_q, col0=hf * 64, ncols=64)
+    return (out + out_lo) if n_splits == 1 else merge(part_o, part_lse, n_splits)
+
+
+# ---------------------------------------------------------------- tc_attn2_kernel
+def run_pair(c, bug=None):
+    """tc_attn2_kernel: a head pair (one head for odd groups) x 128 rows x 64-key chunks,
+    three 32 KB slots, per head S/P buffers at 256 hl + 64 b and O at 256 hl + 128."""
+    nq, nkv, n_q, pos0, n_keys, causal = (c[k] for k in ("nq", "nkv", "n_q", "pos0", "n_keys", "causal"))
+    m = maps(c)
+    group = nq // nkv
+    n_splits, cps = splits_pair(n_q, nq, group, n_keys)
+    W, QBLK, KBLK = 64, 128 * 128, 64 * 128
+    QHEAD, VOFF = 4 * QBLK, 2 * KBLK
+    SLOT = VOFF + QBLK
+    SLOTS = 3
+    sQ, sSlot = 0, 2 * QHEAD
+    a2_sp = (lambda hl, b: hl * 256) if bug == "one_sp_buffer" else (lambda hl, b: hl * 256 + b * 64)
+    a2_o = lambda hl: hl * 256 + 128
+    if bug == "p_lo_offset":
+        p_lo = 16
+    else:
+        p_lo = 32
+    scale = np.float32(1.4426950408889634 / math.sqrt(D))
+    nh = 2 if group % 2 == 0 else 1
+    out = np.zeros((n_q, nq * D), np.float32)
+    out_lo = np.zeros_like(out)
+    part_o = np.zeros((n_splits, nq, n_q, D), np.float32)
+    part_lse = np.full((n_splits, nq, n_q), NEG, np.float32)
+    for qt in range(-(-n_q // 128)):
+        for y in range(nq // nh):
+            h0 = y * nh
+            kvh = h0 // group
+            for sp in range(n_splits):
+                q_row0 = qt * 128
+                rows_here = min(128, n_q - q_row0)
+                kv_end = min(n_keys, pos0 + q_row0 + rows_here) if causal else n_keys
+                nch_total = -(-kv_end // W)
+                c_begin = sp * cps
+                nck = min(nch_total, c_begin + cps) - c_begin
+                rows = q_row0 + np.arange(128)
+                if nck <= 0:
+                    continue
+                sm, tm = T.Smem(2 * QHEAD + SLOTS * SLOT), T.Tmem()
+                is_cur = lambda j: (c_begin + j) * W >= c["base"]
+                for hl in range(nh):
+                    q = sQ + hl * QHEAD
+                    for off, mp, x in ((0, "Q", 0), (QBLK, "Q", 64), (2 * QBLK, "Ql", 0), (3 * QBLK, "Ql", 64)):
+                        sm.tma_load_3d(q + off, m[mp], x, q_row0, h0 + hl, 64, 128)
+                # the slot plan (SlotPlan::take), and which chunk's PV frees each slot use
+                plan, nxt, uses = [], 0, [0] * SLOTS
+                for j in range(nck):
+                    parts = []
+                    for _ in range(2 if is_cur(j) else 1):
+                        parts.append((nxt, uses[nxt]))
+                        uses[nxt] += 1
+                        nxt = (nxt + 1) % SLOTS
+                    plan.append(parts)
+                if bug == "two_slots":                        # a ring one slot short, same plan
+                    plan = [[(s % 2, u) for s, u in parts] for parts in plan]
+                holder = {}                                   # slot -> chunk whose loads it holds until its PV
+                loaded = [0]                                  # chunks loaded so far (in order)
+
+                def pump():
+                    """The load warp: the next chunk's slots, each once its previous use was freed."""
+                    while loaded[0] < nck:
+                        j = loaded[0]
+                        if any(s in holder for s, _ in plan[j]):
+                            return
+                        key0 = (c_begin + j) * W
+                        for i, (s, _) in enumerate(plan[j]):
+                            k = sSlot + s * SLOT
+                            mk, mv = ("K", "Vt") if i == 0 else ("Kl", "Vtl")
+                            krow = key0 if i == 0 else key0 - c["base"]
+                            sm.tma_load_3d(k, m[mk], 0, krow, kvh, 64, 64)
+                            sm.tma_load_3d(k + KBLK, m[mk], 64, krow, kvh, 64, 64)
+                            sm.tma_load_3d(k + VOFF, m[mv], krow, 0, kvh, 64, 128)
+                            holder[s] = j
+                        loaded[0] += 1
+
+                def issue_s(hl, j):
+                    b = j & 1
+                    cur = len(plan[j]) == 2
+                    d = a2_sp(hl, b)
+                    q, ql = sQ + hl * QHEAD, sQ + hl * QHEAD + 2 * QBLK
+                    k = sSlot + plan[j][0][0] * SLOT
+                    kl = sSlot + plan[j][1][0] * SLOT if cur else 0
+                    for kb in range(2):
+                        for kk in range(4):
+                            oq, okb = kb * QBLK + kk * 32, kb * KBLK + kk * 32
+                            T.mma_ss(tm, sm, d, q + oq, k + okb, 128, W, (kb | kk) != 0)
+                            T.mma_ss(tm, sm, d, ql + oq, k + okb, 128, W, True)
+                            if cur:
+                                T.mma_ss(tm, sm, d, q + oq, kl + okb, 128, W, True)
+
+                def issue_pv(hl, k_):
+                    b = k_ & 1
+                    cur = len(plan[k_]) == 2
+                    o, pp = a2_o(hl), a2_sp(hl, b)
+                    v = sSlot + plan[k_][0][0] * SLOT + VOFF
+                    vl = sSlot + plan[k_][1][0] * SLOT + VOFF if cur else 0
+                    for kk in range(4):
+                        vd = v + kk * 32
+                        T.mma_ts(tm, sm, o, pp + kk * 8, vd, 128, D, k_ > 0 or kk != 0)
+                        T.mma_ts(tm, sm, o, pp + p_lo + kk * 8, vd, 128, D, True)
+                        if cur:
+                            T.mma_ts(tm, sm, o, pp + kk * 8, vl + kk * 32, 128, D, True)
+
+                def pv_run(k_):
+                    for hl in range(nh):
+                        issue_pv(hl, k_)
+                    for s, _ in plan[k_]:                    # the commits free chunk k_'s slots
+                        if holder.get(s) == k_:
+                            del holder[s]
+                    pump()
+
+                # issued PVs run on the tensor pipe later: deferred until the next MMA issue
+                # (in-order pipe), an O rescale, a wait for a slot, or the end
+                pending = []
+
+                def flush():
+                    while pending:
+                        pv_run(pending.pop(0))
+
+                def pv_chunk(k_):
+                    pending.append(k_)
+
+                m_used = [np.full(128, NEG, np.float32) for _ in range(nh)]
+                lsum = [np.zeros(128, np.float32) for _ in range(nh)]
+                key_lim = np.array([c["key_lim"][r] if r < n_q else n_keys for r in rows])
+
+                def softmax(hl, j):
+                    b = j & 1
+                    spa = a2_sp(hl, b)
+                    raw = np.concatenate([tm.t[:, spa + cc * 16:spa + cc * 16 + 16] for cc in range(4)], axis=1)
+                    s = softmax_chunk(raw, (c_begin + j) * W, key_lim, scale, None, None)
+
+                    def rescale(any_w, alpha):
+                        if j > 0 and any_w.any():
+                            flush()                           # waits for PV(j - 1)
+                            blk = tm.f32(a2_o(hl), D)
+                            blk[any_w] = (blk[any_w] * alpha[any_w, None]).astype(np.float32)
+                    m_used[hl], lsum[hl] = lazy_update(s.max(axis=1), m_used[hl], lsum[hl], rescale)
+                    wh, wl, lsum[hl] = p_words(s, m_used[hl], lsum[hl])
+                    tm.t[:, spa:spa + 32] = wh                # P over this row's S: hi, then lo
+                    tm.t[:, spa + p_lo:spa + p_lo + 32] = wl
+
+                pump()
+                for j in range(nck):
+                    pv_first = j >= 1 and len(plan[j - 1]) + len(plan[j]) > SLOTS
+                    if bug == "no_pv_first":
+                        pv_first = False
+                    if pv_first:
+                        pv_chunk(j - 1)
+                    if loaded[0] <= j:
+                        flush()                               # the slots come free as pending PVs complete
+                    assert loaded[0] > j, "the MMA warp would wait for a chunk the load warp cannot load"
+                    flush()
+                    for hl in range(nh):
+                        issue_s(hl, j)
+                    if j >= 1 and not pv_first:
+                        pv_chunk(j - 1)
+                    for hl in range(nh):
+                        softmax(hl, j)
+                pv_chunk(nck - 1)
+                flush()
+                for hl in range(nh):
+                    epilogue(tm, a2_o(hl), lsum[hl], m_used[hl], rows, out, out_lo, part_o, part_lse, sp, h0 + hl,
+                             n_splits, nq, n_q)
+    return (out + out_lo) if n_splits == 1 else merge(part_o, part_lse, n_splits)
+
+
+CASES = [
+    # seed, nq, nkv, n_q, pos0, n_keys, causal
+    (1, 4, 2, 100, 200, 300, False),       # canvas over a ragged prefix, head pairs, own-key chunks
+    (2, 4, 1, 200, 50, 250, True),         # causal prefill rows, ragged tiles
+    (3, 2, 2, 64, 600, 664, False),        # group 1: one head per CTA
+    (4, 2, 1, 128, 1536, 1664, False),     # long prefix: several splits and a merge
+    (5, 2, 1, 300, 0, 300, True),          # causal from an empty cache: own keys throughout
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_validated_kernel_replay_matches_the_oracle(case):
+    """The control: the kernel that passes on a B200 passes in the model too."""
+    c = build(*case)
+    assert within(run_single(c), oracle(c))
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_head_pair_kernel_replay_matches_the_oracle(case):
+    c = build(*case)
+    assert within(run_pair(c), oracle(c))
+
+
+@pytest.mark.parametrize("bug", ["p_lo_offset", "no_pv_first"])
+def test_planted_mistakes_in_the_head_pair_replay_are_caught(bug):
+    """A P lo block written half-way into the hi block, or the plain issue order where two
+    own-key chunks follow each other: either gives a wrong result or cannot proceed."""
+    c = build(5, 2, 1, 300, 0, 300, True)
+    try:
+        ok = within(run_pair(c, bug=bug), oracle(c))
+    except AssertionError:
+        ok = False
+    assert not ok
+
+
+@pytest.mark.parametrize("kernel,bug", [("single", "one_p_buffer"), ("pair", "one_sp_buffer")])
+def test_a_single_p_buffer_is_caught(kernel, bug):
+    """One P buffer where the kernels keep two: the next chunk's softmax writes its P while
+    the previous chunk's PV is still to run, which the replay's order allows."""
+    c = build(4, 2, 1, 128, 1536, 1664, False)
+    run = run_single if kernel == "single" else run_pair
+    assert within(run(c), oracle(c))
+    assert not within(run(c, bug=bug), oracle(c))
+
+
+def test_a_ring_one_slot_short_is_caught():
+    """Two slots for the three-slot plan: chunks overwrite K/V still to be read."""
+    c = build(1, 4, 2, 100, 200, 300, False)
+    try:
+        ok = within(run_pair(c, bug="two_slots"), oracle(c))
+    except AssertionError:
+        ok = False
+    assert not ok
