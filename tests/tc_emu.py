@@ -36,6 +36,13 @@ def sw128(addr: np.ndarray) -> np.ndarray:
     return addr ^ (((addr >> 7) & 7) << 4)
 
 
+def swizzle(addr: np.ndarray, span: int) -> np.ndarray:
+    """TMA swizzle modes: 16-byte chunk bits XORed with the bits above 128 bytes, three
+    (128-byte span), two (64) or one (32); span 0 is no swizzle."""
+    mask = {128: 7, 64: 3, 32: 1, 0: 0}[span]
+    return addr ^ (((addr >> 7) & mask) << 4)
+
+
 class Smem:
     def __init__(self, nbytes: int):
         self.b = np.zeros(nbytes, dtype=np.uint8)
@@ -59,6 +66,31 @@ class Smem:
         raw = box.view(np.uint8).reshape(by, row_bytes)
         L = dst + np.arange(by)[:, None] * row_bytes + np.arange(row_bytes)[None, :]
         phys = sw128(L) if swizzle else L
+        assert phys.max() < self.b.size
+        self.b[phys.ravel()] = raw.ravel()
+        self.bytes_loaded += by * row_bytes
+
+    def tma_load(self, dst: int, tensor: np.ndarray, coords, box, span: int):
+        """Tile load of a 2-D or 3-D tensor (numpy, innermost axis last) at coords (x, y[, z])
+        with box (bx, by[, 1]); rows of the box are bx elements, written one after another
+        from dst through the given swizzle; elements outside the tensor read as zero."""
+        es = tensor.dtype.itemsize
+        x, y = coords[0], coords[1]
+        z = coords[2] if len(coords) > 2 else 0
+        bx, by = box[0], box[1]
+        assert (x * es) % 16 == 0, "TMA x coordinate not on a 16-byte boundary"
+        assert span == 0 or (bx * es == span and dst % (8 * span if span else 1) == 0 and dst % 128 == 0)
+        t3 = tensor if tensor.ndim == 3 else tensor[None]
+        d2, d1, d0 = t3.shape
+        blk = np.zeros((by, bx), dtype=tensor.dtype)
+        ys, xs = np.arange(y, y + by), np.arange(x, x + bx)
+        okr, okc = (ys >= 0) & (ys < d1), (xs >= 0) & (xs < d0)
+        if 0 <= z < d2:
+            blk[np.ix_(okr, okc)] = t3[z][np.ix_(ys[okr], xs[okc])]
+        row_bytes = bx * es
+        raw = blk.view(np.uint8).reshape(by, row_bytes)
+        L = dst + np.arange(by)[:, None] * row_bytes + np.arange(row_bytes)[None, :]
+        phys = swizzle(L, span)
         assert phys.max() < self.b.size
         self.b[phys.ravel()] = raw.ravel()
         self.bytes_loaded += by * row_bytes
