@@ -274,13 +274,17 @@ def run_variant(args, cfg, name):
     world, rank = ranks.world, ranks.rank
     from block_diffusion_lm_masked_b200 import dg
 
-    B, lowp = args.canvases, args.experts
+    B, lowp, vlowp = args.canvases, args.experts, args.vocab
     P, C, V, k = cfg["prefix"], cfg["canvas"], cfg["vocab"], cfg["top_k"]
     model = dg.Model(synth.Model(cfg), dev)
     if lowp == "mx8":
         model.set_experts_mx8(synth.mx8_experts(cfg))
     elif lowp == "nv4":
         model.set_experts_nv4(synth.nv4_experts(cfg))
+    if vlowp == "mx8":
+        model.set_vocab_mx8(synth.mx8_vocab(cfg))
+    elif vlowp == "nv4":
+        model.set_vocab_nv4(synth.nv4_vocab(cfg))
     caches = []
     for b in range(B):
         c = dg.KVCache(cfg, ((P + C + 7) // 8) * 8, dev)
@@ -364,8 +368,9 @@ def run_variant(args, cfg, name):
 
     hbm, tf_burst, _, peak_src = _peaks()
     ew = {"mx8": RF.MX8_WBYTES, "nv4": RF.NV4_WBYTES}.get(lowp)
+    vw = {"mx8": RF.MX8_WBYTES, "nv4": RF.NV4_WBYTES}.get(vlowp)
     flops = B * RF.pass_flops(cfg, P, C)
-    nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew) + B * 8 * C
+    nbytes = RF.pass_bytes_batched(cfg, [P] * B, C, unions_h, ew, vw) + B * 8 * C
     if args.fused_update:  # no logits written or read back: the tile records instead
         nbytes += 2 * 16 * C * ((V + 127) // 128) - 2 * 4 * C * V
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
@@ -387,6 +392,8 @@ def run_variant(args, cfg, name):
                    "update": "fused into the vocabulary projection" if args.fused_update else "two kernels on logits",
                    "experts": {"bf16": "bf16", "mx8": "mx8 (E4M3 + E8M0 per 32, synthetic codes)",
                                "nv4": "nv4 (E2M1 + E4M3 per 16 + fp32 tensor scale, synthetic codes)"}[lowp],
+                   "vocab_weights": {"bf16": "bf16", "mx8": "mx8 (E4M3 + E8M0 per 32, synthetic codes)",
+                                     "nv4": "nv4 (E2M1 + E4M3 per 16 + fp32 tensor scale, synthetic codes)"}[vlowp],
                    "l2": "flushed between steps (256 MB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "expert_union": unions_h},
         "roofline": roof,
@@ -419,6 +426,8 @@ def main():
                          "projection's epilogue (no logits)")
     ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8", "nv4"],
                     help="expert weight storage; mx8 and nv4 run through the batched calls")
+    ap.add_argument("--vocab", default="bf16", choices=["bf16", "mx8", "nv4"],
+                    help="output-matrix storage; mx8 and nv4 run through the batched calls")
     args = ap.parse_args()
     name = args.workload
     cfg = CF.CONFIGS[name]
@@ -426,9 +435,9 @@ def main():
         return run_reference(args, cfg, name)
     if args.canvases < 1:
         ap.error("--canvases must be >= 1")
-    if args.fused_update and (args.canvases > 1 or args.experts != "bf16"):
-        ap.error("--fused-update runs one canvas with bf16 experts")
-    if args.canvases > 1 or args.experts != "bf16" or args.fused_update:
+    if args.fused_update and (args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16"):
+        ap.error("--fused-update runs one canvas with bf16 experts and output matrix")
+    if args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16" or args.fused_update:
         return run_variant(args, cfg, name)
 
     import torch

@@ -248,6 +248,14 @@ struct LowpMaps {
   int fmt;
   float g_gate, g_up, g_down;
 };
+// the output matrix in low precision: codes and block scales of W_out [V][H], the format
+// and the 4-bit tensor scale
+struct VocabLowp {
+  CUtensorMap codes, scales;
+  int fmt = 0;
+  float g = 1.0f;
+  bool on = false;
+};
 struct dg_model {
   dg_config cfg;
   const void* embed;
@@ -256,6 +264,7 @@ struct dg_model {
   std::vector<LayerMaps> maps;
   CUtensorMap out_map;
   std::vector<LowpMaps> lowp;  // non-empty: the batched calls run the experts from low-precision weights
+  VocabLowp vocab_lowp;        // on: the batched calls project to the vocabulary from low-precision weights
   bool taps_on = false;
   std::vector<float*> tap_x_attn, tap_x_out, tap_topk_w;
   std::vector<int32_t*> tap_topk_idx, tap_counts, tap_perm;
@@ -1289,7 +1298,14 @@ extern "C" dg_status dg_denoise_pass_batched(dg_model* m, const dg_kv_cache* cac
   s = is_bf16(c) ? run_stack_batched<bf16>(m, caches, B, d_canvases, C, false, ws, st)
                  : run_stack_batched<float>(m, caches, B, d_canvases, C, false, ws, st);
   if (s != DG_OK) return s;
-  if (is_bf16(c)) {
+  if (is_bf16(c) && m->vocab_lowp.on) {
+    // dense low-precision GEMM: tokens in chunks of 64, tiles weight tile major
+    const VocabLowp& Vl = m->vocab_lowp;
+    GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &Vl.codes, nullptr, ws.at<void>(ws.L.xn), nullptr, n, c.hidden,
+               c.vocab, nullptr, nullptr, ceil_div(n, kItemRowsMx8), kItemRowsMx8, d_logits, nullptr, c.vocab, 1, 0,
+               kSmemGemm};
+    if ((s = gemm_lowp(g, Vl.fmt, &Vl.scales, nullptr, Vl.g, 1.0f, ws.err(), st)) != DG_OK) return s;
+  } else if (is_bf16(c)) {
     GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, n, c.hidden,
                c.vocab, nullptr, nullptr, 0, 256, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm};
     if ((s = gemm_bf16(g, ws.err(), st)) != DG_OK) return s;
@@ -1388,6 +1404,38 @@ extern "C" dg_status dg_model_set_experts_nv4(dg_model* m, const dg_expert_weigh
                                               const float* tensor_scales) {
   DG_CHECK_ARG(!layers || tensor_scales, "4-bit experts need their tensor scales");
   return set_experts_lowp(m, dg::FMT_NV4, layers, tensor_scales);
+}
+
+static dg_status set_vocab_lowp(dg_model* m, int fmt, const void* codes, const void* scales, float g) {
+  DG_CHECK_ARG(m, "model is NULL");
+  if (!codes) {
+    m->vocab_lowp.on = false;
+    return DG_OK;
+  }
+  const dg_config& c = m->cfg;
+  DG_CHECK_ARG(is_bf16(c), "low-precision vocabulary weights need a bf16 model");
+  auto a16 = [](const void* q) { return q && (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  DG_CHECK_ARG(a16(codes) && a16(scales), "vocabulary codes and scales must be non-NULL and 16-byte aligned");
+  DG_CHECK_ARG(isfinite(g), "the tensor scale must be finite");
+  VocabLowp v;
+  const uint64_t V = c.vocab, H = c.hidden;
+  dg_status s = fmt == dg::FMT_NV4 ? map_codes4(&v.codes, codes, 1, V, H) : map_codes(&v.codes, codes, 1, V, H);
+  if (s == DG_OK)
+    s = fmt == dg::FMT_NV4 ? map_scales4(&v.scales, scales, 1, V, H) : map_scales(&v.scales, scales, 1, V, H);
+  if (s != DG_OK) return s;
+  v.fmt = fmt;
+  v.g = g;
+  v.on = true;
+  m->vocab_lowp = v;
+  return DG_OK;
+}
+
+extern "C" dg_status dg_model_set_vocab_mx8(dg_model* m, const void* codes, const void* scales) {
+  return set_vocab_lowp(m, dg::FMT_MX8, codes, scales, 1.0f);
+}
+
+extern "C" dg_status dg_model_set_vocab_nv4(dg_model* m, const void* codes, const void* scales, float tensor_scale) {
+  return set_vocab_lowp(m, dg::FMT_NV4, codes, scales, tensor_scale);
 }
 
 extern "C" dg_status dg_generate_canvases_masked(dg_model* m, dg_kv_cache* caches, int32_t B, int32_t* d_canvases,

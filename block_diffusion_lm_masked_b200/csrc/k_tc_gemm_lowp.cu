@@ -66,19 +66,23 @@ __device__ __forceinline__ int mx_total_items(const TcGemmParams& p) {
   return (p.n_tokens + p.n_max - 1) / p.n_max;
 }
 
-// tile t -> (work item t / m_tiles, weight tile t % m_tiles)
+// Grouped: tile t -> (work item t / m_tiles, weight tile t % m_tiles), so the tiles running
+// together cover one item's weight rows.  Dense (one weight matrix, tokens in chunks of
+// n_max): tile t -> (weight tile t / chunks, token chunk t % chunks), so the CTAs that share
+// a weight tile run together and read it from DRAM once between them (L2 serves the rest).
 __device__ __forceinline__ MxTile mx_decode_tile(const TcGemmParams& p, int t) {
   MxTile ti;
-  const int item = t / p.m_tiles;
-  ti.m = t % p.m_tiles;
   if (p.items) {
-    const TcWorkItem it = p.items[item];
+    const TcWorkItem it = p.items[t / p.m_tiles];
+    ti.m = t % p.m_tiles;
     ti.g = it.group;
     ti.row0 = it.row0;
     ti.rows = it.rows;
   } else {
+    const int chunks = (p.n_tokens + p.n_max - 1) / p.n_max;
+    ti.m = t / chunks;
     ti.g = 0;
-    ti.row0 = item * p.n_max;
+    ti.row0 = (t % chunks) * p.n_max;
     ti.rows = min(p.n_max, p.n_tokens - ti.row0);
   }
   return ti;

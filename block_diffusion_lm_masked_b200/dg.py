@@ -91,6 +91,8 @@ def _load():
         "dg_generate_canvases_masked": (I32, [P, P, I32, P, I32, I32, F32, F32, I32, I32, P, P, SZ, P]),
         "dg_model_set_experts_mx8": (I32, [P, P]),
         "dg_model_set_experts_nv4": (I32, [P, P, P]),
+        "dg_model_set_vocab_mx8": (I32, [P, P, P]),
+        "dg_model_set_vocab_nv4": (I32, [P, P, P, F32]),
         "dg_device_status": (I32, [P, P]),
         "dg_last_error": (ctypes.c_char_p, []),
         "dg_set_taps": (I32, [P, ctypes.POINTER(Taps)]),
@@ -225,6 +227,33 @@ class Model:
         g_arr = (ctypes.c_float * len(gs))(*gs)
         _check(lib.dg_model_set_experts_nv4(self.handle, arr, g_arr))
         self._lowp = keep
+
+    def set_vocab_mx8(self, vocab: tuple | None):
+        """vocab: (codes uint8 [V][H], block exponents [V][H / 32]) for the output matrix;
+        None returns to the bf16 W_out.  Used by the batched calls."""
+        if vocab is None:
+            _check(lib.dg_model_set_vocab_mx8(self.handle, None, None))
+            self._lowp_vocab = None
+            return
+        codes, exps = vocab
+        c = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).to(self.device)
+        sc = torch.from_numpy(pack_mx8_scales(np.asarray(exps)[None])[0]).to(self.device)
+        _check(lib.dg_model_set_vocab_mx8(self.handle, ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(sc.data_ptr())))
+        self._lowp_vocab = (c, sc)
+
+    def set_vocab_nv4(self, vocab: tuple | None):
+        """vocab: (codes uint8 [V][H] one 4-bit code per byte, E4M3 block-scale codes
+        [V][H / 16], tensor scale g); None returns to the bf16 W_out."""
+        if vocab is None:
+            _check(lib.dg_model_set_vocab_nv4(self.handle, None, None, 1.0))
+            self._lowp_vocab = None
+            return
+        codes, sc, g = vocab
+        c = torch.from_numpy(pack_nv4_codes(np.asarray(codes)[None])[0]).to(self.device)
+        s_ = torch.from_numpy(pack_nv4_scales(np.asarray(sc)[None])[0]).to(self.device)
+        _check(lib.dg_model_set_vocab_nv4(self.handle, ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(s_.data_ptr()),
+                                          float(g)))
+        self._lowp_vocab = (c, s_)
 
     def set_taps(self, taps: dict | None):
         """taps: name -> list (per layer) of device tensors sized for taps['rows'] tokens,

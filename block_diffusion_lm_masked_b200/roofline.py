@@ -77,9 +77,11 @@ def pass_bytes(cfg: dict, P: int, C: int, unions, ew: float | None = None) -> fl
     return pass_bytes_batched(cfg, [P], C, unions, ew)
 
 
-def pass_bytes_batched(cfg: dict, prefixes, C: int, unions, ew: float | None = None) -> float:
+def pass_bytes_batched(cfg: dict, prefixes, C: int, unions, ew: float | None = None,
+                       vw: float | None = None) -> float:
     """A pass over one canvas of C positions per cache prefix in `prefixes`: every weight
-    once (the experts of the batch's union), each canvas's K/V and logits traffic."""
+    once (the experts of the batch's union), each canvas's K/V and logits traffic.  `ew`
+    and `vw`: bytes per expert and per output-matrix weight (default: the model dtype's)."""
     H, nkv, d, E, V = cfg["hidden"], cfg["n_kv_heads"], cfg["head_dim"], cfg["n_experts"], cfg["vocab"]
     b = wbytes(cfg)
     B = len(prefixes)
@@ -89,7 +91,7 @@ def pass_bytes_batched(cfg: dict, prefixes, C: int, unions, ew: float | None = N
         for P in prefixes:
             total += b * 2 * nkv * d * (P + C)    # K/V read (cached prefix + canvas)
             total += b * 2 * nkv * d * C          # canvas K/V written
-    total += b * V * H + B * (4 * C * V + 4 * C * V)   # output matrix, logits write + read
+    total += (b if vw is None else vw) * V * H + B * (4 * C * V + 4 * C * V)   # output matrix, logits write + read
     return total
 
 

@@ -110,6 +110,8 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 TID_EMBED = 1
 TID_W_OUT = 2
 TID_PREFIX_TOKENS = 3
+TID_W_OUT_MX8 = 4
+TID_W_OUT_NV4 = 5
 
 
 def tid_canvas_noise(canvas_index: int) -> int:
@@ -205,6 +207,21 @@ def nv4_experts(cfg: dict, seed: int = SEED_WEIGHTS):
                        2.0 ** -6)
         out.append(d)
     return out
+
+
+def mx8_vocab(cfg: dict, seed: int = SEED_WEIGHTS):
+    """Synthetic 8-bit output matrix drawn directly as MX-FP8 data, as mx8_experts: codes
+    uint8 [V][H] and every block exponent -12 (one per 32 elements)."""
+    V, H = cfg["vocab"], cfg["hidden"]
+    return _codes8(seed, TID_W_OUT_MX8, (V, H), 0x70), np.full((V, H // 32), -12, dtype=np.int32)
+
+
+def nv4_vocab(cfg: dict, seed: int = SEED_WEIGHTS):
+    """Synthetic 4-bit output matrix drawn directly as NVFP4-style data, as nv4_experts:
+    one E2M1 code per byte [V][H], every block scale code 0x28 (0.25), tensor scale 2^-6."""
+    V, H = cfg["vocab"], cfg["hidden"]
+    b = _codes8(seed, TID_W_OUT_NV4, (V, H), 8)
+    return (((b >> 4) & 0x8) | (b & 0x7)).astype(np.uint8), np.full((V, H // 16), 0x28, dtype=np.uint8), 2.0 ** -6
 
 
 def prefix_cache(cfg: dict, P: int, seed: int = SEED_WEIGHTS):

@@ -246,6 +246,20 @@ dg_status dg_model_set_experts_mx8(dg_model* m, const dg_expert_weights_mx8* lay
  * quarter of bf16's. */
 dg_status dg_model_set_experts_nv4(dg_model* m, const dg_expert_weights_mx8* layers, const float* tensor_scales);
 
+/* Project to the vocabulary from an 8-bit output matrix (NULL codes returns to the bf16
+ * W_out given at creation).  bf16 models only; applies to the batched calls, like the
+ * low-precision experts.  codes: E4M3 [V][H] (row v = vocabulary id v); scales: E8M0
+ * [H / 64][V][2], entry [j][v][b] the scale of elements 64 j + 32 b .. + 31 of row v, each
+ * in [0, 134] (block scale 2^(s - 127) <= 2^7); codes 0x7F / 0xFF (NaN) must not occur.
+ * Each weight is value(code) * 2^(scale - 127), decoded exactly to bf16 for s >= 9.  The
+ * output matrix's stream is about half of bf16's.  Both pointers device, 16-byte aligned,
+ * caller-owned and kept alive while the model uses them. */
+dg_status dg_model_set_vocab_mx8(dg_model* m, const void* codes, const void* scales);
+/* The same from a 4-bit output matrix: codes E2M1 two per byte [V][H / 2] (element 2 i in
+ * the low nibble of byte i), scales E4M3 [H / 64][V][4] (non-negative, not NaN), one finite
+ * tensor scale; each weight is e2m1(code) * e4m3(scale) * tensor_scale. */
+dg_status dg_model_set_vocab_nv4(dg_model* m, const void* codes, const void* scales, float tensor_scale);
+
 /* The re-noise count dg_generate_canvas uses after pass `step` of S (pure host arithmetic). */
 int32_t dg_renoise_count(int32_t C, int32_t S, int32_t step, float r_start, float r_end);
 

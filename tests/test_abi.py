@@ -263,6 +263,26 @@ def test_mx8_gemm_validation_on_host():
     assert L.dg_launch_count() == launches
 
 
+@pytest.mark.parametrize("fmt", ["mx8", "nv4"])
+def test_set_vocab_lowp_validation_on_host(fmt):
+    """dg_model_set_vocab_mx8 / _nv4 refuse an fp32 model and a NULL model before encoding
+    anything; NULL codes turns the low-precision output matrix off."""
+    st, h = _fake_model(CF.CONFIGS["tiny_fp32"])
+    assert st == dg.DG_OK
+    P = ctypes.c_void_p(1 << 28)
+    try:
+        if fmt == "mx8":
+            f = lambda m, c, s: dg.lib.dg_model_set_vocab_mx8(m, c, s)
+        else:
+            f = lambda m, c, s: dg.lib.dg_model_set_vocab_nv4(m, c, s, 0.5)
+        assert f(h, P, P) == dg.DG_ERR_INVALID_ARG                           # fp32 model
+        assert "bf16" in dg.lib.dg_last_error().decode()
+        assert f(h, None, None) == dg.DG_OK
+        assert f(None, P, P) == dg.DG_ERR_INVALID_ARG
+    finally:
+        dg.lib.dg_model_destroy(h)
+
+
 def test_set_experts_mx8_validation_on_host():
     """dg_model_set_experts_mx8 refuses an fp32 model, NULL or misaligned pointers before
     encoding anything; NULL layers turns the 8-bit experts off."""

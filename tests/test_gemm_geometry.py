@@ -37,8 +37,10 @@ def lowp_stage(fmt, n_max, terms, n_a):
 def test_lowp_gemm_geometry(name, fmt):
     c = CF.CONFIGS[name]
     H, F, E, k = c["hidden"], c["expert_ffn"], c["n_experts"], c["top_k"]
-    for dual_a, K, rows in ((1, H, F), (0, F, H)):        # gate/up, down
-        terms, n_max = 2, ITEM_ROWS_LOWP
+    V = c["vocab"]
+    # gate/up and down (two-term tokens), and the dense vocabulary projection (one term)
+    for dual_a, K, rows, terms in ((1, H, F, 2), (0, F, H, 2), (0, H, V, 1)):
+        n_max = ITEM_ROWS_LOWP
         # host checks of launch_tc_gemm_lowp
         assert K % 64 == 0 and 16 <= n_max <= 64 and n_max % 16 == 0
         stage, a_bytes, s_bytes = lowp_stage(fmt, n_max, terms, 1 + dual_a)
@@ -113,3 +115,22 @@ def test_fused_vocab_update_geometry(name, C):
         while r < n_pad:
             assert row0 + r < C
             r += 16
+
+
+@pytest.mark.parametrize("name", BF16_CONFIGS)
+def test_dense_lowp_tiles_are_weight_tile_major(name):
+    """Dense mode (the vocabulary projection): tile t takes weight tile t / chunks and token
+    chunk t % chunks, so the CTAs of one wave cover whole weight tiles with all their token
+    chunks; every (weight tile, chunk) pair is taken exactly once."""
+    c = CF.CONFIGS[name]
+    V, C = c["vocab"], c["canvas"]
+    for n in (C, 4 * C, 37):
+        chunks, m_tiles = -(-n // ITEM_ROWS_LOWP), -(-V // 128)
+        seen = set()
+        for t in range(chunks * m_tiles):
+            m, row0 = t // chunks, (t % chunks) * ITEM_ROWS_LOWP
+            assert m < m_tiles and row0 < n
+            seen.add((m, row0))
+        assert len(seen) == chunks * m_tiles
+        # one wave of 148 CTAs reads about 148 / chunks distinct weight tiles
+        assert len({t // chunks for t in range(min(148, chunks * m_tiles))}) == -(-min(148, chunks * m_tiles) // chunks)

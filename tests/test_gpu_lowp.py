@@ -245,3 +245,36 @@ def test_pass_with_nv4_experts_matches_oracle(dg, cfg, prefixes, C):
     tensor scale applied once to the accumulator on the GPU, to every weight in the oracle:
     rounding differences only)."""
     PL.check_batched_pass(dg, cfg, prefixes, C, prepare=_experts_to_nv4)
+
+
+# ---------------------------------------------------------------- low-precision output matrix
+
+def _vocab_to_mx8(setup):
+    """Quantise the output matrix with the oracle's MX-E4M3 quantiser: codes to the GPU model
+    (the batched calls' vocabulary projection), decoded weights to the oracle model."""
+    codes, exps = O.mx_e4m3_quantize(O.widen(setup.host.w_out))
+    setup.host.w_out = O.mx_e4m3_dequantize(codes, exps)
+    setup.model.set_vocab_mx8((codes, exps))
+
+
+def _vocab_to_nv4(setup):
+    codes, sc, g = O.nvfp4_quantize(O.widen(setup.host.w_out))
+    setup.host.w_out = O.nvfp4_dequantize(codes, sc, g)
+    setup.model.set_vocab_nv4((codes, sc, g))
+
+
+@pytest.mark.parametrize("fmt", ["mx8", "nv4"])
+@pytest.mark.parametrize("cfg,prefixes,C", [(SMALL_BF16, [200], 100), (SMALL_BF16, [64, 0, 131], 37),
+                                            (CF.CONFIGS["layer1_bf16"], [1024], 256)])
+def test_pass_with_low_precision_vocab_matches_oracle(dg, fmt, cfg, prefixes, C):
+    """The batched pass projecting to the vocabulary from an 8- or 4-bit output matrix
+    (dense mode of the low-precision GEMM, tiles weight tile major) against the oracle
+    pass over the decoded matrix, under the bf16 path's parity rules."""
+    PL.check_batched_pass(dg, cfg, prefixes, C, prepare=_vocab_to_mx8 if fmt == "mx8" else _vocab_to_nv4)
+
+
+def test_pass_with_8bit_experts_and_vocab_matches_oracle(dg):
+    def prep(setup):
+        _experts_to_mx8(setup)
+        _vocab_to_mx8(setup)
+    PL.check_batched_pass(dg, SMALL_BF16, [64, 0, 131], 37, prepare=prep)

@@ -34,7 +34,9 @@ def decode_nv4(codes, sc):
 def run_lowp(fmt, W, S, X_hi, X_lo, items, rows_a, K, ld_out, W2=None, S2=None, g=1.0, g2=1.0, n_max=64,
              smem_budget=200 * 1024, grid=3, bug=None):
     """W / W2: codes as the library stores them (8-bit [G][rows][K]; 4-bit packed
-    [G][rows][K / 2]); S / S2: the library's scale bytes; items: (group, row0, rows)."""
+    [G][rows][K / 2]); S / S2: the library's scale bytes; items: (group, row0, rows), or
+    None for the dense mode (one weight matrix, tokens in chunks of n_max, tiles ordered
+    weight tile major)."""
     nv4 = fmt == "nv4"
     A_BYTES = BM * BK // 2 if nv4 else BM * BK
     S_BYTES = BM * 4 if nv4 else BM * 2
@@ -67,7 +69,9 @@ def run_lowp(fmt, W, S, X_hi, X_lo, items, rows_a, K, ld_out, W2=None, S2=None, 
     swz_span = 32 if nv4 else 64
     out = np.full((n_tokens, ld_out), np.nan)
     out_lo = np.zeros((n_tokens, ld_out))
-    n_tiles = len(items) * m_tiles
+    dense = items is None
+    chunks = -(-n_tokens // n_max)
+    n_tiles = chunks * m_tiles if dense else len(items) * m_tiles
     for cta in range(min(grid, n_tiles)):
         sm, tm = T.Smem(stages * stage_bytes), T.Tmem(tmem_cols)
         tiles = list(range(cta, n_tiles, grid))
@@ -76,6 +80,9 @@ def run_lowp(fmt, W, S, X_hi, X_lo, items, rows_a, K, ld_out, W2=None, S2=None, 
         pending_epi = []                                         # (tile index j, tile) awaiting their epilogue
 
         def tile_of(t):
+            if dense:
+                row0 = (t % chunks) * n_max
+                return 0, row0, min(n_max, n_tokens - row0), t // chunks
             g_, row0, rows = items[t // m_tiles]
             return g_, row0, rows, t % m_tiles
 
@@ -289,3 +296,21 @@ def test_a_planted_decode_column_mistake_is_caught():
     out, out_lo = run_lowp("mx8", cg, sg, hi, lo, items, F, K, F, W2=cu, S2=su, bug="dec_col")
     ref = O.silu(x[:20] @ wg[0].T) * (x[:20] @ wu[0].T)
     assert np.abs((out + out_lo)[:20] - ref).max() / np.abs(ref).max() > 1e-2
+
+
+@pytest.mark.parametrize("fmt", ["mx8", "nv4"])
+def test_dense_vocab_gemm_replay(fmt):
+    """The dense mode as the vocabulary projection uses it: one weight matrix of V rows,
+    the canvas rows in chunks of 64 tokens (one term), tiles ordered weight tile major."""
+    rng = np.random.default_rng(11)
+    n, V, H = 150, 640, 128
+    x, hi, _ = tokens(rng, n, H)
+    x = T.bf16_value(hi).astype(np.float64)
+    if fmt == "mx8":
+        codes, S, wq = mx8_weights(rng, 1, V, H)
+        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, grid=7)
+    else:
+        codes, S, g, wq = nv4_weights(rng, 1, V, H)
+        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, g=g, grid=7)
+    ref = x @ wq[0].T
+    assert np.abs(out - ref).max() / np.abs(ref).max() < 2e-5

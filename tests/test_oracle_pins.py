@@ -786,6 +786,9 @@ def test_roofline_batch_and_8bit_accounting():
     assert R.pass_bytes_batched(cfg, [P] * 4, C, U) == one + 3 * per_canvas
     assert one - R.pass_bytes(cfg, P, C, U, ew=R.MX8_WBYTES) == (2 - 1 - 1 / 32) * 3 * H * F * 52
     assert R.gate_up_bytes(cfg, 52, 1024, ew=1.0) == 2 * H * F * 52 + 2 * 1024 * (H + F)
+    # a 4-bit output matrix: 1/2 + 1/16 bytes per weight instead of 2, counted once per batch
+    saved = (2 - 0.5 - 1 / 16) * V * H
+    assert R.pass_bytes_batched(cfg, [P] * 4, C, U) - R.pass_bytes_batched(cfg, [P] * 4, C, U, vw=R.NV4_WBYTES) == saved
 
 
 def test_roofline_reproduces_exercise_arithmetic():

@@ -57,3 +57,20 @@ def test_nv4_experts_are_uniform_4bit_codes():
         assert cnt.min() > 0.8 * codes.size / 16 and cnt.max() < 1.2 * codes.size / 16
         assert sc.shape == shape[:-1] + (shape[-1] // 16,) and (sc == 0x28).all() and g == 2.0 ** -6
     np.testing.assert_array_equal(a[0]["gate"][0], synth.nv4_experts(cfg)[0]["gate"][0])
+
+
+def test_low_precision_vocab_matrices():
+    """The 8- and 4-bit output matrices: shapes, valid codes, their own streams (not the
+    experts'), deterministic."""
+    cfg = dict(n_layers=1, hidden=128, n_experts=2, expert_ffn=64, vocab=256)
+    codes, exps = synth.mx8_vocab(cfg)
+    assert codes.shape == (256, 128) and exps.shape == (256, 4) and (exps == -12).all()
+    assert not np.isin(codes, [0x7F, 0xFF]).any() and (codes & 0x7F).max() == 0x6F
+    np.testing.assert_array_equal(codes, synth.mx8_vocab(cfg)[0])
+    c4, sc, g = synth.nv4_vocab(cfg)
+    assert c4.shape == (256, 128) and c4.max() < 16 and sc.shape == (256, 8) and (sc == 0x28).all()
+    cnt = np.bincount(c4.ravel(), minlength=16)
+    assert cnt.min() > 0.8 * c4.size / 16 and cnt.max() < 1.2 * c4.size / 16
+    # distinct streams from the experts' codes of the same shape
+    e8 = synth.mx8_experts(dict(cfg, n_experts=1, expert_ffn=256))[0]["down"][0]   # [1][128][256]
+    assert (e8[0].T != codes).mean() > 0.9
