@@ -1299,11 +1299,12 @@ extern "C" dg_status dg_denoise_pass_batched(dg_model* m, const dg_kv_cache* cac
                  : run_stack_batched<float>(m, caches, B, d_canvases, C, false, ws, st);
   if (s != DG_OK) return s;
   if (is_bf16(c) && m->vocab_lowp.on) {
-    // dense low-precision GEMM: tokens in chunks of 64, tiles weight tile major
+    // dense low-precision GEMM: tokens in chunks of up to 128 (each chunk decodes the weight
+    // tiles again, so fewer chunks mean less decode work), tiles weight tile major
     const VocabLowp& Vl = m->vocab_lowp;
+    const int chunk = n <= 64 ? ((n + 15) & ~15) : 128;
     GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &Vl.codes, nullptr, ws.at<void>(ws.L.xn), nullptr, n, c.hidden,
-               c.vocab, nullptr, nullptr, ceil_div(n, kItemRowsMx8), kItemRowsMx8, d_logits, nullptr, c.vocab, 1, 0,
-               kSmemGemm};
+               c.vocab, nullptr, nullptr, ceil_div(n, chunk), chunk, d_logits, nullptr, c.vocab, 1, 0, kSmemGemm};
     if ((s = gemm_lowp(g, Vl.fmt, &Vl.scales, nullptr, Vl.g, 1.0f, ws.err(), st)) != DG_OK) return s;
   } else if (is_bf16(c)) {
     GemmCall g{DG_K_GEMM_VOCAB, dg::EPI_STORE_F32, &m->out_map, nullptr, ws.at<void>(ws.L.xn), nullptr, n, c.hidden,

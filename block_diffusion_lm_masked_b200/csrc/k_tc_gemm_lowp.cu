@@ -492,8 +492,11 @@ cudaError_t launch_tc_gemm_lowp(int fmt, int epi, const CUtensorMap& A, const CU
                                 const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p, float g_a,
                                 float g_a2, int max_tiles, cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
+  // TMEM: two accumulators of n_max columns per weight matrix and four decoded stages of 32
+  // columns per matrix fit 512 columns for n_max <= 64 with two matrices, <= 128 with one
   if ((fmt != FMT_MX8 && fmt != FMT_NV4) || p.k_splits != 1 || p.K % MX_BK != 0 || p.K <= 0 || p.n_max < 16 ||
-      p.n_max > 64 || (p.n_max % 16) != 0 || p.m_tiles < 1 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
+      p.n_max > (p.dual_a ? 64 : 128) || (p.n_max % 16) != 0 || p.m_tiles < 1 ||
+      (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
     return cudaErrorInvalidValue;
   const int n_a = p.dual_a ? 2 : 1;
   const int terms = p.two_terms ? 2 : 1;

@@ -39,10 +39,10 @@ def test_lowp_gemm_geometry(name, fmt):
     H, F, E, k = c["hidden"], c["expert_ffn"], c["n_experts"], c["top_k"]
     V = c["vocab"]
     # gate/up and down (two-term tokens), and the dense vocabulary projection (one term)
-    for dual_a, K, rows, terms in ((1, H, F, 2), (0, F, H, 2), (0, H, V, 1)):
-        n_max = ITEM_ROWS_LOWP
+    for dual_a, K, rows, terms, n_max in ((1, H, F, 2, ITEM_ROWS_LOWP), (0, F, H, 2, ITEM_ROWS_LOWP),
+                                          (0, H, V, 1, 128)):
         # host checks of launch_tc_gemm_lowp
-        assert K % 64 == 0 and 16 <= n_max <= 64 and n_max % 16 == 0
+        assert K % 64 == 0 and 16 <= n_max <= (64 if dual_a else 128) and n_max % 16 == 0
         stage, a_bytes, s_bytes = lowp_stage(fmt, n_max, terms, 1 + dual_a)
         assert SMEM_GEMM >= 2 * stage
         stages = min(SMEM_GEMM // stage, 8)
@@ -125,10 +125,11 @@ def test_dense_lowp_tiles_are_weight_tile_major(name):
     c = CF.CONFIGS[name]
     V, C = c["vocab"], c["canvas"]
     for n in (C, 4 * C, 37):
-        chunks, m_tiles = -(-n // ITEM_ROWS_LOWP), -(-V // 128)
+        chunk = ((n + 15) & ~15) if n <= 64 else 128          # the host's token chunk
+        chunks, m_tiles = -(-n // chunk), -(-V // 128)
         seen = set()
         for t in range(chunks * m_tiles):
-            m, row0 = t // chunks, (t % chunks) * ITEM_ROWS_LOWP
+            m, row0 = t // chunks, (t % chunks) * chunk
             assert m < m_tiles and row0 < n
             seen.add((m, row0))
         assert len(seen) == chunks * m_tiles

@@ -298,19 +298,19 @@ def test_a_planted_decode_column_mistake_is_caught():
     assert np.abs((out + out_lo)[:20] - ref).max() / np.abs(ref).max() > 1e-2
 
 
-@pytest.mark.parametrize("fmt", ["mx8", "nv4"])
-def test_dense_vocab_gemm_replay(fmt):
+@pytest.mark.parametrize("fmt,n_max", [("mx8", 64), ("mx8", 128), ("nv4", 128)])
+def test_dense_vocab_gemm_replay(fmt, n_max):
     """The dense mode as the vocabulary projection uses it: one weight matrix of V rows,
-    the canvas rows in chunks of 64 tokens (one term), tiles ordered weight tile major."""
+    the canvas rows in chunks of up to 128 tokens (one term), tiles weight tile major."""
     rng = np.random.default_rng(11)
     n, V, H = 150, 640, 128
     x, hi, _ = tokens(rng, n, H)
     x = T.bf16_value(hi).astype(np.float64)
     if fmt == "mx8":
         codes, S, wq = mx8_weights(rng, 1, V, H)
-        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, grid=7)
+        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, grid=7, n_max=n_max)
     else:
         codes, S, g, wq = nv4_weights(rng, 1, V, H)
-        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, g=g, grid=7)
+        out, _ = run_lowp(fmt, codes, S, hi, None, None, V, H, V, g=g, grid=7, n_max=n_max)
     ref = x @ wq[0].T
     assert np.abs(out - ref).max() / np.abs(ref).max() < 2e-5
