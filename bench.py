@@ -388,7 +388,7 @@ def run_variant(args, cfg, name):
         "metric": METRIC, "value": job_value(world, B * C, args.steps, total_ms), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
-        "config": {"workload": _workload_desc(name, cfg), "canvases_per_pass": B,
+        "config": {"workload": _workload_desc(name, cfg), "canvases_per_pass": B, "attention": _attention_kind(),
                    "update": "fused into the vocabulary projection" if args.fused_update else "two kernels on logits",
                    "experts": {"bf16": "bf16", "mx8": "mx8 (E4M3 + E8M0 per 32, synthetic codes)",
                                "nv4": "nv4 (E2M1 + E4M3 per 16 + fp32 tensor scale, synthetic codes)"}[lowp],
@@ -411,6 +411,12 @@ def run_variant(args, cfg, name):
     return 0
 
 
+def _attention_kind():
+    """Which attention kernel the library runs (DG_ATTN_PAIR=1: the head-pair kernel)."""
+    return ("head pairs, 64-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
+            else "one head, 128-key chunks")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -428,7 +434,11 @@ def main():
                     help="expert weight storage; mx8 and nv4 run through the batched calls")
     ap.add_argument("--vocab", default="bf16", choices=["bf16", "mx8", "nv4"],
                     help="output-matrix storage; mx8 and nv4 run through the batched calls")
+    ap.add_argument("--attn-pair", action="store_true",
+                    help="run the pass's attention through the head-pair kernel (sets DG_ATTN_PAIR=1)")
     args = ap.parse_args()
+    if args.attn_pair:  # read by the library at its first attention call
+        os.environ["DG_ATTN_PAIR"] = "1"
     name = args.workload
     cfg = CF.CONFIGS[name]
     if args.impl == "reference":
@@ -628,7 +638,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": _workload_desc(name, cfg), "l2": "flushed between steps (256 MB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "expert_union": unions_h},
+                   "attention": _attention_kind(), "expert_union": unions_h},
         "roofline": roof,
         "pass_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof * 1e3 / ms_step, "flops": flops,
                           "bytes": nbytes, "bound": "hbm" if nbytes / (hbm * 1e9) > flops / (tf_burst * 1e12)

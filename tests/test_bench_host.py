@@ -92,3 +92,12 @@ def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
 def test_job_value_counts_every_rank_over_the_slowest():
     assert bench.job_value(1, 256, 1000, 347.6) == pytest.approx(256 * 1000 / 0.3476)
     assert bench.job_value(8, 256, 1000, 400.0) == pytest.approx(8 * 256 * 1000 / 0.4)
+
+
+def test_attention_kind_follows_the_switch(monkeypatch):
+    monkeypatch.delenv("DG_ATTN_PAIR", raising=False)
+    assert bench._attention_kind().startswith("one head")
+    monkeypatch.setenv("DG_ATTN_PAIR", "1")
+    assert bench._attention_kind().startswith("head pairs")
+    monkeypatch.setenv("DG_ATTN_PAIR", "0")
+    assert bench._attention_kind().startswith("one head")
