@@ -635,8 +635,8 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
-           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),
-                                 ws.at<bf16>(ws.L.o_lo), st));
+           dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, ws.at<bf16>(ws.L.o),
+                                  ws.at<bf16>(ws.L.o_lo), st));
   return DG_OK;
 }
 

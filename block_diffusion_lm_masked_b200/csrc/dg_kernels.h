@@ -99,6 +99,10 @@ cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, co
                                  const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
                                  const TcAttnParams& p, cudaStream_t st);
 int attn2_head_groups(int nq, int group);
+// the head-pair path's split merge (same inputs and outputs as launch_attn_merge, d = 128):
+// one warp per (row, head), n_splits <= 32
+cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
+                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 
 // ---------------------------------------------------------------- SIMT kernels (any dtype)
 // T = float (fp32 model) or __nv_bfloat16; an activation for a bf16 GEMM is written as
