@@ -287,7 +287,10 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     bool ok = true;
     for (int j = 0; j < nck && ok; ++j) {
       const int b = j & 1;
-      ok = mbar_wait(&s_full[hl][b], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      // every wait's outcome is made warp-uniform: the tcgen05.ld / st that follow are
+      // warp-collective, so a lane that gave up must take its whole warp with it
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&s_full[hl][b], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
       if (!ok) break;
       tc_fence_after();
       const uint32_t spa = tmem + a2_sp(hl, b) + lane_off;
@@ -312,8 +315,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       // tcgen05.ld/st are warp-collective: the warp rescales its rows of O if any row must,
       // once the previous chunk's PV is complete (O stable; PV(j) waits for this P)
       if (__any_sync(0xffffffffu, upd && j > 0)) {
-        ok = mbar_wait(&pv_done[hl][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s, p.err,
-                       DG_DEVERR_TIMEOUT_ATTN);
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s,
+                                               p.err, DG_DEVERR_TIMEOUT_ATTN));
         if (!ok) break;
         tc_fence_after();
         const uint32_t oa = tmem + a2_o(hl) + lane_off;
@@ -356,8 +359,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       if (lane == 0) mbar_arrive(&p_ready[hl][b]);
     }
     if (ok)
-      ok = mbar_wait(&pv_done[hl][(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s, p.err,
-                     DG_DEVERR_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl][(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s,
+                                             p.err, DG_DEVERR_TIMEOUT_ATTN));
     if (ok) {
       tc_fence_after();
       const bool valid = my_row < p.n_q;
