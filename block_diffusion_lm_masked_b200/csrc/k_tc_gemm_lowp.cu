@@ -343,7 +343,10 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
       const MxTile ti = mx_decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;
       const int buf = j & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)) break;
+      // each wait's outcome is made warp-uniform: the tcgen05.ld below is warp-collective
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)))
+        break;
       tc_fence_after();
       const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
       const int f = ti.m * MX_BM + row;  // weight row = output feature
@@ -395,9 +398,11 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
     while (ok && walk.next(t)) {
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % stages, ts = it % MX_T_STAGES;
-        if (!mbar_wait(&f_full[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL) ||
-            !mbar_wait(&t_empty[ts], ((uint32_t)(it / MX_T_STAGES) & 1u) ^ 1u, &abort_s, p.err,
-                       DG_DEVERR_TIMEOUT_EMPTY)) {
+        const bool got =
+            mbar_wait(&f_full[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL) &&
+            mbar_wait(&t_empty[ts], ((uint32_t)(it / MX_T_STAGES) & 1u) ^ 1u, &abort_s, p.err,
+                      DG_DEVERR_TIMEOUT_EMPTY);
+        if (!__all_sync(0xffffffffu, got)) {  // the tcgen05.st below is warp-collective
           ok = false;
           break;
         }
