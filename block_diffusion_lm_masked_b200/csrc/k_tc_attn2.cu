@@ -239,7 +239,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         }
         tc_commit(&pv_done[hl][b]);
       };
-      // PV of chunk k for every head once its P is written, then free chunk k's slots
+      // PV of chunk k for every head once its P is written, then free chunk k's slots (the
+      // last chunk's slots are not reused: no commit nobody waits for)
       auto pv_chunk = [&](int k) {
         for (int hl = 0; hl < nh; ++hl) {
           if (!mbar_wait(&p_ready[hl][k & 1], (uint32_t)(k >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
@@ -247,7 +248,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           tc_fence_after();
           issue_pv(hl, k);
         }
-        for (int i = 0; i < mp.n[k & 1]; ++i) tc_commit(&kv_free[mp.slot[k & 1][i]]);
+        if (k + 1 < nck)
+          for (int i = 0; i < mp.n[k & 1]; ++i) tc_commit(&kv_free[mp.slot[k & 1][i]]);
         return true;
       };
 
@@ -413,17 +415,17 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     }
   }
   __syncthreads();
-  if (abort_s) {
-    // wind down: let issued loads and MMAs land before the smem / TMEM go away
-    if (tid == A2_LOAD_WARP * 32) {
-      if (q_issued) mbar_wait_drain(&q_bar, 0);
-      for (int s = 0; s < A2_SLOTS; ++s)
-        if (loaded[s] > 0) mbar_wait_drain(&kv_full[s], (uint32_t)(loaded[s] - 1) & 1u);
-    }
-    if (tid == A2_MMA_WARP * 32) {
-      tc_commit(&drain_bar);
-      mbar_wait_drain(&drain_bar, 0);
-    }
+  // wind down: every MMA and commit the MMA thread issued has landed (also on the normal
+  // path, so that no mbarrier arrive reaches this CTA's shared memory after it is gone),
+  // and after an abort the loads the load thread issued have landed too
+  if (tid == A2_MMA_WARP * 32) {
+    tc_commit(&drain_bar);
+    mbar_wait_drain(&drain_bar, 0);
+  }
+  if (abort_s && tid == A2_LOAD_WARP * 32) {
+    if (q_issued) mbar_wait_drain(&q_bar, 0);
+    for (int s = 0; s < A2_SLOTS; ++s)
+      if (loaded[s] > 0) mbar_wait_drain(&kv_full[s], (uint32_t)(loaded[s] - 1) & 1u);
   }
   tc_fence_before();
   __syncthreads();

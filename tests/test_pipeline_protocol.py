@@ -88,12 +88,16 @@ class Async:
             self.loads.pop(rng.randrange(len(self.loads)))()
 
 
-def run(roles, q, seed, max_steps=200000):
-    """roles: name -> generator of steps; q: the Async the roles hand delayed completions to."""
+def run(roles, q, seed, max_steps=200000, end_check=False):
+    """roles: name -> generator of steps; q: the Async the roles hand delayed completions to.
+    end_check: when every role has finished (the CTA leaves), no load or MMA completion may
+    still be pending (it would land in released shared or tensor memory)."""
     rng = random.Random(seed)
     blocked = {}
     live = dict(roles)
     for _ in range(max_steps):
+        if not live and end_check:
+            assert not q, f"{len(q.loads)} loads and {len(q.mma)} MMA completions pending after the last role left"
         if not live and not q:
             return
         ready = []
@@ -608,13 +612,15 @@ def fused_epilogue_with_abort(n_tiles, nkb, stages, chunks, rng, vote=True):
     return roles, q, flags
 
 
-def run_ab(roles, q, flags, seed, max_steps=200000):
+def run_ab(roles, q, flags, seed, max_steps=200000, end_check=False):
     """run() where an abort-aware wait also passes once the abort flag is set."""
     rng = random.Random(seed)
     blocked = {}
     live = dict(roles)
     for _ in range(max_steps):
         if not live:
+            if end_check:
+                assert not q, f"{len(q.loads)} loads and {len(q.mma)} MMA completions pending after the last role left"
             return
         ready = []
         for name in live:
@@ -677,19 +683,27 @@ def slot_plan(nck, cur_from, slots):
     return plan
 
 
-def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_first_rule=True):
-    """The redesigned attention's hand-offs: a load warp fills `slots` K/V slots; the MMA
-    warp issues S_A(j), S_B(j) into S/P buffer j & 1 of each head, then PV_A(j-1),
+def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_first_rule=True, flags=None,
+                        give_up_at=None, final_slot_commits=False, drain=True, load_drain=True):
+    """The head-pair attention kernel's hand-offs: a load warp fills `slots` K/V slots; the
+    MMA warp issues S_A(j), S_B(j) into S/P buffer j & 1 of each head, then PV_A(j-1),
     PV_B(j-1), then frees chunk j-1's slots with a commit; each head's softmax warps read
     S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  Before S_h(j)
     reuses buffer j & 1, the MMA warp waits for PV_h(j-2), the last reader of that P.
     When chunks j-1 and j together need more slots than the ring has (two current chunks
     in three slots), chunk j cannot load before chunk j-1's slots are free, so the MMA
-    warp issues PV(j-1) before S(j) (`pv_first_rule`; without it that case deadlocks)."""
+    warp issues PV(j-1) before S(j) (`pv_first_rule`; without it that case deadlocks).
+    The last chunk's slots get no release commit (`final_slot_commits` adds them) and the
+    MMA warp drains its commits before the CTA leaves (`drain`).
+
+    flags: abort mode -- every bounded wait also passes once flags["abort"] is set, the
+    give_up_at-th wait raises it (a timeout), a role whose wait failed leaves its loop,
+    and the load warp then waits for the loads it issued (`load_drain`)."""
     rng = random.Random(seed * 104729 + nck)
     plan = slot_plan(nck, nck if cur_from is None else cur_from, slots)
     kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
     kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
+    drain_bar = Barrier("drain", 1)
     H = 2
     s_full = [[Barrier(f"s_full{h}{b}", 1) for b in range(2)] for h in range(H)]
     p_ready = [[Barrier(f"p_ready{h}{b}", warps_per_head) for b in range(2)] for h in range(H)]
@@ -697,14 +711,40 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_
     bufs, q = Buffers(), Async()
     st = {"pv_done": [0, 0], "pv_issued": [0, 0], "s_done": [0, 0]}
     p_writes = {}
+    steps = [0]
+
+    def bw(bar, parity, phase):
+        """A bounded wait (abort-aware in abort mode)."""
+        if flags is None:
+            return wait(bar, parity, phase)
+        steps[0] += 1
+        if steps[0] == give_up_at:
+            flags["abort"] = True
+        return ("waitab", bar, parity, phase)
+
+    def passed(bar, parity):
+        return flags is None or (bar.completed % 2) != parity
 
     def load():
+        loaded = [0] * slots
+        ok = True
         for j in range(nck):
             for s, u in plan[j]:
-                yield wait(kv_free[s], (u & 1) ^ 1, u - 1)
+                if u >= 1:
+                    yield bw(kv_free[s], (u & 1) ^ 1, u - 1)
+                    if not passed(kv_free[s], (u & 1) ^ 1):
+                        ok = False
+                        break
                 bufs.fill(("slot", s), 2 * H)         # S_A, S_B, PV_A, PV_B of chunk j read it
                 kv_full[s].arrive_expect_tx(32)
                 q.loads.append(lambda s=s: kv_full[s].complete_tx(32))
+                loaded[s] += 1
+            if not ok:
+                break
+        if flags is not None and flags["abort"] and load_drain:
+            for s in range(slots):                    # the wind-down: the last load of each slot
+                if loaded[s]:
+                    yield wait(kv_full[s], (loaded[s] - 1) & 1, None)
 
     def mma():
         def issue_pv(h, k):
@@ -720,22 +760,37 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_
                 pv_done[h][k & 1].arrive()
             q.mma.append(done)
 
-        def pv_prev(j):
+        def pv_chunk(k):
             for h in range(H):
-                yield wait(p_ready[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
-                issue_pv(h, j - 1)
-            for x, _ in plan[j - 1]:                   # one commit per slot of chunk j-1
-                q.mma.append(lambda x=x: kv_free[x].arrive())
+                yield bw(p_ready[h][k & 1], (k >> 1) & 1, k >> 1)
+                if not passed(p_ready[h][k & 1], (k >> 1) & 1):
+                    return False
+                issue_pv(h, k)
+            if k + 1 < nck or final_slot_commits:     # one commit per slot of chunk k
+                for x, _ in plan[k]:
+                    q.mma.append(lambda x=x: kv_free[x].arrive())
+            return True
 
+        ok = True
         for j in range(nck):
             pv_first = pv_first_rule and j >= 1 and len(plan[j - 1]) + len(plan[j]) > slots
             if pv_first:
-                yield from pv_prev(j)
+                ok = yield from pv_chunk(j - 1)
+                if not ok:
+                    break
             for x, u in plan[j]:
-                yield wait(kv_full[x], u & 1, u)
+                yield bw(kv_full[x], u & 1, u)
+                if not passed(kv_full[x], u & 1):
+                    ok = False
+                    break
             for h in range(H):
+                if not ok:
+                    break
                 if j >= 2:
-                    yield wait(pv_done[h][j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
+                    yield bw(pv_done[h][j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
+                    if not passed(pv_done[h][j & 1], ((j >> 1) - 1) & 1):
+                        ok = False
+                        break
                 for w in range(warps_per_head):       # S: each warp reads its own 32 lanes
                     bufs.fill(("sp", h, j & 1, w), 1)
 
@@ -745,25 +800,36 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_
                         bufs.release(("slot", x))
                     s_full[h][j & 1].arrive()
                 q.mma.append(s_done)
+            if not ok:
+                break
             if j >= 1 and not pv_first:
-                yield from pv_prev(j)
-        for h in range(H):
-            yield wait(p_ready[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
-            issue_pv(h, nck - 1)
+                ok = yield from pv_chunk(j - 1)
+                if not ok:
+                    break
+        if ok:
+            yield from pv_chunk(nck - 1)
+        if drain:                                     # every commit issued above has landed
+            q.mma.append(lambda: drain_bar.arrive())
+            yield wait(drain_bar, 0, 0)
 
     def softmax(h, w):
         for j in range(nck):
-            yield wait(s_full[h][j & 1], (j >> 1) & 1, j >> 1)
+            yield bw(s_full[h][j & 1], (j >> 1) & 1, j >> 1)
+            if not passed(s_full[h][j & 1], (j >> 1) & 1):
+                return
             bufs.release(("sp", h, j & 1, w))          # this warp's lanes of S read into registers
             if j > 0 and rng.random() < 0.4:           # the row max grew: rescale O after PV(j-1)
-                yield wait(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                yield bw(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
+                if not passed(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1):
+                    return
                 assert st["pv_done"][h] >= j and st["pv_issued"][h] <= j, "O rescaled while a PV may write it"
             bufs.fill(("sp", h, j & 1, w), 1)         # P over this warp's lanes of S, read by PV(j)
             last, n = p_writes.get((h, j & 1), (None, 0))
             p_writes[(h, j & 1)] = (j, 1) if last != j else (j, n + 1)
             p_ready[h][j & 1].arrive()
-        yield wait(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
-        assert st["pv_done"][h] == nck
+        yield bw(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
+        if passed(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1):
+            assert st["pv_done"][h] == nck
 
     roles = {"load": load(), "mma": mma()}
     for h in range(H):
@@ -778,7 +844,7 @@ def test_attention_redesign_protocol(nck, cur_from):
     read, no P read before all its writers, no O rescaled under a PV."""
     for seed in range(40):
         roles, q = attention_two_heads(nck, seed, cur_from=cur_from)
-        run(roles, q, seed)
+        run(roles, q, seed, end_check=True)
 
 
 def test_attention_redesign_needs_pv_first_for_two_current_chunks():
@@ -791,3 +857,45 @@ def test_attention_redesign_needs_pv_first_for_two_current_chunks():
     for seed in range(20):
         roles, q = attention_two_heads(5, seed, cur_from=4, pv_first_rule=False)
         run(roles, q, seed)
+
+
+def test_attention_redesign_leaves_nothing_in_flight():
+    """When the last role leaves, no MMA completion or commit may still be pending (it would
+    arrive on released shared memory).  With the drain that holds in every interleaving;
+    the earlier design -- release commits for the last chunk's slots and no drain on the
+    normal path -- leaves commits behind in some."""
+    for seed in range(60):
+        roles, q = attention_two_heads(6, seed, cur_from=4)
+        run(roles, q, seed, end_check=True)
+    left = 0
+    for seed in range(60):
+        roles, q = attention_two_heads(6, seed, cur_from=4, final_slot_commits=True, drain=False)
+        try:
+            run(roles, q, seed, end_check=True)
+        except AssertionError as e:
+            left += "pending" in str(e)
+    assert left > 0
+
+
+@pytest.mark.parametrize("nck,cur_from", [(4, 2), (7, 4), (6, 0)])
+def test_attention_redesign_winds_down_after_a_timeout(nck, cur_from):
+    """A bounded wait gives up at a random point: every role leaves (no deadlock), and with
+    the load warp's drain and the MMA warp's drain nothing is in flight when they have.
+    Without the load drain, some timeout leaves a load landing after the CTA is gone."""
+    for seed in range(150):
+        rng = random.Random(seed)
+        flags = {"abort": False}
+        roles, q = attention_two_heads(nck, seed, cur_from=cur_from, flags=flags,
+                                       give_up_at=rng.randrange(1, 12 * nck))
+        run_ab(roles, q, flags, seed, end_check=True)
+    left = 0
+    for seed in range(150):
+        rng = random.Random(seed)
+        flags = {"abort": False}
+        roles, q = attention_two_heads(nck, seed, cur_from=cur_from, flags=flags,
+                                       give_up_at=rng.randrange(1, 12 * nck), load_drain=False)
+        try:
+            run_ab(roles, q, flags, seed, end_check=True)
+        except AssertionError as e:
+            left += "pending" in str(e)
+    assert left > 0
