@@ -264,7 +264,7 @@ def lowp_gemm(n_tiles, nkb, stages, t_stages=4, dec_warps=8):
 def test_bf16_gemm_protocol(n_tiles, nkb, stages):
     for seed in range(30):
         roles, q = bf16_gemm(n_tiles, nkb, stages)
-        run(roles, q, seed)
+        run(roles, q, seed, end_check=True)
 
 
 @pytest.mark.parametrize("n_tiles,nkb,stages", [(1, 1, 2), (3, 1, 6), (2, 5, 3), (5, 4, 6), (3, 16, 6), (6, 3, 2),
@@ -272,7 +272,7 @@ def test_bf16_gemm_protocol(n_tiles, nkb, stages):
 def test_lowp_gemm_protocol(n_tiles, nkb, stages):
     for seed in range(30):
         roles, q = lowp_gemm(n_tiles, nkb, stages)
-        run(roles, q, seed)
+        run(roles, q, seed, end_check=True)
 
 
 def _lowp_with_count(f_empty_count, seed):
@@ -447,7 +447,7 @@ def attention(nck, cur_from, seed, n_warps=8):
 def test_attention_protocol(nck, cur_from):
     for seed in range(25):
         roles, q = attention(nck, cur_from, seed)
-        run(roles, q, seed)
+        run(roles, q, seed, end_check=True)
 
 
 # ---------------------------------------------------------------- the fused vocabulary/update GEMM (k_tc_vocab_update.cu)
