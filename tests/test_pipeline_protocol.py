@@ -549,36 +549,51 @@ def fused_epilogue_with_abort(n_tiles, nkb, stages, chunks, rng, vote=True):
     def ok_after(bar, parity):
         return (bar.completed % 2) != parity
 
+    drain_bar = Barrier("drain", 1)
+
     def producer():
         it = 0
-        for t in range(n_tiles):
-            for kb in range(nkb):
-                s = it % stages
-                par = ((it // stages) & 1) ^ 1
-                yield wait_ab(empty[s], par, None)
-                if not ok_after(empty[s], par):
-                    return
-                full[s].arrive_expect_tx(64)
-                q.loads.append(lambda s=s: full[s].complete_tx(64))
-                it += 1
+
+        def issue_all():
+            nonlocal it
+            for t in range(n_tiles):
+                for kb in range(nkb):
+                    s = it % stages
+                    par = ((it // stages) & 1) ^ 1
+                    yield wait_ab(empty[s], par, None)
+                    if not ok_after(empty[s], par):
+                        return
+                    full[s].arrive_expect_tx(64)
+                    q.loads.append(lambda s=s: full[s].complete_tx(64))
+                    it += 1
+        yield from issue_all()
+        if flags["abort"]:                            # the wind-down: the newest load of every stage
+            for i in range(max(0, it - stages), it):
+                yield wait(full[i % stages], (i // stages) & 1, None)
 
     def mma():
         it = 0
-        for j in range(n_tiles):
-            buf = j & 1
-            par = ((j >> 1) & 1) ^ 1
-            yield wait_ab(acc_empty[buf], par, None)
-            if not ok_after(acc_empty[buf], par):
-                return
-            for kb in range(nkb):
-                s = it % stages
-                par2 = (it // stages) & 1
-                yield wait_ab(full[s], par2, None)
-                if not ok_after(full[s], par2):
+
+        def issue_all():
+            nonlocal it
+            for j in range(n_tiles):
+                buf = j & 1
+                par = ((j >> 1) & 1) ^ 1
+                yield wait_ab(acc_empty[buf], par, None)
+                if not ok_after(acc_empty[buf], par):
                     return
-                q.mma.append(lambda s=s: empty[s].arrive())
-                it += 1
-            q.mma.append(lambda b=buf: acc_full[b].arrive())
+                for kb in range(nkb):
+                    s = it % stages
+                    par2 = (it // stages) & 1
+                    yield wait_ab(full[s], par2, None)
+                    if not ok_after(full[s], par2):
+                        return
+                    q.mma.append(lambda s=s: empty[s].arrive())
+                    it += 1
+                q.mma.append(lambda b=buf: acc_full[b].arrive())
+        yield from issue_all()
+        q.mma.append(lambda: drain_bar.arrive())      # the final commit, waited for before the CTA leaves
+        yield wait(drain_bar, 0, 0)
 
     def epilogue(w):
         k = 0
@@ -655,7 +670,7 @@ def test_fused_epilogue_warps_leave_together_on_a_timeout():
     for seed in range(300):
         rng = random.Random(seed)
         roles, q, flags = fused_epilogue_with_abort(3, 3, 2, 2, rng, vote=True)
-        run_ab(roles, q, flags, seed)
+        run_ab(roles, q, flags, seed, end_check=True)
     hung = 0
     for seed in range(300):
         rng = random.Random(seed)
