@@ -1,0 +1,217 @@
+"""The bf16 GEMM (tc_gemm_kernel, validated on a B200) replayed at the address level on the
+CPU (tests/tc_emu.py): the control for the GEMM half of the hardware model, and a CPU
+check for later changes to the kernel.
+
+Transcribed from the kernel source: the persistent tile walk (grouped: item-major;
+dense: token chunk, then split, then weight tile), the k-block rotation within a split,
+the stage layout (one or two weight tiles, then one or two token terms of n_max rows),
+the MMAs into one of two accumulator buffers (a second weight matrix n_max columns on),
+and the epilogue's indices: fp32 stores into the split's slab, or SwiGLU with bf16 hi /
+lo.  The producer runs as far ahead as the stage ring allows and each epilogue as late as
+its accumulator buffer allows.  Results are compared with fp64 products of the same bf16
+values.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import tc_emu as T
+from oracle import dg_oracle as O
+
+BM, BK = 128, 64
+
+
+def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1, W2=None, split_stride=0,
+             smem_budget=200 * 1024, grid=5, bug=None):
+    """W / W2: bf16 bits [G][rows][K]; X_hi / X_lo: bf16 bits [n][K]; items: (group, row0,
+    rows) or None (dense).  Returns the output array as the kernel writes it."""
+    terms = 2 if X_lo is not None else 1
+    n_a = 2 if W2 is not None else 1
+    a_bytes = BM * BK * 2
+    bmax_bytes = n_max * 128
+    stage_bytes = n_a * a_bytes + terms * bmax_bytes
+    stages = min(smem_budget // stage_bytes, 16)
+    acc_cols = n_max * n_a
+    tmem_cols = 32
+    while tmem_cols < 2 * acc_cols:
+        tmem_cols <<= 1
+    assert tmem_cols <= 512
+    nkb = K // BK // k_splits
+    m_tiles = -(-rows_a // BM)
+    n_tokens = X_hi.shape[0]
+    dense = items is None
+    chunks = -(-n_tokens // n_max)
+    n_items = chunks * k_splits if dense else len(items)
+    n_tiles = n_items * m_tiles
+    swiglu = W2 is not None
+    if swiglu:
+        out = np.full((n_tokens, ld_out), np.nan)
+        out_lo = np.zeros((n_tokens, ld_out))
+    else:
+        out = np.full(k_splits * split_stride if k_splits > 1 else n_tokens * ld_out, np.nan)
+        out_lo = None
+
+    def tile_of(t):
+        item, m = t // m_tiles, t % m_tiles
+        if dense:
+            chunk, split = item // k_splits, item % k_splits
+            row0 = chunk * n_max
+            return 0, row0, min(n_max, n_tokens - row0), split, m
+        g, row0, rows = items[item]
+        return g, row0, rows, 0, m
+
+    for cta in range(min(grid, n_tiles)):
+        sm, tm = T.Smem(stages * stage_bytes), T.Tmem(tmem_cols)
+        tiles = list(range(cta, n_tiles, grid))
+        its = [(t, kb) for t in tiles for kb in range(nkb)]
+        loaded = mma_done = 0
+        pending = []
+
+        def load(it):
+            t, kb = its[it]
+            g, row0, rows, split, m = tile_of(t)
+            n_pad = (rows + 15) & ~15
+            sa = (it % stages) * stage_bytes
+            sb = sa + n_a * a_bytes
+            kx = (split * nkb + (kb + t) % nkb) * BK
+            sm.tma_load(sa, W, (kx, m * BM, g), (64, 128, 1), 128)
+            if n_a == 2:
+                sm.tma_load(sa + a_bytes, W2, (kx, m * BM, g), (64, 128, 1), 128)
+            r = 0
+            lo_off = bmax_bytes if bug != "lo_offset" else n_pad * 64
+            while r + 64 <= n_pad:
+                sm.tma_load(sb + r * 128, X_hi, (kx, row0 + r), (64, 64), 128)
+                if terms == 2:
+                    sm.tma_load(sb + lo_off + r * 128, X_lo, (kx, row0 + r), (64, 64), 128)
+                r += 64
+            while r < n_pad:
+                sm.tma_load(sb + r * 128, X_hi, (kx, row0 + r), (64, 16), 128)
+                if terms == 2:
+                    sm.tma_load(sb + lo_off + r * 128, X_lo, (kx, row0 + r), (64, 16), 128)
+                r += 16
+
+        def epilogue(j, t):
+            g, row0, rows, split, m = tile_of(t)
+            d0 = (j & 1) * acc_cols
+            f = m * BM + np.arange(BM)
+            ok = f < rows_a
+            for col in range(rows):
+                a = tm.f32(d0 + col, 1)[:, 0].astype(np.float64)
+                if swiglu:
+                    b = tm.f32(d0 + n_max + col, 1)[:, 0].astype(np.float64)
+                    hv = (a / (1.0 + np.exp(-a)) * b).astype(np.float32)
+                    hi = T.bf16_value(T.bf16_bits(hv)).astype(np.float64)
+                    out[row0 + col, f[ok]] = hi[ok]
+                    out_lo[row0 + col, f[ok]] = T.bf16_value(T.bf16_bits((hv - hi).astype(np.float32)))[ok]
+                else:
+                    slab = split * split_stride if bug != "no_slab" else 0
+                    out[slab + (row0 + col) * ld_out + f[ok]] = a[ok]
+
+        for it in range(len(its)):
+            while loaded < len(its) and loaded < mma_done + stages:
+                load(loaded)
+                loaded += 1
+            t, kb = its[it]
+            j = tiles.index(t)
+            if kb == 0:
+                while pending and pending[0][0] <= j - 2:
+                    epilogue(*pending.pop(0))
+            g, row0, rows, split, m = tile_of(t)
+            n_pad = (rows + 15) & ~15
+            d0 = (j & 1) * acc_cols
+            d1 = d0 + (n_max if bug != "d1" else acc_cols // 4)
+            sa = (it % stages) * stage_bytes
+            sb = sa + n_a * a_bytes
+            for kk in range(BK // 16):
+                acc = kb != 0 or kk != 0
+                T.mma_ss(tm, sm, d0, sa + kk * 32, sb + kk * 32, BM, n_pad, acc)
+                if terms == 2:
+                    T.mma_ss(tm, sm, d0, sa + kk * 32, sb + bmax_bytes + kk * 32, BM, n_pad, True)
+                if n_a == 2:
+                    T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + kk * 32, BM, n_pad, acc)
+                    if terms == 2:
+                        T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + bmax_bytes + kk * 32, BM, n_pad, True)
+            mma_done += 1
+            if kb == nkb - 1:
+                pending.append((j, t))
+        while pending:
+            epilogue(*pending.pop(0))
+    return out, out_lo
+
+
+def bf16_pair(rng, n, K):
+    x = rng.standard_normal((n, K)).astype(np.float32)
+    hi = T.bf16_bits(x)
+    lo = T.bf16_bits((x - T.bf16_value(hi)).astype(np.float32))
+    return T.bf16_value(hi).astype(np.float64) + T.bf16_value(lo), hi, lo
+
+
+def weights(rng, G, rows, K):
+    w = T.bf16_bits((rng.standard_normal((G, rows, K)) * 0.05).astype(np.float32))
+    return w, T.bf16_value(w).astype(np.float64)
+
+
+def test_dense_two_term_split_k_gemm_replay():
+    """The QKV / output projection shape: dense tokens in chunks, two terms, split-K slabs
+    (their sum is the product)."""
+    rng = np.random.default_rng(1)
+    n, rows, K, ks = 150, 320, 512, 2
+    x, hi, lo = bf16_pair(rng, n, K)
+    W, w = weights(rng, 1, rows, K)
+    out, _ = run_gemm(W, hi, lo, rows, K, rows, n_max=128, k_splits=ks, split_stride=n * rows)
+    got = out.reshape(ks, n, rows).sum(axis=0)
+    ref = x @ w[0].T
+    assert np.abs(got - ref).max() / np.abs(ref).max() < 2e-6
+
+
+def test_grouped_gate_up_swiglu_replay():
+    rng = np.random.default_rng(2)
+    counts, F, K = [20, 0, 150, 7], 192, 256
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
+    items = [(e, r0, min(128, off[e + 1] - r0)) for e in range(4) for r0 in range(off[e], off[e + 1], 128)]
+    x, hi, lo = bf16_pair(rng, int(off[-1]), K)
+    Wg, wg = weights(rng, 4, F, K)
+    Wu, wu = weights(rng, 4, F, K)
+    out, out_lo = run_gemm(Wg, hi, lo, F, K, F, items=items, n_max=128, W2=Wu)
+    got = out + out_lo
+    for e in range(4):
+        xe = x[off[e]:off[e + 1]]
+        if len(xe):
+            ref = O.silu(xe @ wg[e].T) * (xe @ wu[e].T)
+            assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-4, e
+
+
+def test_vocab_single_term_replay():
+    """The vocabulary projection shape: one term, all tokens in one chunk of up to 256."""
+    rng = np.random.default_rng(3)
+    n, V, K = 200, 384, 128
+    _, hi, _ = bf16_pair(rng, n, K)
+    x = T.bf16_value(hi).astype(np.float64)
+    W, w = weights(rng, 1, V, K)
+    out, _ = run_gemm(W, hi, None, V, K, V, n_max=208)
+    ref = x @ w[0].T
+    assert np.abs(out.reshape(n, V) - ref).max() / np.abs(ref).max() < 2e-6
+
+
+@pytest.mark.parametrize("bug", ["d1", "no_slab", "lo_offset"])
+def test_planted_mistakes_in_the_gemm_replay_are_caught(bug):
+    rng = np.random.default_rng(4)
+    if bug == "d1":
+        counts, F, K = [40, 90], 128, 128
+        off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
+        items = [(e, r0, min(64, off[e + 1] - r0)) for e in range(2) for r0 in range(off[e], off[e + 1], 64)]
+        x, hi, lo = bf16_pair(rng, int(off[-1]), K)
+        Wg, wg = weights(rng, 2, F, K)
+        Wu, wu = weights(rng, 2, F, K)
+        out, out_lo = run_gemm(Wg, hi, lo, F, K, F, items=items, n_max=64, W2=Wu, bug=bug)
+        ref = O.silu(x[:40] @ wg[0].T) * (x[:40] @ wu[0].T)
+        got = (out + out_lo)[:40]
+    else:
+        n, rows, K, ks = 60, 128, 256, 2
+        x, hi, lo = bf16_pair(rng, n, K)
+        W, w = weights(rng, 1, rows, K)
+        out, _ = run_gemm(W, hi, lo, rows, K, rows, n_max=64, k_splits=ks, split_stride=n * rows, bug=bug)
+        got = np.nan_to_num(out.reshape(ks, n, rows)).sum(axis=0)
+        ref = x @ w[0].T
+    assert np.abs(got - ref).max() / np.abs(ref).max() > 1e-3
