@@ -539,6 +539,63 @@ MUTANTS = {
 }
 
 
+def _qkv_rope_on_v(model, l, x, positions, prec):
+    q, k, v = _orig["_qkv"](model, l, x, positions, prec)
+    return q, k, O.rope(v, positions, model.cfg["rope_theta"])
+
+
+def _qkv_no_rope_on_k(model, l, x, positions, prec):
+    q, _, v = _orig["_qkv"](model, l, x, positions, prec)
+    _, k, _ = _orig["_qkv"](model, l, x, np.zeros_like(positions), prec)   # position 0: no rotation
+    return q, k, v
+
+
+def _qkv_no_rope(model, l, x, positions, prec):
+    return _orig["_qkv"](model, l, x, np.zeros_like(positions), prec)
+
+
+def _attn_out_heads_not_gathered(model, l, o, prec):
+    return o.reshape(o.shape[1], -1) @ O.widen(model.layers[l]["w_o"]).T
+
+
+def _mx_deq_neighbour_scale(codes, exp, block=32):
+    return _orig["mx_e4m3_dequantize"](codes, np.roll(exp, 1, axis=-1), block)
+
+
+def _mx_deq_row_scale(codes, exp, block=32):
+    return _orig["mx_e4m3_dequantize"](codes, np.broadcast_to(exp.max(axis=-1, keepdims=True), exp.shape), block)
+
+
+def _nv_deq_neighbour_scale(codes, sc, g, block=16):
+    return _orig["nvfp4_dequantize"](codes, np.roll(sc, 1, axis=-1), g, block)
+
+
+def _full_states_causal(model, prefix_tokens, canvas, prec):
+    saved = O.block_mask
+    O.block_mask = lambda P, C: O.causal_rows(0, P + C)
+    try:
+        return _orig["full_sequence_states"](model, prefix_tokens, canvas, prec)
+    finally:
+        O.block_mask = saved
+
+
+MUTANTS.update({
+    "RoPE applied to v": ("_qkv", _qkv_rope_on_v, ["test_attention_sees_relative_positions_only"]),
+    "no RoPE on k": ("_qkv", _qkv_no_rope_on_k, ["test_attention_sees_relative_positions_only"]),
+    "no RoPE at all": ("_qkv", _qkv_no_rope, ["test_attention_sees_relative_positions_only"]),
+    "heads not gathered before the output projection": (
+        "_attn_out", _attn_out_heads_not_gathered, ["test_prefix_kv_reuse_equals_full_recompute"]),
+    "mx dequantised with the neighbouring block's scale": (
+        "mx_e4m3_dequantize", _mx_deq_neighbour_scale, ["test_block_scales_stay_with_their_blocks"]),
+    "mx dequantised with one scale per row": (
+        "mx_e4m3_dequantize", _mx_deq_row_scale, ["test_block_scales_stay_with_their_blocks"]),
+    "nvfp4 dequantised with the neighbouring block's scale": (
+        "nvfp4_dequantize", _nv_deq_neighbour_scale, ["test_block_scales_stay_with_their_blocks"]),
+    "full recompute with a causal mask over the canvas": (
+        "full_sequence_states", _full_states_causal, ["test_prefix_kv_reuse_equals_full_recompute"]),
+})
+
+
 def _run_pins(names):
     failed = []
     for n in names:

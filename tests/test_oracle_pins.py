@@ -358,6 +358,51 @@ def test_single_token_pass_closed_form():
     np.testing.assert_allclose(logits[0], nrm(x) @ m.w_out.T, rtol=1e-11, atol=1e-12)
 
 
+def test_attention_sees_relative_positions_only():
+    """RoPE rotates q and k by their absolute positions, so q.k depends on the positions'
+    difference only: shifting every position by the same amount leaves the attention
+    output unchanged, while changing the spacing changes it.  (Rotating v as well, or
+    leaving k unrotated, breaks the first; no rotation at all breaks the second.)"""
+    cfg = _tiny_cfg(n_q_heads=2, n_kv_heads=1)
+    m = _M(cfg)
+    x = np.random.default_rng(5).standard_normal((6, cfg["hidden"]))
+    prec = O.Precision("f32")
+    allowed = np.ones((6, 6), dtype=bool)
+
+    def out(pos):
+        q, k, v = O._qkv(m, 0, x, np.asarray(pos), prec)
+        return O._attn_out(m, 0, O.attention(q, k, v, allowed), prec)
+    base = out(np.arange(6) + 3)
+    np.testing.assert_allclose(out(np.arange(6) + 1000), base, rtol=1e-9, atol=1e-12)
+    assert np.abs(out(2 * np.arange(6) + 3) - base).max() > 1e-3 * np.abs(base).max()
+
+
+def test_block_scales_stay_with_their_blocks():
+    """Rows whose 32- (MX) or 16-element (NVFP4) blocks differ in magnitude by powers of two:
+    every dequantised element is within its own block's rounding bound, which a scale
+    taken from the neighbouring block, or one scale per row, violates."""
+    rng = np.random.default_rng(47)
+    kx = rng.integers(-12, 13, size=(5, 8))                                # per-block magnitudes
+    w = rng.standard_normal((5, 8, 32)) * np.ldexp(1.0, kx)[..., None]
+    w = w.reshape(5, 256)
+    codes, exp = O.mx_e4m3_quantize(w)
+    dq = O.mx_e4m3_dequantize(codes, exp)
+    amax = np.repeat(np.abs(w).reshape(5, 8, 32).max(axis=-1), 32, axis=-1).reshape(w.shape)
+    X = np.repeat(np.ldexp(1.0, exp), 32, axis=-1).reshape(w.shape)
+    # E4M3 keeps 3 mantissa bits down to 2^-6 of the scale: each error within 2^-4 |w| or the
+    # subnormal step 2^-9 X (X <= amax / 2^8), plus what saturation at 448 X cuts off
+    sat = np.maximum(np.abs(w) - 448.0 * X, 0.0)
+    assert np.all(np.abs(dq - w) <= 2.0 ** -4 * np.abs(w) + 2.0 ** -17 * amax + sat)
+    kn = rng.integers(-6, 7, size=(4, 8))
+    w4 = (rng.standard_normal((4, 8, 16)) * np.ldexp(1.0, kn)[..., None]).reshape(4, 128)
+    c4, sc4, g4 = O.nvfp4_quantize(w4)
+    dq4 = O.nvfp4_dequantize(c4, sc4, g4)
+    amax4 = np.repeat(np.abs(w4).reshape(4, 8, 16).max(axis=-1), 16, axis=-1).reshape(w4.shape)
+    # E2M1: half a step, at most a sixth of the block's largest magnitude, plus the block
+    # scale's own E4M3 rounding
+    assert np.all(np.abs(dq4 - w4) <= (1 / 6 + 2.0 ** -4) * amax4 + 1e-12)
+
+
 def test_zero_mixing_weights_pass_is_embedding_readout():
     cfg = _tiny_cfg(n_layers=2)
     m = _M(cfg)
