@@ -215,7 +215,12 @@ dg_status dg_generate_canvases_masked(dg_model* m, dg_kv_cache* caches, int32_t 
 
 /* 8-bit expert weights (MX-FP8 storage: E4M3 codes with one E8M0 power-of-two scale per
  * 32 consecutive K elements of a row; see dg_debug_gemm_mx8 in dg_debug.h for the byte
- * layouts and limits).  Per layer:
+ * layouts and limits).  The pages name FP8 and NVFP4 deployments of the model without a
+ * format ("Module 12. Diffusion Language Models" exercises, the MoE remark); these are the
+ * OCP MX and NVFP4-style block formats, weight-only.  Errors (for these and the output-
+ * matrix setters below): DG_ERR_INVALID_ARG for a NULL model, an fp32 model, NULL or
+ * misaligned pointers or a non-finite tensor scale; DG_ERR_CUDA if a tensor map cannot be
+ * encoded; on any error the model keeps its previous weights.  Per layer:
  *   gate, up     codes [E][F][H],  scales [E][H / 64][F][2]
  *   down         codes [E][H][F],  scales [E][F / 64][H][2]
  * all device pointers, 16-byte aligned, alive and unchanged while set.  Each weight is
