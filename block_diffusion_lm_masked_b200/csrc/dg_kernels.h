@@ -47,7 +47,8 @@ cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2,
                            const CUtensorMap& B2, const CUtensorMap& Bb, const CUtensorMap& B2b, const TcGemmParams& p,
                            int max_tiles, cudaStream_t st);
 // The same GEMM over low-precision weights decoded exactly to bf16 (token maps, work list
-// and epilogues as launch_tc_gemm; n_max <= 64, k_splits == 1).  A / A2: weight codes,
+// and epilogues as launch_tc_gemm; n_max <= 64 with two weight matrices, <= 128 with one;
+// k_splits == 1; dense tiles always weight tile first).  A / A2: weight codes,
 // S / S2: their block scales, as byte tensors.
 //   FMT_MX8: E4M3 codes, 3-D maps (K bytes, rows, groups), box 64 x 128 x 1, 64-byte swizzle;
 //            E8M0 scales [groups][K / 64][rows][2], 3-D maps (2 rows, K / 64, groups), box 256 x 1 x 1.
