@@ -502,6 +502,8 @@ CASES = [
     (3, 2, 2, 64, 600, 664, False),        # group 1: one head per CTA
     (4, 2, 1, 128, 1536, 1664, False),     # long prefix: several splits and a merge
     (5, 2, 1, 300, 0, 300, True),          # causal from an empty cache: own keys throughout
+    (21, 4, 2, 128, 3584, 3712, False),    # long prefix: 12 splits of 5 chunks, slots reused many times
+    (22, 2, 2, 256, 2048, 2304, True),     # causal, two query tiles: the first tile's later splits are empty
 ]
 
 
