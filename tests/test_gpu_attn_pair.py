@@ -68,6 +68,7 @@ CASES = [
     (2, 1, 300, 0, 300, True),         # prefill from an empty cache
     (8, 2, 256, 16128, 16384, False),  # long prefix: the most splits the workspace holds
     (2, 1, 1024, 0, 1024, True),       # causal prefill with splits: early tiles' later splits are empty
+    (16, 8, 256, 32768, 33024, False), # the large model's shape: head pairs of group 2, 9 splits of 58 chunks
 ]
 
 
