@@ -50,6 +50,13 @@ def test_layer1_bf16_batched_full_size(dg):
     PL.check_batched_pass(dg, cfg, [cfg["prefix"], cfg["prefix"] // 2], cfg["canvas"])
 
 
+def test_layer1_bf16_four_canvases_as_the_bench_runs_them(dg):
+    """The bench variant's shape: four canvases over full prefixes (1024 rows, four
+    vocabulary chunks of 256)."""
+    cfg = CF.CONFIGS["layer1_bf16"]
+    PL.check_batched_pass(dg, cfg, [cfg["prefix"]] * 4, cfg["canvas"])
+
+
 def test_batched_pass_equals_single_passes(dg):
     """Canvas b of a batch against the single-canvas call on the same cache: the fp32
     model's kernels compute every row alone, so the logits agree to fp32 rounding; the
