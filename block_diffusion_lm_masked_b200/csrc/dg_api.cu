@@ -559,9 +559,9 @@ int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
 
 // split-KV factor of the head-pair kernel: one wave of CTAs, at least four 64-key chunks
 // per CTA (each CTA loads its query tiles once)
-int attn_pair_splits(int n_q, int nq, int group, int n_keys, int* chunks_per_split) {
+int attn_pair_splits(int n_q, int nq, int group, int pair_heads, int n_keys, int* chunks_per_split) {
   const int nch = ceil_div(n_keys, 64);
-  const int base = ceil_div(n_q, 128) * dg::attn2_head_groups(nq, group);
+  const int base = ceil_div(n_q, 128) * dg::attn2_head_groups(nq, group, pair_heads);
   int splits = dg::num_sms() / base;
   if (splits > kMaxAttnSplits) splits = kMaxAttnSplits;
   if (splits > nch / 4) splits = nch / 4;
@@ -623,7 +623,18 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.causal = causal;
   p.group = nq / nkv;
   p.nq = nq;
-  p.n_splits = attn_pair_splits(n_q, nq, p.group, n_keys, &p.chunks_per_split);
+  // head pairs share each K/V chunk and overlap one head's softmax with the other's MMAs;
+  // single heads give twice the CTAs.  Take whichever fills more of the machine in one
+  // wave (pairs unless single heads fill at least a quarter more SMs).
+  int cps_pair = 0, cps_single = 0;
+  const int sp_pair = attn_pair_splits(n_q, nq, p.group, 1, n_keys, &cps_pair);
+  const int sp_single = attn_pair_splits(n_q, nq, p.group, 0, n_keys, &cps_single);
+  const int q_tiles = ceil_div(n_q, 128);
+  const int ctas_pair = q_tiles * dg::attn2_head_groups(nq, p.group, 1) * sp_pair;
+  const int ctas_single = q_tiles * nq * sp_single;
+  const int pair_heads = (p.group % 2 == 0 && 4 * ctas_single < 5 * ctas_pair) ? 1 : 0;
+  p.n_splits = pair_heads ? sp_pair : sp_single;
+  p.chunks_per_split = pair_heads ? cps_pair : cps_single;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   p.has_lo = 1;
   p.base = base;
@@ -632,7 +643,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.part_o = ws.at<float>(ws.L.part_o);
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
-  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, st));
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, pair_heads, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
            dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, ws.at<bf16>(ws.L.o),

@@ -95,11 +95,13 @@ cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, con
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 // Head-pair variant (same parameters and outputs; chunks_per_split counts 64-key chunks):
-// K / Kl maps with 64-row boxes, Vt / Vtl as above.  Grid y = attn2_head_groups(nq, group).
+// K / Kl maps with 64-row boxes, Vt / Vtl as above.  pair_heads = 1: two heads of one KV
+// head per CTA where the group is even; 0: one head per CTA.  Grid y =
+// attn2_head_groups(nq, group, pair_heads).
 cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
                                  const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
-                                 const TcAttnParams& p, cudaStream_t st);
-int attn2_head_groups(int nq, int group);
+                                 const TcAttnParams& p, int pair_heads, cudaStream_t st);
+int attn2_head_groups(int nq, int group, int pair_heads);
 // the head-pair path's split merge (same inputs and outputs as launch_attn_merge, d = 128):
 // one warp per (row, head), n_splits <= 32
 cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,

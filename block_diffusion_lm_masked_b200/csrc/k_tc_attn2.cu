@@ -2,9 +2,9 @@
 // modes, the same hi + lo precision terms, the same lazy rescale and split-KV partials),
 // organised for more tensor-core overlap per CTA.
 //
-// One CTA = two query heads of one KV head (one head when the GQA group is odd) x 128
-// query rows x a contiguous range of 64-key chunks.  Each K/V chunk is loaded once for
-// both heads.  Warps 0-3 run the softmax of the first head and warps 4-7 that of the
+// One CTA = two query heads of one KV head (one head when the GQA group is odd, or when
+// the host asks for single heads because they fill more SMs) x 128 query rows x a
+// contiguous range of 64-key chunks.  Each K/V chunk is loaded once for both heads.  Warps 0-3 run the softmax of the first head and warps 4-7 that of the
 // second, one query row per thread over the whole 64-key chunk, so no row statistics are
 // exchanged between warps.  Warp 8 issues the TMA loads, warp 9 the MMAs.
 //
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
                     const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
-                    const TcAttnParams p) {
+                    const TcAttnParams p, const int pair_heads) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_bar;
   __shared__ __align__(8) uint64_t kv_full[A2_SLOTS];  // the slot's TMA loads have landed
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, sp = blockIdx.z;
-  const int nh = (p.group % 2 == 0) ? 2 : 1;
+  const int nh = (pair_heads && p.group % 2 == 0) ? 2 : 1;
   const int h0 = blockIdx.y * nh;
   const int kvh = h0 / p.group;
   const int q_row0 = qt * A2_BQ;
@@ -486,15 +486,15 @@ cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n
                   out, out_lo);
 }
 
-int attn2_head_groups(int nq, int group) { return (group % 2 == 0) ? nq / 2 : nq; }
+int attn2_head_groups(int nq, int group, int pair_heads) { return (pair_heads && group % 2 == 0) ? nq / 2 : nq; }
 
 cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
                                  const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
-                                 const TcAttnParams& p, cudaStream_t st) {
+                                 const TcAttnParams& p, int pair_heads, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(tc_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, A2_SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.n_q + A2_BQ - 1) / A2_BQ, attn2_head_groups(p.nq, p.group), p.n_splits);
-  return launch_k(tc_attn2_kernel, grid, dim3(A2_THREADS), A2_SMEM, st, Q, Ql, K, Vt, Kl, Vtl, p);
+  dim3 grid((p.n_q + A2_BQ - 1) / A2_BQ, attn2_head_groups(p.nq, p.group, pair_heads), p.n_splits);
+  return launch_k(tc_attn2_kernel, grid, dim3(A2_THREADS), A2_SMEM, st, Q, Ql, K, Vt, Kl, Vtl, p, pair_heads);
 }
 
 }  // namespace dg

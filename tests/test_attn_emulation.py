@@ -19,7 +19,7 @@ import pytest
 
 import tc_emu as T
 from oracle import dg_oracle as O
-from test_attn_geometry import lo_rows, splits_pair, splits_single
+from test_attn_geometry import choose_pair, lo_rows, splits_single
 
 D = 128
 NEG = np.float32(-np.inf)
@@ -328,13 +328,17 @@ def run_single(c, bug=None):
 
 
 # ---------------------------------------------------------------- tc_attn2_kernel
-def run_pair(c, bug=None):
+def run_pair(c, bug=None, force_pair=None):
     """tc_attn2_kernel: a head pair (one head for odd groups) x 128 rows x 64-key chunks,
     three 32 KB slots, per head S/P buffers at 256 hl + 64 b and O at 256 hl + 128."""
     nq, nkv, n_q, pos0, n_keys, causal = (c[k] for k in ("nq", "nkv", "n_q", "pos0", "n_keys", "causal"))
     m = maps(c)
     group = nq // nkv
-    n_splits, cps = splits_pair(n_q, nq, group, n_keys)
+    pair, n_splits, cps = choose_pair(n_q, nq, group, n_keys)
+    if force_pair is not None:                       # either mode, whatever the host would choose
+        from test_attn_geometry import splits_pair
+        pair = force_pair and group % 2 == 0
+        n_splits, cps = splits_pair(n_q, nq, group, n_keys, pair)
     W, QBLK, KBLK = 64, 128 * 128, 64 * 128
     QHEAD, VOFF = 4 * QBLK, 2 * KBLK
     SLOT = VOFF + QBLK
@@ -347,7 +351,7 @@ def run_pair(c, bug=None):
     else:
         p_lo = 32
     scale = np.float32(1.4426950408889634 / math.sqrt(D))
-    nh = 2 if group % 2 == 0 else 1
+    nh = 2 if pair else 1
     out = np.zeros((n_q, nq * D), np.float32)
     out_lo = np.zeros_like(out)
     part_o = np.zeros((n_splits, nq, n_q, D), np.float32)
@@ -514,10 +518,12 @@ def test_validated_kernel_replay_matches_the_oracle(case):
     assert within(run_single(c), oracle(c))
 
 
+@pytest.mark.parametrize("force_pair", [None, True, False])
 @pytest.mark.parametrize("case", CASES)
-def test_head_pair_kernel_replay_matches_the_oracle(case):
+def test_head_pair_kernel_replay_matches_the_oracle(case, force_pair):
+    """As the host chooses, and in both modes (two heads per CTA, one head per CTA)."""
     c = build(*case)
-    assert within(run_pair(c), oracle(c))
+    assert within(run_pair(c, force_pair=force_pair), oracle(c))
 
 
 @pytest.mark.parametrize("bug", ["p_lo_offset", "no_pv_first"])
