@@ -88,6 +88,8 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
   uint32_t tmem_cols = 32;
   while (tmem_cols < (uint32_t)(2 * acc_cols)) tmem_cols <<= 1;
   const int nkb = p.K / VU_BK;
+  // tile t = (id tile t / chunks, token chunk t % chunks): the CTAs that share an id tile's
+  // weights run together, so the output matrix is read from DRAM once for all chunks
   const int chunks = (p.n_tokens + p.n_max - 1) / p.n_max;
   const int n_tiles = chunks * p.m_tiles;
 
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const int m = t % p.m_tiles, row0 = (t / p.m_tiles) * p.n_max;
+        const int m = t / chunks, row0 = (t % chunks) * p.n_max;
         const int rows = min(p.n_max, p.n_tokens - row0);
         const int n_pad = (rows + 15) & ~15;
         const uint32_t tx = a_bytes + (uint32_t)n_pad * 128u;
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
       int it = 0, j = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++j) {
-        const int row0 = (t / p.m_tiles) * p.n_max;
+        const int row0 = (t % chunks) * p.n_max;
         const int n_pad = (min(p.n_max, p.n_tokens - row0) + 15) & ~15;
         const int buf = j & 1;
         if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     int j = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++j) {
-      const int m = t % p.m_tiles, row0 = (t / p.m_tiles) * p.n_max;
+      const int m = t / chunks, row0 = (t % chunks) * p.n_max;
       const int rows = min(p.n_max, p.n_tokens - row0);
       const int n_pad = (rows + 15) & ~15;
       const int buf = j & 1;

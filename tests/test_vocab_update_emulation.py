@@ -1,8 +1,8 @@
 """The fused vocabulary/update kernel (tc_vocab_update_kernel, then upd_merge_rows_kernel)
 replayed at the address level on the CPU (tests/tc_emu.py), against the oracle's update.
 
-Transcribed from the kernel source: the persistent walk over (token chunk, 128-id tile)
-tiles with its k-block rotation, the stage layout (weight tile, then token boxes of 64
+Transcribed from the kernel source: the persistent walk over (128-id tile, token chunk)
+tiles, id tile first, with its k-block rotation, the stage layout (weight tile, then token boxes of 64
 and 16 rows), the MMAs into one of two accumulator buffers, and the statistics epilogue:
 warp lg's lane holds id m 128 + 32 lg + lane, each 16-column chunk is reduced per column
 by butterflies (max with the first argmax, the candidate skipping an excluded id, the sum
@@ -79,7 +79,7 @@ def run_vocab_update(Wout, X, V, excl, n_max, smem_budget=200 * 1024, grid=5, bu
         pending = []
 
         def geom(t):
-            m, row0 = t % m_tiles, (t // m_tiles) * n_max
+            m, row0 = t // chunks, (t % chunks) * n_max            # id tile first, then token chunk
             rows = min(n_max, C - row0)
             return m, row0, rows, (rows + 15) & ~15
 
