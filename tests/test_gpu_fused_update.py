@@ -58,10 +58,14 @@ def test_fused_update_equals_the_two_call_path(dg, cfg, P, C):
     (ta, ca, logits), (tb, cb) = _both(dg, st, canvas0, n)
     np.testing.assert_allclose(cb, ca, rtol=2e-5)
     order = np.argsort(ca, kind="stable")
-    cut_lo, cut_hi = ca[order[n - 1]], ca[order[n]] if n < C else np.inf
-    close = np.abs(ca - cut_lo) < 1e-4 * cut_lo or np.abs(ca - cut_hi) < 1e-4 * cut_hi
+    cut_lo, cut_hi = ca[order[n - 1]], (ca[order[n]] if n < C else np.inf)
+    close = (np.abs(ca - cut_lo) < 1e-4 * cut_lo) | (np.abs(ca - cut_hi) < 1e-4 * cut_hi)
+    # the two paths' GEMMs may round the logits differently: a position whose top two
+    # logits are that close may take either id
+    top2 = np.sort(logits, axis=1)[:, -2:]
+    near_tie = (top2[:, 1] - top2[:, 0]) <= 1e-5 * np.maximum(np.abs(top2[:, 1]), 1e-30)
     for i in range(C):
-        if not close[i]:
+        if not close[i] and not near_tie[i]:
             assert ta[i] == tb[i], i
 
 
@@ -78,16 +82,23 @@ def test_fused_masked_update_equals_the_two_call_path(dg):
 
 
 def test_fused_update_matches_the_oracle_full_size(dg):
+    """The fused call against the oracle's pass and update.  The rows exempt from the
+    comparison (routing at a near tie, under the pass's parity rules) come from a tapped
+    two-call pass over the same input: the layer stack is the same in both calls."""
     cfg = CF.CONFIGS["layer1_bf16"]
     st = PL.Setup(cfg, cfg["prefix"])
-    C = cfg["canvas"]
+    C, V = cfg["canvas"], cfg["vocab"]
     canvas0 = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
     n = O.renoise_count(C, 1, 0, 0.25, 0.25)
     ws = st.workspace(C)
+    taps = st.taps(C)
+    logits = torch.empty(C, V, device="cuda")
+    dg.denoise_pass(st.model, st.cache, torch.from_numpy(canvas0.astype(np.int32)).cuda(), logits, ws)
+    logits_o, taps_o = O.denoise_pass(st.host, st.ocache, canvas0, st.prec)
+    exempt = PL.compare_pass(cfg, taps, logits.cpu().numpy(), taps_o, logits_o)
     out = torch.from_numpy(canvas0.astype(np.int32)).cuda()
     conf = torch.empty(C, device="cuda")
     dg.denoise_update(st.model, st.cache, out, n, ws, seed=synth.SEED_RENOISE, step=0, conf=conf)
     dg.device_status(ws)
-    logits_o, _ = O.denoise_pass(st.host, st.ocache, canvas0, st.prec)
     upd_o = O.canvas_update(logits_o, n, synth.SEED_RENOISE, 0)
-    PL.compare_update(out.cpu().numpy(), conf.cpu().numpy(), upd_o, set(), n)
+    PL.compare_update(out.cpu().numpy(), conf.cpu().numpy(), upd_o, exempt, n)
