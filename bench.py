@@ -351,12 +351,15 @@ def run_variant(args, cfg, name):
             kern[kname] = {"launches": n, "avg_us": ms * 1e3 / n, "share": ms / max(prof_ms, 1e-9)}
 
     h_in, h_out = noise.clone().pin_memory(), torch.empty_like(noise).pin_memory()
+    # the step's input: the canvases the batched pass reads, or for the fused call the canvas
+    # it reads and overwrites
+    dst_in = canv_out if args.fused_update else canv_in
     e2e_ms = []
     for s_ in range(args.steps + args.warmup):
         flush.zero_()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        canv_in.copy_(h_in, non_blocking=True)
+        dst_in.copy_(h_in, non_blocking=True)
         step(s_)
         h_out.copy_(canv_out, non_blocking=True)
         b_.record(stream)
