@@ -61,3 +61,11 @@ def test_the_parser_sees_the_known_shapes():
                                                          "float tensor_scale"])
     assert d["dg_launch_count"][1] == [] and d["dg_last_error"][0] == "const char*"
     assert len(d["dg_debug_attention_pair_bf16"][1]) == 15
+
+
+def test_kernel_kinds_follow_the_library_numbering():
+    """The binding's kernel-kind names (used to label the bench's per-kernel times) are the
+    library's, in its order, and cover every kind."""
+    got = [dg.lib.dg_kernel_name(i).decode() for i in range(len(dg.KERNEL_KINDS))]
+    assert got == dg.KERNEL_KINDS
+    assert dg.lib.dg_kernel_name(len(dg.KERNEL_KINDS)).decode() == "?"
