@@ -414,6 +414,58 @@ def run_variant(args, cfg, name):
     return 0
 
 
+def run_kernel_attention(args):
+    """--kernel attention: the block-masked attention launch alone (debug entry: the
+    attention kernel and its split-KV merge) on synthetic bf16 data, the canvas's queries
+    at the last positions of the key range, bidirectional.  One JSON line: median
+    CUDA-event time per call and the algorithmic FLOP rate 4 * queries * heads * d * keys
+    / time against the bf16 peak.  Used for ncu captures of attention at a chosen key
+    count without the rest of the model on the device."""
+    import torch
+
+    from block_diffusion_lm_masked_b200 import dg
+
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(7)
+    d, n_q, n_keys, nq, nkv = 128, args.queries, args.keys, args.heads, args.kv_heads
+    cap = ((n_keys + 7) // 8) * 8
+    q = torch.randn(nq, n_q, d, generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn(nkv, cap, d, generator=g, device=dev).to(torch.bfloat16)
+    vt = torch.randn(nkv, d, cap, generator=g, device=dev).to(torch.bfloat16)
+    cfg = dict(CF.CONFIGS["layer1_bf16"], n_q_heads=nq, n_kv_heads=nkv, hidden=128, expert_ffn=64, n_experts=1,
+               top_k=1, vocab=128, n_layers=1)
+    ws = dg.Workspace(cfg, n_q, dev)
+    out = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device=dev)
+    lo = torch.zeros_like(out)
+    fn = dg.debug_attention_pair_bf16 if args.attn_pair else dg.debug_attention_bf16
+    for _ in range(args.warmup):
+        fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo)
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    dg.device_status(ws)
+    us = statistics.median(ts)
+    hbm, tf_burst, _, peak_src = _peaks()
+    fl = 4.0 * n_q * nq * d * n_keys
+    tf = fl / (us * 1e-6) / 1e12
+    line = {"metric": "block-masked attention call latency (attention + split-KV merge)", "value": us, "unit": "us",
+            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+            "data": "synthetic: q, K, V ~ N(0,1) bf16",
+            "config": {"workload": f"attention: {n_q} queries x {nq} heads ({nkv} KV heads) d{d} over {n_keys} keys, "
+                                   f"bidirectional", "attention": "head pairs, 64-key chunks" if args.attn_pair
+                       else "one head, 128-key chunks", "l2": "K/V re-read between calls"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s", "frac": tf / tf_burst,
+                         "flops_per_call": fl, "peak_source": f"{peak_src} bf16_tflops"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def _attention_kind():
     """Which attention kernel the library runs (DG_ATTN_PAIR=1: the head-pair kernel)."""
     return ("head pairs, 64-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
@@ -439,7 +491,16 @@ def main():
                     help="output-matrix storage; mx8 and nv4 run through the batched calls")
     ap.add_argument("--attn-pair", action="store_true",
                     help="run the pass's attention through the head-pair kernel (sets DG_ATTN_PAIR=1)")
+    ap.add_argument("--kernel", choices=["attention"], default=None,
+                    help="time one kernel alone on synthetic data instead of the step (attention: the "
+                         "block-masked attention call over --keys keys)")
+    ap.add_argument("--keys", type=int, default=8192, help="--kernel attention: key count")
+    ap.add_argument("--queries", type=int, default=256, help="--kernel attention: canvas queries")
+    ap.add_argument("--heads", type=int, default=16, help="--kernel attention: query heads")
+    ap.add_argument("--kv-heads", type=int, default=8, help="--kernel attention: KV heads")
     args = ap.parse_args()
+    if args.kernel == "attention":
+        return run_kernel_attention(args)
     if args.attn_pair:  # read by the library at its first attention call
         os.environ["DG_ATTN_PAIR"] = "1"
     name = args.workload

@@ -146,6 +146,21 @@ bool inject_launch_fault() {
     if (_e != cudaSuccess) return fail(DG_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(_e));          \
   } while (0)
 
+namespace dg {
+// one launch through the same wrapper as every other entry point (fault injection,
+// launch count, NVTX range, per-kind event timing), for entry points in other files
+dg_status launch_wrapped(int kind, cudaStream_t st, const char* what, cudaError_t (*fn)(void*), void* arg) {
+  if (inject_launch_fault()) return fail(DG_ERR_CUDA, "%s: injected launch failure", what);
+  cudaError_t e;
+  {
+    ProfScope ps(kind, st);
+    e = fn(arg);
+  }
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return DG_OK;
+}
+}  // namespace dg
+
 // ---------------------------------------------------------------- tensor maps
 static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode{nullptr};
 static std::mutex g_encode_mu;
