@@ -125,12 +125,10 @@ def _oracle_step(host, ocache, canvas, n, prec, step):
     return O.canvas_update(logits, n, synth.SEED_RENOISE, step)
 
 
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max(i.get("num_threads", 1) for i in threadpool_info())
-    except Exception:
-        return os.cpu_count() or 1
+def _oracle_threads():
+    """Host threads the C++ oracle's OpenMP loops run on."""
+    from oracle import dg_oracle as O
+    return O.num_threads()
 
 
 REF_BUDGET_S = 90.0
@@ -178,8 +176,8 @@ def run_reference(args, cfg, name):
     dt = time.perf_counter() - t0
     ms = dt * 1e3 / done
     value = C / (ms / 1e3)
-    cores = _blas_threads()
-    sample = (f"{done} of {args.steps} requested whole oracle steps (pass + update, fp64 numpy) of the workload, "
+    cores = _oracle_threads()
+    sample = (f"{done} of {args.steps} requested whole oracle steps (pass + update, fp64 C++ with OpenMP) of the workload, "
               f"{REF_BUDGET_S:.0f} s budget")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -207,8 +205,8 @@ def cpu_baseline(cfg, budget_s=30.0):
         _oracle_step(host, ocache, canvas, n, prec, 0)
         times.append(time.perf_counter() - t0)
     ms = statistics.median(times) * 1e3
-    return {"value": C / (ms / 1e3), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{len(times)} whole oracle steps (denoising pass + update, fp64 numpy) of the workload; "
+    return {"value": C / (ms / 1e3), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{len(times)} whole oracle steps (denoising pass + update, fp64 C++ with OpenMP) of the workload; "
                       f"median {ms:.0f} ms per step"}
 
 

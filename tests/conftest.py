@@ -16,6 +16,9 @@ def pytest_configure(config):
     from block_diffusion_lm_masked_b200 import build as B
     if not os.path.exists(B.LIB):
         B.build()
+    # the C++ oracle likewise (test infrastructure; rebuilt when its source is newer)
+    from oracle import build as OB
+    OB.build()
 
 
 def golden_path(name):

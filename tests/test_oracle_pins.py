@@ -304,6 +304,23 @@ def test_moe_identical_experts_equals_dense_swiglu():
     np.testing.assert_allclose(got, _swiglu(xn, L["w_gate"][0], L["w_up"][0], L["w_down"][0]), rtol=1e-12, atol=1e-13)
 
 
+def test_moe_router_reads_the_normed_residual():
+    """Pre-norm MoE (reading #1): the block sees the residual only through its RMSNorm, so
+    with eps = 0 scaling a token's residual by any c > 0 changes neither its routing (the
+    router logits, hence the top-k and their softmax weights) nor its FFN output."""
+    cfg = _tiny_cfg(rms_eps=0.0, n_experts=6, top_k=3)
+    m = _M(cfg)
+    x = np.random.default_rng(21).standard_normal((8, cfg["hidden"]))
+    c = np.array([0.25, 0.5, 1.0, 3.0, 7.0, 0.1, 2.0, 40.0])[:, None]
+    a = O.moe_block(m, 0, x, O.Precision("f32"))
+    b = O.moe_block(m, 0, c * x, O.Precision("f32"))
+    np.testing.assert_allclose(b["router_logits"], a["router_logits"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(b["topk_idx"], a["topk_idx"])
+    np.testing.assert_allclose(b["topk_w"], a["topk_w"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(b["ffn"], a["ffn"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(b["x_out"], c * x + a["ffn"], rtol=1e-11, atol=1e-11)
+
+
 def test_moe_k1_routes_each_token_to_its_argmax_expert():
     cfg = _tiny_cfg(top_k=1)
     m = _M(cfg)
@@ -464,7 +481,9 @@ def _is_nearest_bf16(stored, exact):
 def test_bf16_storage_rounds_what_prefill_writes_and_nothing_in_flight():
     """The storage rule in a bf16 model: prefill rounds the K/V it writes to the nearest
     bf16 value and nothing else, so its residual stream matches the f32 model's; a
-    denoising pass rounds only the vocabulary input, never the canvas K/V it computes."""
+    denoising pass rounds nothing at all (canvas K/V, vocabulary input in flight), so
+    against a given cache the two precisions give the same logits, the plain product of
+    the normed final state and the output matrix."""
     cfg = _tiny_cfg(n_layers=2)
     m = _M(cfg)
     toks = np.array([4, 8, 15, 16, 23, 2])
@@ -475,8 +494,6 @@ def test_bf16_storage_rounds_what_prefill_writes_and_nothing_in_flight():
         for a, b in ((stored.k[l], exact.k[l]), (stored.v[l], exact.v[l])):
             assert _is_nearest_bf16(a, b)
             assert np.abs(a - b).max() > 0
-    # a pass against a given cache: identical residual streams, logits differ only by the
-    # rounding of the final normed state
     can = np.array([7, 30, 1])
     lf, tf = O.denoise_pass(m, stored, can, f32)
     lb, tb = O.denoise_pass(m, stored, can, b16)
@@ -484,8 +501,8 @@ def test_bf16_storage_rounds_what_prefill_writes_and_nothing_in_flight():
         for key in ("attn_o", "x_attn", "x_out"):
             np.testing.assert_array_equal(a[key], b[key])
     xn = O.rms_norm(tf[-1]["x_out"], cfg["rms_eps"])
-    np.testing.assert_allclose(lb, O.round_bf16(xn) @ m.w_out.T, rtol=1e-12, atol=1e-13)
-    assert np.abs(lb - lf).max() > 0
+    np.testing.assert_allclose(lb, xn @ m.w_out.T, rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(lb, lf)
 
 
 def test_denoise_pass_leaves_cache_untouched():
