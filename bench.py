@@ -2,13 +2,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 
-Workload (default): the single-layer bf16 pass -- hidden 2048, 16 query / 4 KV heads
-of 128, 64 experts top-4 with FFN 1024, vocabulary 32768, 1024 cached prefix
-positions (K/V ~ N(0,1)), a 256-slot canvas of uniform random tokens; one step =
-dg_denoise_pass + dg_canvas_update (25% re-noised).  Weights are seeded N(0, 0.02)
-bf16 (synthetic, random init).  The metric is canvas tokens per second per pass
-(C / step latency), summed over ranks; each rank runs its own replica (no data-path
-collective: the pass does not shard), so scaling is weak.
+Workload (default): the large pass -- 4 layers, hidden 2816, 16 query / 8 KV heads of
+128, 128 experts top-8 with FFN 704, vocabulary 262144, 32768 cached prefix positions
+(K/V ~ N(0,1)), a 256-slot canvas of uniform random tokens; one step = dg_denoise_pass +
+dg_canvas_update (the first of its 8 steps: 50% re-noised).  The largest of the five
+workloads that fits one GPU.  `--workload layer1_bf16` runs the single-layer pass
+(hidden 2048, 64 experts top-4, vocabulary 32768, prefix 1024), `denoise8_bf16` the
+8-layer one (prefix 2048), and `chained8_bf16` whole chains: a 512-token prompt
+prefilled, then 4 canvases of 16 passes each, every canvas appended by prefill.
+Weights are seeded N(0, 0.02) bf16 (synthetic, random init).  The metric is canvas
+tokens per second per pass (C / step latency), summed over ranks; each rank runs its
+own replica (no data-path collective: the pass does not shard), so scaling is weak.
 
 Prints ONE JSON line on rank 0.  --impl reference times the CPU oracle instead (a
 bounded sample of the same workload on the host cores).
@@ -47,9 +51,10 @@ def _peaks():
 
 
 def _workload_desc(name, cfg):
+    where = f"prompt {cfg['prompt']} then {cfg['n_canvases']} canvases" if "prompt" in cfg else f"P{cfg['prefix']}"
     return (f"{name}: {cfg['n_layers']} layer(s), H{cfg['hidden']}, {cfg['n_q_heads']}q/{cfg['n_kv_heads']}kv "
             f"d{cfg['head_dim']}, E{cfg['n_experts']} top-{cfg['top_k']}, F{cfg['expert_ffn']}, V{cfg['vocab']}, "
-            f"P{cfg['prefix']}, C{cfg['canvas']}; step = 1 denoising pass + canvas update")
+            f"{where}, C{cfg['canvas']}; step = 1 denoising pass + canvas update")
 
 
 class Clocks:
@@ -133,23 +138,44 @@ def _oracle_threads():
 
 REF_BUDGET_S = 90.0
 
-# DRAM bytes (read + write) of one gate/up GEMM launch from an ncu capture of this
-# workload, valid only for the kernel source it was taken on (sha256 prefix of
-# k_tc_gemm.cu); any other source reports null.
-NCU_TRAFFIC = {"layer1_bf16": ("8f9740b8fc51d669", 457.380608e6 + 6.031104e6)}
+# DRAM bytes (read + write) of one launch of a kernel from an ncu capture of this
+# workload, valid only for the kernel source it was taken on (sha256 prefix of the
+# kernel's source file); any other source reports null.
+NCU_TRAFFIC = {("layer1_bf16", "gemm_gate_up"): ("k_tc_gemm.cu", "8f9740b8fc51d669", 457.380608e6 + 6.031104e6)}
 
 
-def _ncu_traffic(workload):
+def _ncu_traffic(workload, kernel):
     import hashlib
-    entry = NCU_TRAFFIC.get(workload)
+    entry = NCU_TRAFFIC.get((workload, kernel))
     if entry is None:
         return None
-    src = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", "k_tc_gemm.cu")
+    src = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", entry[0])
     try:
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except OSError:
         return None
-    return entry[1] if digest == entry[0] else None
+    return entry[2] if digest == entry[1] else None
+
+
+def _oracle_sample(cfg, host=None):
+    """The oracle's inputs for a bounded sample of the workload: (model, cache, canvas,
+    re-noise count, precision, what the sample is).  A denoising workload's cached prefix
+    is its seeded N(0,1) K/V; the chained workload's first canvas runs after the oracle's
+    own prefill of the 512-token prompt (set-up, not timed)."""
+    from oracle import dg_oracle as O
+    C = cfg["canvas"]
+    host = host if host is not None else synth.Model(cfg)
+    prec = O.Precision(cfg["dtype"])
+    if "prompt" in cfg:
+        prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, cfg["prompt"], cfg["vocab"])
+        ocache = O.prefill_append(host, O.Cache.empty(cfg), prompt, prec)
+        what = "passes + updates of the first canvas after the prompt's prefill (set-up, untimed)"
+    else:
+        ocache = O.Cache(synth.prefix_cache(cfg, cfg["prefix"]))
+        what = "whole oracle steps (denoising pass + update)"
+    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
+    n = O.renoise_count(C, cfg["steps"], 0, cfg["renoise_start"], cfg["renoise_end"])
+    return host, ocache, canvas, n, prec, what
 
 
 def run_reference(args, cfg, name):
@@ -157,13 +183,8 @@ def run_reference(args, cfg, name):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from oracle import dg_oracle as O
-    P, C = cfg["prefix"], cfg["canvas"]
-    host = synth.Model(cfg)
-    ocache = O.Cache(synth.prefix_cache(cfg, P))
-    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
-    prec = O.Precision(cfg["dtype"])
-    n = O.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+    C = cfg["canvas"]
+    host, ocache, canvas, n, prec, what = _oracle_sample(cfg)
     # a bounded sample: at most one warm-up step, then whole steps until K are done or
     # REF_BUDGET_S seconds have passed (at least one)
     for w in range(min(args.warmup, 1)):
@@ -177,7 +198,7 @@ def run_reference(args, cfg, name):
     ms = dt * 1e3 / done
     value = C / (ms / 1e3)
     cores = _oracle_threads()
-    sample = (f"{done} of {args.steps} requested whole oracle steps (pass + update, fp64 C++ with OpenMP) of the workload, "
+    sample = (f"{done} of {args.steps} requested {what}, fp64 C++ with OpenMP, of the workload, "
               f"{REF_BUDGET_S:.0f} s budget")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -189,15 +210,11 @@ def run_reference(args, cfg, name):
     return 0
 
 
-def cpu_baseline(cfg, budget_s=30.0):
-    """Time the oracle as it stands on a bounded sample: whole oracle steps until ~budget."""
-    from oracle import dg_oracle as O
-    P, C = cfg["prefix"], cfg["canvas"]
-    host = synth.Model(cfg)
-    ocache = O.Cache(synth.prefix_cache(cfg, P))
-    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
-    prec = O.Precision(cfg["dtype"])
-    n = O.renoise_count(C, 1, 0, cfg["renoise_start"], cfg["renoise_end"])
+def cpu_baseline(cfg, budget_s=30.0, host=None):
+    """Time the oracle as it stands on a bounded sample: whole oracle steps until ~budget
+    (at least one).  `host`: the synthetic model already built for the GPU run."""
+    C = cfg["canvas"]
+    host, ocache, canvas, n, prec, what = _oracle_sample(cfg, host)
     times = []
     t_start = time.perf_counter()
     while not times or (time.perf_counter() - t_start < budget_s / 2 and len(times) < 5):
@@ -206,8 +223,7 @@ def cpu_baseline(cfg, budget_s=30.0):
         times.append(time.perf_counter() - t0)
     ms = statistics.median(times) * 1e3
     return {"value": C / (ms / 1e3), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{len(times)} whole oracle steps (denoising pass + update, fp64 C++ with OpenMP) of the workload; "
-                      f"median {ms:.0f} ms per step"}
+            "sample": f"{len(times)} {what} of the workload, fp64 C++ with OpenMP; median {ms:.0f} ms per step"}
 
 
 class Ranks:
@@ -412,6 +428,196 @@ def run_variant(args, cfg, name):
     return 0
 
 
+def run_chained(args, cfg, name):
+    """--workload chained8_bf16: one step = one whole chain through the public calls --
+    the prompt's prefill (dg_prefill_append), then for each canvas dg_generate_canvas (16
+    passes with re-noising, then the canvas appended by prefill).  The line's value is
+    canvas tokens per second over the chain's passes (canvases x steps x C / chain time,
+    prefills included); the chain's end-to-end time, its prefill times and the passes'
+    median latency are reported beside it."""
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    from block_diffusion_lm_masked_b200 import dg
+
+    T0, C, S, NC, V = cfg["prompt"], cfg["canvas"], cfg["steps"], cfg["n_canvases"], cfg["vocab"]
+    r0, r1 = cfg["renoise_start"], cfg["renoise_end"]
+    cap = T0 + NC * C
+    host = synth.Model(cfg)
+    model = dg.Model(host, dev)
+    cache = dg.KVCache(cfg, cap, dev)
+    ws = dg.Workspace(cfg, max(T0, C), dev)
+    prompt_h = torch.from_numpy(synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, T0, V)).pin_memory()
+    noise_h = torch.from_numpy(np.stack([synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(rank * NC + c), C, V)
+                                         for c in range(NC)])).pin_memory()
+    prompt = prompt_h.to(dev)
+    noise = noise_h.to(dev)
+    canv = noise.clone()
+    logits = torch.empty(C, V, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def chain(s, marks=None):
+        cache.len = 0
+        dg.prefill_append(model, cache, prompt, ws)
+        if marks is not None:
+            marks[0].record(stream)
+        for c in range(NC):
+            canv[c].copy_(noise[c])
+            dg.generate_canvas(model, cache, canv[c], S, r0, r1, synth.SEED_RENOISE + s, True, logits, ws)
+            if marks is not None:
+                marks[c + 1].record(stream)
+
+    for w in range(args.warmup):
+        chain(w)
+    dg.device_status(ws)
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    clk = Clocks(dev)
+    clk.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(NC + 1)] for _ in range(args.steps)]
+    l0 = dg.launch_count()
+    for s_ in range(args.steps):
+        flush.zero_()
+        ev[s_][0].record(stream)
+        chain(s_, marks[s_])
+        ev[s_][1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = dg.launch_count() - l0
+    clocks = clk.stop()
+    dg.device_status(ws)
+    chain_ms = [a.elapsed_time(b) for a, b in ev]
+    prompt_ms = statistics.median(ev[i][0].elapsed_time(marks[i][0]) for i in range(args.steps))
+    canvas_ms = [statistics.median(marks[i][c].elapsed_time(marks[i][c + 1]) for i in range(args.steps))
+                 for c in range(NC)]
+    total_ms = ranks.max(sum(chain_ms))
+    ranks.barrier()
+
+    # the passes alone, and one append, at each canvas's prefix length (per-kernel profile)
+    dg.profile_reset()
+    dg.profile_enable(True)
+    chain(0)
+    torch.cuda.synchronize(dev)
+    dg.profile_enable(False)
+    kern = {}
+    tot = 0.0
+    for kname in dg.KERNEL_KINDS:
+        ms, n = dg.profile_read(kname)
+        if n:
+            kern[kname] = {"launches": n, "avg_us": ms * 1e3 / n}
+            tot += ms
+    for v in kern.values():
+        v["share"] = v["avg_us"] * v["launches"] / 1e3 / max(tot, 1e-9)
+
+    # end to end through the public calls with host buffers: prompt and noise canvases in,
+    # finished canvases out, every chain
+    out_h = torch.empty_like(noise_h).pin_memory()
+    e2e_ms = []
+    for s_ in range(args.steps + args.warmup):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        prompt.copy_(prompt_h, non_blocking=True)
+        noise.copy_(noise_h, non_blocking=True)
+        chain(s_)
+        out_h.copy_(canv, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if s_ >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_total = ranks.max(sum(e2e_ms))
+    dg.device_status(ws)
+
+    hbm, tf_burst, tf_sust, peak_src = _peaks()
+    # roofline of the chain: every pass at its prefix length (expert unions taken as E,
+    # the near-full coverage random routing gives), every prefill
+    E = cfg["n_experts"]
+    t_roof = 0.0
+    flops_total = bytes_total = 0.0
+    for c in range(NC):
+        P = T0 + c * C
+        f = RF.pass_flops(cfg, P, C)
+        b = RF.pass_bytes(cfg, P, C, [E] * cfg["n_layers"]) + 8 * C
+        t_roof += S * RF.time_bound(f, b, tf_burst * 1e12, hbm * 1e9)
+        flops_total += S * f
+        bytes_total += S * b
+    for P, T in [(0, T0)] + [(T0 + c * C, C) for c in range(NC)]:
+        f = RF.prefill_flops(cfg, P, T)
+        b = RF.prefill_bytes(cfg, P, T, [E] * cfg["n_layers"])
+        t_roof += RF.time_bound(f, b, tf_burst * 1e12, hbm * 1e9)
+        flops_total += f
+        bytes_total += b
+    ms_chain = total_ms / args.steps
+    passes = NC * S
+    value = job_value(world, passes * C, args.steps, total_ms)
+    kroof = kernel_rooflines(cfg, T0 + (NC - 1) * C / 2, C, [E] * cfg["n_layers"], kern, hbm, tf_sust, peak_src)
+    roof = None
+    if kroof:
+        dom = max(kroof, key=lambda n: kern[n]["share"])
+        roof = dict(kroof[dom], kernel=dom, traffic=_ncu_traffic(name, dom),
+                    note="per-launch averages over the chain; attention FLOPs at the mean prefix length")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_chain, "pass_latency_us": statistics.median(canvas_ms) * 1e3 / S,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": (f"{name}: {cfg['n_layers']} layers of H{cfg['hidden']}, E{cfg['n_experts']} "
+                                f"top-{cfg['top_k']}, V{V}; a {T0}-token prompt prefilled, then {NC} canvases of "
+                                f"{C} x {S} passes, each appended by prefill; step = one whole chain"),
+                   "l2": "flushed between chains (256 MB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "chain_ms": {"median": statistics.median(chain_ms), "prompt_prefill": prompt_ms,
+                     "per_canvas_incl_append": canvas_ms},
+        "roofline": roof,
+        "chain_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_chain, "flops": flops_total,
+                           "bytes": bytes_total, "peak_source": peak_src},
+        "kernels": kern, "kernel_rooflines": kroof,
+        "e2e": {"value": job_value(world, passes * C, args.steps, e2e_total), "unit": UNIT,
+                "h2d_bytes_per_step": 4 * (T0 + NC * C), "d2h_bytes_per_step": 4 * NC * C,
+                "chain_ms": e2e_total / args.steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, host=host)
+    ranks.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None):
+    """Achieved rate and fraction of its bound for each big kernel of the step: the expert
+    and vocabulary GEMMs and the update statistics against HBM bandwidth (algorithmic
+    bytes per launch), attention against the bf16 tensor peak (algorithmic FLOPs)."""
+    rows = C if rows is None else rows
+    k, L = cfg["top_k"], cfg["n_layers"]
+    out = {}
+
+    def hbm_entry(kname, nbytes_launch):
+        if kname in kern:
+            a = nbytes_launch / (kern[kname]["avg_us"] * 1e-6) / 1e9
+            out[kname] = {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+                          "bytes_per_launch": nbytes_launch, "peak_source": f"{peak_src} hbm_gbs"}
+    hbm_entry("gemm_gate_up", sum(RF.gate_up_bytes(cfg, u, rows * k) for u in unions) / L)
+    hbm_entry("gemm_down", sum(RF.down_bytes(cfg, u, rows * k) for u in unions) / L)
+    hbm_entry("gemm_vocab", RF.vocab_bytes(cfg, rows))
+    hbm_entry("update_partial", RF.update_bytes(cfg, rows))
+    if "attention" in kern:
+        fl = RF.attention_flops(cfg, P, C)
+        a = fl / (kern["attention"]["avg_us"] * 1e-6) / 1e12
+        out["attention"] = {"bound": "tensor", "achieved": a, "peak": tf_peak, "unit": "TFLOP/s",
+                            "frac": a / tf_peak, "flops_per_launch": fl,
+                            "peak_source": f"{peak_src} bf16_tflops_sustained (timed inside the step)",
+                            "note": "algorithmic QK^T and PV FLOPs; the kernel issues about twice as many "
+                                    "(query and probabilities as bf16 hi + lo terms)"}
+    return out
+
+
 def run_kernel_attention(args):
     """--kernel attention: the block-masked attention launch alone (debug entry: the
     attention kernel and its split-KV merge) on synthetic bf16 data, the canvas's queries
@@ -476,7 +682,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
-    ap.add_argument("--workload", default="layer1_bf16", choices=[n for n in CF.ORDER if n != "chained8_bf16"])
+    ap.add_argument("--workload", default="large4_bf16", choices=CF.ORDER,
+                    help="default: the 4-layer, 262K-vocabulary pass over a 32768-position prefix, the largest "
+                         "single-GPU workload; chained8_bf16 times whole chains (prompt prefill, then canvases of "
+                         "16 passes each appended)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per pass (each its own request and cache) through the batched calls")
@@ -505,6 +714,8 @@ def main():
     cfg = CF.CONFIGS[name]
     if args.impl == "reference":
         return run_reference(args, cfg, name)
+    if name == "chained8_bf16":
+        return run_chained(args, cfg, name)
     if args.canvases < 1:
         ap.error("--canvases must be >= 1")
     if args.fused_update and (args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16"):
@@ -665,34 +876,15 @@ def main():
     # update adds its canvas in / out
     nbytes = RF.pass_bytes(cfg, P, C, unions_h) + 8 * C
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
-    # dominant kernel: the gate/up grouped GEMM, HBM-bound on the union of expert weights
-    gu = kern.get("gemm_gate_up")
+    # every big kernel against its own bound: algorithmic units per launch / average
+    # CUDA-event duration of its launches inside the step (the per-layer expert union
+    # varies, so the expert GEMMs' bytes per launch are the layers' average)
+    kroof = kernel_rooflines(cfg, P, C, unions_h, kern, hbm, tf_sust, peak_src)
+    # the dominant kernel (largest share of the step) is the line's roofline
     roof = None
-    if gu:
-        per_launch = RF.gate_up_bytes(cfg, unions_h[0], C * cfg["top_k"])
-        achieved = per_launch / (gu["avg_us"] * 1e-6) / 1e9
-        roof = {"kernel": "gemm_gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": _ncu_traffic(name), "peak_source": f"{peak_src} hbm_gbs",
-                "bytes_per_launch": per_launch}
-
-    # the other big kernels against their own bounds (algorithmic units per launch / average time)
-    kroof = {}
-    def _hbm(kname, nbytes_launch):
-        if kname in kern:
-            a = nbytes_launch / (kern[kname]["avg_us"] * 1e-6) / 1e9
-            kroof[kname] = {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
-                            "bytes_per_launch": nbytes_launch}
-    if len(set(unions_h)) == 1:
-        _hbm("gemm_down", RF.down_bytes(cfg, unions_h[0], C * cfg["top_k"]))
-    _hbm("gemm_vocab", RF.vocab_bytes(cfg, C))
-    _hbm("update_partial", RF.update_bytes(cfg, C))
-    if "attention" in kern:
-        fl = 4.0 * C * cfg["n_q_heads"] * cfg["head_dim"] * (P + C)
-        a = fl / (kern["attention"]["avg_us"] * 1e-6) / 1e12
-        kroof["attention"] = {"bound": "tensor", "achieved": a, "peak": tf_burst, "unit": "TFLOP/s",
-                              "frac": a / tf_burst, "flops_per_launch": fl,
-                              "note": "algorithmic QK^T and PV FLOPs; the kernel issues about twice as many "
-                                      "(query and probabilities as bf16 hi + lo terms)"}
+    if kroof:
+        dom = max(kroof, key=lambda n: kern[n]["share"])
+        roof = dict(kroof[dom], kernel=dom, traffic=_ncu_traffic(name, dom))
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

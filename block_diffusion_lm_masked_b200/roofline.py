@@ -72,6 +72,31 @@ def pass_flops(cfg: dict, P: int, C: int) -> float:
     return cfg["n_layers"] * per_layer + 2.0 * C * H * V
 
 
+def prefill_flops(cfg: dict, P: int, T: int) -> float:
+    """Causal prefill of T tokens after P cached ones: every layer's projections; below
+    the last layer (which stops after its K/V) causal attention (token i reads P + i + 1
+    keys), the output projection, the router and the k routed experts per token."""
+    H, nq, nkv, d = cfg["hidden"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    E, k, F, L = cfg["n_experts"], cfg["top_k"], cfg["expert_ffn"], cfg["n_layers"]
+    keys = T * P + T * (T + 1) / 2.0
+    return (L * 2.0 * T * H * (nq + 2 * nkv) * d
+            + (L - 1) * (4.0 * nq * d * keys + 2.0 * T * nq * d * H + 2.0 * T * H * E + 6.0 * H * F * T * k))
+
+
+def prefill_bytes(cfg: dict, P: int, T: int, unions) -> float:
+    """Causal prefill's bytes: every layer's QKV weights and the K/V it writes; below the
+    last layer the output projection, the router, the union of experts and the cached K/V."""
+    H, nq, nkv, d, E, L = (cfg["hidden"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"], cfg["n_experts"],
+                           cfg["n_layers"])
+    b = wbytes(cfg)
+    total = 0.0
+    for l in range(L):
+        total += b * H * (nq + 2 * nkv) * d + b * 2 * nkv * d * T
+        if l < L - 1:
+            total += b * nq * d * H + 4 * H * E + expert_bytes(cfg, unions[l]) + b * 2 * nkv * d * (P + T)
+    return total
+
+
 def pass_bytes(cfg: dict, P: int, C: int, unions, ew: float | None = None) -> float:
     """`unions`: the expert union size of each layer (one int per layer)."""
     return pass_bytes_batched(cfg, [P], C, unions, ew)

@@ -9,10 +9,7 @@ import sys
 import pytest
 import torch
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
-                                 reason="the head-pair attention kernel has not yet run on a B200: "
-                                        "DG_RUN_NEW_GPU_TESTS=1 runs it")]
+pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 

@@ -6,7 +6,6 @@ ragged ones.  The batch's taps hold all B C rows; the oracle's per-canvas taps a
 merged the same way (rows stacked, experts grouped over the batch) and compared with
 the single-pass rules of parity_lib.
 """
-import os
 
 import numpy as np
 import pytest
@@ -18,10 +17,7 @@ from oracle import dg_oracle as O
 
 import parity_lib as PL
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
-                                 reason="the batched entry points have not yet run on a B200: "
-                                        "DG_RUN_NEW_GPU_TESTS=1 runs them")]
+pytestmark = pytest.mark.gpu
 
 SMALL_BF16 = dict(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=128, n_experts=8, top_k=2,
                   expert_ffn=192, vocab=2048, rope_theta=10000.0, rms_eps=1e-6, dtype="bf16")

@@ -1,6 +1,5 @@
 """dg_denoise_update (the pass with the update's statistics as the vocabulary
 projection's epilogue, no logits) against the two-call path and against the oracle."""
-import os
 
 import numpy as np
 import pytest
@@ -12,10 +11,7 @@ from oracle import dg_oracle as O
 
 import parity_lib as PL
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
-                                 reason="the fused update has not yet run on a B200: "
-                                        "DG_RUN_NEW_GPU_TESTS=1 runs it")]
+pytestmark = pytest.mark.gpu
 
 SMALL_BF16 = dict(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=128, n_experts=8, top_k=2,
                   expert_ffn=192, vocab=2048, rope_theta=10000.0, rms_eps=1e-6, dtype="bf16")
@@ -98,7 +94,10 @@ def test_fused_update_matches_the_oracle_full_size(dg):
     exempt = PL.compare_pass(cfg, taps, logits.cpu().numpy(), taps_o, logits_o)
     out = torch.from_numpy(canvas0.astype(np.int32)).cuda()
     conf = torch.empty(C, device="cuda")
+    taps_f = st.taps(C)   # the fused call's own layer stack, teacher-forced stage by stage
     dg.denoise_update(st.model, st.cache, out, n, ws, seed=synth.SEED_RENOISE, step=0, conf=conf)
     dg.device_status(ws)
+    stats = PL.forced_pass_check(cfg, st.host, st.prec, st.ocache, canvas0, taps_f, None, label="fused pass")
+    print("forced layers of the fused call:", PL.summary(stats))
     upd_o = O.canvas_update(logits_o, n, synth.SEED_RENOISE, 0)
     PL.compare_update(out.cpu().numpy(), conf.cpu().numpy(), upd_o, exempt, n)

@@ -4,7 +4,6 @@ the oracle's quantisers, the expected products computed in fp64 from the oracle'
 decoding of the same codes.  Exact where the arithmetic allows it (decoding: identity
 activations give the decoded weights themselves), fp32-accumulation close elsewhere;
 and whole passes with 8-bit experts."""
-import os
 
 import numpy as np
 import pytest
@@ -15,10 +14,7 @@ from oracle import dg_oracle as O
 
 import parity_lib as PL
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
-                                 reason="the low-precision-weight GEMMs have not yet run on a B200: "
-                                        "DG_RUN_NEW_GPU_TESTS=1 runs them")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

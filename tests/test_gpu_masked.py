@@ -46,10 +46,11 @@ def test_masked_update_matches_oracle(dg, C, V, frac, n_keep, mask_id):
     for i in masked:
         if i in kept_g or i in kept_o:
             continue
-        if want["top_margin"][i] > PL.TOKEN_MARGIN:
-            assert got[i] == want["canvas"][i], (i, got[i], want["canvas"][i])
+        # both sides take the argmax of the same logits (ties to the lowest id): identical
+        assert got[i] == want["canvas"][i], (i, got[i], want["canvas"][i])
         assert got[i] != mask_id
-    np.testing.assert_allclose(conf.cpu().numpy()[masked], want["conf"][masked], rtol=5e-2, atol=1e-30)
+    # confidences of identical logits: fp32 against fp64 arithmetic
+    np.testing.assert_allclose(conf.cpu().numpy()[masked], want["conf"][masked], rtol=PL.CONF_RTOL, atol=1e-30)
 
 
 def test_generate_masked_matches_oracle_and_step_loop(dg):

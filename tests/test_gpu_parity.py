@@ -44,16 +44,20 @@ def _gpu_pass(dg, st, canvas_np, n, step=0, taps=True):
 
 
 def _check_one_pass(dg, cfg, P, C):
+    """One pass + update: every stage teacher-forced against the oracle, and the whole
+    pass free-running against the oracle's pass from the same canvas."""
     st = PL.Setup(cfg, P)
     canvas0 = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(0), C, cfg["vocab"])
     n = O.renoise_count(C, 1, 0, 0.25, 0.25)
     taps, logits, canvas, conf = _gpu_pass(dg, st, canvas0, n)
+    stats = PL.forced_pass_check(cfg, st.host, st.prec, st.ocache, canvas0, taps, logits, canvas, conf, n,
+                                 synth.SEED_RENOISE, 0)
     logits_o, taps_o = O.denoise_pass(st.host, st.ocache, canvas0, st.prec)
     upd_o = O.canvas_update(logits_o, n, synth.SEED_RENOISE, 0)
     report = []
     exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, report)
     PL.compare_update(canvas, conf, upd_o, exempt, n)
-    print(report, "exempt rows:", sorted(exempt))
+    print("forced:", PL.summary(stats), "| free-running:", report, "exempt rows:", sorted(exempt))
     return st
 
 
@@ -77,6 +81,9 @@ def test_layer1_bf16_full_size(dg):
 
 
 def test_prefill_append_matches_oracle(dg):
+    """Two prefills (77 tokens into an empty cache, then 150 more): every layer's stored
+    K/V and every stage teacher-forced against the oracle; the whole chain free-running
+    up to the causal reach of a near-tie routing difference."""
     cfg = SMALL_BF16
     st = PL.Setup(cfg, 0, capacity=512, with_prefix=False)
     ws = st.workspace(300)
@@ -85,12 +92,15 @@ def test_prefill_append_matches_oracle(dg):
     runs = []
     for toks in (prompt, more):
         P0 = st.ocache.len
-        topk = PL.prefill_topk(st, len(toks))
+        before = PL.oracle_cache_from_gpu(st.cache)
+        tp = st.taps(len(toks))
         dg.prefill_append(st.model, st.cache, torch.from_numpy(toks).cuda(), ws)
+        dg.device_status(ws)
+        stats = PL.forced_prefill_check(cfg, st.host, st.prec, before, toks, tp, st.cache, P0)
+        print(f"prefill at {P0}: forced", PL.summary(stats))
         taps = []
         st.ocache = O.prefill_append(st.host, st.ocache, toks, st.prec, taps)
-        runs.append((P0, [t.cpu().numpy() for t in topk], taps))
-    dg.device_status(ws)
+        runs.append((P0, [t.cpu().numpy() for t in tp["topk_idx"]], taps))
     assert st.cache.len == 227 == st.ocache.len
     seen = PL.kv_close_causal(st.cache, st.ocache, PL.causal_reach(runs, cfg["n_layers"]), "prefill")
     assert seen >= 0.5
@@ -114,41 +124,38 @@ def test_mask_worked_example_on_gpu(dg):
 
 
 def test_chained_canvases_small(dg):
-    """prompt prefill -> (S denoising steps with re-noising -> append) x 2, step by step.
-
-    Every pass starts both sides from the oracle's canvas: one token that legitimately
-    comes out different (a near-tie top-1/top-2 margin) changes every row of the next
-    pass through block attention, so a free-running comparison would compare different
-    problems.  The appended canvas is the oracle's as well."""
+    """prompt prefill -> (S denoising steps with re-noising -> append) x 2, the GPU running
+    its own chain: every pass and every append teacher-forced against the oracle, each
+    stage on the GPU's own input (its canvas, its cache)."""
     cfg = dict(SMALL_BF16, n_layers=2)
     C, S, n_can = 64, 3, 2
     st = PL.Setup(cfg, 0, capacity=512, with_prefix=False)
     ws = st.workspace(96)
     prompt = synth.tokens(synth.SEED_TOKENS, synth.TID_PREFIX_TOKENS, 96, cfg["vocab"])
-    topk = PL.prefill_topk(st, 96)
-    dg.prefill_append(st.model, st.cache, torch.from_numpy(prompt).cuda(), ws)
-    taps = []
-    oc = O.prefill_append(st.host, st.ocache, prompt, st.prec, taps)
-    runs = [(0, [t.cpu().numpy() for t in topk], taps)]
+    _forced_append(dg, st, prompt, ws, "prompt")
     for c in range(n_can):
         cur = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(c), C, cfg["vocab"])
+        oc = PL.oracle_cache_from_gpu(st.cache)
         for s in range(S):
             n = O.renoise_count(C, S, s, 0.5, 0.0)
             taps, logits, nxt_g, conf = _gpu_pass(dg, st, cur, n, step=s)
-            logits_o, taps_o = O.denoise_pass(st.host, oc, cur, st.prec)
-            upd = O.canvas_update(logits_o, n, synth.SEED_RENOISE, s)
-            exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o)
-            PL.compare_update(nxt_g, conf, upd, exempt, n)
-            cur = upd["canvas"]
-        topk = PL.prefill_topk(st, C)
-        dg.prefill_append(st.model, st.cache, torch.from_numpy(cur.astype(np.int32)).cuda(), ws)
-        taps = []
-        runs.append((oc.len, [t.cpu().numpy() for t in topk], taps))
-        oc = O.prefill_append(st.host, oc, cur, st.prec, taps)
+            stats = PL.forced_pass_check(cfg, st.host, st.prec, oc, cur, taps, logits, nxt_g, conf, n,
+                                         synth.SEED_RENOISE, s, label=f"canvas {c} pass {s}")
+            print(f"canvas {c} pass {s}: forced", PL.summary(stats))
+            cur = nxt_g
+        _forced_append(dg, st, cur, ws, f"append {c}")
     dg.device_status(ws)
-    assert st.cache.len == oc.len == 96 + n_can * C
-    seen = PL.kv_close_causal(st.cache, oc, PL.causal_reach(runs, cfg["n_layers"]), "chained")
-    assert seen >= 0.5
+    assert st.cache.len == 96 + n_can * C
+
+
+def _forced_append(dg, st, toks, ws, label):
+    P0 = st.cache.len
+    before = PL.oracle_cache_from_gpu(st.cache)
+    tp = st.taps(len(toks))
+    dg.prefill_append(st.model, st.cache, torch.from_numpy(np.asarray(toks, dtype=np.int32)).cuda(), ws)
+    dg.device_status(ws)
+    stats = PL.forced_prefill_check(st.cfg, st.host, st.prec, before, toks, tp, st.cache, P0, label=label)
+    print(f"{label}: forced", PL.summary(stats))
 
 
 def test_generate_canvas_equals_step_loop(dg):

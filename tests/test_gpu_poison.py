@@ -1,7 +1,6 @@
 """No kernel reads workspace it has not written in the same call: a pass and its update
 with the workspace filled with NaN bytes (the error word cleared) give bit-identical
 logits and canvas to a zero-filled workspace."""
-import os
 
 import numpy as np
 import pytest
@@ -12,10 +11,7 @@ from block_diffusion_lm_masked_b200 import synth
 
 import parity_lib as PL
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DG_RUN_NEW_GPU_TESTS") != "1",
-                                 reason="the poisoned-workspace check has not yet run on a B200: "
-                                        "DG_RUN_NEW_GPU_TESTS=1 runs it")]
+pytestmark = pytest.mark.gpu
 
 SMALL_BF16 = dict(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=128, n_experts=8, top_k=2,
                   expert_ffn=192, vocab=2048, rope_theta=10000.0, rms_eps=1e-6, dtype="bf16")

@@ -1,7 +1,9 @@
 """The comparison rules of the GPU parity tests, checked on planted CPU data (no GPU):
-an allowed routing difference switches the rest of a pass to structure-only checks, a
-routing difference at a clear margin fails, and the causal reach of a prefill starts at
-the first position whose routing actually differs."""
+in the free-running comparison an allowed routing difference switches the rest of a pass
+to structure-only checks, a routing difference at a clear margin fails, and the causal
+reach of a prefill starts at the first position whose routing actually differs; the
+teacher-forced stage checks accept the oracle's own pass dressed as GPU taps and reject
+a wrong layer, a wrong route and a wrong token."""
 import numpy as np
 import pytest
 import torch
@@ -105,3 +107,70 @@ def test_causal_reach_from_actual_flips():
     taps[0]["router_margin"][3] = 1.0
     with pytest.raises(AssertionError, match="prefill layer 0 position 13"):
         PL.causal_reach([(10, g_topk, taps)], 3)
+
+
+# ---------------------------------------------------------------- teacher-forced checks
+
+from oracle import dg_oracle as O  # noqa: E402
+from block_diffusion_lm_masked_b200 import synth  # noqa: E402
+
+SMALL = dict(n_layers=2, hidden=64, n_q_heads=4, n_kv_heads=2, head_dim=16, n_experts=6, top_k=2,
+             expert_ffn=48, vocab=256, rope_theta=10000.0, rms_eps=1e-6, dtype="bf16")
+
+
+def _oracle_as_gpu(cfg, P, C, seed=3):
+    """A pass computed by the oracle and dressed as the GPU's taps (fp32 tensors), so the
+    forced checks see 'GPU' stages that are exact up to fp32 storage."""
+    host = synth.Model(cfg)
+    kv = synth.prefix_cache(cfg, P)
+    oc = O.Cache(kv)
+    canvas = synth.tokens(synth.SEED_TOKENS, synth.tid_canvas_noise(seed), C, cfg["vocab"])
+    prec = O.Precision(cfg["dtype"])
+    logits, taps = O.denoise_pass(host, oc, canvas, prec)
+    t = dict(x_attn=[torch.tensor(x["x_attn"], dtype=torch.float32) for x in taps],
+             x_out=[torch.tensor(x["x_out"], dtype=torch.float32) for x in taps],
+             topk_idx=[torch.tensor(x["topk_idx"], dtype=torch.int32) for x in taps],
+             topk_w=[torch.tensor(x["topk_w"], dtype=torch.float32) for x in taps],
+             counts=[torch.tensor(x["counts"], dtype=torch.int32) for x in taps],
+             perm=[torch.tensor(x["perm"], dtype=torch.int32) for x in taps],
+             unions=torch.tensor([x["union"] for x in taps], dtype=torch.int32))
+    return host, oc, canvas, prec, logits.astype(np.float32), t
+
+
+def test_forced_check_accepts_the_oracle_itself():
+    host, oc, canvas, prec, logits, t = _oracle_as_gpu(SMALL, 40, 24)
+    n = 6
+    upd = O.canvas_update(logits.astype(np.float64), n, 77, 1)
+    stats = PL.forced_pass_check(SMALL, host, prec, oc, canvas, t, logits, upd["canvas"], upd["conf"], n, 77, 1)
+    assert max(stats["attn"]) < 1e-6 and max(stats["moe"]) < 1e-6 and stats["logits"] < 1e-6
+
+
+def test_forced_check_sees_a_wrong_layer_a_wrong_route_and_a_wrong_token():
+    host, oc, canvas, prec, logits, t = _oracle_as_gpu(SMALL, 40, 24)
+    n = 6
+    upd = O.canvas_update(logits.astype(np.float64), n, 77, 1)
+    # a residual off by 5% in the second layer's attention stage
+    bad = dict(t, x_attn=list(t["x_attn"]))
+    bad["x_attn"][1] = bad["x_attn"][1] * 1.05
+    with pytest.raises(AssertionError, match="layer 1"):
+        PL.forced_pass_check(SMALL, host, prec, oc, canvas, bad, logits)
+    # a row routed to another expert at a clear margin (its counts / permutation follow it)
+    bad = dict(t, topk_idx=[x.clone() for x in t["topk_idx"]], counts=list(t["counts"]), perm=list(t["perm"]),
+               unions=t["unions"].clone())
+    m = O.moe_block(host, 0, t["x_attn"][0].double().numpy(), prec)
+    row = int(np.argmax(m["router_margin"]))
+    gi = bad["topk_idx"][0].numpy()
+    gi[row, 0] = [e for e in range(SMALL["n_experts"]) if e not in gi[row]][0]
+    c = np.bincount(gi.reshape(-1), minlength=SMALL["n_experts"])
+    bad["counts"][0] = torch.tensor(c, dtype=torch.int32)
+    flat = gi.reshape(-1)
+    bad["perm"][0] = torch.tensor(sorted(range(flat.size), key=lambda a: (int(flat[a]), a)), dtype=torch.int32)
+    bad["unions"][0] = int((c > 0).sum())
+    with pytest.raises(AssertionError, match="routing"):
+        PL.forced_pass_check(SMALL, host, prec, oc, canvas, bad, logits)
+    # a token that is not the argmax of the same logits, away from the re-noise cut
+    out = upd["canvas"].copy()
+    i = int(np.argmax(np.where(np.isin(np.arange(24), upd["renoised"]), -np.inf, upd["cut_margin"])))
+    out[i] = (out[i] + 1) % SMALL["vocab"]
+    with pytest.raises(AssertionError, match="tokens differ"):
+        PL.forced_pass_check(SMALL, host, prec, oc, canvas, t, logits, out, upd["conf"], n, 77, 1)
