@@ -1772,6 +1772,18 @@ extern "C" dg_status dg_debug_attention_pair_bf16(const void* q, const void* k, 
                          true);
 }
 
+extern "C" dg_status dg_debug_set_wait_limit(uint64_t limit_ns) {
+  DG_CHECK_ARG(limit_ns <= DG_WAIT_NS, "limit_ns must be at most %llu", (unsigned long long)DG_WAIT_NS);
+  cudaError_t (*const setters[])(uint64_t) = {dg::set_wait_limit_attn, dg::set_wait_limit_attn2,
+                                              dg::set_wait_limit_gemm, dg::set_wait_limit_gemm_lowp,
+                                              dg::set_wait_limit_vocab_update};
+  for (auto f : setters) {
+    cudaError_t e = f(limit_ns);
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "setting the wait limit: %s", cudaGetErrorString(e));
+  }
+  return DG_OK;
+}
+
 extern "C" dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream) {
   DG_CHECK_ARG(d_ws, "workspace is NULL");
   DG_CHECK_ARG(timeout_ms >= 1 && timeout_ms <= 10000, "timeout_ms must be in [1, 10000]");

@@ -151,16 +151,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The limit of mbar_wait below.  Each kernel file has its own copy (no relocatable
+// device code): DG_WAIT_NS unless a failure test shortens it through
+// dg_debug_set_wait_limit, which calls every file's set_wait_limit_* (dg_kernels.h).
+static __device__ uint64_t g_dg_wait_limit_ns = DG_WAIT_NS;
+static inline cudaError_t set_wait_limit_this_file(uint64_t ns) {
+  return cudaMemcpyToSymbol(g_dg_wait_limit_ns, &ns, sizeof ns);
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (and sets the
 // abort flag / error word) on timeout or when another thread already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
                                           int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = *(volatile uint64_t*)&g_dg_wait_limit_ns;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > DG_WAIT_NS) {
+    if (globaltimer() - t0 > limit) {
       *abort_flag = 1;
       if (err) atomicCAS(err, 0, code);
       return false;

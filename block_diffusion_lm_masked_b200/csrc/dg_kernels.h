@@ -179,4 +179,11 @@ cudaError_t launch_fill_i32(int32_t* p, int n, int32_t v, cudaStream_t st);
 
 cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 
+// the bounded-wait limit of each kernel file (default DG_WAIT_NS; failure tests shorten it)
+cudaError_t set_wait_limit_attn(uint64_t ns);
+cudaError_t set_wait_limit_attn2(uint64_t ns);
+cudaError_t set_wait_limit_gemm(uint64_t ns);
+cudaError_t set_wait_limit_gemm_lowp(uint64_t ns);
+cudaError_t set_wait_limit_vocab_update(uint64_t ns);
+
 }  // namespace dg

@@ -263,7 +263,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
     __syncwarp();
   } else {
-    // ================= softmax warps: query row `row` (TMEM lane), keys 64 hf .. + 63 of each chunk
+    // ================= softmax warps: query row `row` (TMEM lane), keys 64 hf .. + 63 of each chunk.
+    // Every bounded wait is voted on by the whole warp (__all_sync): the TMEM loads and
+    // stores that follow are warp-collective, so no lane may go on alone after another
+    // lane's wait gave up.
     const int row = (warp & 3) * 32 + lane, hf = warp >> 2;
     const int my_row = q_row0 + row;
     const int my_pos = p.q_pos0 + my_row;
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const int key_lim = p.causal ? min(p.n_keys, my_pos + 1) : p.n_keys;
     bool ok = true;
     for (int j = 0; j < nck && ok; ++j) {
-      ok = mbar_wait(&s_full, (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full, (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
       if (!ok) break;
       tc_fence_after();
       float s[AT_BKEYS / 2];
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       x_max[j & 1][hf][row] = hmax;
       __syncwarp();
       if (lane == 0) mbar_arrive(&x_bar[j & 1]);
-      ok = mbar_wait(&x_bar[j & 1], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, mbar_wait(&x_bar[j & 1], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
       if (!ok) break;
       const float rmax = fmaxf(hmax, x_max[j & 1][hf ^ 1][row]);
       const bool upd = rmax > m_used + 8.0f;
@@ -306,7 +309,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       // tcgen05.ld/st are warp-collective: the whole warp rescales its half of O if any of
       // its rows must, once the previous chunk's PV is complete (O stable)
       if (__any_sync(0xffffffffu, upd && j > 0)) {
-        ok = mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       // P buffer j & 1 was last read by the PV of chunk j - 2
       if (j >= 2) {
-        ok = mbar_wait(&pv_done[j & 1], (uint32_t)((j >> 1) - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], (uint32_t)((j >> 1) - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
         if (!ok) break;
         tc_fence_after();
       }
@@ -354,13 +357,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       if (lane == 0) mbar_arrive(&p_ready[j & 1]);
     }
     if (ok)
-      ok = mbar_wait(&pv_done[(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
     if (ok) {
       // the row sum over both key halves
       x_sum[hf][row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&l_bar);
-      ok = mbar_wait(&l_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, mbar_wait(&l_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
     }
     if (ok) {
       l += x_sum[hf ^ 1][row];
@@ -467,5 +470,7 @@ cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_
   return launch_k(attn_merge_kernel, dim3(n_q, nq), dim3(128), 0, st, part_o, part_lse, n_splits, nq, n_q, d, out,
                   out_lo);
 }
+
+cudaError_t set_wait_limit_attn(uint64_t ns) { return set_wait_limit_this_file(ns); }
 
 }  // namespace dg

@@ -497,4 +497,6 @@ cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, co
   return launch_k(tc_attn2_kernel, grid, dim3(A2_THREADS), A2_SMEM, st, Q, Ql, K, Vt, Kl, Vtl, p, pair_heads);
 }
 
+cudaError_t set_wait_limit_attn2(uint64_t ns) { return set_wait_limit_this_file(ns); }
+
 }  // namespace dg

@@ -227,7 +227,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const TileInfo ti = decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;
       const int buf = j & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM)) break;
+      // the warp votes on the wait's outcome: tcgen05.ld below is warp-collective, so no lane
+      // may go on alone after another gave up
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err,
+                                             DG_DEVERR_TIMEOUT_ACCUM)))
+        break;
       tc_fence_after();
       const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
       const int f = ti.m * TC_BM + row;  // weight row = output feature
@@ -355,5 +359,7 @@ cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2,
   }
   return cudaGetLastError();
 }
+
+cudaError_t set_wait_limit_gemm(uint64_t ns) { return set_wait_limit_this_file(ns); }
 
 }  // namespace dg

@@ -514,4 +514,6 @@ cudaError_t launch_tc_gemm_lowp(int fmt, int epi, const CUtensorMap& A, const CU
                         : launch_fmt<FMT_MX8>(epi, A, A2, S, S2, B, B2, Bb, B2b, p, g_a, g_a2, grid, smem, st);
 }
 
+cudaError_t set_wait_limit_gemm_lowp(uint64_t ns) { return set_wait_limit_this_file(ns); }
+
 }  // namespace dg

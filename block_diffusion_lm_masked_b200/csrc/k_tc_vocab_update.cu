@@ -319,4 +319,6 @@ cudaError_t launch_upd_merge_rows(const UpdPart* part, int C, int tiles, UpdPart
   return launch_k(upd_merge_rows_kernel, dim3((C + 7) / 8), dim3(256), 0, st, part, C, tiles, out);
 }
 
+cudaError_t set_wait_limit_vocab_update(uint64_t ns) { return set_wait_limit_this_file(ns); }
+
 }  // namespace dg

@@ -103,6 +103,7 @@ def _load():
         "dg_launch_count": (ctypes.c_int64, []),
         "dg_renoise_count": (I32, [I32, I32, I32, F32, F32]),
         "dg_debug_bounded_wait": (I32, [P, I32, P]),
+        "dg_debug_set_wait_limit": (I32, [U64]),
         "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_scratch_bytes": (SZ, [I32, I32]),
         "dg_debug_gemm_mx8": (I32, [P, P, P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
@@ -562,3 +563,11 @@ def debug_bounded_wait(ws, timeout_ms, stream=None):
     """Launch the bounded-wait self-test kernel (see include/dg_debug.h)."""
     ptr = ws.ptr if isinstance(ws, Workspace) else ctypes.c_void_p(ws.data_ptr())
     _check(lib.dg_debug_bounded_wait(ptr, timeout_ms, _stream(stream)))
+
+
+WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
+def debug_set_wait_limit(limit_ns: int):
+    """Limit of the tensor-core kernels' bounded waits for later launches (see include/dg_debug.h)."""
+    _check(lib.dg_debug_set_wait_limit(int(limit_ns)))

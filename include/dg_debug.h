@@ -147,6 +147,15 @@ dg_status dg_debug_attention_pair_bf16(const void* q, const void* k, const void*
  * returns DG_ERR_TIMEOUT.  timeout_ms in [1, 10000]. */
 dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream);
 
+/* Failure-detection control: sets the limit of every bounded wait in the tensor-core
+ * kernels (GEMMs, attention, fused vocabulary/update) to limit_ns, for every later
+ * launch on the current device, until set again; the default is 2 s (2000000000).  A
+ * limit of 0 makes a wait that is not already satisfied give up at once, so the next
+ * launch records a timeout code in its error word and winds down (no trap, no hang):
+ * the failure tests use it to show that each kernel's abort path returns.  Not for use
+ * while kernels run.  DG_ERR_INVALID_ARG above 2 s; DG_ERR_CUDA if a copy fails. */
+dg_status dg_debug_set_wait_limit(uint64_t limit_ns);
+
 /* Kernels launched by the library since it was loaded (all kinds, profiling or not). */
 int64_t dg_launch_count(void);
 
