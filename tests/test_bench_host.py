@@ -67,17 +67,27 @@ def test_clock_sampler_reports_why_it_is_unavailable(monkeypatch):
 
 
 def test_ncu_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
-    assert bench._ncu_traffic("layer1_bf16", "gemm_gate_up") == pytest.approx(457.380608e6 + 6.031104e6)
-    assert bench._ncu_traffic("large4_bf16", "attention") is None       # no capture for it
-    src = os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", "k_tc_gemm.cu")
+    """A captured DRAM-traffic figure is reported only while the kernel's source file still
+    hashes to the value recorded with it."""
+    import hashlib
     fake = tmp_path / "block_diffusion_lm_masked_b200" / "csrc"
     fake.mkdir(parents=True)
-    shutil.copy(src, fake / "k_tc_gemm.cu")
+    (fake / "k_x.cu").write_text("// a kernel\n")
+    digest = hashlib.sha256((fake / "k_x.cu").read_bytes()).hexdigest()[:16]
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench._ncu_traffic("layer1_bf16", "gemm_gate_up") is not None   # same bytes, same hash
-    with open(fake / "k_tc_gemm.cu", "a") as f:
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {("w", "kern"): ("k_x.cu", digest, 123.0e6)})
+    assert bench._ncu_traffic("w", "kern") == pytest.approx(123.0e6)
+    assert bench._ncu_traffic("w", "other") is None                    # no capture for it
+    assert bench._ncu_traffic("v", "kern") is None
+    with open(fake / "k_x.cu", "a") as f:
         f.write("\n// changed\n")
-    assert bench._ncu_traffic("layer1_bf16", "gemm_gate_up") is None       # the kernel changed since
+    assert bench._ncu_traffic("w", "kern") is None                     # the kernel changed since
+
+
+def test_recorded_traffic_names_existing_sources():
+    for (workload, kernel), (src, digest, nbytes) in bench.NCU_TRAFFIC.items():
+        assert os.path.exists(os.path.join(ROOT, "block_diffusion_lm_masked_b200", "csrc", src)), src
+        assert len(digest) == 16 and nbytes > 0
 
 
 def test_peaks_fall_back_without_the_measured_file(tmp_path, monkeypatch):
