@@ -652,6 +652,8 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.chunks_per_split = pair_heads ? cps_pair : cps_single;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   p.has_lo = 1;
+  p.q = ws.at<bf16>(ws.L.q);
+  p.q_lo = ws.at<bf16>(ws.L.q_lo);
   p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
@@ -677,17 +679,10 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
                                          n_keys, causal, nq, nkv, d, ws.at<float>(ws.L.o), st));
     return DG_OK;
   }
-  CUtensorMap mq, mql, mk, mv, mkl, mvl;
+  CUtensorMap mk, mv, mkl, mvl;
   dg_status s;
   const int base = (pos0 / 128) * 128;  // the low-term window starts at this chunk
   const int Lc = ws.L.lo_rows;
-  {
-    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
-    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)n_q * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mq, ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
-    if ((s = encode_bf16(&mql, ws.at<void>(ws.L.q_lo), 3, dims, str, box)) != DG_OK) return s;
-  }
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
@@ -722,13 +717,15 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
   p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   p.has_lo = 1;
+  p.q = ws.at<bf16>(ws.L.q);
+  p.q_lo = ws.at<bf16>(ws.L.q_lo);
   p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
   p.part_o = ws.at<float>(ws.L.part_o);
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
-  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mq, mql, mk, mv, mkl, mvl, p, st));
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mk, mv, mkl, mvl, p, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
            dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),

@@ -80,6 +80,8 @@ struct TcAttnParams {
   int n_splits;
   float scale_log2;    // log2(e) / sqrt(d)
   int has_lo;          // query and current K/V carry low terms (bf16 model)
+  const __nv_bfloat16* q;     // query hi [nq][n_q][128] (read directly by tc_attn_kernel)
+  const __nv_bfloat16* q_lo;  // query lo, same layout
   int base;            // 128-aligned start of the low-term window (<= q_pos0)
   __nv_bfloat16* out;     // [n_q][nq * 128] when n_splits == 1 (hi part)
   __nv_bfloat16* out_lo;  // lo part, or null
@@ -87,11 +89,10 @@ struct TcAttnParams {
   float* part_lse;     // [n_splits][nq][n_q], log2 domain
   int* err;
 };
-// Q / Ql: query hi / lo [nq][n_q][128]; K / Vt: the cache; Kl / Vtl: low terms of the
-// current K/V, rows (keys) counted from `base`
-cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
-                                const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
-                                const TcAttnParams& p, cudaStream_t st);
+// K / Vt: the cache; Kl / Vtl: low terms of the current K/V, rows (keys) counted from
+// `base`; the query comes from p.q / p.q_lo
+cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, const CUtensorMap& Kl,
+                                const CUtensorMap& Vtl, const TcAttnParams& p, cudaStream_t st);
 cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 // Head-pair variant (same parameters and outputs; chunks_per_split counts 64-key chunks):

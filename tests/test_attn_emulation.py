@@ -3,8 +3,9 @@ TMA box, shared-memory offset, descriptor start, TMEM column, packed-P layout an
 index as the kernel source computes it, in an order the kernel's barriers allow, against
 the oracle's attention at the GPU test's tolerance.
 
-tc_attn_kernel (validated on a B200) is the control: its transcription passing shows the
-hardware model is right.  The head-pair kernel (tc_attn2_kernel, not yet run) is replayed
+The head-pair kernel (tc_attn2_kernel, validated on a B200) is the control for the
+model; tc_attn_kernel, restructured (query tile in TMEM, three-slot ring, separate load
+and MMA warps), is replayed the same way before its first run.  The head-pair kernel (tc_attn2_kernel, not yet run) is replayed
 with its load warp running as far ahead as its slot plan lets it, so a slot reused too
 early, an S/P buffer overwritten before its PV, or a wrong column or offset changes the
 result.  Planted mistakes in the transcription are caught, which shows the replay is
@@ -176,21 +177,38 @@ def merge2(part_o, part_lse, n_splits):
 
 # ---------------------------------------------------------------- tc_attn_kernel
 def run_single(c, bug=None):
-    """tc_attn_kernel: one head x 128 rows x 128-key chunks, two 64 KB slots (a current
-    chunk takes both), S in TMEM 0..127, P in 128.. / 384.. (hi, lo + 64), O in 256."""
+    """tc_attn_kernel: one head x 128 rows x 128-key chunks; the query tile in TMEM (hi at
+    column 0, lo at 64, packed bf16 pairs along d, stored by the softmax warps), S at 128,
+    O at 256, one P buffer (hi at 384, lo at 448); three 64 KB K/V slots in the slot plan
+    (a current chunk takes two), the load warp running as far ahead as freed slots allow.
+
+    bug: "no_p_wait" -- the softmax writes P(j) without waiting for PV(j - 1);
+    "q_lo_cols" -- the lo query terms stored over the hi ones' columns; "no_pv_first" --
+    the plain issue order where two own-key chunks follow each other."""
     nq, nkv, n_q, pos0, n_keys, causal = (c[k] for k in ("nq", "nkv", "n_q", "pos0", "n_keys", "causal"))
     m = maps(c)
     group = nq // nkv
     n_splits, cps = splits_single(n_q, nq, n_keys)
-    HALF, SLOT = 128 * 128, 4 * 128 * 128
-    sQ, sQl, sSlot = 0, 2 * HALF, 4 * HALF
-    TM_S, TM_O = 0, 256
-    tm_phi = (lambda j: 128) if bug == "one_p_buffer" else (lambda j: 384 if j & 1 else 128)
+    HALF, SLOT, SLOTS = 128 * 128, 4 * 128 * 128, 3
+    sSlot = 0
+    TM_QHI, TM_QLO, TM_S, TM_O, TM_PHI, TM_PLO = 0, 64, 128, 256, 384, 448
+    if bug == "q_lo_cols":
+        TM_QLO = 32
     scale = np.float32(1.4426950408889634 / math.sqrt(D))
     out = np.zeros((n_q, nq * D), np.float32)
     out_lo = np.zeros_like(out)
     part_o = np.zeros((n_splits, nq, n_q, D), np.float32)
     part_lse = np.full((n_splits, nq, n_q), NEG, np.float32)
+
+    def q_words(bits, h, q_row0):
+        """The query rows of one head as the softmax warps store them: word c of a row holds
+        elements 2c (low half) and 2c + 1 (high half); rows past n_q are zero."""
+        rows = np.zeros((128, D), np.uint16)
+        n = min(128, n_q - q_row0)
+        rows[:n] = bits[h, q_row0:q_row0 + n]
+        r32 = rows.astype(np.uint32)
+        return (r32[:, 0::2] | (r32[:, 1::2] << 16)).astype(np.uint32)
+
     for qt in range(-(-n_q // 128)):
         for h in range(nq):
             for sp in range(n_splits):
@@ -204,68 +222,77 @@ def run_single(c, bug=None):
                 rows = q_row0 + np.arange(128)
                 if nck <= 0:
                     continue                                  # empty partial: zeros, lse -inf
-                sm, tm = T.Smem(4 * HALF + 2 * SLOT), T.Tmem()
+                sm, tm = T.Smem(SLOTS * SLOT), T.Tmem()
                 is_cur = lambda j: (c_begin + j) * 128 >= c["base"]
-                for off, mp, x in ((sQ, "Q", 0), (sQ + HALF, "Q", 64), (sQl, "Ql", 0), (sQl + HALF, "Ql", 64)):
-                    sm.tma_load_3d(off, m[mp], x, q_row0, h, 64, 128)
+                tm.t[:, TM_QHI:TM_QHI + 64] = q_words(c["q_hi"], h, q_row0)
+                tm.t[:, TM_QLO:TM_QLO + 64] = q_words(c["q_lo"], h, q_row0)
+                # the slot plan (AtSlotPlan::take), and which chunk's PV frees each slot use
+                plan, nxt, uses = [], 0, [0] * SLOTS
+                for j in range(nck):
+                    parts = []
+                    for _ in range(2 if is_cur(j) else 1):
+                        parts.append((nxt, uses[nxt]))
+                        uses[nxt] += 1
+                        nxt = (nxt + 1) % SLOTS
+                    plan.append(parts)
+                holder = {}
+                loaded = [0]
 
-                def load_slot(slot, mk, mv, krow, vx):
-                    k = sSlot + slot * SLOT
-                    v = k + 2 * HALF
-                    sm.tma_load_3d(k, m[mk], 0, krow, kvh, 64, 128)
-                    sm.tma_load_3d(k + HALF, m[mk], 64, krow, kvh, 64, 128)
-                    sm.tma_load_3d(v, m[mv], vx, 0, kvh, 64, 128)
-                    sm.tma_load_3d(v + HALF, m[mv], vx + 64, 0, kvh, 64, 128)
-
-                issued = [0]
-
-                def issue(j):
-                    key0 = (c_begin + j) * 128
-                    if is_cur(j):
-                        load_slot(0, "K", "Vt", key0, key0)
-                        load_slot(1, "Kl", "Vtl", key0 - c["base"], key0 - c["base"])
-                    else:
-                        load_slot(j & 1, "K", "Vt", key0, key0)
-                    issued[0] = j + 1
+                def pump():
+                    """The load warp: the next chunk's slots, each once its previous use was freed."""
+                    while loaded[0] < nck:
+                        j = loaded[0]
+                        if any(s in holder for s, _ in plan[j]):
+                            return
+                        key0 = (c_begin + j) * 128
+                        for i, (s, _) in enumerate(plan[j]):
+                            k = sSlot + s * SLOT
+                            v = k + 2 * HALF
+                            mk, mv = ("K", "Vt") if i == 0 else ("Kl", "Vtl")
+                            krow = key0 if i == 0 else key0 - c["base"]
+                            sm.tma_load_3d(k, m[mk], 0, krow, kvh, 64, 128)
+                            sm.tma_load_3d(k + HALF, m[mk], 64, krow, kvh, 64, 128)
+                            sm.tma_load_3d(v, m[mv], krow, 0, kvh, 64, 128)
+                            sm.tma_load_3d(v + HALF, m[mv], krow + 64, 0, kvh, 64, 128)
+                            holder[s] = j
+                        loaded[0] += 1
 
                 def issue_s(j):
-                    cur = is_cur(j)
-                    s_hi = 0 if cur else (j & 1)
-                    k, kl = sSlot + s_hi * SLOT, sSlot + SLOT
+                    cur = len(plan[j]) == 2
+                    k = sSlot + plan[j][0][0] * SLOT
+                    kl = sSlot + plan[j][1][0] * SLOT if cur else 0
                     for kb in range(2):
                         for kk in range(4):
-                            off = kb * HALF + kk * 32
-                            T.mma_ss(tm, sm, TM_S, sQ + off, k + off, 128, 128, (kb | kk) != 0)
-                            T.mma_ss(tm, sm, TM_S, sQl + off, k + off, 128, 128, True)
+                            qc, off = kb * 32 + kk * 8, kb * HALF + kk * 32
+                            T.mma_ts(tm, sm, TM_S, TM_QHI + qc, k + off, 128, 128, (kb | kk) != 0)
+                            T.mma_ts(tm, sm, TM_S, TM_QLO + qc, k + off, 128, 128, True)
                             if cur:
-                                T.mma_ss(tm, sm, TM_S, sQ + off, kl + off, 128, 128, True)
+                                T.mma_ts(tm, sm, TM_S, TM_QHI + qc, kl + off, 128, 128, True)
 
-                def issue_pv(j):
-                    cur = is_cur(j)
-                    s_hi = 0 if cur else (j & 1)
-                    v = sSlot + s_hi * SLOT + 2 * HALF
-                    vl = sSlot + SLOT + 2 * HALF
+                def issue_pv(k_):
+                    cur = len(plan[k_]) == 2
+                    v = sSlot + plan[k_][0][0] * SLOT + 2 * HALF
+                    vl = sSlot + plan[k_][1][0] * SLOT + 2 * HALF if cur else 0
                     for kb in range(2):
                         for kk in range(4):
-                            pcol = kb * 32 + kk * 8
-                            vd = v + kb * HALF + kk * 32
-                            T.mma_ts(tm, sm, TM_O, tm_phi(j) + pcol, vd, 128, 128, j > 0 or (kb | kk) != 0)
-                            T.mma_ts(tm, sm, TM_O, tm_phi(j) + 64 + pcol, vd, 128, 128, True)
+                            pcol, vd = kb * 32 + kk * 8, v + kb * HALF + kk * 32
+                            T.mma_ts(tm, sm, TM_O, TM_PHI + pcol, vd, 128, D, k_ > 0 or (kb | kk) != 0)
+                            T.mma_ts(tm, sm, TM_O, TM_PLO + pcol, vd, 128, D, True)
                             if cur:
-                                T.mma_ts(tm, sm, TM_O, tm_phi(j) + pcol, vl + kb * HALF + kk * 32, 128, 128, True)
+                                T.mma_ts(tm, sm, TM_O, TM_PHI + pcol, vl + kb * HALF + kk * 32, 128, D, True)
+                    for s, _ in plan[k_]:                    # the commits free chunk k_'s slots
+                        if holder.get(s) == k_:
+                            del holder[s]
+                    pump()
 
-                # a PV issued by the control warp runs on the tensor pipe later: it is deferred
-                # until the next MMA issue (in-order pipe), an O rescale or the end, so the
-                # softmax of the next chunk writes its P while the PV is still pending
+                # issued PVs run on the tensor pipe later: deferred until the next MMA issue
+                # (in-order pipe), the softmax's wait for the previous PV, a wait for a slot,
+                # or the end
                 pending = []
 
                 def flush():
                     while pending:
                         issue_pv(pending.pop(0))
-
-                def mma_s(j):
-                    flush()
-                    issue_s(j)
 
                 m_used = np.full(128, NEG, np.float32)
                 lsum = [np.zeros(128, np.float32), np.zeros(128, np.float32)]
@@ -281,44 +308,36 @@ def run_single(c, bug=None):
                         s_h.append(s)
                         hmax.append(s.max(axis=1))
                     rmax = np.maximum(hmax[0], hmax[1])
+                    if j > 0 and bug != "no_p_wait":
+                        flush()                               # PV(j - 1) has read P and added into O
                     for hf in range(2):
                         def rescale(any_w, alpha, hf=hf):
                             if j > 0 and any_w.any():
-                                flush()                       # waits for PV(j - 1)
-                                sel = any_w
                                 blk = tm.f32(TM_O + hf * 64, 64)
-                                blk[sel] = (blk[sel] * alpha[sel, None]).astype(np.float32)
+                                blk[any_w] = (blk[any_w] * alpha[any_w, None]).astype(np.float32)
                         mu, lsum[hf] = lazy_update(rmax, m_used, lsum[hf], rescale)
                     m_used = mu
                     for hf in range(2):
                         wh, wl, lsum[hf] = p_words(s_h[hf], m_used, lsum[hf])
-                        tm.t[:, tm_phi(j) + hf * 32:tm_phi(j) + hf * 32 + 32] = wh
-                        tm.t[:, tm_phi(j) + 64 + hf * 32:tm_phi(j) + 64 + hf * 32 + 32] = wl
+                        tm.t[:, TM_PHI + hf * 32:TM_PHI + hf * 32 + 32] = wh
+                        tm.t[:, TM_PLO + hf * 32:TM_PLO + hf * 32 + 32] = wl
 
-                issue(0)
-                if nck > 1 and not is_cur(0) and not is_cur(1):
-                    issue(1)
-                pv_next = 0
+                pump()
                 for j in range(nck):
-                    cur = is_cur(j)
-                    if issued[0] <= j:
-                        if j >= 1 and pv_next == j - 1:
-                            pending.append(j - 1)             # do_pv waits for its completion
-                            flush()
-                            pv_next = j
-                        issue(j)
-                    mma_s(j)
-                    # the softmax warps need only S(j): they may write P(j) before PV(j - 1),
-                    # which the control warp issues after S(j), has run
-                    softmax(j)
-                    if j >= 1 and pv_next == j - 1:
+                    pv_first = j >= 1 and len(plan[j - 1]) + len(plan[j]) > SLOTS
+                    if bug == "no_pv_first":
+                        pv_first = False
+                    if pv_first:
                         pending.append(j - 1)
-                        flush()                               # do_pv waits for it before any load
-                        pv_next = j
-                    if issued[0] == j + 1 and j + 1 < nck and not cur and not is_cur(j + 1):
-                        issue(j + 1)
-                if pv_next == nck - 1:
-                    pending.append(nck - 1)
+                    if loaded[0] <= j:
+                        flush()                               # the slots come free as pending PVs complete
+                    assert loaded[0] > j, "the MMA warp would wait for a chunk the load warp cannot load"
+                    flush()
+                    issue_s(j)
+                    if j >= 1 and not pv_first:
+                        pending.append(j - 1)
+                    softmax(j)
+                pending.append(nck - 1)
                 flush()
                 l = (lsum[0] + lsum[1]).astype(np.float32)
                 for hf in range(2):
@@ -538,14 +557,28 @@ def test_planted_mistakes_in_the_head_pair_replay_are_caught(bug):
     assert not ok
 
 
-@pytest.mark.parametrize("kernel,bug", [("single", "one_p_buffer"), ("pair", "one_sp_buffer")])
-def test_a_single_p_buffer_is_caught(kernel, bug):
-    """One P buffer where the kernels keep two: the next chunk's softmax writes its P while
-    the previous chunk's PV is still to run, which the replay's order allows."""
+def test_a_single_s_p_buffer_in_the_head_pair_kernel_is_caught():
+    """One S/P buffer where the head-pair kernel keeps two: the next chunk's S lands while the
+    previous chunk's PV is still to read its P, which the replay's order allows."""
     c = build(4, 2, 1, 128, 1536, 1664, False)
-    run = run_single if kernel == "single" else run_pair
-    assert within(run(c), oracle(c))
-    assert not within(run(c, bug=bug), oracle(c))
+    assert within(run_pair(c), oracle(c))
+    assert not within(run_pair(c, bug="one_sp_buffer"), oracle(c))
+
+
+@pytest.mark.parametrize("bug,case", [("no_p_wait", (4, 2, 1, 128, 1536, 1664, False)),
+                                      ("q_lo_cols", (5, 2, 1, 300, 0, 300, True)),
+                                      ("no_pv_first", (5, 2, 1, 300, 0, 300, True))])
+def test_planted_mistakes_in_the_attention_replay_are_caught(bug, case):
+    """P written before the previous PV read it (cached chunks, where S(j) runs before
+    PV(j - 1)), the query's lo terms over its hi columns, or the plain issue order for two
+    own-key chunks in a row: a wrong result or no progress."""
+    c = build(*case)
+    assert within(run_single(c), oracle(c))
+    try:
+        ok = within(run_single(c, bug=bug), oracle(c))
+    except AssertionError:
+        ok = False
+    assert not ok
 
 
 def test_a_ring_one_slot_short_is_caught():

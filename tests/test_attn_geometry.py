@@ -72,7 +72,7 @@ def debug_entry_accepts(n_q, pos0, n_keys, causal, cap, nq, nkv):
 
 
 class SlotPlan:
-    """The head-pair kernel's slot plan (SlotPlan::take)."""
+    """The attention kernels' slot plan (SlotPlan::take, AtSlotPlan::take)."""
 
     def __init__(self, slots=3):
         self.nxt, self.uses, self.slots = 0, [0] * slots, slots
@@ -109,6 +109,13 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
     else:
         n_splits, cps = splits_single(n_q, nq, n_keys)
         nh, ys = 1, nq
+        slot_bytes, slots = 65536, 3
+        smem_total = 1024 + slots * slot_bytes                 # the query tile lives in TMEM
+        assert smem_total <= 227 * 1024 - 1024
+        # TMEM columns: Q hi 0..63, lo 64..127, S 128..255, O 256..383, P hi 384..447, lo 448..511
+        cols = [(0, 64), (64, 64), (128, 128), (256, 128), (384, 64), (448, 64)]
+        assert sorted(cols) == cols and all(a + n <= b for (a, n), (b, _) in zip(cols, cols[1:]))
+        assert cols[-1][0] + cols[-1][1] <= 512
     assert 1 <= n_splits <= MAX_SPLITS
     part_o_len = MAX_SPLITS * nq * T * D
     out_len = n_q * nq * D
@@ -123,9 +130,16 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
             kvh = h0 // group
             assert kvh < nkv and h0 + nh <= nq
             assert all((h0 + i) // group == kvh for i in range(nh)), "a CTA's heads span two KV heads"
-            for hl in range(nh):
-                check_tma(0, q_row0, 2, n_q)
-                check_tma(64, q_row0, 2, n_q)
+            if kernel == "pair":
+                for hl in range(nh):
+                    check_tma(0, q_row0, 2, n_q)
+                    check_tma(64, q_row0, 2, n_q)
+            else:
+                # the softmax warps read their query rows (16-byte loads) for rows below n_q
+                for r in (q_row0, q_row0 + rows_here - 1):
+                    for hf in (0, 1):
+                        off = ((h0 * n_q + r) * D + hf * 64) * 2
+                        assert off % 16 == 0 and off + 128 <= nq * n_q * D * 2
             for sp in range(n_splits):
                 c_begin = sp * cps
                 nck = min(nch_total, c_begin + cps) - c_begin
@@ -140,7 +154,7 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                     key0 = (c_begin + j) * W
                     assert key0 < kv_end
                     cur = key0 >= base
-                    parts = plan.take(cur) if kernel == "pair" else [(0, 0)] + ([(1, 0)] if cur else [])
+                    parts = plan.take(cur)
                     for i, (s, _) in enumerate(parts):
                         krow = key0 if i == 0 else key0 - base
                         extent = n_keys if i == 0 else n_keys - base
@@ -151,6 +165,8 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                         assert krow < extent
                         if kernel == "pair":
                             assert s < slots and smem_q + (s + 1) * slot_bytes <= smem_total - 1024
+                        else:
+                            assert s < slots and (s + 1) * slot_bytes <= smem_total - 1024
                     chunks_seen += 1
                 if kernel == "pair":
                     for hl in range(nh):

@@ -305,105 +305,142 @@ def test_the_checker_catches_a_wrong_count():
 
 # ---------------------------------------------------------------- the attention kernel (k_tc_attn.cu)
 
-def attention(nck, cur_from, seed, n_warps=8):
-    """Chunks [cur_from, nck) are the call's own keys ("current": hi and lo parts, both
-    smem slots); earlier chunks are cached keys alternating the two slots."""
+def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, flags=None, give_up_at=None,
+              drain=True, load_drain=True, p_wait=True):
+    """tc_attn_kernel's hand-offs: the softmax warps store the query tile in TMEM and signal
+    (q_ready); a load warp fills `slots` K/V slots in plan order as they are freed; the MMA
+    warp issues S(j) into the one S buffer once the softmax warps have read S(j - 1), then
+    PV(j - 1) from the one P buffer and a commit per slot of chunk j - 1 that frees it
+    (PV(j - 1) first where chunks j - 1 and j need more slots than the ring has); each
+    softmax warp reads its half of S(j), exchanges its half-row max, waits for PV(j - 1)
+    (the last reader of P, and O stable for a rescale), writes its half of P and signals.
+    Chunks [cur_from, nck) are current (two slots each).  flags / give_up_at / load_drain:
+    abort mode as in attention_two_heads below; p_wait=False drops the softmax's wait for
+    PV(j - 1) before overwriting P."""
     rng = random.Random(seed * 7919 + nck)
-    q_bar = Barrier("q_bar", 1)
-    kv = [Barrier(f"kv{s}", 1) for s in range(2)]
+    plan = slot_plan(nck, nck if cur_from is None else cur_from, slots)
+    q_ready = Barrier("q_ready", n_warps)
+    kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
+    kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
     s_full, s_free = Barrier("s_full", 1), Barrier("s_free", n_warps)
-    p_ready = [Barrier(f"p_ready{b}", n_warps) for b in range(2)]
-    pv_done = [Barrier(f"pv_done{b}", 1) for b in range(2)]
+    p_ready, pv_done = Barrier("p_ready", n_warps), Barrier("pv_done", 1)
     x_bar = [Barrier(f"x_bar{b}", n_warps) for b in range(2)]
-    l_bar = Barrier("l_bar", n_warps)
+    l_bar, drain_bar = Barrier("l_bar", n_warps), Barrier("drain", 1)
+    exit_bar = Barrier("exit", n_warps + 2)            # the __syncthreads every role reaches at the end
     bufs, q = Buffers(), Async()
-    st = dict(pv_issued=0, pv_completed=0, s_issued=0, s_completed=0)
+    st = dict(pv_issued=0, pv_done=0, s_done=0)
     p_writes, x_writes = {}, {}
+    steps = [0]
 
-    def is_cur(j):
-        return j >= cur_from
+    def bw(bar, parity, phase):
+        if flags is None:
+            return wait(bar, parity, phase)
+        steps[0] += 1
+        if steps[0] == give_up_at:
+            flags["abort"] = True
+        return ("waitab", bar, parity, phase)
 
-    def control():
-        slot_loads = [0, 0]
-        par = {}
-        issued = 0
-        pv_next = 0
+    def passed(bar, parity):
+        return flags is None or (bar.completed % 2) != parity
 
-        def issue(j):
-            nonlocal issued
-            slots = (0, 1) if is_cur(j) else (j & 1,)
-            for s_ in slots:
-                par[(j & 1, s_)] = slot_loads[s_] & 1
-                slot_loads[s_] += 1
-                bufs.fill(("slot", s_), 2)     # read by the S MMA and the PV MMA of chunk j
-                kv[s_].arrive_expect_tx(32)
-                q.loads.append(lambda s_=s_: kv[s_].complete_tx(32))
-            issued = j + 1
-
-        def issue_pv(k):
-            assert st["pv_issued"] == k and st["s_completed"] >= k + 1
-            st["pv_issued"] += 1
-            assert p_writes.get(k & 1) == (k, n_warps), "PV read a P buffer not fully written"
-            slots = (0, 1) if is_cur(k) else (k & 1,)
-
-            def done(k=k, slots=slots):
-                st["pv_completed"] += 1
-                bufs.release(("p", k & 1))
-                for s_ in slots:
-                    bufs.release(("slot", s_))
-                pv_done[k & 1].arrive()
-            q.mma.append(done)
-
-        def do_pv(k):
-            nonlocal pv_next
-            yield wait(p_ready[k & 1], (k >> 1) & 1, k >> 1)
-            issue_pv(k)
-            pv_next = k + 1
-            yield wait(pv_done[k & 1], (k >> 1) & 1, k >> 1)
-
-        q_bar.arrive_expect_tx(16)
-        q.loads.append(lambda: q_bar.complete_tx(16))
-        issue(0)
-        if nck > 1 and not is_cur(0) and not is_cur(1):
-            issue(1)
+    def load():
+        loaded = [0] * slots
+        ok = True
         for j in range(nck):
-            cur = is_cur(j)
-            s_hi = 0 if cur else (j & 1)
-            if issued <= j:
-                if j >= 1 and pv_next == j - 1:
-                    yield from do_pv(j - 1)
-                issue(j)
-            if j == 0:
-                yield wait(q_bar, 0, 0)
-            yield wait(kv[s_hi], par[(j & 1, s_hi)], None)
-            if cur:
-                yield wait(kv[1], par[(j & 1, 1)], None)
-            if j >= 1:
-                yield wait(s_free, (j - 1) & 1, j - 1)
-            bufs.fill(("S",), n_warps)
-            st["s_issued"] += 1
+            for x, u in plan[j]:
+                if u >= 1:
+                    yield bw(kv_free[x], (u - 1) & 1, u - 1)
+                    if not passed(kv_free[x], (u - 1) & 1):
+                        ok = False
+                        break
+                bufs.fill(("slot", x), 2)              # the S MMA and the PV MMA of chunk j read it
+                kv_full[x].arrive_expect_tx(32)
+                q.loads.append(lambda x=x: kv_full[x].complete_tx(32))
+                loaded[x] += 1
+            if not ok:
+                break
+        # the kernel decides on the wind-down after every role has reached the exit barrier
+        exit_bar.arrive()
+        yield wait(exit_bar, 0, 0)
+        if flags is not None and flags["abort"] and load_drain:
+            for x in range(slots):
+                if loaded[x]:
+                    yield wait(kv_full[x], (loaded[x] - 1) & 1, None)
 
-            def s_done(j=j, cur=cur, s_hi=s_hi):
-                st["s_completed"] += 1
-                for s_ in ((0, 1) if cur else (s_hi,)):
-                    bufs.release(("slot", s_))
+    def leaving(body):
+        """A role that reaches the exit barrier however its body ends."""
+        try:
+            yield from body
+        finally:
+            exit_bar.arrive()
+
+    def mma():
+        def pv_chunk(k):
+            yield bw(p_ready, k & 1, k)
+            if not passed(p_ready, k & 1):
+                return False
+            assert p_writes.get("p") == (k, n_warps), "PV read a P not fully written"
+            st["pv_issued"] += 1
+
+            def done(k=k):
+                st["pv_done"] += 1
+                for w in range(n_warps):
+                    bufs.release(("p", w))
+                for x, _ in plan[k]:
+                    bufs.release(("slot", x))
+                pv_done.arrive()
+            q.mma.append(done)
+            if k + 1 < nck:                            # the last chunk's slots are not reused
+                for x, _ in plan[k]:
+                    q.mma.append(lambda x=x: kv_free[x].arrive())
+            return True
+
+        yield bw(q_ready, 0, 0)
+        ok = passed(q_ready, 0)
+        for j in range(nck if ok else 0):
+            pv_first = pv_first_rule and j >= 1 and len(plan[j - 1]) + len(plan[j]) > slots
+            if pv_first:
+                ok = yield from pv_chunk(j - 1)
+                if not ok:
+                    break
+            for x, u in plan[j]:
+                yield bw(kv_full[x], u & 1, u)
+                if not passed(kv_full[x], u & 1):
+                    ok = False
+                    break
+            if ok and j >= 1:
+                yield bw(s_free, (j - 1) & 1, j - 1)
+                ok = passed(s_free, (j - 1) & 1)
+            if not ok:
+                break
+            for w in range(n_warps):                   # S: each softmax warp reads its half of its lanes
+                bufs.fill(("S", w), 1)
+
+            def s_done(j=j):
+                st["s_done"] += 1
+                for x, _ in plan[j]:
+                    bufs.release(("slot", x))
                 s_full.arrive()
             q.mma.append(s_done)
-            if j >= 1 and pv_next == j - 1:
-                yield from do_pv(j - 1)
-            if issued == j + 1 and j + 1 < nck and not cur and not is_cur(j + 1):
-                issue(j + 1)
-        if pv_next == nck - 1:
-            yield wait(p_ready[(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
-            issue_pv(nck - 1)
+            if j >= 1 and not pv_first:
+                ok = yield from pv_chunk(j - 1)
+                if not ok:
+                    break
+        if ok:
+            yield from pv_chunk(nck - 1)
+        if drain:
+            q.mma.append(lambda: drain_bar.arrive())
+            yield wait(drain_bar, 0, 0)
 
     def softmax(w):
+        q_ready.arrive()                               # this warp's part of the query tile is in TMEM
         for j in range(nck):
-            yield wait(s_full, j & 1, j)
-            assert st["s_completed"] == j + 1
-            bufs.release(("S",))
+            yield bw(s_full, j & 1, j)
+            if not passed(s_full, j & 1):
+                return
+            assert st["s_done"] == j + 1
+            bufs.release(("S", w))
             s_free.arrive()
-            # the row max exchange through x_max[j & 1]
             last, n = x_writes.get(j & 1, (None, 0))
             if last != j:
                 bufs.fill(("x", j & 1), n_warps)
@@ -411,43 +448,68 @@ def attention(nck, cur_from, seed, n_warps=8):
             else:
                 x_writes[j & 1] = (j, n + 1)
             x_bar[j & 1].arrive()
-            yield wait(x_bar[j & 1], (j >> 1) & 1, j >> 1)
+            yield bw(x_bar[j & 1], (j >> 1) & 1, j >> 1)
+            if not passed(x_bar[j & 1], (j >> 1) & 1):
+                return
             assert x_writes[j & 1] == (j, n_warps), "a row max read before both halves posted"
             bufs.release(("x", j & 1))
-            if j > 0 and rng.random() < 0.5:   # some row of this warp needs O rescaled
-                yield wait(pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
-                assert st["pv_completed"] >= j and st["pv_issued"] <= j, "O rescaled while a PV may write it"
-            if j >= 2:
-                yield wait(pv_done[j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
-            last, n = p_writes.get(j & 1, (None, 0))
-            if last != j:
-                bufs.fill(("p", j & 1), 1)     # read by the PV of chunk j
-                p_writes[j & 1] = (j, 1)
-            else:
-                p_writes[j & 1] = (j, n + 1)
-            p_ready[j & 1].arrive()
-        yield wait(pv_done[(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
-        assert st["pv_completed"] == nck
+            if j >= 1 and p_wait:
+                yield bw(pv_done, (j - 1) & 1, j - 1)
+                if not passed(pv_done, (j - 1) & 1):
+                    return
+                if rng.random() < 0.4:                 # some row's max grew: O is rescaled here
+                    assert st["pv_done"] >= j and st["pv_issued"] <= j, "O rescaled while a PV may write it"
+            bufs.fill(("p", w), 1)                     # this warp's half of P, read by PV(j)
+            last, n = p_writes.get("p", (None, 0))
+            p_writes["p"] = (j, 1) if last != j else (j, n + 1)
+            p_ready.arrive()
+        yield bw(pv_done, (nck - 1) & 1, nck - 1)
+        if not passed(pv_done, (nck - 1) & 1):
+            return
+        assert st["pv_done"] == nck
         l_bar.arrive()
-        yield wait(l_bar, 0, 0)
+        yield bw(l_bar, 0, 0)
 
-    roles = {"ctrl": control()}
-    roles.update({f"sm{w}": softmax(w) for w in range(n_warps)})
+    roles = {"load": load(), "mma": leaving(mma())}
+    roles.update({f"sm{w}": leaving(softmax(w)) for w in range(n_warps)})
     return roles, q
 
 
-# What the simulation shows about this protocol: dropping the softmax's wait for the S
-# buffer or for a finished PV before rescaling O is caught; dropping its wait for the PV
-# two chunks back (before reusing that P buffer) is not, because the control warp waits
-# for every PV to complete before issuing the next S, which the softmax waits for first.
-# That wait is therefore redundant, and the control warp's wait is what serialises a PV's
-# completion against the next S on the tensor pipe.
-@pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (2, 1), (2, 0), (3, 3), (5, 3), (6, 0), (7, 5),
-                                          (9, 9), (12, 10)])
+@pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (2, 1), (2, 0), (3, 3), (4, 2), (5, 3), (6, 0),
+                                          (7, 5), (9, 9), (12, 10)])
 def test_attention_protocol(nck, cur_from):
-    for seed in range(25):
-        roles, q = attention(nck, cur_from, seed)
+    """No deadlock, no overrun, no K/V slot, S or P refilled while read, no P read before all
+    its writers, no O rescaled under a PV, nothing in flight when the CTA leaves."""
+    for seed in range(30):
+        roles, q = attention(nck, seed, cur_from=cur_from)
         run(roles, q, seed, end_check=True)
+
+
+def test_attention_protocol_catches_its_planted_mistakes():
+    """Without the PV-first rule two current chunks deadlock the three-slot ring; without the
+    softmax's wait for the previous PV, P is overwritten while that PV reads it."""
+    with pytest.raises(AssertionError, match="deadlock"):
+        roles, q = attention(4, 0, cur_from=2, pv_first_rule=False)
+        run(roles, q, 0)
+    caught = 0
+    for seed in range(30):
+        roles, q = attention(5, seed, p_wait=False)
+        try:
+            run(roles, q, seed)
+        except AssertionError as e:
+            caught += "overwritten" in str(e) or "PV read" in str(e)
+    assert caught > 0
+
+
+@pytest.mark.parametrize("nck,cur_from", [(4, 2), (7, 4), (6, 0), (3, 3)])
+def test_attention_winds_down_after_a_timeout(nck, cur_from):
+    """A bounded wait gives up at a random point: every role leaves and, with the load and
+    MMA drains, nothing is in flight when they have."""
+    for seed in range(150):
+        rng = random.Random(seed)
+        flags = {"abort": False}
+        roles, q = attention(nck, seed, cur_from=cur_from, flags=flags, give_up_at=rng.randrange(1, 14 * nck))
+        run_ab(roles, q, flags, seed, end_check=True)
 
 
 # ---------------------------------------------------------------- the fused vocabulary/update GEMM (k_tc_vocab_update.cu)
