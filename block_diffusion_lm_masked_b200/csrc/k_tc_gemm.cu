@@ -4,7 +4,7 @@
 // small, so weights sit on the 128-row M side of the MMA and tokens on N: a tile is
 // 128 weight rows x (up to n_max) token rows.
 //
-// One CTA per SM walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Roles
+// One CTA per SM walks its share of the tiles (TileWalk: rounds of gridDim.x).  Roles
 // (192 threads): warp 0 issues TMA loads into a ring of smem stages; warp 1 owns
 // the TMEM allocation and issues tcgen05.mma into one of two accumulator buffers;
 // warps 2-5 drain the other buffer through the epilogue, so the loads and MMAs of
@@ -61,15 +61,36 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmParams& p, int t) {
   return ti;
 }
 
-// This CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+// This CTA's tiles.  The tiles are dealt to the CTAs in rounds of gridDim.x, every other
+// round in reverse CTA order (a serpentine), from a list with the whole weight tiles
+// first and, when the weight rows are not a multiple of 128 (the expert FFN of 704
+// rows), each work item's partial last weight tile at the end: the partial tiles, which
+// stream fewer weight bytes, then even out the last rounds.  At the large model's
+// gate/up GEMM (128 items x 5.5 weight tiles) the busiest CTA streams 5 tiles' weights
+// instead of 6.
 struct TileWalk {
-  int t, n_tiles;
-  __device__ TileWalk(int n_tiles_) : t(blockIdx.x), n_tiles(n_tiles_) {}
+  int r, n_tiles, m_tiles, full;
+  __device__ TileWalk(const TcGemmParams& p, int n_tiles_) : r(0), n_tiles(n_tiles_), m_tiles(p.m_tiles) {
+    const bool partial = p.m_tiles > 1 && p.a_rows_per_group % TC_BM != 0;
+    full = partial ? n_tiles - n_tiles / p.m_tiles : n_tiles;
+  }
+  // the k-th tile of the list -> tile index (work item * m_tiles + weight tile)
+  __device__ int order(int k) const {
+    if (full == n_tiles) return k;
+    if (k < full) return (k / (m_tiles - 1)) * m_tiles + k % (m_tiles - 1);
+    return (k - full) * m_tiles + (m_tiles - 1);
+  }
   __device__ bool next(int& tile) {
-    if (t >= n_tiles) return false;
-    tile = t;
-    t += gridDim.x;
-    return true;
+    while ((long long)r * gridDim.x < n_tiles) {
+      const int c = (r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+      const long long k = (long long)r * gridDim.x + c;
+      ++r;
+      if (k < n_tiles) {
+        tile = order((int)k);
+        return true;
+      }
+    }
+    return false;
   }
 };
 
@@ -139,7 +160,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       int it = 0, t;
       bool ok = true;
-      TileWalk walk(n_tiles);
+      TileWalk walk(p, n_tiles);
       while (ok && walk.next(t)) {
         const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
@@ -175,7 +196,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // ---------------- MMA issuer
       int it = 0, j = 0, t;
       bool ok = true;
-      TileWalk walk(n_tiles);
+      TileWalk walk(p, n_tiles);
       for (; ok && walk.next(t); ++j) {
         const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
@@ -222,7 +243,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int row = lg * 32 + lane;  // row of the 128-row tile this thread drains
     const uint32_t lane_off = (uint32_t)(lg * 32) << 16;
     int j = 0, t;
-    TileWalk walk(n_tiles);
+    TileWalk walk(p, n_tiles);
     for (; walk.next(t); ++j) {
       const TileInfo ti = decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;

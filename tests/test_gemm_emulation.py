@@ -3,7 +3,8 @@ CPU (tests/tc_emu.py): the control for the GEMM half of the hardware model, and 
 check for later changes to the kernel.
 
 Transcribed from the kernel source: the persistent tile walk (grouped: item-major;
-dense: token chunk, then split, then weight tile), the k-block rotation within a split,
+dense: token chunk, then split, then weight tile; dealt in serpentine rounds with the
+partial weight tiles last), the k-block rotation within a split,
 the stage layout (one or two weight tiles, then one or two token terms of n_max rows),
 the MMAs into one of two accumulator buffers (a second weight matrix n_max columns on),
 and the epilogue's indices: fp32 stores into the split's slab, or SwiGLU with bf16 hi /
@@ -20,6 +21,29 @@ import tc_emu as T
 from oracle import dg_oracle as O
 
 BM, BK = 128, 64
+
+
+def tile_walk(cta, grid, n_tiles, m_tiles, rows_a):
+    """TileWalk: rounds of `grid` tiles, every other round in reverse CTA order, over a list
+    with the whole weight tiles first and each work item's partial last weight tile (when
+    rows_a is not a multiple of 128) at the end."""
+    partial = m_tiles > 1 and rows_a % BM != 0
+    full = n_tiles - n_tiles // m_tiles if partial else n_tiles
+
+    def order(k):
+        if full == n_tiles:
+            return k
+        if k < full:
+            return (k // (m_tiles - 1)) * m_tiles + k % (m_tiles - 1)
+        return (k - full) * m_tiles + (m_tiles - 1)
+    out, r = [], 0
+    while r * grid < n_tiles:
+        c = grid - 1 - cta if r & 1 else cta
+        k = r * grid + c
+        r += 1
+        if k < n_tiles:
+            out.append(order(k))
+    return out
 
 
 def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1, W2=None, split_stride=0,
@@ -63,7 +87,7 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
 
     for cta in range(min(grid, n_tiles)):
         sm, tm = T.Smem(stages * stage_bytes), T.Tmem(tmem_cols)
-        tiles = list(range(cta, n_tiles, grid))
+        tiles = tile_walk(cta, grid, n_tiles, m_tiles, rows_a)
         its = [(t, kb) for t in tiles for kb in range(nkb)]
         loaded = mma_done = 0
         pending = []
@@ -215,3 +239,23 @@ def test_planted_mistakes_in_the_gemm_replay_are_caught(bug):
         got = np.nan_to_num(out.reshape(ks, n, rows)).sum(axis=0)
         ref = x @ w[0].T
     assert np.abs(got - ref).max() / np.abs(ref).max() > 1e-3
+
+
+@pytest.mark.parametrize("n_items,m_tiles,rows_a,grid", [(128, 6, 704, 148), (54, 8, 1024, 148), (7, 6, 704, 5),
+                                                        (1, 22, 2816, 148), (3, 1, 100, 148)])
+def test_tile_walk_covers_every_tile_once_and_balances_the_weight_bytes(n_items, m_tiles, rows_a, grid):
+    """Every tile is walked by exactly one CTA, and no CTA streams more weight rows than the
+    ceiling of the average plus one partial tile (the large model's gate/up GEMM: 5 whole
+    tiles' worth at most, where the plain strided walk gives some CTA 6)."""
+    n_tiles = n_items * m_tiles
+    walks = [tile_walk(c, grid, n_tiles, m_tiles, rows_a) for c in range(grid)]
+    seen = sorted(t for w in walks for t in w)
+    assert seen == list(range(n_tiles))
+    rows = lambda t: min(BM, rows_a - (t % m_tiles) * BM)
+    load = [sum(rows(t) for t in w) for w in walks]
+    avg = sum(load) / grid
+    assert max(load) <= -(-avg // BM) * BM + BM // 2
+    if (n_items, m_tiles, grid) == (128, 6, 148):
+        assert max(load) == 5 * BM
+        strided = [sum(rows(t) for t in range(c, n_tiles, grid)) for c in range(grid)]
+        assert max(strided) == 6 * BM
