@@ -375,7 +375,7 @@ constexpr int kItemRowsMx8 = 64;         // the same for the 8-bit-weight expert
 
 
 struct WsLayout {
-  size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
+  size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, attn_cnt, opart, topk_idx,
       topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, vtiles, total;
   int lo_rows;  // rows of the current-token K/V low-term window
 };
@@ -410,6 +410,7 @@ WsLayout layout(const dg_config& c, int T) {
   L.o_lo = take(bf ? (size_t)T * c.n_q_heads * d * 2 : 0);
   L.part_o = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
   L.part_lse = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * 4 : 0);
+  L.attn_cnt = take((size_t)((T + 127) / 128) * c.n_q_heads * 4);  // attention's split tickets
   L.opart = take((size_t)(bf ? kMaxKsO : 1) * T * H * 4);
   L.topk_idx = take((size_t)T * k * 4);
   L.topk_w = take((size_t)T * k * 4);
@@ -654,6 +655,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.has_lo = 1;
   p.q = ws.at<bf16>(ws.L.q);
   p.q_lo = ws.at<bf16>(ws.L.q_lo);
+  p.merge_cnt = nullptr;  // merged by attn_merge2_kernel
   p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
@@ -719,17 +721,15 @@ dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int c
   p.has_lo = 1;
   p.q = ws.at<bf16>(ws.L.q);
   p.q_lo = ws.at<bf16>(ws.L.q_lo);
+  p.merge_cnt = ws.at<int>(ws.L.attn_cnt);  // zeroed by the RoPE kernel before every attention
   p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
   p.part_o = ws.at<float>(ws.L.part_o);
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
+  // the kernel merges its split-KV partials itself (the last split of each tile and head)
   LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mk, mv, mkl, mvl, p, st));
-  if (p.n_splits > 1)
-    LAUNCH(DG_K_ATTN_MERGE, st,
-           dg::launch_attn_merge(p.part_o, p.part_lse, p.n_splits, nq, n_q, d, ws.at<bf16>(ws.L.o),
-                                 ws.at<bf16>(ws.L.o_lo), st));
   return DG_OK;
 }
 
@@ -764,7 +764,8 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
          dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), ks_qkv, (size_t)n * QR, n, nq, nkv, d, pos0, c.rope_theta,
                                     ws.at<T>(ws.L.q), (T*)kc, (T*)vtc, cap, bf ? ws.at<T>(ws.L.q_lo) : nullptr,
                                     bf ? ws.at<T>(ws.L.k_lo) : nullptr, bf ? ws.at<T>(ws.L.vt_lo) : nullptr,
-                                    (pos0 / 128) * 128, ws.L.lo_rows, st));
+                                    (pos0 / 128) * 128, ws.L.lo_rows, ws.at<int>(ws.L.attn_cnt),
+                                    ((n + 127) / 128) * nq, st));
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
@@ -952,7 +953,8 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
            dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv) + (size_t)b * C * QR, ks_qkv, (size_t)n * QR, C, nq, nkv,
                                       d, g.pos0, c.rope_theta, wb.at<T>(wb.L.q), (T*)g.kc, (T*)g.vtc, g.cap,
                                       bf ? wb.at<T>(wb.L.q_lo) : nullptr, bf ? ws.at<T>(ws.L.k_lo) : nullptr,
-                                      bf ? ws.at<T>(ws.L.vt_lo) : nullptr, (g.pos0 / 128) * 128, ws.L.lo_rows, st));
+                                      bf ? ws.at<T>(ws.L.vt_lo) : nullptr, (g.pos0 / 128) * 128, ws.L.lo_rows,
+                                      ws.at<int>(ws.L.attn_cnt), ((C + 127) / 128) * nq, st));
     if (stop_after_kv) continue;
     if ((s = attention(c, wb, g.kc, g.vtc, g.cap, C, g.pos0, g.pos0 + C, causal, st)) != DG_OK) return s;
   }
@@ -1741,6 +1743,8 @@ static dg_status debug_attention(const void* q, const void* k, const void* vt, i
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.q_lo), 0, (size_t)nq * n_q * 128 * 2, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.k_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.vt_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
+  // the split tickets the pass's RoPE kernel would zero
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.attn_cnt), 0, (size_t)((n_q + 127) / 128) * nq * 4, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy q: %s", cudaGetErrorString(e));
   void* kc = const_cast<void*>(k);
   void* vtc = const_cast<void*>(vt);

@@ -82,6 +82,9 @@ struct TcAttnParams {
   int has_lo;          // query and current K/V carry low terms (bf16 model)
   const __nv_bfloat16* q;     // query hi [nq][n_q][128] (read directly by tc_attn_kernel)
   const __nv_bfloat16* q_lo;  // query lo, same layout
+  int* merge_cnt;             // [q tiles][nq] split tickets, zero on entry (tc_attn_kernel merges its
+                              // splits itself when n_splits > 1; the last split of a tile and head
+                              // to finish does it and leaves the ticket at zero)
   int base;            // 128-aligned start of the low-term window (<= q_pos0)
   __nv_bfloat16* out;     // [n_q][nq * 128] when n_splits == 1 (hi part)
   __nv_bfloat16* out_lo;  // lo part, or null
@@ -120,7 +123,7 @@ cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int 
 template <typename T>
 cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
                                 int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
-                                T* vt_lo, int lo_base, int lo_rows, cudaStream_t st);
+                                T* vt_lo, int lo_base, int lo_rows, int* zero_p, int zero_n, cudaStream_t st);
 cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, const int* group_off, int n_groups,
                                  int max_rows_per_group, int n_tokens, int M, int K, float* out, int ld_out,
                                  cudaStream_t st);

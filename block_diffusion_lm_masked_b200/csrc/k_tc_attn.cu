@@ -3,8 +3,9 @@
 //                   keys (bidirectional block rows of the prefix/block mask);
 //   prefill mode:   new tokens see keys up to their own position (causal rows).
 // One CTA = one query head x 128 query rows x a contiguous range of 128-key chunks
-// (split-KV; partial results merged by attn_merge_kernel).  V is kept transposed in the
-// cache ([d][position]) so the B operands of both MMAs are K-major in shared memory.
+// (split-KV; the last split of a tile and head to finish merges the partial results).
+// V is kept transposed in the cache ([d][position]) so the B operands of both MMAs are
+// K-major in shared memory.
 //
 // Precision.  Cached keys/values are bf16 (the cache's storage format).  The query and
 // the keys/values of the tokens the call itself processes are in flight at fp32
@@ -87,6 +88,57 @@ struct AtSlotPlan {
   }
 };
 
+// Split-KV merge by the last split of a (query tile, head) to finish: every split has
+// written its partial output and log2-sum-exp; the split whose ticket comes last combines
+// them (weights 2^(lse_s - max)) into the bf16 hi + lo output and resets the ticket for
+// the next launch.  Block-wide; called by every CTA of the grid as it leaves.
+__device__ __forceinline__ void merge_splits_if_last(const TcAttnParams& p, int qt, int h) {
+  __shared__ int last_s;
+  __threadfence();  // this CTA's partials are visible device-wide before its ticket
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(&p.merge_cnt[qt * p.nq + h], 1) == p.n_splits - 1;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  const int q_row0 = qt * AT_BQ;
+  const int rows = min(AT_BQ, p.n_q - q_row0);
+  for (int idx = threadIdx.x; idx < rows * (AT_D / 4); idx += blockDim.x) {
+    const int row = q_row0 + idx / (AT_D / 4), c4 = idx % (AT_D / 4);
+    float mx = -INFINITY;
+    for (int sp = 0; sp < p.n_splits; ++sp) mx = fmaxf(mx, __ldcg(&p.part_lse[((size_t)sp * p.nq + h) * p.n_q + row]));
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.0f;
+    if (mx != -INFINITY) {
+      for (int sp = 0; sp < p.n_splits; ++sp) {
+        const float lse = __ldcg(&p.part_lse[((size_t)sp * p.nq + h) * p.n_q + row]);
+        if (lse == -INFINITY) continue;
+        const float w = exp2f(lse - mx);
+        const float4 o =
+            __ldcg(reinterpret_cast<const float4*>(p.part_o + (((size_t)sp * p.nq + h) * p.n_q + row) * AT_D) + c4);
+        num.x += w * o.x;
+        num.y += w * o.y;
+        num.z += w * o.z;
+        num.w += w * o.w;
+        den += w;
+      }
+    }
+    const float v[4] = {den > 0.f ? num.x / den : 0.f, den > 0.f ? num.y / den : 0.f, den > 0.f ? num.z / den : 0.f,
+                        den > 0.f ? num.w / den : 0.f};
+    uint32_t w[2], wl[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v[2 * e] - __low2float(hi), v[2 * e + 1] - __high2float(hi));
+      w[e] = *reinterpret_cast<const uint32_t*>(&hi);
+      wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+    }
+    const size_t o = (size_t)row * p.nq * AT_D + (size_t)h * AT_D + 4 * c4;
+    *reinterpret_cast<uint2*>(p.out + o) = make_uint2(w[0], w[1]);
+    if (p.out_lo) *reinterpret_cast<uint2*>(p.out_lo + o) = make_uint2(wl[0], wl[1]);
+  }
+  if (threadIdx.x == 0) p.merge_cnt[qt * p.nq + h] = 0;  // ready for the next launch
+}
+
 __global__ void __launch_bounds__(AT_THREADS, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
                    const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
@@ -127,6 +179,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (int i = 0; i < AT_D; ++i) po[i] = 0.0f;
       p.part_lse[((size_t)sp * p.nq + h) * p.n_q + qrow] = -INFINITY;
     }
+    if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h);
     return;
   }
 
@@ -471,6 +524,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
+  if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h);
 }
 
 __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_splits,

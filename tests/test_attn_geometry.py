@@ -135,6 +135,8 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                     check_tma(0, q_row0, 2, n_q)
                     check_tma(64, q_row0, 2, n_q)
             else:
+                # the split ticket of this tile and head lies in the workspace's ticket array
+                assert qt * nq + h0 < cdiv(T, 128) * nq
                 # the softmax warps read their query rows (16-byte loads) for rows below n_q
                 for r in (q_row0, q_row0 + rows_here - 1):
                     for hf in (0, 1):
