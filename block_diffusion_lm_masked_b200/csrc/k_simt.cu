@@ -82,6 +82,10 @@ cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int 
 // qkv[t] = [q heads | k heads | v heads] (fp32).  Rotate-half RoPE at position pos0 + t
 // (angles in double precision), then q -> q[h][t][:], k -> K[kvh][pos][:],
 // v -> V^T[kvh][:][pos], all in the activation dtype.
+// most split-K partial slabs a consumer sums (the projections' split-K factors are at
+// most 4 and 8; launches with more are refused)
+constexpr int kMaxSumParts = 8;
+
 template <typename T>
 __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, size_t part_stride, int nq, int nkv,
                                     int d, int pos0, float theta, int n, T* __restrict__ q, T* __restrict__ kc,
@@ -106,14 +110,20 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, 
   const int W = (nq + 2 * nkv) * d;
   float* row = cs + d;  // qkv row = sum of the split-K partials, in a fixed order
   for (int i = threadIdx.x; i < W / 4; i += blockDim.x) {
+    // every partial's load issued before the first add (the sum keeps its fixed order)
+    float4 a[kMaxSumParts];
+#pragma unroll
+    for (int s = 0; s < kMaxSumParts; ++s)
+      if (s < n_parts) a[s] = reinterpret_cast<const float4*>(qkv + s * part_stride + (size_t)t * W)[i];
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_parts; ++s) {
-      const float4 a = reinterpret_cast<const float4*>(qkv + s * part_stride + (size_t)t * W)[i];
-      v.x += a.x;
-      v.y += a.y;
-      v.z += a.z;
-      v.w += a.w;
-    }
+#pragma unroll
+    for (int s = 0; s < kMaxSumParts; ++s)
+      if (s < n_parts) {
+        v.x += a[s].x;
+        v.y += a[s].y;
+        v.z += a[s].z;
+        v.w += a[s].w;
+      }
     reinterpret_cast<float4*>(row)[i] = v;
   }
   __syncthreads();
@@ -163,6 +173,7 @@ cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_strid
                                 int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
                                 T* vt_lo, int lo_base, int lo_rows, int* zero_p, int zero_n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
+  if (n_parts < 1 || n_parts > kMaxSumParts) return cudaErrorInvalidValue;
   const size_t smem = (size_t)(d + (nq + 2 * nkv) * d) * sizeof(float);
   return launch_k(rope_scatter_kernel<T>, dim3(n), dim3(256), smem, st, qkv, n_parts, part_stride, nq, nkv, d, pos0,
                   theta, n, q, kcache, vtcache, cap, q_lo, k_lo, vt_lo, lo_base, lo_rows, zero_p, zero_n);
@@ -341,14 +352,20 @@ __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     const size_t ps4 = part_stride / 4;
     float4* own4 = reinterpret_cast<float4*>(own);
     for (int i = threadIdx.x; i < no * H4; i += RT_THREADS) {
+      // every partial's load issued before the first add (the sum keeps its fixed order)
+      float4 a[kMaxSumParts];
+#pragma unroll
+      for (int s = 0; s < kMaxSumParts; ++s)
+        if (s < n_parts) a[s] = p4[s * ps4 + i];
       float4 v = x4[i];
-      for (int s = 0; s < n_parts; ++s) {
-        const float4 a = p4[s * ps4 + i];
-        v.x += a.x;
-        v.y += a.y;
-        v.z += a.z;
-        v.w += a.w;
-      }
+#pragma unroll
+      for (int s = 0; s < kMaxSumParts; ++s)
+        if (s < n_parts) {
+          v.x += a[s].x;
+          v.y += a[s].y;
+          v.z += a[s].z;
+          v.w += a[s].w;
+        }
       x4[i] = v;
       own4[i] = v;
     }
@@ -464,6 +481,7 @@ cudaError_t launch_router_fused(float* x, const float* parts, int n_parts, size_
                                 T* xn, T* xn_lo, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   if (E > 256 || E % RT_G != 0 || k > 16 || k > E || (H % 4) != 0) return cudaErrorInvalidValue;
+  if (n_parts < 0 || n_parts > kMaxSumParts) return cudaErrorInvalidValue;
   const size_t smem = ((size_t)(RT_OWN + RT_TOK) * H + (size_t)RT_TOK * (E / RT_G)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(router_fused_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
