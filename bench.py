@@ -670,6 +670,83 @@ def run_kernel_attention(args):
     return 0
 
 
+def run_kernel_gemm(args):
+    """--kernel gemm --gemm vocab|gate_up|down: one GEMM launch of the large model's shapes
+    through the debug entry (the pass's persistent tcgen05 kernel) on synthetic bf16 data:
+    the vocabulary projection (262144 x 2816 weights, 256 tokens, fp32 out), or the grouped
+    expert GEMMs over 128 experts with 16 rows each (gate/up with the SwiGLU epilogue, two-term
+    tokens; down, fp32 out).  One JSON line: median CUDA-event time per launch and the
+    algorithmic bytes per launch against the HBM bandwidth.  Used for ncu captures of the
+    GEMMs at the large model's sizes without the rest of the model on the device."""
+    import torch
+
+    from block_diffusion_lm_masked_b200 import dg
+
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(11)
+    cfg = CF.CONFIGS["large4_bf16"]
+    H, F, V, E, k, C = cfg["hidden"], cfg["expert_ffn"], cfg["vocab"], cfg["n_experts"], cfg["top_k"], cfg["canvas"]
+    rows = C * k
+
+    def bf(*shape, scale=0.02):
+        return (torch.randn(*shape, generator=g, device=dev) * scale).to(torch.bfloat16)
+
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    if args.gemm == "vocab":
+        W, X = bf(1, V, H), bf(C, H, scale=1.0)
+        out = torch.empty(C, V, device=dev)
+        scratch = dg.debug_gemm_scratch(C, 1)
+        call = lambda: dg.debug_gemm_bf16(W, X, out, V, err, scratch)
+        nbytes = RF.vocab_bytes(cfg, C)
+    else:
+        off = torch.arange(0, rows + 1, rows // E, dtype=torch.int32, device=dev)
+        if args.gemm == "gate_up":
+            W, W2 = bf(E, F, H), bf(E, F, H)
+            Xf = torch.randn(rows, H, generator=g, device=dev)
+            X = Xf.to(torch.bfloat16)
+            X_lo = (Xf - X.float()).to(torch.bfloat16)
+            out = torch.empty(rows, F, dtype=torch.bfloat16, device=dev)
+            out_lo = torch.empty_like(out)
+            scratch = dg.debug_gemm_scratch(rows, E)
+            call = lambda: dg.debug_gemm_bf16(W, X, out, F, err, scratch, W2=W2, X_lo=X_lo, group_off=off,
+                                              out_lo=out_lo)
+            nbytes = RF.gate_up_bytes(cfg, E, rows)
+        else:
+            W = bf(E, H, F)
+            Xf = torch.randn(rows, F, generator=g, device=dev)
+            X = Xf.to(torch.bfloat16)
+            X_lo = (Xf - X.float()).to(torch.bfloat16)
+            out = torch.empty(rows, H, device=dev)
+            scratch = dg.debug_gemm_scratch(rows, E)
+            call = lambda: dg.debug_gemm_bf16(W, X, out, H, err, scratch, X_lo=X_lo, group_off=off)
+            nbytes = RF.down_bytes(cfg, E, rows)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    if err.item() != 0:
+        raise RuntimeError(f"GEMM error word {err.item()}")
+    us = statistics.median(ts)
+    hbm, _, _, peak_src = _peaks()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    line = {"metric": f"GEMM launch latency ({args.gemm}, large model's shape)", "value": us, "unit": "us",
+            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+            "data": "synthetic: weights N(0, 0.02), tokens N(0, 1), bf16",
+            "config": {"workload": f"gemm {args.gemm}: H{H}, F{F}, V{V}, {E} experts x {rows // E} rows, C{C}",
+                       "l2": "weights larger than L2 except the debug entry's token operand"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "bytes_per_launch": nbytes, "peak_source": f"{peak_src} hbm_gbs"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def _attention_kind():
     """Which attention kernel the library runs (DG_ATTN_PAIR=1: the head-pair kernel)."""
     return ("head pairs, 64-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
@@ -698,9 +775,12 @@ def main():
                     help="output-matrix storage; mx8 and nv4 run through the batched calls")
     ap.add_argument("--attn-pair", action="store_true",
                     help="run the pass's attention through the head-pair kernel (sets DG_ATTN_PAIR=1)")
-    ap.add_argument("--kernel", choices=["attention"], default=None,
+    ap.add_argument("--kernel", choices=["attention", "gemm"], default=None,
                     help="time one kernel alone on synthetic data instead of the step (attention: the "
-                         "block-masked attention call over --keys keys)")
+                         "block-masked attention call over --keys keys; gemm: one GEMM of the large model's "
+                         "shapes, --gemm)")
+    ap.add_argument("--gemm", choices=["vocab", "gate_up", "down"], default="vocab",
+                    help="--kernel gemm: which GEMM")
     ap.add_argument("--keys", type=int, default=8192, help="--kernel attention: key count")
     ap.add_argument("--queries", type=int, default=256, help="--kernel attention: canvas queries")
     ap.add_argument("--heads", type=int, default=16, help="--kernel attention: query heads")
@@ -708,6 +788,8 @@ def main():
     args = ap.parse_args()
     if args.kernel == "attention":
         return run_kernel_attention(args)
+    if args.kernel == "gemm":
+        return run_kernel_gemm(args)
     if args.attn_pair:  # read by the library at its first attention call
         os.environ["DG_ATTN_PAIR"] = "1"
     name = args.workload
