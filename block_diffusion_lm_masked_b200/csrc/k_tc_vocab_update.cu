@@ -11,8 +11,9 @@
 // Roles (192 threads, one CTA per SM, tiles blockIdx.x, blockIdx.x + gridDim.x, ...):
 // warp 0 TMA (weights 128 rows x 64, tokens in boxes of 64 then 16 rows, single term),
 // warp 1 MMA into one of two TMEM accumulators, warps 2-5 the statistics epilogue of the
-// other: each warp reduces its 32 ids per token column with butterfly shuffles, the four
-// warps' records are merged in id order through shared memory.  Every wait is bounded.
+// other: each warp reduces its 32 ids for 32 token columns at a time with transposed
+// shuffles (lane L ends with column L), the four warps' records are merged in id order
+// through shared memory.  Every wait is bounded.
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -49,15 +50,36 @@ __device__ __forceinline__ void vu_cand_merge(float& m2, int& a, float om2, int 
   }
 }
 
-// the warp's (max, first argmax) over one value per lane, ties to the lower id
-__device__ __forceinline__ void vu_warp_argmax(float& m, int& a) {
+// Transposed warp reductions over 32 token columns: lane L enters with its id's value
+// for each of the 32 columns and leaves with column L's result over the warp's 32 ids.
+// At the stage with offset o each lane keeps one half of its current columns (the upper
+// half when bit o of its lane is set), sends the other half to lane L ^ o and merges what
+// it receives into what it keeps; after five stages the one column left is column L.
+// 31 exchanges per value for 32 columns, all of a stage independent of each other.
+__device__ __forceinline__ void vu_tr_argmax(float (&m)[32], int (&a)[32], int lane) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    const float om = __shfl_xor_sync(0xffffffffu, m, o);
-    const int oa = __shfl_xor_sync(0xffffffffu, a, o);
-    if (om > m || (om == m && oa < a)) {
-      m = om;
-      a = oa;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float km = up ? m[j + o] : m[j], sm = up ? m[j] : m[j + o];
+      const int ka = up ? a[j + o] : a[j], sa = up ? a[j] : a[j + o];
+      const float rm = __shfl_xor_sync(0xffffffffu, sm, o);
+      const int ra = __shfl_xor_sync(0xffffffffu, sa, o);
+      const bool take = rm > km || (rm == km && ra < ka);  // ties to the lower id
+      m[j] = take ? rm : km;
+      a[j] = take ? ra : ka;
+    }
+  }
+}
+__device__ __forceinline__ void vu_tr_sum(float (&e)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float ke = up ? e[j + o] : e[j], se = up ? e[j] : e[j + o];
+      e[j] = ke + __shfl_xor_sync(0xffffffffu, se, o);
     }
   }
 }
@@ -71,7 +93,7 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
   __shared__ __align__(8) uint64_t acc_full[2];
   __shared__ __align__(8) uint64_t acc_empty[2];
   __shared__ __align__(8) uint64_t drain_bar;
-  __shared__ UpdPart red[4][16];  // one 16-column chunk's records of the four epilogue warps
+  __shared__ UpdPart red[4][32];  // one 32-column group's records of the four epilogue warps
   __shared__ int epi_ok[4];       // each epilogue warp's wait result, so that all four leave together
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
@@ -207,37 +229,62 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
       const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
       const int id = m * VU_BM + lg * 32 + lane;  // this lane's vocabulary id
       const bool valid_id = id < p.V;
-      for (int c0 = 0; c0 < n_pad; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(t0 + c0, r);
-        tc_wait_ld();
-        UpdPart mine = {-INFINITY, 0.0f, 0x7fffffff, -INFINITY};  // lane q: column c0 + q's record
+      // the excluded id's lane, when it lies in this warp's 32 ids (warp-uniform)
+      const bool excl_here = p.excl >= 0 && p.excl >= m * VU_BM + lg * 32 && p.excl < m * VU_BM + lg * 32 + 32;
+      for (int c0 = 0; c0 < n_pad; c0 += 32) {
+        // this lane's id's logits for 32 token columns (16 when only 16 are left; the
+        // others count as -inf and their records are not stored)
+        float v[32], mm[32], e[32];
+        int aa[32];
+        {
+          uint32_t r[16];
+          tmem_ld16(t0 + c0, r);
+          tc_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float v = valid_id ? __uint_as_float(r[q]) : -INFINITY;
-          float wm = v;
-          int wa = valid_id ? id : 0x7fffffff;
-          vu_warp_argmax(wm, wa);
-          float cm = wm;
-          int ca = wa;
-          if (p.excl >= 0) {
-            cm = (id == p.excl) ? -INFINITY : v;
-            ca = (id == p.excl || !valid_id) ? 0x7fffffff : id;
-            vu_warp_argmax(cm, ca);
-          }
-          float e = (v == -INFINITY) ? 0.0f : __expf(v - wm);
+          for (int q = 0; q < 16; ++q) v[q] = valid_id ? __uint_as_float(r[q]) : -INFINITY;
+          if (c0 + 16 < n_pad) {
+            tmem_ld16(t0 + c0 + 16, r);
+            tc_wait_ld();
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-          if (lane == q) {
-            mine.m = wm;
-            mine.s = e;
-            mine.a = ca;
-            mine.m2 = cm;
+            for (int q = 0; q < 16; ++q) v[16 + q] = valid_id ? __uint_as_float(r[q]) : -INFINITY;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[16 + q] = -INFINITY;
           }
         }
-        if (lane < 16) red[lg][lane] = mine;
+        // column lane: the largest logit over the warp's ids and its first id
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          mm[q] = v[q];
+          aa[q] = valid_id ? id : 0x7fffffff;
+        }
+        vu_tr_argmax(mm, aa, lane);
+        const float col_m = mm[0];
+        const int col_a = aa[0];
+        // sum of exp(l - column max) over the warp's ids
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const float cm = __shfl_sync(0xffffffffu, col_m, q);
+          e[q] = (v[q] == -INFINITY) ? 0.0f : __expf(v[q] - cm);
+        }
+        vu_tr_sum(e, lane);
+        // the candidate: the argmax, or where the excluded id is one of this warp's, the
+        // argmax over the others
+        float cand_m = col_m;
+        int cand_a = col_a;
+        if (excl_here) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            mm[q] = (id == p.excl) ? -INFINITY : v[q];
+            aa[q] = (id == p.excl || !valid_id) ? 0x7fffffff : id;
+          }
+          vu_tr_argmax(mm, aa, lane);
+          cand_m = mm[0];
+          cand_a = aa[0];
+        }
+        red[lg][lane] = UpdPart{col_m, e[0], cand_a, cand_m};
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
-        if (lg == 0 && lane < 16 && c0 + lane < rows &&
+        if (lg == 0 && c0 + lane < rows &&
             DG_GUARD(row0 + c0 + lane < p.n_tokens && m < p.m_tiles && c0 + lane < n_pad, p.err)) {
           UpdPart o = red[0][lane];
 #pragma unroll
@@ -248,7 +295,7 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
           }
           p.part[(size_t)(row0 + c0 + lane) * p.m_tiles + m] = o;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // red is rewritten by the next chunk
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // red is rewritten by the next group
       }
       tc_fence_before();
       __syncwarp();

@@ -4,10 +4,11 @@ replayed at the address level on the CPU (tests/tc_emu.py), against the oracle's
 Transcribed from the kernel source: the persistent walk over (128-id tile, token chunk)
 tiles, id tile first, with its k-block rotation, the stage layout (weight tile, then token boxes of 64
 and 16 rows), the MMAs into one of two accumulator buffers, and the statistics epilogue:
-warp lg's lane holds id m 128 + 32 lg + lane, each 16-column chunk is reduced per column
-by butterflies (max with the first argmax, the candidate skipping an excluded id, the sum
-of exp(l - warp max)), lane q keeps column q's record, and warp 0 merges the four warps'
-records in id order into part[token][tile].  The row merge then reduces a token's tile
+warp lg's lane holds id m 128 + 32 lg + lane, each group of 32 token columns is reduced
+by transposed shuffles (max with the first argmax, the sum of exp(l - column max), and
+where the excluded id is one of the warp's, the candidate skipping it), lane L ends with
+column L's record, and warp 0 merges the four warps' records in id order into
+part[token][tile].  The row merge then reduces a token's tile
 records in lane order and a butterfly.  The records must give the oracle's argmax /
 candidate exactly and its confidence to rounding; each epilogue runs as late as its
 accumulator buffer allows.  The butterflies use float64 exp (the device exponential is
@@ -42,6 +43,42 @@ def ms_merge(m, s, om, os):
 
 def cand_merge(m2, a, om2, oa):
     return (om2, oa) if (om2 > m2 or (om2 == m2 and oa < a)) else (m2, a)
+
+
+def tr_argmax(m, a, bug=None):
+    """vu_tr_argmax over the warp: m, a [lane][32 columns] -> (max, first argmax) of column L
+    in lane L.  At the stage with offset o a lane keeps the upper half of its columns when
+    bit o of its lane is set, and merges the partner's values for that half into it."""
+    m, a = m.astype(np.float64), a.astype(np.int64)
+    o = 16
+    while o:
+        lanes = np.arange(32)
+        up = (lanes & o) != 0
+        if bug == "kept_half":
+            up = ~up
+        km = np.where(up[:, None], m[:, o:2 * o], m[:, :o])
+        ka = np.where(up[:, None], a[:, o:2 * o], a[:, :o])
+        sm = np.where(up[:, None], m[:, :o], m[:, o:2 * o])
+        sa = np.where(up[:, None], a[:, :o], a[:, o:2 * o])
+        rm, ra = sm[lanes ^ o], sa[lanes ^ o]
+        take = (rm > km) | ((rm == km) & (ra < ka))
+        m = np.where(take, rm, km)
+        a = np.where(take, ra, ka)
+        o >>= 1
+    return m[:, 0], a[:, 0]
+
+
+def tr_sum(e):
+    """vu_tr_sum: e [lane][32 columns] -> column L's sum in lane L (same exchange pattern)."""
+    o = 16
+    while o:
+        lanes = np.arange(32)
+        up = (lanes & o) != 0
+        ke = np.where(up[:, None], e[:, o:2 * o], e[:, :o])
+        se = np.where(up[:, None], e[:, :o], e[:, o:2 * o])
+        e = ke + se[lanes ^ o]
+        o >>= 1
+    return e[:, 0]
 
 
 def warp_argmax(v, ids):
@@ -101,23 +138,28 @@ def run_vocab_update(Wout, X, V, excl, n_max, smem_budget=200 * 1024, grid=5, bu
         def epilogue(j, t):
             m, row0, rows, n_pad = geom(t)
             d0 = (j & 1) * acc_cols
-            for c0 in range(0, n_pad, 16):
-                red = [[None] * 16 for _ in range(4)]
+            for c0 in range(0, n_pad, 32):
+                width = 32 if c0 + 16 < n_pad else 16      # the last group may hold 16 columns
+                red = [[None] * 32 for _ in range(4)]
                 for lg in range(4):
-                    ids = [m * BM + lg * 32 + ln for ln in range(32)]
-                    valid = [i < V for i in ids]
-                    vals = tm.f32(d0 + c0, 16)[lg * 32:lg * 32 + 32].astype(np.float64)   # [lane][q]
-                    for q in range(16):
-                        v = [float(vals[ln, q]) if valid[ln] else NEG for ln in range(32)]
-                        wm, wa = warp_argmax(v, [ids[ln] if valid[ln] else BIG for ln in range(32)])
-                        cm, ca = wm, wa
-                        if excl >= 0:
-                            cm, ca = warp_argmax([NEG if ids[ln] == excl else v[ln] for ln in range(32)],
-                                                 [BIG if (ids[ln] == excl or not valid[ln]) else ids[ln]
-                                                  for ln in range(32)])
-                        e = sum(0.0 if x == NEG else math.exp(x - wm) for x in v)
-                        red[lg][q] = (wm, e, ca, cm)
-                for ln in range(16):
+                    ids = np.array([m * BM + lg * 32 + ln for ln in range(32)])
+                    valid = ids < V
+                    vals = np.full((32, 32), NEG)              # [lane][column]
+                    vals[:, :width] = tm.f32(d0 + c0, width)[lg * 32:lg * 32 + 32].astype(np.float64)
+                    vals[~valid] = NEG
+                    aid = np.where(valid, ids, BIG)[:, None].repeat(32, axis=1)
+                    col_m, col_a = tr_argmax(vals.copy(), aid.copy(), bug)
+                    with np.errstate(invalid="ignore"):             # -inf - -inf where a column is empty
+                        e = np.where(vals == NEG, 0.0, np.exp(vals - col_m[None, :]))  # column q's max from lane q
+                    col_s = tr_sum(e)
+                    cand_m, cand_a = col_m, col_a
+                    if excl >= 0 and excl in ids:
+                        ev = np.where((ids == excl)[:, None], NEG, vals)
+                        ea = np.where(((ids == excl) | ~valid)[:, None], BIG, aid)
+                        cand_m, cand_a = tr_argmax(ev, ea, bug)
+                    for ln in range(32):
+                        red[lg][ln] = (col_m[ln], col_s[ln], cand_a[ln], cand_m[ln])
+                for ln in range(32):
                     if c0 + ln < rows:
                         mm, ss, aa, m2 = red[0][ln]
                         for w2 in range(1, 4):
@@ -211,10 +253,11 @@ def test_fused_masked_records_replay_gives_the_oracle_update():
     assert rec[0][0] > rec[0][3]                      # token 0: its maximum is the excluded id
 
 
-@pytest.mark.parametrize("bug", ["record_tile", "one_acc"])
+@pytest.mark.parametrize("bug", ["record_tile", "one_acc", "kept_half"])
 def test_planted_mistakes_in_the_fused_replay_are_caught(bug):
-    """Every tile's record written to tile 0, or one accumulator buffer for two tiles in
-    flight: the update differs from the oracle's (or records are missing)."""
+    """Every tile's record written to tile 0, one accumulator buffer for two tiles in
+    flight, or the transposed reduction keeping the wrong half (column L's record lands in
+    another lane): the update differs from the oracle's (or records are missing)."""
     C, V, K = 40, 512, 128
     W, X, lg = inputs(3, C, V, K)
     want = O.canvas_update(lg, 0, 1, 0)
