@@ -605,15 +605,30 @@ __global__ void gather_rows_kernel(const T* __restrict__ xn, const T* __restrict
   const int p = blockIdx.x;
   const int t = perm[p] / k;
   const int nv = H * (int)sizeof(T) / 16;
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * H);
-    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
-  }
-  if (xn_lo) {
-    const uint4* src = reinterpret_cast<const uint4*>(xn_lo + (size_t)t * H);
-    uint4* dst = reinterpret_cast<uint4*>(xs_lo + (size_t)p * H);
-    for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
+  const uint4* src = reinterpret_cast<const uint4*>(xn + (size_t)t * H);
+  const uint4* src_lo = xn_lo ? reinterpret_cast<const uint4*>(xn_lo + (size_t)t * H) : nullptr;
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
+  uint4* dst_lo = xn_lo ? reinterpret_cast<uint4*>(xs_lo + (size_t)p * H) : nullptr;
+  // four 16-byte loads of each term in flight per thread before the stores
+  constexpr int U = 4;
+  for (int i0 = threadIdx.x; i0 < nv; i0 += U * blockDim.x) {
+    uint4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < nv) {
+        a[u] = src[i];
+        if (src_lo) b[u] = src_lo[i];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < nv) {
+        dst[i] = a[u];
+        if (src_lo) dst_lo[i] = b[u];
+      }
+    }
   }
 }
 
@@ -639,6 +654,8 @@ cudaError_t launch_swiglu_f32(const float* g, const float* u, int rows, int F, f
   return launch_k(swiglu_f32_kernel, dim3(rows), dim3(256), 0, st, g, u, F, h);
 }
 
+constexpr int kMaxCombineSlots = 16;  // top-k limit of the router kernel
+
 // x[t] += sum_j w[t][j] * ys[inv[t*k + j]] (slots in order j = 0..k-1), then
 // xn[t] = x[t] / rms(x[t]) for the next consumer (next layer's QKV, or the vocabulary
 // projection with xn_lo = null).
@@ -659,14 +676,20 @@ __global__ void combine_norm_kernel(const float* __restrict__ ys, const int32_t*
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * H);
   float ss = 0.0f;
   for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
+    // every slot's row load issued before the first multiply-add (slots still added in order)
+    float4 y[kMaxCombineSlots];
+#pragma unroll
+    for (int j = 0; j < kMaxCombineSlots; ++j)
+      if (j < k) y[j] = reinterpret_cast<const float4*>(ys + (size_t)rows[j] * H)[i];
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 y = reinterpret_cast<const float4*>(ys + (size_t)rows[j] * H)[i];
-      acc.x = fmaf(ws[j], y.x, acc.x);
-      acc.y = fmaf(ws[j], y.y, acc.y);
-      acc.z = fmaf(ws[j], y.z, acc.z);
-      acc.w = fmaf(ws[j], y.w, acc.w);
-    }
+#pragma unroll
+    for (int j = 0; j < kMaxCombineSlots; ++j)
+      if (j < k) {
+        acc.x = fmaf(ws[j], y[j].x, acc.x);
+        acc.y = fmaf(ws[j], y[j].y, acc.y);
+        acc.z = fmaf(ws[j], y[j].z, acc.z);
+        acc.w = fmaf(ws[j], y[j].w, acc.w);
+      }
     float4 v = xr[i];
     v.x += acc.x;
     v.y += acc.y;
