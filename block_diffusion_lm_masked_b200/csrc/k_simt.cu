@@ -654,7 +654,7 @@ cudaError_t launch_swiglu_f32(const float* g, const float* u, int rows, int F, f
   return launch_k(swiglu_f32_kernel, dim3(rows), dim3(256), 0, st, g, u, F, h);
 }
 
-constexpr int kMaxCombineSlots = 16;  // top-k limit of the router kernel
+constexpr int kCombineBatch = 8;  // slot rows loaded together
 
 // x[t] += sum_j w[t][j] * ys[inv[t*k + j]] (slots in order j = 0..k-1), then
 // xn[t] = x[t] / rms(x[t]) for the next consumer (next layer's QKV, or the vocabulary
@@ -676,20 +676,23 @@ __global__ void combine_norm_kernel(const float* __restrict__ ys, const int32_t*
   float4* xr = reinterpret_cast<float4*>(x + (size_t)t * H);
   float ss = 0.0f;
   for (int i = threadIdx.x; i < H / 4; i += blockDim.x) {
-    // every slot's row load issued before the first multiply-add (slots still added in order)
-    float4 y[kMaxCombineSlots];
-#pragma unroll
-    for (int j = 0; j < kMaxCombineSlots; ++j)
-      if (j < k) y[j] = reinterpret_cast<const float4*>(ys + (size_t)rows[j] * H)[i];
+    // up to eight slots' row loads issued before their multiply-adds (slots still added in
+    // order)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
+      float4 y[kCombineBatch];
 #pragma unroll
-    for (int j = 0; j < kMaxCombineSlots; ++j)
-      if (j < k) {
-        acc.x = fmaf(ws[j], y[j].x, acc.x);
-        acc.y = fmaf(ws[j], y[j].y, acc.y);
-        acc.z = fmaf(ws[j], y[j].z, acc.z);
-        acc.w = fmaf(ws[j], y[j].w, acc.w);
-      }
+      for (int j = 0; j < kCombineBatch; ++j)
+        if (j0 + j < k) y[j] = reinterpret_cast<const float4*>(ys + (size_t)rows[j0 + j] * H)[i];
+#pragma unroll
+      for (int j = 0; j < kCombineBatch; ++j)
+        if (j0 + j < k) {
+          acc.x = fmaf(ws[j0 + j], y[j].x, acc.x);
+          acc.y = fmaf(ws[j0 + j], y[j].y, acc.y);
+          acc.z = fmaf(ws[j0 + j], y[j].z, acc.z);
+          acc.w = fmaf(ws[j0 + j], y[j].w, acc.w);
+        }
+    }
     float4 v = xr[i];
     v.x += acc.x;
     v.y += acc.y;
