@@ -487,6 +487,15 @@ struct GemmCall {
   int smem_budget;
 };
 
+// dense projections (no work list, one weight matrix, fp32 store) of at least two weight
+// tiles take them in pairs that share each token load
+bool pair_weight_tiles(int a_rows, bool grouped, bool dual, int epi) {
+  return !grouped && !dual && epi == dg::EPI_STORE_F32 && a_rows >= 256;
+}
+// weight tiles of a dense projection as the GEMM walks them (pairs where they are paired)
+int dense_weight_tiles(int a_rows) { return ceil_div(a_rows, pair_weight_tiles(a_rows, false, false,
+                                                                                  dg::EPI_STORE_F32) ? 256 : 128); }
+
 dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   CUtensorMap B, B2, Bb, B2b;
   dg_status s;
@@ -502,7 +511,8 @@ dg_status gemm_bf16(const GemmCall& g, int* err, cudaStream_t st) {
   dg::TcGemmParams p{};
   p.K = g.K;
   p.a_rows_per_group = g.a_rows_per_group;
-  p.m_tiles = ceil_div(g.a_rows_per_group, 128);
+  p.m_pair = pair_weight_tiles(g.a_rows_per_group, g.items != nullptr, g.A2 != nullptr, g.epi) ? 1 : 0;
+  p.m_tiles = ceil_div(g.a_rows_per_group, p.m_pair ? 256 : 128);
   p.n_max = g.n_max;
   p.n_tokens = g.x_rows;
   p.k_splits = g.k_splits;
@@ -751,7 +761,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   // ---- attention block: QKV (split-K partials) -> RoPE + K/V into the cache -> attention -> output projection
   int ks_qkv = 1, ks_o = 1;
   if (bf) {
-    ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
+    ks_qkv = pick_ksplit(dense_weight_tiles(QR), ceil_div(n, 128), H / 64, kMaxKsQkv);
     GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
                nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
@@ -769,7 +779,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
-    ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
+    ks_o = pick_ksplit(dense_weight_tiles(H), ceil_div(n, 128), nq * d / 64, kMaxKsO);
     GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
                n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
                kSmemGemm};
@@ -935,7 +945,7 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
   dg_status s;
   int ks_qkv = 1, ks_o = 1;
   if (bf) {
-    ks_qkv = pick_ksplit(QR / 128, ceil_div(n, 128), H / 64, kMaxKsQkv);
+    ks_qkv = pick_ksplit(dense_weight_tiles(QR), ceil_div(n, 128), H / 64, kMaxKsQkv);
     GemmCall g{DG_K_GEMM_QKV, dg::EPI_STORE_F32, &m->maps[l].qkv, nullptr, ws.at<void>(ws.L.xn), xn_lo, n, H, QR,
                nullptr, nullptr, 0, 128, ws.at<float>(ws.L.qkv), nullptr, QR, ks_qkv, (size_t)n * QR, kSmemGemm};
     if ((s = gemm_bf16(g, err, st)) != DG_OK) return s;
@@ -960,7 +970,7 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
   }
   if (stop_after_kv) return DG_OK;
   if (bf) {
-    ks_o = pick_ksplit(H / 128, ceil_div(n, 128), nq * d / 64, kMaxKsO);
+    ks_o = pick_ksplit(dense_weight_tiles(H), ceil_div(n, 128), nq * d / 64, kMaxKsO);
     GemmCall g{DG_K_GEMM_O, dg::EPI_STORE_F32, &m->maps[l].o, nullptr, ws.at<void>(ws.L.o), ws.at<void>(ws.L.o_lo),
                n, nq * d, H, nullptr, nullptr, 0, 128, ws.at<float>(ws.L.opart), nullptr, H, ks_o, (size_t)n * H,
                kSmemGemm};

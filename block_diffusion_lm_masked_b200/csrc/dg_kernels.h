@@ -33,6 +33,7 @@ struct TcGemmParams {
   const TcWorkItem* items;  // grouped: device work list (null: dense)
   const int* n_items;       // grouped: device count
   int dual_a;
+  int m_pair;            // a tile = two consecutive 128-row weight tiles (m_tiles counts pairs)
   int two_terms;
   void* out;
   void* out_lo;

@@ -12,7 +12,11 @@
 //
 // Options: two_terms (tokens given as bf16 hi + lo, both accumulated: fp32-precision
 // activations against bf16 weights); dual_a (gate and up weight tiles accumulated
-// into two TMEM regions, SwiGLU epilogue); k_splits (split-K, one output slab per split).
+// into two TMEM regions, SwiGLU epilogue); m_pair (a tile is two consecutive 128-row
+// weight tiles of one matrix sharing each token load: the dense projections, whose
+// token operand is re-read once per weight tile, read it half as often); k_splits
+// (split-K, one output slab per split).  Two accumulator buffers when they fit in the 512
+// TMEM columns, else one (the loads of the next tile still run during the epilogue).
 //
 // Each tile starts its K walk at a different k-block (tile index mod k-blocks): tiles
 // that run at the same time then read different k-blocks of the token operand, which
@@ -71,7 +75,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmParams& p, int t) {
 struct TileWalk {
   int r, n_tiles, m_tiles, full;
   __device__ TileWalk(const TcGemmParams& p, int n_tiles_) : r(0), n_tiles(n_tiles_), m_tiles(p.m_tiles) {
-    const bool partial = p.m_tiles > 1 && p.a_rows_per_group % TC_BM != 0;
+    const bool partial = p.m_tiles > 1 && p.a_rows_per_group % (p.m_pair ? 2 * TC_BM : TC_BM) != 0;
     full = partial ? n_tiles - n_tiles / p.m_tiles : n_tiles;
   }
   // the k-th tile of the list -> tile index (work item * m_tiles + weight tile)
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int terms = p.two_terms ? 2 : 1;
-  const int n_a = p.dual_a ? 2 : 1;
+  const int n_a = (p.dual_a || p.m_pair) ? 2 : 1;
   const uint32_t a_bytes = TC_BM * TC_BK * 2;           // one weight tile per k-block
   const uint32_t bmax_bytes = (uint32_t)p.n_max * 128;  // one token term per k-block, n_max rows
   const uint32_t stage_bytes = n_a * a_bytes + terms * bmax_bytes;
@@ -120,8 +124,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int acc_cols = p.n_max * n_a;  // one accumulator buffer
+  const int nbuf = 2 * acc_cols <= 512 ? 2 : 1;
   uint32_t tmem_cols = 32;
-  while (tmem_cols < (uint32_t)(2 * acc_cols)) tmem_cols <<= 1;
+  while (tmem_cols < (uint32_t)(nbuf * acc_cols)) tmem_cols <<= 1;
+  const int rows_per_tile = p.m_pair ? 2 * TC_BM : TC_BM;  // weight rows of one tile
   const int nkb = p.K / TC_BK / p.k_splits;
 
   if (warp == 1) tmem_alloc(&tmem_base_s, tmem_cols);
@@ -176,8 +182,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           uint8_t* sb = sa + n_a * a_bytes;
           const int kx = (ti.split * nkb + (kb + t) % nkb) * TC_BK;
           mbar_arrive_expect_tx(&full_bar[s], tx);
-          tma_load_3d(sa, &tmA, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
-          if (p.dual_a) tma_load_3d(sa + a_bytes, &tmA2, kx, ti.m * TC_BM, ti.g, &full_bar[s]);
+          const int arow = ti.m * rows_per_tile;
+          tma_load_3d(sa, &tmA, kx, arow, ti.g, &full_bar[s]);
+          if (p.dual_a) tma_load_3d(sa + a_bytes, &tmA2, kx, arow, ti.g, &full_bar[s]);
+          if (p.m_pair) tma_load_3d(sa + a_bytes, &tmA, kx, arow + TC_BM, ti.g, &full_bar[s]);
           int r = 0;
           for (; r + TC_B_BOX_BIG <= n_pad; r += TC_B_BOX_BIG) {
             tma_load_2d(sb + r * 128, &tmBb, kx, ti.row0 + r, &full_bar[s]);
@@ -200,8 +208,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (; ok && walk.next(t); ++j) {
         const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
-        const int buf = j & 1;
-        if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
+        const int buf = j % nbuf;
+        if (!mbar_wait(&acc_empty[buf], ((uint32_t)(j / nbuf) & 1u) ^ 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ACCUM))
           break;
         tc_fence_after();
         const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
@@ -224,7 +232,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint64_t bd2 = sw128_kmajor_desc(sb + bmax_bytes + kk * 32);
             tc_mma(d0, ad, bd, idesc, acc);
             if (terms == 2) tc_mma(d0, ad, bd2, idesc, 1u);
-            if (p.dual_a) {
+            if (n_a == 2) {
               const uint64_t ad2 = sw128_kmajor_desc(sa + a_bytes + kk * 32);
               tc_mma(d1, ad2, bd, idesc, acc);
               if (terms == 2) tc_mma(d1, ad2, bd2, idesc, 1u);
@@ -247,35 +255,38 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (; walk.next(t); ++j) {
       const TileInfo ti = decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;
-      const int buf = j & 1;
+      const int buf = j % nbuf;
       // the warp votes on the wait's outcome: tcgen05.ld below is warp-collective, so no lane
       // may go on alone after another gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, &abort_s, p.err,
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (uint32_t)(j / nbuf) & 1u, &abort_s, p.err,
                                              DG_DEVERR_TIMEOUT_ACCUM)))
         break;
       tc_fence_after();
-      const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols) + lane_off;
-      const int f = ti.m * TC_BM + row;  // weight row = output feature
-      const bool fvalid = f < p.a_rows_per_group;
-      for (int c0 = 0; c0 < n_pad; c0 += 16) {
-        uint32_t ra[16], rb[16];
-        tmem_ld16(t0 + c0, ra);
-        if (EPI == EPI_SWIGLU_BF16) tmem_ld16(t0 + p.n_max + c0, rb);
-        tc_wait_ld();
+      // paired weight tiles: the second accumulator holds weight rows 128 .. 255 of the tile
+      for (int half = 0; half < (p.m_pair ? 2 : 1); ++half) {
+        const uint32_t t0 = tmem + (uint32_t)(buf * acc_cols + half * p.n_max) + lane_off;
+        const int f = ti.m * rows_per_tile + half * TC_BM + row;  // weight row = output feature
+        const bool fvalid = f < p.a_rows_per_group;
+        for (int c0 = 0; c0 < n_pad; c0 += 16) {
+          uint32_t ra[16], rb[16];
+          tmem_ld16(t0 + c0, ra);
+          if (EPI == EPI_SWIGLU_BF16) tmem_ld16(t0 + p.n_max + c0, rb);
+          tc_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int col = c0 + q;
-          const float a = __uint_as_float(ra[q]);
-          const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
-          if (!fvalid || col >= ti.rows) continue;
-          const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
-          if (EPI == EPI_STORE_F32) {
-            reinterpret_cast<float*>(p.out)[(size_t)ti.split * p.split_stride + o] = a;
-          } else {
-            const float hv = a / (1.0f + expf(-a)) * b;
-            const bf16 hi = __float2bfloat16_rn(hv);
-            reinterpret_cast<bf16*>(p.out)[o] = hi;
-            if (p.out_lo) reinterpret_cast<bf16*>(p.out_lo)[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+          for (int q = 0; q < 16; ++q) {
+            const int col = c0 + q;
+            const float a = __uint_as_float(ra[q]);
+            const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
+            if (!fvalid || col >= ti.rows) continue;
+            const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
+            if (EPI == EPI_STORE_F32) {
+              reinterpret_cast<float*>(p.out)[(size_t)ti.split * p.split_stride + o] = a;
+            } else {
+              const float hv = a / (1.0f + expf(-a)) * b;
+              const bf16 hi = __float2bfloat16_rn(hv);
+              reinterpret_cast<bf16*>(p.out)[o] = hi;
+              if (p.out_lo) reinterpret_cast<bf16*>(p.out_lo)[o] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+            }
           }
         }
       }
@@ -356,9 +367,10 @@ cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2,
   if (p.k_splits < 1 || (p.K / TC_BK) % p.k_splits != 0 || (p.k_splits > 1 && p.items) || p.n_max < 16 ||
       p.n_max > 256 || (p.n_max % 16) != 0 || p.m_tiles < 1)
     return cudaErrorInvalidValue;
-  const int n_a = p.dual_a ? 2 : 1;
+  const int n_a = (p.dual_a || p.m_pair) ? 2 : 1;
   const int stage = n_a * TC_BM * TC_BK * 2 + (p.two_terms ? 2 : 1) * p.n_max * 128;
-  if (p.smem_budget < stage || 2 * p.n_max * n_a > 512 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0))
+  if (p.smem_budget < stage || p.n_max * n_a > 512 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0) ||
+      (p.m_pair && (p.dual_a || epi != EPI_STORE_F32)))
     return cudaErrorInvalidValue;
   const int smem = p.smem_budget + 1024;
   const int sms = num_sms();

@@ -23,11 +23,11 @@ from oracle import dg_oracle as O
 BM, BK = 128, 64
 
 
-def tile_walk(cta, grid, n_tiles, m_tiles, rows_a):
+def tile_walk(cta, grid, n_tiles, m_tiles, rows_a, tile_rows=BM):
     """TileWalk: rounds of `grid` tiles, every other round in reverse CTA order, over a list
     with the whole weight tiles first and each work item's partial last weight tile (when
-    rows_a is not a multiple of 128) at the end."""
-    partial = m_tiles > 1 and rows_a % BM != 0
+    rows_a is not a multiple of the tile's weight rows) at the end."""
+    partial = m_tiles > 1 and rows_a % tile_rows != 0
     full = n_tiles - n_tiles // m_tiles if partial else n_tiles
 
     def order(k):
@@ -47,22 +47,28 @@ def tile_walk(cta, grid, n_tiles, m_tiles, rows_a):
 
 
 def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1, W2=None, split_stride=0,
-             smem_budget=200 * 1024, grid=5, bug=None):
+             smem_budget=200 * 1024, grid=5, bug=None, m_pair=None):
     """W / W2: bf16 bits [G][rows][K]; X_hi / X_lo: bf16 bits [n][K]; items: (group, row0,
-    rows) or None (dense).  Returns the output array as the kernel writes it."""
+    rows) or None (dense).  m_pair: tiles of two consecutive 128-row weight tiles (default:
+    as the host chooses, dense fp32-store GEMMs of at least 256 weight rows).  Returns the
+    output array as the kernel writes it."""
     terms = 2 if X_lo is not None else 1
-    n_a = 2 if W2 is not None else 1
+    if m_pair is None:
+        m_pair = items is None and W2 is None and rows_a >= 256
+    n_a = 2 if (W2 is not None or m_pair) else 1
+    tile_rows = 2 * BM if m_pair else BM
     a_bytes = BM * BK * 2
     bmax_bytes = n_max * 128
     stage_bytes = n_a * a_bytes + terms * bmax_bytes
     stages = min(smem_budget // stage_bytes, 16)
     acc_cols = n_max * n_a
+    nbuf = 2 if 2 * acc_cols <= 512 else 1
     tmem_cols = 32
-    while tmem_cols < 2 * acc_cols:
+    while tmem_cols < nbuf * acc_cols:
         tmem_cols <<= 1
     assert tmem_cols <= 512
     nkb = K // BK // k_splits
-    m_tiles = -(-rows_a // BM)
+    m_tiles = -(-rows_a // tile_rows)
     n_tokens = X_hi.shape[0]
     dense = items is None
     chunks = -(-n_tokens // n_max)
@@ -87,7 +93,7 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
 
     for cta in range(min(grid, n_tiles)):
         sm, tm = T.Smem(stages * stage_bytes), T.Tmem(tmem_cols)
-        tiles = tile_walk(cta, grid, n_tiles, m_tiles, rows_a)
+        tiles = tile_walk(cta, grid, n_tiles, m_tiles, rows_a, tile_rows)
         its = [(t, kb) for t in tiles for kb in range(nkb)]
         loaded = mma_done = 0
         pending = []
@@ -99,9 +105,11 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
             sa = (it % stages) * stage_bytes
             sb = sa + n_a * a_bytes
             kx = (split * nkb + (kb + t) % nkb) * BK
-            sm.tma_load(sa, W, (kx, m * BM, g), (64, 128, 1), 128)
-            if n_a == 2:
-                sm.tma_load(sa + a_bytes, W2, (kx, m * BM, g), (64, 128, 1), 128)
+            sm.tma_load(sa, W, (kx, m * tile_rows, g), (64, 128, 1), 128)
+            if W2 is not None:
+                sm.tma_load(sa + a_bytes, W2, (kx, m * tile_rows, g), (64, 128, 1), 128)
+            if m_pair:
+                sm.tma_load(sa + a_bytes, W, (kx, m * tile_rows + BM, g), (64, 128, 1), 128)
             r = 0
             lo_off = bmax_bytes if bug != "lo_offset" else n_pad * 64
             while r + 64 <= n_pad:
@@ -117,8 +125,13 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
 
         def epilogue(j, t):
             g, row0, rows, split, m = tile_of(t)
-            d0 = (j & 1) * acc_cols
-            f = m * BM + np.arange(BM)
+            for half in range(2 if m_pair else 1):
+                epilogue_half(j, t, half)
+
+        def epilogue_half(j, t, half):
+            g, row0, rows, split, m = tile_of(t)
+            d0 = (j % nbuf) * acc_cols + half * n_max
+            f = m * tile_rows + half * BM + np.arange(BM)
             ok = f < rows_a
             for col in range(rows):
                 a = tm.f32(d0 + col, 1)[:, 0].astype(np.float64)
@@ -139,11 +152,11 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
             t, kb = its[it]
             j = tiles.index(t)
             if kb == 0:
-                while pending and pending[0][0] <= j - 2:
+                while pending and pending[0][0] <= j - nbuf:
                     epilogue(*pending.pop(0))
             g, row0, rows, split, m = tile_of(t)
             n_pad = (rows + 15) & ~15
-            d0 = (j & 1) * acc_cols
+            d0 = (j % nbuf) * acc_cols
             d1 = d0 + (n_max if bug != "d1" else acc_cols // 4)
             sa = (it % stages) * stage_bytes
             sb = sa + n_a * a_bytes
@@ -259,3 +272,24 @@ def test_tile_walk_covers_every_tile_once_and_balances_the_weight_bytes(n_items,
         assert max(load) == 5 * BM
         strided = [sum(rows(t) for t in range(c, n_tiles, grid)) for c in range(grid)]
         assert max(strided) == 6 * BM
+
+
+@pytest.mark.parametrize("rows,n,terms,n_max", [(320, 150, 2, 128), (704, 37, 2, 128), (384, 200, 1, 256),
+                                               (256, 16, 1, 256)])
+def test_paired_weight_tiles_replay(rows, n, terms, n_max):
+    """Dense projections with paired weight tiles (two 128-row tiles sharing each token
+    load; a partial pair where the rows end mid-pair); with 256 tokens per tile the two
+    accumulators fill TMEM and the kernel keeps one buffer.  The unpaired replay agrees to
+    fp32 summation order (a tile's k-blocks start at a rotation that depends on its index)."""
+    rng = np.random.default_rng(rows + n)
+    K = 256
+    x, hi, lo = bf16_pair(rng, n, K)
+    if terms == 1:
+        lo = None
+        x = T.bf16_value(hi).astype(np.float64)
+    W, w = weights(rng, 1, rows, K)
+    out, _ = run_gemm(W, hi, lo, rows, K, rows, n_max=n_max, m_pair=True)
+    ref = x @ w[0].T
+    assert np.abs(out.reshape(n, rows) - ref).max() / np.abs(ref).max() < 2e-6
+    plain, _ = run_gemm(W, hi, lo, rows, K, rows, n_max=n_max, m_pair=False)
+    assert np.abs(out - plain).max() / np.abs(ref).max() < 2e-6

@@ -124,11 +124,13 @@ def run(roles, q, seed, max_steps=200000, end_check=False):
 
 # ---------------------------------------------------------------- the bf16 GEMM (k_tc_gemm.cu)
 
-def bf16_gemm(n_tiles, nkb, stages):
+def bf16_gemm(n_tiles, nkb, stages, nbuf=2):
+    """nbuf: accumulator buffers (one where two do not fit in TMEM: paired weight tiles of
+    256 token columns)."""
     full = [Barrier(f"full{s}", 1) for s in range(stages)]
     empty = [Barrier(f"empty{s}", 1) for s in range(stages)]
-    acc_full = [Barrier(f"acc_full{b}", 1) for b in range(2)]
-    acc_empty = [Barrier(f"acc_empty{b}", 4) for b in range(2)]
+    acc_full = [Barrier(f"acc_full{b}", 1) for b in range(nbuf)]
+    acc_empty = [Barrier(f"acc_empty{b}", 4) for b in range(nbuf)]
     bufs, q = Buffers(), Async()
     acc_done = {}
 
@@ -146,8 +148,8 @@ def bf16_gemm(n_tiles, nkb, stages):
     def mma():
         it = 0
         for j in range(n_tiles):
-            buf = j & 1
-            yield wait(acc_empty[buf], ((j >> 1) & 1) ^ 1, (j >> 1) - 1)
+            buf = j % nbuf
+            yield wait(acc_empty[buf], ((j // nbuf) & 1) ^ 1, j // nbuf - 1)
             bufs.fill(("acc", buf), 4)
             acc_done[buf] = 0
             for kb in range(nkb):
@@ -164,8 +166,8 @@ def bf16_gemm(n_tiles, nkb, stages):
 
     def epilogue(w):
         for j in range(n_tiles):
-            buf = j & 1
-            yield wait(acc_full[buf], (j >> 1) & 1, j >> 1)
+            buf = j % nbuf
+            yield wait(acc_full[buf], (j // nbuf) & 1, j // nbuf)
             assert acc_done[buf] == nkb, "epilogue read an accumulator before its MMAs completed"
             bufs.release(("acc", buf))
             acc_empty[buf].arrive()
@@ -261,9 +263,10 @@ def lowp_gemm(n_tiles, nkb, stages, t_stages=4, dec_warps=8):
 
 
 @pytest.mark.parametrize("n_tiles,nkb,stages", [(1, 1, 2), (3, 1, 3), (2, 5, 3), (5, 4, 6), (4, 32, 3), (7, 3, 8)])
-def test_bf16_gemm_protocol(n_tiles, nkb, stages):
+@pytest.mark.parametrize("nbuf", [2, 1])
+def test_bf16_gemm_protocol(n_tiles, nkb, stages, nbuf):
     for seed in range(30):
-        roles, q = bf16_gemm(n_tiles, nkb, stages)
+        roles, q = bf16_gemm(n_tiles, nkb, stages, nbuf)
         run(roles, q, seed, end_check=True)
 
 
