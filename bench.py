@@ -618,6 +618,37 @@ def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None)
     return out
 
 
+def _graph_time(call, steps, warmup):
+    """Median device time (us) of one `call`, captured once into a CUDA graph and replayed
+    with CUDA events around each replay: the host work of the call (tensor-map encoding,
+    argument checks) stays out of the timed region, which then holds only the call's
+    device work."""
+    import torch
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            call()
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    del graph
+    return statistics.median(ts)
+
+
 def run_kernel_attention(args):
     """--kernel attention: the block-masked attention launch alone (debug entry: the
     attention kernel and its split-KV merge) on synthetic bf16 data, the canvas's queries
@@ -642,19 +673,9 @@ def run_kernel_attention(args):
     out = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device=dev)
     lo = torch.zeros_like(out)
     fn = dg.debug_attention_pair_bf16 if args.attn_pair else dg.debug_attention_bf16
-    for _ in range(args.warmup):
-        fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo)
-    torch.cuda.synchronize(dev)
-    ts = []
-    for _ in range(args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo)
-        e1.record()
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) * 1e3)
+    us = _graph_time(lambda: fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo), args.steps,
+                     args.warmup)
     dg.device_status(ws)
-    us = statistics.median(ts)
     hbm, tf_burst, _, peak_src = _peaks()
     fl = 4.0 * n_q * nq * d * n_keys
     tf = fl / (us * 1e-6) / 1e12
@@ -720,20 +741,9 @@ def run_kernel_gemm(args):
             scratch = dg.debug_gemm_scratch(rows, E)
             call = lambda: dg.debug_gemm_bf16(W, X, out, H, err, scratch, X_lo=X_lo, group_off=off)
             nbytes = RF.down_bytes(cfg, E, rows)
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize(dev)
-    ts = []
-    for _ in range(args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        call()
-        e1.record()
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) * 1e3)
+    us = _graph_time(call, args.steps, args.warmup)
     if err.item() != 0:
         raise RuntimeError(f"GEMM error word {err.item()}")
-    us = statistics.median(ts)
     hbm, _, _, peak_src = _peaks()
     gbs = nbytes / (us * 1e-6) / 1e9
     line = {"metric": f"GEMM launch latency ({args.gemm}, large model's shape)", "value": us, "unit": "us",

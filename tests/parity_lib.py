@@ -18,14 +18,18 @@ compared numerically:
   * routing weights within 2e-2 relative; hidden states and logits within
     max |gpu - oracle| / rms(oracle) <= 2e-2 (bf16) or 1e-4 (fp32);
   * canvas tokens exactly (the argmax of identical logits), confidences within 1e-5;
-  * stored K/V within one bf16 rounding step (identical inputs round alike except at
-    a rounding boundary).
+  * stored K/V: each element within half a bf16 step (its rounding) plus the fp32
+    tolerance (1e-4 of the rms) of the exact value, and at most 1% of the elements
+    different from the exact value's own rounding (values computed in fp32 from the same
+    input round alike except near a rounding boundary).
 
 Free-running comparison (`compare_pass`, `compare_update`) -- reported beside it: the
 oracle's whole pass from the same canvas and cache against the GPU's.  Routing
 differences at near ties are allowed; after one at a layer before the last, the two
 sides compute different problems, so the rest of that free-running pass is checked
-for structure only (the forced checks above still cover every stage).
+for structure only (the forced checks above still cover every stage).  The update is
+compared with margins widened to the measured logit difference of the two passes
+(`logit_shift`): each side updates its own logits.
 """
 from __future__ import annotations
 
@@ -267,31 +271,48 @@ def kv_close(gpu, ref, skip_positions=(), tol_rms=2e-2):
     return (not bad.any()) and frac < 0.2, frac, worst
 
 
-def compare_update(canvas_gpu, conf_gpu, upd_o, exempt, n):
-    """Canvas after the update: tokens, re-noise set and confidences."""
+def logit_shift(logits_gpu, logits_o, exempt=()):
+    """Largest |gpu - oracle| logit over the rows not exempt (0 when none is left)."""
+    g = np.asarray(logits_gpu, dtype=np.float64)
+    r = np.asarray(logits_o, dtype=np.float64)
+    keep = np.ones(r.shape[0], dtype=bool)
+    keep[[i for i in exempt if i < r.shape[0]]] = False
+    return float(np.abs(g[keep] - r[keep]).max()) if keep.any() else 0.0
+
+
+def compare_update(canvas_gpu, conf_gpu, upd_o, exempt, n, logit_err=0.0):
+    """Canvas after the update, free-running: the GPU's update of its own logits against
+    the oracle's update of the oracle's logits, which differ by at most `logit_err` per
+    element (measured).  A log-confidence (the top logit minus the log-sum-exp of the
+    row) then moves by at most 2 * logit_err on each side, so a position keeps its side
+    of the re-noise cut wherever its cut margin exceeds 4 * logit_err, its argmax
+    wherever the top-1 minus top-2 logit exceeds 2 * logit_err, and its confidence is
+    within a factor exp(2 * logit_err).  Those margins never go below the forced
+    check's (1e-3 for the cut, 1e-2 for tokens)."""
     canvas_gpu = np.asarray(canvas_gpu)
     C = canvas_gpu.shape[0]
+    cut_m = max(CUT_MARGIN, 4.0 * logit_err * 1.0001)
+    tok_m = max(TOKEN_MARGIN, 2.0 * logit_err * 1.0001)
     ren_o = set(upd_o["renoised"].tolist())
     for i in range(C):
         if i in exempt:
             continue
-        if upd_o["cut_margin"][i] < CUT_MARGIN:
+        if upd_o["cut_margin"][i] < cut_m:
             continue
         if i in ren_o:
             assert canvas_gpu[i] == upd_o["canvas"][i], f"re-noised position {i}: {canvas_gpu[i]} vs {upd_o['canvas'][i]}"
-        elif upd_o["top_margin"][i] > TOKEN_MARGIN:
+        elif upd_o["top_margin"][i] > tok_m:
             assert canvas_gpu[i] == upd_o["canvas"][i], f"position {i}: token {canvas_gpu[i]} vs {upd_o['canvas'][i]}"
     if conf_gpu is not None:
         c = np.asarray(conf_gpu, dtype=np.float64)
         # the set the GPU re-noised, read from its own confidences with the stated rule
         gpu_set = set(np.argsort(c, kind="stable")[:n].tolist())
         for i in gpu_set ^ ren_o:
-            assert i in exempt or upd_o["cut_margin"][i] < CUT_MARGIN, (
-                f"re-noise set differs at {i}: cut margin {upd_o['cut_margin'][i]:.3e}")
+            assert i in exempt or upd_o["cut_margin"][i] < cut_m, (
+                f"re-noise set differs at {i}: cut margin {upd_o['cut_margin'][i]:.3e} (bound {cut_m:.3e})")
         keep = [i for i in range(C) if i not in exempt]
-        # free-running: the two sides' logits differ by up to the 2e-2 rms tolerance, and a
-        # confidence (the largest softmax probability) moves by about twice a logit's error
-        np.testing.assert_allclose(c[keep], upd_o["conf"][keep], rtol=5e-2)
+        rtol = max(CONF_RTOL, float(np.expm1(2.0 * logit_err)) * 1.0001)
+        np.testing.assert_allclose(c[keep], upd_o["conf"][keep], rtol=rtol)
 
 
 # ---------------------------------------------------------------- several canvases
@@ -356,7 +377,7 @@ def check_batched_pass(dg, cfg, prefixes, C, prepare=None):
     for b in range(B):
         upd_o = O.canvas_update(res[b][0], n, synth.SEED_RENOISE + b, 0)
         ex_b = {r - b * C for r in exempt if b * C <= r < (b + 1) * C}
-        compare_update(out_np[b], conf_np[b], upd_o, ex_b, n)
+        compare_update(out_np[b], conf_np[b], upd_o, ex_b, n, logit_shift(lg_np[b], res[b][0], ex_b))
     print(report, "exempt rows:", len(exempt))
     # the caches' committed prefixes are untouched and their lengths unchanged
     for c, P in zip(bt.caches, prefixes):
@@ -547,19 +568,22 @@ def forced_prefill_check(cfg, host, prec, cache_before, tokens, taps_gpu, cache_
 
 
 def kv_stored_close(gpu, exact, prec, max_frac=0.01):
-    """K/V the GPU stored against the oracle's unrounded K/V from the same input: bf16
-    storage holds the value's rounding, and a GPU value a few ulps of fp32 away from the
-    oracle's may round to the neighbouring bf16 value, so each element lies within one
-    bf16 step of the exact value and only a small fraction differs from the oracle's own
-    rounding; fp32 storage within 1e-4 relative to the rms."""
+    """K/V the GPU stored against the oracle's unrounded K/V from the same input.  The GPU
+    computes the value in fp32 (within the fp32 tolerance, 1e-4 of the rms, of the exact
+    value) and bf16 storage holds its rounding (within half a bf16 step of it), so each
+    element lies within half a step plus that tolerance of the exact value, and only a
+    small fraction differs from the exact value's own rounding; fp32 storage within 1e-4
+    relative to the rms."""
     g = np.asarray(gpu, np.float64)
     r = np.asarray(exact, np.float64)
+    rms = np.sqrt(np.mean(r * r))
     if prec.dtype != "bf16":
-        err = np.abs(g - r).max() / np.sqrt(np.mean(r * r))
+        err = np.abs(g - r).max() / rms
         return err <= 1e-4, float(err), ""
     stored = O.round_bf16(r)
     d = np.abs(g - r)
-    bad = d > bf16_spacing(r) * 1.0001
+    half_step = 0.5 * bf16_spacing(np.maximum(np.abs(g), np.abs(r)))
+    bad = d > half_step * 1.0001 + 1e-4 * rms
     frac = float((g != stored).mean())
     worst = ""
     if bad.any():

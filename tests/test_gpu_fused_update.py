@@ -100,4 +100,7 @@ def test_fused_update_matches_the_oracle_full_size(dg):
     stats = PL.forced_pass_check(cfg, st.host, st.prec, st.ocache, canvas0, taps_f, None, label="fused pass")
     print("forced layers of the fused call:", PL.summary(stats))
     upd_o = O.canvas_update(logits_o, n, synth.SEED_RENOISE, 0)
-    PL.compare_update(out.cpu().numpy(), conf.cpu().numpy(), upd_o, exempt, n)
+    # the fused call's logits (never written) come from the same single-term input and
+    # weights as the separate pass's, in another fp32 summation order: 1% slack
+    shift = 1.01 * PL.logit_shift(logits.cpu().numpy(), logits_o, exempt)
+    PL.compare_update(out.cpu().numpy(), conf.cpu().numpy(), upd_o, exempt, n, shift)

@@ -56,7 +56,7 @@ def _check_one_pass(dg, cfg, P, C):
     upd_o = O.canvas_update(logits_o, n, synth.SEED_RENOISE, 0)
     report = []
     exempt = PL.compare_pass(cfg, taps, logits, taps_o, logits_o, report)
-    PL.compare_update(canvas, conf, upd_o, exempt, n)
+    PL.compare_update(canvas, conf, upd_o, exempt, n, PL.logit_shift(logits, logits_o, exempt))
     print("forced:", PL.summary(stats), "| free-running:", report, "exempt rows:", sorted(exempt))
     return st
 

@@ -174,3 +174,66 @@ def test_forced_check_sees_a_wrong_layer_a_wrong_route_and_a_wrong_token():
     out[i] = (out[i] + 1) % SMALL["vocab"]
     with pytest.raises(AssertionError, match="tokens differ"):
         PL.forced_pass_check(SMALL, host, prec, oc, canvas, t, logits, out, upd["conf"], n, 77, 1)
+
+
+def test_stored_kv_rule():
+    """A stored bf16 value is the rounding of an fp32 value within the fp32 tolerance of
+    the exact one: a tiny element whose exact value sits just short of a rounding boundary
+    may round to the neighbour (half a step plus 1e-4 of the rms away); an element a
+    whole step off at a large magnitude, or too many neighbour roundings, fail."""
+    from oracle import dg_oracle as O
+    prec = O.Precision("bf16")
+    rng = np.random.default_rng(3)
+    exact = rng.standard_normal((2, 64, 16)) * 0.3
+    stored = O.round_bf16(exact)
+    assert PL.kv_stored_close(stored, exact, prec)[0]
+    # a tiny element just below a rounding boundary, stored one step up
+    e2, s2 = exact.copy(), stored.copy()
+    sp = PL.bf16_spacing(2.8e-4)
+    e2[0, 0, 0] = -(2.44140625e-4 + 18.977 * sp)
+    s2[0, 0, 0] = -(2.44140625e-4 + 20 * sp)
+    ok, frac, _ = PL.kv_stored_close(s2, e2, prec)
+    assert ok and frac > 0
+    # a large element one whole step off
+    s3 = stored.copy()
+    i = np.unravel_index(np.argmax(np.abs(exact)), exact.shape)
+    s3[i] = stored[i] + np.sign(stored[i]) * PL.bf16_spacing(stored[i])
+    assert not PL.kv_stored_close(s3, exact, prec)[0]
+    # neighbour roundings on more than 1% of the elements
+    s4 = stored.copy()
+    flat = s4.reshape(-1)
+    idx = np.argsort(np.abs(exact).reshape(-1))[:40]   # the smallest: inside the rms floor
+    flat[idx] += PL.bf16_spacing(flat[idx])
+    ok, frac, _ = PL.kv_stored_close(s4, exact, prec)
+    assert not ok and frac > 0.01
+
+
+def _update(logits, n):
+    from oracle import dg_oracle as O
+    return O.canvas_update(logits, n, 11, 0)
+
+
+def test_free_running_update_margins_follow_the_logit_shift():
+    """The free-running update check widens its margins to the measured logit difference:
+    the oracle's update of logits shifted by delta passes against the unshifted update
+    when delta is passed, and a token changed at a clear margin still fails."""
+    rng = np.random.default_rng(5)
+    C, V, n = 48, 64, 12
+    lo = rng.standard_normal((C, V))
+    delta = 2e-2
+    lg = lo + rng.uniform(-delta, delta, size=lo.shape)
+    up_o, up_g = _update(lo, n), _update(lg, n)
+    PL.compare_update(up_g["canvas"], up_g["conf"], up_o, set(), n, PL.logit_shift(lg, lo))
+    # a kept position given another token although its top margin is large
+    kept = [i for i in range(C) if i not in set(up_o["renoised"].tolist())
+            and up_o["top_margin"][i] > 10 * delta and up_o["cut_margin"][i] > 10 * delta]
+    assert kept
+    bad = up_g["canvas"].copy()
+    bad[kept[0]] = (bad[kept[0]] + 1) % V
+    with pytest.raises(AssertionError):
+        PL.compare_update(bad, up_g["conf"], up_o, set(), n, PL.logit_shift(lg, lo))
+    # a confidence off by more than exp(2 delta)
+    conf = np.asarray(up_g["conf"], dtype=np.float64).copy()
+    conf[kept[0]] *= 1.2
+    with pytest.raises(AssertionError):
+        PL.compare_update(up_g["canvas"], conf, up_o, set(), n, PL.logit_shift(lg, lo))
