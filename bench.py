@@ -534,33 +534,70 @@ def run_chained(args, cfg, name):
     dg.device_status(ws)
 
     hbm, tf_burst, tf_sust, peak_src = _peaks()
-    # roofline of the chain: every pass at its prefix length (expert unions taken as E,
-    # the near-full coverage random routing gives), every prefill
-    E = cfg["n_experts"]
+    # the expert union of every layer of every call of one chain (an untimed chain run
+    # call by call with the union tap; the same passes as dg_generate_canvas): converging
+    # canvases repeat tokens, so later passes touch fewer experts
+    L = cfg["n_layers"]
+    uni = torch.zeros(L, dtype=torch.int32, device=dev)
+    model.set_taps({"unions": uni, "rows": max(T0, C)})
+
+    def unions_now():
+        torch.cuda.synchronize(dev)
+        return [int(u) for u in uni.cpu()]
+
+    cache.len = 0
+    dg.prefill_append(model, cache, prompt, ws)
+    prefill_unions = [unions_now()]
+    pass_unions = []
+    for c in range(NC):
+        canv[c].copy_(noise[c])
+        per = []
+        for st_ in range(S):
+            dg.denoise_pass(model, cache, canv[c], logits, ws)
+            per.append(unions_now())
+            dg.canvas_update(logits, dg.renoise_count(C, S, st_, r0, r1), synth.SEED_RENOISE, st_, canv[c], ws)
+        pass_unions.append(per)
+        dg.prefill_append(model, cache, canv[c], ws)
+        prefill_unions.append(unions_now())
+    model.set_taps(None)
+    dg.device_status(ws)
+
+    # roofline of the chain: every pass at its prefix length, every prefill, with the
+    # measured unions
     t_roof = 0.0
     flops_total = bytes_total = 0.0
     for c in range(NC):
         P = T0 + c * C
         f = RF.pass_flops(cfg, P, C)
-        b = RF.pass_bytes(cfg, P, C, [E] * cfg["n_layers"]) + 8 * C
-        t_roof += S * RF.time_bound(f, b, tf_burst * 1e12, hbm * 1e9)
-        flops_total += S * f
-        bytes_total += S * b
-    for P, T in [(0, T0)] + [(T0 + c * C, C) for c in range(NC)]:
+        for u in pass_unions[c]:
+            b = RF.pass_bytes(cfg, P, C, u) + 8 * C
+            t_roof += RF.time_bound(f, b, tf_burst * 1e12, hbm * 1e9)
+            flops_total += f
+            bytes_total += b
+    for (P, T), u in zip([(0, T0)] + [(T0 + c * C, C) for c in range(NC)], prefill_unions):
         f = RF.prefill_flops(cfg, P, T)
-        b = RF.prefill_bytes(cfg, P, T, [E] * cfg["n_layers"])
+        b = RF.prefill_bytes(cfg, P, T, u)
         t_roof += RF.time_bound(f, b, tf_burst * 1e12, hbm * 1e9)
         flops_total += f
         bytes_total += b
     ms_chain = total_ms / args.steps
     passes = NC * S
     value = job_value(world, passes * C, args.steps, total_ms)
-    kroof = kernel_rooflines(cfg, T0 + (NC - 1) * C / 2, C, [E] * cfg["n_layers"], kern, hbm, tf_sust, peak_src)
+    # per-launch algorithmic bytes of the expert GEMMs, averaged over the chain's launches
+    # (each pass: L launches of C rows; each prefill: L - 1 launches of T rows)
+    k = cfg["top_k"]
+    eg = [(u, C * k) for per in pass_unions for us in per for u in us]
+    eg += [(u, T * k) for T, us in zip([T0] + [C] * NC, prefill_unions) for u in us[:L - 1]]
+    expert_bytes = {"gemm_gate_up": sum(RF.gate_up_bytes(cfg, u, r) for u, r in eg) / len(eg),
+                    "gemm_down": sum(RF.down_bytes(cfg, u, r) for u, r in eg) / len(eg)}
+    kroof = kernel_rooflines(cfg, T0 + (NC - 1) * C / 2, C, None, kern, hbm, tf_sust, peak_src,
+                             expert_bytes=expert_bytes)
     roof = None
     if kroof:
         dom = max(kroof, key=lambda n: kern[n]["share"])
         roof = dict(kroof[dom], kernel=dom, traffic=_ncu_traffic(name, dom),
-                    note="per-launch averages over the chain; attention FLOPs at the mean prefix length")
+                    note="per-launch averages over the chain (expert GEMM bytes from the measured unions of every "
+                         "call); attention FLOPs at the mean prefix length")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_chain, "pass_latency_us": statistics.median(canvas_ms) * 1e3 / S,
@@ -590,10 +627,12 @@ def run_chained(args, cfg, name):
     return 0
 
 
-def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None):
+def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None, expert_bytes=None):
     """Achieved rate and fraction of its bound for each big kernel of the step: the expert
     and vocabulary GEMMs and the update statistics against HBM bandwidth (algorithmic
-    bytes per launch), attention against the bf16 tensor peak (algorithmic FLOPs)."""
+    bytes per launch), attention against the bf16 tensor peak (algorithmic FLOPs).
+    `expert_bytes`: per-launch bytes of the expert GEMMs when they are not those of one
+    pass with per-layer `unions`."""
     rows = C if rows is None else rows
     k, L = cfg["top_k"], cfg["n_layers"]
     out = {}
@@ -603,8 +642,11 @@ def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None)
             a = nbytes_launch / (kern[kname]["avg_us"] * 1e-6) / 1e9
             out[kname] = {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
                           "bytes_per_launch": nbytes_launch, "peak_source": f"{peak_src} hbm_gbs"}
-    hbm_entry("gemm_gate_up", sum(RF.gate_up_bytes(cfg, u, rows * k) for u in unions) / L)
-    hbm_entry("gemm_down", sum(RF.down_bytes(cfg, u, rows * k) for u in unions) / L)
+    if expert_bytes is None:
+        expert_bytes = {"gemm_gate_up": sum(RF.gate_up_bytes(cfg, u, rows * k) for u in unions) / L,
+                        "gemm_down": sum(RF.down_bytes(cfg, u, rows * k) for u in unions) / L}
+    for kname, nb in expert_bytes.items():
+        hbm_entry(kname, nb)
     hbm_entry("gemm_vocab", RF.vocab_bytes(cfg, rows))
     hbm_entry("update_partial", RF.update_bytes(cfg, rows))
     if "attention" in kern:

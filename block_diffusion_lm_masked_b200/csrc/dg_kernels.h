@@ -83,9 +83,9 @@ struct TcAttnParams {
   int has_lo;          // query and current K/V carry low terms (bf16 model)
   const __nv_bfloat16* q;     // query hi [nq][n_q][128] (read directly by tc_attn_kernel)
   const __nv_bfloat16* q_lo;  // query lo, same layout
-  int* merge_cnt;             // [q tiles][nq] split tickets, zero on entry (tc_attn_kernel merges its
-                              // splits itself when n_splits > 1; the last split of a tile and head
-                              // to finish does it and leaves the ticket at zero)
+  int* merge_cnt;             // [q tiles][nq] split tickets, zero on entry: when n_splits > 1 the
+                              // last split of a tile and head (head pair: ticket of its first
+                              // head) to finish merges the splits and leaves the ticket at zero
   int base;            // 128-aligned start of the low-term window (<= q_pos0)
   __nv_bfloat16* out;     // [n_q][nq * 128] when n_splits == 1 (hi part)
   __nv_bfloat16* out_lo;  // lo part, or null
@@ -97,8 +97,6 @@ struct TcAttnParams {
 // `base`; the query comes from p.q / p.q_lo
 cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, const CUtensorMap& Kl,
                                 const CUtensorMap& Vtl, const TcAttnParams& p, cudaStream_t st);
-cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
-                              __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 // Head-pair variant (same parameters and outputs; chunks_per_split counts 64-key chunks):
 // K / Kl maps with 64-row boxes, Vt / Vtl as above.  pair_heads = 1: two heads of one KV
 // head per CTA where the group is even; 0: one head per CTA.  Grid y =
@@ -107,11 +105,6 @@ cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, co
                                  const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
                                  const TcAttnParams& p, int pair_heads, cudaStream_t st);
 int attn2_head_groups(int nq, int group, int pair_heads);
-// the head-pair path's split merge (same inputs and outputs as launch_attn_merge, d = 128):
-// one warp per (row, head), n_splits <= 32
-cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
-                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
-
 // ---------------------------------------------------------------- SIMT kernels (any dtype)
 // T = float (fp32 model) or __nv_bfloat16; an activation for a bf16 GEMM is written as
 // hi + lo bf16 tensors (lo pointers may be null: single term).

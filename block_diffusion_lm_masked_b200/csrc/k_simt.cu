@@ -317,13 +317,16 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
 // each CTA streams only E / RT_G rows of the router matrix: CTA r adds the residual and
 // normalises its own RT_TOK / RT_G tokens, the normalised rows are shared through
 // distributed shared memory, every CTA computes its experts' logits for all RT_TOK
-// tokens (one expert per warp, eight float4 loads per lane in flight), and CTA r runs
+// tokens (four experts per warp at once, each token row read from shared memory once per
+// four experts, eight float4 weight loads per lane in flight), and CTA r runs
 // the top-k of its own tokens over the logits of all CTAs.  Each logit is one lane-
 // strided fp32 dot product followed by a warp sum, as in a single-CTA version.
 constexpr int RT_G = 4;
 constexpr int RT_TOK = 8;
 constexpr int RT_OWN = RT_TOK / RT_G;
-constexpr int RT_THREADS = 512;
+constexpr int RT_THREADS = 256;
+constexpr int RT_EB = 4;   // experts per warp at once
+constexpr int RT_PF = 2;   // float4 steps of the weights loaded ahead (RT_PF * RT_EB loads)
 template <typename T>
 __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
@@ -392,35 +395,44 @@ __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
   }
   __syncthreads();
   const float4* xs4 = reinterpret_cast<const float4*>(xs);
-  for (int j = warp; j < Eg; j += NW) {
-    const float4* w4 = reinterpret_cast<const float4*>(wr + (size_t)(rank * Eg + j) * H);
-    float acc[RT_TOK] = {};
-    for (int i0 = lane; i0 < H4; i0 += 32 * 8) {
-      float4 u[8];
+  // RT_EB experts per warp at once: each token row read from shared memory serves all of
+  // them (shared-memory reads, not FMAs, bound a one-expert-per-warp loop)
+  for (int j0 = warp * RT_EB; j0 < Eg; j0 += NW * RT_EB) {
+    const float4* w4[RT_EB];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+    for (int b = 0; b < RT_EB; ++b) w4[b] = reinterpret_cast<const float4*>(wr + (size_t)(rank * Eg + min(j0 + b, Eg - 1)) * H);
+    float acc[RT_EB][RT_TOK] = {};
+    for (int i0 = lane; i0 < H4; i0 += 32 * RT_PF) {
+      float4 u[RT_PF][RT_EB];
+#pragma unroll
+      for (int q = 0; q < RT_PF; ++q) {
         const int i = i0 + 32 * q;
-        u[q] = i < H4 ? w4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int b = 0; b < RT_EB; ++b) u[q][b] = i < H4 ? w4[b][i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < RT_PF; ++q) {
         const int i = i0 + 32 * q;
         if (i < H4) {
 #pragma unroll
           for (int a = 0; a < RT_TOK; ++a) {
             if (a < nt) {
               const float4 v = xs4[a * H4 + i];
-              acc[a] = fmaf(u[q].x, v.x, fmaf(u[q].y, v.y, fmaf(u[q].z, v.z, fmaf(u[q].w, v.w, acc[a]))));
+#pragma unroll
+              for (int b = 0; b < RT_EB; ++b)
+                acc[b][a] = fmaf(u[q][b].x, v.x, fmaf(u[q][b].y, v.y, fmaf(u[q][b].z, v.z, fmaf(u[q][b].w, v.w, acc[b][a]))));
             }
           }
         }
       }
     }
 #pragma unroll
-    for (int a = 0; a < RT_TOK; ++a) {
-      const float r = warp_sum(acc[a]);
-      if (lane == 0) lg[a * Eg + j] = r;
-    }
+    for (int b = 0; b < RT_EB; ++b)
+#pragma unroll
+      for (int a = 0; a < RT_TOK; ++a) {
+        const float r = warp_sum(acc[b][a]);
+        if (lane == 0 && j0 + b < Eg) lg[a * Eg + j0 + b] = r;
+      }
   }
   cl.sync();  // every CTA's logits are in place
   // top-k: warp w < no selects for owned token w; lane takes experts lane + 32 i

@@ -33,6 +33,8 @@
 // in, and writes P once PV(j - 1) has read the previous P.  Hand-offs are mbarriers.
 #include <math.h>
 
+#include "attn_merge.cuh"
+#include "attn_softmax.cuh"
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -51,14 +53,6 @@ constexpr int AT_SM_WARPS = 8;
 constexpr int AT_MMA_WARP = AT_SM_WARPS;
 constexpr int AT_LOAD_WARP = AT_SM_WARPS + 1;
 constexpr int AT_THREADS = 32 * (AT_LOAD_WARP + 1);
-
-// 2^x by the hardware's approximate exponential (relative error about 2^-22; results
-// below 2^-126 flush to zero, far below what the bf16 hi + lo probabilities resolve)
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // A operand from TMEM (Q or P), B from shared memory (K or V^T), fp32 accumulate in TMEM
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -87,57 +81,6 @@ struct AtSlotPlan {
     }
   }
 };
-
-// Split-KV merge by the last split of a (query tile, head) to finish: every split has
-// written its partial output and log2-sum-exp; the split whose ticket comes last combines
-// them (weights 2^(lse_s - max)) into the bf16 hi + lo output and resets the ticket for
-// the next launch.  Block-wide; called by every CTA of the grid as it leaves.
-__device__ __forceinline__ void merge_splits_if_last(const TcAttnParams& p, int qt, int h) {
-  __shared__ int last_s;
-  __threadfence();  // this CTA's partials are visible device-wide before its ticket
-  __syncthreads();
-  if (threadIdx.x == 0) last_s = atomicAdd(&p.merge_cnt[qt * p.nq + h], 1) == p.n_splits - 1;
-  __syncthreads();
-  if (!last_s) return;
-  __threadfence();
-  const int q_row0 = qt * AT_BQ;
-  const int rows = min(AT_BQ, p.n_q - q_row0);
-  for (int idx = threadIdx.x; idx < rows * (AT_D / 4); idx += blockDim.x) {
-    const int row = q_row0 + idx / (AT_D / 4), c4 = idx % (AT_D / 4);
-    float mx = -INFINITY;
-    for (int sp = 0; sp < p.n_splits; ++sp) mx = fmaxf(mx, __ldcg(&p.part_lse[((size_t)sp * p.nq + h) * p.n_q + row]));
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.0f;
-    if (mx != -INFINITY) {
-      for (int sp = 0; sp < p.n_splits; ++sp) {
-        const float lse = __ldcg(&p.part_lse[((size_t)sp * p.nq + h) * p.n_q + row]);
-        if (lse == -INFINITY) continue;
-        const float w = exp2f(lse - mx);
-        const float4 o =
-            __ldcg(reinterpret_cast<const float4*>(p.part_o + (((size_t)sp * p.nq + h) * p.n_q + row) * AT_D) + c4);
-        num.x += w * o.x;
-        num.y += w * o.y;
-        num.z += w * o.z;
-        num.w += w * o.w;
-        den += w;
-      }
-    }
-    const float v[4] = {den > 0.f ? num.x / den : 0.f, den > 0.f ? num.y / den : 0.f, den > 0.f ? num.z / den : 0.f,
-                        den > 0.f ? num.w / den : 0.f};
-    uint32_t w[2], wl[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(v[2 * e] - __low2float(hi), v[2 * e + 1] - __high2float(hi));
-      w[e] = *reinterpret_cast<const uint32_t*>(&hi);
-      wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
-    }
-    const size_t o = (size_t)row * p.nq * AT_D + (size_t)h * AT_D + 4 * c4;
-    *reinterpret_cast<uint2*>(p.out + o) = make_uint2(w[0], w[1]);
-    if (p.out_lo) *reinterpret_cast<uint2*>(p.out_lo + o) = make_uint2(wl[0], wl[1]);
-  }
-  if (threadIdx.x == 0) p.merge_cnt[qt * p.nq + h] = 0;  // ready for the next launch
-}
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
@@ -179,7 +122,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (int i = 0; i < AT_D; ++i) po[i] = 0.0f;
       p.part_lse[((size_t)sp * p.nq + h) * p.n_q + qrow] = -INFINITY;
     }
-    if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h);
+    if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h, 1);
     return;
   }
 
@@ -524,32 +467,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
-  if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h);
-}
-
-__global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_splits,
-                                  int nq, int n_q, int d, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
-  griddep_sync();
-  const int qrow = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
-  float mx = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, part_lse[((size_t)s * nq + h) * n_q + qrow]);
-  for (int dd = t; dd < d; dd += blockDim.x) {
-    float num = 0.0f, den = 0.0f;
-    if (mx != -INFINITY) {
-      for (int s = 0; s < n_splits; ++s) {
-        const float lse = part_lse[((size_t)s * nq + h) * n_q + qrow];
-        if (lse == -INFINITY) continue;
-        const float w = exp2f(lse - mx);
-        num += w * part_o[(((size_t)s * nq + h) * n_q + qrow) * d + dd];
-        den += w;
-      }
-    }
-    const float v = den > 0.0f ? num / den : 0.0f;
-    const size_t o = (size_t)qrow * nq * d + (size_t)h * d + dd;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    out[o] = hi;
-    if (out_lo) out_lo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
-  }
+  if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h, 1);
 }
 
 cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, const CUtensorMap& Kl,
@@ -558,12 +476,6 @@ cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, con
   if (e != cudaSuccess) return e;
   dim3 grid((p.n_q + AT_BQ - 1) / AT_BQ, p.nq, p.n_splits);
   return launch_k(tc_attn_kernel, grid, dim3(AT_THREADS), AT_SMEM, st, K, Vt, Kl, Vtl, p);
-}
-
-cudaError_t launch_attn_merge(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q, int d,
-                              __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
-  return launch_k(attn_merge_kernel, dim3(n_q, nq), dim3(128), 0, st, part_o, part_lse, n_splits, nq, n_q, d, out,
-                  out_lo);
 }
 
 cudaError_t set_wait_limit_attn(uint64_t ns) { return set_wait_limit_this_file(ns); }

@@ -25,6 +25,8 @@
 // plain order deadlocks in that case.
 #include <math.h>
 
+#include "attn_merge.cuh"
+#include "attn_softmax.cuh"
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         for (int i = 0; i < A2_D; ++i) po[i] = 0.0f;
         p.part_lse[((size_t)sp * p.nq + h0 + hl) * p.n_q + qrow] = -INFINITY;
       }
+    if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h0, nh);
     return;
   }
 
@@ -285,7 +288,9 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     const int my_pos = p.q_pos0 + my_row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int key_lim = p.causal ? min(p.n_keys, my_pos + 1) : p.n_keys;
-    float m_used = -INFINITY, l = 0.0f;
+    float m_used = -INFINITY;
+    uint64_t l2 = f2_pack(0.0f, 0.0f);  // the row sum as two partial sums (even and odd keys)
+    const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int j = 0; j < nck && ok; ++j) {
       const int b = j & 1;
@@ -296,24 +301,27 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t spa = tmem + a2_sp(hl, b) + lane_off;
-      float s[A2_W];
+      // the chunk's raw scores, all four loads in flight before the one wait
+      uint32_t r[A2_W / 16][16];
 #pragma unroll
-      for (int c = 0; c < A2_W / 16; ++c) {
-        uint32_t r[16];
-        tmem_ld16(spa + c * 16, r);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[i]) * p.scale_log2;
-      }
+      for (int c = 0; c < A2_W / 16; ++c) tmem_ld16(spa + c * 16, r[c]);
+      tc_wait_ld();
       const int key0 = (c_begin + j) * A2_W;
-      float cmax = -INFINITY;
+      // keys at or past the row's limit (only in the chunk that holds the limit)
+      if (__any_sync(0xffffffffu, key0 + A2_W > key_lim)) {
 #pragma unroll
-      for (int i = 0; i < A2_W; ++i) {
-        if (key0 + i >= key_lim) s[i] = -INFINITY;
-        cmax = fmaxf(cmax, s[i]);
+        for (int i = 0; i < A2_W; ++i)
+          if (key0 + i >= key_lim) r[i / 16][i % 16] = __float_as_uint(-INFINITY);
       }
+      // the row maximum of the raw scores, then scaled (the scale is positive and
+      // rounding monotone, so this is the maximum of the scaled scores)
+      float cm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < A2_W; i += 2)
+        cm = max3f(cm, __uint_as_float(r[i / 16][i % 16]), __uint_as_float(r[i / 16][i % 16 + 1]));
+      const float cmax = cm * p.scale_log2;
       const bool upd = cmax > m_used + 8.0f;
-      const float alpha = upd ? exp2f(m_used - cmax) : 1.0f;  // 0 while nothing was visible yet
+      const float alpha = upd ? ex2_approx(m_used - cmax) : 1.0f;  // 0 while nothing was visible yet
       // tcgen05.ld/st are warp-collective: the warp rescales its rows of O if any row must,
       // once the previous chunk's PV is complete (O stable; PV(j) waits for this P)
       if (__any_sync(0xffffffffu, upd && j > 0)) {
@@ -324,33 +332,41 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         const uint32_t oa = tmem + a2_o(hl) + lane_off;
 #pragma unroll
         for (int c = 0; c < A2_D / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(oa + c * 16, r);
+          uint32_t o[16];
+          tmem_ld16(oa + c * 16, o);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st16(oa + c * 16, r);
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16(oa + c * 16, o);
         }
       }
       if (upd) {
-        l *= alpha;
+        l2 = f2_mul(l2, f2_pack(alpha, alpha));
         m_used = cmax;
       }
-      // P = exp2(s - m_used) as packed bf16 pairs over this row's S: hi in columns 0..31,
-      // lo in 32..63 (S was read into registers above)
+      // P = 2^(s * scale - m_used) (one rounding), packed bf16 pairs over this row's S: hi
+      // in columns 0..31, lo in 32..63.  A row that has seen no key has m_used = -inf and
+      // only -inf scores: its offset is taken as 0, so that every P is 2^-inf = 0.
+      const float neg_m = (m_used == -INFINITY) ? 0.0f : -m_used;
+      const uint64_t nm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // 32 keys -> 16 packed columns per store
         uint32_t wh[16], wl[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int i0 = c * 32 + 2 * e;
-          const float p0 = (s[i0] == -INFINITY) ? 0.0f : exp2f(s[i0] - m_used);
-          const float p1 = (s[i0 + 1] == -INFINITY) ? 0.0f : exp2f(s[i0 + 1] - m_used);
-          l += p0 + p1;
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-          const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
-          wh[e] = *reinterpret_cast<const uint32_t*>(&hi);
-          wl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+          const uint64_t t = f2_fma(f2_pack(__uint_as_float(r[i0 / 16][i0 % 16]),
+                                            __uint_as_float(r[i0 / 16][i0 % 16 + 1])), scale2, nm2);
+          float t0, t1;
+          f2_unpack(t, t0, t1);
+          const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+          const uint64_t pp = f2_pack(p0, p1);
+          l2 = f2_add(l2, pp);
+          const uint32_t hi = bf16x2_pack(p0, p1);
+          float lo0, lo1;
+          f2_unpack(f2_sub(pp, bf16x2_widen(hi)), lo0, lo1);
+          wh[e] = hi;
+          wl[e] = bf16x2_pack(lo0, lo1);
         }
         tmem_st16(spa + c * 16, wh);
         tmem_st16(spa + 32 + c * 16, wl);
@@ -363,6 +379,9 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl][(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s,
                                              p.err, DG_DEVERR_TIMEOUT_ATTN));
+    float l0, l1;
+    f2_unpack(l2, l0, l1);
+    const float l = l0 + l1;
     if (ok) {
       tc_fence_after();
       const bool valid = my_row < p.n_q;
@@ -430,60 +449,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == A2_MMA_WARP) tmem_dealloc(tmem, 512);
-}
-
-// Split-KV merge, one warp per (query row, head): lane s < n_splits reads split s's
-// log2-sum-exp, the warp takes their maximum and the weights exp2(lse_s - max) by
-// shuffles, and each lane merges four of the 128 output columns over the splits (the
-// splits' loads independent of one another), then writes the bf16 hi and lo parts.
-// Rows with no visible key (every lse -inf) are written as zeros.
-__global__ void __launch_bounds__(256) attn_merge2_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_lse, int n_splits, int nq,
-                                                          int n_q, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
-  griddep_sync();
-  const int lane = threadIdx.x & 31;
-  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (w >= nq * n_q) return;
-  const int h = w / n_q, row = w % n_q;
-  const float lse = lane < n_splits ? part_lse[((size_t)lane * nq + h) * n_q + row] : -INFINITY;
-  float mx = lse;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const float wt = (lse == -INFINITY) ? 0.0f : exp2f(lse - mx);
-  float den = wt;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sp = 0; sp < n_splits; ++sp) {
-    const float ws = __shfl_sync(0xffffffffu, wt, sp);
-    if (ws == 0.0f) continue;  // uniform across the warp
-    const float4 v = reinterpret_cast<const float4*>(part_o + (((size_t)sp * nq + h) * n_q + row) * A2_D)[lane];
-    acc.x += ws * v.x;
-    acc.y += ws * v.y;
-    acc.z += ws * v.z;
-    acc.w += ws * v.w;
-  }
-  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  const float a[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-  uint32_t hw[2], lw[2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(a[2 * e], a[2 * e + 1]);
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(a[2 * e] - __low2float(hi), a[2 * e + 1] - __high2float(hi));
-    hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
-    lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
-  }
-  const size_t o = (size_t)row * nq * A2_D + (size_t)h * A2_D + 4 * lane;
-  *reinterpret_cast<uint2*>(out + o) = make_uint2(hw[0], hw[1]);
-  if (out_lo) *reinterpret_cast<uint2*>(out_lo + o) = make_uint2(lw[0], lw[1]);
-}
-
-cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
-                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
-  if (n_splits < 1 || n_splits > 32) return cudaErrorInvalidValue;
-  const int warps = nq * n_q;
-  return launch_k(attn_merge2_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, part_o, part_lse, n_splits, nq, n_q,
-                  out, out_lo);
+  if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h0, nh);
 }
 
 int attn2_head_groups(int nq, int group, int pair_heads) { return (pair_heads && group % 2 == 0) ? nq / 2 : nq; }

@@ -112,6 +112,32 @@ def lazy_update(rmax, m_used, l, warp_rescale):
     return m_used, l
 
 
+def softmax_chunk_raw(raw, key0, key_lim):
+    """The head-pair kernel's chunk: raw scores (fp32), -inf at or past each row's key
+    limit; the row maximum is taken on the raw scores and scaled afterwards."""
+    s = raw.view(np.float32).copy()
+    keys = key0 + np.arange(s.shape[1])
+    return np.where(keys[None, :] >= key_lim[:, None], NEG, s).astype(np.float32)
+
+
+def p_words_fma(s_raw, scale, m_used, l_pair):
+    """P = 2^(fma(s, scale, -m)) (one rounding; offset 0 where the row has seen no key),
+    packed hi / lo, and the row sum as two fp32 partial sums (even and odd keys)."""
+    neg_m = np.where(np.isneginf(m_used), np.float32(0), -m_used).astype(np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        t = (s_raw.astype(np.float64) * np.float64(scale) + neg_m[:, None]).astype(np.float32)
+        p = np.exp2(t.astype(np.float64)).astype(np.float32)
+    le, lo_ = l_pair
+    for e in range(0, p.shape[1], 2):
+        le = (le + p[:, e]).astype(np.float32)
+        lo_ = (lo_ + p[:, e + 1]).astype(np.float32)
+    hi = T.bf16_value(T.bf16_bits(p))
+    lo = (p - hi).astype(np.float32)
+    wh = T.pack_bf16x2(p[:, 0::2], p[:, 1::2])
+    wl = T.pack_bf16x2(lo[:, 0::2], lo[:, 1::2])
+    return wh, wl, (le, lo_)
+
+
 def epilogue(tm, o_cols, l, m_used, rows, out, out_lo, part_o, part_lse, sp, h, n_splits, nq, n_q, col0=0, ncols=128):
     inv = np.where(l > 0, (np.float32(1.0) / np.where(l > 0, l, 1)).astype(np.float32), np.float32(0)).astype(np.float32)
     o = (tm.f32(o_cols, ncols) * inv[:, None]).astype(np.float32)
@@ -143,35 +169,6 @@ def merge(part_o, part_lse, n_splits):
     hi = T.bf16_value(T.bf16_bits(v))
     lo = T.bf16_value(T.bf16_bits((v - hi).astype(np.float32)))
     nq, n_q = v.shape[0], v.shape[1]
-    return (hi + lo).transpose(1, 0, 2).reshape(n_q, nq * D)
-
-
-def merge2(part_o, part_lse, n_splits):
-    """attn_merge2_kernel: per (row, head) warp, lane s holds split s's lse; maximum and the
-    weight sum by butterflies, the columns accumulated over the splits in order, times the
-    reciprocal of the sum."""
-    nq, n_q = part_lse.shape[1], part_lse.shape[2]
-    lanes = np.full((32, nq, n_q), NEG, np.float32)
-    lanes[:n_splits] = part_lse[:n_splits]
-    mx = lanes.copy()
-    o = 16
-    while o:
-        mx = np.maximum(mx, mx[np.arange(32) ^ o])
-        o >>= 1
-    with np.errstate(invalid="ignore"):
-        wt = np.where(np.isneginf(lanes), np.float32(0), np.exp2((lanes - mx).astype(np.float32))).astype(np.float32)
-    den = wt.copy()
-    o = 16
-    while o:
-        den = (den + den[np.arange(32) ^ o]).astype(np.float32)
-        o >>= 1
-    acc = np.zeros(part_o.shape[1:], np.float32)
-    for sp in range(n_splits):
-        acc = (acc + wt[sp][..., None] * part_o[sp]).astype(np.float32)
-    inv = np.where(den[0] > 0, (np.float32(1) / np.where(den[0] > 0, den[0], 1)).astype(np.float32), np.float32(0))
-    v = (acc * inv[..., None]).astype(np.float32)
-    hi = T.bf16_value(T.bf16_bits(v))
-    lo = T.bf16_value(T.bf16_bits((v - hi).astype(np.float32)))
     return (hi + lo).transpose(1, 0, 2).reshape(n_q, nq * D)
 
 
@@ -474,22 +471,25 @@ def run_pair(c, bug=None, force_pair=None):
                     pending.append(k_)
 
                 m_used = [np.full(128, NEG, np.float32) for _ in range(nh)]
-                lsum = [np.zeros(128, np.float32) for _ in range(nh)]
+                lpair = [(np.zeros(128, np.float32), np.zeros(128, np.float32)) for _ in range(nh)]
                 key_lim = np.array([c["key_lim"][r] if r < n_q else n_keys for r in rows])
 
                 def softmax(hl, j):
                     b = j & 1
                     spa = a2_sp(hl, b)
                     raw = np.concatenate([tm.t[:, spa + cc * 16:spa + cc * 16 + 16] for cc in range(4)], axis=1)
-                    s = softmax_chunk(raw, (c_begin + j) * W, key_lim, scale, None, None)
+                    s = softmax_chunk_raw(raw, (c_begin + j) * W, key_lim)
 
                     def rescale(any_w, alpha):
                         if j > 0 and any_w.any():
                             flush()                           # waits for PV(j - 1)
                             blk = tm.f32(a2_o(hl), D)
                             blk[any_w] = (blk[any_w] * alpha[any_w, None]).astype(np.float32)
-                    m_used[hl], lsum[hl] = lazy_update(s.max(axis=1), m_used[hl], lsum[hl], rescale)
-                    wh, wl, lsum[hl] = p_words(s, m_used[hl], lsum[hl])
+                    le, lo_ = lpair[hl]
+                    m_old = m_used[hl]
+                    m_used[hl], le = lazy_update((s.max(axis=1) * scale).astype(np.float32), m_old, le, rescale)
+                    _, lo_ = lazy_update((s.max(axis=1) * scale).astype(np.float32), m_old, lo_, lambda a, b: None)
+                    wh, wl, lpair[hl] = p_words_fma(s, scale, m_used[hl], (le, lo_))
                     tm.t[:, spa:spa + 32] = wh                # P over this row's S: hi, then lo
                     tm.t[:, spa + p_lo:spa + p_lo + 32] = wl
 
@@ -513,9 +513,10 @@ def run_pair(c, bug=None, force_pair=None):
                 pv_chunk(nck - 1)
                 flush()
                 for hl in range(nh):
-                    epilogue(tm, a2_o(hl), lsum[hl], m_used[hl], rows, out, out_lo, part_o, part_lse, sp, h0 + hl,
+                    lsum = (lpair[hl][0] + lpair[hl][1]).astype(np.float32)
+                    epilogue(tm, a2_o(hl), lsum, m_used[hl], rows, out, out_lo, part_o, part_lse, sp, h0 + hl,
                              n_splits, nq, n_q)
-    return (out + out_lo) if n_splits == 1 else merge2(part_o, part_lse, n_splits)
+    return (out + out_lo) if n_splits == 1 else merge(part_o, part_lse, n_splits)
 
 
 CASES = [
