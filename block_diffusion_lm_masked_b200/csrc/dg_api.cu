@@ -665,7 +665,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.has_lo = 1;
   p.q = ws.at<bf16>(ws.L.q);
   p.q_lo = ws.at<bf16>(ws.L.q_lo);
-  p.merge_cnt = ws.at<int>(ws.L.attn_cnt);  // the last split of each tile merges (zeroed by the RoPE kernel)
+  p.merge_cnt = nullptr;  // merged by attn_merge2_kernel
   p.base = base;
   p.out = ws.at<bf16>(ws.L.o);
   p.out_lo = ws.at<bf16>(ws.L.o_lo);
@@ -673,6 +673,10 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   p.part_lse = ws.at<float>(ws.L.part_lse);
   p.err = ws.err();
   LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, pair_heads, st));
+  if (p.n_splits > 1)
+    LAUNCH(DG_K_ATTN_MERGE, st,
+           dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, ws.at<bf16>(ws.L.o),
+                                  ws.at<bf16>(ws.L.o_lo), st));
   return DG_OK;
 }
 

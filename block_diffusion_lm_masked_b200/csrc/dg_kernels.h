@@ -105,6 +105,10 @@ cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, co
                                  const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
                                  const TcAttnParams& p, int pair_heads, cudaStream_t st);
 int attn2_head_groups(int nq, int group, int pair_heads);
+// the head-pair path's split merge, one warp per (row, head) over the GPU, d = 128,
+// n_splits <= 32
+cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
+                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 // ---------------------------------------------------------------- SIMT kernels (any dtype)
 // T = float (fp32 model) or __nv_bfloat16; an activation for a bf16 GEMM is written as
 // hi + lo bf16 tensors (lo pointers may be null: single term).

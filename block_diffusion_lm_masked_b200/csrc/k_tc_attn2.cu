@@ -25,7 +25,6 @@
 // plain order deadlocks in that case.
 #include <math.h>
 
-#include "attn_merge.cuh"
 #include "attn_softmax.cuh"
 #include "dg_common.cuh"
 #include "dg_kernels.h"
@@ -118,7 +117,6 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         for (int i = 0; i < A2_D; ++i) po[i] = 0.0f;
         p.part_lse[((size_t)sp * p.nq + h0 + hl) * p.n_q + qrow] = -INFINITY;
       }
-    if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h0, nh);
     return;
   }
 
@@ -449,7 +447,63 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == A2_MMA_WARP) tmem_dealloc(tmem, 512);
-  if (p.n_splits > 1 && p.merge_cnt) merge_splits_if_last(p, qt, h0, nh);
+}
+
+// Split-KV merge in a kernel of its own (the head-pair kernel's splits write partials):
+// one warp per (query row, head), spread over the whole GPU -- a merge by the last split
+// of each tile would leave one CTA to read every split's partial rows (about 1 MB at the
+// large model's nine splits), a tail of tens of microseconds.  Lane s < n_splits reads split s's
+// log2-sum-exp, the warp takes their maximum and the weights exp2(lse_s - max) by
+// shuffles, and each lane merges four of the 128 output columns over the splits (the
+// splits' loads independent of one another), then writes the bf16 hi and lo parts.
+// Rows with no visible key (every lse -inf) are written as zeros.
+__global__ void __launch_bounds__(256) attn_merge2_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int n_splits, int nq,
+                                                          int n_q, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
+  griddep_sync();
+  const int lane = threadIdx.x & 31;
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (w >= nq * n_q) return;
+  const int h = w / n_q, row = w % n_q;
+  const float lse = lane < n_splits ? part_lse[((size_t)lane * nq + h) * n_q + row] : -INFINITY;
+  float mx = lse;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float wt = (lse == -INFINITY) ? 0.0f : exp2f(lse - mx);
+  float den = wt;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp = 0; sp < n_splits; ++sp) {
+    const float ws = __shfl_sync(0xffffffffu, wt, sp);
+    if (ws == 0.0f) continue;  // uniform across the warp
+    const float4 v = reinterpret_cast<const float4*>(part_o + (((size_t)sp * nq + h) * n_q + row) * A2_D)[lane];
+    acc.x += ws * v.x;
+    acc.y += ws * v.y;
+    acc.z += ws * v.z;
+    acc.w += ws * v.w;
+  }
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  const float a[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  uint32_t hw[2], lw[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(a[2 * e], a[2 * e + 1]);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(a[2 * e] - __low2float(hi), a[2 * e + 1] - __high2float(hi));
+    hw[e] = *reinterpret_cast<const uint32_t*>(&hi);
+    lw[e] = *reinterpret_cast<const uint32_t*>(&lo);
+  }
+  const size_t o = (size_t)row * nq * A2_D + (size_t)h * A2_D + 4 * lane;
+  *reinterpret_cast<uint2*>(out + o) = make_uint2(hw[0], hw[1]);
+  if (out_lo) *reinterpret_cast<uint2*>(out_lo + o) = make_uint2(lw[0], lw[1]);
+}
+
+cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
+                               __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
+  if (n_splits < 1 || n_splits > 32) return cudaErrorInvalidValue;
+  const int warps = nq * n_q;
+  return launch_k(attn_merge2_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, part_o, part_lse, n_splits, nq, n_q,
+                  out, out_lo);
 }
 
 int attn2_head_groups(int nq, int group, int pair_heads) { return (pair_heads && group % 2 == 0) ? nq / 2 : nq; }

@@ -22,6 +22,12 @@
 // that run at the same time then read different k-blocks of the token operand, which
 // all of them share, instead of hammering the same L2 lines in lockstep.
 //
+// The shared memory holds a ring of variable-size k-block buffers (KbRing): a k-block
+// takes its weight boxes (16 KB each) and its token boxes of the tile's own padded row
+// count, contiguously, so that an expert tile of 16 token rows takes 36 KB instead of a
+// stage sized for the largest tile (64 KB): more weight bytes are in flight per SM when
+// the tiles are small.  Up to 16 k-blocks are in flight, one pair of barriers each.
+//
 #include "dg_common.cuh"
 #include "dg_kernels.h"
 
@@ -31,8 +37,22 @@ constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
 constexpr int TC_B_BOX = 16;      // token rows per small TMA box
 constexpr int TC_B_BOX_BIG = 64;  // token rows per large TMA box
-constexpr int TC_MAX_STAGES = 16;
+constexpr int TC_MAX_STAGES = 16;  // k-blocks in flight at most (barrier pairs)
 constexpr int TC_THREADS = 192;
+
+// The k-block buffers' offsets in the ring, in the order both the producer and the MMA
+// warp walk the k-blocks: a buffer starts where the previous one ended, or at 0 when it
+// would run past the end.  Sizes are multiples of 2 KB, so every buffer (and each box
+// in it) starts on a 1024-byte swizzle atom.
+struct KbRing {
+  uint32_t cap, head;
+  __device__ explicit KbRing(uint32_t c) : cap(c), head(0) {}
+  __device__ uint32_t take(uint32_t bytes) {
+    const uint32_t off = head + bytes > cap ? 0u : head;
+    head = off + bytes;
+    return off;
+  }
+};
 
 struct TileInfo {
   int g, row0, rows, split, m;
@@ -117,11 +137,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int terms = p.two_terms ? 2 : 1;
   const int n_a = (p.dual_a || p.m_pair) ? 2 : 1;
-  const uint32_t a_bytes = TC_BM * TC_BK * 2;           // one weight tile per k-block
-  const uint32_t bmax_bytes = (uint32_t)p.n_max * 128;  // one token term per k-block, n_max rows
-  const uint32_t stage_bytes = n_a * a_bytes + terms * bmax_bytes;
-  int stages = p.smem_budget / (int)stage_bytes;
-  if (stages > TC_MAX_STAGES) stages = TC_MAX_STAGES;
+  const uint32_t a_bytes = TC_BM * TC_BK * 2;  // one weight tile per k-block
+  // a k-block buffer of a tile with n_pad token rows: weight boxes, then each token term
+  auto kb_bytes = [&](int n_pad) { return n_a * a_bytes + (uint32_t)(terms * n_pad * 128); };
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int acc_cols = p.n_max * n_a;  // one accumulator buffer
   const int nbuf = 2 * acc_cols <= 512 ? 2 : 1;
@@ -132,7 +150,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 1) tmem_alloc(&tmem_base_s, tmem_cols);
   if (tid == 0) {
-    for (int s = 0; s < stages; ++s) {
+    for (int s = 0; s < TC_MAX_STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -165,20 +183,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prefetch_tmap(&tmB2b);
       }
       int it = 0, t;
+      int released = 0;  // k-blocks whose buffers the MMAs have released (in order)
+      uint32_t q_off[TC_MAX_STAGES], q_len[TC_MAX_STAGES];  // buffers of k-blocks released .. it - 1
       bool ok = true;
+      KbRing ring((uint32_t)p.smem_budget);
       TileWalk walk(p, n_tiles);
       while (ok && walk.next(t)) {
         const TileInfo ti = decode_tile(p, t);
         const int n_pad = (ti.rows + 15) & ~15;
-        const uint32_t tx = n_a * a_bytes + terms * (uint32_t)n_pad * 128;
+        const uint32_t tx = kb_bytes(n_pad);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % stages;
-          if (!mbar_wait(&empty_bar[s], ((uint32_t)(it / stages) & 1u) ^ 1u, &abort_s, p.err,
-                         DG_DEVERR_TIMEOUT_EMPTY)) {
-            ok = false;
-            break;
+          const int s = it % TC_MAX_STAGES;
+          const uint32_t off = ring.take(tx);
+          // wait for the oldest k-blocks until none in flight overlaps this buffer and
+          // fewer than TC_MAX_STAGES are in flight (buffers are released in order)
+          while (released < it) {
+            bool clash = it - released >= TC_MAX_STAGES;
+            for (int q = released; q < it && !clash; ++q)
+              clash = off < q_off[q % TC_MAX_STAGES] + q_len[q % TC_MAX_STAGES] && q_off[q % TC_MAX_STAGES] < off + tx;
+            if (!clash) break;
+            if (!mbar_wait(&empty_bar[released % TC_MAX_STAGES], (uint32_t)(released / TC_MAX_STAGES) & 1u, &abort_s,
+                           p.err, DG_DEVERR_TIMEOUT_EMPTY)) {
+              ok = false;
+              break;
+            }
+            ++released;
           }
-          uint8_t* sa = smem + (size_t)s * stage_bytes;
+          if (!ok) break;
+          q_off[s] = off;
+          q_len[s] = tx;
+          uint8_t* sa = smem + off;
           uint8_t* sb = sa + n_a * a_bytes;
           const int kx = (ti.split * nkb + (kb + t) % nkb) * TC_BK;
           mbar_arrive_expect_tx(&full_bar[s], tx);
@@ -189,11 +223,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           int r = 0;
           for (; r + TC_B_BOX_BIG <= n_pad; r += TC_B_BOX_BIG) {
             tma_load_2d(sb + r * 128, &tmBb, kx, ti.row0 + r, &full_bar[s]);
-            if (terms == 2) tma_load_2d(sb + bmax_bytes + r * 128, &tmB2b, kx, ti.row0 + r, &full_bar[s]);
+            if (terms == 2) tma_load_2d(sb + n_pad * 128 + r * 128, &tmB2b, kx, ti.row0 + r, &full_bar[s]);
           }
           for (; r < n_pad; r += TC_B_BOX) {
             tma_load_2d(sb + r * 128, &tmB, kx, ti.row0 + r, &full_bar[s]);
-            if (terms == 2) tma_load_2d(sb + bmax_bytes + r * 128, &tmB2, kx, ti.row0 + r, &full_bar[s]);
+            if (terms == 2) tma_load_2d(sb + n_pad * 128 + r * 128, &tmB2, kx, ti.row0 + r, &full_bar[s]);
           }
           n_issued_s = it + 1;
         }
@@ -204,6 +238,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // ---------------- MMA issuer
       int it = 0, j = 0, t;
       bool ok = true;
+      KbRing ring((uint32_t)p.smem_budget);
       TileWalk walk(p, n_tiles);
       for (; ok && walk.next(t); ++j) {
         const TileInfo ti = decode_tile(p, t);
@@ -215,21 +250,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
         const uint32_t d1 = d0 + (uint32_t)p.n_max;
         const uint32_t idesc = idesc_bf16_f32(TC_BM, n_pad);
+        const uint32_t tx = kb_bytes(n_pad);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % stages;
-          if (!mbar_wait(&full_bar[s], (uint32_t)(it / stages) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
+          const int s = it % TC_MAX_STAGES;
+          const uint32_t off = ring.take(tx);
+          if (!mbar_wait(&full_bar[s], (uint32_t)(it / TC_MAX_STAGES) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+          const uint32_t sa = smem_u32(smem + off);
           const uint32_t sb = sa + n_a * a_bytes;
 #pragma unroll
           for (int kk = 0; kk < TC_BK / 16; ++kk) {
             const uint32_t acc = (kb != 0 || kk != 0) ? 1u : 0u;
             const uint64_t ad = sw128_kmajor_desc(sa + kk * 32);
             const uint64_t bd = sw128_kmajor_desc(sb + kk * 32);
-            const uint64_t bd2 = sw128_kmajor_desc(sb + bmax_bytes + kk * 32);
+            const uint64_t bd2 = sw128_kmajor_desc(sb + (uint32_t)n_pad * 128 + kk * 32);
             tc_mma(d0, ad, bd, idesc, acc);
             if (terms == 2) tc_mma(d0, ad, bd2, idesc, 1u);
             if (n_a == 2) {
@@ -300,7 +337,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (abort_s && tid == 0) {
     // wind down: let issued loads land before the smem goes away
     for (int i = n_consumed_s; i < n_issued_s; ++i)
-      mbar_wait_drain(&full_bar[i % stages], (uint32_t)(i / stages) & 1u);
+      mbar_wait_drain(&full_bar[i % TC_MAX_STAGES], (uint32_t)(i / TC_MAX_STAGES) & 1u);
   }
   if (tid == 32) mbar_wait_drain(&drain_bar, 0);  // every issued MMA has landed
   tc_fence_before();
@@ -368,8 +405,8 @@ cudaError_t launch_tc_gemm(int epi, const CUtensorMap& A, const CUtensorMap& A2,
       p.n_max > 256 || (p.n_max % 16) != 0 || p.m_tiles < 1)
     return cudaErrorInvalidValue;
   const int n_a = (p.dual_a || p.m_pair) ? 2 : 1;
-  const int stage = n_a * TC_BM * TC_BK * 2 + (p.two_terms ? 2 : 1) * p.n_max * 128;
-  if (p.smem_budget < stage || p.n_max * n_a > 512 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0) ||
+  const int stage = n_a * TC_BM * TC_BK * 2 + (p.two_terms ? 2 : 1) * p.n_max * 128;  // the largest k-block
+  if (p.smem_budget < stage || p.smem_budget % 2048 != 0 || p.n_max * n_a > 512 || (epi == EPI_SWIGLU_BF16) != (p.dual_a != 0) ||
       (p.m_pair && (p.dual_a || epi != EPI_STORE_F32)))
     return cudaErrorInvalidValue;
   const int smem = p.smem_budget + 1024;

@@ -172,6 +172,35 @@ def merge(part_o, part_lse, n_splits):
     return (hi + lo).transpose(1, 0, 2).reshape(n_q, nq * D)
 
 
+def merge2(part_o, part_lse, n_splits):
+    """attn_merge2_kernel: per (row, head) warp, lane s holds split s's lse; maximum and the
+    weight sum by butterflies, the columns accumulated over the splits in order, times the
+    reciprocal of the sum."""
+    nq, n_q = part_lse.shape[1], part_lse.shape[2]
+    lanes = np.full((32, nq, n_q), NEG, np.float32)
+    lanes[:n_splits] = part_lse[:n_splits]
+    mx = lanes.copy()
+    o = 16
+    while o:
+        mx = np.maximum(mx, mx[np.arange(32) ^ o])
+        o >>= 1
+    with np.errstate(invalid="ignore"):
+        wt = np.where(np.isneginf(lanes), np.float32(0), np.exp2((lanes - mx).astype(np.float32))).astype(np.float32)
+    den = wt.copy()
+    o = 16
+    while o:
+        den = (den + den[np.arange(32) ^ o]).astype(np.float32)
+        o >>= 1
+    acc = np.zeros(part_o.shape[1:], np.float32)
+    for sp in range(n_splits):
+        acc = (acc + wt[sp][..., None] * part_o[sp]).astype(np.float32)
+    inv = np.where(den[0] > 0, (np.float32(1) / np.where(den[0] > 0, den[0], 1)).astype(np.float32), np.float32(0))
+    v = (acc * inv[..., None]).astype(np.float32)
+    hi = T.bf16_value(T.bf16_bits(v))
+    lo = T.bf16_value(T.bf16_bits((v - hi).astype(np.float32)))
+    return (hi + lo).transpose(1, 0, 2).reshape(n_q, nq * D)
+
+
 # ---------------------------------------------------------------- tc_attn_kernel
 def run_single(c, bug=None):
     """tc_attn_kernel: one head x 128 rows x 128-key chunks; the query tile in TMEM (hi at
@@ -516,7 +545,7 @@ def run_pair(c, bug=None, force_pair=None):
                     lsum = (lpair[hl][0] + lpair[hl][1]).astype(np.float32)
                     epilogue(tm, a2_o(hl), lsum, m_used[hl], rows, out, out_lo, part_o, part_lse, sp, h0 + hl,
                              n_splits, nq, n_q)
-    return (out + out_lo) if n_splits == 1 else merge(part_o, part_lse, n_splits)
+    return (out + out_lo) if n_splits == 1 else merge2(part_o, part_lse, n_splits)
 
 
 CASES = [

@@ -5,10 +5,12 @@ check for later changes to the kernel.
 Transcribed from the kernel source: the persistent tile walk (grouped: item-major;
 dense: token chunk, then split, then weight tile; dealt in serpentine rounds with the
 partial weight tiles last), the k-block rotation within a split,
-the stage layout (one or two weight tiles, then one or two token terms of n_max rows),
+the k-block ring (each k-block's buffer: one or two weight tiles, then one or two token
+terms of the tile's padded rows, at the next offset of the ring or at 0 when it would run
+past the end; a buffer is loaded only once no k-block in flight overlaps it),
 the MMAs into one of two accumulator buffers (a second weight matrix n_max columns on),
 and the epilogue's indices: fp32 stores into the split's slab, or SwiGLU with bf16 hi /
-lo.  The producer runs as far ahead as the stage ring allows and each epilogue as late as
+lo.  The producer runs as far ahead as the ring allows and each epilogue as late as
 its accumulator buffer allows.  Results are compared with fp64 products of the same bf16
 values.
 """
@@ -58,9 +60,6 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
     n_a = 2 if (W2 is not None or m_pair) else 1
     tile_rows = 2 * BM if m_pair else BM
     a_bytes = BM * BK * 2
-    bmax_bytes = n_max * 128
-    stage_bytes = n_a * a_bytes + terms * bmax_bytes
-    stages = min(smem_budget // stage_bytes, 16)
     acc_cols = n_max * n_a
     nbuf = 2 if 2 * acc_cols <= 512 else 1
     tmem_cols = 32
@@ -91,18 +90,36 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
         g, row0, rows = items[item]
         return g, row0, rows, 0, m
 
+    def kb_bytes(t):
+        n_pad = (tile_of(t)[2] + 15) & ~15
+        return n_a * a_bytes + terms * n_pad * 128
+
     for cta in range(min(grid, n_tiles)):
-        sm, tm = T.Smem(stages * stage_bytes), T.Tmem(tmem_cols)
+        sm, tm = T.Smem(smem_budget), T.Tmem(tmem_cols)
         tiles = tile_walk(cta, grid, n_tiles, m_tiles, rows_a, tile_rows)
         its = [(t, kb) for t in tiles for kb in range(nkb)]
+        offs, head = [], 0                    # KbRing: each k-block's buffer offset and size
+        for t, _ in its:
+            n = kb_bytes(t)
+            off = 0 if head + n > smem_budget else head
+            head = off + n
+            offs.append((off, n))
         loaded = mma_done = 0
         pending = []
+
+        def can_load(it):
+            """No k-block in flight (loaded, not yet consumed) overlaps this buffer, and
+            fewer than 16 are in flight."""
+            if it - mma_done >= 16:
+                return False
+            off, n = offs[it]
+            return all(off + n <= o or o + m <= off for o, m in offs[mma_done:it])
 
         def load(it):
             t, kb = its[it]
             g, row0, rows, split, m = tile_of(t)
             n_pad = (rows + 15) & ~15
-            sa = (it % stages) * stage_bytes
+            sa = offs[it][0]
             sb = sa + n_a * a_bytes
             kx = (split * nkb + (kb + t) % nkb) * BK
             sm.tma_load(sa, W, (kx, m * tile_rows, g), (64, 128, 1), 128)
@@ -111,7 +128,7 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
             if m_pair:
                 sm.tma_load(sa + a_bytes, W, (kx, m * tile_rows + BM, g), (64, 128, 1), 128)
             r = 0
-            lo_off = bmax_bytes if bug != "lo_offset" else n_pad * 64
+            lo_off = n_pad * 128 if bug != "lo_offset" else n_pad * 64
             while r + 64 <= n_pad:
                 sm.tma_load(sb + r * 128, X_hi, (kx, row0 + r), (64, 64), 128)
                 if terms == 2:
@@ -146,9 +163,10 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
                     out[slab + (row0 + col) * ld_out + f[ok]] = a[ok]
 
         for it in range(len(its)):
-            while loaded < len(its) and loaded < mma_done + stages:
+            while loaded < len(its) and can_load(loaded):
                 load(loaded)
                 loaded += 1
+            assert loaded > it, "the MMA warp would wait for a k-block the producer cannot load"
             t, kb = its[it]
             j = tiles.index(t)
             if kb == 0:
@@ -158,17 +176,17 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
             n_pad = (rows + 15) & ~15
             d0 = (j % nbuf) * acc_cols
             d1 = d0 + (n_max if bug != "d1" else acc_cols // 4)
-            sa = (it % stages) * stage_bytes
+            sa = offs[it][0]
             sb = sa + n_a * a_bytes
             for kk in range(BK // 16):
                 acc = kb != 0 or kk != 0
                 T.mma_ss(tm, sm, d0, sa + kk * 32, sb + kk * 32, BM, n_pad, acc)
                 if terms == 2:
-                    T.mma_ss(tm, sm, d0, sa + kk * 32, sb + bmax_bytes + kk * 32, BM, n_pad, True)
+                    T.mma_ss(tm, sm, d0, sa + kk * 32, sb + n_pad * 128 + kk * 32, BM, n_pad, True)
                 if n_a == 2:
                     T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + kk * 32, BM, n_pad, acc)
                     if terms == 2:
-                        T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + bmax_bytes + kk * 32, BM, n_pad, True)
+                        T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + n_pad * 128 + kk * 32, BM, n_pad, True)
             mma_done += 1
             if kb == nkb - 1:
                 pending.append((j, t))
@@ -213,6 +231,28 @@ def test_grouped_gate_up_swiglu_replay():
     out, out_lo = run_gemm(Wg, hi, lo, F, K, F, items=items, n_max=128, W2=Wu)
     got = out + out_lo
     for e in range(4):
+        xe = x[off[e]:off[e + 1]]
+        if len(xe):
+            ref = O.silu(xe @ wg[e].T) * (xe @ wu[e].T)
+            assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-4, e
+
+
+@pytest.mark.parametrize("smem_budget", [200 * 1024, 96 * 1024, 64 * 1024])
+def test_grouped_ring_of_mixed_tiles_replay(smem_budget):
+    """Expert tiles of 16 to 128 token rows in one launch: k-block buffers of 36 to 64 KB
+    wrap around a ring that holds five, two or one of them, and a buffer is loaded only
+    once the k-blocks it overlaps are consumed."""
+    rng = np.random.default_rng(12)
+    counts, F, K = [16, 3, 128, 40, 0, 77, 16, 9], 256, 384
+    E = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
+    items = [(e, r0, min(128, off[e + 1] - r0)) for e in range(E) for r0 in range(off[e], off[e + 1], 128)]
+    x, hi, lo = bf16_pair(rng, int(off[-1]), K)
+    Wg, wg = weights(rng, E, F, K)
+    Wu, wu = weights(rng, E, F, K)
+    out, out_lo = run_gemm(Wg, hi, lo, F, K, F, items=items, n_max=128, W2=Wu, smem_budget=smem_budget, grid=3)
+    got = out + out_lo
+    for e in range(E):
         xe = x[off[e]:off[e + 1]]
         if len(xe):
             ref = O.silu(xe @ wg[e].T) * (xe @ wu[e].T)

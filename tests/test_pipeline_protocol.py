@@ -124,41 +124,79 @@ def run(roles, q, seed, max_steps=200000, end_check=False):
 
 # ---------------------------------------------------------------- the bf16 GEMM (k_tc_gemm.cu)
 
-def bf16_gemm(n_tiles, nkb, stages, nbuf=2):
-    """nbuf: accumulator buffers (one where two do not fit in TMEM: paired weight tiles of
-    256 token columns)."""
-    full = [Barrier(f"full{s}", 1) for s in range(stages)]
-    empty = [Barrier(f"empty{s}", 1) for s in range(stages)]
+class Ranges:
+    """Byte ranges of a shared-memory ring still being read; a producer may only fill a
+    range that overlaps none of them."""
+
+    def __init__(self):
+        self.live = []
+
+    def fill(self, off, n):
+        for o, m in self.live:
+            assert off + n <= o or o + m <= off, f"[{off}, {off + n}) overwrites [{o}, {o + m}) while it is read"
+        self.live.append((off, n))
+
+    def release(self, off, n):
+        self.live.remove((off, n))
+
+
+def bf16_gemm(tile_bytes, nkb, cap, slots=16, nbuf=2, bug=None):
+    """tile_bytes: the k-block buffer size of each tile (weight boxes + token terms of its
+    padded rows); cap: the ring's bytes; slots: barrier pairs (k-blocks in flight at most);
+    nbuf: accumulator buffers (one where two do not fit in TMEM: paired weight tiles of
+    256 token columns).  The producer allocates each k-block's buffer from the ring (KbRing)
+    and waits for the oldest k-blocks until none in flight overlaps it."""
+    n_tiles = len(tile_bytes)
+    full = [Barrier(f"full{s}", 1) for s in range(slots)]
+    empty = [Barrier(f"empty{s}", 1) for s in range(slots)]
     acc_full = [Barrier(f"acc_full{b}", 1) for b in range(nbuf)]
     acc_empty = [Barrier(f"acc_empty{b}", 4) for b in range(nbuf)]
-    bufs, q = Buffers(), Async()
+    bufs, ranges, q = Buffers(), Ranges(), Async()
     acc_done = {}
 
-    def producer():
-        it = 0
+    def ring():
+        head = 0
         for t in range(n_tiles):
-            for kb in range(nkb):
-                s = it % stages
-                yield wait(empty[s], ((it // stages) & 1) ^ 1, it // stages - 1)
-                bufs.fill(("smem", s), 1)
-                full[s].arrive_expect_tx(64)
-                q.loads.append(lambda s=s: full[s].complete_tx(64))
-                it += 1
+            for _ in range(nkb):
+                n = tile_bytes[t]
+                off = 0 if head + n > cap else head
+                head = off + n
+                yield off, n
+
+    def producer():
+        released, inflight = 0, {}
+        for it, (off, n) in enumerate(ring()):
+            s = it % slots
+            while released < it:
+                clash = it - released >= slots
+                if bug != "no_overlap_check":
+                    clash = clash or any(off < o + m and o < off + n for o, m in
+                                         (inflight[b] for b in range(released, it)))
+                if not clash:
+                    break
+                yield wait(empty[released % slots], (released // slots) & 1, released // slots)
+                released += 1
+            ranges.fill(off, n)
+            inflight[it] = (off, n)
+            full[s].arrive_expect_tx(n)
+            q.loads.append(lambda s=s, n=n: full[s].complete_tx(n))
 
     def mma():
         it = 0
+        offs = ring()
         for j in range(n_tiles):
             buf = j % nbuf
             yield wait(acc_empty[buf], ((j // nbuf) & 1) ^ 1, j // nbuf - 1)
             bufs.fill(("acc", buf), 4)
             acc_done[buf] = 0
             for kb in range(nkb):
-                s = it % stages
-                yield wait(full[s], (it // stages) & 1, it // stages)
+                s = it % slots
+                off, n = next(offs)
+                yield wait(full[s], (it // slots) & 1, it // slots)
 
-                def done(s=s, buf=buf):
+                def done(s=s, buf=buf, off=off, n=n):
                     acc_done[buf] += 1
-                    bufs.release(("smem", s))
+                    ranges.release(off, n)
                     empty[s].arrive()
                 q.mma.append(done)
                 it += 1
@@ -262,12 +300,37 @@ def lowp_gemm(n_tiles, nkb, stages, t_stages=4, dec_warps=8):
     return roles, q
 
 
-@pytest.mark.parametrize("n_tiles,nkb,stages", [(1, 1, 2), (3, 1, 3), (2, 5, 3), (5, 4, 6), (4, 32, 3), (7, 3, 8)])
+KB = 1024
+# k-block buffer sizes (weight boxes + token terms): a 16-row expert tile of the gate/up
+# GEMM (36 KB), of the down GEMM (20 KB), a full 128-row gate/up tile (64 KB), a paired
+# dense tile of 256 single-term rows (64 KB), a two-term one (96 KB)
+GEMM_CASES = [
+    ([36 * KB] * 3, 1, 200 * KB), ([36 * KB, 64 * KB, 36 * KB, 20 * KB], 5, 200 * KB),
+    ([20 * KB] * 5, 4, 200 * KB), ([64 * KB] * 4, 32, 200 * KB), ([96 * KB] * 2, 6, 200 * KB),
+    ([36 * KB, 44 * KB, 64 * KB, 52 * KB, 36 * KB, 20 * KB, 28 * KB], 3, 200 * KB),
+    ([64 * KB, 36 * KB], 7, 64 * KB),      # one k-block in flight at a time
+    ([4 * KB] * 3, 40, 200 * KB),           # more k-blocks than barrier pairs fit
+]
+
+
+@pytest.mark.parametrize("tile_bytes,nkb,cap", GEMM_CASES)
 @pytest.mark.parametrize("nbuf", [2, 1])
-def test_bf16_gemm_protocol(n_tiles, nkb, stages, nbuf):
+def test_bf16_gemm_protocol(tile_bytes, nkb, cap, nbuf):
     for seed in range(30):
-        roles, q = bf16_gemm(n_tiles, nkb, stages, nbuf)
+        roles, q = bf16_gemm(tile_bytes, nkb, cap, nbuf=nbuf)
         run(roles, q, seed, end_check=True)
+
+
+def test_the_checker_catches_a_ring_without_the_overlap_check():
+    """A producer that counts barrier pairs but not bytes overwrites a buffer still read."""
+    caught = 0
+    for seed in range(60):
+        roles, q = bf16_gemm([36 * KB, 64 * KB, 20 * KB], 6, 128 * KB, bug="no_overlap_check")
+        try:
+            run(roles, q, seed, end_check=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("n_tiles,nkb,stages", [(1, 1, 2), (3, 1, 6), (2, 5, 3), (5, 4, 6), (3, 16, 6), (6, 3, 2),
