@@ -725,7 +725,7 @@ def run_kernel_attention(args):
             "higher_is_better": False, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
             "data": "synthetic: q, K, V ~ N(0,1) bf16",
             "config": {"workload": f"attention: {n_q} queries x {nq} heads ({nkv} KV heads) d{d} over {n_keys} keys, "
-                                   f"bidirectional", "attention": "head pairs, 64-key chunks" if args.attn_pair
+                                   f"bidirectional", "attention": "head pairs, 128-key chunks" if args.attn_pair
                        else "one head, 128-key chunks", "l2": "K/V re-read between calls"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s", "frac": tf / tf_burst,
                          "flops_per_call": fl, "peak_source": f"{peak_src} bf16_tflops"}}
@@ -801,7 +801,7 @@ def run_kernel_gemm(args):
 
 def _attention_kind():
     """Which attention kernel the library runs (DG_ATTN_PAIR=1: the head-pair kernel)."""
-    return ("head pairs, 64-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
+    return ("head pairs, 128-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
             else "one head, 128-key chunks")
 
 

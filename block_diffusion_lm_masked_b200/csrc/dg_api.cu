@@ -583,14 +583,14 @@ int attn_splits(int n_q, int nq, int n_keys, int* chunks_per_split) {
   return splits;
 }
 
-// split-KV factor of the head-pair kernel: one wave of CTAs, at least four 64-key chunks
+// split-KV factor of the head-pair kernel: one wave of CTAs, at least two 128-key chunks
 // per CTA (each CTA loads its query tiles once)
 int attn_pair_splits(int n_q, int nq, int group, int pair_heads, int n_keys, int* chunks_per_split) {
-  const int nch = ceil_div(n_keys, 64);
+  const int nch = ceil_div(n_keys, 128);
   const int base = ceil_div(n_q, 128) * dg::attn2_head_groups(nq, group, pair_heads);
   int splits = dg::num_sms() / base;
   if (splits > kMaxAttnSplits) splits = kMaxAttnSplits;
-  if (splits > nch / 4) splits = nch / 4;
+  if (splits > nch / 2) splits = nch / 2;
   if (splits < 1) splits = 1;
   *chunks_per_split = ceil_div(nch, splits);
   splits = ceil_div(nch, *chunks_per_split);
@@ -609,7 +609,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
   CUtensorMap mq, mql, mk, mv, mkl, mvl;
   dg_status s;
-  const int base = (pos0 / 128) * 128;  // the low-term window starts here (a multiple of 64)
+  const int base = (pos0 / 128) * 128;  // the low-term window starts here (a multiple of the 128-key chunk)
   const int Lc = ws.L.lo_rows;
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
@@ -621,7 +621,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
-    const uint32_t box[3] = {64, 64, 1};
+    const uint32_t box[3] = {64, 128, 1};
     if ((s = encode_bf16(&mk, kc, 3, dims, str, box)) != DG_OK) return s;
   }
   {
@@ -633,7 +633,7 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)(n_keys - base), (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)Lc * d * 2};
-    const uint32_t box[3] = {64, 64, 1};
+    const uint32_t box[3] = {64, 128, 1};
     if ((s = encode_bf16(&mkl, ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
   }
   {

@@ -97,8 +97,8 @@ struct TcAttnParams {
 // `base`; the query comes from p.q / p.q_lo
 cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, const CUtensorMap& Kl,
                                 const CUtensorMap& Vtl, const TcAttnParams& p, cudaStream_t st);
-// Head-pair variant (same parameters and outputs; chunks_per_split counts 64-key chunks):
-// K / Kl maps with 64-row boxes, Vt / Vtl as above.  pair_heads = 1: two heads of one KV
+// Head-pair variant (same parameters and outputs; chunks_per_split counts 128-key chunks):
+// K / Kl maps with 128-row boxes (64 d wide), Vt / Vtl as above.  pair_heads = 1: two heads of one KV
 // head per CTA where the group is even; 0: one head per CTA.  Grid y =
 // attn2_head_groups(nq, group, pair_heads).
 cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,

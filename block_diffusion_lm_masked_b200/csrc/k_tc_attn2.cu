@@ -1,28 +1,29 @@
-// tcgen05 flash attention, head-pair variant: the same attention as tc_attn_kernel (both
+// tcgen05 flash attention, head-pair kernel: the same attention as tc_attn_kernel (both
 // modes, the same hi + lo precision terms, the same lazy rescale and split-KV partials),
-// organised for more tensor-core overlap per CTA.
+// organised so that the tensor cores stay busy while the softmax runs.
 //
 // One CTA = two query heads of one KV head (one head when the GQA group is odd, or when
 // the host asks for single heads because they fill more SMs) x 128 query rows x a
-// contiguous range of 64-key chunks.  Each K/V chunk is loaded once for both heads.  Warps 0-3 run the softmax of the first head and warps 4-7 that of the
-// second, one query row per thread over the whole 64-key chunk, so no row statistics are
-// exchanged between warps.  Warp 8 issues the TMA loads, warp 9 the MMAs.
+// contiguous range of 128-key chunks.  Each K/V chunk is loaded once for both heads.
+// Warps 0-3 run the softmax of the first head and warps 4-7 that of the second, one query
+// row per thread over the whole 128-key chunk, so no row statistics are exchanged between
+// warps.  Warp 8 issues the TMA loads, warp 9 the MMAs.
 //
-// TMEM (512 columns): per head, two S/P buffers of 64 columns and O (128 columns).  The
-// softmax reads S (fp32, 64 keys) into registers and writes P over it as packed bf16
-// pairs, hi in the first 32 columns and lo in the next 32; the PV MMAs read P from there.
-// Shared memory: the query tiles (hi + lo, 64 KB per head) and three 32 KB K/V slots
-// (K [64 keys][128 d] and V^T [128 d][64 keys]).  A chunk of cached keys takes one slot; a
-// chunk of the call's own keys takes two (hi K/V in the first, lo in the second).
+// TMEM (512 columns): per head one S/P region of 128 columns and O (128 columns).  The
+// softmax reads S (fp32, 128 keys) into registers and writes P over it as packed bf16
+// pairs, hi in the first 64 columns and lo in the next 64; the PV MMAs read P from there.
+// Shared memory: the query tiles (hi + lo, 64 KB per head) and a ring of three 32 KB
+// half-slots, each holding one chunk's K [128 keys][128 d] or V^T [128 d][128 keys] (two
+// 16 KB swizzled blocks); a chunk of the call's own keys also takes its K and V low terms.
+// Ring order per chunk: K (and K lo), then V (and V lo).
 //
-// Issue order of the MMA warp: S_A(j), S_B(j), then PV_A(j-1), PV_B(j-1) and a commit per
-// slot of chunk j-1 that frees it, so the PVs of one chunk run beside the softmax of the
-// next.  Before S_h(j) reuses buffer j & 1 it waits for PV_h(j-2), the last reader of that
-// P.  Where chunks j-1 and j together need more than the three slots (two chunks of own
-// keys in a row), chunk j cannot load until chunk j-1's slots are free, so PV(j-1) goes
-// first there.  That order was checked in a barrier simulation over random interleavings
-// (no deadlock, no slot or S/P buffer refilled while read, no O rescaled under a PV); the
-// plain order deadlocks in that case.
+// Issue order of the MMA warp per chunk j: S_A(j), S_B(j) (each once PV(j-1) of its head
+// has completed, which also means its softmax has read S(j-1) and written P(j-1)), a
+// commit freeing the K half-slots, then PV_A(j), PV_B(j) (each once its head's softmax of
+// chunk j has written P) and a commit freeing the V half-slots.  While the softmax of one
+// head works on S(j), the tensor cores run the other head's S or PV, so with the MMAs of
+// two heads per chunk (two-term S and PV: 33.6 MFLOP, about 3.1 us at the per-SM peak)
+// the tensor pipe waits on a softmax only if it takes longer than one head's S or PV.
 #include <math.h>
 
 #include "attn_softmax.cuh"
@@ -32,22 +33,20 @@
 namespace dg {
 
 constexpr int A2_BQ = 128;
-constexpr int A2_W = 64;                              // keys per chunk
+constexpr int A2_W = 128;                       // keys per chunk
 constexpr int A2_D = 128;
-constexpr int A2_SLOTS = 3;
-constexpr uint32_t A2_QBLK = 128 * 128;               // [128 rows][64 bf16] swizzled: 16 KB
-constexpr uint32_t A2_QHEAD = 4 * A2_QBLK;            // Q hi (2 blocks) + Q lo (2 blocks)
-constexpr uint32_t A2_KBLK = 64 * 128;                // [64 keys][64 d]: 8 KB
-constexpr uint32_t A2_VOFF = 2 * A2_KBLK;             // V^T block [128 d][64 keys]: 16 KB
-constexpr uint32_t A2_SLOT = A2_VOFF + A2_QBLK;       // 32 KB
-constexpr int A2_SMEM = 1024 + 2 * A2_QHEAD + A2_SLOTS * A2_SLOT;
+constexpr int A2_HSLOTS = 3;                    // half-slots of the K/V ring
+constexpr uint32_t A2_BLK = 128 * 128;          // [128 rows][64 bf16] swizzled block: 16 KB
+constexpr uint32_t A2_QHEAD = 4 * A2_BLK;       // Q hi (two d blocks) + Q lo: 64 KB
+constexpr uint32_t A2_HSLOT = 2 * A2_BLK;       // K (two d blocks) or V^T (two key blocks): 32 KB
+constexpr int A2_SMEM = 1024 + 2 * A2_QHEAD + A2_HSLOTS * A2_HSLOT;
 constexpr int A2_LOAD_WARP = 8;
 constexpr int A2_MMA_WARP = 9;
 constexpr int A2_THREADS = 32 * 10;
 static_assert(A2_SMEM <= 227 * 1024 - 512, "shared memory budget");
 
-// TMEM column offsets: head hl's S/P buffer b, and its O
-__device__ __forceinline__ uint32_t a2_sp(int hl, int b) { return (uint32_t)(hl * 256 + b * 64); }
+// TMEM column offsets: head hl's S/P region and its O
+__device__ __forceinline__ uint32_t a2_sp(int hl) { return (uint32_t)(hl * 256); }
 __device__ __forceinline__ uint32_t a2_o(int hl) { return (uint32_t)(hl * 256 + 128); }
 
 // A operand from TMEM (P), B from shared memory (V^T), fp32 accumulate in TMEM
@@ -61,35 +60,41 @@ __device__ __forceinline__ void a2_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// The slot plan both the load and the MMA warp follow: chunk j takes the next one slot
-// (cached keys) or two (own keys) of the ring, in order.
-struct SlotPlan {
+// The half-slot plan both the load and the MMA warp follow: chunk j takes the next one
+// (cached keys) or two (own keys: hi, lo) half-slots for its K, then as many for its V^T.
+struct HalfSlotPlan {
   int nxt = 0;
-  int uses[A2_SLOTS] = {0, 0, 0};
-  int slot[2][2], use[2][2], n[2];  // [j & 1][part]: slot, its use index; parts of chunk j
-  __device__ void take(int j, bool cur) {
-    const int b = j & 1;
-    n[b] = cur ? 2 : 1;
-    for (int i = 0; i < n[b]; ++i) {
-      slot[b][i] = nxt;
-      use[b][i] = uses[nxt]++;
-      nxt = nxt + 1 == A2_SLOTS ? 0 : nxt + 1;
+  int uses[A2_HSLOTS] = {0, 0, 0};
+  int n;                    // parts per operand: 1, or 2 for a chunk of own keys
+  int ks[2], ku[2];         // K parts: half-slot, its use index
+  int vs[2], vu[2];         // V^T parts
+  __device__ void take(bool cur) {
+    n = cur ? 2 : 1;
+    for (int i = 0; i < n; ++i) {
+      ks[i] = nxt;
+      ku[i] = uses[nxt]++;
+      nxt = nxt + 1 == A2_HSLOTS ? 0 : nxt + 1;
+    }
+    for (int i = 0; i < n; ++i) {
+      vs[i] = nxt;
+      vu[i] = uses[nxt]++;
+      nxt = nxt + 1 == A2_HSLOTS ? 0 : nxt + 1;
     }
   }
 };
 
-__global__ void __launch_bounds__(A2_THREADS, 1)
+__global__ void __maxnreg__(200)
     tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
                     const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
                     const TcAttnParams p, const int pair_heads) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_bar;
-  __shared__ __align__(8) uint64_t kv_full[A2_SLOTS];  // the slot's TMA loads have landed
-  __shared__ __align__(8) uint64_t kv_free[A2_SLOTS];  // the MMAs reading the slot are complete
-  __shared__ __align__(8) uint64_t s_full[2][2];       // [head][buffer]: S is in TMEM
-  __shared__ __align__(8) uint64_t p_ready[2][2];      // [head][buffer]: P is in TMEM (4 warps)
-  __shared__ __align__(8) uint64_t pv_done[2][2];      // [head][buffer]: the PV reading P is complete
+  __shared__ __align__(8) uint64_t hs_full[A2_HSLOTS];  // the half-slot's TMA loads have landed
+  __shared__ __align__(8) uint64_t hs_free[A2_HSLOTS];  // the MMAs reading the half-slot are complete
+  __shared__ __align__(8) uint64_t s_full[2];           // [head]: S of the chunk is in TMEM
+  __shared__ __align__(8) uint64_t p_ready[2];          // [head]: P of the chunk is in TMEM (4 warps)
+  __shared__ __align__(8) uint64_t pv_done[2];          // [head]: the PV of the chunk is complete
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
@@ -121,22 +126,21 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   }
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                       // [head][Q hi blk0, blk1, Q lo blk0, blk1]
-  uint8_t* sSlot = smem + 2 * A2_QHEAD;     // [slot][K blk0, K blk1, V^T]
+  uint8_t* sQ = smem;                   // [head][Q hi blk0, blk1, Q lo blk0, blk1]
+  uint8_t* sHalf = smem + 2 * A2_QHEAD;  // [half-slot][blk0, blk1]
 
   if (warp == A2_MMA_WARP) tmem_alloc(&tmem_base_s, 512);
   if (tid == A2_LOAD_WARP * 32) {
     mbar_init(&q_bar, 1);
-    for (int s = 0; s < A2_SLOTS; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_free[s], 1);
+    for (int s = 0; s < A2_HSLOTS; ++s) {
+      mbar_init(&hs_full[s], 1);
+      mbar_init(&hs_free[s], 1);
     }
-    for (int hl = 0; hl < 2; ++hl)
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&s_full[hl][b], 1);
-        mbar_init(&p_ready[hl][b], 4);
-        mbar_init(&pv_done[hl][b], 1);
-      }
+    for (int hl = 0; hl < 2; ++hl) {
+      mbar_init(&s_full[hl], 1);
+      mbar_init(&p_ready[hl], 4);
+      mbar_init(&pv_done[hl], 1);
+    }
     mbar_init(&drain_bar, 1);
     abort_s = 0;
     fence_barrier_init();
@@ -148,14 +152,13 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   const uint32_t tmem = tmem_base_s;
 
   auto is_cur = [&](int j) { return p.has_lo && (c_begin + j) * A2_W >= p.base; };
-  const uint32_t idesc_s = idesc_bf16_f32(A2_BQ, A2_W);
-  const uint32_t idesc_pv = idesc_bf16_f32(A2_BQ, A2_D);
-  int loaded[A2_SLOTS] = {0, 0, 0};  // loads the load thread issued into each slot (for the wind-down)
+  const uint32_t idesc = idesc_bf16_f32(A2_BQ, A2_W);  // S: 128 rows x 128 keys; PV: 128 rows x 128 d
+  int loaded[A2_HSLOTS] = {0, 0, 0};  // loads the load thread issued into each half-slot (for the wind-down)
   bool q_issued = false;
 
   if (warp == A2_LOAD_WARP) {
     if (lane == 0) {
-      // ================= loads: the query tiles, then each chunk's slots in plan order
+      // ================= loads: the query tiles, then each chunk's K and V^T in plan order
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmQl);
       prefetch_tmap(&tmK);
@@ -168,117 +171,111 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       for (int hl = 0; hl < nh; ++hl) {
         uint8_t* q = sQ + hl * A2_QHEAD;
         tma_load_3d(q, &tmQ, 0, q_row0, h0 + hl, &q_bar);
-        tma_load_3d(q + A2_QBLK, &tmQ, 64, q_row0, h0 + hl, &q_bar);
-        tma_load_3d(q + 2 * A2_QBLK, &tmQl, 0, q_row0, h0 + hl, &q_bar);
-        tma_load_3d(q + 3 * A2_QBLK, &tmQl, 64, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + A2_BLK, &tmQ, 64, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + 2 * A2_BLK, &tmQl, 0, q_row0, h0 + hl, &q_bar);
+        tma_load_3d(q + 3 * A2_BLK, &tmQl, 64, q_row0, h0 + hl, &q_bar);
       }
       q_issued = true;
-      SlotPlan lp;
+      HalfSlotPlan lp;
       bool ok = true;
+      // one half-slot: wait until its previous use was freed, then its two 16 KB blocks
+      auto load_half = [&](int s, int u, const CUtensorMap* map, bool is_v, int krow) {
+        if (u >= 1 && !mbar_wait(&hs_free[s], (uint32_t)(u - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
+          return false;
+        if (!DG_GUARD(krow >= 0 && krow % A2_W == 0, p.err)) {
+          abort_s = 1;
+          return false;
+        }
+        uint8_t* dst = sHalf + s * A2_HSLOT;
+        loaded[s] += 1;
+        mbar_arrive_expect_tx(&hs_full[s], A2_HSLOT);
+        if (is_v) {  // V^T [128 d][64 keys] blocks: keys krow .. +63, +64 .. +127
+          tma_load_3d(dst, map, krow, 0, kvh, &hs_full[s]);
+          tma_load_3d(dst + A2_BLK, map, krow + 64, 0, kvh, &hs_full[s]);
+        } else {     // K [128 keys][64 d] blocks: d 0 .. 63, 64 .. 127
+          tma_load_3d(dst, map, 0, krow, kvh, &hs_full[s]);
+          tma_load_3d(dst + A2_BLK, map, 64, krow, kvh, &hs_full[s]);
+        }
+        return true;
+      };
       for (int j = 0; j < nck && ok; ++j) {
         const int key0 = (c_begin + j) * A2_W;
-        lp.take(j, is_cur(j));
-        for (int i = 0; i < lp.n[j & 1] && ok; ++i) {
-          const int s = lp.slot[j & 1][i], u = lp.use[j & 1][i];
-          // the slot's previous chunk was freed by the MMAs that read it
-          if (u >= 1 && !(ok = mbar_wait(&kv_free[s], (uint32_t)(u - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN)))
-            break;
-          uint8_t* k = sSlot + s * A2_SLOT;
-          const CUtensorMap* mk = (i == 0) ? &tmK : &tmKl;
-          const CUtensorMap* mv = (i == 0) ? &tmVt : &tmVtl;
-          const int krow = (i == 0) ? key0 : key0 - p.base;  // the low-term window starts at `base`
-          if (!DG_GUARD(krow >= 0 && krow % A2_W == 0, p.err)) {
-            ok = false;
-            abort_s = 1;
-            break;
-          }
-          loaded[s] += 1;
-          mbar_arrive_expect_tx(&kv_full[s], A2_SLOT);
-          tma_load_3d(k, mk, 0, krow, kvh, &kv_full[s]);
-          tma_load_3d(k + A2_KBLK, mk, 64, krow, kvh, &kv_full[s]);
-          tma_load_3d(k + A2_VOFF, mv, krow, 0, kvh, &kv_full[s]);
-        }
+        lp.take(is_cur(j));
+        // part 0: the cache's bf16 keys; part 1: the low terms, rows counted from `base`
+        for (int i = 0; i < lp.n && ok; ++i)
+          ok = load_half(lp.ks[i], lp.ku[i], i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
+        for (int i = 0; i < lp.n && ok; ++i)
+          ok = load_half(lp.vs[i], lp.vu[i], i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
       }
     }
     __syncwarp();
   } else if (warp == A2_MMA_WARP) {
     if (lane == 0) {
       // ================= MMAs
-      SlotPlan mp;
-      auto slot_addr = [&](int s) { return smem_u32(sSlot + s * A2_SLOT); };
-      auto issue_s = [&](int hl, int j) {
-        const int b = j & 1;
-        const bool cur = mp.n[b] == 2;
-        const uint32_t d = tmem + a2_sp(hl, b);
-        const uint32_t q = smem_u32(sQ + hl * A2_QHEAD), ql = q + 2 * A2_QBLK;
-        const uint32_t k = slot_addr(mp.slot[b][0]);
-        const uint32_t kl = cur ? slot_addr(mp.slot[b][1]) : 0u;
+      HalfSlotPlan mp;
+      auto half_addr = [&](int s) { return smem_u32(sHalf + s * A2_HSLOT); };
+      auto issue_s = [&](int hl) {
+        const uint32_t d = tmem + a2_sp(hl);
+        const uint32_t q = smem_u32(sQ + hl * A2_QHEAD), ql = q + 2 * A2_BLK;
+        const uint32_t k = half_addr(mp.ks[0]);
+        const uint32_t kl = mp.n == 2 ? half_addr(mp.ks[1]) : 0u;
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t oq = kb * A2_QBLK + kk * 32, okb = kb * A2_KBLK + kk * 32;
-            const uint64_t kd = sw128_kmajor_desc(k + okb);
-            tc_mma(d, sw128_kmajor_desc(q + oq), kd, idesc_s, (kb | kk) != 0 ? 1u : 0u);
-            tc_mma(d, sw128_kmajor_desc(ql + oq), kd, idesc_s, 1u);
-            if (cur) tc_mma(d, sw128_kmajor_desc(q + oq), sw128_kmajor_desc(kl + okb), idesc_s, 1u);
+            const uint32_t o = kb * A2_BLK + kk * 32;
+            const uint64_t kd = sw128_kmajor_desc(k + o);
+            tc_mma(d, sw128_kmajor_desc(q + o), kd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma(d, sw128_kmajor_desc(ql + o), kd, idesc, 1u);
+            if (mp.n == 2) tc_mma(d, sw128_kmajor_desc(q + o), sw128_kmajor_desc(kl + o), idesc, 1u);
           }
-        tc_commit(&s_full[hl][b]);
+        tc_commit(&s_full[hl]);
       };
-      auto issue_pv = [&](int hl, int k) {
-        const int b = k & 1;
-        const bool cur = mp.n[b] == 2;
-        const uint32_t o = tmem + a2_o(hl), pp = tmem + a2_sp(hl, b);
-        const uint32_t v = slot_addr(mp.slot[b][0]) + A2_VOFF;
-        const uint32_t vl = cur ? slot_addr(mp.slot[b][1]) + A2_VOFF : 0u;
+      auto issue_pv = [&](int hl, int j) {
+        const uint32_t o = tmem + a2_o(hl), pp = tmem + a2_sp(hl);
+        const uint32_t v = half_addr(mp.vs[0]);
+        const uint32_t vl = mp.n == 2 ? half_addr(mp.vs[1]) : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 16 keys = 8 packed P columns per MMA
-          const uint64_t vd = sw128_kmajor_desc(v + kk * 32);
-          a2_mma_ts(o, pp + kk * 8, vd, idesc_pv, (k > 0 || kk != 0) ? 1u : 0u);
-          a2_mma_ts(o, pp + 32 + kk * 8, vd, idesc_pv, 1u);
-          if (cur) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + kk * 32), idesc_pv, 1u);
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys = 8 packed P columns per MMA
+          const uint32_t vo = (kk >> 2) * A2_BLK + (kk & 3) * 32;
+          const uint64_t vd = sw128_kmajor_desc(v + vo);
+          a2_mma_ts(o, pp + kk * 8, vd, idesc, (j > 0 || kk != 0) ? 1u : 0u);
+          a2_mma_ts(o, pp + 64 + kk * 8, vd, idesc, 1u);
+          if (mp.n == 2) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
         }
-        tc_commit(&pv_done[hl][b]);
-      };
-      // PV of chunk k for every head once its P is written, then free chunk k's slots (the
-      // last chunk's slots are not reused: no commit nobody waits for)
-      auto pv_chunk = [&](int k) {
-        for (int hl = 0; hl < nh; ++hl) {
-          if (!mbar_wait(&p_ready[hl][k & 1], (uint32_t)(k >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
-            return false;
-          tc_fence_after();
-          issue_pv(hl, k);
-        }
-        if (k + 1 < nck)
-          for (int i = 0; i < mp.n[k & 1]; ++i) tc_commit(&kv_free[mp.slot[k & 1][i]]);
-        return true;
+        tc_commit(&pv_done[hl]);
       };
 
       bool ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
       for (int j = 0; j < nck && ok; ++j) {
-        mp.take(j, is_cur(j));
-        const bool pv_first = j >= 1 && mp.n[(j - 1) & 1] + mp.n[j & 1] > A2_SLOTS;
-        if (pv_first && !(ok = pv_chunk(j - 1))) break;
-        for (int i = 0; i < mp.n[j & 1] && ok; ++i)
-          ok = mbar_wait(&kv_full[mp.slot[j & 1][i]], (uint32_t)mp.use[j & 1][i] & 1u, &abort_s, p.err,
-                         DG_DEVERR_TIMEOUT_ATTN);
+        mp.take(is_cur(j));
+        for (int i = 0; i < mp.n && ok; ++i)
+          ok = mbar_wait(&hs_full[mp.ks[i]], (uint32_t)mp.ku[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         for (int hl = 0; hl < nh && ok; ++hl) {
-          // S/P buffer j & 1 was last read by PV(j - 2)
-          if (j >= 2)
-            ok = mbar_wait(&pv_done[hl][j & 1], (uint32_t)((j >> 1) - 1) & 1u, &abort_s, p.err,
-                           DG_DEVERR_TIMEOUT_ATTN);
+          // the head's S/P region was last read by PV(j - 1)
+          if (j >= 1)
+            ok = mbar_wait(&pv_done[hl], (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
           if (!ok) break;
           tc_fence_after();
-          issue_s(hl, j);
+          issue_s(hl);
         }
         if (!ok) break;
-        if (j >= 1 && !pv_first) ok = pv_chunk(j - 1);
+        for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.ks[i]]);
+        for (int i = 0; i < mp.n && ok; ++i)
+          ok = mbar_wait(&hs_full[mp.vs[i]], (uint32_t)mp.vu[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        for (int hl = 0; hl < nh && ok; ++hl) {
+          ok = mbar_wait(&p_ready[hl], (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(hl, j);
+        }
+        if (!ok) break;
+        for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.vs[i]]);
       }
-      if (ok) pv_chunk(nck - 1);
     }
     __syncwarp();
   } else if ((warp >> 2) < nh) {
-    // ================= softmax: head hl, query row `row` (TMEM lane), all 64 keys of a chunk
+    // ================= softmax: head hl, query row `row` (TMEM lane), all 128 keys of a chunk
     const int hl = warp >> 2;
     const int h = h0 + hl;
     const int row = (warp & 3) * 32 + lane;
@@ -286,20 +283,19 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     const int my_pos = p.q_pos0 + my_row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int key_lim = p.causal ? min(p.n_keys, my_pos + 1) : p.n_keys;
+    const uint32_t spa = tmem + a2_sp(hl) + lane_off;
     float m_used = -INFINITY;
     uint64_t l2 = f2_pack(0.0f, 0.0f);  // the row sum as two partial sums (even and odd keys)
     const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int j = 0; j < nck && ok; ++j) {
-      const int b = j & 1;
       // every wait's outcome is made warp-uniform: the tcgen05.ld / st that follow are
       // warp-collective, so a lane that gave up must take its whole warp with it
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(&s_full[hl][b], (uint32_t)(j >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
+                      mbar_wait(&s_full[hl], (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t spa = tmem + a2_sp(hl, b) + lane_off;
-      // the chunk's raw scores, all four loads in flight before the one wait
+      // the chunk's raw scores, all eight loads in flight before the one wait
       uint32_t r[A2_W / 16][16];
 #pragma unroll
       for (int c = 0; c < A2_W / 16; ++c) tmem_ld16(spa + c * 16, r[c]);
@@ -311,24 +307,28 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         for (int i = 0; i < A2_W; ++i)
           if (key0 + i >= key_lim) r[i / 16][i % 16] = __float_as_uint(-INFINITY);
       }
-      // the row maximum of the raw scores, then scaled (the scale is positive and
-      // rounding monotone, so this is the maximum of the scaled scores)
-      float cm = -INFINITY;
+      // the row maximum of the raw scores (four independent chains), then scaled: the
+      // scale is positive and rounding monotone, so this is the maximum of the scaled scores
+      float cm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int i = 0; i < A2_W; i += 2)
-        cm = max3f(cm, __uint_as_float(r[i / 16][i % 16]), __uint_as_float(r[i / 16][i % 16 + 1]));
-      const float cmax = cm * p.scale_log2;
+      for (int i = 0; i < A2_W; i += 8)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          cm4[c] = max3f(cm4[c], __uint_as_float(r[(i + 2 * c) / 16][(i + 2 * c) % 16]),
+                         __uint_as_float(r[(i + 2 * c) / 16][(i + 2 * c) % 16 + 1]));
+      const float cmax = fmaxf(fmaxf(cm4[0], cm4[1]), fmaxf(cm4[2], cm4[3])) * p.scale_log2;
       const bool upd = cmax > m_used + 8.0f;
       const float alpha = upd ? ex2_approx(m_used - cmax) : 1.0f;  // 0 while nothing was visible yet
       // tcgen05.ld/st are warp-collective: the warp rescales its rows of O if any row must,
       // once the previous chunk's PV is complete (O stable; PV(j) waits for this P)
       if (__any_sync(0xffffffffu, upd && j > 0)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, &abort_s,
-                                               p.err, DG_DEVERR_TIMEOUT_ATTN));
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl], (uint32_t)(j - 1) & 1u, &abort_s, p.err,
+                                               DG_DEVERR_TIMEOUT_ATTN));
         if (!ok) break;
         tc_fence_after();
         const uint32_t oa = tmem + a2_o(hl) + lane_off;
-#pragma unroll
+        // (16 columns at a time: the chunk's 128 scores stay live in registers meanwhile)
+#pragma unroll 1
         for (int c = 0; c < A2_D / 16; ++c) {
           uint32_t o[16];
           tmem_ld16(oa + c * 16, o);
@@ -343,16 +343,16 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         m_used = cmax;
       }
       // P = 2^(s * scale - m_used) (one rounding), packed bf16 pairs over this row's S: hi
-      // in columns 0..31, lo in 32..63.  A row that has seen no key has m_used = -inf and
+      // in columns 0..63, lo in 64..127.  A row that has seen no key has m_used = -inf and
       // only -inf scores: its offset is taken as 0, so that every P is 2^-inf = 0.
       const float neg_m = (m_used == -INFINITY) ? 0.0f : -m_used;
       const uint64_t nm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {  // 32 keys -> 16 packed columns per store
-        uint32_t wh[16], wl[16];
+      for (int c = 0; c < A2_W / 16; ++c) {  // 16 keys -> 8 packed columns per store
+        uint32_t wh[8], wl[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i0 = c * 32 + 2 * e;
+        for (int e = 0; e < 8; ++e) {
+          const int i0 = c * 16 + 2 * e;
           const uint64_t t = f2_fma(f2_pack(__uint_as_float(r[i0 / 16][i0 % 16]),
                                             __uint_as_float(r[i0 / 16][i0 % 16 + 1])), scale2, nm2);
           float t0, t1;
@@ -366,17 +366,17 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           wh[e] = hi;
           wl[e] = bf16x2_pack(lo0, lo1);
         }
-        tmem_st16(spa + c * 16, wh);
-        tmem_st16(spa + 32 + c * 16, wl);
+        tmem_st8(spa + c * 8, wh);
+        tmem_st8(spa + 64 + c * 8, wl);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[hl][b]);
+      if (lane == 0) mbar_arrive(&p_ready[hl]);
     }
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl][(nck - 1) & 1], (uint32_t)((nck - 1) >> 1) & 1u, &abort_s,
-                                             p.err, DG_DEVERR_TIMEOUT_ATTN));
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[hl], (uint32_t)(nck - 1) & 1u, &abort_s, p.err,
+                                             DG_DEVERR_TIMEOUT_ATTN));
     float l0, l1;
     f2_unpack(l2, l0, l1);
     const float l = l0 + l1;
@@ -441,8 +441,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   }
   if (abort_s && tid == A2_LOAD_WARP * 32) {
     if (q_issued) mbar_wait_drain(&q_bar, 0);
-    for (int s = 0; s < A2_SLOTS; ++s)
-      if (loaded[s] > 0) mbar_wait_drain(&kv_full[s], (uint32_t)(loaded[s] - 1) & 1u);
+    for (int s = 0; s < A2_HSLOTS; ++s)
+      if (loaded[s] > 0) mbar_wait_drain(&hs_full[s], (uint32_t)(loaded[s] - 1) & 1u);
   }
   tc_fence_before();
   __syncthreads();

@@ -133,7 +133,7 @@ dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, 
 
 /* The same attention through the head-pair kernel: two query heads of one KV head per CTA
  * (one when nq / nkv is odd, or when single heads fill at least a quarter more SMs in the
- * one wave of CTAs), 64-key chunks, the same precision terms, outputs, workspace and
+ * one wave of CTAs), 128-key chunks, the same precision terms, outputs, workspace and
  * errors as dg_debug_attention_bf16.  Setting DG_ATTN_PAIR=1 in the environment
  * (read once per process) routes the bf16 pass's attention through this kernel too. */
 dg_status dg_debug_attention_pair_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,

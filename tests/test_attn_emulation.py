@@ -374,8 +374,9 @@ def run_single(c, bug=None):
 
 # ---------------------------------------------------------------- tc_attn2_kernel
 def run_pair(c, bug=None, force_pair=None):
-    """tc_attn2_kernel: a head pair (one head for odd groups) x 128 rows x 64-key chunks,
-    three 32 KB slots, per head S/P buffers at 256 hl + 64 b and O at 256 hl + 128."""
+    """tc_attn2_kernel: a head pair (one head for odd groups) x 128 rows x 128-key chunks,
+    a ring of three 32 KB half-slots (a chunk's K, then its V^T, each with its low term
+    for own keys), per head one S/P region at 256 hl and O at 256 hl + 128."""
     nq, nkv, n_q, pos0, n_keys, causal = (c[k] for k in ("nq", "nkv", "n_q", "pos0", "n_keys", "causal"))
     m = maps(c)
     group = nq // nkv
@@ -384,17 +385,14 @@ def run_pair(c, bug=None, force_pair=None):
         from test_attn_geometry import splits_pair
         pair = force_pair and group % 2 == 0
         n_splits, cps = splits_pair(n_q, nq, group, n_keys, pair)
-    W, QBLK, KBLK = 64, 128 * 128, 64 * 128
-    QHEAD, VOFF = 4 * QBLK, 2 * KBLK
-    SLOT = VOFF + QBLK
-    SLOTS = 3
-    sQ, sSlot = 0, 2 * QHEAD
-    a2_sp = (lambda hl, b: hl * 256) if bug == "one_sp_buffer" else (lambda hl, b: hl * 256 + b * 64)
+    W, BLK = 128, 128 * 128
+    QHEAD, HSLOT = 4 * BLK, 2 * BLK
+    HSLOTS = 3
+    phys = (lambda s_: s_ % 2) if bug == "two_slots" else (lambda s_: s_)   # a ring one half-slot short
+    sQ, sHalf = 0, 2 * QHEAD
+    a2_sp = lambda hl: hl * 256
     a2_o = lambda hl: hl * 256 + 128
-    if bug == "p_lo_offset":
-        p_lo = 16
-    else:
-        p_lo = 32
+    p_lo = 32 if bug == "p_lo_offset" else 64
     scale = np.float32(1.4426950408889634 / math.sqrt(D))
     nh = 2 if pair else 1
     out = np.zeros((n_q, nq * D), np.float32)
@@ -415,132 +413,120 @@ def run_pair(c, bug=None, force_pair=None):
                 rows = q_row0 + np.arange(128)
                 if nck <= 0:
                     continue
-                sm, tm = T.Smem(2 * QHEAD + SLOTS * SLOT), T.Tmem()
+                sm, tm = T.Smem(2 * QHEAD + 3 * HSLOT), T.Tmem()
                 is_cur = lambda j: (c_begin + j) * W >= c["base"]
                 for hl in range(nh):
                     q = sQ + hl * QHEAD
-                    for off, mp, x in ((0, "Q", 0), (QBLK, "Q", 64), (2 * QBLK, "Ql", 0), (3 * QBLK, "Ql", 64)):
+                    for off, mp, x in ((0, "Q", 0), (BLK, "Q", 64), (2 * BLK, "Ql", 0), (3 * BLK, "Ql", 64)):
                         sm.tma_load_3d(q + off, m[mp], x, q_row0, h0 + hl, 64, 128)
-                # the slot plan (SlotPlan::take), and which chunk's PV frees each slot use
-                plan, nxt, uses = [], 0, [0] * SLOTS
+                # the half-slot plan (HalfSlotPlan::take): per chunk its K parts, then its V parts
+                plan, items, nxt = [], [], 0
                 for j in range(nck):
-                    parts = []
-                    for _ in range(2 if is_cur(j) else 1):
-                        parts.append((nxt, uses[nxt]))
-                        uses[nxt] += 1
-                        nxt = (nxt + 1) % SLOTS
-                    plan.append(parts)
-                if bug == "two_slots":                        # a ring one slot short, same plan
-                    plan = [[(s % 2, u) for s, u in parts] for parts in plan]
-                holder = {}                                   # slot -> chunk whose loads it holds until its PV
-                loaded = [0]                                  # chunks loaded so far (in order)
+                    n = 2 if is_cur(j) else 1
+                    ks, vs = [], []
+                    for lst in (ks, vs):
+                        for i in range(n):
+                            lst.append(nxt)
+                            items.append((j, "K" if lst is ks else "V", i, nxt))
+                            nxt = (nxt + 1) % HSLOTS
+                    plan.append((ks, vs))
+                holder = {}                                   # half-slot -> (chunk, operand) held until freed
+                loaded = [0]                                  # items loaded so far (in order)
 
                 def pump():
-                    """The load warp: the next chunk's slots, each once its previous use was freed."""
-                    while loaded[0] < nck:
-                        j = loaded[0]
-                        if any(s in holder for s, _ in plan[j]):
+                    """The load warp: the next items, each once its half-slot's previous use was freed."""
+                    while loaded[0] < len(items):
+                        j, op, i, s = items[loaded[0]]
+                        if s in holder:
                             return
                         key0 = (c_begin + j) * W
-                        for i, (s, _) in enumerate(plan[j]):
-                            k = sSlot + s * SLOT
-                            mk, mv = ("K", "Vt") if i == 0 else ("Kl", "Vtl")
-                            krow = key0 if i == 0 else key0 - c["base"]
-                            sm.tma_load_3d(k, m[mk], 0, krow, kvh, 64, 64)
-                            sm.tma_load_3d(k + KBLK, m[mk], 64, krow, kvh, 64, 64)
-                            sm.tma_load_3d(k + VOFF, m[mv], krow, 0, kvh, 64, 128)
-                            holder[s] = j
+                        krow = key0 if i == 0 else key0 - c["base"]
+                        dst = sHalf + phys(s) * HSLOT
+                        if op == "K":
+                            mk = "K" if i == 0 else "Kl"
+                            sm.tma_load_3d(dst, m[mk], 0, krow, kvh, 64, 128)
+                            sm.tma_load_3d(dst + BLK, m[mk], 64, krow, kvh, 64, 128)
+                        else:
+                            mv = "Vt" if i == 0 else "Vtl"
+                            sm.tma_load_3d(dst, m[mv], krow, 0, kvh, 64, 128)
+                            sm.tma_load_3d(dst + BLK, m[mv], krow + 64, 0, kvh, 64, 128)
+                        holder[s] = (j, op)
                         loaded[0] += 1
 
-                def issue_s(hl, j):
-                    b = j & 1
-                    cur = len(plan[j]) == 2
-                    d = a2_sp(hl, b)
-                    q, ql = sQ + hl * QHEAD, sQ + hl * QHEAD + 2 * QBLK
-                    k = sSlot + plan[j][0][0] * SLOT
-                    kl = sSlot + plan[j][1][0] * SLOT if cur else 0
-                    for kb in range(2):
-                        for kk in range(4):
-                            oq, okb = kb * QBLK + kk * 32, kb * KBLK + kk * 32
-                            T.mma_ss(tm, sm, d, q + oq, k + okb, 128, W, (kb | kk) != 0)
-                            T.mma_ss(tm, sm, d, ql + oq, k + okb, 128, W, True)
-                            if cur:
-                                T.mma_ss(tm, sm, d, q + oq, kl + okb, 128, W, True)
+                def ready(j, op):
+                    pump()
+                    need = [it for it in items if it[0] == j and it[1] == op]
+                    assert all(items.index(it) < loaded[0] for it in need), \
+                        "the MMA warp would wait for a half-slot the load warp cannot fill"
 
-                def issue_pv(hl, k_):
-                    b = k_ & 1
-                    cur = len(plan[k_]) == 2
-                    o, pp = a2_o(hl), a2_sp(hl, b)
-                    v = sSlot + plan[k_][0][0] * SLOT + VOFF
-                    vl = sSlot + plan[k_][1][0] * SLOT + VOFF if cur else 0
-                    for kk in range(4):
-                        vd = v + kk * 32
-                        T.mma_ts(tm, sm, o, pp + kk * 8, vd, 128, D, k_ > 0 or kk != 0)
-                        T.mma_ts(tm, sm, o, pp + p_lo + kk * 8, vd, 128, D, True)
-                        if cur:
-                            T.mma_ts(tm, sm, o, pp + kk * 8, vl + kk * 32, 128, D, True)
-
-                def pv_run(k_):
-                    for hl in range(nh):
-                        issue_pv(hl, k_)
-                    for s, _ in plan[k_]:                    # the commits free chunk k_'s slots
-                        if holder.get(s) == k_:
+                def free(j, op):
+                    for s in (plan[j][0] if op == "K" else plan[j][1]):
+                        if holder.get(s) == (j, op):
                             del holder[s]
                     pump()
 
-                # issued PVs run on the tensor pipe later: deferred until the next MMA issue
-                # (in-order pipe), an O rescale, a wait for a slot, or the end
-                pending = []
+                def issue_s(hl, j):
+                    ks = plan[j][0]
+                    d = a2_sp(hl)
+                    q, ql = sQ + hl * QHEAD, sQ + hl * QHEAD + 2 * BLK
+                    k = sHalf + phys(ks[0]) * HSLOT
+                    kl = sHalf + phys(ks[1]) * HSLOT if len(ks) == 2 else 0
+                    for kb in range(2):
+                        for kk in range(4):
+                            o = kb * BLK + kk * 32
+                            T.mma_ss(tm, sm, d, q + o, k + o, 128, W, (kb | kk) != 0)
+                            T.mma_ss(tm, sm, d, ql + o, k + o, 128, W, True)
+                            if len(ks) == 2:
+                                T.mma_ss(tm, sm, d, q + o, kl + o, 128, W, True)
 
-                def flush():
-                    while pending:
-                        pv_run(pending.pop(0))
-
-                def pv_chunk(k_):
-                    pending.append(k_)
+                def issue_pv(hl, j):
+                    vs = plan[j][1]
+                    o, pp = a2_o(hl), a2_sp(hl)
+                    v = sHalf + phys(vs[0]) * HSLOT
+                    vl = sHalf + phys(vs[1]) * HSLOT if len(vs) == 2 else 0
+                    for kk in range(8):
+                        vo = (kk >> 2) * BLK + (kk & 3) * 32
+                        T.mma_ts(tm, sm, o, pp + kk * 8, v + vo, 128, D, j > 0 or kk != 0)
+                        T.mma_ts(tm, sm, o, pp + p_lo + kk * 8, v + vo, 128, D, True)
+                        if len(vs) == 2:
+                            T.mma_ts(tm, sm, o, pp + kk * 8, vl + vo, 128, D, True)
 
                 m_used = [np.full(128, NEG, np.float32) for _ in range(nh)]
                 lpair = [(np.zeros(128, np.float32), np.zeros(128, np.float32)) for _ in range(nh)]
                 key_lim = np.array([c["key_lim"][r] if r < n_q else n_keys for r in rows])
 
                 def softmax(hl, j):
-                    b = j & 1
-                    spa = a2_sp(hl, b)
-                    raw = np.concatenate([tm.t[:, spa + cc * 16:spa + cc * 16 + 16] for cc in range(4)], axis=1)
+                    spa = a2_sp(hl)
+                    raw = np.concatenate([tm.t[:, spa + cc * 16:spa + cc * 16 + 16] for cc in range(8)], axis=1)
                     s = softmax_chunk_raw(raw, (c_begin + j) * W, key_lim)
 
                     def rescale(any_w, alpha):
-                        if j > 0 and any_w.any():
-                            flush()                           # waits for PV(j - 1)
+                        if j > 0 and any_w.any():                 # PV(j - 1) has completed
                             blk = tm.f32(a2_o(hl), D)
                             blk[any_w] = (blk[any_w] * alpha[any_w, None]).astype(np.float32)
                     le, lo_ = lpair[hl]
                     m_old = m_used[hl]
-                    m_used[hl], le = lazy_update((s.max(axis=1) * scale).astype(np.float32), m_old, le, rescale)
-                    _, lo_ = lazy_update((s.max(axis=1) * scale).astype(np.float32), m_old, lo_, lambda a, b: None)
+                    rmax = (s.max(axis=1) * scale).astype(np.float32)
+                    m_used[hl], le = lazy_update(rmax, m_old, le, rescale)
+                    _, lo_ = lazy_update(rmax, m_old, lo_, lambda a, b: None)
                     wh, wl, lpair[hl] = p_words_fma(s, scale, m_used[hl], (le, lo_))
-                    tm.t[:, spa:spa + 32] = wh                # P over this row's S: hi, then lo
-                    tm.t[:, spa + p_lo:spa + p_lo + 32] = wl
+                    tm.t[:, spa:spa + 64] = wh                # P over this row's S: hi, then lo
+                    tm.t[:, spa + p_lo:spa + p_lo + 64] = wl
 
                 pump()
                 for j in range(nck):
-                    pv_first = j >= 1 and len(plan[j - 1]) + len(plan[j]) > SLOTS
-                    if bug == "no_pv_first":
-                        pv_first = False
-                    if pv_first:
-                        pv_chunk(j - 1)
-                    if loaded[0] <= j:
-                        flush()                               # the slots come free as pending PVs complete
-                    assert loaded[0] > j, "the MMA warp would wait for a chunk the load warp cannot load"
-                    flush()
+                    ready(j, "K")
                     for hl in range(nh):
                         issue_s(hl, j)
-                    if j >= 1 and not pv_first:
-                        pv_chunk(j - 1)
+                        if bug == "k_free_after_first_head" and hl == 0:
+                            free(j, "K")                      # the commit placed before the second head's S
+                    free(j, "K")
                     for hl in range(nh):
                         softmax(hl, j)
-                pv_chunk(nck - 1)
-                flush()
+                    ready(j, "V")
+                    for hl in range(nh):
+                        issue_pv(hl, j)
+                    free(j, "V")
                 for hl in range(nh):
                     lsum = (lpair[hl][0] + lpair[hl][1]).astype(np.float32)
                     epilogue(tm, a2_o(hl), lsum, m_used[hl], rows, out, out_lo, part_o, part_lse, sp, h0 + hl,
@@ -575,24 +561,18 @@ def test_head_pair_kernel_replay_matches_the_oracle(case, force_pair):
     assert within(run_pair(c, force_pair=force_pair), oracle(c))
 
 
-@pytest.mark.parametrize("bug", ["p_lo_offset", "no_pv_first"])
+@pytest.mark.parametrize("bug", ["p_lo_offset", "k_free_after_first_head"])
 def test_planted_mistakes_in_the_head_pair_replay_are_caught(bug):
-    """A P lo block written half-way into the hi block, or the plain issue order where two
-    own-key chunks follow each other: either gives a wrong result or cannot proceed."""
-    c = build(5, 2, 1, 300, 0, 300, True)
+    """A P lo block written half-way into the hi block, or the K half-slots freed after the
+    first head's S MMAs (the load warp then fills them before the second head reads K):
+    either gives a wrong result or cannot proceed."""
+    c = build(6, 4, 2, 100, 200, 300, False)
+    assert within(run_pair(c, force_pair=True), oracle(c))
     try:
-        ok = within(run_pair(c, bug=bug), oracle(c))
+        ok = within(run_pair(c, bug=bug, force_pair=True), oracle(c))
     except AssertionError:
         ok = False
     assert not ok
-
-
-def test_a_single_s_p_buffer_in_the_head_pair_kernel_is_caught():
-    """One S/P buffer where the head-pair kernel keeps two: the next chunk's S lands while the
-    previous chunk's PV is still to read its P, which the replay's order allows."""
-    c = build(4, 2, 1, 128, 1536, 1664, False)
-    assert within(run_pair(c), oracle(c))
-    assert not within(run_pair(c, bug="one_sp_buffer"), oracle(c))
 
 
 @pytest.mark.parametrize("bug,case", [("no_p_wait", (4, 2, 1, 128, 1536, 1664, False)),

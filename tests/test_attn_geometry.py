@@ -43,9 +43,9 @@ def head_groups(nq, group, pair=True):
 
 
 def splits_pair(n_q, nq, group, n_keys, pair=True):
-    nch = cdiv(n_keys, 64)
+    nch = cdiv(n_keys, 128)
     s = NUM_SMS // (cdiv(n_q, 128) * head_groups(nq, group, pair))
-    s = max(min(s, MAX_SPLITS, nch // 4), 1)
+    s = max(min(s, MAX_SPLITS, nch // 2), 1)
     cps = cdiv(nch, s)
     return cdiv(nch, cps), cps
 
@@ -71,8 +71,25 @@ def debug_entry_accepts(n_q, pos0, n_keys, causal, cap, nq, nkv):
     return n_keys - (pos0 // 128) * 128 <= lo_rows(n_q)
 
 
+class HalfSlotPlan:
+    """The head-pair kernel's half-slot plan (HalfSlotPlan::take): a chunk's K parts, then
+    its V^T parts, each the next half-slot of the ring."""
+
+    def __init__(self, slots=3):
+        self.nxt, self.uses, self.slots = 0, [0] * slots, slots
+
+    def take(self, cur):
+        k, v = [], []
+        for lst in (k, v):
+            for _ in range(2 if cur else 1):
+                lst.append((self.nxt, self.uses[self.nxt]))
+                self.uses[self.nxt] += 1
+                self.nxt = (self.nxt + 1) % self.slots
+        return k, v
+
+
 class SlotPlan:
-    """The attention kernels' slot plan (SlotPlan::take, AtSlotPlan::take)."""
+    """The single-head kernel's slot plan (AtSlotPlan::take)."""
 
     def __init__(self, slots=3):
         self.nxt, self.uses, self.slots = 0, [0] * slots, slots
@@ -98,12 +115,12 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
     base = (pos0 // 128) * 128
     Lc = lo_rows(T)
     assert 0 <= n_keys - base <= Lc, "the low-term window exceeds the workspace's"
-    W = 64 if kernel == "pair" else 128
+    W = 128
     if kernel == "pair":
         pair, n_splits, cps = choose_pair(n_q, nq, group, n_keys)
         nh = 2 if pair else 1
         ys = head_groups(nq, group, pair)
-        smem_q, slot_bytes, slots = 2 * 4 * 16384, 32768, 3
+        smem_q, slot_bytes, slots = 2 * 4 * 16384, 32768, 3      # half-slots of 32 KB
         smem_total = 1024 + smem_q + slots * slot_bytes
         assert smem_total <= 227 * 1024 - 512
     else:
@@ -151,30 +168,39 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                         for r in rows:
                             assert ((sp * nq + h) * n_q + r + 1) * D <= part_o_len
                     continue
-                plan = SlotPlan()
+                plan = HalfSlotPlan() if kernel == "pair" else SlotPlan()
                 for j in range(nck):
                     key0 = (c_begin + j) * W
                     assert key0 < kv_end
                     cur = key0 >= base
-                    parts = plan.take(cur)
-                    for i, (s, _) in enumerate(parts):
-                        krow = key0 if i == 0 else key0 - base
-                        extent = n_keys if i == 0 else n_keys - base
-                        assert krow % W == 0
-                        check_tma(0, krow, 2, extent)           # K: x = d offset 0 / 64, y = key row
-                        check_tma(64, krow, 2, extent)
-                        check_tma(krow, 0, 2, extent + 1)       # V^T: x = key, y = d row 0
-                        assert krow < extent
-                        if kernel == "pair":
-                            assert s < slots and smem_q + (s + 1) * slot_bytes <= smem_total - 1024
-                        else:
+                    if kernel == "pair":
+                        k_parts, v_parts = plan.take(cur)
+                        for i, ((sk, _), (sv, _)) in enumerate(zip(k_parts, v_parts)):
+                            krow = key0 if i == 0 else key0 - base
+                            extent = n_keys if i == 0 else n_keys - base
+                            assert krow % W == 0 and krow < extent
+                            check_tma(0, krow, 2, extent)       # K blocks: x = d 0 / 64, y = key row
+                            check_tma(64, krow, 2, extent)
+                            check_tma(krow, 0, 2, extent + 1)   # V^T blocks: x = key, key + 64; y = d 0
+                            check_tma(krow + 64, 0, 2, extent + 64)
+                            for hs in (sk, sv):
+                                assert hs < slots and smem_q + (hs + 1) * slot_bytes <= smem_total - 1024
+                    else:
+                        parts = plan.take(cur)
+                        for i, (s, _) in enumerate(parts):
+                            krow = key0 if i == 0 else key0 - base
+                            extent = n_keys if i == 0 else n_keys - base
+                            assert krow % W == 0
+                            check_tma(0, krow, 2, extent)           # K: x = d offset 0 / 64, y = key row
+                            check_tma(64, krow, 2, extent)
+                            check_tma(krow, 0, 2, extent + 1)       # V^T: x = key, y = d row 0
+                            assert krow < extent
                             assert s < slots and (s + 1) * slot_bytes <= smem_total - 1024
                     chunks_seen += 1
                 if kernel == "pair":
                     for hl in range(nh):
-                        for b in range(2):
-                            assert hl * 256 + b * 64 + 64 <= 512
-                        assert hl * 256 + 128 + 128 <= 512
+                        assert hl * 256 + 128 <= 512           # S/P region: S 128 fp32, P hi 64 + lo 64
+                        assert hl * 256 + 128 + 128 <= 512     # O
                 for h in range(h0, h0 + nh):
                     for r in (rows[0], rows[-1]):
                         if n_splits == 1:
@@ -277,9 +303,9 @@ def test_debug_entries_refuse_a_low_term_window_past_the_workspace():
 @pytest.mark.parametrize("nck,cur_from", [(5, 2), (9, 0), (12, 8), (3, 3)])
 def test_kernel_slot_plan_is_the_simulated_one(nck, cur_from):
     import test_pipeline_protocol as TP
-    plan = SlotPlan()
+    plan = HalfSlotPlan()
     got = [plan.take(j >= cur_from) for j in range(nck)]
-    assert got == [list(map(tuple, x)) for x in TP.slot_plan(nck, cur_from, 3)]
+    assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, 3)]
 
 
 def test_splits_fill_about_one_wave():

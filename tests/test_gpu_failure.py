@@ -27,7 +27,9 @@ TIMEOUT_CODES = (1, 2, 3, 4)
 
 
 def _gemm_case(dg, g):
-    K, M, n = 256, 384, 70
+    # long enough that the epilogue's first wait (for the first tile's MMAs over 128
+    # k-blocks) lasts tens of microseconds, far beyond the timer's resolution
+    K, M, n = 8192, 2048, 70
     W = (torch.randn(1, M, K, generator=g, device="cuda") * 0.05).to(torch.bfloat16)
     X = torch.randn(n, K, generator=g, device="cuda").to(torch.bfloat16)
     out = torch.full((n, M), float("nan"), device="cuda")

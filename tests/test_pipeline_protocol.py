@@ -371,6 +371,21 @@ def test_the_checker_catches_a_wrong_count():
 
 # ---------------------------------------------------------------- the attention kernel (k_tc_attn.cu)
 
+def slot_plan(nck, cur_from, slots):
+    """Slots of each chunk (tc_attn_kernel): a cached chunk takes the next slot, a current
+    chunk (the call's own keys: hi and lo parts) the next two; returns [(slots of chunk j,
+    use index of each)]."""
+    nxt, uses, plan = 0, [0] * slots, []
+    for j in range(nck):
+        k = 2 if j >= cur_from else 1
+        ss = [(nxt + i) % slots for i in range(k)]
+        plan.append([(x, uses[x]) for x in ss])
+        for x in ss:
+            uses[x] += 1
+        nxt = (nxt + k) % slots
+    return plan
+
+
 def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, flags=None, give_up_at=None,
               drain=True, load_drain=True, p_wait=True):
     """tc_attn_kernel's hand-offs: the softmax warps store the query tile in TMEM and signal
@@ -812,47 +827,52 @@ def test_fused_epilogue_warps_leave_together_on_a_timeout():
 
 # ---------------------------------------------------------------- the attention redesign (on paper)
 
-def slot_plan(nck, cur_from, slots):
-    """Slots of each chunk: a cached chunk takes the next slot, a current chunk (the call's
-    own keys: hi and lo parts) the next two; returns [(slots of chunk j, use index of each)]."""
+def half_slot_plan(nck, cur_from, slots):
+    """The head-pair kernel's ring: chunk j takes the next one half-slot (cached keys) or
+    two (own keys: hi and lo parts) for its K, then as many for its V^T; returns
+    [(K parts, V parts)], each part (half-slot, its use index)."""
     nxt, uses, plan = 0, [0] * slots, []
     for j in range(nck):
-        k = 2 if j >= cur_from else 1
-        ss = [(nxt + i) % slots for i in range(k)]
-        plan.append([(x, uses[x]) for x in ss])
-        for x in ss:
-            uses[x] += 1
-        nxt = (nxt + k) % slots
+        n = 2 if j >= cur_from else 1
+        parts = []
+        for _ in range(2):
+            lst = []
+            for _ in range(n):
+                lst.append((nxt, uses[nxt]))
+                uses[nxt] += 1
+                nxt = (nxt + 1) % slots
+            parts.append(lst)
+        plan.append(tuple(parts))
     return plan
 
 
-def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_first_rule=True, flags=None,
-                        give_up_at=None, final_slot_commits=False, drain=True, load_drain=True):
-    """The head-pair attention kernel's hand-offs: a load warp fills `slots` K/V slots; the
-    MMA warp issues S_A(j), S_B(j) into S/P buffer j & 1 of each head, then PV_A(j-1),
-    PV_B(j-1), then frees chunk j-1's slots with a commit; each head's softmax warps read
-    S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  Before S_h(j)
-    reuses buffer j & 1, the MMA warp waits for PV_h(j-2), the last reader of that P.
-    When chunks j-1 and j together need more slots than the ring has (two current chunks
-    in three slots), chunk j cannot load before chunk j-1's slots are free, so the MMA
-    warp issues PV(j-1) before S(j) (`pv_first_rule`; without it that case deadlocks).
-    The last chunk's slots get no release commit (`final_slot_commits` adds them) and the
-    MMA warp drains its commits before the CTA leaves (`drain`).
+def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, flags=None, give_up_at=None,
+                        drain=True, load_drain=True, bug=None):
+    """The head-pair attention kernel's hand-offs (128-key chunks): a load warp fills a ring
+    of `slots` half-slots, each chunk's K then its V^T; per chunk the MMA warp issues S_A(j),
+    S_B(j) -- each once PV(j-1) of its head has completed, since S overwrites the head's one
+    S/P region -- commits the K half-slots free, then PV_A(j), PV_B(j) once each head's
+    softmax warps have written P(j), and commits the V half-slots free.  Each head's softmax
+    warps read S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  The MMA
+    warp drains its commits before the CTA leaves (`drain`).
+
+    bug: "no_pv_wait" -- S(j) issued without waiting for PV(j-1); "k_free_early" -- the K
+    half-slots freed after the first head's S.
 
     flags: abort mode -- every bounded wait also passes once flags["abort"] is set, the
     give_up_at-th wait raises it (a timeout), a role whose wait failed leaves its loop,
     and the load warp then waits for the loads it issued (`load_drain`)."""
     rng = random.Random(seed * 104729 + nck)
-    plan = slot_plan(nck, nck if cur_from is None else cur_from, slots)
-    kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
-    kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
+    plan = half_slot_plan(nck, nck if cur_from is None else cur_from, slots)
+    hs_full = [Barrier(f"hs_full{s}", 1) for s in range(slots)]
+    hs_free = [Barrier(f"hs_free{s}", 1) for s in range(slots)]
     drain_bar = Barrier("drain", 1)
     H = 2
-    s_full = [[Barrier(f"s_full{h}{b}", 1) for b in range(2)] for h in range(H)]
-    p_ready = [[Barrier(f"p_ready{h}{b}", warps_per_head) for b in range(2)] for h in range(H)]
-    pv_done = [[Barrier(f"pv_done{h}{b}", 1) for b in range(2)] for h in range(H)]
+    s_full = [Barrier(f"s_full{h}", 1) for h in range(H)]
+    p_ready = [Barrier(f"p_ready{h}", warps_per_head) for h in range(H)]
+    pv_done = [Barrier(f"pv_done{h}", 1) for h in range(H)]
     bufs, q = Buffers(), Async()
-    st = {"pv_done": [0, 0], "pv_issued": [0, 0], "s_done": [0, 0]}
+    st = {"pv_done": [0, 0], "pv_issued": [0, 0]}
     p_writes = {}
     steps = [0]
 
@@ -872,106 +892,107 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_
         loaded = [0] * slots
         ok = True
         for j in range(nck):
-            for s, u in plan[j]:
-                if u >= 1:
-                    yield bw(kv_free[s], (u & 1) ^ 1, u - 1)
-                    if not passed(kv_free[s], (u & 1) ^ 1):
-                        ok = False
-                        break
-                bufs.fill(("slot", s), 2 * H)         # S_A, S_B, PV_A, PV_B of chunk j read it
-                kv_full[s].arrive_expect_tx(32)
-                q.loads.append(lambda s=s: kv_full[s].complete_tx(32))
-                loaded[s] += 1
+            for parts in plan[j]:
+                for s, u in parts:
+                    if u >= 1:
+                        yield bw(hs_free[s], (u - 1) & 1, u - 1)
+                        if not passed(hs_free[s], (u - 1) & 1):
+                            ok = False
+                            break
+                    bufs.fill(("hs", s), H)           # K: S_A and S_B read it; V^T: PV_A and PV_B
+                    hs_full[s].arrive_expect_tx(32)
+                    q.loads.append(lambda s=s: hs_full[s].complete_tx(32))
+                    loaded[s] += 1
+                if not ok:
+                    break
             if not ok:
                 break
         if flags is not None and flags["abort"] and load_drain:
-            for s in range(slots):                    # the wind-down: the last load of each slot
+            for s in range(slots):                    # the wind-down: the last load of each half-slot
                 if loaded[s]:
-                    yield wait(kv_full[s], (loaded[s] - 1) & 1, None)
+                    yield wait(hs_full[s], (loaded[s] - 1) & 1, None)
 
     def mma():
-        def issue_pv(h, k):
-            assert p_writes.get((h, k & 1)) == (k, warps_per_head), "PV read a P not fully written"
-            st["pv_issued"][h] += 1
-
-            def done(h=h, k=k):
-                st["pv_done"][h] += 1
-                for w in range(warps_per_head):       # every warp's lanes of P(k) were read
-                    bufs.release(("sp", h, k & 1, w))
-                for x, _ in plan[k]:
-                    bufs.release(("slot", x))
-                pv_done[h][k & 1].arrive()
-            q.mma.append(done)
-
-        def pv_chunk(k):
-            for h in range(H):
-                yield bw(p_ready[h][k & 1], (k >> 1) & 1, k >> 1)
-                if not passed(p_ready[h][k & 1], (k >> 1) & 1):
-                    return False
-                issue_pv(h, k)
-            if k + 1 < nck or final_slot_commits:     # one commit per slot of chunk k
-                for x, _ in plan[k]:
-                    q.mma.append(lambda x=x: kv_free[x].arrive())
-            return True
-
         ok = True
         for j in range(nck):
-            pv_first = pv_first_rule and j >= 1 and len(plan[j - 1]) + len(plan[j]) > slots
-            if pv_first:
-                ok = yield from pv_chunk(j - 1)
-                if not ok:
-                    break
-            for x, u in plan[j]:
-                yield bw(kv_full[x], u & 1, u)
-                if not passed(kv_full[x], u & 1):
+            k_parts, v_parts = plan[j]
+            for x, u in k_parts:
+                yield bw(hs_full[x], u & 1, u)
+                if not passed(hs_full[x], u & 1):
                     ok = False
                     break
             for h in range(H):
                 if not ok:
                     break
-                if j >= 2:
-                    yield bw(pv_done[h][j & 1], ((j >> 1) - 1) & 1, (j >> 1) - 1)
-                    if not passed(pv_done[h][j & 1], ((j >> 1) - 1) & 1):
+                if j >= 1 and bug != "no_pv_wait":
+                    yield bw(pv_done[h], (j - 1) & 1, j - 1)
+                    if not passed(pv_done[h], (j - 1) & 1):
                         ok = False
                         break
                 for w in range(warps_per_head):       # S: each warp reads its own 32 lanes
-                    bufs.fill(("sp", h, j & 1, w), 1)
+                    bufs.fill(("sp", h, w), 1)
 
                 def s_done(h=h, j=j):
-                    st["s_done"][h] += 1
-                    for x, _ in plan[j]:
-                        bufs.release(("slot", x))
-                    s_full[h][j & 1].arrive()
+                    for x, _ in plan[j][0]:
+                        bufs.release(("hs", x))
+                    s_full[h].arrive()
                 q.mma.append(s_done)
+                if bug == "k_free_early" and h == 0:
+                    for x, _ in k_parts:
+                        q.mma.append(lambda x=x: hs_free[x].arrive())
             if not ok:
                 break
-            if j >= 1 and not pv_first:
-                ok = yield from pv_chunk(j - 1)
+            if bug != "k_free_early":
+                for x, _ in k_parts:                  # one commit per K half-slot
+                    q.mma.append(lambda x=x: hs_free[x].arrive())
+            for x, u in v_parts:
+                yield bw(hs_full[x], u & 1, u)
+                if not passed(hs_full[x], u & 1):
+                    ok = False
+                    break
+            for h in range(H):
                 if not ok:
                     break
-        if ok:
-            yield from pv_chunk(nck - 1)
+                yield bw(p_ready[h], j & 1, j)
+                if not passed(p_ready[h], j & 1):
+                    ok = False
+                    break
+                assert p_writes.get(h) == (j, warps_per_head), "PV read a P not fully written"
+                st["pv_issued"][h] += 1
+
+                def pv_fin(h=h, j=j):
+                    st["pv_done"][h] += 1
+                    for w in range(warps_per_head):   # every warp's lanes of P(j) were read
+                        bufs.release(("sp", h, w))
+                    for x, _ in plan[j][1]:
+                        bufs.release(("hs", x))
+                    pv_done[h].arrive()
+                q.mma.append(pv_fin)
+            if not ok:
+                break
+            for x, _ in v_parts:                      # one commit per V^T half-slot
+                q.mma.append(lambda x=x: hs_free[x].arrive())
         if drain:                                     # every commit issued above has landed
             q.mma.append(lambda: drain_bar.arrive())
             yield wait(drain_bar, 0, 0)
 
     def softmax(h, w):
         for j in range(nck):
-            yield bw(s_full[h][j & 1], (j >> 1) & 1, j >> 1)
-            if not passed(s_full[h][j & 1], (j >> 1) & 1):
+            yield bw(s_full[h], j & 1, j)
+            if not passed(s_full[h], j & 1):
                 return
-            bufs.release(("sp", h, j & 1, w))          # this warp's lanes of S read into registers
-            if j > 0 and rng.random() < 0.4:           # the row max grew: rescale O after PV(j-1)
-                yield bw(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1, (j - 1) >> 1)
-                if not passed(pv_done[h][(j - 1) & 1], ((j - 1) >> 1) & 1):
+            bufs.release(("sp", h, w))                # this warp's lanes of S read into registers
+            if j > 0 and rng.random() < 0.4:          # the row max grew: rescale O after PV(j-1)
+                yield bw(pv_done[h], (j - 1) & 1, j - 1)
+                if not passed(pv_done[h], (j - 1) & 1):
                     return
                 assert st["pv_done"][h] >= j and st["pv_issued"][h] <= j, "O rescaled while a PV may write it"
-            bufs.fill(("sp", h, j & 1, w), 1)         # P over this warp's lanes of S, read by PV(j)
-            last, n = p_writes.get((h, j & 1), (None, 0))
-            p_writes[(h, j & 1)] = (j, 1) if last != j else (j, n + 1)
-            p_ready[h][j & 1].arrive()
-        yield bw(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1, (nck - 1) >> 1)
-        if passed(pv_done[h][(nck - 1) & 1], ((nck - 1) >> 1) & 1):
+            bufs.fill(("sp", h, w), 1)                # P over this warp's lanes of S, read by PV(j)
+            last, n = p_writes.get(h, (None, 0))
+            p_writes[h] = (j, 1) if last != j else (j, n + 1)
+            p_ready[h].arrive()
+        yield bw(pv_done[h], (nck - 1) & 1, nck - 1)
+        if passed(pv_done[h], (nck - 1) & 1):
             assert st["pv_done"][h] == nck
 
     roles = {"load": load(), "mma": mma()}
@@ -981,38 +1002,40 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, pv_
 
 
 @pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (3, 3), (4, 2), (7, 7), (7, 4), (12, 8), (6, 0)])
-def test_attention_redesign_protocol(nck, cur_from):
-    """The protocol planned for the attention redesign, cached chunks in one slot and the
-    call's own (current) chunks in two: no deadlock, no overrun, no buffer refilled while
-    read, no P read before all its writers, no O rescaled under a PV."""
+def test_head_pair_attention_protocol(nck, cur_from):
+    """Cached chunks in one half-slot per operand, the call's own (current) chunks in two:
+    no deadlock, no overrun, no buffer refilled while read, no P read before all its
+    writers, no O rescaled under a PV."""
     for seed in range(40):
         roles, q = attention_two_heads(nck, seed, cur_from=cur_from)
         run(roles, q, seed, end_check=True)
 
 
-def test_attention_redesign_needs_pv_first_for_two_current_chunks():
-    """Two current chunks in a row hold four slots of three if S(j) runs before PV(j-1):
-    the simulator finds the deadlock the issue-order rule avoids."""
-    with pytest.raises(AssertionError, match="deadlock"):
-        roles, q = attention_two_heads(4, 0, cur_from=2, pv_first_rule=False)
-        run(roles, q, 0)
-    # one current chunk after cached ones fits: the rule never fires there
-    for seed in range(20):
-        roles, q = attention_two_heads(5, seed, cur_from=4, pv_first_rule=False)
-        run(roles, q, seed)
+@pytest.mark.parametrize("bug", ["no_pv_wait", "k_free_early"])
+def test_head_pair_attention_protocol_catches_its_planted_mistakes(bug):
+    """S(j) issued before PV(j-1) has read P(j-1) from the same TMEM region, or the K
+    half-slots freed before the second head's S: some interleaving overwrites a buffer that
+    is still read."""
+    caught = 0
+    for seed in range(80):
+        roles, q = attention_two_heads(6, seed, cur_from=4, bug=bug)
+        try:
+            run(roles, q, seed, end_check=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
-def test_attention_redesign_leaves_nothing_in_flight():
+def test_head_pair_attention_leaves_nothing_in_flight():
     """When the last role leaves, no MMA completion or commit may still be pending (it would
-    arrive on released shared memory).  With the drain that holds in every interleaving;
-    the earlier design -- release commits for the last chunk's slots and no drain on the
-    normal path -- leaves commits behind in some."""
+    arrive on released shared memory): the MMA warp's drain makes that hold in every
+    interleaving; without it some interleaving leaves a commit behind."""
     for seed in range(60):
         roles, q = attention_two_heads(6, seed, cur_from=4)
         run(roles, q, seed, end_check=True)
     left = 0
     for seed in range(60):
-        roles, q = attention_two_heads(6, seed, cur_from=4, final_slot_commits=True, drain=False)
+        roles, q = attention_two_heads(6, seed, cur_from=4, drain=False)
         try:
             run(roles, q, seed, end_check=True)
         except AssertionError as e:
@@ -1021,7 +1044,7 @@ def test_attention_redesign_leaves_nothing_in_flight():
 
 
 @pytest.mark.parametrize("nck,cur_from", [(4, 2), (7, 4), (6, 0)])
-def test_attention_redesign_winds_down_after_a_timeout(nck, cur_from):
+def test_head_pair_attention_winds_down_after_a_timeout(nck, cur_from):
     """A bounded wait gives up at a random point: every role leaves (no deadlock), and with
     the load warp's drain and the MMA warp's drain nothing is in flight when they have.
     Without the load drain, some timeout leaves a load landing after the CTA is gone."""
