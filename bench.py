@@ -627,7 +627,7 @@ def run_chained(args, cfg, name):
     return 0
 
 
-def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None, expert_bytes=None):
+def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None, expert_bytes=None, fused=False):
     """Achieved rate and fraction of its bound for each big kernel of the step: the expert
     and vocabulary GEMMs and the update statistics against HBM bandwidth (algorithmic
     bytes per launch), attention against the bf16 tensor peak (algorithmic FLOPs).
@@ -647,8 +647,12 @@ def kernel_rooflines(cfg, P, C, unions, kern, hbm, tf_peak, peak_src, rows=None,
                         "gemm_down": sum(RF.down_bytes(cfg, u, rows * k) for u in unions) / L}
     for kname, nb in expert_bytes.items():
         hbm_entry(kname, nb)
-    hbm_entry("gemm_vocab", RF.vocab_bytes(cfg, rows))
-    hbm_entry("update_partial", RF.update_bytes(cfg, rows))
+    if fused:   # the vocabulary GEMM writes tile records; the row merge reads them
+        hbm_entry("gemm_vocab", RF.vocab_bytes(cfg, rows) - 4 * rows * cfg["vocab"] + RF.update_record_bytes(cfg, rows))
+        hbm_entry("update_partial", RF.update_record_bytes(cfg, rows))
+    else:
+        hbm_entry("gemm_vocab", RF.vocab_bytes(cfg, rows))
+        hbm_entry("update_partial", RF.update_bytes(cfg, rows))
     if "attention" in kern:
         fl = RF.attention_flops(cfg, P, C)
         a = fl / (kern["attention"]["avg_us"] * 1e-6) / 1e12
@@ -818,9 +822,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per pass (each its own request and cache) through the batched calls")
-    ap.add_argument("--fused-update", action="store_true",
-                    help="one call per step: the pass with the update's statistics as the vocabulary "
-                         "projection's epilogue (no logits)")
+    ap.add_argument("--update", choices=["fused", "two-call"], default="fused",
+                    help="fused (default): one call per step, the pass with the update's statistics as the "
+                         "vocabulary projection's epilogue (no logits); two-call: dg_denoise_pass writes the "
+                         "logits and dg_canvas_update reads them (always so for several canvases or 8/4-bit "
+                         "weights)")
     ap.add_argument("--experts", default="bf16", choices=["bf16", "mx8", "nv4"],
                     help="expert weight storage; mx8 and nv4 run through the batched calls")
     ap.add_argument("--vocab", default="bf16", choices=["bf16", "mx8", "nv4"],
@@ -852,9 +858,10 @@ def main():
         return run_chained(args, cfg, name)
     if args.canvases < 1:
         ap.error("--canvases must be >= 1")
-    if args.fused_update and (args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16"):
-        ap.error("--fused-update runs one canvas with bf16 experts and output matrix")
-    if args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16" or args.fused_update:
+    variant = args.canvases > 1 or args.experts != "bf16" or args.vocab != "bf16"
+    # the fused call runs one canvas with bf16 experts and output matrix
+    args.fused_update = args.update == "fused" and not variant
+    if variant:
         return run_variant(args, cfg, name)
 
     import torch
@@ -880,13 +887,22 @@ def main():
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
 
-    # every step denoises the same input canvas; the update writes a second buffer
-    canvas_in = canvas
-    canvas_out = torch.empty_like(canvas)
+    fused = args.fused_update
+    if fused:
+        # one call per step reads the canvas and writes the updated one in place: each step
+        # denoises the previous step's result (the same shapes and work every step)
+        canvas_in = canvas_out = canvas
 
-    def step(s):
-        dg.denoise_pass(model, cache, canvas_in, logits, ws)
-        dg.canvas_update(logits, n_ren, synth.SEED_RENOISE, s, canvas_out, ws)
+        def step(s):
+            dg.denoise_update(model, cache, canvas, n_ren, ws, seed=synth.SEED_RENOISE, step=s)
+    else:
+        # every step denoises the same input canvas; the update writes a second buffer
+        canvas_in = canvas
+        canvas_out = torch.empty_like(canvas)
+
+        def step(s):
+            dg.denoise_pass(model, cache, canvas_in, logits, ws)
+            dg.canvas_update(logits, n_ren, synth.SEED_RENOISE, s, canvas_out, ws)
 
     # expert union per layer of this input (read once, outside the timed region)
     unions = torch.zeros(cfg["n_layers"], dtype=torch.int32, device=dev)
@@ -1007,13 +1023,16 @@ def main():
     # whole-pass roofline (slower of FLOPs at the bf16 peak and bytes at HBM bandwidth)
     flops = RF.pass_flops(cfg, P, C)
     # the pass's bytes already hold the logits' write and the update's read of them; the
-    # update adds its canvas in / out
+    # update adds its canvas in / out; the fused step writes and reads 16-byte tile records
+    # (one per token and 128 vocabulary ids) instead of the logits
     nbytes = RF.pass_bytes(cfg, P, C, unions_h) + 8 * C
+    if fused:
+        nbytes += 2 * RF.update_record_bytes(cfg, C) - 2 * 4 * C * V
     t_roof = RF.time_bound(flops, nbytes, tf_burst * 1e12, hbm * 1e9)
     # every big kernel against its own bound: algorithmic units per launch / average
     # CUDA-event duration of its launches inside the step (the per-layer expert union
     # varies, so the expert GEMMs' bytes per launch are the layers' average)
-    kroof = kernel_rooflines(cfg, P, C, unions_h, kern, hbm, tf_sust, peak_src)
+    kroof = kernel_rooflines(cfg, P, C, unions_h, kern, hbm, tf_sust, peak_src, fused=fused)
     # the dominant kernel (largest share of the step) is the line's roofline
     roof = None
     if kroof:
@@ -1026,7 +1045,9 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": _workload_desc(name, cfg), "l2": "flushed between steps (256 MB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "attention": _attention_kind(), "expert_union": unions_h},
+                   "attention": _attention_kind(), "expert_union": unions_h,
+                   "update": "fused into the vocabulary projection (one call per step)" if fused
+                   else "two calls: logits written, then read by the update"},
         "roofline": roof,
         "pass_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof * 1e3 / ms_step, "flops": flops,
                           "bytes": nbytes, "bound": "hbm" if nbytes / (hbm * 1e9) > flops / (tf_burst * 1e12)
@@ -1035,7 +1056,8 @@ def main():
         "kernel_rooflines": kroof,
         "step_median_us": step_median_us,
         "step_p10_p90_us": [step_p10_us, step_p90_us],
-        "pass_only_us": {"median": statistics.median(pass_us), "mean": sum(pass_us) / len(pass_us), "steps": k2},
+        "pass_only_us": {"median": statistics.median(pass_us), "mean": sum(pass_us) / len(pass_us), "steps": k2,
+                         "note": "dg_denoise_pass alone (logits written), no update"},
         "graph_step_us": graph,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": C * 4, "d2h_bytes_per_step": C * 4},
         "gpu_launches": launches,

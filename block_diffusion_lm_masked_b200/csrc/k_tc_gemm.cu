@@ -42,15 +42,23 @@ constexpr int TC_THREADS = 192;
 
 // The k-block buffers' offsets in the ring, in the order both the producer and the MMA
 // warp walk the k-blocks: a buffer starts where the previous one ended, or at 0 when it
-// would run past the end.  Sizes are multiples of 2 KB, so every buffer (and each box
-// in it) starts on a 1024-byte swizzle atom.
+// would run past the end (the skipped tail then counts in its footprint).  Buffers are
+// released in allocation order, so the bytes in use are the footprints of the k-blocks in
+// flight, and a new buffer overlaps none of them exactly when that sum stays within the
+// ring.  Sizes are multiples of 2 KB, so every buffer (and each box in it) starts on a
+// 1024-byte swizzle atom.
 struct KbRing {
   uint32_t cap, head;
   __device__ explicit KbRing(uint32_t c) : cap(c), head(0) {}
-  __device__ uint32_t take(uint32_t bytes) {
-    const uint32_t off = head + bytes > cap ? 0u : head;
-    head = off + bytes;
-    return off;
+  __device__ uint32_t take(uint32_t bytes, uint32_t* foot) {
+    if (head + bytes > cap) {
+      *foot = cap - head + bytes;
+      head = bytes;
+      return 0u;
+    }
+    *foot = bytes;
+    head += bytes;
+    return head - bytes;
   }
 };
 
@@ -133,6 +141,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ int n_issued_s, n_consumed_s;
+  __shared__ uint32_t kb_foot[TC_MAX_STAGES];  // ring footprint of each k-block in flight (producer only)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int terms = p.two_terms ? 2 : 1;
@@ -183,8 +192,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prefetch_tmap(&tmB2b);
       }
       int it = 0, t;
-      int released = 0;  // k-blocks whose buffers the MMAs have released (in order)
-      uint32_t q_off[TC_MAX_STAGES], q_len[TC_MAX_STAGES];  // buffers of k-blocks released .. it - 1
+      int released = 0;     // k-blocks whose buffers the MMAs have released (in order)
+      uint32_t in_use = 0;  // ring bytes of the k-blocks released .. it - 1 (footprints)
       bool ok = true;
       KbRing ring((uint32_t)p.smem_budget);
       TileWalk walk(p, n_tiles);
@@ -194,24 +203,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t tx = kb_bytes(n_pad);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % TC_MAX_STAGES;
-          const uint32_t off = ring.take(tx);
-          // wait for the oldest k-blocks until none in flight overlaps this buffer and
-          // fewer than TC_MAX_STAGES are in flight (buffers are released in order)
-          while (released < it) {
-            bool clash = it - released >= TC_MAX_STAGES;
-            for (int q = released; q < it && !clash; ++q)
-              clash = off < q_off[q % TC_MAX_STAGES] + q_len[q % TC_MAX_STAGES] && q_off[q % TC_MAX_STAGES] < off + tx;
-            if (!clash) break;
+          uint32_t foot;
+          const uint32_t off = ring.take(tx, &foot);
+          in_use += foot;
+          // wait for the oldest k-blocks until this buffer fits beside those still in flight
+          // and fewer than TC_MAX_STAGES are in flight
+          while (released < it && (in_use > (uint32_t)p.smem_budget || it - released >= TC_MAX_STAGES)) {
             if (!mbar_wait(&empty_bar[released % TC_MAX_STAGES], (uint32_t)(released / TC_MAX_STAGES) & 1u, &abort_s,
                            p.err, DG_DEVERR_TIMEOUT_EMPTY)) {
               ok = false;
               break;
             }
+            in_use -= kb_foot[released % TC_MAX_STAGES];
             ++released;
           }
           if (!ok) break;
-          q_off[s] = off;
-          q_len[s] = tx;
+          kb_foot[s] = foot;
           uint8_t* sa = smem + off;
           uint8_t* sb = sa + n_a * a_bytes;
           const int kx = (ti.split * nkb + (kb + t) % nkb) * TC_BK;
@@ -253,7 +260,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t tx = kb_bytes(n_pad);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % TC_MAX_STAGES;
-          const uint32_t off = ring.take(tx);
+          uint32_t foot;
+          const uint32_t off = ring.take(tx, &foot);
           if (!mbar_wait(&full_bar[s], (uint32_t)(it / TC_MAX_STAGES) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_FULL)) {
             ok = false;
             break;

@@ -315,18 +315,36 @@ __global__ void __launch_bounds__(VU_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 }
 
-// one warp per token: its tile records merged in id order (lane l takes tiles l, l + 32,
-// ...; then the lanes in a fixed butterfly), one record out
-__global__ void upd_merge_rows_kernel(const UpdPart* __restrict__ part, int C, int tiles, UpdPart* __restrict__ out) {
+// One CTA of UM_THREADS threads per token: thread t merges the token's tile records t,
+// t + UM_THREADS, ... in id order (UM_BATCH loads in flight before the merges), each
+// warp combines its lanes in a fixed butterfly, and thread 0 merges the warps' records
+// in warp order: one record out.  (One warp per token, one load in flight per lane, left
+// each lane 64 dependent loads at the large vocabulary.)
+constexpr int UM_THREADS = 128;
+constexpr int UM_BATCH = 8;
+__global__ void __launch_bounds__(UM_THREADS) upd_merge_rows_kernel(const UpdPart* __restrict__ part, int C,
+                                                                    int tiles, UpdPart* __restrict__ out) {
   griddep_sync();
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  __shared__ UpdPart wrec[UM_THREADS / 32];
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (row >= C) return;
+  const UpdPart* pr = part + (size_t)row * tiles;
   float m = -INFINITY, s = 0.0f, m2 = -INFINITY;
   int a = 0x7fffffff;
-  for (int t = lane; t < tiles; t += 32) {
-    const UpdPart x = part[(size_t)row * tiles + t];
-    vu_ms_merge(m, s, x.m, x.s);
-    vu_cand_merge(m2, a, x.m2, x.a);
+  for (int t0 = tid; t0 < tiles; t0 += UM_THREADS * UM_BATCH) {
+    UpdPart x[UM_BATCH];
+#pragma unroll
+    for (int i = 0; i < UM_BATCH; ++i) {
+      const int t = t0 + i * UM_THREADS;
+      if (t < tiles) x[i] = pr[t];
+    }
+#pragma unroll
+    for (int i = 0; i < UM_BATCH; ++i) {
+      if (t0 + i * UM_THREADS < tiles) {
+        vu_ms_merge(m, s, x[i].m, x[i].s);
+        vu_cand_merge(m2, a, x[i].m2, x[i].a);
+      }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -343,6 +361,15 @@ __global__ void upd_merge_rows_kernel(const UpdPart* __restrict__ part, int C, i
     r.s = s;
     r.a = a;
     r.m2 = m2;
+    wrec[warp] = r;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    UpdPart r = wrec[0];
+    for (int w = 1; w < UM_THREADS / 32; ++w) {
+      vu_ms_merge(r.m, r.s, wrec[w].m, wrec[w].s);
+      vu_cand_merge(r.m2, r.a, wrec[w].m2, wrec[w].a);
+    }
     out[row] = r;
   }
 }
@@ -363,7 +390,7 @@ cudaError_t launch_vocab_update(const CUtensorMap& A, const CUtensorMap& B, cons
 
 cudaError_t launch_upd_merge_rows(const UpdPart* part, int C, int tiles, UpdPart* out, cudaStream_t st) {
   if (C <= 0) return cudaSuccess;
-  return launch_k(upd_merge_rows_kernel, dim3((C + 7) / 8), dim3(256), 0, st, part, C, tiles, out);
+  return launch_k(upd_merge_rows_kernel, dim3(C), dim3(UM_THREADS), 0, st, part, C, tiles, out);
 }
 
 cudaError_t set_wait_limit_vocab_update(uint64_t ns) { return set_wait_limit_this_file(ns); }

@@ -59,6 +59,11 @@ def update_bytes(cfg: dict, C: int) -> int:
     return 4 * C * cfg["vocab"] + 8 * C
 
 
+def update_record_bytes(cfg: dict, C: int) -> int:
+    """The fused update's tile records: one 16-byte record per token and 128 vocabulary ids."""
+    return 16 * C * ((cfg["vocab"] + 127) // 128)
+
+
 def attention_flops(cfg: dict, P: int, C: int) -> float:
     """Canvas queries over P + C keys: QK^T and PV, per layer."""
     return 4.0 * C * cfg["n_q_heads"] * cfg["head_dim"] * (P + C)

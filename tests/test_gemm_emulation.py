@@ -98,22 +98,27 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
         sm, tm = T.Smem(smem_budget), T.Tmem(tmem_cols)
         tiles = tile_walk(cta, grid, n_tiles, m_tiles, rows_a, tile_rows)
         its = [(t, kb) for t in tiles for kb in range(nkb)]
-        offs, head = [], 0                    # KbRing: each k-block's buffer offset and size
+        offs, foots, head = [], [], 0         # KbRing: each k-block's offset, size and footprint
         for t, _ in its:
             n = kb_bytes(t)
-            off = 0 if head + n > smem_budget else head
-            head = off + n
+            if head + n > smem_budget:
+                foots.append(smem_budget - head + n)
+                off, head = 0, n
+            else:
+                foots.append(n)
+                off, head = head, head + n
             offs.append((off, n))
         loaded = mma_done = 0
         pending = []
 
         def can_load(it):
-            """No k-block in flight (loaded, not yet consumed) overlaps this buffer, and
-            fewer than 16 are in flight."""
+            """The buffer's footprint fits beside those of the k-blocks in flight (loaded, not
+            yet consumed), and fewer than 16 are in flight."""
+            if it == mma_done:                 # nothing in flight: the producer waits for nothing
+                return True
             if it - mma_done >= 16:
                 return False
-            off, n = offs[it]
-            return all(off + n <= o or o + m <= off for o, m in offs[mma_done:it])
+            return sum(foots[mma_done:it + 1]) <= smem_budget
 
         def load(it):
             t, kb = its[it]

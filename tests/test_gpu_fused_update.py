@@ -44,7 +44,8 @@ def _both(dg, st, canvas_np, n, mask_id=-1, step=3):
     return (a.cpu().numpy(), ca.cpu().numpy(), logits.cpu().numpy()), (b.cpu().numpy(), cb.cpu().numpy())
 
 
-@pytest.mark.parametrize("cfg,P,C", [(SMALL_BF16, 200, 100), (SMALL_BF16, 0, 37), (CF.CONFIGS["layer1_bf16"], 1024, 256)])
+@pytest.mark.parametrize("cfg,P,C", [(SMALL_BF16, 200, 100), (SMALL_BF16, 0, 37), (CF.CONFIGS["layer1_bf16"], 1024, 256),
+                                     (CF.CONFIGS["large4_bf16"], 32768, 256)])
 def test_fused_update_equals_the_two_call_path(dg, cfg, P, C):
     """The same accumulators feed both paths, so ids agree exactly and confidences to fp32
     summation order; the re-noise sets agree except where two confidences are that close."""

@@ -145,7 +145,8 @@ def bf16_gemm(tile_bytes, nkb, cap, slots=16, nbuf=2, bug=None):
     padded rows); cap: the ring's bytes; slots: barrier pairs (k-blocks in flight at most);
     nbuf: accumulator buffers (one where two do not fit in TMEM: paired weight tiles of
     256 token columns).  The producer allocates each k-block's buffer from the ring (KbRing)
-    and waits for the oldest k-blocks until none in flight overlaps it."""
+    and waits for the oldest k-blocks until its footprint fits beside theirs (buffers are
+    released in allocation order, so that is exactly when it overlaps none of them)."""
     n_tiles = len(tile_bytes)
     full = [Barrier(f"full{s}", 1) for s in range(slots)]
     empty = [Barrier(f"empty{s}", 1) for s in range(slots)]
@@ -155,35 +156,34 @@ def bf16_gemm(tile_bytes, nkb, cap, slots=16, nbuf=2, bug=None):
     acc_done = {}
 
     def ring():
+        """KbRing::take: (offset, bytes, footprint incl. a skipped tail)."""
         head = 0
         for t in range(n_tiles):
             for _ in range(nkb):
                 n = tile_bytes[t]
-                off = 0 if head + n > cap else head
-                head = off + n
-                yield off, n
+                if head + n > cap:
+                    foot, off, head = cap - head + n, 0, n
+                else:
+                    foot, off, head = n, head, head + n
+                yield off, n, foot
 
     def producer():
-        released, inflight = 0, {}
-        for it, (off, n) in enumerate(ring()):
+        released, in_use, foot_of = 0, 0, {}
+        for it, (off, n, foot) in enumerate(ring()):
             s = it % slots
-            while released < it:
-                clash = it - released >= slots
-                if bug != "no_overlap_check":
-                    clash = clash or any(off < o + m and o < off + n for o, m in
-                                         (inflight[b] for b in range(released, it)))
-                if not clash:
-                    break
+            in_use += foot
+            while released < it and ((in_use > cap and bug != "no_footprint_check") or it - released >= slots):
                 yield wait(empty[released % slots], (released // slots) & 1, released // slots)
+                in_use -= foot_of[released]
                 released += 1
             ranges.fill(off, n)
-            inflight[it] = (off, n)
+            foot_of[it] = foot
             full[s].arrive_expect_tx(n)
             q.loads.append(lambda s=s, n=n: full[s].complete_tx(n))
 
     def mma():
         it = 0
-        offs = ring()
+        offs = ((o, n) for o, n, _ in ring())
         for j in range(n_tiles):
             buf = j % nbuf
             yield wait(acc_empty[buf], ((j // nbuf) & 1) ^ 1, j // nbuf - 1)
@@ -321,11 +321,11 @@ def test_bf16_gemm_protocol(tile_bytes, nkb, cap, nbuf):
         run(roles, q, seed, end_check=True)
 
 
-def test_the_checker_catches_a_ring_without_the_overlap_check():
+def test_the_checker_catches_a_ring_without_the_footprint_check():
     """A producer that counts barrier pairs but not bytes overwrites a buffer still read."""
     caught = 0
     for seed in range(60):
-        roles, q = bf16_gemm([36 * KB, 64 * KB, 20 * KB], 6, 128 * KB, bug="no_overlap_check")
+        roles, q = bf16_gemm([36 * KB, 64 * KB, 20 * KB], 6, 128 * KB, bug="no_footprint_check")
         try:
             run(roles, q, seed, end_check=True)
         except AssertionError:

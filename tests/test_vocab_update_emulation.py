@@ -188,29 +188,38 @@ def run_vocab_update(Wout, X, V, excl, n_max, smem_budget=200 * 1024, grid=5, bu
                 pending.append((j, t))
         while pending:
             epilogue(*pending.pop(0))
-    # the row merge: lane l takes tiles l, l + 32, ...; then a butterfly across lanes
+    # the row merge: thread t of 128 takes tiles t, t + 128, ...; a butterfly within each
+    # warp; then the four warps' records in warp order
     out = []
     for row in range(C):
-        lanes = []
-        for ln in range(32):
+        thr = []
+        for t_ in range(128):
             mm, ss, m2, aa = NEG, 0.0, NEG, BIG
-            for t in range(ln, m_tiles, 32):
+            for t in range(t_, m_tiles, 128):
                 xm, xs, xa, xm2 = part[row][t]
                 mm, ss = ms_merge(mm, ss, xm, xs)
                 m2, aa = cand_merge(m2, aa, xm2, xa)
-            lanes.append((mm, ss, m2, aa))
-        o = 16
-        while o:
-            new = []
-            for ln in range(32):
-                mm, ss, m2, aa = lanes[ln]
-                om, os, om2, oa = lanes[ln ^ o]
-                mm, ss = ms_merge(mm, ss, om, os)
-                m2, aa = cand_merge(m2, aa, om2, oa)
-                new.append((mm, ss, m2, aa))
-            lanes = new
-            o >>= 1
-        mm, ss, m2, aa = lanes[0]
+            thr.append((mm, ss, m2, aa))
+        warps = []
+        for w in range(4):
+            lanes = thr[32 * w:32 * w + 32]
+            o = 16
+            while o:
+                new = []
+                for ln in range(32):
+                    mm, ss, m2, aa = lanes[ln]
+                    om, os, om2, oa = lanes[ln ^ o]
+                    mm, ss = ms_merge(mm, ss, om, os)
+                    m2, aa = cand_merge(m2, aa, om2, oa)
+                    new.append((mm, ss, m2, aa))
+                lanes = new
+                o >>= 1
+            warps.append(lanes[0])
+        mm, ss, m2, aa = warps[0]
+        for w in range(1, 4):
+            om, os, om2, oa = warps[w]
+            mm, ss = ms_merge(mm, ss, om, os)
+            m2, aa = cand_merge(m2, aa, om2, oa)
         out.append((mm, ss, aa, m2))
     return out
 
