@@ -83,7 +83,7 @@ struct HalfSlotPlan {
   }
 };
 
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(192)
     tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
                     const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
