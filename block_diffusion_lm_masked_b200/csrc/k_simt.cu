@@ -318,7 +318,7 @@ cudaError_t launch_simt_attention_f32(const float* q, const float* kcache, const
 // normalises its own RT_TOK / RT_G tokens, the normalised rows are shared through
 // distributed shared memory, every CTA computes its experts' logits for all RT_TOK
 // tokens (four experts per warp at once, each token row read from shared memory once per
-// four experts, eight float4 weight loads per lane in flight), and CTA r runs
+// four experts, sixteen float4 weight loads per lane in flight), and CTA r runs
 // the top-k of its own tokens over the logits of all CTAs.  Each logit is one lane-
 // strided fp32 dot product followed by a warp sum, as in a single-CTA version.
 constexpr int RT_G = 4;
@@ -326,7 +326,7 @@ constexpr int RT_TOK = 8;
 constexpr int RT_OWN = RT_TOK / RT_G;
 constexpr int RT_THREADS = 256;
 constexpr int RT_EB = 4;   // experts per warp at once
-constexpr int RT_PF = 2;   // float4 steps of the weights loaded ahead (RT_PF * RT_EB loads)
+constexpr int RT_PF = 4;   // float4 steps of the weights loaded ahead (RT_PF * RT_EB loads)
 template <typename T>
 __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     float* __restrict__ x, const float* __restrict__ parts, int n_parts, size_t part_stride,
@@ -354,23 +354,36 @@ __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     const float4* p4 = reinterpret_cast<const float4*>(parts + (size_t)o0 * H);
     const size_t ps4 = part_stride / 4;
     float4* own4 = reinterpret_cast<float4*>(own);
-    for (int i = threadIdx.x; i < no * H4; i += RT_THREADS) {
-      // every partial's load issued before the first add (the sum keeps its fixed order)
-      float4 a[kMaxSumParts];
+    // two elements per thread and step: every partial's load of both issued before the
+    // first add (each sum keeps its fixed order)
+    for (int i0 = threadIdx.x; i0 < no * H4; i0 += 2 * RT_THREADS) {
+      float4 a[2][kMaxSumParts], v[2];
 #pragma unroll
-      for (int s = 0; s < kMaxSumParts; ++s)
-        if (s < n_parts) a[s] = p4[s * ps4 + i];
-      float4 v = x4[i];
+      for (int e = 0; e < 2; ++e) {
+        const int i = i0 + e * RT_THREADS;
+        if (i < no * H4) {
 #pragma unroll
-      for (int s = 0; s < kMaxSumParts; ++s)
-        if (s < n_parts) {
-          v.x += a[s].x;
-          v.y += a[s].y;
-          v.z += a[s].z;
-          v.w += a[s].w;
+          for (int s = 0; s < kMaxSumParts; ++s)
+            if (s < n_parts) a[e][s] = p4[s * ps4 + i];
+          v[e] = x4[i];
         }
-      x4[i] = v;
-      own4[i] = v;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = i0 + e * RT_THREADS;
+        if (i < no * H4) {
+#pragma unroll
+          for (int s = 0; s < kMaxSumParts; ++s)
+            if (s < n_parts) {
+              v[e].x += a[e][s].x;
+              v[e].y += a[e][s].y;
+              v[e].z += a[e][s].z;
+              v[e].w += a[e][s].w;
+            }
+          x4[i] = v[e];
+          own4[i] = v[e];
+        }
+      }
     }
   }
   __syncthreads();
@@ -387,11 +400,29 @@ __global__ void __launch_bounds__(RT_THREADS) router_fused_kernel(
     store_act(xn, xn_lo, (size_t)o0 * H + i, v);
   }
   cl.sync();  // every CTA's rows are normalised
-  for (int r = 0; r < RT_G; ++r) {
-    const int nr = max(0, min(RT_OWN, nt - r * RT_OWN));
-    const float4* src = reinterpret_cast<const float4*>(cl.map_shared_rank(own, r));
-    float4* dst = reinterpret_cast<float4*>(xs + (size_t)r * RT_OWN * H);
-    for (int i = threadIdx.x; i < nr * H4; i += RT_THREADS) dst[i] = src[i];
+  // the cluster's rows into this CTA's shared memory: eight remote loads in flight per
+  // thread before their stores (rank r's rows land at r * RT_OWN)
+  {
+    const float4* src[RT_G];
+#pragma unroll
+    for (int r = 0; r < RT_G; ++r) src[r] = reinterpret_cast<const float4*>(cl.map_shared_rank(own, r));
+    float4* dst = reinterpret_cast<float4*>(xs);
+    const int per = RT_OWN * H4;  // float4 of one rank's rows
+    const int total = nt * H4;
+    constexpr int CB = 8;
+    for (int i0 = threadIdx.x; i0 < total; i0 += CB * RT_THREADS) {
+      float4 v[CB];
+#pragma unroll
+      for (int c = 0; c < CB; ++c) {
+        const int i = i0 + c * RT_THREADS;
+        if (i < total) v[c] = src[i / per][i % per];
+      }
+#pragma unroll
+      for (int c = 0; c < CB; ++c) {
+        const int i = i0 + c * RT_THREADS;
+        if (i < total) dst[i] = v[c];
+      }
+    }
   }
   __syncthreads();
   const float4* xs4 = reinterpret_cast<const float4*>(xs);

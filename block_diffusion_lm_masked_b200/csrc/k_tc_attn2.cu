@@ -83,7 +83,7 @@ struct HalfSlotPlan {
   }
 };
 
-__global__ void __maxnreg__(192)
+__global__ void __launch_bounds__(A2_THREADS, 1)
     tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
                     const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVtl,
