@@ -597,10 +597,11 @@ int attn_pair_splits(int n_q, int nq, int group, int pair_heads, int n_keys, int
   return splits;
 }
 
-// DG_ATTN_PAIR=1 routes the bf16 pass's attention through the head-pair kernel
+// The bf16 pass's attention runs the head-pair kernel; DG_ATTN_SINGLE=1 routes it
+// through the single-head kernel (tc_attn_kernel) instead
 bool attn_pair_enabled() {
-  static const bool on = getenv("DG_ATTN_PAIR") != nullptr && getenv("DG_ATTN_PAIR")[0] == '1';
-  return on;
+  static const bool single = getenv("DG_ATTN_SINGLE") != nullptr && getenv("DG_ATTN_SINGLE")[0] == '1';
+  return !single;
 }
 
 // attention() through the head-pair kernel: the same inputs, outputs and workspace

@@ -1,7 +1,7 @@
-"""The head-pair attention kernel (dg_debug_attention_pair_bf16) against a plain fp32
-reference of the same attention and against today's kernel on the same inputs, then
-whole passes with it (DG_ATTN_PAIR=1) against the oracle, in a child process since the
-switch is read once per process."""
+"""The head-pair attention kernel (dg_debug_attention_pair_bf16, the pass's default)
+against a plain fp64 reference of the same attention and against the single-head kernel
+on the same inputs, then whole passes with the single-head kernel (DG_ATTN_SINGLE=1)
+against the oracle, in a child process since the switch is read once per process."""
 import os
 import subprocess
 import sys
@@ -87,14 +87,14 @@ def test_pair_kernel_agrees_with_the_single_head_kernel(dg, nq, nkv, n_q, pos0, 
     assert ((a - b).abs() <= 2e-5 * b.abs() + 2e-5 * rms).all(), (a - b).abs().max().item()
 
 
-def test_passes_with_pair_kernel_match_the_oracle():
+def test_passes_with_the_single_head_kernel_match_the_oracle():
     """The pass parity tests (own-key low terms, causal prefill, chained canvases) with the
-    pass's attention routed through the head-pair kernel; the child must have run them (a
-    child whose tests all skipped proves nothing)."""
+    pass's attention routed through the single-head kernel; the child must have run them
+    (a child whose tests all skipped proves nothing)."""
     import re
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    env = dict(os.environ, DG_ATTN_PAIR="1")
+    env = dict(os.environ, DG_ATTN_SINGLE="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "tests/test_gpu_parity.py",
                         "-k", "small_bf16 or layer1_bf16 or prefill_append or chained"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
