@@ -7,7 +7,7 @@
 // contiguous range of 128-key chunks.  Each K/V chunk is loaded once for both heads.
 // Warps 0-3 run the softmax of the first head and warps 4-7 that of the second, one query
 // row per thread over the whole 128-key chunk, so no row statistics are exchanged between
-// warps.  Warp 8 issues the TMA loads, warp 9 the MMAs.
+// warps.  Warp 8 issues the TMA loads; warps 9 and 10 issue the MMAs, one per head.
 //
 // TMEM (512 columns): per head one S/P region of 128 columns and O (128 columns).  The
 // softmax reads S (fp32, 128 keys) into registers and writes P over it as packed bf16
@@ -17,13 +17,14 @@
 // 16 KB swizzled blocks); a chunk of the call's own keys also takes its K and V low terms.
 // Ring order per chunk: K (and K lo), then V (and V lo).
 //
-// Issue order of the MMA warp per chunk j: S_A(j), S_B(j) (each once PV(j-1) of its head
-// has completed, which also means its softmax has read S(j-1) and written P(j-1)), a
-// commit freeing the K half-slots, then PV_A(j), PV_B(j) (each once its head's softmax of
-// chunk j has written P) and a commit freeing the V half-slots.  While the softmax of one
-// head works on S(j), the tensor cores run the other head's S or PV, so with the MMAs of
-// two heads per chunk (two-term S and PV: 33.6 MFLOP, about 3.1 us at the per-SM peak)
-// the tensor pipe waits on a softmax only if it takes longer than one head's S or PV.
+// Each head's MMA thread, per chunk j: S(j) once PV(j-1) of its head has completed (which
+// also means its softmax has read S(j-1) and written P(j-1)), a commit towards freeing the
+// K half-slots, then PV(j) once its softmax has written P(j), and a commit towards freeing
+// the V half-slots; a half-slot is free once both heads' commits have arrived.  The two
+// threads run side by side: each bounded wait and commit costs a few hundred nanoseconds
+// (measured), and with one issuing thread for both heads those costs, twelve per chunk,
+// added up to about 2.4 of the chunk's 5.6 us.  While the softmax of one head works on
+// S(j), the tensor cores run the other head's MMAs.
 #include <math.h>
 
 #include "attn_softmax.cuh"
@@ -41,8 +42,8 @@ constexpr uint32_t A2_QHEAD = 4 * A2_BLK;       // Q hi (two d blocks) + Q lo: 6
 constexpr uint32_t A2_HSLOT = 2 * A2_BLK;       // K (two d blocks) or V^T (two key blocks): 32 KB
 constexpr int A2_SMEM = 1024 + 2 * A2_QHEAD + A2_HSLOTS * A2_HSLOT;
 constexpr int A2_LOAD_WARP = 8;
-constexpr int A2_MMA_WARP = 9;
-constexpr int A2_THREADS = 32 * 10;
+constexpr int A2_MMA_WARP = 9;   // the MMAs of the first head; warp 10 those of the second
+constexpr int A2_THREADS = 32 * 11;
 static_assert(A2_SMEM <= 227 * 1024 - 512, "shared memory budget");
 
 // TMEM column offsets: head hl's S/P region and its O
@@ -134,14 +135,14 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     mbar_init(&q_bar, 1);
     for (int s = 0; s < A2_HSLOTS; ++s) {
       mbar_init(&hs_full[s], 1);
-      mbar_init(&hs_free[s], 1);
+      mbar_init(&hs_free[s], nh);  // one commit per head's MMA thread
     }
     for (int hl = 0; hl < 2; ++hl) {
       mbar_init(&s_full[hl], 1);
       mbar_init(&p_ready[hl], 4);
       mbar_init(&pv_done[hl], 1);
     }
-    mbar_init(&drain_bar, 1);
+    mbar_init(&drain_bar, nh);
     abort_s = 0;
     fence_barrier_init();
   }
@@ -209,12 +210,14 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == A2_MMA_WARP) {
-    if (lane == 0) {
-      // ================= MMAs
+  } else if (warp == A2_MMA_WARP || warp == A2_MMA_WARP + 1) {
+    const int hl = warp - A2_MMA_WARP;  // this warp's head
+    if (lane == 0 && hl < nh) {
+      // ================= MMAs of head hl: one issuing thread per head, so that each
+      // head's waits, MMAs and commits run beside the other head's
       HalfSlotPlan mp;
       auto half_addr = [&](int s) { return smem_u32(sHalf + s * A2_HSLOT); };
-      auto issue_s = [&](int hl) {
+      auto issue_s = [&]() {
         const uint32_t d = tmem + a2_sp(hl);
         const uint32_t q = smem_u32(sQ + hl * A2_QHEAD), ql = q + 2 * A2_BLK;
         const uint32_t k = half_addr(mp.ks[0]);
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           }
         tc_commit(&s_full[hl]);
       };
-      auto issue_pv = [&](int hl, int j) {
+      auto issue_pv = [&](int j) {
         const uint32_t o = tmem + a2_o(hl), pp = tmem + a2_sp(hl);
         const uint32_t v = half_addr(mp.vs[0]);
         const uint32_t vl = mp.n == 2 ? half_addr(mp.vs[1]) : 0u;
@@ -251,25 +254,20 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         mp.take(is_cur(j));
         for (int i = 0; i < mp.n && ok; ++i)
           ok = mbar_wait(&hs_full[mp.ks[i]], (uint32_t)mp.ku[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-        for (int hl = 0; hl < nh && ok; ++hl) {
-          // the head's S/P region was last read by PV(j - 1)
-          if (j >= 1)
-            ok = mbar_wait(&pv_done[hl], (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(hl);
-        }
+        // the head's S/P region was last read by PV(j - 1)
+        if (ok && j >= 1)
+          ok = mbar_wait(&pv_done[hl], (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (!ok) break;
+        tc_fence_after();
+        issue_s();
+        // a K half-slot is free once both heads' S MMAs have read it (count: one per head)
         for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.ks[i]]);
         for (int i = 0; i < mp.n && ok; ++i)
           ok = mbar_wait(&hs_full[mp.vs[i]], (uint32_t)mp.vu[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-        for (int hl = 0; hl < nh && ok; ++hl) {
-          ok = mbar_wait(&p_ready[hl], (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(hl, j);
-        }
+        if (ok) ok = mbar_wait(&p_ready[hl], (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (!ok) break;
+        tc_fence_after();
+        issue_pv(j);
         for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.vs[i]]);
       }
     }
@@ -435,10 +433,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   // wind down: every MMA and commit the MMA thread issued has landed (also on the normal
   // path, so that no mbarrier arrive reaches this CTA's shared memory after it is gone),
   // and after an abort the loads the load thread issued have landed too
-  if (tid == A2_MMA_WARP * 32) {
-    tc_commit(&drain_bar);
-    mbar_wait_drain(&drain_bar, 0);
-  }
+  if (lane == 0 && (warp == A2_MMA_WARP || (nh == 2 && warp == A2_MMA_WARP + 1))) tc_commit(&drain_bar);
+  if (tid == A2_MMA_WARP * 32) mbar_wait_drain(&drain_bar, 0);
   if (abort_s && tid == A2_LOAD_WARP * 32) {
     if (q_issued) mbar_wait_drain(&q_bar, 0);
     for (int s = 0; s < A2_HSLOTS; ++s)

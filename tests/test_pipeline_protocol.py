@@ -846,32 +846,53 @@ def half_slot_plan(nck, cur_from, slots):
     return plan
 
 
+class AsyncPerThread(Async):
+    """Completions of several issuing threads: each thread's MMAs and commits complete in its
+    own issue order, the threads' streams interleave in any order."""
+
+    def __init__(self, n):
+        super().__init__()
+        self.by = [[] for _ in range(n)]
+
+    def __bool__(self):
+        return bool(self.loads or any(self.by))
+
+    def step(self, rng):
+        busy = [q for q in self.by if q]
+        if busy and (not self.loads or rng.random() < 0.5):
+            rng.choice(busy).pop(0)()
+        else:
+            self.loads.pop(rng.randrange(len(self.loads)))()
+
+
 def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, flags=None, give_up_at=None,
                         drain=True, load_drain=True, bug=None):
     """The head-pair attention kernel's hand-offs (128-key chunks): a load warp fills a ring
-    of `slots` half-slots, each chunk's K then its V^T; per chunk the MMA warp issues S_A(j),
-    S_B(j) -- each once PV(j-1) of its head has completed, since S overwrites the head's one
-    S/P region -- commits the K half-slots free, then PV_A(j), PV_B(j) once each head's
-    softmax warps have written P(j), and commits the V half-slots free.  Each head's softmax
-    warps read S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  The MMA
-    warp drains its commits before the CTA leaves (`drain`).
+    of `slots` half-slots, each chunk's K then its V^T; one MMA thread per head issues, per
+    chunk, its S(j) -- once its PV(j-1) has completed, since S overwrites the head's one
+    S/P region -- and a commit towards freeing the K half-slots, then its PV(j) once its
+    softmax warps have written P(j), and a commit towards freeing the V half-slots; a
+    half-slot's free barrier counts one commit per head.  Each head's softmax warps read
+    S(j), maybe rescale O (after PV(j-1)), write P over S and signal.  Each MMA thread
+    drains its commits before the CTA leaves (`drain`).
 
-    bug: "no_pv_wait" -- S(j) issued without waiting for PV(j-1); "k_free_early" -- the K
-    half-slots freed after the first head's S.
+    bug: "no_pv_wait" -- S(j) issued without waiting for PV(j-1); "free_count_one" -- the
+    half-slots' free barriers count one commit, so the first head's frees the slot.
 
     flags: abort mode -- every bounded wait also passes once flags["abort"] is set, the
     give_up_at-th wait raises it (a timeout), a role whose wait failed leaves its loop,
     and the load warp then waits for the loads it issued (`load_drain`)."""
     rng = random.Random(seed * 104729 + nck)
     plan = half_slot_plan(nck, nck if cur_from is None else cur_from, slots)
-    hs_full = [Barrier(f"hs_full{s}", 1) for s in range(slots)]
-    hs_free = [Barrier(f"hs_free{s}", 1) for s in range(slots)]
-    drain_bar = Barrier("drain", 1)
     H = 2
+    free_count = 1 if bug == "free_count_one" else H
+    hs_full = [Barrier(f"hs_full{s}", 1) for s in range(slots)]
+    hs_free = [Barrier(f"hs_free{s}", free_count) for s in range(slots)]
+    drain_bar = Barrier("drain", H)
     s_full = [Barrier(f"s_full{h}", 1) for h in range(H)]
     p_ready = [Barrier(f"p_ready{h}", warps_per_head) for h in range(H)]
     pv_done = [Barrier(f"pv_done{h}", 1) for h in range(H)]
-    bufs, q = Buffers(), Async()
+    bufs, q = Buffers(), AsyncPerThread(H)
     st = {"pv_done": [0, 0], "pv_issued": [0, 0]}
     p_writes = {}
     steps = [0]
@@ -899,7 +920,7 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                         if not passed(hs_free[s], (u - 1) & 1):
                             ok = False
                             break
-                    bufs.fill(("hs", s), H)           # K: S_A and S_B read it; V^T: PV_A and PV_B
+                    bufs.fill(("hs", s), H)           # K: both heads' S read it; V^T: both PVs
                     hs_full[s].arrive_expect_tx(32)
                     q.loads.append(lambda s=s: hs_full[s].complete_tx(32))
                     loaded[s] += 1
@@ -912,7 +933,8 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                 if loaded[s]:
                     yield wait(hs_full[s], (loaded[s] - 1) & 1, None)
 
-    def mma():
+    def mma(h):
+        mq = q.by[h]
         ok = True
         for j in range(nck):
             k_parts, v_parts = plan[j]
@@ -921,60 +943,48 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                 if not passed(hs_full[x], u & 1):
                     ok = False
                     break
-            for h in range(H):
-                if not ok:
-                    break
-                if j >= 1 and bug != "no_pv_wait":
-                    yield bw(pv_done[h], (j - 1) & 1, j - 1)
-                    if not passed(pv_done[h], (j - 1) & 1):
-                        ok = False
-                        break
-                for w in range(warps_per_head):       # S: each warp reads its own 32 lanes
-                    bufs.fill(("sp", h, w), 1)
-
-                def s_done(h=h, j=j):
-                    for x, _ in plan[j][0]:
-                        bufs.release(("hs", x))
-                    s_full[h].arrive()
-                q.mma.append(s_done)
-                if bug == "k_free_early" and h == 0:
-                    for x, _ in k_parts:
-                        q.mma.append(lambda x=x: hs_free[x].arrive())
+            if ok and j >= 1 and bug != "no_pv_wait":
+                yield bw(pv_done[h], (j - 1) & 1, j - 1)
+                ok = passed(pv_done[h], (j - 1) & 1)
             if not ok:
                 break
-            if bug != "k_free_early":
-                for x, _ in k_parts:                  # one commit per K half-slot
-                    q.mma.append(lambda x=x: hs_free[x].arrive())
+            for w in range(warps_per_head):           # S: each warp reads its own 32 lanes
+                bufs.fill(("sp", h, w), 1)
+
+            def s_done(h=h, j=j):
+                for x, _ in plan[j][0]:
+                    bufs.release(("hs", x))
+                s_full[h].arrive()
+            mq.append(s_done)
+            for x, _ in k_parts:                      # this head's commit per K half-slot
+                mq.append(lambda x=x: hs_free[x].arrive())
             for x, u in v_parts:
                 yield bw(hs_full[x], u & 1, u)
                 if not passed(hs_full[x], u & 1):
                     ok = False
                     break
-            for h in range(H):
-                if not ok:
-                    break
-                yield bw(p_ready[h], j & 1, j)
-                if not passed(p_ready[h], j & 1):
-                    ok = False
-                    break
-                assert p_writes.get(h) == (j, warps_per_head), "PV read a P not fully written"
-                st["pv_issued"][h] += 1
-
-                def pv_fin(h=h, j=j):
-                    st["pv_done"][h] += 1
-                    for w in range(warps_per_head):   # every warp's lanes of P(j) were read
-                        bufs.release(("sp", h, w))
-                    for x, _ in plan[j][1]:
-                        bufs.release(("hs", x))
-                    pv_done[h].arrive()
-                q.mma.append(pv_fin)
             if not ok:
                 break
-            for x, _ in v_parts:                      # one commit per V^T half-slot
-                q.mma.append(lambda x=x: hs_free[x].arrive())
+            yield bw(p_ready[h], j & 1, j)
+            if not passed(p_ready[h], j & 1):
+                break
+            assert p_writes.get(h) == (j, warps_per_head), "PV read a P not fully written"
+            st["pv_issued"][h] += 1
+
+            def pv_fin(h=h, j=j):
+                st["pv_done"][h] += 1
+                for w in range(warps_per_head):       # every warp's lanes of P(j) were read
+                    bufs.release(("sp", h, w))
+                for x, _ in plan[j][1]:
+                    bufs.release(("hs", x))
+                pv_done[h].arrive()
+            mq.append(pv_fin)
+            for x, _ in v_parts:                      # this head's commit per V^T half-slot
+                mq.append(lambda x=x: hs_free[x].arrive())
         if drain:                                     # every commit issued above has landed
-            q.mma.append(lambda: drain_bar.arrive())
-            yield wait(drain_bar, 0, 0)
+            mq.append(lambda: drain_bar.arrive())
+            if h == 0:
+                yield wait(drain_bar, 0, 0)
 
     def softmax(h, w):
         for j in range(nck):
@@ -995,8 +1005,9 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
         if passed(pv_done[h], (nck - 1) & 1):
             assert st["pv_done"][h] == nck
 
-    roles = {"load": load(), "mma": mma()}
+    roles = {"load": load()}
     for h in range(H):
+        roles[f"mma{h}"] = mma(h)
         roles.update({f"sm{h}{w}": softmax(h, w) for w in range(warps_per_head)})
     return roles, q
 
@@ -1011,11 +1022,11 @@ def test_head_pair_attention_protocol(nck, cur_from):
         run(roles, q, seed, end_check=True)
 
 
-@pytest.mark.parametrize("bug", ["no_pv_wait", "k_free_early"])
+@pytest.mark.parametrize("bug", ["no_pv_wait", "free_count_one"])
 def test_head_pair_attention_protocol_catches_its_planted_mistakes(bug):
-    """S(j) issued before PV(j-1) has read P(j-1) from the same TMEM region, or the K
-    half-slots freed before the second head's S: some interleaving overwrites a buffer that
-    is still read."""
+    """S(j) issued before PV(j-1) has read P(j-1) from the same TMEM region, or a half-slot
+    freed by the first head's commit before the other head's MMAs read it: some
+    interleaving overwrites a buffer that is still read."""
     caught = 0
     for seed in range(80):
         roles, q = attention_two_heads(6, seed, cur_from=4, bug=bug)
