@@ -489,8 +489,13 @@ struct GemmCall {
 
 // dense projections (no work list, one weight matrix, fp32 store) of at least two weight
 // tiles take them in pairs that share each token load
+// weight tiles taken in pairs that share each token load: every fp32-store GEMM of at
+// least 256 weight rows (the dense projections and the grouped expert down projection,
+// whose short tiles -- 11 k-blocks of 16 token rows at the large model -- then halve their
+// per-tile hand-offs and token loads); the gate/up GEMM already pairs its two matrices
 bool pair_weight_tiles(int a_rows, bool grouped, bool dual, int epi) {
-  return !grouped && !dual && epi == dg::EPI_STORE_F32 && a_rows >= 256;
+  (void)grouped;
+  return !dual && epi == dg::EPI_STORE_F32 && a_rows >= 256;
 }
 // weight tiles of a dense projection as the GEMM walks them (pairs where they are paired)
 int dense_weight_tiles(int a_rows) { return ceil_div(a_rows, pair_weight_tiles(a_rows, false, false,

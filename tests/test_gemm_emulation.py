@@ -52,11 +52,11 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
              smem_budget=200 * 1024, grid=5, bug=None, m_pair=None):
     """W / W2: bf16 bits [G][rows][K]; X_hi / X_lo: bf16 bits [n][K]; items: (group, row0,
     rows) or None (dense).  m_pair: tiles of two consecutive 128-row weight tiles (default:
-    as the host chooses, dense fp32-store GEMMs of at least 256 weight rows).  Returns the
+    as the host chooses, fp32-store GEMMs of at least 256 weight rows, dense or grouped).  Returns the
     output array as the kernel writes it."""
     terms = 2 if X_lo is not None else 1
     if m_pair is None:
-        m_pair = items is None and W2 is None and rows_a >= 256
+        m_pair = W2 is None and rows_a >= 256
     n_a = 2 if (W2 is not None or m_pair) else 1
     tile_rows = 2 * BM if m_pair else BM
     a_bytes = BM * BK * 2
@@ -338,3 +338,24 @@ def test_paired_weight_tiles_replay(rows, n, terms, n_max):
     assert np.abs(out.reshape(n, rows) - ref).max() / np.abs(ref).max() < 2e-6
     plain, _ = run_gemm(W, hi, lo, rows, K, rows, n_max=n_max, m_pair=False)
     assert np.abs(out - plain).max() / np.abs(ref).max() < 2e-6
+
+
+@pytest.mark.parametrize("m_pair", [True, False])
+def test_grouped_down_projection_in_weight_tile_pairs_replay(m_pair):
+    """The expert down projection's shape (fp32 store, grouped, 16-ish token rows per
+    expert) with its weight tiles paired, as the host runs it, and unpaired: both match
+    fp64 products; weight rows (384) not a multiple of the pair (256) leave a partial pair."""
+    rng = np.random.default_rng(13)
+    counts, H, F = [16, 0, 40, 9, 130], 384, 192
+    E = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
+    items = [(e, r0, min(128, off[e + 1] - r0)) for e in range(E) for r0 in range(off[e], off[e + 1], 128)]
+    x, hi, lo = bf16_pair(rng, int(off[-1]), F)
+    W, w = weights(rng, E, H, F)
+    out, _ = run_gemm(W, hi, lo, H, F, H, items=items, n_max=128, m_pair=m_pair, grid=3)
+    got = out.reshape(int(off[-1]), H)
+    for e in range(E):
+        xe = x[off[e]:off[e + 1]]
+        if len(xe):
+            ref = xe @ w[e].T
+            assert np.abs(got[off[e]:off[e + 1]] - ref).max() / np.abs(ref).max() < 1e-5, e
