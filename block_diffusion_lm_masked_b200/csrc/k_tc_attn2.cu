@@ -11,7 +11,12 @@
 //
 // TMEM (512 columns): per head one S/P region of 128 columns and O (128 columns).  The
 // softmax reads S (fp32, 128 keys) into registers and writes P over it as packed bf16
-// pairs, hi in the first 64 columns and lo in the next 64; the PV MMAs read P from there.
+// pairs (64 columns); the PV MMAs read P from there.  P enters the PV product as one bf16
+// term (the query keeps its hi + lo terms): each probability is rounded once (relative
+// error at most 2^-8), and the row sum adds the rounded values, so the output is an exact
+// weighted mean of V whose weights are off by at most 2^-8 relative -- at most
+// 2^-8 * sum_j p_j |v_j - o| / sum_j p_j per element, a few thousandths of the output's
+// RMS, against the two-term P's fp32 level and at a quarter fewer MMAs.
 // Shared memory: the query tiles (hi + lo, 64 KB per head) and a ring of three 32 KB
 // half-slots, each holding one chunk's K [128 keys][128 d] or V^T [128 d][128 keys] (two
 // 16 KB swizzled blocks); a chunk of the call's own keys also takes its K and V low terms.
@@ -243,7 +248,6 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           const uint32_t vo = (kk >> 2) * A2_BLK + (kk & 3) * 32;
           const uint64_t vd = sw128_kmajor_desc(v + vo);
           a2_mma_ts(o, pp + kk * 8, vd, idesc, (j > 0 || kk != 0) ? 1u : 0u);
-          a2_mma_ts(o, pp + 64 + kk * 8, vd, idesc, 1u);
           if (mp.n == 2) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
         }
         tc_commit(&pv_done[hl]);
@@ -340,14 +344,14 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         l2 = f2_mul(l2, f2_pack(alpha, alpha));
         m_used = cmax;
       }
-      // P = 2^(s * scale - m_used) (one rounding), packed bf16 pairs over this row's S: hi
-      // in columns 0..63, lo in 64..127.  A row that has seen no key has m_used = -inf and
+      // P = 2^(s * scale - m_used) (one rounding), rounded to bf16 and packed in pairs over
+      // this row's S (columns 0..63).  A row that has seen no key has m_used = -inf and
       // only -inf scores: its offset is taken as 0, so that every P is 2^-inf = 0.
       const float neg_m = (m_used == -INFINITY) ? 0.0f : -m_used;
       const uint64_t nm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < A2_W / 16; ++c) {  // 16 keys -> 8 packed columns per store
-        uint32_t wh[8], wl[8];
+        uint32_t wh[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int i0 = c * 16 + 2 * e;
@@ -356,16 +360,13 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           float t0, t1;
           f2_unpack(t, t0, t1);
           const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-          const uint64_t pp = f2_pack(p0, p1);
-          l2 = f2_add(l2, pp);
+          // the PV product takes P in one bf16 term; the row sum adds the same rounded
+          // values, so the output is their exact weighted mean of V
           const uint32_t hi = bf16x2_pack(p0, p1);
-          float lo0, lo1;
-          f2_unpack(f2_sub(pp, bf16x2_widen(hi)), lo0, lo1);
+          l2 = f2_add(l2, bf16x2_widen(hi));
           wh[e] = hi;
-          wl[e] = bf16x2_pack(lo0, lo1);
         }
         tmem_st8(spa + c * 8, wh);
-        tmem_st8(spa + 64 + c * 8, wl);
       }
       tc_wait_st();
       tc_fence_before();
