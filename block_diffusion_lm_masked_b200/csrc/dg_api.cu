@@ -375,7 +375,7 @@ constexpr int kItemRowsMx8 = 64;         // the same for the 8-bit-weight expert
 
 
 struct WsLayout {
-  size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, attn_cnt, opart, topk_idx,
+  size_t err, upd, x, xn, xn_lo, qkv, q, q_lo, k_lo, vt_lo, o, o_lo, part_o, part_lse, opart, topk_idx,
       topk_w, counts, offsets, perm, inv, uni, items, n_items, xs, xs_lo, h, h_lo, gu, ys, vtiles, total;
   int lo_rows;  // rows of the current-token K/V low-term window
 };
@@ -410,7 +410,6 @@ WsLayout layout(const dg_config& c, int T) {
   L.o_lo = take(bf ? (size_t)T * c.n_q_heads * d * 2 : 0);
   L.part_o = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * d * 4 : 0);
   L.part_lse = take(bf ? (size_t)kMaxAttnSplits * c.n_q_heads * T * 4 : 0);
-  L.attn_cnt = take((size_t)((T + 127) / 128) * c.n_q_heads * 4);  // attention's split tickets
   L.opart = take((size_t)(bf ? kMaxKsO : 1) * T * H * 4);
   L.topk_idx = take((size_t)T * k * 4);
   L.topk_w = take((size_t)T * k * 4);
@@ -609,52 +608,76 @@ bool attn_pair_enabled() {
   return !single;
 }
 
-// attention() through the head-pair kernel: the same inputs, outputs and workspace
-dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0,
-                         int n_keys, int causal, cudaStream_t st) {
+// The tensor maps both attention kernels read: the query hi / lo [nq][n_q][128], the
+// cache's K [nkv][cap][128] and V^T [nkv][128][cap], the low terms of the current K / V^T
+// (rows counted from `base`); every box is 64 x 128 (128-byte swizzled rows)
+dg_status attn_maps(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int n_keys, int base,
+                    CUtensorMap* m) {
   const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
-  CUtensorMap mq, mql, mk, mv, mkl, mvl;
-  dg_status s;
-  const int base = (pos0 / 128) * 128;  // the low-term window starts here (a multiple of the 128-key chunk)
   const int Lc = ws.L.lo_rows;
+  const uint32_t box[3] = {64, 128, 1};
+  dg_status s;
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_q, (uint64_t)nq};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)n_q * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mq, ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
-    if ((s = encode_bf16(&mql, ws.at<void>(ws.L.q_lo), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[0], ws.at<void>(ws.L.q), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[1], ws.at<void>(ws.L.q_lo), 3, dims, str, box)) != DG_OK) return s;
   }
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mk, kc, 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[2], kc, 3, dims, str, box)) != DG_OK) return s;
   }
   {
     const uint64_t dims[3] = {(uint64_t)n_keys, (uint64_t)d, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)cap * 2, (uint64_t)d * cap * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mv, vtc, 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[3], vtc, 3, dims, str, box)) != DG_OK) return s;
   }
   {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)(n_keys - base), (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)Lc * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mkl, ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[4], ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
   }
   {
     const uint64_t dims[3] = {(uint64_t)(n_keys - base), (uint64_t)d, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)Lc * 2, (uint64_t)d * Lc * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mvl, ws.at<void>(ws.L.vt_lo), 3, dims, str, box)) != DG_OK) return s;
+    if ((s = encode_bf16(&m[5], ws.at<void>(ws.L.vt_lo), 3, dims, str, box)) != DG_OK) return s;
   }
+  return DG_OK;
+}
+
+// the parameters both attention kernels share (the split layout is the caller's)
+dg::TcAttnParams attn_params(const dg_config& c, const Ws& ws, int n_q, int pos0, int n_keys, int causal, int base) {
+  const int nq = c.n_q_heads, d = c.head_dim;
   dg::TcAttnParams p;
   p.n_q = n_q;
   p.q_pos0 = pos0;
   p.n_keys = n_keys;
   p.causal = causal;
-  p.group = nq / nkv;
+  p.group = nq / c.n_kv_heads;
   p.nq = nq;
+  p.n_splits = 1;
+  p.chunks_per_split = 1;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  p.has_lo = 1;
+  p.base = base;
+  p.out = ws.at<bf16>(ws.L.o);
+  p.out_lo = ws.at<bf16>(ws.L.o_lo);
+  p.part_o = ws.at<float>(ws.L.part_o);
+  p.part_lse = ws.at<float>(ws.L.part_lse);
+  p.err = ws.err();
+  return p;
+}
+
+// attention() through the head-pair kernel: the same inputs, outputs and workspace
+dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0,
+                         int n_keys, int causal, cudaStream_t st) {
+  const int nq = c.n_q_heads;
+  const int base = (pos0 / 128) * 128;  // the low-term window starts here (a multiple of the 128-key chunk)
+  CUtensorMap m[6];
+  dg_status s;
+  if ((s = attn_maps(c, ws, kc, vtc, cap, n_q, n_keys, base, m)) != DG_OK) return s;
+  dg::TcAttnParams p = attn_params(c, ws, n_q, pos0, n_keys, causal, base);
   // head pairs share each K/V chunk and overlap one head's softmax with the other's MMAs;
   // single heads give twice the CTAs.  Take whichever fills more of the machine in one
   // wave (pairs unless single heads fill at least a quarter more SMs).
@@ -667,85 +690,40 @@ dg_status attention_pair(const dg_config& c, const Ws& ws, void* kc, void* vtc, 
   const int pair_heads = (p.group % 2 == 0 && 4 * ctas_single < 5 * ctas_pair) ? 1 : 0;
   p.n_splits = pair_heads ? sp_pair : sp_single;
   p.chunks_per_split = pair_heads ? cps_pair : cps_single;
-  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-  p.has_lo = 1;
-  p.q = ws.at<bf16>(ws.L.q);
-  p.q_lo = ws.at<bf16>(ws.L.q_lo);
-  p.merge_cnt = nullptr;  // merged by attn_merge2_kernel
-  p.base = base;
-  p.out = ws.at<bf16>(ws.L.o);
-  p.out_lo = ws.at<bf16>(ws.L.o_lo);
-  p.part_o = ws.at<float>(ws.L.part_o);
-  p.part_lse = ws.at<float>(ws.L.part_lse);
-  p.err = ws.err();
-  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(mq, mql, mk, mv, mkl, mvl, p, pair_heads, st));
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention2(m[0], m[1], m[2], m[3], m[4], m[5], p, pair_heads, st));
   if (p.n_splits > 1)
     LAUNCH(DG_K_ATTN_MERGE, st,
-           dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, ws.at<bf16>(ws.L.o),
-                                  ws.at<bf16>(ws.L.o_lo), st));
+           dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, p.out, p.out_lo, st));
+  return DG_OK;
+}
+
+// attention() through the single-head kernel: the same inputs, outputs and workspace
+dg_status attention_single(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0,
+                           int n_keys, int causal, cudaStream_t st) {
+  const int nq = c.n_q_heads;
+  const int base = (pos0 / 128) * 128;  // the low-term window starts at this chunk
+  CUtensorMap m[6];
+  dg_status s;
+  if ((s = attn_maps(c, ws, kc, vtc, cap, n_q, n_keys, base, m)) != DG_OK) return s;
+  dg::TcAttnParams p = attn_params(c, ws, n_q, pos0, n_keys, causal, base);
+  p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
+  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(m[0], m[1], m[2], m[3], m[4], m[5], p, st));
+  if (p.n_splits > 1)
+    LAUNCH(DG_K_ATTN_MERGE, st,
+           dg::launch_attn_merge2(p.part_o, p.part_lse, p.n_splits, nq, n_q, p.out, p.out_lo, st));
   return DG_OK;
 }
 
 // attention of n_q new rows at positions pos0.. over cache keys [0, n_keys) -> ws.o (+ ws.o_lo)
 dg_status attention(const dg_config& c, const Ws& ws, void* kc, void* vtc, int cap, int n_q, int pos0, int n_keys,
                     int causal, cudaStream_t st) {
-  const int nq = c.n_q_heads, nkv = c.n_kv_heads, d = c.head_dim;
-  if (is_bf16(c) && attn_pair_enabled()) return attention_pair(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st);
-  if (!is_bf16(c)) {
-    LAUNCH(DG_K_ATTENTION, st,
-           dg::launch_simt_attention_f32(ws.at<float>(ws.L.q), (const float*)kc, (const float*)vtc, cap, n_q, pos0,
-                                         n_keys, causal, nq, nkv, d, ws.at<float>(ws.L.o), st));
-    return DG_OK;
-  }
-  CUtensorMap mk, mv, mkl, mvl;
-  dg_status s;
-  const int base = (pos0 / 128) * 128;  // the low-term window starts at this chunk
-  const int Lc = ws.L.lo_rows;
-  {
-    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)n_keys, (uint64_t)nkv};
-    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)cap * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mk, kc, 3, dims, str, box)) != DG_OK) return s;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)n_keys, (uint64_t)d, (uint64_t)nkv};
-    const uint64_t str[2] = {(uint64_t)cap * 2, (uint64_t)d * cap * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mv, vtc, 3, dims, str, box)) != DG_OK) return s;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)(n_keys - base), (uint64_t)nkv};
-    const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)Lc * d * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mkl, ws.at<void>(ws.L.k_lo), 3, dims, str, box)) != DG_OK) return s;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)(n_keys - base), (uint64_t)d, (uint64_t)nkv};
-    const uint64_t str[2] = {(uint64_t)Lc * 2, (uint64_t)d * Lc * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if ((s = encode_bf16(&mvl, ws.at<void>(ws.L.vt_lo), 3, dims, str, box)) != DG_OK) return s;
-  }
-  dg::TcAttnParams p;
-  p.n_q = n_q;
-  p.q_pos0 = pos0;
-  p.n_keys = n_keys;
-  p.causal = causal;
-  p.group = nq / nkv;
-  p.nq = nq;
-  p.n_splits = attn_splits(n_q, nq, n_keys, &p.chunks_per_split);
-  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-  p.has_lo = 1;
-  p.q = ws.at<bf16>(ws.L.q);
-  p.q_lo = ws.at<bf16>(ws.L.q_lo);
-  p.merge_cnt = ws.at<int>(ws.L.attn_cnt);  // zeroed by the RoPE kernel before every attention
-  p.base = base;
-  p.out = ws.at<bf16>(ws.L.o);
-  p.out_lo = ws.at<bf16>(ws.L.o_lo);
-  p.part_o = ws.at<float>(ws.L.part_o);
-  p.part_lse = ws.at<float>(ws.L.part_lse);
-  p.err = ws.err();
-  // the kernel merges its split-KV partials itself (the last split of each tile and head)
-  LAUNCH(DG_K_ATTENTION, st, dg::launch_tc_attention(mk, mv, mkl, mvl, p, st));
+  if (is_bf16(c))
+    return attn_pair_enabled() ? attention_pair(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)
+                               : attention_single(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st);
+  LAUNCH(DG_K_ATTENTION, st,
+         dg::launch_simt_attention_f32(ws.at<float>(ws.L.q), (const float*)kc, (const float*)vtc, cap, n_q, pos0,
+                                       n_keys, causal, c.n_q_heads, c.n_kv_heads, c.head_dim, ws.at<float>(ws.L.o),
+                                       st));
   return DG_OK;
 }
 
@@ -780,8 +758,7 @@ dg_status layer(dg_model* m, int l, const Ws& ws, void* kc, void* vtc, int cap, 
          dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv), ks_qkv, (size_t)n * QR, n, nq, nkv, d, pos0, c.rope_theta,
                                     ws.at<T>(ws.L.q), (T*)kc, (T*)vtc, cap, bf ? ws.at<T>(ws.L.q_lo) : nullptr,
                                     bf ? ws.at<T>(ws.L.k_lo) : nullptr, bf ? ws.at<T>(ws.L.vt_lo) : nullptr,
-                                    (pos0 / 128) * 128, ws.L.lo_rows, ws.at<int>(ws.L.attn_cnt),
-                                    ((n + 127) / 128) * nq, st));
+                                    (pos0 / 128) * 128, ws.L.lo_rows, st));
   if (stop_after_kv) return DG_OK;
   if ((s = attention(c, ws, kc, vtc, cap, n, pos0, pos0 + n, causal, st)) != DG_OK) return s;
   if (bf) {
@@ -969,8 +946,7 @@ dg_status layer_batched(dg_model* m, int l, const Ws& ws, const std::vector<Seg>
            dg::launch_rope_scatter<T>(ws.at<float>(ws.L.qkv) + (size_t)b * C * QR, ks_qkv, (size_t)n * QR, C, nq, nkv,
                                       d, g.pos0, c.rope_theta, wb.at<T>(wb.L.q), (T*)g.kc, (T*)g.vtc, g.cap,
                                       bf ? wb.at<T>(wb.L.q_lo) : nullptr, bf ? ws.at<T>(ws.L.k_lo) : nullptr,
-                                      bf ? ws.at<T>(ws.L.vt_lo) : nullptr, (g.pos0 / 128) * 128, ws.L.lo_rows,
-                                      ws.at<int>(ws.L.attn_cnt), ((C + 127) / 128) * nq, st));
+                                      bf ? ws.at<T>(ws.L.vt_lo) : nullptr, (g.pos0 / 128) * 128, ws.L.lo_rows, st));
     if (stop_after_kv) continue;
     if ((s = attention(c, wb, g.kc, g.vtc, g.cap, C, g.pos0, g.pos0 + C, causal, st)) != DG_OK) return s;
   }
@@ -1759,13 +1735,11 @@ static dg_status debug_attention(const void* q, const void* k, const void* vt, i
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.q_lo), 0, (size_t)nq * n_q * 128 * 2, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.k_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.vt_lo), 0, (size_t)nkv * ws.L.lo_rows * 128 * 2, st);
-  // the split tickets the pass's RoPE kernel would zero
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws.at<void>(ws.L.attn_cnt), 0, (size_t)((n_q + 127) / 128) * nq * 4, st);
   if (e != cudaSuccess) return fail(DG_ERR_CUDA, "copy q: %s", cudaGetErrorString(e));
   void* kc = const_cast<void*>(k);
   void* vtc = const_cast<void*>(vt);
   if ((s = pair ? attention_pair(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)
-                : attention(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
+                : attention_single(c, ws, kc, vtc, cap, n_q, pos0, n_keys, causal, st)) != DG_OK)
     return s;
   e = cudaMemcpyAsync(out, ws.at<void>(ws.L.o), (size_t)n_q * nq * 128 * 2, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess && out_lo)

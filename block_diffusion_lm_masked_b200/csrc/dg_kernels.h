@@ -81,11 +81,6 @@ struct TcAttnParams {
   int n_splits;
   float scale_log2;    // log2(e) / sqrt(d)
   int has_lo;          // query and current K/V carry low terms (bf16 model)
-  const __nv_bfloat16* q;     // query hi [nq][n_q][128] (read directly by tc_attn_kernel)
-  const __nv_bfloat16* q_lo;  // query lo, same layout
-  int* merge_cnt;             // [q tiles][nq] split tickets, zero on entry: when n_splits > 1 the
-                              // last split of a tile and head (head pair: ticket of its first
-                              // head) to finish merges the splits and leaves the ticket at zero
   int base;            // 128-aligned start of the low-term window (<= q_pos0)
   __nv_bfloat16* out;     // [n_q][nq * 128] when n_splits == 1 (hi part)
   __nv_bfloat16* out_lo;  // lo part, or null
@@ -93,10 +88,13 @@ struct TcAttnParams {
   float* part_lse;     // [n_splits][nq][n_q], log2 domain
   int* err;
 };
-// K / Vt: the cache; Kl / Vtl: low terms of the current K/V, rows (keys) counted from
-// `base`; the query comes from p.q / p.q_lo
-cudaError_t launch_tc_attention(const CUtensorMap& K, const CUtensorMap& Vt, const CUtensorMap& Kl,
-                                const CUtensorMap& Vtl, const TcAttnParams& p, cudaStream_t st);
+// Single-head kernel (chunks_per_split counts 128-key chunks; with n_splits > 1 the
+// partials go to part_o / part_lse for launch_attn_merge2).  Q / Ql: the query hi / lo
+// [nq][n_q][128]; K / Vt: the cache; Kl / Vtl: low terms of the current K/V, rows (keys)
+// counted from `base`; every map with 64 x 128 boxes.
+cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,
+                                const CUtensorMap& Vt, const CUtensorMap& Kl, const CUtensorMap& Vtl,
+                                const TcAttnParams& p, cudaStream_t st);
 // Head-pair variant (same parameters and outputs; chunks_per_split counts 128-key chunks):
 // K / Kl maps with 128-row boxes (64 d wide), Vt / Vtl as above.  pair_heads = 1: two heads of one KV
 // head per CTA where the group is even; 0: one head per CTA.  Grid y =
@@ -106,7 +104,7 @@ cudaError_t launch_tc_attention2(const CUtensorMap& Q, const CUtensorMap& Ql, co
                                  const TcAttnParams& p, int pair_heads, cudaStream_t st);
 int attn2_head_groups(int nq, int group, int pair_heads);
 // the head-pair path's split merge, one warp per (row, head) over the GPU, d = 128,
-// n_splits <= 32
+// n_splits <= 16
 cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
                                __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st);
 // ---------------------------------------------------------------- SIMT kernels (any dtype)
@@ -121,7 +119,7 @@ cudaError_t launch_embed_norm(const int32_t* tokens, const T* embed, int n, int 
 template <typename T>
 cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
                                 int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
-                                T* vt_lo, int lo_base, int lo_rows, int* zero_p, int zero_n, cudaStream_t st);
+                                T* vt_lo, int lo_base, int lo_rows, cudaStream_t st);
 cudaError_t launch_simt_gemm_f32(int epi_add, const float* W, const float* X, const int* group_off, int n_groups,
                                  int max_rows_per_group, int n_tokens, int M, int K, float* out, int ld_out,
                                  cudaStream_t st);

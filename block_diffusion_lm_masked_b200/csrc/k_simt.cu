@@ -90,12 +90,8 @@ template <typename T>
 __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, size_t part_stride, int nq, int nkv,
                                     int d, int pos0, float theta, int n, T* __restrict__ q, T* __restrict__ kc,
                                     T* __restrict__ vtc, int cap, T* __restrict__ q_lo, T* __restrict__ k_lo,
-                                    T* __restrict__ vt_lo, int lo_base, int lo_rows, int* __restrict__ zero_p,
-                                    int zero_n) {
+                                    T* __restrict__ vt_lo, int lo_base, int lo_rows) {
   griddep_sync();
-  // the next kernel's (attention's) split tickets start at zero
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero_p[i] = 0;
   extern __shared__ float cs[];  // [d/2] cos, [d/2] sin, then the summed qkv row
   const int t = blockIdx.x;
   const int half = d / 2;
@@ -171,12 +167,12 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int n_parts, 
 template <typename T>
 cudaError_t launch_rope_scatter(const float* qkv, int n_parts, size_t part_stride, int n, int nq, int nkv, int d,
                                 int pos0, float theta, T* q, T* kcache, T* vtcache, int cap, T* q_lo, T* k_lo,
-                                T* vt_lo, int lo_base, int lo_rows, int* zero_p, int zero_n, cudaStream_t st) {
+                                T* vt_lo, int lo_base, int lo_rows, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   if (n_parts < 1 || n_parts > kMaxSumParts) return cudaErrorInvalidValue;
   const size_t smem = (size_t)(d + (nq + 2 * nkv) * d) * sizeof(float);
   return launch_k(rope_scatter_kernel<T>, dim3(n), dim3(256), smem, st, qkv, n_parts, part_stride, nq, nkv, d, pos0,
-                  theta, n, q, kcache, vtcache, cap, q_lo, k_lo, vt_lo, lo_base, lo_rows, zero_p, zero_n);
+                  theta, n, q, kcache, vtcache, cap, q_lo, k_lo, vt_lo, lo_base, lo_rows);
 }
 
 // ---------------------------------------------------------------- fp32 GEMM (fp32 model)
@@ -1013,7 +1009,7 @@ cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream
   template cudaError_t launch_embed_norm<T>(const int32_t*, const T*, int, int, int, float, float*, T*, T*, int*, \
                                             cudaStream_t);                                                        \
   template cudaError_t launch_rope_scatter<T>(const float*, int, size_t, int, int, int, int, int, float, T*, T*,  \
-                                              T*, int, T*, T*, T*, int, int, int*, int, cudaStream_t);            \
+                                              T*, int, T*, T*, T*, int, int, cudaStream_t);                       \
   template cudaError_t launch_router_fused<T>(float*, const float*, int, size_t, const float*, int, int, int, int, \
                                               float, float*, int32_t*, float*, T*, T*, cudaStream_t);             \
   template cudaError_t launch_gather_rows<T>(const T*, const T*, const int32_t*, int, int, int, T*, T*,          \

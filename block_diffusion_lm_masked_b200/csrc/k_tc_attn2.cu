@@ -11,12 +11,7 @@
 //
 // TMEM (512 columns): per head one S/P region of 128 columns and O (128 columns).  The
 // softmax reads S (fp32, 128 keys) into registers and writes P over it as packed bf16
-// pairs (64 columns); the PV MMAs read P from there.  P enters the PV product as one bf16
-// term (the query keeps its hi + lo terms): each probability is rounded once (relative
-// error at most 2^-8), and the row sum adds the rounded values, so the output is an exact
-// weighted mean of V whose weights are off by at most 2^-8 relative -- at most
-// 2^-8 * sum_j p_j |v_j - o| / sum_j p_j per element, a few thousandths of the output's
-// RMS, against the two-term P's fp32 level and at a quarter fewer MMAs.
+// pairs, hi in the first 64 columns and lo in the next 64; the PV MMAs read P from there.
 // Shared memory: the query tiles (hi + lo, 64 KB per head) and a ring of three 32 KB
 // half-slots, each holding one chunk's K [128 keys][128 d] or V^T [128 d][128 keys] (two
 // 16 KB swizzled blocks); a chunk of the call's own keys also takes its K and V low terms.
@@ -248,6 +243,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           const uint32_t vo = (kk >> 2) * A2_BLK + (kk & 3) * 32;
           const uint64_t vd = sw128_kmajor_desc(v + vo);
           a2_mma_ts(o, pp + kk * 8, vd, idesc, (j > 0 || kk != 0) ? 1u : 0u);
+          a2_mma_ts(o, pp + 64 + kk * 8, vd, idesc, 1u);
           if (mp.n == 2) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
         }
         tc_commit(&pv_done[hl]);
@@ -344,14 +340,14 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         l2 = f2_mul(l2, f2_pack(alpha, alpha));
         m_used = cmax;
       }
-      // P = 2^(s * scale - m_used) (one rounding), rounded to bf16 and packed in pairs over
-      // this row's S (columns 0..63).  A row that has seen no key has m_used = -inf and
+      // P = 2^(s * scale - m_used) (one rounding), packed bf16 pairs over this row's S: hi
+      // in columns 0..63, lo in 64..127.  A row that has seen no key has m_used = -inf and
       // only -inf scores: its offset is taken as 0, so that every P is 2^-inf = 0.
       const float neg_m = (m_used == -INFINITY) ? 0.0f : -m_used;
       const uint64_t nm2 = f2_pack(neg_m, neg_m);
 #pragma unroll
       for (int c = 0; c < A2_W / 16; ++c) {  // 16 keys -> 8 packed columns per store
-        uint32_t wh[8];
+        uint32_t wh[8], wl[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int i0 = c * 16 + 2 * e;
@@ -360,13 +356,16 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
           float t0, t1;
           f2_unpack(t, t0, t1);
           const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-          // the PV product takes P in one bf16 term; the row sum adds the same rounded
-          // values, so the output is their exact weighted mean of V
+          const uint64_t pp = f2_pack(p0, p1);
+          l2 = f2_add(l2, pp);
           const uint32_t hi = bf16x2_pack(p0, p1);
-          l2 = f2_add(l2, bf16x2_widen(hi));
+          float lo0, lo1;
+          f2_unpack(f2_sub(pp, bf16x2_widen(hi)), lo0, lo1);
           wh[e] = hi;
+          wl[e] = bf16x2_pack(lo0, lo1);
         }
         tmem_st8(spa + c * 8, wh);
+        tmem_st8(spa + 64 + c * 8, wl);
       }
       tc_wait_st();
       tc_fence_before();
@@ -451,8 +450,8 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
 // of each tile would leave one CTA to read every split's partial rows (about 1 MB at the
 // large model's nine splits), a tail of tens of microseconds.  Lane s < n_splits reads split s's
 // log2-sum-exp, the warp takes their maximum and the weights exp2(lse_s - max) by
-// shuffles, and each lane merges four of the 128 output columns over the splits (the
-// splits' loads independent of one another), then writes the bf16 hi and lo parts.
+// shuffles, and each lane merges four of the 128 output columns over the splits (all the
+// splits' loads issued before the first product), then writes the bf16 hi and lo parts.
 // Rows with no visible key (every lse -inf) are written as zeros.
 __global__ void __launch_bounds__(256) attn_merge2_kernel(const float* __restrict__ part_o,
                                                           const float* __restrict__ part_lse, int n_splits, int nq,
@@ -470,15 +469,22 @@ __global__ void __launch_bounds__(256) attn_merge2_kernel(const float* __restric
   float den = wt;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  // every split's row slice loaded before the first product (same summation order)
+  constexpr int MAXS = 16;
+  float4 v[MAXS];
+#pragma unroll
+  for (int sp = 0; sp < MAXS; ++sp)
+    if (sp < n_splits) v[sp] = reinterpret_cast<const float4*>(part_o + (((size_t)sp * nq + h) * n_q + row) * A2_D)[lane];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sp = 0; sp < n_splits; ++sp) {
+#pragma unroll
+  for (int sp = 0; sp < MAXS; ++sp) {
+    if (sp >= n_splits) break;
     const float ws = __shfl_sync(0xffffffffu, wt, sp);
     if (ws == 0.0f) continue;  // uniform across the warp
-    const float4 v = reinterpret_cast<const float4*>(part_o + (((size_t)sp * nq + h) * n_q + row) * A2_D)[lane];
-    acc.x += ws * v.x;
-    acc.y += ws * v.y;
-    acc.z += ws * v.z;
-    acc.w += ws * v.w;
+    acc.x += ws * v[sp].x;
+    acc.y += ws * v[sp].y;
+    acc.z += ws * v[sp].z;
+    acc.w += ws * v[sp].w;
   }
   const float inv = den > 0.0f ? 1.0f / den : 0.0f;
   const float a[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
@@ -497,7 +503,7 @@ __global__ void __launch_bounds__(256) attn_merge2_kernel(const float* __restric
 
 cudaError_t launch_attn_merge2(const float* part_o, const float* part_lse, int n_splits, int nq, int n_q,
                                __nv_bfloat16* out, __nv_bfloat16* out_lo, cudaStream_t st) {
-  if (n_splits < 1 || n_splits > 32) return cudaErrorInvalidValue;
+  if (n_splits < 1 || n_splits > 16) return cudaErrorInvalidValue;
   const int warps = nq * n_q;
   return launch_k(attn_merge2_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, part_o, part_lse, n_splits, nq, n_q,
                   out, out_lo);

@@ -118,7 +118,8 @@ dg_status dg_debug_gemm_nv4(const void* W, const void* W_scales, float g, const 
                             int32_t x_rows, int32_t K, const int32_t* group_off, void* out, void* out_lo,
                             int32_t ld_out, void* d_scratch, size_t scratch_bytes, int32_t* d_err, dg_stream stream);
 
-/* One attention launch (bf16, head_dim 128), as in the pass: q [nq][n_q][128],
+/* One attention launch (bf16, head_dim 128) through the single-head kernel (one query
+ * head x 128 rows per CTA, two S buffers in TMEM), as in the pass: q [nq][n_q][128],
  * K [nkv][cap][128], Vt [nkv][128][cap]; queries at positions pos0.. over keys
  * [0, n_keys), causal or not.  out bf16 [n_q][nq * 128] (hi part); out_lo (nullable)
  * receives the lo part, out + out_lo = the fp32 attention output to ~16 bits.  d_ws: a

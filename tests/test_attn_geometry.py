@@ -10,7 +10,7 @@ the buffer or tensor map it addresses:
 - slots and query tiles stay inside the kernel's shared memory, TMEM columns below 512;
 - heads stay inside one KV head's group, and every output and partial index stays
   inside its buffer (partials: at most 16 splits of [nq][rows][128] fp32).
-The head-pair kernel's slot plan is also checked against the barrier simulation's.
+Both kernels' half-slot plans are also checked against the barrier simulation's.
 """
 
 import pytest
@@ -72,8 +72,9 @@ def debug_entry_accepts(n_q, pos0, n_keys, causal, cap, nq, nkv):
 
 
 class HalfSlotPlan:
-    """The head-pair kernel's half-slot plan (HalfSlotPlan::take): a chunk's K parts, then
-    its V^T parts, each the next half-slot of the ring."""
+    """The half-slot plan of both kernels (HalfSlotPlan::take in the head-pair kernel,
+    three half-slots; AtPlan::take in the single-head kernel, five): a chunk's K parts,
+    then its V^T parts, each the next half-slot of the ring."""
 
     def __init__(self, slots=3):
         self.nxt, self.uses, self.slots = 0, [0] * slots, slots
@@ -86,21 +87,6 @@ class HalfSlotPlan:
                 self.uses[self.nxt] += 1
                 self.nxt = (self.nxt + 1) % self.slots
         return k, v
-
-
-class SlotPlan:
-    """The single-head kernel's slot plan (AtSlotPlan::take)."""
-
-    def __init__(self, slots=3):
-        self.nxt, self.uses, self.slots = 0, [0] * slots, slots
-
-    def take(self, cur):
-        out = []
-        for _ in range(2 if cur else 1):
-            out.append((self.nxt, self.uses[self.nxt]))
-            self.uses[self.nxt] += 1
-            self.nxt = (self.nxt + 1) % self.slots
-        return out
 
 
 def check_tma(x, y, elem_bytes, y_extent):
@@ -126,11 +112,11 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
     else:
         n_splits, cps = splits_single(n_q, nq, n_keys)
         nh, ys = 1, nq
-        slot_bytes, slots = 65536, 3
-        smem_total = 1024 + slots * slot_bytes                 # the query tile lives in TMEM
-        assert smem_total <= 227 * 1024 - 1024
-        # TMEM columns: Q hi 0..63, lo 64..127, S 128..255, O 256..383, P hi 384..447, lo 448..511
-        cols = [(0, 64), (64, 64), (128, 128), (256, 128), (384, 64), (448, 64)]
+        smem_q, slot_bytes, slots = 4 * 16384, 32768, 5         # the query tile, five half-slots
+        smem_total = 1024 + smem_q + slots * slot_bytes
+        assert smem_total <= 227 * 1024 - 512
+        # TMEM columns: S buffers 0..127 and 128..255, O 256..383, P buffers 384..447 and 448..511
+        cols = [(0, 128), (128, 128), (256, 128), (384, 64), (448, 64)]
         assert sorted(cols) == cols and all(a + n <= b for (a, n), (b, _) in zip(cols, cols[1:]))
         assert cols[-1][0] + cols[-1][1] <= 512
     assert 1 <= n_splits <= MAX_SPLITS
@@ -147,18 +133,10 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
             kvh = h0 // group
             assert kvh < nkv and h0 + nh <= nq
             assert all((h0 + i) // group == kvh for i in range(nh)), "a CTA's heads span two KV heads"
-            if kernel == "pair":
-                for hl in range(nh):
-                    check_tma(0, q_row0, 2, n_q)
-                    check_tma(64, q_row0, 2, n_q)
-            else:
-                # the split ticket of this tile and head lies in the workspace's ticket array
-                assert qt * nq + h0 < cdiv(T, 128) * nq
-                # the softmax warps read their query rows (16-byte loads) for rows below n_q
-                for r in (q_row0, q_row0 + rows_here - 1):
-                    for hf in (0, 1):
-                        off = ((h0 * n_q + r) * D + hf * 64) * 2
-                        assert off % 16 == 0 and off + 128 <= nq * n_q * D * 2
+            for hl in range(nh):  # the query tiles (hi and lo maps: x = d 0 / 64, y = row, z = head)
+                assert h0 + hl < nq
+                check_tma(0, q_row0, 2, n_q)
+                check_tma(64, q_row0, 2, n_q)
             for sp in range(n_splits):
                 c_begin = sp * cps
                 nck = min(nch_total, c_begin + cps) - c_begin
@@ -168,34 +146,22 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                         for r in rows:
                             assert ((sp * nq + h) * n_q + r + 1) * D <= part_o_len
                     continue
-                plan = HalfSlotPlan() if kernel == "pair" else SlotPlan()
+                plan = HalfSlotPlan(slots)
                 for j in range(nck):
                     key0 = (c_begin + j) * W
                     assert key0 < kv_end
                     cur = key0 >= base
-                    if kernel == "pair":
-                        k_parts, v_parts = plan.take(cur)
-                        for i, ((sk, _), (sv, _)) in enumerate(zip(k_parts, v_parts)):
-                            krow = key0 if i == 0 else key0 - base
-                            extent = n_keys if i == 0 else n_keys - base
-                            assert krow % W == 0 and krow < extent
-                            check_tma(0, krow, 2, extent)       # K blocks: x = d 0 / 64, y = key row
-                            check_tma(64, krow, 2, extent)
-                            check_tma(krow, 0, 2, extent + 1)   # V^T blocks: x = key, key + 64; y = d 0
-                            check_tma(krow + 64, 0, 2, extent + 64)
-                            for hs in (sk, sv):
-                                assert hs < slots and smem_q + (hs + 1) * slot_bytes <= smem_total - 1024
-                    else:
-                        parts = plan.take(cur)
-                        for i, (s, _) in enumerate(parts):
-                            krow = key0 if i == 0 else key0 - base
-                            extent = n_keys if i == 0 else n_keys - base
-                            assert krow % W == 0
-                            check_tma(0, krow, 2, extent)           # K: x = d offset 0 / 64, y = key row
-                            check_tma(64, krow, 2, extent)
-                            check_tma(krow, 0, 2, extent + 1)       # V^T: x = key, y = d row 0
-                            assert krow < extent
-                            assert s < slots and (s + 1) * slot_bytes <= smem_total - 1024
+                    k_parts, v_parts = plan.take(cur)
+                    for i, ((sk, _), (sv, _)) in enumerate(zip(k_parts, v_parts)):
+                        krow = key0 if i == 0 else key0 - base
+                        extent = n_keys if i == 0 else n_keys - base
+                        assert krow % W == 0 and krow < extent
+                        check_tma(0, krow, 2, extent)       # K blocks: x = d 0 / 64, y = key row
+                        check_tma(64, krow, 2, extent)
+                        check_tma(krow, 0, 2, extent + 1)   # V^T blocks: x = key, key + 64; y = d 0
+                        check_tma(krow + 64, 0, 2, extent + 64)
+                        for hs in (sk, sv):
+                            assert hs < slots and smem_q + (hs + 1) * slot_bytes <= smem_total - 1024
                     chunks_seen += 1
                 if kernel == "pair":
                     for hl in range(nh):
@@ -300,12 +266,13 @@ def test_debug_entries_refuse_a_low_term_window_past_the_workspace():
         assert f(P, P, P, 4096, 64, 4097, 4096, 0, 2, 1, P, None, P, 1 << 30, None) == dg.DG_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("slots", [3, 5])
 @pytest.mark.parametrize("nck,cur_from", [(5, 2), (9, 0), (12, 8), (3, 3)])
-def test_kernel_slot_plan_is_the_simulated_one(nck, cur_from):
+def test_kernel_slot_plan_is_the_simulated_one(nck, cur_from, slots):
     import test_pipeline_protocol as TP
-    plan = HalfSlotPlan()
+    plan = HalfSlotPlan(slots)
     got = [plan.take(j >= cur_from) for j in range(nck)]
-    assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, 3)]
+    assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, slots)]
 
 
 def test_splits_fill_about_one_wave():

@@ -369,48 +369,35 @@ def test_the_checker_catches_a_wrong_count():
         _lowp_with_count(9, seed)
 
 
-# ---------------------------------------------------------------- the attention kernel (k_tc_attn.cu)
+# ---------------------------------------------------------------- the single-head attention kernel (k_tc_attn.cu)
 
-def slot_plan(nck, cur_from, slots):
-    """Slots of each chunk (tc_attn_kernel): a cached chunk takes the next slot, a current
-    chunk (the call's own keys: hi and lo parts) the next two; returns [(slots of chunk j,
-    use index of each)]."""
-    nxt, uses, plan = 0, [0] * slots, []
-    for j in range(nck):
-        k = 2 if j >= cur_from else 1
-        ss = [(nxt + i) % slots for i in range(k)]
-        plan.append([(x, uses[x]) for x in ss])
-        for x in ss:
-            uses[x] += 1
-        nxt = (nxt + k) % slots
-    return plan
+def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_at=None, drain=True,
+              load_drain=True, bug=None):
+    """tc_attn_kernel's hand-offs (128-key chunks, two S buffers, one P buffer): a load warp
+    fills the query tile, then a ring of `slots` half-slots with each chunk's K then its V^T;
+    the MMA thread issues S(j) into S buffer j & 1 (no wait of its own: PV(j - 2), issued
+    before it, waited for P(j - 2), which the softmax writes after reading S(j - 2)), a
+    commit freeing the K half-slots, then PV(j - 1) once P(j - 1) is written, and a commit
+    freeing its V half-slots; each softmax warp reads S(j), then -- once PV(j - 1) is
+    complete (O stable, P read) -- maybe rescales O, writes P(j) and signals.  Chunks [cur_from, nck) are the call's own (two half-slots per operand).
+    Every role reaches the exit barrier; the MMA thread drains its commits (`drain`), and
+    after an abort the load warp waits for the loads it issued (`load_drain`).
 
-
-def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, flags=None, give_up_at=None,
-              drain=True, load_drain=True, p_wait=True):
-    """tc_attn_kernel's hand-offs: the softmax warps store the query tile in TMEM and signal
-    (q_ready); a load warp fills `slots` K/V slots in plan order as they are freed; the MMA
-    warp issues S(j) into the one S buffer once the softmax warps have read S(j - 1), then
-    PV(j - 1) from the one P buffer and a commit per slot of chunk j - 1 that frees it
-    (PV(j - 1) first where chunks j - 1 and j need more slots than the ring has); each
-    softmax warp reads its half of S(j), exchanges its half-row max, waits for PV(j - 1)
-    (the last reader of P, and O stable for a rescale), writes its half of P and signals.
-    Chunks [cur_from, nck) are current (two slots each).  flags / give_up_at / load_drain:
-    abort mode as in attention_two_heads below; p_wait=False drops the softmax's wait for
-    PV(j - 1) before overwriting P."""
+    bug: "lag2" -- PV lags two chunks behind S (S(j), then PV(j - 2)), so S(j) no longer
+    follows P(j - 2); "no_pv_wait" -- P(j) written without waiting for PV(j - 1).
+    flags / give_up_at: abort mode as in attention_two_heads below."""
     rng = random.Random(seed * 7919 + nck)
-    plan = slot_plan(nck, nck if cur_from is None else cur_from, slots)
-    q_ready = Barrier("q_ready", n_warps)
-    kv_full = [Barrier(f"kv_full{s}", 1) for s in range(slots)]
-    kv_free = [Barrier(f"kv_free{s}", 1) for s in range(slots)]
-    s_full, s_free = Barrier("s_full", 1), Barrier("s_free", n_warps)
+    plan = half_slot_plan(nck, nck if cur_from is None else cur_from, slots)
+    q_bar = Barrier("q", 1)
+    hs_full = [Barrier(f"hs_full{s}", 1) for s in range(slots)]
+    hs_free = [Barrier(f"hs_free{s}", 1) for s in range(slots)]
+    s_full = [Barrier(f"s_full{b}", 1) for b in range(2)]
     p_ready, pv_done = Barrier("p_ready", n_warps), Barrier("pv_done", 1)
-    x_bar = [Barrier(f"x_bar{b}", n_warps) for b in range(2)]
-    l_bar, drain_bar = Barrier("l_bar", n_warps), Barrier("drain", 1)
+    drain_bar = Barrier("drain", 1)
     exit_bar = Barrier("exit", n_warps + 2)            # the __syncthreads every role reaches at the end
     bufs, q = Buffers(), Async()
-    st = dict(pv_issued=0, pv_done=0, s_done=0)
-    p_writes, x_writes = {}, {}
+    st = dict(pv_issued=0, pv_done=0)
+    p_writes = {}
     steps = [0]
 
     def bw(bar, parity, phase):
@@ -425,28 +412,34 @@ def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, 
         return flags is None or (bar.completed % 2) != parity
 
     def load():
+        q_bar.arrive_expect_tx(64)
+        q.loads.append(lambda: q_bar.complete_tx(64))
         loaded = [0] * slots
         ok = True
         for j in range(nck):
-            for x, u in plan[j]:
-                if u >= 1:
-                    yield bw(kv_free[x], (u - 1) & 1, u - 1)
-                    if not passed(kv_free[x], (u - 1) & 1):
-                        ok = False
-                        break
-                bufs.fill(("slot", x), 2)              # the S MMA and the PV MMA of chunk j read it
-                kv_full[x].arrive_expect_tx(32)
-                q.loads.append(lambda x=x: kv_full[x].complete_tx(32))
-                loaded[x] += 1
+            for parts in plan[j]:
+                for x, u in parts:
+                    if u >= 1:
+                        yield bw(hs_free[x], (u - 1) & 1, u - 1)
+                        if not passed(hs_free[x], (u - 1) & 1):
+                            ok = False
+                            break
+                    bufs.fill(("hs", x), 1)             # K: read by S(j); V^T: by PV(j)
+                    hs_full[x].arrive_expect_tx(32)
+                    q.loads.append(lambda x=x: hs_full[x].complete_tx(32))
+                    loaded[x] += 1
+                if not ok:
+                    break
             if not ok:
                 break
         # the kernel decides on the wind-down after every role has reached the exit barrier
         exit_bar.arrive()
         yield wait(exit_bar, 0, 0)
         if flags is not None and flags["abort"] and load_drain:
+            yield wait(q_bar, 0, None)
             for x in range(slots):
                 if loaded[x]:
-                    yield wait(kv_full[x], (loaded[x] - 1) & 1, None)
+                    yield wait(hs_full[x], (loaded[x] - 1) & 1, None)
 
     def leaving(body):
         """A role that reaches the exit barrier however its body ends."""
@@ -456,100 +449,83 @@ def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, 
             exit_bar.arrive()
 
     def mma():
-        def pv_chunk(k):
-            yield bw(p_ready, k & 1, k)
-            if not passed(p_ready, k & 1):
+        def do_pv(i):
+            for x, u in plan[i][1]:
+                yield bw(hs_full[x], u & 1, u)
+                if not passed(hs_full[x], u & 1):
+                    return False
+            yield bw(p_ready, i & 1, i)
+            if not passed(p_ready, i & 1):
                 return False
-            assert p_writes.get("p") == (k, n_warps), "PV read a P not fully written"
+            assert p_writes.get("p") == (i, n_warps), "PV read a P not fully written"
             st["pv_issued"] += 1
 
-            def done(k=k):
+            def fin(i=i):
                 st["pv_done"] += 1
                 for w in range(n_warps):
                     bufs.release(("p", w))
-                for x, _ in plan[k]:
-                    bufs.release(("slot", x))
+                for x, _ in plan[i][1]:
+                    bufs.release(("hs", x))
                 pv_done.arrive()
-            q.mma.append(done)
-            if k + 1 < nck:                            # the last chunk's slots are not reused
-                for x, _ in plan[k]:
-                    q.mma.append(lambda x=x: kv_free[x].arrive())
+            q.mma.append(fin)
+            for x, _ in plan[i][1]:
+                q.mma.append(lambda x=x: hs_free[x].arrive())
             return True
 
-        yield bw(q_ready, 0, 0)
-        ok = passed(q_ready, 0)
+        yield bw(q_bar, 0, 0)
+        ok = passed(q_bar, 0)
         for j in range(nck if ok else 0):
-            pv_first = pv_first_rule and j >= 1 and len(plan[j - 1]) + len(plan[j]) > slots
-            if pv_first:
-                ok = yield from pv_chunk(j - 1)
-                if not ok:
-                    break
-            for x, u in plan[j]:
-                yield bw(kv_full[x], u & 1, u)
-                if not passed(kv_full[x], u & 1):
+            b = j & 1
+            for x, u in plan[j][0]:
+                yield bw(hs_full[x], u & 1, u)
+                if not passed(hs_full[x], u & 1):
                     ok = False
                     break
-            if ok and j >= 1:
-                yield bw(s_free, (j - 1) & 1, j - 1)
-                ok = passed(s_free, (j - 1) & 1)
             if not ok:
                 break
-            for w in range(n_warps):                   # S: each softmax warp reads its half of its lanes
-                bufs.fill(("S", w), 1)
+            for w in range(n_warps):                   # S(j): each softmax warp reads its 32 lanes
+                bufs.fill(("S", b, w), 1)
 
-            def s_done(j=j):
-                st["s_done"] += 1
-                for x, _ in plan[j]:
-                    bufs.release(("slot", x))
-                s_full.arrive()
+            def s_done(j=j, b=b):
+                for x, _ in plan[j][0]:
+                    bufs.release(("hs", x))
+                s_full[b].arrive()
             q.mma.append(s_done)
-            if j >= 1 and not pv_first:
-                ok = yield from pv_chunk(j - 1)
+            for x, _ in plan[j][0]:
+                q.mma.append(lambda x=x: hs_free[x].arrive())
+            lag = 2 if bug == "lag2" else 1
+            if j >= lag:
+                ok = yield from do_pv(j - lag)
                 if not ok:
                     break
-        if ok:
-            yield from pv_chunk(nck - 1)
+        for i in range(max(nck - (2 if bug == "lag2" else 1), 0), nck):
+            if not ok:
+                break
+            ok = yield from do_pv(i)
         if drain:
             q.mma.append(lambda: drain_bar.arrive())
             yield wait(drain_bar, 0, 0)
 
     def softmax(w):
-        q_ready.arrive()                               # this warp's part of the query tile is in TMEM
         for j in range(nck):
-            yield bw(s_full, j & 1, j)
-            if not passed(s_full, j & 1):
+            b = j & 1
+            yield bw(s_full[b], (j >> 1) & 1, j >> 1)
+            if not passed(s_full[b], (j >> 1) & 1):
                 return
-            assert st["s_done"] == j + 1
-            bufs.release(("S", w))
-            s_free.arrive()
-            last, n = x_writes.get(j & 1, (None, 0))
-            if last != j:
-                bufs.fill(("x", j & 1), n_warps)
-                x_writes[j & 1] = (j, 1)
-            else:
-                x_writes[j & 1] = (j, n + 1)
-            x_bar[j & 1].arrive()
-            yield bw(x_bar[j & 1], (j >> 1) & 1, j >> 1)
-            if not passed(x_bar[j & 1], (j >> 1) & 1):
-                return
-            assert x_writes[j & 1] == (j, n_warps), "a row max read before both halves posted"
-            bufs.release(("x", j & 1))
-            if j >= 1 and p_wait:
+            bufs.release(("S", b, w))                  # this warp's lanes of S(j) read into registers
+            if j > 0 and bug != "no_pv_wait":
                 yield bw(pv_done, (j - 1) & 1, j - 1)
                 if not passed(pv_done, (j - 1) & 1):
                     return
                 if rng.random() < 0.4:                 # some row's max grew: O is rescaled here
                     assert st["pv_done"] >= j and st["pv_issued"] <= j, "O rescaled while a PV may write it"
-            bufs.fill(("p", w), 1)                     # this warp's half of P, read by PV(j)
+            bufs.fill(("p", w), 1)                     # this warp's lanes of P(j), read by PV(j)
             last, n = p_writes.get("p", (None, 0))
             p_writes["p"] = (j, 1) if last != j else (j, n + 1)
             p_ready.arrive()
         yield bw(pv_done, (nck - 1) & 1, nck - 1)
-        if not passed(pv_done, (nck - 1) & 1):
-            return
-        assert st["pv_done"] == nck
-        l_bar.arrive()
-        yield bw(l_bar, 0, 0)
+        if passed(pv_done, (nck - 1) & 1):
+            assert st["pv_done"] == nck
 
     roles = {"load": load(), "mma": leaving(mma())}
     roles.update({f"sm{w}": leaving(softmax(w)) for w in range(n_warps)})
@@ -559,27 +535,50 @@ def attention(nck, seed, cur_from=None, slots=3, n_warps=8, pv_first_rule=True, 
 @pytest.mark.parametrize("nck,cur_from", [(1, 1), (1, 0), (2, 2), (2, 1), (2, 0), (3, 3), (4, 2), (5, 3), (6, 0),
                                           (7, 5), (9, 9), (12, 10)])
 def test_attention_protocol(nck, cur_from):
-    """No deadlock, no overrun, no K/V slot, S or P refilled while read, no P read before all
-    its writers, no O rescaled under a PV, nothing in flight when the CTA leaves."""
+    """No deadlock, no overrun, no half-slot, S or P buffer refilled while read, no P read
+    before all its writers, no O rescaled under a PV, nothing in flight when the CTA leaves."""
     for seed in range(30):
         roles, q = attention(nck, seed, cur_from=cur_from)
         run(roles, q, seed, end_check=True)
 
 
-def test_attention_protocol_catches_its_planted_mistakes():
-    """Without the PV-first rule two current chunks deadlock the three-slot ring; without the
-    softmax's wait for the previous PV, P is overwritten while that PV reads it."""
-    with pytest.raises(AssertionError, match="deadlock"):
-        roles, q = attention(4, 0, cur_from=2, pv_first_rule=False)
-        run(roles, q, 0)
+@pytest.mark.parametrize("bug", ["lag2", "no_pv_wait"])
+def test_attention_protocol_catches_its_planted_mistakes(bug):
+    """S(j) issued before the softmax has read S(j - 2) from the same buffer (PV lagging two
+    chunks), or P(j) written before PV(j - 1) has read P(j - 1): some interleaving
+    overwrites a buffer still read, or deadlocks."""
     caught = 0
-    for seed in range(30):
-        roles, q = attention(5, seed, p_wait=False)
+    for seed in range(60):
+        roles, q = attention(6, seed, cur_from=4, bug=bug)
         try:
-            run(roles, q, seed)
+            run(roles, q, seed, end_check=True)
         except AssertionError as e:
-            caught += "overwritten" in str(e) or "PV read" in str(e)
+            caught += any(m in str(e) for m in ("overwritten", "PV read", "rescaled", "deadlock"))
     assert caught > 0
+
+
+def test_attention_with_a_smaller_ring_deadlocks():
+    """The ring must hold chunk j's K beside chunk j - 1's unread V^T: two chunks of own keys
+    need four half-slots, and a ring of three deadlocks on them."""
+    with pytest.raises(AssertionError, match="deadlock"):
+        roles, q = attention(4, 0, cur_from=2, slots=3)
+        run(roles, q, 0)
+    for seed in range(20):
+        roles, q = attention(6, seed, cur_from=2, slots=4)
+        run(roles, q, seed, end_check=True)
+
+
+def test_attention_leaves_nothing_in_flight():
+    """Without the MMA thread's drain some interleaving leaves a commit landing after the
+    CTA is gone."""
+    left = 0
+    for seed in range(60):
+        roles, q = attention(6, seed, cur_from=4, drain=False)
+        try:
+            run(roles, q, seed, end_check=True)
+        except AssertionError as e:
+            left += "pending" in str(e)
+    assert left > 0
 
 
 @pytest.mark.parametrize("nck,cur_from", [(4, 2), (7, 4), (6, 0), (3, 3)])
