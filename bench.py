@@ -718,7 +718,7 @@ def run_kernel_attention(args):
     ws = dg.Workspace(cfg, n_q, dev)
     out = torch.zeros(n_q, nq * d, dtype=torch.bfloat16, device=dev)
     lo = torch.zeros_like(out)
-    fn = dg.debug_attention_bf16 if args.attn_single else dg.debug_attention_pair_bf16
+    fn = dg.debug_attention_pair_bf16 if args.attn_pair else dg.debug_attention_bf16
     us = _graph_time(lambda: fn(q, k, vt, n_keys, n_keys - n_q, False, out, ws, out_lo=lo), args.steps,
                      args.warmup)
     dg.device_status(ws)
@@ -729,7 +729,7 @@ def run_kernel_attention(args):
             "higher_is_better": False, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
             "data": "synthetic: q, K, V ~ N(0,1) bf16",
             "config": {"workload": f"attention: {n_q} queries x {nq} heads ({nkv} KV heads) d{d} over {n_keys} keys, "
-                                   f"bidirectional", "attention": "head pairs, 128-key chunks" if not args.attn_single
+                                   f"bidirectional", "attention": "head pairs, 128-key chunks" if args.attn_pair
                        else "one head, 128-key chunks", "l2": "K/V re-read between calls"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s", "frac": tf / tf_burst,
                          "flops_per_call": fl, "peak_source": f"{peak_src} bf16_tflops"}}
@@ -804,8 +804,8 @@ def run_kernel_gemm(args):
 
 
 def _attention_kind():
-    """Which attention kernel the library runs (DG_ATTN_SINGLE=1: the single-head kernel)."""
-    return ("head pairs, 128-key chunks" if os.environ.get("DG_ATTN_SINGLE", "")[:1] != "1"
+    """Which attention kernel the library runs (DG_ATTN_PAIR=1: the head-pair kernel)."""
+    return ("head pairs, 128-key chunks" if os.environ.get("DG_ATTN_PAIR", "")[:1] == "1"
             else "one head, 128-key chunks")
 
 
@@ -831,9 +831,9 @@ def main():
                     help="expert weight storage; mx8 and nv4 run through the batched calls")
     ap.add_argument("--vocab", default="bf16", choices=["bf16", "mx8", "nv4"],
                     help="output-matrix storage; mx8 and nv4 run through the batched calls")
-    ap.add_argument("--attn-single", action="store_true",
-                    help="run attention through the single-head kernel instead of the head-pair kernel "
-                         "(sets DG_ATTN_SINGLE=1)")
+    ap.add_argument("--attn-pair", action="store_true",
+                    help="run attention through the head-pair kernel instead of the single-head kernel "
+                         "(sets DG_ATTN_PAIR=1)")
     ap.add_argument("--kernel", choices=["attention", "gemm"], default=None,
                     help="time one kernel alone on synthetic data instead of the step (attention: the "
                          "block-masked attention call over --keys keys; gemm: one GEMM of the large model's "
@@ -849,8 +849,8 @@ def main():
         return run_kernel_attention(args)
     if args.kernel == "gemm":
         return run_kernel_gemm(args)
-    if args.attn_single:  # read by the library at its first attention call
-        os.environ["DG_ATTN_SINGLE"] = "1"
+    if args.attn_pair:  # read by the library at its first attention call
+        os.environ["DG_ATTN_PAIR"] = "1"
     name = args.workload
     cfg = CF.CONFIGS[name]
     if args.impl == "reference":

@@ -601,11 +601,11 @@ int attn_pair_splits(int n_q, int nq, int group, int pair_heads, int n_keys, int
   return splits;
 }
 
-// The bf16 pass's attention runs the head-pair kernel; DG_ATTN_SINGLE=1 routes it
-// through the single-head kernel (tc_attn_kernel) instead
+// The bf16 pass's attention runs the single-head kernel (tc_attn_kernel); DG_ATTN_PAIR=1
+// routes it through the head-pair kernel (tc_attn2_kernel) instead
 bool attn_pair_enabled() {
-  static const bool single = getenv("DG_ATTN_SINGLE") != nullptr && getenv("DG_ATTN_SINGLE")[0] == '1';
-  return !single;
+  static const bool pair = getenv("DG_ATTN_PAIR") != nullptr && getenv("DG_ATTN_PAIR")[0] == '1';
+  return pair;
 }
 
 // The tensor maps both attention kernels read: the query hi / lo [nq][n_q][128], the

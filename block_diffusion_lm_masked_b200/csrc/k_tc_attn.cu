@@ -16,27 +16,26 @@
 // start `base` at or below the first current position; rows before the first current
 // position are zero there.
 //
-// Layout.  Shared memory: the query tile (hi + lo, 64 KB, TMA) and a ring of five 32 KB
-// half-slots, each holding one chunk's K [128 keys][128 d] or V^T [128 d][128 keys] (two
-// 16 KB blocks, 128-byte swizzled); a chunk of the call's own keys also takes its K and V
-// low terms.  Ring order per chunk: K (and K lo), then V (and V lo).
+// Layout.  Shared memory: the query tile (hi + lo, 64 KB, TMA), a ring of two 32 KB
+// half-slots for K [128 keys][128 d] and one of three for V^T [128 d][128 keys] (two 16 KB
+// blocks each, 128-byte swizzled); a chunk of the call's own keys takes two entries of
+// each ring (hi, then lo).
 // TMEM (512 columns): two S buffers (fp32, 128 keys) at 0 and 128, O at 256, and P at 384
 // (packed bf16 pairs along the keys: hi in 384..447, lo in 448..511).  Chunk j uses S
 // buffer j & 1.
 //
 // Roles.  Warps 0-3 run the softmax, one query row per thread (its TMEM lane) over the
 // whole 128-key chunk, so no row statistics are exchanged between warps; warp 4 issues the
-// TMA loads; warp 5 the MMAs.  The MMA thread issues S(0), then per chunk j >= 1: S(j), a
-// commit freeing chunk j's K half-slots, then PV(j - 1) once the softmax has written
-// P(j - 1), and a commit freeing its V half-slots.  S(j) needs no wait of its own for its
-// buffer: it is issued after PV(j - 2), which waited for P(j - 2), and the softmax writes
-// P(j - 2) only after it has read S(j - 2) out of that buffer.  So the tensor cores compute
-// S(j + 1) while the softmax works on S(j),
-// and the softmax takes chunk j + 1 as soon as it has handed P(j) over.  The softmax of
-// chunk j computes P(j) in registers, then, once PV(j - 1) is complete, rescales O (lazily,
-// when its row maximum grew by more than 2^8) and writes P(j) over P(j - 1); so the tensor
-// cores run PV(j - 1) and S(j + 1) while the softmax computes.  Hand-offs are mbarriers
-// with bounded waits.
+// TMA loads; warps 5 and 6 issue the MMAs, one thread each: warp 5 the S MMAs, S(j) once
+// chunk j's K has landed and the softmax has read S(j - 2) out of the same buffer, then a
+// commit freeing the K half-slots; warp 6 the PV MMAs, PV(j) once chunk j's V^T has landed
+// and the softmax has written P(j), then a commit freeing the V^T half-slots.  Each issuing
+// thread's waits and commits (a few hundred nanoseconds each, measured) then run while the
+// tensor cores execute the other thread's MMAs, and the tensor cores compute S(j + 1) and
+// PV(j - 1) while the softmax works on S(j).  The softmax of chunk j computes P(j) in
+// registers, then, once PV(j - 1) is complete, rescales O (lazily, when its row maximum
+// grew by more than 2^8) and writes P(j) over P(j - 1).  Hand-offs are mbarriers with
+// bounded waits.
 #include <math.h>
 
 #include "attn_softmax.cuh"
@@ -48,15 +47,18 @@ namespace dg {
 constexpr int AT_BQ = 128;
 constexpr int AT_W = 128;                       // keys per chunk
 constexpr int AT_D = 128;
-constexpr int AT_HSLOTS = 5;                    // half-slots of the K/V ring
+constexpr int AT_KSLOTS = 2;                    // half-slots of the K ring
+constexpr int AT_VSLOTS = 3;                    // half-slots of the V^T ring (after the K ring's)
+constexpr int AT_HSLOTS = AT_KSLOTS + AT_VSLOTS;
 constexpr uint32_t AT_BLK = 128 * 128;          // [128 rows][64 bf16] swizzled block: 16 KB
 constexpr uint32_t AT_QTILE = 4 * AT_BLK;       // Q hi (two d blocks) + Q lo (two d blocks): 64 KB
 constexpr uint32_t AT_HSLOT = 2 * AT_BLK;       // K (two d blocks) or V^T (two key blocks): 32 KB
 constexpr int AT_SMEM = 1024 + AT_QTILE + AT_HSLOTS * AT_HSLOT;
 constexpr int AT_SM_WARPS = 4;
 constexpr int AT_LOAD_WARP = 4;
-constexpr int AT_MMA_WARP = 5;
-constexpr int AT_THREADS = 32 * 6;
+constexpr int AT_S_WARP = 5;    // issues the S MMAs (and holds the TMEM allocation)
+constexpr int AT_PV_WARP = 6;   // issues the PV MMAs
+constexpr int AT_THREADS = 32 * 7;
 static_assert(AT_SMEM <= 227 * 1024 - 512, "shared memory budget");
 
 // TMEM column offsets
@@ -75,30 +77,19 @@ __device__ __forceinline__ void at_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// The half-slot plan both the load and the MMA warp follow: chunk j takes the next one
-// (cached keys) or two (own keys: hi, lo) half-slots for its K, then as many for its V^T.
-// The MMA thread holds chunk j's K parts and chunk j - 1's V parts at once: entries [j & 1].
-struct AtPlan {
-  int nxt = 0;
-  int uses[AT_HSLOTS] = {0, 0, 0, 0, 0};
-  int n[2];                // parts per operand: 1, or 2 for a chunk of own keys
-  int ks[2][2], ku[2][2];  // [j & 1][part]: K half-slot, its use index
-  int vs[2][2], vu[2][2];  // V^T half-slots
-  __device__ void take(int j, bool cur) {
-    const int b = j & 1;
-    n[b] = cur ? 2 : 1;
-    for (int i = 0; i < n[b]; ++i) {
-      ks[b][i] = nxt;
-      ku[b][i] = uses[nxt]++;
-      nxt = nxt + 1 == AT_HSLOTS ? 0 : nxt + 1;
-    }
-    for (int i = 0; i < n[b]; ++i) {
-      vs[b][i] = nxt;
-      vu[b][i] = uses[nxt]++;
-      nxt = nxt + 1 == AT_HSLOTS ? 0 : nxt + 1;
-    }
-  }
-};
+// The two half-slot rings, as plain arithmetic (no indexed arrays, so nothing spills to
+// local memory).  Chunk j's K parts (one, or two for own keys: hi, lo) take the next
+// entries of the K ring, its V^T parts those of the V^T ring; K entry e lives in half-slot
+// e % AT_KSLOTS, V^T entry e in half-slot AT_KSLOTS + e % AT_VSLOTS, as that half-slot's
+// use e / (ring size).  Each ring has one consumer (the S thread, the PV thread), which
+// waits for its entries in order: so no wait can meet a half-slot whose previous use has
+// not landed yet (a parity wait there would pass at once).
+__device__ __forceinline__ int at_kslot(int e) { return e % AT_KSLOTS; }
+__device__ __forceinline__ int at_vslot(int e) { return AT_KSLOTS + e % AT_VSLOTS; }
+__device__ __forceinline__ uint32_t at_kparity(int e) { return (uint32_t)(e / AT_KSLOTS) & 1u; }
+__device__ __forceinline__ uint32_t at_vparity(int e) { return (uint32_t)(e / AT_VSLOTS) & 1u; }
+// loads issued into the ring's slot r (0-based within the ring) when its first n entries were issued
+__device__ __forceinline__ int at_loads_into(int r, int n, int ring) { return n > r ? (n - 1 - r) / ring + 1 : 0; }
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
@@ -110,6 +101,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __shared__ __align__(8) uint64_t hs_full[AT_HSLOTS];  // the half-slot's TMA loads have landed
   __shared__ __align__(8) uint64_t hs_free[AT_HSLOTS];  // the MMAs reading the half-slot are complete
   __shared__ __align__(8) uint64_t s_full[2];           // [buffer]: S of the chunk is in TMEM
+  __shared__ __align__(8) uint64_t s_free[2];           // [buffer]: the softmax warps have read S
   __shared__ __align__(8) uint64_t p_ready;             // P of the chunk is in TMEM
   __shared__ __align__(8) uint64_t pv_done;             // the PV of the chunk is complete
   __shared__ __align__(8) uint64_t drain_bar;
@@ -143,7 +135,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint8_t* sQ = smem;                // [Q hi blk0, blk1, Q lo blk0, blk1]
   uint8_t* sHalf = smem + AT_QTILE;  // [half-slot][blk0, blk1]
 
-  if (warp == AT_MMA_WARP) tmem_alloc(&tmem_base_s, 512);
+  if (warp == AT_S_WARP) tmem_alloc(&tmem_base_s, 512);
   if (tid == AT_LOAD_WARP * 32) {
     mbar_init(&q_bar, 1);
     for (int s = 0; s < AT_HSLOTS; ++s) {
@@ -152,10 +144,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], AT_SM_WARPS);
     }
     mbar_init(&p_ready, AT_SM_WARPS);
     mbar_init(&pv_done, 1);
-    mbar_init(&drain_bar, 1);
+    mbar_init(&drain_bar, 2);  // one commit per issuing thread
     abort_s = 0;
     fence_barrier_init();
   }
@@ -169,7 +162,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   // own keys (key0 >= base) also carry low terms and take two half-slots per operand
   auto is_cur = [&](int j) { return p.has_lo && (c_begin + j) * AT_W >= p.base; };
   const uint32_t idesc = idesc_bf16_f32(AT_BQ, AT_W);  // S: 128 rows x 128 keys; PV: 128 rows x 128 d
-  int loaded[AT_HSLOTS] = {0, 0, 0, 0, 0};  // loads the load thread issued into each half-slot
+  int issued_k = 0, issued_v = 0;  // ring entries the load thread issued loads for (for the wind-down)
   bool q_issued = false;
 
   if (warp == AT_LOAD_WARP) {
@@ -189,18 +182,21 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tma_load_3d(sQ + 2 * AT_BLK, &tmQl, 0, q_row0, h, &q_bar);
       tma_load_3d(sQ + 3 * AT_BLK, &tmQl, 64, q_row0, h, &q_bar);
       q_issued = true;
-      AtPlan lp;
       bool ok = true;
-      // one half-slot: wait until its previous use was freed, then its two 16 KB blocks
-      auto load_half = [&](int s, int u, const CUtensorMap* map, bool is_v, int krow) {
-        if (u >= 1 && !mbar_wait(&hs_free[s], (uint32_t)(u - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
+      // entry e of the K (or V^T) ring: wait until its half-slot's previous use was freed,
+      // then its two 16 KB blocks
+      auto load_half = [&](int e, const CUtensorMap* map, bool is_v, int krow) {
+        const int ring = is_v ? AT_VSLOTS : AT_KSLOTS;
+        const int s = is_v ? at_vslot(e) : at_kslot(e);
+        if (e >= ring && !mbar_wait(&hs_free[s], is_v ? at_vparity(e - ring) : at_kparity(e - ring), &abort_s,
+                                    p.err, DG_DEVERR_TIMEOUT_ATTN))
           return false;
         if (!DG_GUARD(krow >= 0 && krow % AT_W == 0, p.err)) {
           abort_s = 1;
           return false;
         }
         uint8_t* dst = sHalf + s * AT_HSLOT;
-        loaded[s] += 1;
+        (is_v ? issued_v : issued_k) = e + 1;
         mbar_arrive_expect_tx(&hs_full[s], AT_HSLOT);
         if (is_v) {  // V^T [128 d][64 keys] blocks: keys krow .. +63, +64 .. +127
           tma_load_3d(dst, map, krow, 0, kvh, &hs_full[s]);
@@ -211,29 +207,28 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         }
         return true;
       };
-      for (int j = 0; j < nck && ok; ++j) {
+      for (int j = 0, e = 0; j < nck && ok; ++j) {  // e: chunk j's first entry in either ring
         const int key0 = (c_begin + j) * AT_W;
-        const int b = j & 1;
-        lp.take(j, is_cur(j));
+        const int n = is_cur(j) ? 2 : 1;
         // part 0: the cache's bf16 keys; part 1: the low terms, rows counted from `base`
-        for (int i = 0; i < lp.n[b] && ok; ++i)
-          ok = load_half(lp.ks[b][i], lp.ku[b][i], i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
-        for (int i = 0; i < lp.n[b] && ok; ++i)
-          ok = load_half(lp.vs[b][i], lp.vu[b][i], i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
+        for (int i = 0; i < n && ok; ++i)
+          ok = load_half(e + i, i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
+        for (int i = 0; i < n && ok; ++i)
+          ok = load_half(e + i, i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
+        e += n;
       }
     }
     __syncwarp();
-  } else if (warp == AT_MMA_WARP) {
+  } else if (warp == AT_S_WARP || warp == AT_PV_WARP) {
     if (lane == 0) {
-      // ================= MMAs: S(0); per chunk j >= 1: S(j), PV(j - 1); then PV(last)
-      AtPlan mp;
+      // ================= MMAs: warp 5 the S MMAs, warp 6 the PV MMAs, in chunk order
       auto half_addr = [&](int s) { return smem_u32(sHalf + s * AT_HSLOT); };
       const uint32_t q = smem_u32(sQ), ql = q + 2 * AT_BLK;
-      auto issue_s = [&](int j) {
-        const int b = j & 1;
-        const uint32_t d = tmem + at_s(b);
-        const uint32_t k = half_addr(mp.ks[b][0]);
-        const uint32_t kl = mp.n[b] == 2 ? half_addr(mp.ks[b][1]) : 0u;
+      // S(j): K parts at ring entries ek, ek + 1
+      auto issue_s = [&](int j, int ek, int n) {
+        const uint32_t d = tmem + at_s(j & 1);
+        const uint32_t k = half_addr(at_kslot(ek));
+        const uint32_t kl = n == 2 ? half_addr(at_kslot(ek + 1)) : 0u;
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -242,51 +237,58 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             const uint64_t kd = sw128_kmajor_desc(k + o);
             tc_mma(d, sw128_kmajor_desc(q + o), kd, idesc, (kb | kk) != 0 ? 1u : 0u);
             tc_mma(d, sw128_kmajor_desc(ql + o), kd, idesc, 1u);
-            if (mp.n[b] == 2) tc_mma(d, sw128_kmajor_desc(q + o), sw128_kmajor_desc(kl + o), idesc, 1u);
+            if (n == 2) tc_mma(d, sw128_kmajor_desc(q + o), sw128_kmajor_desc(kl + o), idesc, 1u);
           }
-        tc_commit(&s_full[b]);
+        tc_commit(&s_full[j & 1]);
       };
-      // PV of chunk i once its V^T has landed and the softmax has written P(i); then the
-      // commits that free its V half-slots
-      auto do_pv = [&](int i) {
-        const int b = i & 1;
+      // PV of chunk i once its V^T (ring entries ev, ev + 1) has landed and the softmax has
+      // written P(i); then the commits that free its V half-slots
+      auto do_pv = [&](int i, int ev, int n) {
         bool ok2 = true;
-        for (int t = 0; t < mp.n[b] && ok2; ++t)
-          ok2 = mbar_wait(&hs_full[mp.vs[b][t]], (uint32_t)mp.vu[b][t] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        for (int t = 0; t < n && ok2; ++t)
+          ok2 = mbar_wait(&hs_full[at_vslot(ev + t)], at_vparity(ev + t), &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (ok2) ok2 = mbar_wait(&p_ready, (uint32_t)i & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (!ok2) return false;
         tc_fence_after();
         const uint32_t o = tmem + AT_O, ph = tmem + AT_PHI, pl = tmem + AT_PLO;
-        const uint32_t v = half_addr(mp.vs[b][0]);
-        const uint32_t vl = mp.n[b] == 2 ? half_addr(mp.vs[b][1]) : 0u;
+        const uint32_t v = half_addr(at_vslot(ev));
+        const uint32_t vl = n == 2 ? half_addr(at_vslot(ev + 1)) : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 16 keys = 8 packed P columns per MMA
           const uint32_t vo = (kk >> 2) * AT_BLK + (kk & 3) * 32;
           const uint64_t vd = sw128_kmajor_desc(v + vo);
           at_mma_ts(o, ph + kk * 8, vd, idesc, (i > 0 || kk != 0) ? 1u : 0u);
           at_mma_ts(o, pl + kk * 8, vd, idesc, 1u);
-          if (mp.n[b] == 2) at_mma_ts(o, ph + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
+          if (n == 2) at_mma_ts(o, ph + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
         }
         tc_commit(&pv_done);
-        for (int t = 0; t < mp.n[b]; ++t) tc_commit(&hs_free[mp.vs[b][t]]);
+        for (int t = 0; t < n; ++t) tc_commit(&hs_free[at_vslot(ev + t)]);
         return true;
       };
 
-      bool ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-      for (int j = 0; j < nck && ok; ++j) {
-        const int b = j & 1;
-        mp.take(j, is_cur(j));
-        for (int t = 0; t < mp.n[b] && ok; ++t)
-          ok = mbar_wait(&hs_full[mp.ks[b][t]], (uint32_t)mp.ku[b][t] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-        // (S buffer b was read by the softmax of chunk j - 2 before it wrote P(j - 2), which
-        // PV(j - 2), issued in the previous iteration, waited for)
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(j);
-        for (int t = 0; t < mp.n[b]; ++t) tc_commit(&hs_free[mp.ks[b][t]]);
-        if (j >= 1) ok = do_pv(j - 1);
+      if (warp == AT_S_WARP) {
+        bool ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        for (int j = 0, e = 0; j < nck && ok; ++j) {  // e: chunk j's first K entry
+          const int n = is_cur(j) ? 2 : 1;
+          for (int t = 0; t < n && ok; ++t)
+            ok = mbar_wait(&hs_full[at_kslot(e + t)], at_kparity(e + t), &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+          // S buffer j & 1 was last read by the softmax of chunk j - 2
+          if (ok && j >= 2)
+            ok = mbar_wait(&s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j, e, n);
+          for (int t = 0; t < n; ++t) tc_commit(&hs_free[at_kslot(e + t)]);
+          e += n;
+        }
+      } else {
+        bool ok = true;
+        for (int j = 0, e = 0; j < nck && ok; ++j) {  // e: chunk j's first V^T entry
+          const int n = is_cur(j) ? 2 : 1;
+          ok = do_pv(j, e, n);
+          e += n;
+        }
       }
-      if (ok) do_pv(nck - 1);
     }
     __syncwarp();
   } else {
@@ -314,6 +316,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
       for (int c = 0; c < AT_W / 16; ++c) tmem_ld16(tmem + at_s(b) + lane_off + c * 16, r[c]);
       tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);  // S(j + 2) may go into this buffer
       const int key0 = (c_begin + j) * AT_W;
       // keys at or past the row's limit (only in the chunk that holds the limit)
       if (__any_sync(0xffffffffu, key0 + AT_W > key_lim)) {
@@ -454,18 +459,22 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   // wind down: every MMA and commit the MMA thread issued has landed (also on the normal
   // path, so that no mbarrier arrive reaches this CTA's shared memory after it is gone),
   // and after an abort the loads the load thread issued have landed too
-  if (tid == AT_MMA_WARP * 32) {
-    tc_commit(&drain_bar);
-    mbar_wait_drain(&drain_bar, 0);
-  }
+  if (lane == 0 && (warp == AT_S_WARP || warp == AT_PV_WARP)) tc_commit(&drain_bar);
+  if (tid == AT_S_WARP * 32) mbar_wait_drain(&drain_bar, 0);
   if (abort_s && tid == AT_LOAD_WARP * 32) {
     if (q_issued) mbar_wait_drain(&q_bar, 0);
-    for (int s = 0; s < AT_HSLOTS; ++s)
-      if (loaded[s] > 0) mbar_wait_drain(&hs_full[s], (uint32_t)(loaded[s] - 1) & 1u);
+    for (int r = 0; r < AT_KSLOTS; ++r) {
+      const int loads = at_loads_into(r, issued_k, AT_KSLOTS);
+      if (loads > 0) mbar_wait_drain(&hs_full[r], (uint32_t)(loads - 1) & 1u);
+    }
+    for (int r = 0; r < AT_VSLOTS; ++r) {
+      const int loads = at_loads_into(r, issued_v, AT_VSLOTS);
+      if (loads > 0) mbar_wait_drain(&hs_full[AT_KSLOTS + r], (uint32_t)(loads - 1) & 1u);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
+  if (warp == AT_S_WARP) tmem_dealloc(tmem, 512);
 }
 
 cudaError_t launch_tc_attention(const CUtensorMap& Q, const CUtensorMap& Ql, const CUtensorMap& K,

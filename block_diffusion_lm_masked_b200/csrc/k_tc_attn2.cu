@@ -61,28 +61,16 @@ __device__ __forceinline__ void a2_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// The half-slot plan both the load and the MMA warp follow: chunk j takes the next one
-// (cached keys) or two (own keys: hi, lo) half-slots for its K, then as many for its V^T.
-struct HalfSlotPlan {
-  int nxt = 0;
-  int uses[A2_HSLOTS] = {0, 0, 0};
-  int n;                    // parts per operand: 1, or 2 for a chunk of own keys
-  int ks[2], ku[2];         // K parts: half-slot, its use index
-  int vs[2], vu[2];         // V^T parts
-  __device__ void take(bool cur) {
-    n = cur ? 2 : 1;
-    for (int i = 0; i < n; ++i) {
-      ks[i] = nxt;
-      ku[i] = uses[nxt]++;
-      nxt = nxt + 1 == A2_HSLOTS ? 0 : nxt + 1;
-    }
-    for (int i = 0; i < n; ++i) {
-      vs[i] = nxt;
-      vu[i] = uses[nxt]++;
-      nxt = nxt + 1 == A2_HSLOTS ? 0 : nxt + 1;
-    }
-  }
-};
+// The half-slot ring the load thread and both MMA threads follow, as plain arithmetic (no
+// indexed arrays, so nothing spills to local memory): ring entries are taken in plan
+// order, chunk j's K parts (one, or two for own keys: hi, lo), then as many V^T parts;
+// entry e lives in half-slot e % A2_HSLOTS and is that half-slot's use e / A2_HSLOTS.
+__device__ __forceinline__ int a2_slot(int e) { return e % A2_HSLOTS; }
+__device__ __forceinline__ uint32_t a2_use_parity(int e) { return (uint32_t)(e / A2_HSLOTS) & 1u; }
+// loads issued into half-slot s when the first n_entries entries were issued
+__device__ __forceinline__ int a2_loads_into(int s, int n_entries) {
+  return n_entries > s ? (n_entries - 1 - s) / A2_HSLOTS + 1 : 0;
+}
 
 __global__ void __launch_bounds__(A2_THREADS, 1)
     tc_attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQl,
@@ -154,7 +142,7 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
 
   auto is_cur = [&](int j) { return p.has_lo && (c_begin + j) * A2_W >= p.base; };
   const uint32_t idesc = idesc_bf16_f32(A2_BQ, A2_W);  // S: 128 rows x 128 keys; PV: 128 rows x 128 d
-  int loaded[A2_HSLOTS] = {0, 0, 0};  // loads the load thread issued into each half-slot (for the wind-down)
+  int issued = 0;  // ring entries the load thread issued loads for (for the wind-down)
   bool q_issued = false;
 
   if (warp == A2_LOAD_WARP) {
@@ -177,18 +165,19 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         tma_load_3d(q + 3 * A2_BLK, &tmQl, 64, q_row0, h0 + hl, &q_bar);
       }
       q_issued = true;
-      HalfSlotPlan lp;
       bool ok = true;
-      // one half-slot: wait until its previous use was freed, then its two 16 KB blocks
-      auto load_half = [&](int s, int u, const CUtensorMap* map, bool is_v, int krow) {
-        if (u >= 1 && !mbar_wait(&hs_free[s], (uint32_t)(u - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
+      // ring entry e: wait until its half-slot's previous use was freed, then its two 16 KB blocks
+      auto load_half = [&](int e, const CUtensorMap* map, bool is_v, int krow) {
+        const int s = a2_slot(e);
+        if (e >= A2_HSLOTS &&
+            !mbar_wait(&hs_free[s], a2_use_parity(e - A2_HSLOTS), &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN))
           return false;
         if (!DG_GUARD(krow >= 0 && krow % A2_W == 0, p.err)) {
           abort_s = 1;
           return false;
         }
         uint8_t* dst = sHalf + s * A2_HSLOT;
-        loaded[s] += 1;
+        issued = e + 1;
         mbar_arrive_expect_tx(&hs_full[s], A2_HSLOT);
         if (is_v) {  // V^T [128 d][64 keys] blocks: keys krow .. +63, +64 .. +127
           tma_load_3d(dst, map, krow, 0, kvh, &hs_full[s]);
@@ -199,14 +188,15 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
         }
         return true;
       };
-      for (int j = 0; j < nck && ok; ++j) {
+      for (int j = 0, e = 0; j < nck && ok; ++j) {
         const int key0 = (c_begin + j) * A2_W;
-        lp.take(is_cur(j));
+        const int n = is_cur(j) ? 2 : 1;
         // part 0: the cache's bf16 keys; part 1: the low terms, rows counted from `base`
-        for (int i = 0; i < lp.n && ok; ++i)
-          ok = load_half(lp.ks[i], lp.ku[i], i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
-        for (int i = 0; i < lp.n && ok; ++i)
-          ok = load_half(lp.vs[i], lp.vu[i], i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
+        for (int i = 0; i < n && ok; ++i)
+          ok = load_half(e + i, i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
+        for (int i = 0; i < n && ok; ++i)
+          ok = load_half(e + n + i, i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
+        e += 2 * n;
       }
     }
     __syncwarp();
@@ -215,13 +205,13 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
     if (lane == 0 && hl < nh) {
       // ================= MMAs of head hl: one issuing thread per head, so that each
       // head's waits, MMAs and commits run beside the other head's
-      HalfSlotPlan mp;
-      auto half_addr = [&](int s) { return smem_u32(sHalf + s * A2_HSLOT); };
-      auto issue_s = [&]() {
+      auto half_addr = [&](int e) { return smem_u32(sHalf + a2_slot(e) * A2_HSLOT); };
+      // S(j): K parts at ring entries ek, ek + 1
+      auto issue_s = [&](int ek, int n) {
         const uint32_t d = tmem + a2_sp(hl);
         const uint32_t q = smem_u32(sQ + hl * A2_QHEAD), ql = q + 2 * A2_BLK;
-        const uint32_t k = half_addr(mp.ks[0]);
-        const uint32_t kl = mp.n == 2 ? half_addr(mp.ks[1]) : 0u;
+        const uint32_t k = half_addr(ek);
+        const uint32_t kl = n == 2 ? half_addr(ek + 1) : 0u;
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -230,45 +220,48 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
             const uint64_t kd = sw128_kmajor_desc(k + o);
             tc_mma(d, sw128_kmajor_desc(q + o), kd, idesc, (kb | kk) != 0 ? 1u : 0u);
             tc_mma(d, sw128_kmajor_desc(ql + o), kd, idesc, 1u);
-            if (mp.n == 2) tc_mma(d, sw128_kmajor_desc(q + o), sw128_kmajor_desc(kl + o), idesc, 1u);
+            if (n == 2) tc_mma(d, sw128_kmajor_desc(q + o), sw128_kmajor_desc(kl + o), idesc, 1u);
           }
         tc_commit(&s_full[hl]);
       };
-      auto issue_pv = [&](int j) {
+      // PV(j): V^T parts at ring entries ev, ev + 1
+      auto issue_pv = [&](int j, int ev, int n) {
         const uint32_t o = tmem + a2_o(hl), pp = tmem + a2_sp(hl);
-        const uint32_t v = half_addr(mp.vs[0]);
-        const uint32_t vl = mp.n == 2 ? half_addr(mp.vs[1]) : 0u;
+        const uint32_t v = half_addr(ev);
+        const uint32_t vl = n == 2 ? half_addr(ev + 1) : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 16 keys = 8 packed P columns per MMA
           const uint32_t vo = (kk >> 2) * A2_BLK + (kk & 3) * 32;
           const uint64_t vd = sw128_kmajor_desc(v + vo);
           a2_mma_ts(o, pp + kk * 8, vd, idesc, (j > 0 || kk != 0) ? 1u : 0u);
           a2_mma_ts(o, pp + 64 + kk * 8, vd, idesc, 1u);
-          if (mp.n == 2) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
+          if (n == 2) a2_mma_ts(o, pp + kk * 8, sw128_kmajor_desc(vl + vo), idesc, 1u);
         }
         tc_commit(&pv_done[hl]);
       };
 
       bool ok = mbar_wait(&q_bar, 0, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
-      for (int j = 0; j < nck && ok; ++j) {
-        mp.take(is_cur(j));
-        for (int i = 0; i < mp.n && ok; ++i)
-          ok = mbar_wait(&hs_full[mp.ks[i]], (uint32_t)mp.ku[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+      for (int j = 0, e = 0; j < nck && ok; ++j) {
+        const int n = is_cur(j) ? 2 : 1;
+        for (int i = 0; i < n && ok; ++i)
+          ok = mbar_wait(&hs_full[a2_slot(e + i)], a2_use_parity(e + i), &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         // the head's S/P region was last read by PV(j - 1)
         if (ok && j >= 1)
           ok = mbar_wait(&pv_done[hl], (uint32_t)(j - 1) & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (!ok) break;
         tc_fence_after();
-        issue_s();
+        issue_s(e, n);
         // a K half-slot is free once both heads' S MMAs have read it (count: one per head)
-        for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.ks[i]]);
-        for (int i = 0; i < mp.n && ok; ++i)
-          ok = mbar_wait(&hs_full[mp.vs[i]], (uint32_t)mp.vu[i] & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
+        for (int i = 0; i < n; ++i) tc_commit(&hs_free[a2_slot(e + i)]);
+        for (int i = 0; i < n && ok; ++i)
+          ok = mbar_wait(&hs_full[a2_slot(e + n + i)], a2_use_parity(e + n + i), &abort_s, p.err,
+                         DG_DEVERR_TIMEOUT_ATTN);
         if (ok) ok = mbar_wait(&p_ready[hl], (uint32_t)j & 1u, &abort_s, p.err, DG_DEVERR_TIMEOUT_ATTN);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(j);
-        for (int i = 0; i < mp.n; ++i) tc_commit(&hs_free[mp.vs[i]]);
+        issue_pv(j, e + n, n);
+        for (int i = 0; i < n; ++i) tc_commit(&hs_free[a2_slot(e + n + i)]);
+        e += 2 * n;
       }
     }
     __syncwarp();
@@ -437,8 +430,10 @@ __global__ void __launch_bounds__(A2_THREADS, 1)
   if (tid == A2_MMA_WARP * 32) mbar_wait_drain(&drain_bar, 0);
   if (abort_s && tid == A2_LOAD_WARP * 32) {
     if (q_issued) mbar_wait_drain(&q_bar, 0);
-    for (int s = 0; s < A2_HSLOTS; ++s)
-      if (loaded[s] > 0) mbar_wait_drain(&hs_full[s], (uint32_t)(loaded[s] - 1) & 1u);
+    for (int s = 0; s < A2_HSLOTS; ++s) {
+      const int loads = a2_loads_into(s, issued);
+      if (loads > 0) mbar_wait_drain(&hs_full[s], (uint32_t)(loads - 1) & 1u);
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -135,9 +135,9 @@ dg_status dg_debug_attention_bf16(const void* q, const void* k, const void* vt, 
 /* The same attention through the head-pair kernel: two query heads of one KV head per CTA
  * (one when nq / nkv is odd, or when single heads fill at least a quarter more SMs in the
  * one wave of CTAs), 128-key chunks, the same precision terms, outputs, workspace and
- * errors as dg_debug_attention_bf16.  The bf16 pass's attention runs this kernel; setting
- * DG_ATTN_SINGLE=1 in the environment (read once per process) routes it through the
- * single-head kernel of dg_debug_attention_bf16 instead. */
+ * errors as dg_debug_attention_bf16.  The bf16 pass's attention runs the single-head kernel
+ * of dg_debug_attention_bf16; setting DG_ATTN_PAIR=1 in the environment (read once per
+ * process) routes it through this kernel instead. */
 dg_status dg_debug_attention_pair_bf16(const void* q, const void* k, const void* vt, int32_t cap, int32_t n_q,
                                        int32_t pos0, int32_t n_keys, int32_t causal, int32_t nq, int32_t nkv,
                                        void* out, void* out_lo, void* d_ws, size_t ws_bytes, dg_stream stream);

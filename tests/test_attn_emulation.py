@@ -208,7 +208,7 @@ def run_pair(c, bug=None, force_pair=None):
                     q = sQ + hl * QHEAD
                     for off, mp, x in ((0, "Q", 0), (BLK, "Q", 64), (2 * BLK, "Ql", 0), (3 * BLK, "Ql", 64)):
                         sm.tma_load_3d(q + off, m[mp], x, q_row0, h0 + hl, 64, 128)
-                # the half-slot plan (HalfSlotPlan::take): per chunk its K parts, then its V parts
+                # the half-slot ring (entry e in half-slot e % 3): per chunk its K parts, then its V parts
                 plan, items, nxt = [], [], 0
                 for j in range(nck):
                     n = 2 if is_cur(j) else 1
@@ -326,11 +326,12 @@ def run_pair(c, bug=None, force_pair=None):
 # ---------------------------------------------------------------- tc_attn_kernel
 def run_single(c, bug=None):
     """tc_attn_kernel: one head x 128 rows x 128-key chunks; the query tile (hi + lo) in
-    shared memory by TMA, then a ring of five 32 KB half-slots (a chunk's K, then its V^T,
-    each with its low term for own keys); TMEM: S buffers at columns 0 and 128, O at 256,
-    P hi at 384 and lo at 448.  Per chunk j the replay computes S(j) before the softmax of
-    chunk j - 1 reads S(j - 1), then PV(j - 1), as the kernel's issue order lets the tensor
-    cores run; the load warp fills half-slots as soon as they are freed.
+    shared memory by TMA, then a ring of two 32 KB half-slots for K and one of three for V^T
+    (with their low terms for own keys); TMEM: S buffers at columns 0 and 128, O at 256,
+    P hi at 384 and lo at 448.  The replay runs S as far ahead as the barriers let it: S(j + 2)
+    lands in S buffer j & 1 as soon as the softmax has read S(j) -- before it writes P(j)
+    where chunk j + 2's K could be loaded by then, else after PV(j) frees half-slots; the
+    load warp fills half-slots as soon as they are freed.
 
     bug: "one_s_buffer" -- both S buffers at column 0; "p_lo_offset" -- P lo at 416, half
     over P hi; "q_lo_block" -- the query's lo MMAs read its hi blocks; "v_free_early" -- a
@@ -340,7 +341,8 @@ def run_single(c, bug=None):
     group = nq // nkv
     n_splits, cps = splits_single(n_q, nq, n_keys)
     W, BLK = 128, 128 * 128
-    QTILE, HSLOT, HSLOTS = 4 * BLK, 2 * BLK, 5
+    QTILE, HSLOT, KSLOTS, VSLOTS = 4 * BLK, 2 * BLK, 2, 3
+    HSLOTS = KSLOTS + VSLOTS
     sQ, sHalf = 0, QTILE
     at_s = (lambda b: 0) if bug == "one_s_buffer" else (lambda b: b * 128)
     AT_O, AT_PHI = 256, 384
@@ -368,17 +370,17 @@ def run_single(c, bug=None):
                 is_cur = lambda j: (c_begin + j) * W >= c["base"]
                 for off, mp, x in ((0, "Q", 0), (BLK, "Q", 64), (2 * BLK, "Ql", 0), (3 * BLK, "Ql", 64)):
                     sm.tma_load_3d(sQ + off, m[mp], x, q_row0, h, 64, 128)
-                # the half-slot plan (AtPlan::take): per chunk its K parts, then its V parts
-                plan, items, nxt = [], [], 0
+                # the rings (K entry e in half-slot e % 2, V^T entry e in 2 + e % 3): per chunk
+                # its K parts, then its V^T parts, in the load warp's order
+                plan, items, ek, ev = [], [], 0, 0
                 for j in range(nck):
                     n = 2 if is_cur(j) else 1
-                    ks, vs = [], []
-                    for lst in (ks, vs):
-                        for i in range(n):
-                            lst.append(nxt)
-                            items.append((j, "K" if lst is ks else "V", i, nxt))
-                            nxt = (nxt + 1) % HSLOTS
+                    ks = [(ek + i) % KSLOTS for i in range(n)]
+                    vs = [KSLOTS + (ev + i) % VSLOTS for i in range(n)]
+                    items += [(j, "K", i, ks[i]) for i in range(n)] + [(j, "V", i, vs[i]) for i in range(n)]
                     plan.append((ks, vs))
+                    ek += n
+                    ev += n
                 holder = {}                                   # half-slot -> (chunk, operand) held until freed
                 loaded = [0]
 
@@ -442,10 +444,12 @@ def run_single(c, bug=None):
                 lpair = (np.zeros(128, np.float32), np.zeros(128, np.float32))
                 key_lim = np.array([c["key_lim"][r] if r < n_q else n_keys for r in rows])
 
-                def softmax(j):
-                    nonlocal m_used, lpair
+                def read_s(j):
                     sb = at_s(j & 1)
-                    raw = np.concatenate([tm.t[:, sb + cc * 16:sb + cc * 16 + 16] for cc in range(8)], axis=1)
+                    return np.concatenate([tm.t[:, sb + cc * 16:sb + cc * 16 + 16] for cc in range(8)], axis=1)
+
+                def softmax(j, raw):
+                    nonlocal m_used, lpair
                     s = softmax_chunk_raw(raw, (c_begin + j) * W, key_lim)
 
                     def rescale(any_w, alpha):
@@ -468,16 +472,27 @@ def run_single(c, bug=None):
                     issue_pv(j)
                     free(j, "V")
 
-                pump()
-                for j in range(nck):
+                def s_mmas(j):
                     ready(j, "K")
                     issue_s(j)
                     free(j, "K")
-                    if j >= 1:
-                        softmax(j - 1)
-                        pv(j - 1)
-                softmax(nck - 1)
-                pv(nck - 1)
+
+                def k_loaded(j):
+                    pump()
+                    return all(items.index(it) < loaded[0] for it in items if it[0] == j and it[1] == "K")
+
+                pump()
+                for j in range(min(nck, 2)):
+                    s_mmas(j)
+                for j in range(nck):
+                    raw = read_s(j)                           # S buffer j & 1 is free again
+                    early = j + 2 < nck and k_loaded(j + 2)
+                    if early:
+                        s_mmas(j + 2)
+                    softmax(j, raw)                           # after PV(j - 1): rescale O, write P(j)
+                    pv(j)
+                    if j + 2 < nck and not early:
+                        s_mmas(j + 2)
                 lsum = (lpair[0] + lpair[1]).astype(np.float32)
                 epilogue(tm, AT_O, lsum, m_used, rows, out, out_lo, part_o, part_lse, sp, h, n_splits, nq, n_q)
     return (out + out_lo) if n_splits == 1 else merge2(part_o, part_lse, n_splits)

@@ -72,9 +72,9 @@ def debug_entry_accepts(n_q, pos0, n_keys, causal, cap, nq, nkv):
 
 
 class HalfSlotPlan:
-    """The half-slot plan of both kernels (HalfSlotPlan::take in the head-pair kernel,
-    three half-slots; AtPlan::take in the single-head kernel, five): a chunk's K parts,
-    then its V^T parts, each the next half-slot of the ring."""
+    """The head-pair kernel's half-slot ring: ring entries taken in plan order (a chunk's K
+    parts, then its V^T parts, two each for own keys), entry e in half-slot e % slots as
+    that half-slot's use e // slots (a2_slot and the use parity in the kernel)."""
 
     def __init__(self, slots=3):
         self.nxt, self.uses, self.slots = 0, [0] * slots, slots
@@ -86,6 +86,24 @@ class HalfSlotPlan:
                 lst.append((self.nxt, self.uses[self.nxt]))
                 self.uses[self.nxt] += 1
                 self.nxt = (self.nxt + 1) % self.slots
+        return k, v
+
+
+class TwoRingPlan:
+    """The single-head kernel's rings: a chunk's K parts take the next entries of a ring of
+    kslots half-slots, its V^T parts those of a ring of vslots half-slots numbered after
+    the K ring's (at_kslot / at_vslot and the use parities in the kernel)."""
+
+    def __init__(self, kslots=2, vslots=3):
+        self.ek = self.ev = 0
+        self.kslots, self.vslots = kslots, vslots
+
+    def take(self, cur):
+        n = 2 if cur else 1
+        k = [((self.ek + i) % self.kslots, (self.ek + i) // self.kslots) for i in range(n)]
+        v = [(self.kslots + (self.ev + i) % self.vslots, (self.ev + i) // self.vslots) for i in range(n)]
+        self.ek += n
+        self.ev += n
         return k, v
 
 
@@ -112,7 +130,7 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
     else:
         n_splits, cps = splits_single(n_q, nq, n_keys)
         nh, ys = 1, nq
-        smem_q, slot_bytes, slots = 4 * 16384, 32768, 5         # the query tile, five half-slots
+        smem_q, slot_bytes, slots = 4 * 16384, 32768, 5         # the query tile, 2 + 3 half-slots
         smem_total = 1024 + smem_q + slots * slot_bytes
         assert smem_total <= 227 * 1024 - 512
         # TMEM columns: S buffers 0..127 and 128..255, O 256..383, P buffers 384..447 and 448..511
@@ -146,7 +164,7 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
                         for r in rows:
                             assert ((sp * nq + h) * n_q + r + 1) * D <= part_o_len
                     continue
-                plan = HalfSlotPlan(slots)
+                plan = HalfSlotPlan(slots) if kernel == "pair" else TwoRingPlan()
                 for j in range(nck):
                     key0 = (c_begin + j) * W
                     assert key0 < kv_end
@@ -266,13 +284,31 @@ def test_debug_entries_refuse_a_low_term_window_past_the_workspace():
         assert f(P, P, P, 4096, 64, 4097, 4096, 0, 2, 1, P, None, P, 1 << 30, None) == dg.DG_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("slots", [3, 5])
+@pytest.mark.parametrize("slots", [2, 3])
+def test_ring_arithmetic_counts_the_loads_of_each_half_slot(slots):
+    """The wind-down's count of loads issued into each half-slot (a2_loads_into /
+    at_loads_into) is the number of ring entries below the issued count in that half-slot,
+    and the last one's use parity is what the drain waits for (rings of 3 in the head-pair
+    kernel, of 2 and 3 in the single-head kernel)."""
+    def loads_into(s, n):
+        return (n - 1 - s) // slots + 1 if n > s else 0
+    for n in range(0, 40):
+        for s in range(slots):
+            mine = [e for e in range(n) if e % slots == s]
+            assert loads_into(s, n) == len(mine)
+            if mine:
+                assert (loads_into(s, n) - 1) & 1 == (mine[-1] // slots) & 1
+
+
 @pytest.mark.parametrize("nck,cur_from", [(5, 2), (9, 0), (12, 8), (3, 3)])
-def test_kernel_slot_plan_is_the_simulated_one(nck, cur_from, slots):
+def test_kernel_slot_plans_are_the_simulated_ones(nck, cur_from):
     import test_pipeline_protocol as TP
-    plan = HalfSlotPlan(slots)
+    plan = HalfSlotPlan(3)
     got = [plan.take(j >= cur_from) for j in range(nck)]
-    assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, slots)]
+    assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, 3)]
+    plan2 = TwoRingPlan(2, 3)
+    got2 = [plan2.take(j >= cur_from) for j in range(nck)]
+    assert got2 == [(list(k), list(v)) for k, v in TP.two_ring_plan(nck, cur_from, 2, 3)]
 
 
 def test_splits_fill_about_one_wave():

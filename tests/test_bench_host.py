@@ -105,9 +105,9 @@ def test_job_value_counts_every_rank_over_the_slowest():
 
 
 def test_attention_kind_follows_the_switch(monkeypatch):
-    monkeypatch.delenv("DG_ATTN_SINGLE", raising=False)
-    assert bench._attention_kind().startswith("head pairs")
-    monkeypatch.setenv("DG_ATTN_SINGLE", "1")
+    monkeypatch.delenv("DG_ATTN_PAIR", raising=False)
     assert bench._attention_kind().startswith("one head")
-    monkeypatch.setenv("DG_ATTN_SINGLE", "0")
+    monkeypatch.setenv("DG_ATTN_PAIR", "1")
     assert bench._attention_kind().startswith("head pairs")
+    monkeypatch.setenv("DG_ATTN_PAIR", "0")
+    assert bench._attention_kind().startswith("one head")

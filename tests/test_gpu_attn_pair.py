@@ -1,8 +1,8 @@
-"""Both attention kernels -- the head-pair kernel (dg_debug_attention_pair_bf16, the
-pass's default) and the single-head kernel (dg_debug_attention_bf16) -- against a plain
-fp64 reference of the same attention, then whole passes with the single-head kernel
-(DG_ATTN_SINGLE=1) against the oracle, in a child process since the switch is read once
-per process."""
+"""Both attention kernels -- the single-head kernel (dg_debug_attention_bf16, the pass's
+default) and the head-pair kernel (dg_debug_attention_pair_bf16) -- against a plain fp64
+reference of the same attention, then whole passes with the head-pair kernel
+(DG_ATTN_PAIR=1) against the oracle, in a child process since the switch is read once per
+process."""
 import os
 import subprocess
 import sys
@@ -85,14 +85,14 @@ def test_kernel_matches_reference(dg, kernel, nq, nkv, n_q, pos0, n_keys, causal
     assert (err <= 1e-4 * ref.abs() + 1e-4 * rms).all(), err.max().item()
 
 
-def test_passes_with_the_single_head_kernel_match_the_oracle():
+def test_passes_with_the_head_pair_kernel_match_the_oracle():
     """The pass parity tests (own-key low terms, causal prefill, chained canvases) with the
-    pass's attention routed through the single-head kernel; the child must have run them
+    pass's attention routed through the head-pair kernel; the child must have run them
     (a child whose tests all skipped proves nothing)."""
     import re
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
-    env = dict(os.environ, DG_ATTN_SINGLE="1")
+    env = dict(os.environ, DG_ATTN_PAIR="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "tests/test_gpu_parity.py",
                         "-k", "small_bf16 or layer1_bf16 or prefill_append or chained"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)

@@ -371,34 +371,60 @@ def test_the_checker_catches_a_wrong_count():
 
 # ---------------------------------------------------------------- the single-head attention kernel (k_tc_attn.cu)
 
-def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_at=None, drain=True,
-              load_drain=True, bug=None):
-    """tc_attn_kernel's hand-offs (128-key chunks, two S buffers, one P buffer): a load warp
-    fills the query tile, then a ring of `slots` half-slots with each chunk's K then its V^T;
-    the MMA thread issues S(j) into S buffer j & 1 (no wait of its own: PV(j - 2), issued
-    before it, waited for P(j - 2), which the softmax writes after reading S(j - 2)), a
-    commit freeing the K half-slots, then PV(j - 1) once P(j - 1) is written, and a commit
-    freeing its V half-slots; each softmax warp reads S(j), then -- once PV(j - 1) is
-    complete (O stable, P read) -- maybe rescales O, writes P(j) and signals.  Chunks [cur_from, nck) are the call's own (two half-slots per operand).
-    Every role reaches the exit barrier; the MMA thread drains its commits (`drain`), and
-    after an abort the load warp waits for the loads it issued (`load_drain`).
+def two_ring_plan(nck, cur_from, kslots, vslots):
+    """The single-head kernel's rings: chunk j's K parts (two for own keys) take the next
+    entries of a ring of `kslots` half-slots, its V^T parts those of a ring of `vslots`
+    half-slots numbered after the K ring's; returns [(K parts, V parts)], each part
+    (half-slot, its use index)."""
+    ek = ev = 0
+    plan = []
+    for j in range(nck):
+        n = 2 if j >= cur_from else 1
+        kp = [((ek + i) % kslots, (ek + i) // kslots) for i in range(n)]
+        vp = [(kslots + (ev + i) % vslots, (ev + i) // vslots) for i in range(n)]
+        plan.append((kp, vp))
+        ek += n
+        ev += n
+    return plan
 
-    bug: "lag2" -- PV lags two chunks behind S (S(j), then PV(j - 2)), so S(j) no longer
-    follows P(j - 2); "no_pv_wait" -- P(j) written without waiting for PV(j - 1).
+
+def attention(nck, seed, cur_from=None, kslots=2, vslots=3, n_warps=4, flags=None, give_up_at=None, drain=True,
+              load_drain=True, bug=None, shared_ring=False):
+    """tc_attn_kernel's hand-offs (128-key chunks, two S buffers, one P buffer): a load warp
+    fills the query tile, then each chunk's K into a ring of `kslots` half-slots and its V^T
+    into a ring of `vslots` (shared_ring: one ring of kslots + vslots half-slots for both,
+    K then V^T per chunk -- which the two issuing threads cannot share, see below).
+    Two issuing threads: the S thread issues S(j) into S buffer j & 1 once chunk j's K has
+    landed and the softmax warps have read S(j - 2) (s_free), then a commit freeing the K
+    half-slots; the PV thread issues PV(j) once chunk j's V^T has landed and P(j) is
+    written, then a commit freeing the V^T half-slots; their completions interleave in any
+    order, each thread's in its own issue order.  Each softmax warp reads S(j) and signals
+    s_free, then -- once PV(j - 1) is complete (O stable, P read) -- maybe rescales O,
+    writes P(j) and signals.  Chunks [cur_from, nck) are the call's own (two half-slots per
+    operand).  Every role reaches the exit barrier; both issuing threads drain their
+    commits (`drain`), and after an abort the load warp waits for the loads it issued
+    (`load_drain`).
+
+    bug: "no_s_free_wait" -- S(j) issued without waiting for the softmax's read of S(j - 2);
+    "no_pv_wait" -- P(j) written without waiting for PV(j - 1).
     flags / give_up_at: abort mode as in attention_two_heads below."""
     rng = random.Random(seed * 7919 + nck)
-    plan = half_slot_plan(nck, nck if cur_from is None else cur_from, slots)
+    cf = nck if cur_from is None else cur_from
+    slots = kslots + vslots
+    plan = half_slot_plan(nck, cf, slots) if shared_ring else two_ring_plan(nck, cf, kslots, vslots)
     q_bar = Barrier("q", 1)
     hs_full = [Barrier(f"hs_full{s}", 1) for s in range(slots)]
     hs_free = [Barrier(f"hs_free{s}", 1) for s in range(slots)]
     s_full = [Barrier(f"s_full{b}", 1) for b in range(2)]
+    s_free = [Barrier(f"s_free{b}", n_warps) for b in range(2)]
     p_ready, pv_done = Barrier("p_ready", n_warps), Barrier("pv_done", 1)
-    drain_bar = Barrier("drain", 1)
-    exit_bar = Barrier("exit", n_warps + 2)            # the __syncthreads every role reaches at the end
-    bufs, q = Buffers(), Async()
+    drain_bar = Barrier("drain", 2)
+    exit_bar = Barrier("exit", n_warps + 3)            # the __syncthreads every role reaches at the end
+    bufs, q = Buffers(), AsyncPerThread(2)
     st = dict(pv_issued=0, pv_done=0)
     p_writes = {}
     steps = [0]
+    uses = {}                                          # half-slot -> use index last loaded into it
 
     def bw(bar, parity, phase):
         if flags is None:
@@ -425,6 +451,7 @@ def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_
                             ok = False
                             break
                     bufs.fill(("hs", x), 1)             # K: read by S(j); V^T: by PV(j)
+                    uses[x] = u
                     hs_full[x].arrive_expect_tx(32)
                     q.loads.append(lambda x=x: hs_full[x].complete_tx(32))
                     loaded[x] += 1
@@ -448,15 +475,52 @@ def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_
         finally:
             exit_bar.arrive()
 
-    def mma():
-        def do_pv(i):
+    def s_thread():
+        mq = q.by[0]
+        yield bw(q_bar, 0, 0)
+        ok = passed(q_bar, 0)
+        for j in range(nck if ok else 0):
+            b = j & 1
+            for x, u in plan[j][0]:
+                yield bw(hs_full[x], u & 1, u)
+                if not passed(hs_full[x], u & 1):
+                    ok = False
+                    break
+                assert uses.get(x) == u and hs_full[x].completed == u + 1, f"S({j}) read half-slot {x} before use {u} landed"
+            if ok and j >= 2 and bug != "no_s_free_wait":
+                yield bw(s_free[b], ((j - 2) >> 1) & 1, (j - 2) >> 1)
+                ok = passed(s_free[b], ((j - 2) >> 1) & 1)
+            if not ok:
+                break
+            for w in range(n_warps):                   # S(j): each softmax warp reads its 32 lanes
+                bufs.fill(("S", b, w), 1)
+
+            def s_done(j=j, b=b):
+                for x, _ in plan[j][0]:
+                    bufs.release(("hs", x))
+                s_full[b].arrive()
+            mq.append(s_done)
+            for x, _ in plan[j][0]:
+                mq.append(lambda x=x: hs_free[x].arrive())
+        if drain:
+            mq.append(lambda: drain_bar.arrive())
+            yield wait(drain_bar, 0, 0)
+
+    def pv_thread():
+        mq = q.by[1]
+        for i in range(nck):
+            ok = True
             for x, u in plan[i][1]:
                 yield bw(hs_full[x], u & 1, u)
                 if not passed(hs_full[x], u & 1):
-                    return False
+                    ok = False
+                    break
+                assert uses.get(x) == u and hs_full[x].completed == u + 1, f"PV({i}) read half-slot {x} before use {u} landed"
+            if not ok:
+                break
             yield bw(p_ready, i & 1, i)
             if not passed(p_ready, i & 1):
-                return False
+                break
             assert p_writes.get("p") == (i, n_warps), "PV read a P not fully written"
             st["pv_issued"] += 1
 
@@ -467,44 +531,11 @@ def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_
                 for x, _ in plan[i][1]:
                     bufs.release(("hs", x))
                 pv_done.arrive()
-            q.mma.append(fin)
+            mq.append(fin)
             for x, _ in plan[i][1]:
-                q.mma.append(lambda x=x: hs_free[x].arrive())
-            return True
-
-        yield bw(q_bar, 0, 0)
-        ok = passed(q_bar, 0)
-        for j in range(nck if ok else 0):
-            b = j & 1
-            for x, u in plan[j][0]:
-                yield bw(hs_full[x], u & 1, u)
-                if not passed(hs_full[x], u & 1):
-                    ok = False
-                    break
-            if not ok:
-                break
-            for w in range(n_warps):                   # S(j): each softmax warp reads its 32 lanes
-                bufs.fill(("S", b, w), 1)
-
-            def s_done(j=j, b=b):
-                for x, _ in plan[j][0]:
-                    bufs.release(("hs", x))
-                s_full[b].arrive()
-            q.mma.append(s_done)
-            for x, _ in plan[j][0]:
-                q.mma.append(lambda x=x: hs_free[x].arrive())
-            lag = 2 if bug == "lag2" else 1
-            if j >= lag:
-                ok = yield from do_pv(j - lag)
-                if not ok:
-                    break
-        for i in range(max(nck - (2 if bug == "lag2" else 1), 0), nck):
-            if not ok:
-                break
-            ok = yield from do_pv(i)
+                mq.append(lambda x=x: hs_free[x].arrive())
         if drain:
-            q.mma.append(lambda: drain_bar.arrive())
-            yield wait(drain_bar, 0, 0)
+            mq.append(lambda: drain_bar.arrive())
 
     def softmax(w):
         for j in range(nck):
@@ -513,6 +544,7 @@ def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_
             if not passed(s_full[b], (j >> 1) & 1):
                 return
             bufs.release(("S", b, w))                  # this warp's lanes of S(j) read into registers
+            s_free[b].arrive()
             if j > 0 and bug != "no_pv_wait":
                 yield bw(pv_done, (j - 1) & 1, j - 1)
                 if not passed(pv_done, (j - 1) & 1):
@@ -527,7 +559,7 @@ def attention(nck, seed, cur_from=None, slots=5, n_warps=4, flags=None, give_up_
         if passed(pv_done, (nck - 1) & 1):
             assert st["pv_done"] == nck
 
-    roles = {"load": load(), "mma": leaving(mma())}
+    roles = {"load": load(), "mma_s": leaving(s_thread()), "mma_pv": leaving(pv_thread())}
     roles.update({f"sm{w}": leaving(softmax(w)) for w in range(n_warps)})
     return roles, q
 
@@ -542,11 +574,11 @@ def test_attention_protocol(nck, cur_from):
         run(roles, q, seed, end_check=True)
 
 
-@pytest.mark.parametrize("bug", ["lag2", "no_pv_wait"])
+@pytest.mark.parametrize("bug", ["no_s_free_wait", "no_pv_wait"])
 def test_attention_protocol_catches_its_planted_mistakes(bug):
-    """S(j) issued before the softmax has read S(j - 2) from the same buffer (PV lagging two
-    chunks), or P(j) written before PV(j - 1) has read P(j - 1): some interleaving
-    overwrites a buffer still read, or deadlocks."""
+    """S(j) issued before the softmax has read S(j - 2) from the same buffer, or P(j)
+    written before PV(j - 1) has read P(j - 1): some interleaving overwrites a buffer
+    still read."""
     caught = 0
     for seed in range(60):
         roles, q = attention(6, seed, cur_from=4, bug=bug)
@@ -557,20 +589,34 @@ def test_attention_protocol_catches_its_planted_mistakes(bug):
     assert caught > 0
 
 
-def test_attention_with_a_smaller_ring_deadlocks():
-    """The ring must hold chunk j's K beside chunk j - 1's unread V^T: two chunks of own keys
-    need four half-slots, and a ring of three deadlocks on them."""
+def test_attention_with_one_shared_ring_reads_a_half_slot_too_early():
+    """One ring for K and V^T with two issuing threads: the S thread can reach a K entry whose
+    half-slot still waits for an earlier V^T use to land, and its parity wait passes at once
+    (a phase behind looks like a completed one).  The separate rings exist for this."""
+    caught = 0
+    for seed in range(60):
+        roles, q = attention(7, seed, cur_from=5, shared_ring=True)
+        try:
+            run(roles, q, seed, end_check=True)
+        except AssertionError as e:
+            caught += "before use" in str(e) or "released twice" in str(e) or "overwritten" in str(e)
+    assert caught > 0
+
+
+def test_attention_with_the_smallest_rings():
+    """One half-slot per ring deadlocks on a chunk of own keys (two parts); two per ring do
+    not."""
     with pytest.raises(AssertionError, match="deadlock"):
-        roles, q = attention(4, 0, cur_from=2, slots=3)
+        roles, q = attention(4, 0, cur_from=2, kslots=1, vslots=1)
         run(roles, q, 0)
     for seed in range(20):
-        roles, q = attention(6, seed, cur_from=2, slots=4)
+        roles, q = attention(6, seed, cur_from=2, kslots=2, vslots=2)
         run(roles, q, seed, end_check=True)
 
 
 def test_attention_leaves_nothing_in_flight():
-    """Without the MMA thread's drain some interleaving leaves a commit landing after the
-    CTA is gone."""
+    """Without the issuing threads' drain some interleaving leaves a commit landing after
+    the CTA is gone."""
     left = 0
     for seed in range(60):
         roles, q = attention(6, seed, cur_from=4, drain=False)
@@ -895,6 +941,7 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
     st = {"pv_done": [0, 0], "pv_issued": [0, 0]}
     p_writes = {}
     steps = [0]
+    uses = {}                                         # half-slot -> use index last loaded into it
 
     def bw(bar, parity, phase):
         """A bounded wait (abort-aware in abort mode)."""
@@ -920,6 +967,7 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                             ok = False
                             break
                     bufs.fill(("hs", s), H)           # K: both heads' S read it; V^T: both PVs
+                    uses[s] = u
                     hs_full[s].arrive_expect_tx(32)
                     q.loads.append(lambda s=s: hs_full[s].complete_tx(32))
                     loaded[s] += 1
@@ -942,6 +990,7 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                 if not passed(hs_full[x], u & 1):
                     ok = False
                     break
+                assert uses.get(x) == u and hs_full[x].completed == u + 1, f"S read half-slot {x} before use {u} landed"
             if ok and j >= 1 and bug != "no_pv_wait":
                 yield bw(pv_done[h], (j - 1) & 1, j - 1)
                 ok = passed(pv_done[h], (j - 1) & 1)
@@ -962,6 +1011,7 @@ def attention_two_heads(nck, seed, slots=3, warps_per_head=4, cur_from=None, fla
                 if not passed(hs_full[x], u & 1):
                     ok = False
                     break
+                assert uses.get(x) == u and hs_full[x].completed == u + 1, f"PV read half-slot {x} before use {u} landed"
             if not ok:
                 break
             yield bw(p_ready[h], j & 1, j)
