@@ -16,8 +16,8 @@
 // start `base` at or below the first current position; rows before the first current
 // position are zero there.
 //
-// Layout.  Shared memory: the query tile (hi + lo, 64 KB, TMA), a ring of two 32 KB
-// half-slots for K [128 keys][128 d] and one of three for V^T [128 d][128 keys] (two 16 KB
+// Layout.  Shared memory: the query tile (hi + lo, 64 KB, TMA), a ring of three 32 KB
+// half-slots for K [128 keys][128 d] and one of two for V^T [128 d][128 keys] (two 16 KB
 // blocks each, 128-byte swizzled); a chunk of the call's own keys takes two entries of
 // each ring (hi, then lo).
 // TMEM (512 columns): two S buffers (fp32, 128 keys) at 0 and 128, O at 256, and P at 384
@@ -25,8 +25,10 @@
 // buffer j & 1.
 //
 // Roles.  Warps 0-3 run the softmax, one query row per thread (its TMEM lane) over the
-// whole 128-key chunk, so no row statistics are exchanged between warps; warp 4 issues the
-// TMA loads; warps 5 and 6 issue the MMAs, one thread each: warp 5 the S MMAs, S(j) once
+// whole 128-key chunk, so no row statistics are exchanged between warps; warps 4 and 7
+// issue the TMA loads of the K ring (and the query tile) and of the V^T ring, each ring in
+// its own order, so that a K load never waits behind a V^T half-slot still being read;
+// warps 5 and 6 issue the MMAs, one thread each: warp 5 the S MMAs, S(j) once
 // chunk j's K has landed and the softmax has read S(j - 2) out of the same buffer, then a
 // commit freeing the K half-slots; warp 6 the PV MMAs, PV(j) once chunk j's V^T has landed
 // and the softmax has written P(j), then a commit freeing the V^T half-slots.  Each issuing
@@ -47,18 +49,19 @@ namespace dg {
 constexpr int AT_BQ = 128;
 constexpr int AT_W = 128;                       // keys per chunk
 constexpr int AT_D = 128;
-constexpr int AT_KSLOTS = 2;                    // half-slots of the K ring
-constexpr int AT_VSLOTS = 3;                    // half-slots of the V^T ring (after the K ring's)
+constexpr int AT_KSLOTS = 3;                    // half-slots of the K ring
+constexpr int AT_VSLOTS = 2;                    // half-slots of the V^T ring (after the K ring's)
 constexpr int AT_HSLOTS = AT_KSLOTS + AT_VSLOTS;
 constexpr uint32_t AT_BLK = 128 * 128;          // [128 rows][64 bf16] swizzled block: 16 KB
 constexpr uint32_t AT_QTILE = 4 * AT_BLK;       // Q hi (two d blocks) + Q lo (two d blocks): 64 KB
 constexpr uint32_t AT_HSLOT = 2 * AT_BLK;       // K (two d blocks) or V^T (two key blocks): 32 KB
 constexpr int AT_SMEM = 1024 + AT_QTILE + AT_HSLOTS * AT_HSLOT;
 constexpr int AT_SM_WARPS = 4;
-constexpr int AT_LOAD_WARP = 4;
+constexpr int AT_LOAD_WARP = 4;   // the query tile and the K ring
+constexpr int AT_VLOAD_WARP = 7;  // the V^T ring
 constexpr int AT_S_WARP = 5;    // issues the S MMAs (and holds the TMEM allocation)
 constexpr int AT_PV_WARP = 6;   // issues the PV MMAs
-constexpr int AT_THREADS = 32 * 7;
+constexpr int AT_THREADS = 32 * 8;
 static_assert(AT_SMEM <= 227 * 1024 - 512, "shared memory budget");
 
 // TMEM column offsets
@@ -165,57 +168,60 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   int issued_k = 0, issued_v = 0;  // ring entries the load thread issued loads for (for the wind-down)
   bool q_issued = false;
 
-  if (warp == AT_LOAD_WARP) {
+  if (warp == AT_LOAD_WARP || warp == AT_VLOAD_WARP) {
     if (lane == 0) {
-      // ================= loads: the query tile, then each chunk's K and V^T in plan order
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmQl);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmVt);
-      if (p.has_lo) {
-        prefetch_tmap(&tmKl);
-        prefetch_tmap(&tmVtl);
+      // ================= loads: warp 4 the query tile, then each chunk's K in plan order;
+      // warp 7 each chunk's V^T
+      const bool is_v = warp == AT_VLOAD_WARP;
+      if (!is_v) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmQl);
+        prefetch_tmap(&tmK);
+        if (p.has_lo) prefetch_tmap(&tmKl);
+        mbar_arrive_expect_tx(&q_bar, AT_QTILE);
+        tma_load_3d(sQ, &tmQ, 0, q_row0, h, &q_bar);
+        tma_load_3d(sQ + AT_BLK, &tmQ, 64, q_row0, h, &q_bar);
+        tma_load_3d(sQ + 2 * AT_BLK, &tmQl, 0, q_row0, h, &q_bar);
+        tma_load_3d(sQ + 3 * AT_BLK, &tmQl, 64, q_row0, h, &q_bar);
+        q_issued = true;
+      } else {
+        prefetch_tmap(&tmVt);
+        if (p.has_lo) prefetch_tmap(&tmVtl);
       }
-      mbar_arrive_expect_tx(&q_bar, AT_QTILE);
-      tma_load_3d(sQ, &tmQ, 0, q_row0, h, &q_bar);
-      tma_load_3d(sQ + AT_BLK, &tmQ, 64, q_row0, h, &q_bar);
-      tma_load_3d(sQ + 2 * AT_BLK, &tmQl, 0, q_row0, h, &q_bar);
-      tma_load_3d(sQ + 3 * AT_BLK, &tmQl, 64, q_row0, h, &q_bar);
-      q_issued = true;
+      const int ring = is_v ? AT_VSLOTS : AT_KSLOTS;
+      const CUtensorMap* map_hi = is_v ? &tmVt : &tmK;
+      const CUtensorMap* map_lo = is_v ? &tmVtl : &tmKl;
       bool ok = true;
-      // entry e of the K (or V^T) ring: wait until its half-slot's previous use was freed,
-      // then its two 16 KB blocks
-      auto load_half = [&](int e, const CUtensorMap* map, bool is_v, int krow) {
-        const int ring = is_v ? AT_VSLOTS : AT_KSLOTS;
-        const int s = is_v ? at_vslot(e) : at_kslot(e);
-        if (e >= ring && !mbar_wait(&hs_free[s], is_v ? at_vparity(e - ring) : at_kparity(e - ring), &abort_s,
-                                    p.err, DG_DEVERR_TIMEOUT_ATTN))
-          return false;
-        if (!DG_GUARD(krow >= 0 && krow % AT_W == 0, p.err)) {
-          abort_s = 1;
-          return false;
-        }
-        uint8_t* dst = sHalf + s * AT_HSLOT;
-        (is_v ? issued_v : issued_k) = e + 1;
-        mbar_arrive_expect_tx(&hs_full[s], AT_HSLOT);
-        if (is_v) {  // V^T [128 d][64 keys] blocks: keys krow .. +63, +64 .. +127
-          tma_load_3d(dst, map, krow, 0, kvh, &hs_full[s]);
-          tma_load_3d(dst + AT_BLK, map, krow + 64, 0, kvh, &hs_full[s]);
-        } else {     // K [128 keys][64 d] blocks: d 0 .. 63, 64 .. 127
-          tma_load_3d(dst, map, 0, krow, kvh, &hs_full[s]);
-          tma_load_3d(dst + AT_BLK, map, 64, krow, kvh, &hs_full[s]);
-        }
-        return true;
-      };
-      for (int j = 0, e = 0; j < nck && ok; ++j) {  // e: chunk j's first entry in either ring
+      for (int j = 0, e = 0; j < nck && ok; ++j) {  // e: chunk j's first entry in this ring
         const int key0 = (c_begin + j) * AT_W;
         const int n = is_cur(j) ? 2 : 1;
         // part 0: the cache's bf16 keys; part 1: the low terms, rows counted from `base`
-        for (int i = 0; i < n && ok; ++i)
-          ok = load_half(e + i, i == 0 ? &tmK : &tmKl, false, i == 0 ? key0 : key0 - p.base);
-        for (int i = 0; i < n && ok; ++i)
-          ok = load_half(e + i, i == 0 ? &tmVt : &tmVtl, true, i == 0 ? key0 : key0 - p.base);
-        e += n;
+        for (int i = 0; i < n && ok; ++i, ++e) {
+          // wait until the half-slot's previous use was freed, then its two 16 KB blocks
+          const int s = is_v ? at_vslot(e) : at_kslot(e);
+          if (e >= ring && !mbar_wait(&hs_free[s], is_v ? at_vparity(e - ring) : at_kparity(e - ring), &abort_s,
+                                      p.err, DG_DEVERR_TIMEOUT_ATTN)) {
+            ok = false;
+            break;
+          }
+          const int krow = i == 0 ? key0 : key0 - p.base;
+          if (!DG_GUARD(krow >= 0 && krow % AT_W == 0, p.err)) {
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sHalf + s * AT_HSLOT;
+          (is_v ? issued_v : issued_k) = e + 1;
+          mbar_arrive_expect_tx(&hs_full[s], AT_HSLOT);
+          const CUtensorMap* map = i == 0 ? map_hi : map_lo;
+          if (is_v) {  // V^T [128 d][64 keys] blocks: keys krow .. +63, +64 .. +127
+            tma_load_3d(dst, map, krow, 0, kvh, &hs_full[s]);
+            tma_load_3d(dst + AT_BLK, map, krow + 64, 0, kvh, &hs_full[s]);
+          } else {     // K [128 keys][64 d] blocks: d 0 .. 63, 64 .. 127
+            tma_load_3d(dst, map, 0, krow, kvh, &hs_full[s]);
+            tma_load_3d(dst + AT_BLK, map, 64, krow, kvh, &hs_full[s]);
+          }
+        }
       }
     }
     __syncwarp();
@@ -467,6 +473,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const int loads = at_loads_into(r, issued_k, AT_KSLOTS);
       if (loads > 0) mbar_wait_drain(&hs_full[r], (uint32_t)(loads - 1) & 1u);
     }
+  }
+  if (abort_s && tid == AT_VLOAD_WARP * 32) {
     for (int r = 0; r < AT_VSLOTS; ++r) {
       const int loads = at_loads_into(r, issued_v, AT_VSLOTS);
       if (loads > 0) mbar_wait_drain(&hs_full[AT_KSLOTS + r], (uint32_t)(loads - 1) & 1u);

@@ -326,12 +326,12 @@ def run_pair(c, bug=None, force_pair=None):
 # ---------------------------------------------------------------- tc_attn_kernel
 def run_single(c, bug=None):
     """tc_attn_kernel: one head x 128 rows x 128-key chunks; the query tile (hi + lo) in
-    shared memory by TMA, then a ring of two 32 KB half-slots for K and one of three for V^T
+    shared memory by TMA, then a ring of three 32 KB half-slots for K and one of two for V^T
     (with their low terms for own keys); TMEM: S buffers at columns 0 and 128, O at 256,
     P hi at 384 and lo at 448.  The replay runs S as far ahead as the barriers let it: S(j + 2)
     lands in S buffer j & 1 as soon as the softmax has read S(j) -- before it writes P(j)
     where chunk j + 2's K could be loaded by then, else after PV(j) frees half-slots; the
-    load warp fills half-slots as soon as they are freed.
+    two load threads fill their rings' half-slots as soon as they are freed.
 
     bug: "one_s_buffer" -- both S buffers at column 0; "p_lo_offset" -- P lo at 416, half
     over P hi; "q_lo_block" -- the query's lo MMAs read its hi blocks; "v_free_early" -- a
@@ -341,7 +341,7 @@ def run_single(c, bug=None):
     group = nq // nkv
     n_splits, cps = splits_single(n_q, nq, n_keys)
     W, BLK = 128, 128 * 128
-    QTILE, HSLOT, KSLOTS, VSLOTS = 4 * BLK, 2 * BLK, 2, 3
+    QTILE, HSLOT, KSLOTS, VSLOTS = 4 * BLK, 2 * BLK, 3, 2
     HSLOTS = KSLOTS + VSLOTS
     sQ, sHalf = 0, QTILE
     at_s = (lambda b: 0) if bug == "one_s_buffer" else (lambda b: b * 128)
@@ -370,7 +370,7 @@ def run_single(c, bug=None):
                 is_cur = lambda j: (c_begin + j) * W >= c["base"]
                 for off, mp, x in ((0, "Q", 0), (BLK, "Q", 64), (2 * BLK, "Ql", 0), (3 * BLK, "Ql", 64)):
                     sm.tma_load_3d(sQ + off, m[mp], x, q_row0, h, 64, 128)
-                # the rings (K entry e in half-slot e % 2, V^T entry e in 2 + e % 3): per chunk
+                # the rings (K entry e in half-slot e % 3, V^T entry e in 3 + e % 2): per chunk
                 # its K parts, then its V^T parts, in the load warp's order
                 plan, items, ek, ev = [], [], 0, 0
                 for j in range(nck):
@@ -382,33 +382,37 @@ def run_single(c, bug=None):
                     ek += n
                     ev += n
                 holder = {}                                   # half-slot -> (chunk, operand) held until freed
-                loaded = [0]
+                queues = {op: [it for it in items if it[1] == op] for op in ("K", "V")}
+                loaded = {"K": 0, "V": 0}                     # entries each load thread issued, in order
 
                 def pump():
-                    """The load warp: the next items, each once its half-slot's previous use was freed."""
-                    while loaded[0] < len(items):
-                        j, op, i, s_ = items[loaded[0]]
-                        if s_ in holder:
-                            return
-                        key0 = (c_begin + j) * W
-                        krow = key0 if i == 0 else key0 - c["base"]
-                        dst = sHalf + s_ * HSLOT
-                        if op == "K":
-                            mk = "K" if i == 0 else "Kl"
-                            sm.tma_load_3d(dst, m[mk], 0, krow, kvh, 64, 128)
-                            sm.tma_load_3d(dst + BLK, m[mk], 64, krow, kvh, 64, 128)
-                        else:
-                            mv = "Vt" if i == 0 else "Vtl"
-                            sm.tma_load_3d(dst, m[mv], krow, 0, kvh, 64, 128)
-                            sm.tma_load_3d(dst + BLK, m[mv], krow + 64, 0, kvh, 64, 128)
-                        holder[s_] = (j, op)
-                        loaded[0] += 1
+                    """The two load threads: the next entries of their rings, each once its
+                    half-slot's previous use was freed."""
+                    for op in ("K", "V"):
+                        qq = queues[op]
+                        while loaded[op] < len(qq):
+                            j, _, i, s_ = qq[loaded[op]]
+                            if s_ in holder:
+                                break
+                            key0 = (c_begin + j) * W
+                            krow = key0 if i == 0 else key0 - c["base"]
+                            dst = sHalf + s_ * HSLOT
+                            if op == "K":
+                                mk = "K" if i == 0 else "Kl"
+                                sm.tma_load_3d(dst, m[mk], 0, krow, kvh, 64, 128)
+                                sm.tma_load_3d(dst + BLK, m[mk], 64, krow, kvh, 64, 128)
+                            else:
+                                mv = "Vt" if i == 0 else "Vtl"
+                                sm.tma_load_3d(dst, m[mv], krow, 0, kvh, 64, 128)
+                                sm.tma_load_3d(dst + BLK, m[mv], krow + 64, 0, kvh, 64, 128)
+                            holder[s_] = (j, op)
+                            loaded[op] += 1
 
                 def ready(j, op):
                     pump()
-                    need = [it for it in items if it[0] == j and it[1] == op]
-                    assert all(items.index(it) < loaded[0] for it in need), \
-                        "the MMA thread would wait for a half-slot the load warp cannot fill"
+                    need = [it for it in queues[op] if it[0] == j]
+                    assert all(queues[op].index(it) < loaded[op] for it in need), \
+                        "the MMA thread would wait for a half-slot the load thread cannot fill"
 
                 def free(j, op):
                     for s_ in (plan[j][0] if op == "K" else plan[j][1]):
@@ -479,7 +483,7 @@ def run_single(c, bug=None):
 
                 def k_loaded(j):
                     pump()
-                    return all(items.index(it) < loaded[0] for it in items if it[0] == j and it[1] == "K")
+                    return all(queues["K"].index(it) < loaded["K"] for it in queues["K"] if it[0] == j)
 
                 pump()
                 for j in range(min(nck, 2)):

@@ -94,7 +94,7 @@ class TwoRingPlan:
     kslots half-slots, its V^T parts those of a ring of vslots half-slots numbered after
     the K ring's (at_kslot / at_vslot and the use parities in the kernel)."""
 
-    def __init__(self, kslots=2, vslots=3):
+    def __init__(self, kslots=3, vslots=2):
         self.ek = self.ev = 0
         self.kslots, self.vslots = kslots, vslots
 
@@ -130,7 +130,7 @@ def audit(kernel, n_q, pos0, n_keys, causal, nq, nkv, T):
     else:
         n_splits, cps = splits_single(n_q, nq, n_keys)
         nh, ys = 1, nq
-        smem_q, slot_bytes, slots = 4 * 16384, 32768, 5         # the query tile, 2 + 3 half-slots
+        smem_q, slot_bytes, slots = 4 * 16384, 32768, 5         # the query tile, 3 + 2 half-slots
         smem_total = 1024 + smem_q + slots * slot_bytes
         assert smem_total <= 227 * 1024 - 512
         # TMEM columns: S buffers 0..127 and 128..255, O 256..383, P buffers 384..447 and 448..511
@@ -289,7 +289,7 @@ def test_ring_arithmetic_counts_the_loads_of_each_half_slot(slots):
     """The wind-down's count of loads issued into each half-slot (a2_loads_into /
     at_loads_into) is the number of ring entries below the issued count in that half-slot,
     and the last one's use parity is what the drain waits for (rings of 3 in the head-pair
-    kernel, of 2 and 3 in the single-head kernel)."""
+    kernel, of 3 and 2 in the single-head kernel)."""
     def loads_into(s, n):
         return (n - 1 - s) // slots + 1 if n > s else 0
     for n in range(0, 40):
@@ -306,9 +306,9 @@ def test_kernel_slot_plans_are_the_simulated_ones(nck, cur_from):
     plan = HalfSlotPlan(3)
     got = [plan.take(j >= cur_from) for j in range(nck)]
     assert got == [(list(k), list(v)) for k, v in TP.half_slot_plan(nck, cur_from, 3)]
-    plan2 = TwoRingPlan(2, 3)
+    plan2 = TwoRingPlan(3, 2)
     got2 = [plan2.take(j >= cur_from) for j in range(nck)]
-    assert got2 == [(list(k), list(v)) for k, v in TP.two_ring_plan(nck, cur_from, 2, 3)]
+    assert got2 == [(list(k), list(v)) for k, v in TP.two_ring_plan(nck, cur_from, 3, 2)]
 
 
 def test_splits_fill_about_one_wave():
