@@ -737,6 +737,32 @@ def run_kernel_attention(args):
     return 0
 
 
+def run_kernel_mma(args):
+    """The tensor-pipe rate probe: one CTA per SM issuing MMAs of 128 x n x 16 back to back
+    (A from shared memory or from TMEM), for the shapes the pass issues; one JSON line per
+    shape with the cycles per instruction and the aggregate rate."""
+    import torch
+    from block_diffusion_lm_masked_b200 import dg
+    torch.cuda.init()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    hbm, tf_burst, _, peak_src = _peaks()
+    count = 1 << 14
+    for a_tmem in (False, True):
+        for n in (64, 128, 256):
+            dg.debug_mma_rate(a_tmem, n, 256, sms)  # warm-up
+            cyc, ms = dg.debug_mma_rate(a_tmem, n, count, sms)
+            tf = 2.0 * 128 * n * 16 * count * sms / (ms * 1e-3) / 1e12
+            print(json.dumps({"metric": "tcgen05 MMA instruction rate (one issuing thread per SM)",
+                              "value": cyc / count, "unit": "cycles per instruction", "higher_is_better": False,
+                              "dtype": "bf16", "data": "zero operands",
+                              "config": {"workload": f"{count} MMAs of 128 x {n} x 16, A from "
+                                                     f"{'TMEM' if a_tmem else 'shared memory'}, B from shared "
+                                                     f"memory, {sms} CTAs"},
+                              "tflops": tf, "frac_of_peak": tf / tf_burst,
+                              "peak_source": f"{peak_src} bf16_tflops"}), flush=True)
+    return 0
+
+
 def run_kernel_gemm(args):
     """--kernel gemm --gemm vocab|gate_up|down: one GEMM launch of the large model's shapes
     through the debug entry (the pass's persistent tcgen05 kernel) on synthetic bf16 data:
@@ -834,10 +860,10 @@ def main():
     ap.add_argument("--attn-pair", action="store_true",
                     help="run attention through the head-pair kernel instead of the single-head kernel "
                          "(sets DG_ATTN_PAIR=1)")
-    ap.add_argument("--kernel", choices=["attention", "gemm"], default=None,
+    ap.add_argument("--kernel", choices=["attention", "gemm", "mma"], default=None,
                     help="time one kernel alone on synthetic data instead of the step (attention: the "
                          "block-masked attention call over --keys keys; gemm: one GEMM of the large model's "
-                         "shapes, --gemm)")
+                         "shapes, --gemm; mma: the tensor-pipe rate probe for 128 x n x 16 instructions)")
     ap.add_argument("--gemm", choices=["vocab", "gate_up", "down"], default="vocab",
                     help="--kernel gemm: which GEMM")
     ap.add_argument("--keys", type=int, default=8192, help="--kernel attention: key count")
@@ -849,6 +875,8 @@ def main():
         return run_kernel_attention(args)
     if args.kernel == "gemm":
         return run_kernel_gemm(args)
+    if args.kernel == "mma":
+        return run_kernel_mma(args)
     if args.attn_pair:  # read by the library at its first attention call
         os.environ["DG_ATTN_PAIR"] = "1"
     name = args.workload

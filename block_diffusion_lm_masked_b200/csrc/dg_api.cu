@@ -1775,6 +1775,43 @@ extern "C" dg_status dg_debug_set_wait_limit(uint64_t limit_ns) {
   return DG_OK;
 }
 
+extern "C" dg_status dg_debug_mma_rate(int32_t a_tmem, int32_t n, int32_t count, int32_t blocks,
+                                       uint64_t* cycles_out, float* ms_out, dg_stream stream) {
+  DG_CHECK_ARG(n == 64 || n == 128 || n == 256, "n must be 64, 128 or 256");
+  DG_CHECK_ARG(count >= 1 && count <= (1 << 20), "count must be in [1, 1048576]");
+  DG_CHECK_ARG(blocks >= 1 && blocks <= 1024, "blocks must be in [1, 1024]");
+  DG_CHECK_ARG(cycles_out && ms_out, "NULL output");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned long long* d_cycles = nullptr;
+  int* d_err = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  cudaError_t e = cudaMalloc(&d_cycles, sizeof(unsigned long long) + sizeof(int));
+  if (e == cudaSuccess) {
+    d_err = reinterpret_cast<int*>(d_cycles + 1);
+    e = cudaMemsetAsync(d_cycles, 0, sizeof(unsigned long long) + sizeof(int), st);
+  }
+  if (e == cudaSuccess) e = cudaEventCreate(&e0);
+  if (e == cudaSuccess) e = cudaEventCreate(&e1);
+  if (e == cudaSuccess) e = cudaEventRecord(e0, st);
+  if (e == cudaSuccess) e = dg::launch_mma_rate(a_tmem ? 1 : 0, n, count, blocks, d_cycles, d_err, st);
+  if (e == cudaSuccess) e = cudaEventRecord(e1, st);
+  if (e == cudaSuccess) e = cudaEventSynchronize(e1);
+  float ms = 0.f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+  unsigned long long cyc = 0;
+  int derr = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&cyc, d_cycles, sizeof(cyc), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&derr, d_err, sizeof(derr), cudaMemcpyDeviceToHost);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (d_cycles) cudaFree(d_cycles);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "mma rate probe: %s", cudaGetErrorString(e));
+  if (derr) return fail(DG_ERR_TIMEOUT, "mma rate probe: the wait for the MMAs gave up");
+  *cycles_out = cyc;
+  *ms_out = ms;
+  return DG_OK;
+}
+
 extern "C" dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream) {
   DG_CHECK_ARG(d_ws, "workspace is NULL");
   DG_CHECK_ARG(timeout_ms >= 1 && timeout_ms <= 10000, "timeout_ms must be in [1, 10000]");

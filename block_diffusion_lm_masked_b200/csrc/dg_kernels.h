@@ -178,6 +178,10 @@ cudaError_t launch_update_select(const UpdPart* part, int C, int V, int splits, 
 cudaError_t launch_fill_i32(int32_t* p, int n, int32_t v, cudaStream_t st);
 
 cudaError_t launch_bounded_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
+// tensor-pipe rate probe (k_probe.cu): `blocks` CTAs, each issuing `count` MMAs of
+// 128 x n x 16 (A from TMEM when a_tmem), n in {64, 128, 256}; block 0's cycles to *cycles
+cudaError_t launch_mma_rate(int a_tmem, int n, int count, int blocks, unsigned long long* cycles, int* err,
+                            cudaStream_t st);
 
 // the bounded-wait limit of each kernel file (default DG_WAIT_NS; failure tests shorten it)
 cudaError_t set_wait_limit_attn(uint64_t ns);

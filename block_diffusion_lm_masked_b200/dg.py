@@ -104,6 +104,7 @@ def _load():
         "dg_renoise_count": (I32, [I32, I32, I32, F32, F32]),
         "dg_debug_bounded_wait": (I32, [P, I32, P]),
         "dg_debug_set_wait_limit": (I32, [U64]),
+        "dg_debug_mma_rate": (I32, [I32, I32, I32, I32, P, P, P]),
         "dg_debug_gemm_bf16": (I32, [P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
         "dg_debug_gemm_scratch_bytes": (SZ, [I32, I32]),
         "dg_debug_gemm_mx8": (I32, [P, P, P, P, I32, I32, P, P, I32, I32, P, P, P, I32, P, SZ, P, P]),
@@ -566,6 +567,16 @@ def debug_bounded_wait(ws, timeout_ms, stream=None):
 
 
 WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
+def debug_mma_rate(a_tmem: bool, n: int, count: int, blocks: int, stream=None):
+    """Tensor-pipe rate probe (include/dg_debug.h): returns (block 0's cycles from the first
+    MMA issue to the completion, the launch's milliseconds)."""
+    cyc = ctypes.c_uint64()
+    ms = ctypes.c_float()
+    _check(lib.dg_debug_mma_rate(1 if a_tmem else 0, int(n), int(count), int(blocks), ctypes.byref(cyc),
+                                 ctypes.byref(ms), _stream(stream)))
+    return int(cyc.value), float(ms.value)
 
 
 def debug_set_wait_limit(limit_ns: int):

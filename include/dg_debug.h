@@ -158,6 +158,18 @@ dg_status dg_debug_bounded_wait(void* d_ws, int32_t timeout_ms, dg_stream stream
  * while kernels run.  DG_ERR_INVALID_ARG above 2 s; DG_ERR_CUDA if a copy fails. */
 dg_status dg_debug_set_wait_limit(uint64_t limit_ns);
 
+/* Tensor-pipe rate probe: `blocks` CTAs (one per SM), each with one thread issuing
+ * `count` tcgen05 MMAs of 128 x n x 16 (bf16 inputs, fp32 accumulation in TMEM) back to
+ * back on operands it zeroes first -- A from shared memory (a_tmem = 0) or from TMEM
+ * (a_tmem = 1), B from shared memory -- then waiting for them (bounded wait, 1 s).
+ * *cycles_out (host): block 0's clock64 cycles from the first issue to the completion;
+ * *ms_out (host): the launch's CUDA-event time.  n in {64, 128, 256}, count in
+ * [1, 1048576], blocks in [1, 1024].  The work is the probe's only output; it measures
+ * the rate the attention kernel's 128 x 128 x 16 instructions can reach.
+ * DG_ERR_INVALID_ARG on a bad argument (nothing launched); DG_ERR_TIMEOUT if the wait gave up. */
+dg_status dg_debug_mma_rate(int32_t a_tmem, int32_t n, int32_t count, int32_t blocks, uint64_t* cycles_out,
+                            float* ms_out, dg_stream stream);
+
 /* Kernels launched by the library since it was loaded (all kinds, profiling or not). */
 int64_t dg_launch_count(void);
 

@@ -425,3 +425,19 @@ def test_debug_attention_validation_on_host(name):
     for args in bad:
         assert f(*args, None) == dg.DG_ERR_INVALID_ARG, args
     assert dg.lib.dg_launch_count() == launches
+
+
+def test_mma_rate_probe_validation_on_host():
+    """The tensor-pipe probe refuses bad shapes and NULL outputs before any CUDA call."""
+    c, m = ctypes.c_uint64(), ctypes.c_float()
+    C, M = ctypes.byref(c), ctypes.byref(m)
+    launches = dg.lib.dg_launch_count()
+    bad = [(0, 96, 16, 1, C, M),        # n not 64, 128 or 256
+           (0, 128, 0, 1, C, M),        # no MMAs
+           (0, 128, 1 << 21, 1, C, M),  # too many
+           (1, 128, 16, 0, C, M),       # no CTAs
+           (1, 128, 16, 2048, C, M),    # too many CTAs
+           (0, 128, 16, 1, None, M)]    # NULL output
+    for args in bad:
+        assert dg.lib.dg_debug_mma_rate(*args, None) == dg.DG_ERR_INVALID_ARG, args
+    assert dg.lib.dg_launch_count() == launches
