@@ -11,7 +11,11 @@
 // tile i+1 overlap the epilogue of tile i.  Every wait is bounded.
 //
 // Options: two_terms (tokens given as bf16 hi + lo, both accumulated: fp32-precision
-// activations against bf16 weights); dual_a (gate and up weight tiles accumulated
+// activations against bf16 weights; where a tile's padded token rows fit twice in its
+// accumulator -- the expert tiles, 16-64 rows against 128 columns -- one MMA of N = 2 x rows
+// takes the hi rows and the lo rows, which sit back to back in shared memory, into two
+// column ranges that the epilogue adds: an MMA instruction costs about the same for any
+// N up to 128 (measured: 96 cycles), so the small tiles issue half the instructions); dual_a (gate and up weight tiles accumulated
 // into two TMEM regions, SwiGLU epilogue); m_pair (a tile is two consecutive 128-row
 // weight tiles of one matrix sharing each token load: the dense projections, whose
 // token operand is re-read once per weight tile, read it half as often); k_splits
@@ -256,7 +260,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_fence_after();
         const uint32_t d0 = tmem + (uint32_t)(buf * acc_cols);
         const uint32_t d1 = d0 + (uint32_t)p.n_max;
-        const uint32_t idesc = idesc_bf16_f32(TC_BM, n_pad);
+        // both token terms in one MMA (columns 0 .. n_pad - 1: hi, n_pad .. 2 n_pad - 1: lo)
+        const bool fuse = terms == 2 && 2 * n_pad <= p.n_max;
+        const uint32_t idesc = idesc_bf16_f32(TC_BM, fuse ? 2 * n_pad : n_pad);
         const uint32_t tx = kb_bytes(n_pad);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % TC_MAX_STAGES;
@@ -276,11 +282,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint64_t bd = sw128_kmajor_desc(sb + kk * 32);
             const uint64_t bd2 = sw128_kmajor_desc(sb + (uint32_t)n_pad * 128 + kk * 32);
             tc_mma(d0, ad, bd, idesc, acc);
-            if (terms == 2) tc_mma(d0, ad, bd2, idesc, 1u);
+            if (terms == 2 && !fuse) tc_mma(d0, ad, bd2, idesc, 1u);
             if (n_a == 2) {
               const uint64_t ad2 = sw128_kmajor_desc(sa + a_bytes + kk * 32);
               tc_mma(d1, ad2, bd, idesc, acc);
-              if (terms == 2) tc_mma(d1, ad2, bd2, idesc, 1u);
+              if (terms == 2 && !fuse) tc_mma(d1, ad2, bd2, idesc, 1u);
             }
           }
           tc_commit(&empty_bar[s]);
@@ -301,6 +307,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const TileInfo ti = decode_tile(p, t);
       const int n_pad = (ti.rows + 15) & ~15;
       const int buf = j % nbuf;
+      const bool fuse = terms == 2 && 2 * n_pad <= p.n_max;  // the lo term's columns follow the hi term's
       // the warp votes on the wait's outcome: tcgen05.ld below is warp-collective, so no lane
       // may go on alone after another gave up
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (uint32_t)(j / nbuf) & 1u, &abort_s, p.err,
@@ -313,15 +320,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int f = ti.m * rows_per_tile + half * TC_BM + row;  // weight row = output feature
         const bool fvalid = f < p.a_rows_per_group;
         for (int c0 = 0; c0 < n_pad; c0 += 16) {
-          uint32_t ra[16], rb[16];
+          uint32_t ra[16], rb[16], ra2[16], rb2[16];
           tmem_ld16(t0 + c0, ra);
           if (EPI == EPI_SWIGLU_BF16) tmem_ld16(t0 + p.n_max + c0, rb);
+          if (fuse) {
+            tmem_ld16(t0 + n_pad + c0, ra2);
+            if (EPI == EPI_SWIGLU_BF16) tmem_ld16(t0 + p.n_max + n_pad + c0, rb2);
+          }
           tc_wait_ld();
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
             const int col = c0 + q;
-            const float a = __uint_as_float(ra[q]);
-            const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) : 0.0f;
+            const float a = __uint_as_float(ra[q]) + (fuse ? __uint_as_float(ra2[q]) : 0.0f);
+            const float b = EPI == EPI_SWIGLU_BF16 ? __uint_as_float(rb[q]) + (fuse ? __uint_as_float(rb2[q]) : 0.0f)
+                                                   : 0.0f;
             if (!fvalid || col >= ti.rows) continue;
             const size_t o = (size_t)(ti.row0 + col) * p.ld_out + f;
             if (EPI == EPI_STORE_F32) {

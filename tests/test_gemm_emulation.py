@@ -152,13 +152,21 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
 
         def epilogue_half(j, t, half):
             g, row0, rows, split, m = tile_of(t)
+            n_pad = (rows + 15) & ~15
+            fuse = terms == 2 and 2 * n_pad <= n_max and bug != "no_fuse_add"
             d0 = (j % nbuf) * acc_cols + half * n_max
             f = m * tile_rows + half * BM + np.arange(BM)
             ok = f < rows_a
+
+            def col_sum(c):
+                v = tm.f32(c, 1)[:, 0]
+                if fuse:                                # the lo term's column, n_pad further on
+                    v = (v + tm.f32(c + n_pad, 1)[:, 0]).astype(np.float32)
+                return v.astype(np.float64)
             for col in range(rows):
-                a = tm.f32(d0 + col, 1)[:, 0].astype(np.float64)
+                a = col_sum(d0 + col)
                 if swiglu:
-                    b = tm.f32(d0 + n_max + col, 1)[:, 0].astype(np.float64)
+                    b = col_sum(d0 + n_max + col)
                     hv = (a / (1.0 + np.exp(-a)) * b).astype(np.float32)
                     hi = T.bf16_value(T.bf16_bits(hv)).astype(np.float64)
                     out[row0 + col, f[ok]] = hi[ok]
@@ -183,14 +191,17 @@ def run_gemm(W, X_hi, X_lo, rows_a, K, ld_out, items=None, n_max=64, k_splits=1,
             d1 = d0 + (n_max if bug != "d1" else acc_cols // 4)
             sa = offs[it][0]
             sb = sa + n_a * a_bytes
+            # both token terms in one MMA of N = 2 n_pad where they fit the accumulator twice
+            fuse = terms == 2 and 2 * n_pad <= n_max
+            nn = 2 * n_pad if fuse else n_pad
             for kk in range(BK // 16):
                 acc = kb != 0 or kk != 0
-                T.mma_ss(tm, sm, d0, sa + kk * 32, sb + kk * 32, BM, n_pad, acc)
-                if terms == 2:
+                T.mma_ss(tm, sm, d0, sa + kk * 32, sb + kk * 32, BM, nn, acc)
+                if terms == 2 and not fuse:
                     T.mma_ss(tm, sm, d0, sa + kk * 32, sb + n_pad * 128 + kk * 32, BM, n_pad, True)
                 if n_a == 2:
-                    T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + kk * 32, BM, n_pad, acc)
-                    if terms == 2:
+                    T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + kk * 32, BM, nn, acc)
+                    if terms == 2 and not fuse:
                         T.mma_ss(tm, sm, d1, sa + a_bytes + kk * 32, sb + n_pad * 128 + kk * 32, BM, n_pad, True)
             mma_done += 1
             if kb == nkb - 1:
@@ -276,10 +287,23 @@ def test_vocab_single_term_replay():
     assert np.abs(out.reshape(n, V) - ref).max() / np.abs(ref).max() < 2e-6
 
 
-@pytest.mark.parametrize("bug", ["d1", "no_slab", "lo_offset"])
+@pytest.mark.parametrize("bug", ["d1", "no_slab", "lo_offset", "no_fuse_add"])
 def test_planted_mistakes_in_the_gemm_replay_are_caught(bug):
+    """An accumulator at the wrong column, split-K slabs over each other, the lo token term
+    half-way into the hi rows, or an epilogue that leaves out the lo term's columns of a
+    tile whose two terms share one MMA: each moves the result well past the fp32 level."""
     rng = np.random.default_rng(4)
-    if bug == "d1":
+    if bug == "no_fuse_add":
+        counts, F, K = [20, 7], 128, 128      # tiles of 32 and 16 rows: both terms in one MMA
+        off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
+        items = [(e, int(off[e]), counts[e]) for e in range(2)]
+        x, hi, lo = bf16_pair(rng, int(off[-1]), K)
+        Wg, wg = weights(rng, 2, F, K)
+        Wu, wu = weights(rng, 2, F, K)
+        out, out_lo = run_gemm(Wg, hi, lo, F, K, F, items=items, n_max=128, W2=Wu, bug=bug)
+        ref = O.silu(x[:20] @ wg[0].T) * (x[:20] @ wu[0].T)
+        got = (out + out_lo)[:20]
+    elif bug == "d1":
         counts, F, K = [40, 90], 128, 128
         off = np.concatenate([[0], np.cumsum(counts)]).astype(int)
         items = [(e, r0, min(64, off[e + 1] - r0)) for e in range(2) for r0 in range(off[e], off[e + 1], 64)]
