@@ -141,7 +141,9 @@ REF_BUDGET_S = 90.0
 # DRAM bytes (read + write) of one launch of a kernel from an ncu capture of this
 # workload, valid only for the kernel source it was taken on (sha256 prefix of the
 # kernel's source file); any other source reports null.
-NCU_TRAFFIC = {("layer1_bf16", "gemm_gate_up"): ("k_tc_gemm.cu", "8f9740b8fc51d669", 457.380608e6 + 6.031104e6)}
+NCU_TRAFFIC = {("layer1_bf16", "gemm_gate_up"): ("k_tc_gemm.cu", "8f9740b8fc51d669", 457.380608e6 + 6.031104e6),
+               # profiles/gemm_gate_up_large4_bf16.md: the launch at the large model's sizes
+               ("large4_bf16", "gemm_gate_up"): ("k_tc_gemm.cu", "dba5f1c440f71225", 1073.691e6 + 9.256448e6)}
 
 
 def _ncu_traffic(workload, kernel):
