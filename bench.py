@@ -124,6 +124,32 @@ class Clocks:
                 "reasons": reasons, "samples": len(self.samples), "source": "NVML, 10 ms"}
 
 
+# clock-event reasons that make a timed region no measurement (a power cap is kept and noted)
+SLOWDOWN_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clocked(ranks, dev, run, sampler=Clocks):
+    """Runs the timed region run() under the clock sampler; returns (run's result, the clock
+    record).  A region that saw a hardware or thermal slowdown on any rank is timed once
+    more, on every rank so that the ranks' collectives stay matched; the second region's
+    record then names the reasons that voided the first under "remeasured_after"."""
+    clk = sampler(dev)
+    clk.start()
+    out = run()
+    clocks = clk.stop()
+    slowed = sorted(set(clocks.get("reasons") or ()) & set(SLOWDOWN_REASONS))
+    if ranks.max(1.0 if slowed else 0.0) > 0:
+        ranks.barrier()
+        if getattr(dev, "type", None) == "cuda":
+            import torch
+            torch.cuda.synchronize(dev)
+        clk = sampler(dev)
+        clk.start()
+        out = run()
+        clocks = dict(clk.stop(), remeasured_after=slowed)
+    return out, clocks
+
+
 def _oracle_step(host, ocache, canvas, n, prec, step):
     from oracle import dg_oracle as O
     logits, _ = O.denoise_pass(host, ocache, canvas, prec)
@@ -352,10 +378,7 @@ def run_variant(args, cfg, name):
 
     ranks.barrier()
     torch.cuda.synchronize(dev)
-    clk = Clocks(dev)
-    clk.start()
-    total_ms, launches = timed(args.steps, profile=False)
-    clocks = clk.stop()
+    (total_ms, launches), clocks = clocked(ranks, dev, lambda: timed(args.steps, profile=False))
     dg.device_status(ws)
     total_ms = ranks.max(total_ms)
     ranks.barrier()
@@ -479,19 +502,20 @@ def run_chained(args, cfg, name):
     dg.device_status(ws)
     ranks.barrier()
     torch.cuda.synchronize(dev)
-    clk = Clocks(dev)
-    clk.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(NC + 1)] for _ in range(args.steps)]
-    l0 = dg.launch_count()
-    for s_ in range(args.steps):
-        flush.zero_()
-        ev[s_][0].record(stream)
-        chain(s_, marks[s_])
-        ev[s_][1].record(stream)
-    torch.cuda.synchronize(dev)
-    launches = dg.launch_count() - l0
-    clocks = clk.stop()
+
+    def timed_chains():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        marks = [[torch.cuda.Event(enable_timing=True) for _ in range(NC + 1)] for _ in range(args.steps)]
+        l0 = dg.launch_count()
+        for s_ in range(args.steps):
+            flush.zero_()
+            ev[s_][0].record(stream)
+            chain(s_, marks[s_])
+            ev[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return ev, marks, dg.launch_count() - l0
+
+    (ev, marks, launches), clocks = clocked(ranks, dev, timed_chains)
     dg.device_status(ws)
     chain_ms = [a.elapsed_time(b) for a, b in ev]
     prompt_ms = statistics.median(ev[i][0].elapsed_time(marks[i][0]) for i in range(args.steps))
@@ -967,10 +991,7 @@ def main():
 
     ranks.barrier()
     torch.cuda.synchronize(dev)
-    clk = Clocks(dev)
-    clk.start()
-    total_ms, launches = timed(args.steps, profile=False)
-    clocks = clk.stop()
+    (total_ms, launches), clocks = clocked(ranks, dev, lambda: timed(args.steps, profile=False))
     dg.device_status(ws)
     total_ms = ranks.max(total_ms)
     ranks.barrier()

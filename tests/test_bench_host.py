@@ -1,6 +1,7 @@
 """bench.py's host-side helpers on the CPU: the NVML clock sampler (against a fake NVML
-module: it only reads), the hash guard that reports ncu traffic only for the kernel
-source it was captured on, the peak-file fallback and the whole-job value."""
+module: it only reads), the one re-measurement of a timed region that saw a hardware or
+thermal slowdown, the hash guard that reports ncu traffic only for the kernel source it
+was captured on, the peak-file fallback and the whole-job value."""
 import os
 import shutil
 import sys
@@ -111,3 +112,63 @@ def test_attention_kind_follows_the_switch(monkeypatch):
     assert bench._attention_kind().startswith("head pairs")
     monkeypatch.setenv("DG_ATTN_PAIR", "0")
     assert bench._attention_kind().startswith("one head")
+
+
+class _FakeSampler:
+    """Stands in for bench.Clocks: each region's record comes from a script."""
+    script = []
+
+    def __init__(self, dev):
+        self.dev = dev
+
+    def start(self):
+        pass
+
+    def stop(self):
+        reasons = _FakeSampler.script.pop(0)
+        return {"sm_mhz": 1900.0, "sm_max_mhz": 1965, "reasons": reasons, "samples": 10}
+
+
+@pytest.fixture
+def one_rank(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    return bench.Ranks("gloo", device="cpu")
+
+
+def _count_runs():
+    runs = []
+
+    def run():
+        runs.append(len(runs))
+        return ("result", len(runs))
+    return runs, run
+
+
+@pytest.mark.parametrize("reasons", [[], ["sw_power_cap"]])
+def test_clean_or_power_capped_region_is_kept(one_rank, reasons):
+    r = one_rank
+    _FakeSampler.script = [list(reasons)]
+    runs, run = _count_runs()
+    out, clocks = bench.clocked(r, "cpu", run, sampler=_FakeSampler)
+    assert runs == [0] and out == ("result", 1)
+    assert clocks["reasons"] == reasons and "remeasured_after" not in clocks
+
+
+@pytest.mark.parametrize("bad", ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"])
+def test_slowed_region_is_timed_once_more(one_rank, bad):
+    r = one_rank
+    _FakeSampler.script = [["sw_power_cap", bad], ["sw_power_cap"]]
+    runs, run = _count_runs()
+    out, clocks = bench.clocked(r, "cpu", run, sampler=_FakeSampler)
+    assert runs == [0, 1] and out == ("result", 2)      # the second region's result and clocks
+    assert clocks["reasons"] == ["sw_power_cap"] and clocks["remeasured_after"] == [bad]
+    assert _FakeSampler.script == []
+
+
+def test_second_slowed_region_is_reported_not_retried(one_rank):
+    r = one_rank
+    _FakeSampler.script = [["hw_slowdown"], ["hw_slowdown"]]
+    runs, run = _count_runs()
+    _, clocks = bench.clocked(r, "cpu", run, sampler=_FakeSampler)
+    assert runs == [0, 1] and clocks["reasons"] == ["hw_slowdown"]   # once more, not again
